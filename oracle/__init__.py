@@ -1,0 +1,193 @@
+"""CPU oracle for the TiDAR decode step -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  It wraps
+``tidar_oracle.c`` (plain C, fp64 arithmetic, unfused loops) through ctypes and
+shares no code with the CUDA library in ``ar_decoding_b200``.
+
+Functions take numpy arrays (fp32 or bf16-as-uint16 for the floating-point
+inputs, int32 for indices) and return numpy arrays.  See ``tidar_oracle.c`` for
+the method each one restates and the pages it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tidar_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+F32, BF16 = 0, 1
+GREEDY, REJECTION = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile tidar_oracle.c into liboracle.so (gcc, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        lib.tidar_oracle_step_key_visible.argtypes = [i, i, i]
+        lib.tidar_oracle_step_key_visible.restype = i
+        lib.tidar_oracle_step_attn.argtypes = [i, i, i, i, i, i, i, ctypes.c_double, P, P, P, i, i,
+                                               P, P, P, P, i, P, P, P, i]
+        lib.tidar_oracle_step_attn.restype = i
+        lib.tidar_oracle_append.argtypes = [i, i, i, i, i, i, P, P, P, i, i, P, P, P]
+        lib.tidar_oracle_append.restype = i
+        lib.tidar_oracle_verify.argtypes = [i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
+        lib.tidar_oracle_verify.restype = i
+        lib.tidar_oracle_commit.argtypes = [i, i, i, i, i, i, P, P, P, i, i, P, P, P, P]
+        lib.tidar_oracle_commit.restype = i
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    raise TypeError(f"oracle inputs are float32 or bf16 stored as uint16, got {a.dtype}")
+
+
+def rows_per_seq(k: int) -> int:
+    """Query rows of one sequence in one step: k drafts + k blocks of k slots (1 if k = 0)."""
+    return 1 if k == 0 else k + k * k
+
+
+def step_key_visible(k: int, row: int, key: int) -> bool:
+    return bool(_load().tidar_oracle_step_key_visible(k, row, key))
+
+
+def step_attn(q, k_blk, v_blk, k_pages, v_pages, page_table, seq_lens, k, *, scale=0.0,
+              sel=None, num_threads=0):
+    """Three-zone step attention in fp64.
+
+    q [B][R][Hq][D], k_blk/v_blk [B][R][Hkv][D], k_pages/v_pages
+    [num_pages][Hkv][page][D] (fp32 or uint16 bf16 bits), page_table
+    [B][max_pages] int32, seq_lens [B] int32.  Returns (out, lse): out
+    [B][R][Hq][D] and lse [B][R][Hq] (natural log), or [n][D] / [n] for the
+    (b, rho, h) triples in ``sel``.
+    """
+    lib = _load()
+    q = np.ascontiguousarray(q)
+    dt = _dtype_code(q)
+    B, R, Hq, D = q.shape
+    Hkv = k_blk.shape[2]
+    num_pages, _, page_size, _ = k_pages.shape
+    assert R == rows_per_seq(k)
+    k_blk, v_blk = np.ascontiguousarray(k_blk), np.ascontiguousarray(v_blk)
+    k_pages, v_pages = np.ascontiguousarray(k_pages), np.ascontiguousarray(v_pages)
+    page_table = np.ascontiguousarray(page_table, dtype=np.int32)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    for a in (k_blk, v_blk, k_pages, v_pages):
+        assert a.dtype == q.dtype
+    if sel is None:
+        n_sel, sel_arr = -1, None
+        out = np.zeros((B, R, Hq, D), np.float64)
+        lse = np.zeros((B, R, Hq), np.float64)
+    else:
+        sel_arr = np.ascontiguousarray(np.asarray(sel, dtype=np.int32).reshape(-1, 3))
+        n_sel = sel_arr.shape[0]
+        out = np.zeros((n_sel, D), np.float64)
+        lse = np.zeros((n_sel,), np.float64)
+    st = lib.tidar_oracle_step_attn(B, Hq, Hkv, D, k, page_size, dt, float(scale), _ptr(k_pages),
+                                    _ptr(v_pages), _ptr(page_table), page_table.shape[1], num_pages,
+                                    _ptr(seq_lens), _ptr(q), _ptr(k_blk), _ptr(v_blk), n_sel,
+                                    _ptr(sel_arr), _ptr(out), _ptr(lse), int(num_threads))
+    if st != 0:
+        raise ValueError(f"oracle step_attn failed with status {st}")
+    return out, lse
+
+
+def append(k_pages, v_pages, page_table, seq_lens, k_blk, v_blk, k):
+    """Return copies of the caches with the draft rows' K/V written at P_b.. P_b+n-1."""
+    lib = _load()
+    kp, vp = np.array(k_pages, copy=True), np.array(v_pages, copy=True)
+    num_pages, Hkv, page_size, D = kp.shape
+    page_table = np.ascontiguousarray(page_table, dtype=np.int32)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    k_blk, v_blk = np.ascontiguousarray(k_blk), np.ascontiguousarray(v_blk)
+    B = seq_lens.shape[0]
+    st = lib.tidar_oracle_append(B, Hkv, D, k, page_size, kp.dtype.itemsize, _ptr(kp), _ptr(vp),
+                                 _ptr(page_table), page_table.shape[1], num_pages, _ptr(seq_lens),
+                                 _ptr(k_blk), _ptr(v_blk))
+    if st != 0:
+        raise ValueError(f"oracle append failed with status {st}")
+    return kp, vp
+
+
+def verify(logits, drafts, k, mode, *, draft_logits=None, uniforms=None, block_guesses=None,
+           with_margins=False):
+    """Left-to-right verification, acceptance and selection (fp64).
+
+    Returns dict(accept_count [B], out_tokens [B][n], next_drafts [B][k],
+    selected_block [B], margins [B][n] if requested).
+    """
+    lib = _load()
+    logits = np.ascontiguousarray(logits)
+    dt = _dtype_code(logits)
+    B, n, V = logits.shape
+    assert n == max(k, 1)
+    drafts = None if drafts is None else np.ascontiguousarray(drafts, dtype=np.int32)
+    if draft_logits is not None:
+        draft_logits = np.ascontiguousarray(draft_logits)
+        assert draft_logits.dtype == logits.dtype
+    if uniforms is not None:
+        uniforms = np.ascontiguousarray(uniforms, dtype=np.float32)
+    if block_guesses is not None:
+        block_guesses = np.ascontiguousarray(block_guesses, dtype=np.int32)
+    acc = np.zeros(B, np.int32)
+    toks = np.zeros((B, n), np.int32)
+    nxt = np.zeros((B, max(k, 1)), np.int32)
+    selb = np.zeros(B, np.int32)
+    marg = np.zeros((B, n), np.float64) if with_margins else None
+    st = lib.tidar_oracle_verify(B, k, V, dt, mode, _ptr(logits), _ptr(drafts), _ptr(draft_logits),
+                                 _ptr(uniforms), _ptr(block_guesses), _ptr(acc), _ptr(toks),
+                                 _ptr(nxt), _ptr(selb), _ptr(marg))
+    if st != 0:
+        raise ValueError(f"oracle verify failed with status {st}")
+    res = dict(accept_count=acc, out_tokens=toks, next_drafts=nxt[:, :k], selected_block=selb)
+    if with_margins:
+        res["margins"] = marg
+    return res
+
+
+def commit(k_pages, v_pages, page_table, seq_lens, accept_count, k):
+    """KV commit/evict on copies.  Returns (k_pages, v_pages, page_table, seq_lens,
+    released, num_released, status)."""
+    lib = _load()
+    kp, vp = np.array(k_pages, copy=True), np.array(v_pages, copy=True)
+    pt = np.array(page_table, dtype=np.int32, copy=True)
+    sl = np.array(seq_lens, dtype=np.int32, copy=True)
+    acc = np.ascontiguousarray(accept_count, dtype=np.int32)
+    num_pages, Hkv, page_size, D = kp.shape
+    B = sl.shape[0]
+    n = max(k, 1)
+    cap = B * ((n + page_size - 1) // page_size + 1)
+    rel = np.zeros(cap, np.int32)
+    nrel = np.zeros(1, np.int32)
+    st = lib.tidar_oracle_commit(B, Hkv, D, k, page_size, kp.dtype.itemsize, _ptr(kp), _ptr(vp),
+                                 _ptr(pt), pt.shape[1], num_pages, _ptr(sl), _ptr(acc), _ptr(rel),
+                                 _ptr(nrel))
+    return kp, vp, pt, sl, rel, int(nrel[0]), st

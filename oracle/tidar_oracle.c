@@ -1,0 +1,450 @@
+/*
+ * tidar_oracle.c -- TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT PATH.
+ *
+ * A plain, slow, CPU restatement of one TiDAR decode step, written from the
+ * description of the method on these web pages (cited below by tag):
+ *
+ *   [EN]   "TiDAR：Nvidia 的擴散＋自回歸混合架構——把閒置的 GPU 算力換成推論加速"
+ *          (engineer-news.pages.dev)
+ *   [MS]   "TiDAR: Think in Diffusion, Talk in Autoregression" (mauroscia.it)
+ *   [NDfr] "TiDAR : l'hybride de NVIDIA qui rédige par diffusion et parle de
+ *          manière autorégressive" (nodesdaily.com, French)
+ *   [FG]   "論文の概要: TiDAR: Think in Diffusion, Talk in Autoregression"
+ *          (fugumt.com, arXiv 2511.08923 abstract)
+ *
+ * Only tests/, the smoke check and the CPU-baseline leg of the benchmark may
+ * load this code.  It shares no source with the CUDA library and never links it.
+ *
+ * Arithmetic: inputs are fp32 or bf16 (bf16 is widened exactly to fp64); every
+ * sum, exponential and division is in fp64.  Loops are unfused and unsplit:
+ * scores for all visible keys, then the maximum, then the normaliser, then the
+ * weighted sum of values, in key order.
+ *
+ * Notation (the pages give none in symbols; this is the plainest reading):
+ *   B batch, Hq query heads, Hkv KV heads, G = Hq/Hkv, D head_dim, P_b the
+ *   settled prefix length of sequence b, k the draft length, n = max(k,1),
+ *   R = k + k*k query rows per sequence (R = 1 when k = 0).
+ *   Rows of a step: draft rows r = 1..k (row index r-1), then mask block
+ *   j = 1..k, slot s = 1..k (row index k + (j-1)k + (s-1)).
+ *   Step keys use the same indices: D_1..D_k are step keys 0..k-1 and
+ *   M_{j,s} is step key k + (j-1)k + (s-1).
+ *
+ * Parity pins: every function here is checked by tests/test_oracle_*.py against
+ * closed forms, independent formulations (dense attention over explicitly
+ * concatenated key sets, numpy/torch library routines), invariants and
+ * chi-squared / exact-enumeration tests of the acceptance rule.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_PAGE 2
+#define ORACLE_ERR_COUNT 3
+
+/* bf16 -> fp64, exact: a bf16 value is the upper half of an fp32 value. */
+static double widen_bf16(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Element idx of a buffer stored as fp32 (dtype 0) or bf16 (dtype 1). */
+static double elem(const void* base, int64_t idx, int dtype) {
+  if (dtype == 0) return (double)((const float*)base)[idx];
+  return widen_bf16(((const uint16_t*)base)[idx]);
+}
+
+/*
+ * Structured mask over the step keys ([MS] §2 "Single Forward Pass &
+ * Structured Attention Mask": three zones, causal for the verified drafts,
+ * bidirectional for the pre-drafts; [NDfr] paragraph on the masking puzzle:
+ * settled tokens strictly causal, each guess block fully visible inside and
+ * seeing the whole settled past; [NDfr] paragraph on betting on every outcome:
+ * one guess block per future "first survives / two survive / all survive").
+ *
+ * Returns 1 if query row `row` may attend step key `key`.  The prefix keys are
+ * visible to every row and are not decided here.  The predicate depends on
+ * zone-relative indices only, never on P_b ([NDfr] masking paragraph: the same
+ * mask slides forward as the text grows).
+ */
+int tidar_oracle_step_key_visible(int k, int row, int key) {
+  if (k == 0) return key == 0;           /* plain AR decode: the newest token sees itself */
+  if (row < k) return key <= row;         /* draft row r sees D_1..D_r (causal) */
+  {
+    int j = (row - k) / k + 1;            /* mask block j in 1..k */
+    int first = k + (j - 1) * k;          /* its slots M_{j,1..k} */
+    if (key < j) return 1;                /* D_1..D_j: the j drafts of this future */
+    return key >= first && key < first + k; /* its own block, bidirectional */
+  }
+}
+
+static int rows_per_seq(int k) { return k == 0 ? 1 : k + k * k; }
+
+/* Address (in elements) of cache row `pos` of KV head g for sequence b, or -1
+ * if the page table does not map it to a valid page. */
+static int64_t cache_row(const int32_t* page_table, int max_pages, int num_pages,
+                         int page_size, int Hkv, int D, int b, int g, int64_t pos) {
+  int64_t pi = pos / page_size;
+  int32_t page;
+  if (pi >= max_pages) return -1;
+  page = page_table[(int64_t)b * max_pages + pi];
+  if (page < 0 || page >= num_pages) return -1;
+  return (((int64_t)page * Hkv + g) * page_size + pos % page_size) * D;
+}
+
+/*
+ * One output row of the step attention: softmax over every visible key of the
+ * scaled dot products, applied to the values (the plain definition of
+ * attention; the prefix zone comes from the KV cache, [MS] "KV Cache",
+ * [NDfr] paragraph on the three zones).  Query head h reads KV head h / G.
+ * Returns ORACLE_ERR_PAGE if a needed prefix page is unmapped.
+ */
+static int attend_one(int b, int rho, int h, int Hq, int Hkv, int D, int k, int page_size,
+                      int dtype, double scale, const void* k_pages, const void* v_pages,
+                      const int32_t* page_table, int max_pages, int num_pages, int P,
+                      const void* q, const void* k_blk, const void* v_blk,
+                      double* s /* scratch, P + R */, double* out, double* lse) {
+  const int R = rows_per_seq(k);
+  const int G = Hq / Hkv;
+  const int g = h / G;
+  const int64_t qoff = (((int64_t)b * R + rho) * Hq + h) * D;
+  int nkeys = 0, i, d;
+  double m = -INFINITY, z = 0.0;
+
+  /* scores: prefix keys 0..P-1, then the visible step keys in index order */
+  for (i = 0; i < P; ++i) {
+    int64_t ko = cache_row(page_table, max_pages, num_pages, page_size, Hkv, D, b, g, i);
+    double dot = 0.0;
+    if (ko < 0) return ORACLE_ERR_PAGE;
+    for (d = 0; d < D; ++d) dot += elem(q, qoff + d, dtype) * elem(k_pages, ko + d, dtype);
+    s[nkeys++] = dot * scale;
+  }
+  for (i = 0; i < R; ++i) {
+    if (tidar_oracle_step_key_visible(k, rho, i)) {
+      int64_t ko = (((int64_t)b * R + i) * Hkv + g) * D;
+      double dot = 0.0;
+      for (d = 0; d < D; ++d) dot += elem(q, qoff + d, dtype) * elem(k_blk, ko + d, dtype);
+      s[nkeys++] = dot * scale;
+    }
+  }
+  for (i = 0; i < nkeys; ++i) if (s[i] > m) m = s[i];
+  for (i = 0; i < nkeys; ++i) { s[i] = exp(s[i] - m); z += s[i]; }
+
+  for (d = 0; d < D; ++d) out[d] = 0.0;
+  nkeys = 0;
+  for (i = 0; i < P; ++i) {
+    int64_t vo = cache_row(page_table, max_pages, num_pages, page_size, Hkv, D, b, g, i);
+    double w = s[nkeys++] / z;
+    for (d = 0; d < D; ++d) out[d] += w * elem(v_pages, vo + d, dtype);
+  }
+  for (i = 0; i < R; ++i) {
+    if (tidar_oracle_step_key_visible(k, rho, i)) {
+      int64_t vo = (((int64_t)b * R + i) * Hkv + g) * D;
+      double w = s[nkeys++] / z;
+      for (d = 0; d < D; ++d) out[d] += w * elem(v_blk, vo + d, dtype);
+    }
+  }
+  *lse = m + log(z);
+  return ORACLE_OK;
+}
+
+/*
+ * Step attention over the three zones.
+ *   q      [B][R][Hq][D]      k_blk, v_blk [B][R][Hkv][D]  (dtype)
+ *   k_pages, v_pages [num_pages][Hkv][page_size][D]; page_table [B][max_pages]
+ *   seq_lens [B] (P_b).
+ * If n_sel < 0 every (b, rho, h) is computed into out [B][R][Hq][D] and
+ * lse [B][R][Hq]; otherwise only the n_sel triples sel[3i..3i+2] = (b, rho, h),
+ * into out [n_sel][D], lse [n_sel].  lse is the natural log of the softmax
+ * normaliser including the maximum.  scale <= 0 selects 1/sqrt(D).
+ */
+int tidar_oracle_step_attn(int B, int Hq, int Hkv, int D, int k, int page_size, int dtype,
+                           double scale, const void* k_pages, const void* v_pages,
+                           const int32_t* page_table, int max_pages, int num_pages,
+                           const int32_t* seq_lens, const void* q, const void* k_blk,
+                           const void* v_blk, int n_sel, const int32_t* sel, double* out,
+                           double* lse, int num_threads) {
+  const int R = rows_per_seq(k);
+  int64_t total, t;
+  int Pmax = 0, b, status = ORACLE_OK;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || k < 0 || page_size <= 0)
+    return ORACLE_ERR_ARG;
+  if (scale <= 0.0) scale = 1.0 / sqrt((double)D);
+  for (b = 0; b < B; ++b) {
+    if (seq_lens[b] < 0) return ORACLE_ERR_ARG;
+    if (seq_lens[b] > Pmax) Pmax = seq_lens[b];
+  }
+  total = n_sel < 0 ? (int64_t)B * R * Hq : n_sel;
+#ifdef _OPENMP
+  if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel
+#endif
+  {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(Pmax + R + 1));
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 4)
+#endif
+    for (t = 0; t < total; ++t) {
+      int bb, rho, h, st;
+      if (n_sel < 0) {
+        h = (int)(t % Hq);
+        rho = (int)((t / Hq) % R);
+        bb = (int)(t / ((int64_t)Hq * R));
+      } else {
+        bb = sel[3 * t]; rho = sel[3 * t + 1]; h = sel[3 * t + 2];
+      }
+      if (!s || bb < 0 || bb >= B || rho < 0 || rho >= R || h < 0 || h >= Hq) {
+        st = ORACLE_ERR_ARG;
+      } else {
+        st = attend_one(bb, rho, h, Hq, Hkv, D, k, page_size, dtype, scale, k_pages, v_pages,
+                        page_table, max_pages, num_pages, seq_lens[bb], q, k_blk, v_blk, s,
+                        out + t * D, lse + t);
+      }
+      if (st != ORACLE_OK) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+        status = st;
+      }
+    }
+    free(s);
+  }
+  return status;
+}
+
+/*
+ * Speculative write of the draft rows' K/V into the cache: the K/V of step rows
+ * 0..n-1 (D_1..D_k; the single row when k = 0) go to cache positions
+ * P_b .. P_b+n-1 of every KV head.  Byte copies (elem_bytes per element).
+ * The carried-over drafts are the second zone of a step ([NDfr] paragraph on
+ * the three zones); keeping their entries is what "reuse the settled cache"
+ * means once they are accepted.
+ */
+int tidar_oracle_append(int B, int Hkv, int D, int k, int page_size, int elem_bytes,
+                        void* k_pages, void* v_pages, const int32_t* page_table, int max_pages,
+                        int num_pages, const int32_t* seq_lens, const void* k_blk,
+                        const void* v_blk) {
+  const int R = rows_per_seq(k);
+  const int n = k > 0 ? k : 1;
+  int b, r, g, status = ORACLE_OK;
+  for (b = 0; b < B; ++b) {
+    for (r = 0; r < n; ++r) {
+      for (g = 0; g < Hkv; ++g) {
+        int64_t dst = cache_row(page_table, max_pages, num_pages, page_size, Hkv, D, b, g,
+                                (int64_t)seq_lens[b] + r);
+        int64_t src = (((int64_t)b * R + r) * Hkv + g) * D;
+        if (dst < 0) { status = ORACLE_ERR_PAGE; continue; }
+        memcpy((char*)k_pages + dst * elem_bytes, (const char*)k_blk + src * elem_bytes,
+               (size_t)D * elem_bytes);
+        memcpy((char*)v_pages + dst * elem_bytes, (const char*)v_blk + src * elem_bytes,
+               (size_t)D * elem_bytes);
+      }
+    }
+  }
+  return status;
+}
+
+/* softmax of one logit row in fp64: writes p[0..V-1] (may be NULL) and returns
+ * nothing else.  Two passes: maximum, then normaliser. */
+static void softmax_row(const void* base, int64_t off, int V, int dtype, double* p) {
+  double m = -INFINITY, z = 0.0;
+  int x;
+  for (x = 0; x < V; ++x) { double v = elem(base, off + x, dtype); if (v > m) m = v; }
+  for (x = 0; x < V; ++x) { p[x] = exp(elem(base, off + x, dtype) - m); z += p[x]; }
+  for (x = 0; x < V; ++x) p[x] /= z;
+}
+
+/* argmax with the lowest index winning ties, on the exact stored values */
+static int argmax_row(const void* base, int64_t off, int V, int dtype) {
+  int x, best = 0;
+  double bv = elem(base, off, dtype);
+  for (x = 1; x < V; ++x) {
+    double v = elem(base, off + x, dtype);
+    if (v > bv) { bv = v; best = x; }
+  }
+  return best;
+}
+
+/*
+ * Verification and acceptance ("Talk in Autoregression"): the drafts are
+ * scored left to right under the strict AR distribution ([NDfr] paragraph on
+ * betting on every outcome: strict left-to-right scoring; [MS] §1: a good
+ * draft is accepted, a bad one corrected); the output must equal plain AR
+ * sampling ([EN] section "TiDAR 在做什麼": mathematically equivalent to pure AR
+ * sampling; [NDfr] last paragraph: accepted text is rescored under the strict
+ * distribution).  The rejection rule is the speculative-sampling rule of the
+ * lineage [MS] names (Leviathan et al., Chen et al.), which keeps the AR
+ * distribution exact.
+ *
+ *   logits [B][n][V]: row i (1-based) is the AR distribution p_i of the token
+ *     after d_1..d_i.  drafts [B][k]: d_1..d_k (d_1 is the token sampled at the
+ *     end of the previous step and is always kept).
+ *   draft_logits [B][k-1][V] (mode 1): row i-1 gives q_i, the distribution d_{i+1}
+ *     was drafted from.   uniforms [B][n] in [0,1) (mode 1).
+ *   block_guesses [B][k][k] or NULL: slot guesses of mask block j (row j-1).
+ *
+ * Algorithm (n = max(k,1)):
+ *   j = 1; for i = 1..n-1: accept d_{i+1} iff
+ *     greedy:    d_{i+1} == argmax l_i (lowest index on ties)
+ *     rejection: u[i-1] * q_i(d_{i+1}) < p_i(d_{i+1})
+ *   and continue while accepted (j = i+1), stop at the first rejection.
+ *   The token t* at row j:
+ *     greedy: argmax l_j;
+ *     rejection, j < n: residual w = max(0, p_j - q_j) (all zero -> w = p_j);
+ *     rejection, j = n: w = p_j (bonus token);
+ *     t* = smallest t with u[n-1] * sum(w) < sum_{x<=t} w(x), summed in index order.
+ *   Emitted tokens: d_2..d_j, then t* (j tokens), -1 padded to n.
+ *   selected_block = j (0 when k = 0, which has no mask blocks).
+ *   next_drafts = [t*, g_{j,2}, .., g_{j,k}] (-1 where block_guesses is NULL).
+ *
+ * margins [B][n] (may be NULL), rejection only: entry i-1 is the relative
+ * distance |u q - p| / p of the i-th accept test (i <= j-1 accepted ones and the
+ * rejecting one), entry n-1 the distance of u*sum(w) to the nearest boundary of
+ * the cumulative sum, divided by sum(w).  Unused entries are +inf.  They let a
+ * test exclude decisions that differ only by summation order.
+ */
+int tidar_oracle_verify(int B, int k, int V, int dtype, int mode, const void* logits,
+                        const int32_t* drafts, const void* draft_logits, const float* uniforms,
+                        const int32_t* block_guesses, int32_t* accept_count, int32_t* out_tokens,
+                        int32_t* next_drafts, int32_t* selected_block, double* margins) {
+  const int n = k > 0 ? k : 1;
+  double *p, *qd, *w;
+  int b;
+  if (B < 0 || k < 0 || V <= 0 || (mode != 0 && mode != 1)) return ORACLE_ERR_ARG;
+  if (k > 1 && !drafts) return ORACLE_ERR_ARG;
+  if (mode == 1 && (!uniforms || (k > 1 && !draft_logits))) return ORACLE_ERR_ARG;
+  p = (double*)malloc(sizeof(double) * V);
+  qd = (double*)malloc(sizeof(double) * V);
+  w = (double*)malloc(sizeof(double) * V);
+  if (!p || !qd || !w) { free(p); free(qd); free(w); return ORACLE_ERR_ARG; }
+
+  for (b = 0; b < B; ++b) {
+    int i, j = 1, x, t_star = 0, e;
+    if (margins) for (i = 0; i < n; ++i) margins[(int64_t)b * n + i] = INFINITY;
+
+    /* accept scan, left to right */
+    for (i = 1; i <= n - 1; ++i) {
+      int d_next = drafts[(int64_t)b * k + i];   /* d_{i+1} */
+      int64_t lrow = ((int64_t)b * n + (i - 1)) * V;
+      int accept;
+      if (d_next < 0 || d_next >= V) { accept = 0; }
+      else if (mode == 0) {
+        accept = (d_next == argmax_row(logits, lrow, V, dtype));
+      } else {
+        double u = (double)uniforms[(int64_t)b * n + (i - 1)];
+        int64_t qrow = ((int64_t)b * (k - 1) + (i - 1)) * V;
+        softmax_row(logits, lrow, V, dtype, p);
+        softmax_row(draft_logits, qrow, V, dtype, qd);
+        accept = (u * qd[d_next] < p[d_next]);
+        if (margins)
+          margins[(int64_t)b * n + (i - 1)] = fabs(u * qd[d_next] - p[d_next]) / p[d_next];
+      }
+      if (!accept) break;
+      j = i + 1;
+    }
+
+    /* the token at row j */
+    {
+      int64_t lrow = ((int64_t)b * n + (j - 1)) * V;
+      if (mode == 0) {
+        t_star = argmax_row(logits, lrow, V, dtype);
+      } else {
+        double u = (double)uniforms[(int64_t)b * n + (n - 1)];
+        double total = 0.0, c = 0.0, target, prev = 0.0;
+        softmax_row(logits, lrow, V, dtype, p);
+        if (j < n) {
+          int64_t qrow = ((int64_t)b * (k - 1) + (j - 1)) * V;
+          softmax_row(draft_logits, qrow, V, dtype, qd);
+          for (x = 0; x < V; ++x) { double r = p[x] - qd[x]; w[x] = r > 0.0 ? r : 0.0; total += w[x]; }
+          if (!(total > 0.0)) { for (x = 0; x < V; ++x) w[x] = p[x]; total = 0.0; for (x = 0; x < V; ++x) total += w[x]; }
+        } else {
+          for (x = 0; x < V; ++x) { w[x] = p[x]; total += w[x]; }
+        }
+        target = u * total;
+        t_star = V - 1;
+        for (x = 0; x < V; ++x) {
+          prev = c;
+          c += w[x];
+          if (target < c) { t_star = x; break; }
+        }
+        if (margins) {
+          double lo = target - prev, hi = c - target;
+          margins[(int64_t)b * n + (n - 1)] = (lo < hi ? lo : hi) / total;
+        }
+      }
+    }
+
+    /* outputs */
+    accept_count[b] = j;
+    for (e = 0; e < n; ++e) out_tokens[(int64_t)b * n + e] = -1;
+    for (e = 0; e < j - 1; ++e) out_tokens[(int64_t)b * n + e] = drafts[(int64_t)b * k + e + 1];
+    out_tokens[(int64_t)b * n + j - 1] = t_star;
+    if (selected_block) selected_block[b] = k > 0 ? j : 0;
+    if (next_drafts && k > 0) {
+      next_drafts[(int64_t)b * k] = t_star;
+      for (e = 1; e < k; ++e)
+        next_drafts[(int64_t)b * k + e] =
+            block_guesses ? block_guesses[((int64_t)b * k + (j - 1)) * k + e] : -1;
+    }
+  }
+  free(p); free(qd); free(w);
+  return ORACLE_OK;
+}
+
+/*
+ * KV commit / evict ("the settled cache is reused, the rejected entries are
+ * evicted", [NDfr] paragraph on the three zones; exact KV cache, [MS] "KV
+ * Cache" and [FG] abstract).  Accepted drafts are always a prefix of the draft
+ * zone ([NDfr]: "only the first survives, two survive, all survive"), so no row
+ * moves.  For each b with c = accept_count[b] in 0..n:
+ *   rows P_b+c .. P_b+n-1 of every KV head are set to zero (K and V);
+ *   seq_lens[b] = P_b + c;
+ *   page-table entries i in [ceil((P_b+c)/ps), ceil((P_b+n)/ps)) -- the pages
+ *   that held only rejected draft rows -- are released: their ids are appended
+ *   to `released` in (b, i) order and the entries set to -1.
+ * `released` holds B*(ceil(n/ps)+1) entries, -1 padded; *num_released counts
+ * the ids written.  A sequence with c out of range, or whose draft rows are
+ * not mapped to valid pages, is left untouched and the call returns an error.
+ */
+int tidar_oracle_commit(int B, int Hkv, int D, int k, int page_size, int elem_bytes,
+                        void* k_pages, void* v_pages, int32_t* page_table, int max_pages,
+                        int num_pages, int32_t* seq_lens, const int32_t* accept_count,
+                        int32_t* released, int32_t* num_released) {
+  const int n = k > 0 ? k : 1;
+  const int cap = B * ((n + page_size - 1) / page_size + 1);
+  int b, status = ORACLE_OK, count = 0, e;
+  for (e = 0; e < cap; ++e) released[e] = -1;
+  for (b = 0; b < B; ++b) {
+    int P = seq_lens[b], c = accept_count[b], r, g, ok = 1;
+    int64_t i, first, last;
+    if (c < 0 || c > n) { status = ORACLE_ERR_COUNT; continue; }
+    for (r = 0; r < n && ok; ++r)
+      if (cache_row(page_table, max_pages, num_pages, page_size, Hkv, D, b, 0, (int64_t)P + r) < 0)
+        ok = 0;
+    if (!ok) { status = ORACLE_ERR_PAGE; continue; }
+    for (r = c; r < n; ++r) {
+      for (g = 0; g < Hkv; ++g) {
+        int64_t row = cache_row(page_table, max_pages, num_pages, page_size, Hkv, D, b, g,
+                                (int64_t)P + r);
+        memset((char*)k_pages + row * elem_bytes, 0, (size_t)D * elem_bytes);
+        memset((char*)v_pages + row * elem_bytes, 0, (size_t)D * elem_bytes);
+      }
+    }
+    seq_lens[b] = P + c;
+    first = ((int64_t)P + c + page_size - 1) / page_size;
+    last = ((int64_t)P + n + page_size - 1) / page_size;
+    for (i = first; i < last; ++i) {
+      int32_t* ent = &page_table[(int64_t)b * max_pages + i];
+      if (*ent >= 0) { released[count++] = *ent; *ent = -1; }
+    }
+  }
+  *num_released = count;
+  return status;
+}

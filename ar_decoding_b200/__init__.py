@@ -1,0 +1,237 @@
+"""Python binding of libtidar.so -- the GPU hot path of one TiDAR decode step.
+
+Argument marshalling only: tensors are passed to the C ABI (include/tidar.h)
+as raw device pointers with the current torch CUDA stream; every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback: if
+libtidar.so is missing or a call fails, an exception is raised.
+
+    out, lse = step_attn(q, k_blk, v_blk, cache, k, max_prefix_len=P)
+    res = verify(logits, drafts, k, "greedy", block_guesses=g)
+    released, n = commit(cache, res["accept_count"], k, max_prefix_len=P)
+
+``cache`` is a mapping with the device tensors ``k_pages``/``v_pages``
+[num_pages][Hkv][page][D], ``page_table`` [B][max_pages] int32 and
+``seq_lens`` [B] int32 (the layout ``synth.make_cache`` produces).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtidar.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "tidar.h")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(6)
+F32, BF16 = 0, 1
+GREEDY, REJECTION = 0, 1
+PATH_AUTO, PATH_SIMT, PATH_TC05 = 0, 1, 2
+DEVERR_BAD_PAGE, DEVERR_BAD_LEN, DEVERR_BAD_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
+_PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tc05": PATH_TC05}
+
+
+class TidarError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: status {status}")
+
+
+class StepDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("max_prefix_len", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("path", ctypes.c_int32)]
+
+
+class KVCacheDesc(ctypes.Structure):
+    _fields_ = [("k_pages", ctypes.c_void_p), ("v_pages", ctypes.c_void_p),
+                ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libtidar.so (built in-tree by ``python -m ar_decoding_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m ar_decoding_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+        L.tidar_step_attn_workspace_bytes.argtypes = [P]
+        L.tidar_step_attn_workspace_bytes.restype = S
+        L.tidar_step_attn.argtypes = [P, P, P, P, P, P, P, P, S, P]
+        L.tidar_step_attn.restype = ctypes.c_int
+        L.tidar_step_attn_plan.argtypes = [P, P, P]
+        L.tidar_step_attn_plan.restype = ctypes.c_int
+        L.tidar_verify_workspace_bytes.argtypes = [I, I, I, ctypes.c_int]
+        L.tidar_verify_workspace_bytes.restype = S
+        L.tidar_verify.argtypes = [I, I, I, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P, P, P,
+                                   S, P]
+        L.tidar_verify.restype = ctypes.c_int
+        L.tidar_commit.argtypes = [P, P, P, P, P, P]
+        L.tidar_commit.restype = ctypes.c_int
+        L.tidar_get_device_status.argtypes = [P, P]
+        L.tidar_get_device_status.restype = ctypes.c_int
+        L.tidar_status_string.argtypes = [ctypes.c_int]
+        L.tidar_status_string.restype = ctypes.c_char_p
+        L.tidar_last_cuda_error.argtypes = []
+        L.tidar_last_cuda_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/tidar.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(tidar_[a-z0-9_]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        L = lib()
+        msg = L.tidar_status_string(status).decode()
+        if status == ERR_CUDA:
+            msg += " (" + L.tidar_last_cuda_error().decode() + ")"
+        raise TidarError(status, f"{what} failed: {msg}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def make_desc(q, k_blk, cache, k, max_prefix_len, scale=0.0, path="auto") -> StepDesc:
+    B, R, Hq, D = q.shape
+    return StepDesc(batch=B, num_q_heads=Hq, num_kv_heads=k_blk.shape[2], head_dim=D, k=k,
+                    page_size=cache["k_pages"].shape[2], max_prefix_len=int(max_prefix_len),
+                    dtype=_dtype_code(q), softmax_scale=float(scale), path=_PATHS[path])
+
+
+def make_cache_desc(cache) -> KVCacheDesc:
+    for n in ("k_pages", "v_pages", "page_table", "seq_lens"):
+        _dev(cache[n], n)
+    if cache["page_table"].dtype != torch.int32 or cache["seq_lens"].dtype != torch.int32:
+        raise ValueError("page_table and seq_lens must be int32")
+    return KVCacheDesc(k_pages=cache["k_pages"].data_ptr(), v_pages=cache["v_pages"].data_ptr(),
+                       page_table=cache["page_table"].data_ptr(),
+                       seq_lens=cache["seq_lens"].data_ptr(),
+                       num_pages=cache["k_pages"].shape[0],
+                       max_pages_per_seq=cache["page_table"].shape[1])
+
+
+def plan(desc: StepDesc) -> tuple[int, int]:
+    path, splits = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().tidar_step_attn_plan(ctypes.byref(desc), ctypes.byref(path), ctypes.byref(splits)),
+           "tidar_step_attn_plan")
+    return path.value, splits.value
+
+
+def step_attn_workspace_bytes(desc: StepDesc) -> int:
+    return int(lib().tidar_step_attn_workspace_bytes(ctypes.byref(desc)))
+
+
+def step_attn(q, k_blk, v_blk, cache, k, *, max_prefix_len, scale=0.0, path="auto", out=None,
+              lse=None, want_lse=True, workspace=None, stream=None):
+    """Three-zone step attention (+ draft-row K/V append).  Returns (out, lse)."""
+    for t, n in ((q, "q"), (k_blk, "k_blk"), (v_blk, "v_blk")):
+        _dev(t, n)
+    desc = make_desc(q, k_blk, cache, k, max_prefix_len, scale, path)
+    cdesc = make_cache_desc(cache)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    need = step_attn_workspace_bytes(desc)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().tidar_step_attn(ctypes.byref(desc), ctypes.byref(cdesc), _ptr(q), _ptr(k_blk),
+                               _ptr(v_blk), _ptr(out), _ptr(lse), _ptr(workspace), wbytes,
+                               _stream_handle(stream))
+    _check(st, "tidar_step_attn")
+    return out, lse
+
+
+def verify_workspace_bytes(B, k, V, mode) -> int:
+    return int(lib().tidar_verify_workspace_bytes(B, k, V, mode))
+
+
+def verify(logits, drafts, k, mode="greedy", *, draft_logits=None, uniforms=None,
+           block_guesses=None, outputs=None, workspace=None, stream=None):
+    """Verification, acceptance and block selection.  Returns a dict of device tensors:
+    accept_count [B], out_tokens [B][n], next_drafts [B][k], selected_block [B]."""
+    m = mode if isinstance(mode, int) else {"greedy": GREEDY, "rejection": REJECTION}[mode]
+    _dev(logits, "logits")
+    B, n, V = logits.shape
+    dev = logits.device
+    if outputs is None:
+        outputs = dict(accept_count=torch.empty(B, dtype=torch.int32, device=dev),
+                       out_tokens=torch.empty((B, n), dtype=torch.int32, device=dev),
+                       next_drafts=torch.empty((B, max(k, 1)), dtype=torch.int32, device=dev),
+                       selected_block=torch.empty(B, dtype=torch.int32, device=dev))
+    need = verify_workspace_bytes(B, k, V, m)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    st = lib().tidar_verify(B, k, V, _dtype_code(logits), m, _ptr(logits), _ptr(drafts),
+                            _ptr(draft_logits), _ptr(uniforms), _ptr(block_guesses),
+                            _ptr(outputs["accept_count"]), _ptr(outputs["out_tokens"]),
+                            _ptr(outputs["next_drafts"]) if k > 0 else None,
+                            _ptr(outputs["selected_block"]), _ptr(workspace),
+                            workspace.numel(), _stream_handle(stream))
+    _check(st, "tidar_verify")
+    return outputs
+
+
+def commit(cache, accept_count, k, *, max_prefix_len, head_dim=None, num_q_heads=None,
+           released=None, num_released=None, stream=None):
+    """KV commit/evict in place.  Returns (released [B*(ceil(n/ps)+1)], num_released [1])."""
+    kp = cache["k_pages"]
+    B = cache["seq_lens"].shape[0]
+    Hkv, ps, D = kp.shape[1], kp.shape[2], kp.shape[3]
+    n = max(k, 1)
+    desc = StepDesc(batch=B, num_q_heads=num_q_heads or Hkv, num_kv_heads=Hkv, head_dim=D, k=k,
+                    page_size=ps, max_prefix_len=int(max_prefix_len), dtype=_dtype_code(kp),
+                    softmax_scale=0.0, path=PATH_AUTO)
+    cdesc = make_cache_desc(cache)
+    cap = B * ((n + ps - 1) // ps + 1)
+    if released is None:
+        released = torch.empty(cap, dtype=torch.int32, device=kp.device)
+    if num_released is None:
+        num_released = torch.empty(1, dtype=torch.int32, device=kp.device)
+    st = lib().tidar_commit(ctypes.byref(desc), ctypes.byref(cdesc), _ptr(accept_count),
+                            _ptr(released), _ptr(num_released), _stream_handle(stream))
+    _check(st, "tidar_commit")
+    return released, num_released
+
+
+def device_status(stream=None) -> tuple[int, int]:
+    """Synchronises the stream; returns (status, error bits) and clears the word."""
+    bits = ctypes.c_uint32()
+    st = lib().tidar_get_device_status(_stream_handle(stream), ctypes.byref(bits))
+    return st, bits.value

@@ -1,0 +1,290 @@
+// api.cu -- the C ABI of libtidar.so: argument checks, launch plans, launches.
+//
+// Every host-checkable condition is tested before anything is queued; the
+// kernels only re-check what depends on device-resident values (page ids,
+// lengths, accept counts) and report it through the per-device error word.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/tidar.h"
+#include "common.cuh"
+#include "kernels.h"
+
+// Per-device error word (one instance per device that loads the library).
+__device__ unsigned int g_tidar_error_word = 0;
+
+namespace {
+
+thread_local char g_cuda_msg[256] = "";
+constexpr int kMaxDevices = 64;
+unsigned int* g_err_ptr[kMaxDevices] = {nullptr};
+
+tidar_status cuda_fail(cudaError_t e) {
+  snprintf(g_cuda_msg, sizeof g_cuda_msg, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return TIDAR_ERR_CUDA;
+}
+
+// Device address of this device's error word (looked up once per device).
+tidar_status error_word(unsigned int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return TIDAR_ERR_UNSUPPORTED;
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_tidar_error_word);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_err_ptr[dev] = static_cast<unsigned int*>(p);
+  }
+  *out = g_err_ptr[dev];
+  return TIDAR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Shape checks shared by step_attn and commit.
+tidar_status check_desc(const tidar_step_desc* d) {
+  if (!d) return TIDAR_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 ||
+      d->num_q_heads % d->num_kv_heads != 0 || d->k < 0 || d->max_prefix_len < 0 ||
+      d->page_size <= 0)
+    return TIDAR_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return TIDAR_ERR_UNSUPPORTED;
+  if (d->k > 16) return TIDAR_ERR_UNSUPPORTED;
+  if (d->page_size != 16 && d->page_size != 32 && d->page_size != 64 && d->page_size != 128)
+    return TIDAR_ERR_UNSUPPORTED;
+  if (d->dtype != TIDAR_F32 && d->dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
+  if (d->path != TIDAR_PATH_AUTO && d->path != TIDAR_PATH_SIMT && d->path != TIDAR_PATH_TC05)
+    return TIDAR_ERR_INVALID_ARG;
+  return TIDAR_OK;
+}
+
+tidar_status check_cache(const tidar_step_desc* d, const tidar_kv_cache* c) {
+  if (!c) return TIDAR_ERR_INVALID_ARG;
+  const int n = d->k > 0 ? d->k : 1;
+  if (c->num_pages <= 0 || c->max_pages_per_seq <= 0) return TIDAR_ERR_INVALID_ARG;
+  const long long need = ((long long)d->max_prefix_len + n + d->page_size - 1) / d->page_size;
+  if (c->max_pages_per_seq < need) return TIDAR_ERR_INVALID_ARG;
+  if (!c->k_pages || !c->v_pages || !c->page_table || !c->seq_lens) return TIDAR_ERR_INVALID_ARG;
+  if (!aligned16(c->k_pages) || !aligned16(c->v_pages)) return TIDAR_ERR_INVALID_ARG;
+  return TIDAR_OK;
+}
+
+constexpr bool kTc05Built = false;
+
+bool tc05_supported(const tidar_step_desc* d) {
+  return kTc05Built && d->dtype == TIDAR_BF16 && d->head_dim == 128 && d->page_size == 64;
+}
+
+constexpr int kNumSMs = 148;
+
+struct Plan {
+  int path;    // 1 SIMT, 2 TC05
+  int nsplit;
+  int keys_per_split;
+};
+
+// Key ranges are multiples of 128 keys.  SIMT: aim for ~2 waves of 4-warp CTAs.
+// TC05: one CTA per (b, kv head, 128-row tile, split); aim for one wave.
+Plan make_plan(const tidar_step_desc* d, int path) {
+  Plan p;
+  p.path = path;
+  const int R = tidar::rows_per_seq(d->k);
+  const int G = d->num_q_heads / d->num_kv_heads;
+  const int M = R * G;
+  const int maxP = d->max_prefix_len;
+  const int blocks128 = (maxP + 127) / 128;
+  long long units;
+  int target;
+  if (path == 2) {
+    const int rows_per_tile = (128 / G) * G;
+    const int tiles = (M + rows_per_tile - 1) / rows_per_tile;
+    units = (long long)d->batch * d->num_kv_heads * tiles;
+    target = kNumSMs;
+  } else {
+    units = (long long)d->batch * d->num_kv_heads * ((M + 3) / 4);
+    target = 2 * kNumSMs * 4;
+  }
+  int ns = 1;
+  if (units > 0 && units < target) ns = (int)((target + units - 1) / units);
+  // at least 2 key blocks of 128 per split (tensor-core path), 1 for SIMT
+  const int min_blocks = path == 2 ? 2 : 1;
+  const int max_ns = blocks128 / min_blocks > 0 ? blocks128 / min_blocks : 1;
+  if (ns > max_ns) ns = max_ns;
+  if (ns > 64) ns = 64;
+  if (ns < 1) ns = 1;
+  const int bps = (blocks128 + ns - 1) / ns;
+  p.keys_per_split = (bps > 0 ? bps : 1) * 128;
+  p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
+  if (p.nsplit < 1) p.nsplit = 1;
+  return p;
+}
+
+int choose_path(const tidar_step_desc* d) {
+  if (d->path == TIDAR_PATH_SIMT) return 1;
+  if (d->path == TIDAR_PATH_TC05) return 2;
+  return tc05_supported(d) ? 2 : 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tidar_status_string(tidar_status s) {
+  switch (s) {
+    case TIDAR_OK: return "ok";
+    case TIDAR_ERR_INVALID_ARG: return "invalid argument";
+    case TIDAR_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TIDAR_ERR_CUDA: return "CUDA error";
+    case TIDAR_ERR_TIMEOUT: return "device-side wait timed out";
+    case TIDAR_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* tidar_last_cuda_error(void) { return g_cuda_msg; }
+
+tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, int32_t* splits) {
+  tidar_status st = check_desc(desc);
+  if (st != TIDAR_OK) return st;
+  const int pth = choose_path(desc);
+  if (pth == 2 && !tc05_supported(desc)) return TIDAR_ERR_UNSUPPORTED;
+  const Plan p = make_plan(desc, pth);
+  if (path) *path = p.path;
+  if (splits) *splits = p.nsplit;
+  return TIDAR_OK;
+}
+
+size_t tidar_step_attn_workspace_bytes(const tidar_step_desc* d) {
+  if (check_desc(d) != TIDAR_OK) return 0;
+  const int pth = choose_path(d);
+  const Plan p = make_plan(d, pth);
+  if (p.nsplit <= 1) return 0;
+  const size_t rows = (size_t)d->batch * tidar::rows_per_seq(d->k) * d->num_q_heads;
+  return align256((size_t)p.nsplit * rows * d->head_dim * sizeof(float)) +
+         align256((size_t)p.nsplit * rows * sizeof(float));
+}
+
+tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, const void* q,
+                             const void* k_blk, const void* v_blk, void* out, float* lse_out,
+                             void* workspace, size_t workspace_bytes, tidar_stream_t stream) {
+  tidar_status st = check_desc(d);
+  if (st != TIDAR_OK) return st;
+  if (d->batch == 0) return TIDAR_OK;
+  if ((st = check_cache(d, c)) != TIDAR_OK) return st;
+  if (!q || !k_blk || !v_blk || !out) return TIDAR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_blk) || !aligned16(v_blk) || !aligned16(out))
+    return TIDAR_ERR_INVALID_ARG;
+  const int pth = choose_path(d);
+  if (pth == 2 && !tc05_supported(d)) return TIDAR_ERR_UNSUPPORTED;
+  const Plan p = make_plan(d, pth);
+  const size_t need = tidar_step_attn_workspace_bytes(d);
+  if (workspace_bytes < need) return TIDAR_ERR_INVALID_ARG;
+  if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+    return TIDAR_ERR_INVALID_ARG;
+  unsigned int* err = nullptr;
+  if ((st = error_word(&err)) != TIDAR_OK) return st;
+
+  tidar::AttnArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = q; a.k_blk = k_blk; a.v_blk = v_blk;
+  a.k_pages = c->k_pages; a.v_pages = c->v_pages;
+  a.page_table = c->page_table; a.seq_lens = c->seq_lens;
+  a.out = out; a.lse_out = lse_out; a.err = err;
+  a.B = d->batch; a.Hq = d->num_q_heads; a.Hkv = d->num_kv_heads; a.G = a.Hq / a.Hkv;
+  a.D = d->head_dim; a.k = d->k; a.R = tidar::rows_per_seq(d->k); a.n = d->k > 0 ? d->k : 1;
+  a.page_size = d->page_size; a.max_pages = c->max_pages_per_seq; a.num_pages = c->num_pages;
+  a.max_prefix = d->max_prefix_len;
+  a.nsplit = p.nsplit; a.keys_per_split = p.keys_per_split;
+  a.bf16 = d->dtype == TIDAR_BF16;
+  a.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->head_dim);
+  if (p.nsplit > 1) {
+    const size_t rows = (size_t)a.B * a.R * a.Hq;
+    a.part_o = static_cast<float*>(workspace);
+    a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          align256((size_t)p.nsplit * rows * a.D * sizeof(float)));
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = pth == 2 ? tidar::launch_attn_tc05(a, s) : tidar::launch_attn_simt(a, s);
+  if (e == cudaErrorNotSupported) return TIDAR_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = tidar::launch_finalize(a, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
+size_t tidar_verify_workspace_bytes(int32_t batch, int32_t k, int32_t vocab, tidar_accept_mode mode) {
+  if (batch <= 0 || k < 0 || k > 16 || vocab <= 0) return 0;
+  return tidar::verify_workspace_bytes(batch, k, vocab, mode);
+}
+
+tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                          tidar_accept_mode mode, const void* logits, const int32_t* drafts,
+                          const void* draft_logits, const float* uniforms,
+                          const int32_t* block_guesses, int32_t* accept_count,
+                          int32_t* out_tokens, int32_t* next_drafts, int32_t* selected_block,
+                          void* workspace, size_t workspace_bytes, tidar_stream_t stream) {
+  if (batch < 0 || k < 0 || vocab <= 0) return TIDAR_ERR_INVALID_ARG;
+  if (k > 16) return TIDAR_ERR_UNSUPPORTED;
+  if (dtype != TIDAR_F32 && dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
+  if (mode != TIDAR_GREEDY && mode != TIDAR_REJECTION) return TIDAR_ERR_INVALID_ARG;
+  if (batch == 0) return TIDAR_OK;
+  if (!logits || !accept_count || !out_tokens) return TIDAR_ERR_INVALID_ARG;
+  if (k > 1 && !drafts) return TIDAR_ERR_INVALID_ARG;
+  if (mode == TIDAR_REJECTION && (!uniforms || (k > 1 && !draft_logits)))
+    return TIDAR_ERR_INVALID_ARG;
+  const size_t need = tidar::verify_workspace_bytes(batch, k, vocab, mode);
+  if (workspace_bytes < need || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return TIDAR_ERR_INVALID_ARG;
+  tidar::VerifyArgs a;
+  a.B = batch; a.k = k; a.n = k > 0 ? k : 1; a.V = vocab; a.bf16 = dtype == TIDAR_BF16; a.mode = mode;
+  a.logits = logits; a.drafts = drafts; a.draft_logits = draft_logits; a.uniforms = uniforms;
+  a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;
+  a.next_drafts = next_drafts; a.selected_block = selected_block; a.workspace = workspace;
+  cudaError_t e = tidar::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
+tidar_status tidar_commit(const tidar_step_desc* d, const tidar_kv_cache* c,
+                          const int32_t* accept_count, int32_t* released_pages,
+                          int32_t* num_released, tidar_stream_t stream) {
+  tidar_status st = check_desc(d);
+  if (st != TIDAR_OK) return st;
+  if (d->batch == 0) return TIDAR_OK;
+  if ((st = check_cache(d, c)) != TIDAR_OK) return st;
+  if (!accept_count || !released_pages || !num_released) return TIDAR_ERR_INVALID_ARG;
+  unsigned int* err = nullptr;
+  if ((st = error_word(&err)) != TIDAR_OK) return st;
+  tidar::CommitArgs a;
+  a.B = d->batch; a.Hkv = d->num_kv_heads; a.D = d->head_dim; a.k = d->k; a.n = d->k > 0 ? d->k : 1;
+  a.page_size = d->page_size; a.elem_bytes = d->dtype == TIDAR_BF16 ? 2 : 4;
+  a.max_pages = c->max_pages_per_seq; a.num_pages = c->num_pages;
+  a.k_pages = c->k_pages; a.v_pages = c->v_pages; a.page_table = c->page_table;
+  a.seq_lens = c->seq_lens; a.accept_count = accept_count; a.released = released_pages;
+  a.num_released = num_released; a.err = err;
+  cudaError_t e = tidar::launch_commit(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
+tidar_status tidar_get_device_status(tidar_stream_t stream, uint32_t* bits_out) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned int bits = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&bits, g_tidar_error_word, sizeof bits);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (bits) {
+    e = cudaMemcpyToSymbol(g_tidar_error_word, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (bits_out) *bits_out = bits;
+  if (bits & TIDAR_DEVERR_TIMEOUT) return TIDAR_ERR_TIMEOUT;
+  if (bits) return TIDAR_ERR_DEVICE;
+  return TIDAR_OK;
+}
+
+}  // extern "C"

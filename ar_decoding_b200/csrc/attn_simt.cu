@@ -1,0 +1,203 @@
+// attn_simt.cu -- CUDA-core step attention, split-KV merge and draft-row append.
+//
+// The step attention of one TiDAR decode step ("TiDAR: Think in Diffusion,
+// Talk in Autoregression", mauroscia.it, section 2 "Single Forward Pass &
+// Structured Attention Mask"; nodesdaily.com (fr), paragraphs on the three
+// zones and on the masking puzzle): every query row attends the whole cached
+// prefix plus the step keys its zone may see.
+//
+// This is the fp32 path (the tiny workload needs 1e-5 agreement, so no tf32
+// tensor cores) and the general fallback for shapes the tensor-core kernel
+// does not take.  One warp owns one packed query row (b, rho, h); lanes split
+// the head dimension; keys are visited in order with an online softmax in
+// fp32 (accurate expf).  Split-KV: blockIdx.y selects a contiguous key range;
+// the last split also takes the step keys.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tidar {
+
+namespace {
+
+constexpr int kWarps = 4;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(AttnArgs a) {
+  constexpr int VPL = D / 32;  // elements per lane
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int bg = blockIdx.z;
+  const int b = bg / a.Hkv, g = bg % a.Hkv;
+  const int M = a.R * a.G;
+  const int m = blockIdx.x * kWarps + warp;
+  if (m >= M) return;
+  const int rho = m / a.G, h = g * a.G + m % a.G;
+  const int split = blockIdx.y;
+
+  int P = a.seq_lens[b];
+  if (P < 0 || P > a.max_prefix) {
+    if (lane == 0 && split == 0 && m == 0) raise_error(a.err, TIDAR_DEVERR_BAD_LEN);
+    P = 0;
+  }
+
+  const T* qp = static_cast<const T*>(a.q) + ((size_t)(b * a.R + rho) * a.Hq + h) * D + lane * VPL;
+  float qv[VPL];
+  load_vec<T, VPL>(qp, qv);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) qv[i] *= a.scale;
+
+  float mx = -INFINITY, l = 0.f, acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+
+  auto update = [&](const T* kp, const T* vp) {
+    float kv[VPL], vv[VPL];
+    load_vec<T, VPL>(kp, kv);
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) dot = fmaf(qv[i], kv[i], dot);
+    const float s = warp_sum(dot);
+    load_vec<T, VPL>(vp, vv);
+    const float mn = fmaxf(mx, s);
+    const float corr = expf(mx - mn);   // 0 on the first key (mx = -inf)
+    const float pe = expf(s - mn);
+    l = fmaf(l, corr, pe);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] = fmaf(acc[i], corr, pe * vv[i]);
+    mx = mn;
+  };
+
+  // prefix keys of this split
+  const int k0 = split * a.keys_per_split;
+  const int k1 = min(P, k0 + a.keys_per_split);
+  const T* kpages = static_cast<const T*>(a.k_pages);
+  const T* vpages = static_cast<const T*>(a.v_pages);
+  const int32_t* table = a.page_table + (size_t)b * a.max_pages;
+  bool bad_page = false;
+  for (int key = k0; key < k1; ++key) {
+    const int page = table[key / a.page_size];
+    if (page < 0 || page >= a.num_pages) { bad_page = true; continue; }
+    const size_t off = ((size_t)(page * a.Hkv + g) * a.page_size + key % a.page_size) * D + lane * VPL;
+    update(kpages + off, vpages + off);
+  }
+  if (bad_page && lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
+
+  // step keys (drafts and mask slots), last split only
+  if (split == a.nsplit - 1) {
+    const StepVis vis = step_visibility(a.k, rho);
+    const T* kb = static_cast<const T*>(a.k_blk);
+    const T* vb = static_cast<const T*>(a.v_blk);
+    for (int key = 0; key < a.R; ++key) {
+      if (!step_visible(vis, key)) continue;
+      const size_t off = ((size_t)(b * a.R + key) * a.Hkv + g) * D + lane * VPL;
+      update(kb + off, vb + off);
+    }
+  }
+
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  float o[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) o[i] = acc[i] * inv;
+  const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
+  const float lse = l > 0.f ? mx + logf(l) : -INFINITY;
+  if (a.nsplit == 1) {
+    store_vec<T, VPL>(static_cast<T*>(a.out) + row * D + lane * VPL, o);
+    if (a.lse_out && lane == 0) a.lse_out[row] = lse;
+  } else {
+    const size_t prow = (size_t)split * a.B * a.R * a.Hq + row;
+    store_vec<float, VPL>(a.part_o + prow * D + lane * VPL, o);
+    if (lane == 0) a.part_lse[prow] = lse;
+  }
+}
+
+// Merge the split partials (weights exp(lse_s - max)) and, in the blocks past
+// the merge, copy the draft rows' K/V into the cache at P_b .. P_b+n-1.
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32) finalize_kernel(AttnArgs a, int merge_blocks) {
+  constexpr int VPL = D / 32;
+  if ((int)blockIdx.x < merge_blocks) {
+    const int lane = threadIdx.x & 31;
+    const size_t rows = (size_t)a.B * a.R * a.Hq;
+    const size_t row = (size_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    float mx = -INFINITY;
+    for (int s = 0; s < a.nsplit; ++s) mx = fmaxf(mx, a.part_lse[s * rows + row]);
+    float acc[VPL], wsum = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+    if (mx > -INFINITY) {
+      for (int s = 0; s < a.nsplit; ++s) {
+        const float ls = a.part_lse[s * rows + row];
+        if (ls == -INFINITY) continue;
+        const float w = expf(ls - mx);
+        float v[VPL];
+        load_vec<float, VPL>(a.part_o + (s * rows + row) * D + lane * VPL, v);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+        wsum += w;
+      }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] *= inv;
+    store_vec<T, VPL>(static_cast<T*>(a.out) + row * D + lane * VPL, acc);
+    if (a.lse_out && lane == 0) a.lse_out[row] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+    return;
+  }
+  // draft-row append: one block per (b, r)
+  const int idx = blockIdx.x - merge_blocks;
+  const int b = idx / a.n, r = idx % a.n;
+  const int P = a.seq_lens[b];
+  if (P < 0 || P > a.max_prefix) return;   // reported by the attention kernel
+  const int pos = P + r;
+  const int page = a.page_table[(size_t)b * a.max_pages + pos / a.page_size];
+  if (page < 0 || page >= a.num_pages) {
+    if (threadIdx.x == 0) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
+    return;
+  }
+  constexpr int kVec = 16 / sizeof(T);     // elements per 16-byte chunk
+  const int chunks = a.Hkv * D / kVec;     // per K (and per V) row
+  for (int c = threadIdx.x; c < 2 * chunks; c += blockDim.x) {
+    const int which = c / chunks, cc = c % chunks;
+    const int g = cc / (D / kVec), e = (cc % (D / kVec)) * kVec;
+    const T* src = static_cast<const T*>(which ? a.v_blk : a.k_blk) +
+                   ((size_t)(b * a.R + r) * a.Hkv + g) * D + e;
+    T* dst = static_cast<T*>(const_cast<void*>(which ? a.v_pages : a.k_pages)) +
+             ((size_t)(page * a.Hkv + g) * a.page_size + pos % a.page_size) * D + e;
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_simt_t(const AttnArgs& a, cudaStream_t s) {
+  const int M = a.R * a.G;
+  dim3 grid((M + kWarps - 1) / kWarps, a.nsplit, a.B * a.Hkv);
+  attn_simt_kernel<T, D><<<grid, kWarps * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_finalize_t(const AttnArgs& a, cudaStream_t s) {
+  const size_t rows = (size_t)a.B * a.R * a.Hq;
+  const int merge_blocks = a.nsplit > 1 ? (int)((rows + kWarps - 1) / kWarps) : 0;
+  const int blocks = merge_blocks + a.B * a.n;
+  if (blocks == 0) return cudaSuccess;
+  finalize_kernel<T, D><<<blocks, kWarps * 32, 0, s>>>(a, merge_blocks);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s) {
+  if (a.bf16) return a.D == 64 ? launch_simt_t<__nv_bfloat16, 64>(a, s) : launch_simt_t<__nv_bfloat16, 128>(a, s);
+  return a.D == 64 ? launch_simt_t<float, 64>(a, s) : launch_simt_t<float, 128>(a, s);
+}
+
+cudaError_t launch_finalize(const AttnArgs& a, cudaStream_t s) {
+  if (a.bf16) return a.D == 64 ? launch_finalize_t<__nv_bfloat16, 64>(a, s) : launch_finalize_t<__nv_bfloat16, 128>(a, s);
+  return a.D == 64 ? launch_finalize_t<float, 64>(a, s) : launch_finalize_t<float, 128>(a, s);
+}
+
+}  // namespace tidar

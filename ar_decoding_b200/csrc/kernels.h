@@ -1,0 +1,66 @@
+// kernels.h -- host-side launch interface between api.cu and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tidar {
+
+// Everything a step-attention kernel needs, in device pointers and sizes.
+struct AttnArgs {
+  const void* q;
+  const void* k_blk;
+  const void* v_blk;
+  const void* k_pages;
+  const void* v_pages;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  void* out;
+  float* lse_out;        // may be null
+  float* part_o;         // [nsplit][B][R][Hq][D] fp32 (nsplit > 1)
+  float* part_lse;       // [nsplit][B][R][Hq]  fp32 (nsplit > 1)
+  unsigned int* err;     // device error word
+  int B, Hq, Hkv, G, D, k, R, n, page_size, max_pages, num_pages, max_prefix;
+  int nsplit, keys_per_split;
+  int bf16;              // 1: bf16 tensors, 0: fp32
+  float scale;           // softmax scale (natural-log domain)
+};
+
+// CUDA-core kernel (fp32 or bf16, D 64 or 128).
+cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
+// tcgen05/TMEM kernel (bf16, D 128, page 64).  Returns cudaErrorNotSupported if
+// the tensor maps cannot be built.
+cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s);
+// Split merge (when nsplit > 1) and the draft-row append, in one launch.
+cudaError_t launch_finalize(const AttnArgs& a, cudaStream_t s);
+
+struct VerifyArgs {
+  int B, k, n, V, bf16, mode;
+  const void* logits;
+  const int32_t* drafts;
+  const void* draft_logits;
+  const float* uniforms;
+  const int32_t* block_guesses;
+  int32_t* accept_count;
+  int32_t* out_tokens;
+  int32_t* next_drafts;
+  int32_t* selected_block;
+  void* workspace;
+};
+size_t verify_workspace_bytes(int B, int k, int V, int mode);
+cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s);
+
+struct CommitArgs {
+  int B, Hkv, D, k, n, page_size, elem_bytes, max_pages, num_pages;
+  void* k_pages;
+  void* v_pages;
+  int32_t* page_table;
+  int32_t* seq_lens;
+  const int32_t* accept_count;
+  int32_t* released;
+  int32_t* num_released;
+  unsigned int* err;
+};
+cudaError_t launch_commit(const CommitArgs& a, cudaStream_t s);
+
+}  // namespace tidar

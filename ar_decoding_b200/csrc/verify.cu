@@ -1,0 +1,408 @@
+// verify.cu -- fused verification / acceptance / block selection over vocab rows.
+//
+// "Talk in Autoregression": the carried drafts are scored strictly left to
+// right under the AR distribution (nodesdaily.com (fr), paragraph on betting
+// on every outcome; mauroscia.it section 1: a good draft is accepted, a bad
+// one corrected), so the emitted text follows plain AR sampling exactly
+// (engineer-news.pages.dev, section "TiDAR 在做什麼").  The rejection rule is
+// the speculative-sampling rule of TiDAR's lineage (Leviathan et al., Chen et
+// al., listed on the mauroscia.it page).  The same scan picks the pre-drafted
+// mask block that matches the accept count.
+//
+// Layout of the work (vocab rows are HBM/latency bound; nothing here is a
+// contraction):
+//   stats:     grid (chunks, rows).  One CTA sweeps CHUNK logits of one row with
+//              16-byte loads: exact max / argmax (lowest index on ties) and,
+//              for rejection, the fp64 sum of exp(x - chunk max).
+//   greedy:    grid (B).  Merges the chunk argmaxes, scans, writes outputs.
+//   rejection: residual (grid (chunks, B)) recomputes the row normalisers from
+//              the chunk stats, runs the accept scan (fp64), and sums the
+//              sampling weights of its chunk; select (grid (B)) locates the
+//              inverse-CDF chunk, scans it in fp64 and writes outputs.
+#include <climits>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tidar {
+
+namespace {
+
+constexpr int kChunk = 4096;
+constexpr int kThreads = 256;
+constexpr int kPer = kChunk / kThreads;   // 16 elements per thread
+
+struct ChunkStat {
+  float max;
+  int arg;
+  double sum;   // sum exp(x - max) over the chunk (rejection only)
+};
+
+template <typename T>
+__device__ __forceinline__ float ld(const T* p, int i) { return to_f32(p[i]); }
+
+// Exact argmax merge: larger value wins, equal values -> lower index.
+__device__ __forceinline__ void amax_merge(float& v, int& i, float v2, int i2) {
+  if (v2 > v || (v2 == v && i2 < i)) { v = v2; i = i2; }
+}
+
+// Loads this thread's kPer elements of the chunk (index order t*8.., strided by
+// 8*kThreads for 16-byte vector loads when the row is vector aligned).
+template <typename T>
+__device__ __forceinline__ int load_chunk(const T* row, int V, int c0, float (&x)[kPer],
+                                          int (&ix)[kPer], bool vec_ok) {
+  constexpr int kVec = 16 / sizeof(T);
+  int cnt = 0;
+  if (vec_ok) {
+#pragma unroll
+    for (int it = 0; it < kPer / kVec; ++it) {
+      const int base = c0 + (it * kThreads + threadIdx.x) * kVec;
+      if (base + kVec <= V) {
+        float v[kVec];
+        load_vec<T, kVec>(row + base, v);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) { x[it * kVec + e] = v[e]; ix[it * kVec + e] = base + e; }
+      } else {
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) {
+          const int id = base + e;
+          x[it * kVec + e] = id < V ? ld(row, id) : -INFINITY;
+          ix[it * kVec + e] = id < V ? id : INT_MAX;
+        }
+      }
+    }
+    cnt = kPer;
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int id = c0 + e * kThreads + threadIdx.x;
+      x[e] = id < V ? ld(row, id) : -INFINITY;
+      ix[e] = id < V ? id : INT_MAX;
+    }
+    cnt = kPer;
+  }
+  return cnt;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat* stats, int nchunk,
+                                                         bool vec_ok) {
+  const int c = blockIdx.x, rr = blockIdx.y;
+  const int prow = a.B * a.n;
+  const T* row = rr < prow ? static_cast<const T*>(a.logits) + (size_t)rr * a.V
+                           : static_cast<const T*>(a.draft_logits) + (size_t)(rr - prow) * a.V;
+  float x[kPer];
+  int ix[kPer];
+  load_chunk<T>(row, a.V, c * kChunk, x, ix, vec_ok);
+  float bv = -INFINITY;
+  int bi = INT_MAX;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) amax_merge(bv, bi, x[e], ix[e]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+    amax_merge(bv, bi, v2, i2);
+  }
+  __shared__ float sv[kThreads / 32];
+  __shared__ int si[kThreads / 32];
+  __shared__ double sd[kThreads / 32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) { sv[w] = bv; si[w] = bi; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < kThreads / 32; ++i) amax_merge(bv, bi, sv[i], si[i]);
+    sv[0] = bv; si[0] = bi;
+  }
+  __syncthreads();
+  const float cmax = sv[0];
+  const int carg = si[0];
+  double sum = 0.0;
+  if (a.mode == TIDAR_REJECTION) {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e)
+      if (ix[e] != INT_MAX) sum += exp((double)x[e] - (double)cmax);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) sd[w] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      sum = 0.0;
+      for (int i = 0; i < kThreads / 32; ++i) sum += sd[i];
+    }
+  }
+  if (threadIdx.x == 0) {
+    ChunkStat st;
+    st.max = cmax; st.arg = carg; st.sum = sum;
+    stats[(size_t)rr * nchunk + c] = st;
+  }
+}
+
+// Writes accept_count, out_tokens, selected_block, next_drafts for sequence b.
+__device__ void write_outputs(const VerifyArgs& a, int b, int j, int t_star) {
+  a.accept_count[b] = j;
+  for (int e = 0; e < a.n; ++e) {
+    int v = -1;
+    if (e < j - 1) v = a.drafts[(size_t)b * a.k + e + 1];
+    else if (e == j - 1) v = t_star;
+    a.out_tokens[(size_t)b * a.n + e] = v;
+  }
+  if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
+  if (a.next_drafts && a.k > 0) {
+    a.next_drafts[(size_t)b * a.k] = t_star;
+    for (int e = 1; e < a.k; ++e)
+      a.next_drafts[(size_t)b * a.k + e] =
+          a.block_guesses ? a.block_guesses[((size_t)b * a.k + (j - 1)) * a.k + e] : -1;
+  }
+}
+
+__global__ void greedy_kernel(VerifyArgs a, const ChunkStat* stats, int nchunk) {
+  const int b = blockIdx.x;
+  __shared__ int am[16];
+  if ((int)threadIdx.x < a.n) {
+    const ChunkStat* st = stats + ((size_t)b * a.n + threadIdx.x) * nchunk;
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    for (int c = 0; c < nchunk; ++c) amax_merge(bv, bi, st[c].max, st[c].arg);
+    am[threadIdx.x] = bi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int j = 1;
+    for (int i = 1; i <= a.n - 1; ++i) {
+      if (a.drafts[(size_t)b * a.k + i] != am[i - 1]) break;
+      j = i + 1;
+    }
+    write_outputs(a, b, j, am[j - 1]);
+  }
+}
+
+// Row normaliser from chunk stats: M = max of chunk maxima, Z = sum_c
+// exp(max_c - M) * sum_c (fp64).
+__device__ void row_norm(const ChunkStat* st, int nchunk, double& M, double& Z) {
+  float mf = -INFINITY;
+  for (int c = 0; c < nchunk; ++c) mf = fmaxf(mf, st[c].max);
+  M = (double)mf;
+  Z = 0.0;
+  for (int c = 0; c < nchunk; ++c) Z += exp((double)st[c].max - M) * st[c].sum;
+}
+
+// The accept scan for sequence b under the rejection rule; returns j.
+template <typename T>
+__device__ int rejection_scan(const VerifyArgs& a, int b, const ChunkStat* stats, int nchunk) {
+  const int prow = a.B * a.n;
+  int j = 1;
+  for (int i = 1; i <= a.n - 1; ++i) {
+    const int d = a.drafts[(size_t)b * a.k + i];
+    if (d < 0 || d >= a.V) break;
+    double Mp, Zp, Mq, Zq;
+    const size_t lrow = (size_t)b * a.n + (i - 1);
+    const size_t qrow = (size_t)b * (a.k - 1) + (i - 1);
+    row_norm(stats + lrow * nchunk, nchunk, Mp, Zp);
+    row_norm(stats + (prow + qrow) * nchunk, nchunk, Mq, Zq);
+    const double p = exp((double)ld(static_cast<const T*>(a.logits) + lrow * a.V, d) - Mp) / Zp;
+    const double q = exp((double)ld(static_cast<const T*>(a.draft_logits) + qrow * a.V, d) - Mq) / Zq;
+    const double u = (double)a.uniforms[(size_t)b * a.n + (i - 1)];
+    if (!(u * q < p)) break;
+    j = i + 1;
+  }
+  return j;
+}
+
+// Per (chunk, b): the sampling weights' chunk sums for both candidate weight
+// laws -- residual max(0, p_j - q_j) (when j < n) and p_j itself.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const ChunkStat* stats,
+                                                            int nchunk, double* wsum, int* jbuf,
+                                                            bool vec_ok) {
+  const int c = blockIdx.x, b = blockIdx.y;
+  __shared__ int sj;
+  __shared__ double sMp, sZp, sMq, sZq;
+  if (threadIdx.x == 0) {
+    const int j = rejection_scan<T>(a, b, stats, nchunk);
+    sj = j;
+    if (c == 0) jbuf[b] = j;
+    row_norm(stats + ((size_t)b * a.n + (j - 1)) * nchunk, nchunk, sMp, sZp);
+    if (j < a.n) {
+      const size_t qrow = (size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1);
+      row_norm(stats + qrow * nchunk, nchunk, sMq, sZq);
+    }
+  }
+  __syncthreads();
+  const int j = sj;
+  const T* prow = static_cast<const T*>(a.logits) + ((size_t)b * a.n + (j - 1)) * a.V;
+  float xp[kPer];
+  int ix[kPer];
+  load_chunk<T>(prow, a.V, c * kChunk, xp, ix, vec_ok);
+  double sr = 0.0, sp = 0.0;
+  const double Mp = sMp, Zp = sZp;
+  if (j < a.n) {
+    const T* qrow = static_cast<const T*>(a.draft_logits) + ((size_t)b * (a.k - 1) + (j - 1)) * a.V;
+    float xq[kPer];
+    int iq[kPer];
+    load_chunk<T>(qrow, a.V, c * kChunk, xq, iq, vec_ok);
+    const double Mq = sMq, Zq = sZq;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      if (ix[e] == INT_MAX) continue;
+      const double p = exp((double)xp[e] - Mp) / Zp;
+      const double q = exp((double)xq[e] - Mq) / Zq;
+      const double r = p - q;
+      sr += r > 0.0 ? r : 0.0;
+      sp += p;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      if (ix[e] == INT_MAX) continue;
+      sp += exp((double)xp[e] - Mp) / Zp;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sr += __shfl_xor_sync(0xffffffffu, sr, o);
+    sp += __shfl_xor_sync(0xffffffffu, sp, o);
+  }
+  __shared__ double s1[kThreads / 32], s2[kThreads / 32];
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) { s1[w] = sr; s2[w] = sp; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    sr = 0.0; sp = 0.0;
+    for (int i = 0; i < kThreads / 32; ++i) { sr += s1[i]; sp += s2[i]; }
+    wsum[((size_t)b * nchunk + c) * 2 + 0] = sr;
+    wsum[((size_t)b * nchunk + c) * 2 + 1] = sp;
+  }
+}
+
+// Inverse CDF: smallest t with u*sum(w) < sum_{x<=t} w(x).  Chunk located from
+// the chunk sums; inside the chunk an fp64 block scan in index order.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const ChunkStat* stats,
+                                                          int nchunk, const double* wsum,
+                                                          const int* jbuf) {
+  const int b = blockIdx.x;
+  const int j = jbuf[b];
+  __shared__ int s_chunk, s_resid, s_found;
+  __shared__ double s_target, sMp, sZp, sMq, sZq;
+  __shared__ double s_scan[kThreads];
+  if (threadIdx.x == 0) {
+    double tr = 0.0, tp = 0.0;
+    for (int c = 0; c < nchunk; ++c) { tr += wsum[((size_t)b * nchunk + c) * 2]; tp += wsum[((size_t)b * nchunk + c) * 2 + 1]; }
+    const int resid = (j < a.n) && (tr > 0.0);
+    const double total = resid ? tr : tp;
+    const double target = (double)a.uniforms[(size_t)b * a.n + (a.n - 1)] * total;
+    double cum = 0.0;
+    int ch = nchunk - 1;
+    for (int c = 0; c < nchunk; ++c) {
+      const double wc = wsum[((size_t)b * nchunk + c) * 2 + (resid ? 0 : 1)];
+      if (target < cum + wc) { ch = c; break; }
+      cum += wc;
+      if (c == nchunk - 1) cum -= wc;   // not found: scan the last chunk
+    }
+    s_chunk = ch;
+    s_resid = resid;
+    s_target = target - cum;
+    s_found = INT_MAX;
+    row_norm(stats + ((size_t)b * a.n + (j - 1)) * nchunk, nchunk, sMp, sZp);
+    if (resid) row_norm(stats + ((size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1)) * nchunk, nchunk, sMq, sZq);
+  }
+  __syncthreads();
+  const int c0 = s_chunk * kChunk;
+  const T* prow = static_cast<const T*>(a.logits) + ((size_t)b * a.n + (j - 1)) * a.V;
+  const T* qrow = s_resid ? static_cast<const T*>(a.draft_logits) + ((size_t)b * (a.k - 1) + (j - 1)) * a.V : nullptr;
+  // contiguous kPer elements per thread so a block scan gives index order
+  double w[kPer];
+  double tsum = 0.0;
+  int last_nz = -1;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int id = c0 + threadIdx.x * kPer + e;
+    double v = 0.0;
+    if (id < a.V) {
+      const double p = exp((double)ld(prow, id) - sMp) / sZp;
+      if (s_resid) {
+        const double q = exp((double)ld(qrow, id) - sMq) / sZq;
+        v = p - q > 0.0 ? p - q : 0.0;
+      } else {
+        v = p;
+      }
+      if (v > 0.0) last_nz = id;
+    }
+    w[e] = v;
+    tsum += v;
+  }
+  s_scan[threadIdx.x] = tsum;
+  __syncthreads();
+  // Hillis-Steele inclusive scan over the per-thread sums
+  for (int off = 1; off < kThreads; off <<= 1) {
+    const double v = threadIdx.x >= (unsigned)off ? s_scan[threadIdx.x - off] : 0.0;
+    __syncthreads();
+    s_scan[threadIdx.x] += v;
+    __syncthreads();
+  }
+  double cum = threadIdx.x ? s_scan[threadIdx.x - 1] : 0.0;
+  const double target = s_target;
+  int hit = INT_MAX;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int id = c0 + threadIdx.x * kPer + e;
+    cum += w[e];
+    if (hit == INT_MAX && id < a.V && target < cum) hit = id;
+  }
+  if (hit != INT_MAX) atomicMin(&s_found, hit);
+  __shared__ int s_last;
+  if (threadIdx.x == 0) s_last = -1;
+  __syncthreads();
+  if (last_nz >= 0) atomicMax(&s_last, last_nz);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = s_found;
+    if (t == INT_MAX) t = s_last >= 0 ? s_last : min(c0 + kChunk, a.V) - 1;
+    write_outputs(a, b, j, t);
+  }
+}
+
+template <typename T>
+cudaError_t launch_t(const VerifyArgs& a, cudaStream_t s) {
+  const int nchunk = (a.V + kChunk - 1) / kChunk;
+  const bool vec_ok = ((size_t)a.V * sizeof(T)) % 16 == 0;
+  ChunkStat* stats = static_cast<ChunkStat*>(a.workspace);
+  const int rows = a.B * a.n + (a.mode == TIDAR_REJECTION ? a.B * (a.k > 1 ? a.k - 1 : 0) : 0);
+  stats_kernel<T><<<dim3(nchunk, rows), kThreads, 0, s>>>(a, stats, nchunk, vec_ok);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.mode == TIDAR_GREEDY) {
+    greedy_kernel<<<a.B, 32, 0, s>>>(a, stats, nchunk);
+    return cudaGetLastError();
+  }
+  char* base = static_cast<char*>(a.workspace) + (((size_t)rows * nchunk * sizeof(ChunkStat) + 255) & ~(size_t)255);
+  double* wsum = reinterpret_cast<double*>(base);
+  int* jbuf = reinterpret_cast<int*>(base + (((size_t)a.B * nchunk * 2 * sizeof(double) + 255) & ~(size_t)255));
+  residual_kernel<T><<<dim3(nchunk, a.B), kThreads, 0, s>>>(a, stats, nchunk, wsum, jbuf, vec_ok);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  select_kernel<T><<<a.B, kThreads, 0, s>>>(a, stats, nchunk, wsum, jbuf);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t verify_workspace_bytes(int B, int k, int V, int mode) {
+  const size_t nchunk = (V + kChunk - 1) / kChunk;
+  const int n = k > 0 ? k : 1;
+  const size_t rows = (size_t)B * n + (mode == TIDAR_REJECTION ? (size_t)B * (k > 1 ? k - 1 : 0) : 0);
+  size_t bytes = ((rows * nchunk * sizeof(ChunkStat) + 255) & ~(size_t)255);
+  if (mode == TIDAR_REJECTION) {
+    bytes += (((size_t)B * nchunk * 2 * sizeof(double) + 255) & ~(size_t)255);
+    bytes += (((size_t)B * sizeof(int) + 255) & ~(size_t)255);
+  }
+  return bytes;
+}
+
+cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s) {
+  return a.bf16 ? launch_t<__nv_bfloat16>(a, s) : launch_t<float>(a, s);
+}
+
+}  // namespace tidar

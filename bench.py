@@ -1,0 +1,480 @@
+"""Benchmark of one TiDAR decode step on B200: step attention (three zones over a
+paged bf16 GQA KV cache, plus the draft-row append), greedy verification with
+block selection, and the KV commit -- all through the C ABI of libtidar.so.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: 8B-class heads (32 q / 8 kv, head_dim 128, bf16), prefix 8192, k = 16
+(16 draft rows + 16 blocks of 16 mask slots = 272 query rows), verification over
+vocab 32768 logits N(0,3) with each draft equal to the row argmax w.p. 0.7.
+Inputs are seeded synthetic tensors generated on the device.  One rank per GPU
+(torchrun); every rank runs its own independent sequence (weak scaling, no
+collective on the data path).
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
+cudaDeviceSynchronize; each step is timed on the device with CUDA events on the
+launching stream, and rotates over enough independent input/cache copies that
+each step's working set is evicted from L2 (126 MB) before it is reused.
+Between steps (outside the events) the copy's prefix length and page table are
+restored so every step does identical work.  ms_per_step / value is the mean
+step time, max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "TiDAR step latency (µs) and achieved HBM GB/s vs draft length k"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--k", type=int, default=16)
+    ap.add_argument("--prefix", type=int, default=8192)
+    ap.add_argument("--no-sweep", action="store_true", help="skip the k sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc05"])
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- setup
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def workload(k: int, prefix: int, rank: int = 0):
+    from ar_decoding_b200 import synth
+    return synth.class_8b(seed=synth.SEED_BASE + 2 + 1000 * rank, k=k, prefix=prefix)
+
+
+def step_key_counts(k: int) -> int:
+    """Visible step keys summed over the rows of one sequence: draft row r sees r
+    drafts; a slot of block j sees j drafts and the k slots of its block."""
+    if k == 0:
+        return 1
+    return k * (k + 1) // 2 + k * sum(j + k for j in range(1, k + 1))
+
+
+def algorithmic(cfg):
+    """Bytes that must move and flops of one step attention: KV prefix read, Q read
+    and O write, step K/V read, draft-row append write; flops 4*D per (row, head,
+    visible key) for QK^T and PV."""
+    e = cfg.elem_bytes
+    P = sum(cfg.prefix)
+    kv = P * cfg.Hkv * cfg.D * 2 * e
+    qo = 2 * cfg.B * cfg.R * cfg.Hq * cfg.D * e
+    stepkv = cfg.B * cfg.R * cfg.Hkv * cfg.D * 2 * e
+    append = cfg.B * cfg.n * cfg.Hkv * cfg.D * 2 * e
+    vis = sum(cfg.R * p + step_key_counts(cfg.k) for p in cfg.prefix)
+    flops = 4 * cfg.D * cfg.Hq * vis
+    return kv + qo + stepkv + append, flops
+
+
+class Step:
+    """Device-resident inputs for `copies` independent instances of the workload,
+    and one decode step (attention, verify, commit) on a chosen copy."""
+
+    def __init__(self, cfg, copies, path="auto"):
+        import ar_decoding_b200 as tidar
+        from ar_decoding_b200 import synth
+        self.tidar, self.cfg, self.path = tidar, cfg, path
+        dev = torch.device("cuda")
+        self.copies = []
+        for c in range(copies):
+            cc = synth.StepConfig(**{**cfg.__dict__, "seed": cfg.seed + 17 * c})
+            cache = synth.make_cache(cc, device=dev)
+            step = synth.make_step(cc, device=dev)
+            vin = synth.make_verify(cc, "greedy")
+            self.copies.append(dict(
+                cache=cache, step=step,
+                logits=vin["logits"].to(dev), drafts=vin["drafts"].to(dev),
+                guesses=vin["block_guesses"].to(dev),
+                seq0=cache["seq_lens"].clone(), pt0=cache["page_table"].clone()))
+        self.max_prefix = max(cfg.prefix)
+        c0 = self.copies[0]
+        self.desc = tidar.make_desc(c0["step"]["q"], c0["step"]["k_blk"], c0["cache"], cfg.k,
+                                    self.max_prefix, path=path)
+        self.path_id, self.splits = tidar.plan(self.desc)
+        need = tidar.step_attn_workspace_bytes(self.desc)
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        self.out = torch.empty_like(c0["step"]["q"])
+        self.lse = torch.empty(c0["step"]["q"].shape[:3], dtype=torch.float32, device=dev)
+        B, n, V = c0["logits"].shape
+        self.vws = torch.empty(max(tidar.verify_workspace_bytes(B, cfg.k, V, 0), 256),
+                               dtype=torch.uint8, device=dev)
+        self.vout = dict(accept_count=torch.empty(B, dtype=torch.int32, device=dev),
+                         out_tokens=torch.empty((B, n), dtype=torch.int32, device=dev),
+                         next_drafts=torch.empty((B, max(cfg.k, 1)), dtype=torch.int32, device=dev),
+                         selected_block=torch.empty(B, dtype=torch.int32, device=dev))
+        cap = cfg.B * ((cfg.n + cfg.page_size - 1) // cfg.page_size + 1)
+        self.rel = torch.empty(cap, dtype=torch.int32, device=dev)
+        self.nrel = torch.empty(1, dtype=torch.int32, device=dev)
+        self.launches_per_step = 2 + 2 + 2   # attention+finalize, stats+accept, scrub+compact
+
+    def attn(self, i):
+        c = self.copies[i]
+        self.tidar.step_attn(c["step"]["q"], c["step"]["k_blk"], c["step"]["v_blk"], c["cache"],
+                             self.cfg.k, max_prefix_len=self.max_prefix, path=self.path,
+                             out=self.out, lse=self.lse, workspace=self.ws)
+
+    def verify_commit(self, i):
+        c = self.copies[i]
+        self.tidar.verify(c["logits"], c["drafts"], self.cfg.k, "greedy",
+                          block_guesses=c["guesses"], outputs=self.vout, workspace=self.vws)
+        self.tidar.commit(c["cache"], self.vout["accept_count"], self.cfg.k,
+                          max_prefix_len=self.max_prefix, released=self.rel,
+                          num_released=self.nrel)
+
+    def restore(self, i):
+        c = self.copies[i]
+        c["cache"]["seq_lens"].copy_(c["seq0"], non_blocking=True)
+        c["cache"]["page_table"].copy_(c["pt0"], non_blocking=True)
+
+
+def copies_for(cfg):
+    per = algorithmic(cfg)[0] + cfg.B * cfg.n * cfg.vocab * cfg.elem_bytes
+    return max(3, math.ceil(3 * L2_BYTES / per))
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.proc = None
+        self.index = index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- timing
+def time_steps(st: Step, K: int, W: int, world: int):
+    """Returns per-step device µs and per-step step_attn µs (lists)."""
+    n = len(st.copies)
+    stream = torch.cuda.current_stream()
+    for i in range(W):
+        st.attn(i % n); st.verify_commit(i % n); st.restore(i % n)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(K):
+        c = (W + i) % n
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        st.attn(c)
+        e1.record(stream)
+        st.verify_commit(c)
+        e2.record(stream)
+        st.restore(c)
+    torch.cuda.synchronize()
+    barrier(world)
+    step_us = [e0.elapsed_time(e2) * 1e3 for e0, _, e2 in ev]
+    attn_us = [e0.elapsed_time(e1) * 1e3 for e0, e1, _ in ev]
+    return step_us, attn_us
+
+
+def time_e2e(st: Step, K: int, W: int):
+    """Same step through the public API with host buffers: the step's inputs are
+    copied from pinned host memory and the verification results read back, inside
+    the timed region.  Returns (µs per step, h2d bytes, d2h bytes)."""
+    c = st.copies[0]
+    host_in = {k: v.cpu().pin_memory() for k, v in
+               (("q", c["step"]["q"]), ("k_blk", c["step"]["k_blk"]), ("v_blk", c["step"]["v_blk"]),
+                ("logits", c["logits"]), ("drafts", c["drafts"]), ("guesses", c["guesses"]))}
+    host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in st.vout.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    stream = torch.cuda.current_stream()
+
+    def one():
+        c["step"]["q"].copy_(host_in["q"], non_blocking=True)
+        c["step"]["k_blk"].copy_(host_in["k_blk"], non_blocking=True)
+        c["step"]["v_blk"].copy_(host_in["v_blk"], non_blocking=True)
+        c["logits"].copy_(host_in["logits"], non_blocking=True)
+        c["drafts"].copy_(host_in["drafts"], non_blocking=True)
+        c["guesses"].copy_(host_in["guesses"], non_blocking=True)
+        st.attn(0)
+        st.verify_commit(0)
+        for k2 in host_out:
+            host_out[k2].copy_(st.vout[k2], non_blocking=True)
+
+    for _ in range(W):
+        one(); st.restore(0)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        one()
+        e1.record(stream)
+        st.restore(0)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    return statistics.mean(ts), h2d, d2h
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_step_seconds(cfg, row_fraction=1.0, threads=0):
+    """Wall time of the oracle doing one step (attention over a fraction of the
+    rows, verification and commit), scaled to the full step."""
+    import numpy as np
+    import oracle
+    from ar_decoding_b200 import synth
+    cache, step = synth.make_cache(cfg), synth.make_step(cfg)
+    vin = synth.make_verify(cfg, "greedy")
+    n = synth.to_np
+    npc = {k: n(v) for k, v in cache.items()}
+    nps = {k: n(v) for k, v in step.items()}
+    rows = [(b, r, h) for b in range(cfg.B) for r in range(cfg.R) for h in range(cfg.Hq)]
+    take = max(1, int(round(len(rows) * row_fraction)))
+    idx = np.linspace(0, len(rows) - 1, take).round().astype(int)
+    sel = [rows[i] for i in idx]
+    t0 = time.perf_counter()
+    oracle.step_attn(nps["q"], nps["k_blk"], nps["v_blk"], npc["k_pages"], npc["v_pages"],
+                     npc["page_table"], npc["seq_lens"], cfg.k, sel=None if take == len(rows) else sel,
+                     num_threads=threads)
+    t_attn = (time.perf_counter() - t0) * len(rows) / take
+    t0 = time.perf_counter()
+    kp, vp = oracle.append(npc["k_pages"], npc["v_pages"], npc["page_table"], npc["seq_lens"],
+                           nps["k_blk"], nps["v_blk"], cfg.k)
+    res = oracle.verify(n(vin["logits"]), n(vin["drafts"]), cfg.k, oracle.GREEDY,
+                        block_guesses=n(vin["block_guesses"]))
+    oracle.commit(kp, vp, npc["page_table"], npc["seq_lens"], res["accept_count"], cfg.k)
+    t_rest = time.perf_counter() - t0
+    return t_attn + t_rest, take, len(rows)
+
+
+def oracle_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- main
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cfg = workload(args.k, args.prefix)
+    cores = oracle_threads()
+    # each step: the oracle on an evenly spaced fraction of the query rows (plus
+    # the whole verification and commit), scaled to one full step
+    frac = 0.25
+    times = []
+    for i in range(args.warmup + args.steps):
+        t, take, total = oracle_step_seconds(cfg, frac)
+        if i >= args.warmup:
+            times.append(t)
+    us = statistics.mean(times) * 1e6
+    sample = (f"oracle on {take} of {total} (b,row,head) attention rows per step (scaled x{total / take:.2f}),"
+              f" full verify+append+commit; {cores} OpenMP threads")
+    line = {"impl": "reference", "metric": METRIC, "value": us, "unit": "us", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": "8B-class TiDAR step", "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv,
+                       "head_dim": cfg.D, "prefix": args.prefix, "k": args.k, "rows": cfg.R,
+                       "vocab": cfg.vocab},
+            "cpu_baseline": {"value": us, "unit": "us", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local):
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    tc_peak = peaks.get("bf16_tflops", 1590.0)
+    peak_src = "measured" if peaks else "fallback"
+
+    cfg = workload(args.k, args.prefix, rank)
+    st = Step(cfg, copies_for(cfg), path=args.path)
+    clocks = ClockSampler(local)
+    clocks.start()
+    step_us, attn_us = time_steps(st, args.steps, args.warmup, world)
+    clk = clocks.stop()
+    mean_step = reduce_max(statistics.mean(step_us), world)
+    mean_attn = reduce_max(statistics.mean(attn_us), world)
+    bytes_, flops = algorithmic(cfg)
+    t_mem = bytes_ / (hbm_peak * 1e9)
+    t_tc = flops / (tc_peak * 1e12)
+    attn_s = mean_attn * 1e-6
+    bound = "tensor" if t_tc > t_mem else "hbm"
+    if bound == "tensor":
+        achieved, peak, unit = flops / attn_s / 1e12, tc_peak, "TFLOP/s"
+    else:
+        achieved, peak, unit = bytes_ / attn_s / 1e9, hbm_peak, "GB/s"
+    e2e_us, h2d, d2h = time_e2e(st, max(5, args.steps // 2), 2)
+    e2e_us = reduce_max(e2e_us, world)
+
+    sweep = []
+    if not args.no_sweep:
+        for kk in (0, 4, 8, 16):
+            c2 = workload(kk, args.prefix, rank)
+            s2 = Step(c2, copies_for(c2), path=args.path)
+            su, au = time_steps(s2, max(10, args.steps // 2), 3, world)
+            b2, f2 = algorithmic(c2)
+            a2 = reduce_max(statistics.mean(au), world) * 1e-6
+            sweep.append({"k": kk, "rows": c2.R, "step_us": reduce_max(statistics.mean(su), world),
+                          "attn_us": a2 * 1e6, "attn_hbm_gbs": b2 / a2 / 1e9,
+                          "hbm_frac": (b2 / a2 / 1e9) / hbm_peak,
+                          "tc_frac": (f2 / a2 / 1e12) / tc_peak,
+                          "roofline_frac": max(b2 / (hbm_peak * 1e9), f2 / (tc_peak * 1e12)) / a2,
+                          "path": "tc05" if s2.path_id == 2 else "simt", "splits": s2.splits})
+            del s2
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, take, total = oracle_step_seconds(cfg, 1.0)
+        cores = oracle_threads()
+        cpu = {"value": t * 1e6, "unit": "us", "cores": cores, "kind": "oracle",
+               "sample": f"one full step of the same workload ({total} attention rows, verify, "
+                         f"append, commit) on {cores} OpenMP threads"}
+
+    agg_gbs = reduce_sum(bytes_ / attn_s / 1e9, world)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": mean_step, "unit": "us", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_step / 1e3,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, generated on device)",
+            "config": {"workload": "8B-class TiDAR step", "B_per_gpu": cfg.B, "Hq": cfg.Hq,
+                       "Hkv": cfg.Hkv, "head_dim": cfg.D, "prefix": args.prefix, "k": args.k,
+                       "rows": cfg.R, "vocab": cfg.vocab, "page": cfg.page_size,
+                       "l2": f"rotating {len(st.copies)} independent input copies (> 3x L2)",
+                       "attn_path": "tc05" if st.path_id == 2 else "simt",
+                       "splits": st.splits},
+            "attn_us": mean_attn, "hbm_gbs_attn": bytes_ / attn_s / 1e9,
+            "hbm_gbs_all_gpus": agg_gbs,
+            "roofline": {"kernel": "tidar_step_attn", "bound": bound, "achieved": achieved,
+                         "peak": peak, "unit": unit, "frac": achieved / peak,
+                         "peak_source": peak_src, "traffic": None,
+                         "algorithmic_bytes": bytes_, "algorithmic_flops": flops,
+                         "roofline_frac_max_of_both": max(t_mem, t_tc) / attn_s},
+            "k_sweep": sweep,
+            "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": st.launches_per_step * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

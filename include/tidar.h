@@ -1,0 +1,212 @@
+/*
+ * tidar.h -- C ABI of libtidar.so, the GPU hot path of one TiDAR decode step.
+ *
+ * The method ("TiDAR: Think in Diffusion, Talk in Autoregression", arXiv
+ * 2511.08923) is described on these pages, cited below by tag:
+ *   [MS]   "TiDAR: Think in Diffusion, Talk in Autoregression" (mauroscia.it)
+ *   [NDfr] "TiDAR : l'hybride de NVIDIA qui rédige par diffusion et parle de
+ *          manière autorégressive" (nodesdaily.com, French)
+ *   [FG]   "論文の概要: TiDAR: Think in Diffusion, Talk in Autoregression"
+ *          (fugumt.com; the paper's abstract)
+ *   [EN]   "TiDAR：Nvidia 的擴散＋自回歸混合架構——把閒置的 GPU 算力換成推論加速"
+ *          (engineer-news.pages.dev)
+ *
+ * One step = tidar_step_attn (one attention pass over three zones, plus the
+ * speculative write of the draft rows' K/V), then tidar_verify (left-to-right
+ * acceptance and selection of the matching pre-drafted block), then
+ * tidar_commit (keep the accepted drafts' cache rows, evict the rest).
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless stated otherwise, on the device
+ *     that is current when the call is made.  The caller owns every buffer
+ *     (cache, tables, inputs, outputs, workspace); the library allocates no
+ *     device memory.  Its only state is a per-device error word (see
+ *     tidar_get_device_status).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and returns after the launches are queued.
+ *   - Argument errors the host can see are returned before anything is
+ *     launched.  Errors that depend on device-resident values (page ids, prefix
+ *     lengths, accept counts) set bits in the device error word; the affected
+ *     work is skipped (outputs of that row/sequence are unspecified but
+ *     finite) and tidar_get_device_status reports them.  Nothing traps.
+ *   - Floating-point tensors are fp32 (TIDAR_F32) or bf16 (TIDAR_BF16),
+ *     row-major, contiguous, 16-byte aligned.
+ *
+ * Shapes (B batch, Hq query heads, Hkv KV heads, G = Hq/Hkv, D head_dim,
+ * k draft length in 0..16, n = max(k,1), R = k + k*k rows per sequence, R = 1
+ * when k = 0):
+ *   query rows of a sequence, in order: the k carried-over drafts d_1..d_k
+ *   (row r-1 for d_r), then mask block j = 1..k, slot s = 1..k at row
+ *   k + (j-1)k + (s-1).  The step keys/values use the same row indices.
+ */
+#ifndef TIDAR_H
+#define TIDAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tidar_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  TIDAR_OK = 0,
+  TIDAR_ERR_INVALID_ARG = 1, /* a host-checkable argument is wrong; nothing launched */
+  TIDAR_ERR_UNSUPPORTED = 2, /* valid but not implemented (dtype/head_dim/page size/path) */
+  TIDAR_ERR_CUDA = 3,        /* a CUDA runtime call failed (message via tidar_last_cuda_error) */
+  TIDAR_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (device error word) */
+  TIDAR_ERR_DEVICE = 5       /* a device-side check failed (device error word) */
+} tidar_status;
+
+typedef enum { TIDAR_F32 = 0, TIDAR_BF16 = 1 } tidar_dtype;
+typedef enum { TIDAR_GREEDY = 0, TIDAR_REJECTION = 1 } tidar_accept_mode;
+
+/* Kernel family for the step attention.  AUTO: tcgen05/TMEM tensor-core
+ * kernel for bf16, head_dim 128, page 64; CUDA-core kernel otherwise. */
+typedef enum { TIDAR_PATH_AUTO = 0, TIDAR_PATH_SIMT = 1, TIDAR_PATH_TC05 = 2 } tidar_attn_path;
+
+/* Bits of the device error word. */
+#define TIDAR_DEVERR_BAD_PAGE 0x1u      /* a needed page-table entry is -1 or >= num_pages */
+#define TIDAR_DEVERR_BAD_LEN 0x2u       /* seq_lens[b] < 0 or > max_prefix_len */
+#define TIDAR_DEVERR_BAD_COUNT 0x4u     /* accept_count[b] outside 0..n (commit) */
+#define TIDAR_DEVERR_TIMEOUT 0x8u       /* a bounded mbarrier wait ran out */
+
+typedef struct {
+  int32_t batch;          /* B >= 0 (0: every call is a no-op) */
+  int32_t num_q_heads;    /* Hq */
+  int32_t num_kv_heads;   /* Hkv, divides Hq; query head h reads KV head h / (Hq/Hkv) */
+  int32_t head_dim;       /* D: 64 or 128 */
+  int32_t k;              /* draft length, 0..16 */
+  int32_t page_size;      /* rows per cache page: 16, 32, 64 or 128 (tensor-core path: 64) */
+  int32_t max_prefix_len; /* upper bound on every seq_lens[b]; sizes the KV split */
+  tidar_dtype dtype;      /* of q, k_blk, v_blk, out and the cache */
+  float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim) */
+  tidar_attn_path path;   /* TIDAR_PATH_AUTO unless a test pins a kernel family */
+} tidar_step_desc;
+
+typedef struct {
+  void* k_pages;             /* [num_pages][Hkv][page_size][D], dtype */
+  void* v_pages;             /* same layout */
+  int32_t* page_table;       /* [batch][max_pages_per_seq]: page id of rows
+                                [i*page_size, (i+1)*page_size) of sequence b, -1 = none */
+  int32_t* seq_lens;         /* [batch]: P_b, the committed (settled) prefix length */
+  int32_t num_pages;
+  int32_t max_pages_per_seq; /* >= ceil((max_prefix_len + n) / page_size) */
+} tidar_kv_cache;
+
+/* ---------------------------------------------------------------------------
+ * Step attention.  [MS] §2 "Single Forward Pass & Structured Attention Mask"
+ * (three zones: causal prefix, verified drafts, bidirectional pre-drafts);
+ * [NDfr] paragraphs on the three zones, on betting on every outcome (one mask
+ * block per possible accept count) and on the masking puzzle (drafts strictly
+ * causal, each block fully visible inside and seeing the whole settled past;
+ * the mask depends only on zone-relative positions, so it slides forward).
+ *
+ * For sequence b, query head h (KV head g = h / G) and row rho:
+ *   out[b][rho][h] = sum over visible keys x of softmax_x(<q, K_x> * scale) V_x
+ * where the visible keys are the prefix rows 0..P_b-1 of the paged cache and
+ * the step keys chosen by the mask:
+ *   draft row r (rho = r-1):          D_1..D_r
+ *   slot (j, s) of mask block j:      D_1..D_j and M_{j,1..k} (its whole block)
+ *   k = 0 (one row):                  D_1 (itself)
+ * lse_out (optional) receives the natural-log normaliser log(sum exp(score)).
+ *
+ * The same call writes the step rows' K/V of the drafts (rows 0..n-1 of k_blk,
+ * v_blk) into cache rows P_b .. P_b+n-1 (the pages must already be reserved in
+ * page_table); tidar_commit later keeps the accepted ones.  The attention
+ * itself reads only cache rows < P_b.
+ *
+ *   q        [B][R][Hq][D]     k_blk, v_blk [B][R][Hkv][D]     (dtype)
+ *   out      [B][R][Hq][D]     (dtype)     lse_out [B][R][Hq] fp32 or NULL
+ *   workspace: device scratch of at least tidar_step_attn_workspace_bytes(desc)
+ *     bytes, 256-byte aligned (may be NULL when that size is 0); contents on
+ *     entry are ignored.  Calls that share a workspace must be stream-ordered.
+ * Device errors: BAD_PAGE (prefix or draft page unmapped), BAD_LEN.
+ * ------------------------------------------------------------------------- */
+size_t tidar_step_attn_workspace_bytes(const tidar_step_desc* desc);
+tidar_status tidar_step_attn(const tidar_step_desc* desc, const tidar_kv_cache* cache,
+                             const void* q, const void* k_blk, const void* v_blk, void* out,
+                             float* lse_out, void* workspace, size_t workspace_bytes,
+                             tidar_stream_t stream);
+
+/* The launch plan the library would use: kernel family (1 SIMT, 2 tensor
+ * core) and number of KV splits.  Host only, no device access. */
+tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, int32_t* splits);
+
+/* ---------------------------------------------------------------------------
+ * Verification, acceptance and selection.  [NDfr] paragraph on betting on
+ * every outcome (strict left-to-right scoring of the carried drafts; a guess
+ * block is waiting for whichever outcome verification confirms); [MS] §1
+ * (a good draft is accepted, a bad one corrected); [EN] section "TiDAR 在做什麼"
+ * and [NDfr] last paragraph (output identical to AR sampling).  The rejection
+ * rule is the speculative-sampling rule of the work [MS] lists as TiDAR's
+ * lineage (Leviathan et al., Chen et al.).
+ *
+ * With n = max(k,1) and row i of `logits` the AR distribution p_i of the token
+ * after d_1..d_i:
+ *   j = 1; for i = 1..n-1, accept d_{i+1} iff
+ *     greedy:    d_{i+1} == argmax logits_i (lowest index on ties)
+ *     rejection: u[i-1] * q_i(d_{i+1}) < p_i(d_{i+1})       (fp64)
+ *   and stop at the first rejection; j = 1 + accepted count.
+ *   t* at row j: greedy argmax; rejection: inverse CDF (smallest t with
+ *   u[n-1]*sum(w) < sum_{x<=t} w) of w = max(0, p_j - q_j) after a rejection
+ *   (w = p_j if that is all zero) or w = p_j when every draft was accepted.
+ *   accept_count[b] = j; out_tokens[b] = d_2..d_j, t*, then -1 up to n;
+ *   selected_block[b] = j (0 when k = 0); next_drafts[b] = t*, g_{j,2..k}.
+ * Probabilities in the rejection test and the inverse CDF are computed in
+ * fp64 (softmax with the row maximum subtracted).  Logits must be finite.
+ *
+ *   logits        [B][n][V] dtype         drafts [B][k] int32 (NULL if k == 0)
+ *   draft_logits  [B][k-1][V] dtype, rejection only (q_i is row i-1)
+ *   uniforms      [B][n] fp32 in [0,1), rejection only
+ *   block_guesses [B][k][k] int32 slot guesses of each mask block, or NULL
+ *   accept_count  [B] int32      out_tokens [B][n] int32
+ *   next_drafts   [B][k] int32 or NULL      selected_block [B] int32 or NULL
+ *   workspace: at least tidar_verify_workspace_bytes(...) bytes, 256-aligned.
+ * A draft token outside [0, V) is never accepted.
+ * ------------------------------------------------------------------------- */
+size_t tidar_verify_workspace_bytes(int32_t batch, int32_t k, int32_t vocab,
+                                    tidar_accept_mode mode);
+tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                          tidar_accept_mode mode, const void* logits, const int32_t* drafts,
+                          const void* draft_logits, const float* uniforms,
+                          const int32_t* block_guesses, int32_t* accept_count,
+                          int32_t* out_tokens, int32_t* next_drafts, int32_t* selected_block,
+                          void* workspace, size_t workspace_bytes, tidar_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * KV commit / evict, in place.  [NDfr] paragraph on the three zones (the
+ * settled cache is reused, rejected entries are evicted); [MS] "KV Cache" and
+ * [FG] abstract (exact KV cache).  Accepted drafts are a prefix of the draft
+ * zone ([NDfr]: the futures run from only the first kept to all kept), so no row
+ * moves.  For each b with c = accept_count[b] in 0..n and P = seq_lens[b]:
+ *   cache rows P+c .. P+n-1 (every KV head, K and V) are zeroed;
+ *   seq_lens[b] = P + c;
+ *   page_table[b][i] for i in [ceil((P+c)/ps), ceil((P+n)/ps)) -- pages that
+ *   held only rejected draft rows -- are set to -1 and their ids returned.
+ *   released_pages: [B * (ceil(n/ps) + 1)] int32, the released ids in
+ *     (b, i) order, then -1; num_released: [1] int32.
+ * tidar_verify produces c in 1..n; c = 0 (evict every draft row) is allowed.
+ * Device errors: BAD_COUNT (c out of range) or BAD_PAGE (a draft row without
+ * a valid page): that sequence is left untouched.
+ * ------------------------------------------------------------------------- */
+tidar_status tidar_commit(const tidar_step_desc* desc, const tidar_kv_cache* cache,
+                          const int32_t* accept_count, int32_t* released_pages,
+                          int32_t* num_released, tidar_stream_t stream);
+
+/* Synchronises `stream`, reads and clears this device's error word.  Returns
+ * TIDAR_ERR_TIMEOUT if the timeout bit was set, TIDAR_ERR_DEVICE for any other
+ * bit, TIDAR_ERR_CUDA if the synchronisation failed, else TIDAR_OK.  bits_out
+ * (host pointer, may be NULL) receives the raw bits. */
+tidar_status tidar_get_device_status(tidar_stream_t stream, uint32_t* bits_out);
+
+const char* tidar_status_string(tidar_status status);
+/* Text of the last CUDA error seen by this thread's calls (host string). */
+const char* tidar_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TIDAR_H */

@@ -1,0 +1,126 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports every
+function include/tidar.h declares, and rejects bad arguments before launching
+anything.  Device pointers here are fake aligned addresses; every call below
+fails validation before any pointer could be used."""
+import ctypes
+
+import pytest
+
+import ar_decoding_b200 as tidar
+from ar_decoding_b200 import build
+
+FAKE = 0x10000          # aligned, never dereferenced
+MISALIGNED = 0x10008
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return tidar.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = tidar.header_functions()
+    assert {"tidar_step_attn", "tidar_verify", "tidar_commit", "tidar_get_device_status"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def _desc(**kw):
+    d = dict(batch=1, num_q_heads=4, num_kv_heads=2, head_dim=128, k=4, page_size=64,
+             max_prefix_len=100, dtype=tidar.BF16, softmax_scale=0.0, path=tidar.PATH_AUTO)
+    d.update(kw)
+    return tidar.StepDesc(**d)
+
+
+def _cache(**kw):
+    c = dict(k_pages=FAKE, v_pages=FAKE, page_table=FAKE, seq_lens=FAKE, num_pages=8,
+             max_pages_per_seq=2)
+    c.update(kw)
+    return tidar.KVCacheDesc(**c)
+
+
+def _attn(L, desc, cache, q=FAKE, out=FAKE, ws=None, wsb=0):
+    return L.tidar_step_attn(ctypes.byref(desc) if desc is not None else None,
+                             ctypes.byref(cache) if cache is not None else None,
+                             q, FAKE, FAKE, out, None, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_q_heads=3), tidar.ERR_INVALID_ARG),          # Hq not a multiple of Hkv
+    (dict(head_dim=96), tidar.ERR_UNSUPPORTED),
+    (dict(k=17), tidar.ERR_UNSUPPORTED),
+    (dict(k=-1), tidar.ERR_INVALID_ARG),
+    (dict(page_size=48), tidar.ERR_UNSUPPORTED),
+    (dict(dtype=7), tidar.ERR_UNSUPPORTED),
+    (dict(path=9), tidar.ERR_INVALID_ARG),
+    (dict(max_prefix_len=-5), tidar.ERR_INVALID_ARG),
+    (dict(max_prefix_len=1000), tidar.ERR_INVALID_ARG),    # table too short for it
+])
+def test_step_attn_rejects_bad_desc(L, kw, status):
+    assert _attn(L, _desc(**kw), _cache()) == status
+
+
+def test_step_attn_rejects_null_and_misaligned(L):
+    assert _attn(L, None, _cache()) == tidar.ERR_INVALID_ARG
+    assert _attn(L, _desc(), None) == tidar.ERR_INVALID_ARG
+    assert _attn(L, _desc(), _cache(), q=None) == tidar.ERR_INVALID_ARG
+    assert _attn(L, _desc(), _cache(), q=MISALIGNED) == tidar.ERR_INVALID_ARG
+    assert _attn(L, _desc(), _cache(k_pages=MISALIGNED)) == tidar.ERR_INVALID_ARG
+    assert _attn(L, _desc(), _cache(num_pages=0)) == tidar.ERR_INVALID_ARG
+
+
+def test_step_attn_rejects_small_workspace(L):
+    d = _desc(max_prefix_len=8192, batch=1, num_q_heads=32, num_kv_heads=8, k=0)
+    c = _cache(max_pages_per_seq=129)
+    need = L.tidar_step_attn_workspace_bytes(ctypes.byref(d))
+    assert need > 0
+    assert _attn(L, d, c, ws=FAKE, wsb=need - 1) == tidar.ERR_INVALID_ARG
+    assert _attn(L, d, c, ws=FAKE + 16, wsb=need) == tidar.ERR_INVALID_ARG   # not 256-aligned
+
+
+def test_batch_zero_is_a_noop(L):
+    assert _attn(L, _desc(batch=0), None) == tidar.OK
+
+
+def test_verify_rejects_bad_args(L):
+    V = L.tidar_verify
+    ws = L.tidar_verify_workspace_bytes(2, 4, 512, tidar.REJECTION)
+    args = lambda **kw: dict(dict(B=2, k=4, V=512, dt=tidar.F32, mode=tidar.REJECTION, logits=FAKE,
+                                  drafts=FAKE, dl=FAKE, u=FAKE, acc=FAKE, toks=FAKE, ws=FAKE,
+                                  wsb=ws), **kw)
+    def call(a):
+        return V(a["B"], a["k"], a["V"], a["dt"], a["mode"], a["logits"], a["drafts"], a["dl"],
+                 a["u"], None, a["acc"], a["toks"], None, None, a["ws"], a["wsb"], None)
+    assert call(args(k=17)) == tidar.ERR_UNSUPPORTED
+    assert call(args(V=0)) == tidar.ERR_INVALID_ARG
+    assert call(args(dl=None)) == tidar.ERR_INVALID_ARG
+    assert call(args(u=None)) == tidar.ERR_INVALID_ARG
+    assert call(args(drafts=None)) == tidar.ERR_INVALID_ARG
+    assert call(args(wsb=ws - 1)) == tidar.ERR_INVALID_ARG
+    assert call(args(ws=FAKE + 8)) == tidar.ERR_INVALID_ARG
+    assert call(args(mode=5)) == tidar.ERR_INVALID_ARG
+    assert call(args(B=0)) == tidar.OK
+
+
+def test_commit_rejects_bad_args(L):
+    d, c = _desc(), _cache()
+    assert L.tidar_commit(ctypes.byref(d), ctypes.byref(c), None, FAKE, FAKE, None) == tidar.ERR_INVALID_ARG
+    assert L.tidar_commit(ctypes.byref(_desc(k=20)), ctypes.byref(c), FAKE, FAKE, FAKE, None) == tidar.ERR_UNSUPPORTED
+    assert L.tidar_commit(ctypes.byref(d), None, FAKE, FAKE, FAKE, None) == tidar.ERR_INVALID_ARG
+
+
+def test_plan_covers_workloads(L):
+    # host-only planning: the 8B-class step fills the machine, small prefixes use one split
+    d = _desc(batch=1, num_q_heads=32, num_kv_heads=8, k=16, max_prefix_len=8192)
+    path, splits = tidar.plan(d)
+    assert path in (1, 2) and splits >= 1
+    d = _desc(max_prefix_len=64)
+    assert tidar.plan(d)[1] == 1
+    d = _desc(dtype=tidar.F32, head_dim=64, path=tidar.PATH_AUTO)
+    assert tidar.plan(d)[0] == 1                        # fp32 -> CUDA-core kernel
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.tidar_status_string(s)

@@ -73,7 +73,7 @@ tidar_status check_cache(const tidar_step_desc* d, const tidar_kv_cache* c) {
   return TIDAR_OK;
 }
 
-constexpr bool kTc05Built = false;
+constexpr bool kTc05Built = true;
 
 bool tc05_supported(const tidar_step_desc* d) {
   return kTc05Built && d->dtype == TIDAR_BF16 && d->head_dim == 128 && d->page_size == 64;
@@ -109,7 +109,12 @@ Plan make_plan(const tidar_step_desc* d, int path) {
     target = 2 * kNumSMs * 4;
   }
   int ns = 1;
-  if (units > 0 && units < target) ns = (int)((target + units - 1) / units);
+  if (path == 2) {
+    // one CTA per SM: as many splits as fit in a single wave
+    if (units > 0 && units < target) ns = (int)(target / units);
+  } else if (units > 0 && units < target) {
+    ns = (int)((target + units - 1) / units);
+  }
   // at least 2 key blocks of 128 per split (tensor-core path), 1 for SIMT
   const int min_blocks = path == 2 ? 2 : 1;
   const int max_ns = blocks128 / min_blocks > 0 ? blocks128 / min_blocks : 1;

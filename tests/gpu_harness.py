@@ -68,6 +68,7 @@ def sample_rows(cfg, count, seed=0):
     """(b, rho, h) triples covering draft rows, first/last slots of blocks, every head."""
     rng = np.random.default_rng(seed)
     R = cfg.R
+    count = min(count, cfg.B * R * cfg.Hq)
     special = {0, R - 1, min(cfg.k, R - 1), max(cfg.k - 1, 0)}
     if cfg.k:
         for j in (1, 2, cfg.k):

@@ -69,9 +69,9 @@ def test_serving_flow(oracle_mod):
     """Serving batch: ragged prefixes, shuffled pages; the previous step's accept
     counts (uniform on 0..k) are committed first, then one full step."""
     cfg = synth.serving()
-    cache = synth.make_cache(cfg)
+    cache = synth.make_cache(cfg, extra_pages=cfg.B)      # spare pages for the next step
     prev = synth.prev_accept_counts(cfg)
-    max_prefix = 16384 + cfg.k
+    max_prefix = max(cfg.prefix) + cfg.n                  # lengths grow by at most n
     # 1) commit the previous step's counts (its draft rows sit at P..P+n-1)
     got, rel, nrel, st, _ = _gpu_commit(cache, prev, cfg.k, max_prefix)
     assert st == tidar.OK
@@ -81,7 +81,7 @@ def test_serving_flow(oracle_mod):
     pt = got["page_table"].clone()
     free = [int(x) for x in rel[:nrel]]
     used = set(int(x) for x in pt[pt >= 0])
-    spare = [p for p in range(cfg.B * 0, got["k_pages"].shape[0]) if p not in used and p not in free]
+    spare = [p for p in range(got["k_pages"].shape[0]) if p not in used and p not in free]
     pool = free + spare
     for b in range(cfg.B):
         P = int(got["seq_lens"][b])

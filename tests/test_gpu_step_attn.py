@@ -15,14 +15,16 @@ from gpu_harness import (compare_attention, oracle_attention, run_attention, sam
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["simt", "auto"]
+PATHS = ["simt", "tc05"]
 
 
-def _bf16_path_ok(cfg, path):
-    return True
+def _tc05_ok(cfg):
+    return cfg.dtype == "bf16" and cfg.D == 128 and cfg.page_size == 64
 
 
 def _check_full(oracle_mod, cfg, path):
+    if path == "tc05" and not _tc05_ok(cfg):
+        return                      # the tensor-core kernel takes bf16, head_dim 128 only
     cache, step = synth.make_cache(cfg), synth.make_step(cfg)
     out, lse, cache_after = run_attention(cfg, path, cache, step)
     want, want_lse = oracle_attention(oracle_mod, cfg, cache, step)
@@ -35,9 +37,9 @@ def _check_full(oracle_mod, cfg, path):
     np.testing.assert_array_equal(n(cache_after["v_pages"]), vp)
 
 
-@pytest.mark.parametrize("path", PATHS)
-def test_tiny_fp32(oracle_mod, path):
-    _check_full(oracle_mod, synth.tiny(), path)
+def test_tiny_fp32(oracle_mod):
+    _check_full(oracle_mod, synth.tiny(), "simt")
+    _check_full(oracle_mod, synth.tiny(), "auto")
 
 
 @pytest.mark.parametrize("path", PATHS)

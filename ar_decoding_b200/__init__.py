@@ -29,7 +29,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(
 F32, BF16 = 0, 1
 GREEDY, REJECTION = 0, 1
 PATH_AUTO, PATH_SIMT, PATH_TC05 = 0, 1, 2
-DEVERR_BAD_PAGE, DEVERR_BAD_LEN, DEVERR_BAD_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_BAD_PAGE, DEVERR_BAD_LEN, DEVERR_BAD_COUNT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 1, 2, 4, 8, 16
 _PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tc05": PATH_TC05}
 
 

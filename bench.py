@@ -12,12 +12,13 @@ Inputs are seeded synthetic tensors generated on the device.  One rank per GPU
 collective on the data path).
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
-cudaDeviceSynchronize; each step is timed on the device with CUDA events on the
-launching stream, and rotates over enough independent input/cache copies that
-each step's working set is evicted from L2 (126 MB) before it is reused.
-Between steps (outside the events) the copy's prefix length and page table are
-restored so every step does identical work.  ms_per_step / value is the mean
-step time, max over ranks.
+cudaDeviceSynchronize.  Each step replays CUDA graphs captured from the public
+API calls (step attention; verify + commit) and is timed on the device with
+CUDA events on the launching stream.  Steps rotate over enough independent
+input/cache copies that each step's working set is evicted from L2 (126 MB)
+before it is reused.  Between steps (outside the events) a third graph restores
+the copy's prefix length and page table so every step does identical work.
+ms_per_step / value is the mean step time, max over ranks.
 
 Prints one JSON line (rank 0).
 """
@@ -186,6 +187,25 @@ class Step:
         c["cache"]["seq_lens"].copy_(c["seq0"], non_blocking=True)
         c["cache"]["page_table"].copy_(c["pt0"], non_blocking=True)
 
+    def capture(self):
+        """One CUDA graph per copy for each of: step attention, verify + commit,
+        restore.  Replaying them keeps the host out of the timed device work."""
+        n = len(self.copies)
+        for i in range(n):          # first calls outside capture (module load, attributes)
+            self.attn(i); self.verify_commit(i); self.restore(i)
+        torch.cuda.synchronize()
+        self.graphs = []
+        for i in range(n):
+            ga, gv, gr = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ga):
+                self.attn(i)
+            with torch.cuda.graph(gv):
+                self.verify_commit(i)
+            with torch.cuda.graph(gr):
+                self.restore(i)
+            self.graphs.append((ga, gv, gr))
+        torch.cuda.synchronize()
+
 
 def copies_for(cfg):
     per = algorithmic(cfg)[0] + cfg.B * cfg.n * cfg.vocab * cfg.elem_bytes
@@ -243,25 +263,29 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- timing
 def time_steps(st: Step, K: int, W: int, world: int):
-    """Returns per-step device µs and per-step step_attn µs (lists)."""
+    """Returns per-step device µs and per-step step_attn µs (lists).  Each step
+    replays the copy's captured graphs; events sit between the graphs on the
+    launching stream, and the restore graph runs outside the timed span."""
     n = len(st.copies)
+    st.capture()
     stream = torch.cuda.current_stream()
     for i in range(W):
-        st.attn(i % n); st.verify_commit(i % n); st.restore(i % n)
+        ga, gv, gr = st.graphs[i % n]
+        ga.replay(); gv.replay(); gr.replay()
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
     for i in range(K):
-        c = (W + i) % n
+        ga, gv, gr = st.graphs[(W + i) % n]
         e0, e1, e2 = ev[i]
         e0.record(stream)
-        st.attn(c)
+        ga.replay()
         e1.record(stream)
-        st.verify_commit(c)
+        gv.replay()
         e2.record(stream)
-        st.restore(c)
+        gr.replay()
     torch.cuda.synchronize()
     barrier(world)
     step_us = [e0.elapsed_time(e2) * 1e3 for e0, _, e2 in ev]

@@ -72,6 +72,7 @@ typedef enum { TIDAR_PATH_AUTO = 0, TIDAR_PATH_SIMT = 1, TIDAR_PATH_TC05 = 2 } t
 #define TIDAR_DEVERR_BAD_LEN 0x2u       /* seq_lens[b] < 0 or > max_prefix_len */
 #define TIDAR_DEVERR_BAD_COUNT 0x4u     /* accept_count[b] outside 0..n (commit) */
 #define TIDAR_DEVERR_TIMEOUT 0x8u       /* a bounded mbarrier wait ran out */
+#define TIDAR_DEVERR_LAYOUT 0x10u       /* a kernel's shared-memory layout check failed (no work done) */
 
 typedef struct {
   int32_t batch;          /* B >= 0 (0: every call is a no-op) */

@@ -97,7 +97,7 @@ def test_8b_class_k_sweep_sampled(oracle_mod, path, k):
 @pytest.mark.parametrize("path", PATHS)
 def test_serving_ragged_sampled(oracle_mod, path):
     cfg = synth.serving()
-    _check_sampled(oracle_mod, cfg, path, 200, max_prefix=16384)
+    _check_sampled(oracle_mod, cfg, path, 200, max_prefix=max(cfg.prefix))
 
 
 def test_step_attn_reports_bad_page_without_fault(oracle_mod):

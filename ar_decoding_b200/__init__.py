@@ -76,6 +76,9 @@ def lib():
         L.tidar_verify.argtypes = [I, I, I, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P, P, P,
                                    S, P]
         L.tidar_verify.restype = ctypes.c_int
+        L.tidar_verify_noalloc.argtypes = [I, I, I, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P,
+                                           P, P, P]
+        L.tidar_verify_noalloc.restype = ctypes.c_int
         L.tidar_commit.argtypes = [P, P, P, P, P, P]
         L.tidar_commit.restype = ctypes.c_int
         L.tidar_get_device_status.argtypes = [P, P]
@@ -205,6 +208,32 @@ def verify(logits, drafts, k, mode="greedy", *, draft_logits=None, uniforms=None
                             _ptr(outputs["selected_block"]), _ptr(workspace),
                             workspace.numel(), _stream_handle(stream))
     _check(st, "tidar_verify")
+    return outputs
+
+
+VERIFY_NOALLOC_MAX_SCRATCH_BYTES = 4 << 20
+
+
+def verify_noalloc(logits, drafts, k, mode="greedy", *, draft_logits=None, uniforms=None,
+                   block_guesses=None, outputs=None, stream=None):
+    """tidar_verify without a workspace: the library's fixed device scratch is used
+    (for callers that cannot allocate at this point, e.g. inside graph capture
+    once the first call on the device has been made outside it)."""
+    m = mode if isinstance(mode, int) else {"greedy": GREEDY, "rejection": REJECTION}[mode]
+    _dev(logits, "logits")
+    B, n, V = logits.shape
+    dev = logits.device
+    if outputs is None:
+        outputs = dict(accept_count=torch.empty(B, dtype=torch.int32, device=dev),
+                       out_tokens=torch.empty((B, n), dtype=torch.int32, device=dev),
+                       next_drafts=torch.empty((B, max(k, 1)), dtype=torch.int32, device=dev),
+                       selected_block=torch.empty(B, dtype=torch.int32, device=dev))
+    st = lib().tidar_verify_noalloc(B, k, V, _dtype_code(logits), m, _ptr(logits), _ptr(drafts),
+                                    _ptr(draft_logits), _ptr(uniforms), _ptr(block_guesses),
+                                    _ptr(outputs["accept_count"]), _ptr(outputs["out_tokens"]),
+                                    _ptr(outputs["next_drafts"]) if k > 0 else None,
+                                    _ptr(outputs["selected_block"]), _stream_handle(stream))
+    _check(st, "tidar_verify_noalloc")
     return outputs
 
 

@@ -406,3 +406,67 @@ cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s) {
 }
 
 }  // namespace tidar
+
+// ---------------------------------------------------------------------------
+// tidar_verify_noalloc: the same verification without a caller workspace.
+//
+// For callers that cannot allocate device memory when they call verify: for
+// example a decode loop being recorded into a CUDA graph, where an allocation
+// would break the capture, or a host runtime that only hands the library
+// tensors it already owns and has no way to create scratch buffers.  The
+// scratch lives in this file's fixed device array instead; every GPU that
+// loads the library keeps it until the process exits.
+//
+// The device address of the array is looked up (cudaGetSymbolAddress) on the
+// first call made with each device current; that first call should therefore
+// happen before any stream capture.  All calls share the one array and it
+// keeps whatever the last call left there.  Verification needs no part of it
+// zeroed: every statistic is written before it is read.  Calls that overlap on
+// the GPU (different streams, no ordering between them) race on the array.
+namespace tidar {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = TIDAR_VERIFY_NOALLOC_MAX_SCRATCH_BYTES;   // per device
+static __device__ __align__(256) unsigned char g_verify_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_verify_scratch_ptr[kNoAllocMaxDevices] = {nullptr};
+
+}  // namespace
+}  // namespace tidar
+
+extern "C" tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                                             tidar_accept_mode mode, const void* logits,
+                                             const int32_t* drafts, const void* draft_logits,
+                                             const float* uniforms, const int32_t* block_guesses,
+                                             int32_t* accept_count, int32_t* out_tokens,
+                                             int32_t* next_drafts, int32_t* selected_block,
+                                             tidar_stream_t stream) {
+  if (batch < 0 || k < 0 || vocab <= 0) return TIDAR_ERR_INVALID_ARG;
+  if (k > 16) return TIDAR_ERR_UNSUPPORTED;
+  if (dtype != TIDAR_F32 && dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
+  if (mode != TIDAR_GREEDY && mode != TIDAR_REJECTION) return TIDAR_ERR_INVALID_ARG;
+  if (batch == 0) return TIDAR_OK;
+  if (!logits || !accept_count || !out_tokens) return TIDAR_ERR_INVALID_ARG;
+  if (k > 1 && !drafts) return TIDAR_ERR_INVALID_ARG;
+  if (mode == TIDAR_REJECTION && (!uniforms || (k > 1 && !draft_logits))) return TIDAR_ERR_INVALID_ARG;
+  // too large for the fixed scratch: refuse before touching the device
+  if (tidar::verify_workspace_bytes(batch, k, vocab, mode) > tidar::kNoAllocScratchBytes)
+    return TIDAR_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TIDAR_ERR_CUDA;
+  if (dev < 0 || dev >= tidar::kNoAllocMaxDevices) return TIDAR_ERR_UNSUPPORTED;
+  if (!tidar::g_verify_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, tidar::g_verify_scratch) != cudaSuccess || !ptr) return TIDAR_ERR_CUDA;
+    tidar::g_verify_scratch_ptr[dev] = ptr;
+  }
+  tidar::VerifyArgs a;
+  a.B = batch; a.k = k; a.n = k > 0 ? k : 1; a.V = vocab; a.bf16 = dtype == TIDAR_BF16; a.mode = mode;
+  a.logits = logits; a.drafts = drafts; a.draft_logits = draft_logits; a.uniforms = uniforms;
+  a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;
+  a.next_drafts = next_drafts; a.selected_block = selected_block;
+  a.workspace = tidar::g_verify_scratch_ptr[dev];
+  if (tidar::launch_verify(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TIDAR_ERR_CUDA;
+  return TIDAR_OK;
+}

@@ -178,6 +178,36 @@ tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype d
                           void* workspace, size_t workspace_bytes, tidar_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Verification without a caller workspace (no counterpart in the paper; a
+ * convenience of this library).
+ *
+ * Same arguments, results and device-side behaviour as tidar_verify, minus
+ * the workspace.  It is for callers that cannot allocate device memory at the
+ * point where they verify: a decode loop being captured into a CUDA graph, or
+ * a host runtime that only passes in tensors it already owns.  The scratch is
+ * a fixed array inside the library of TIDAR_VERIFY_NOALLOC_MAX_SCRATCH_BYTES
+ * (4 MiB) on every GPU that loads the library, held until the process exits.
+ * The call allocates nothing.
+ *   - Returns TIDAR_ERR_UNSUPPORTED, before any launch, when the call needs
+ *     more scratch than that (tidar_verify_workspace_bytes(...) > the maximum).
+ *   - The first call made with a given device current looks the array's
+ *     address up (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.
+ *   - All calls share the array and it keeps the previous call's contents
+ *     (verification reads nothing it did not write).  Calls that can overlap
+ *     on the GPU -- different streams with no ordering between them -- race
+ *     on it; order them on one stream.
+ * ------------------------------------------------------------------------- */
+#define TIDAR_VERIFY_NOALLOC_MAX_SCRATCH_BYTES ((size_t)4 << 20)
+tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                                  tidar_accept_mode mode, const void* logits,
+                                  const int32_t* drafts, const void* draft_logits,
+                                  const float* uniforms, const int32_t* block_guesses,
+                                  int32_t* accept_count, int32_t* out_tokens,
+                                  int32_t* next_drafts, int32_t* selected_block,
+                                  tidar_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * KV commit / evict, in place.  [NDfr] paragraph on the three zones (the
  * settled cache is reused, rejected entries are evicted); [MS] "KV Cache" and
  * [FG] abstract (exact KV cache).  Accepted drafts are a prefix of the draft

@@ -207,6 +207,23 @@ class Step:
         torch.cuda.synchronize()
 
 
+def measured_traffic(k: int):
+    """DRAM bytes of one attention launch from the committed ncu record, if the
+    kernel source is unchanged since the capture; else None."""
+    import hashlib
+    src = os.path.join(ROOT, "ar_decoding_b200", "csrc", "attn_tc05.cu")
+    rec = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        for line in open(rec):
+            parts = line.split()
+            if len(parts) == 3 and not line.startswith("#") and parts[0] == sha and int(parts[1]) == k:
+                return int(parts[2])
+    except OSError:
+        pass
+    return None
+
+
 def copies_for(cfg):
     per = algorithmic(cfg)[0] + cfg.B * cfg.n * cfg.vocab * cfg.elem_bytes
     return max(3, math.ceil(3 * L2_BYTES / per))
@@ -473,7 +490,8 @@ def run_ours(args, rank, world, local):
             "hbm_gbs_all_gpus": agg_gbs,
             "roofline": {"kernel": "tidar_step_attn", "bound": bound, "achieved": achieved,
                          "peak": peak, "unit": unit, "frac": achieved / peak,
-                         "peak_source": peak_src, "traffic": None,
+                         "peak_source": peak_src, "peak_kind": "burst",
+                         "traffic": measured_traffic(args.k) if st.path_id == 2 else None,
                          "algorithmic_bytes": bytes_, "algorithmic_flops": flops,
                          "roofline_frac_max_of_both": max(t_mem, t_tc) / attn_s},
             "k_sweep": sweep,

@@ -40,7 +40,7 @@ namespace tidar {
 
 namespace {
 
-constexpr int kThreads = 320;       // producer, MMA, 8 softmax warps
+constexpr int kThreads = 576;       // producer, MMA, 16 softmax warps
 constexpr int kStages = 3;       // K/V ring depth; also the number of S buffers
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // every mbarrier wait gives up after ~1 s
 constexpr uint32_t kSuspendHintNs = 10000000u;      // one try_wait sleeps at most 10 ms
@@ -55,12 +55,13 @@ constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
 constexpr int BAR_Q = 0;
 constexpr int BAR_KFULL = 1;     // + stage
 constexpr int BAR_VFULL = 4;     // + stage
-constexpr int BAR_EMPTY = 7;     // + stage
+constexpr int BAR_KEMPTY = 7;    // + stage: K stage free again (its S MMA is done)
 constexpr int BAR_SFULL = 10;    // + S buffer
 constexpr int BAR_PFULL = 13;    // + S buffer
 constexpr int BAR_PVDONE = 16;   // + S buffer
 constexpr int BAR_FINAL = 19;
-constexpr int kNumBars = 20;
+constexpr int BAR_VEMPTY = 20;   // + stage: V stage free again (its PV MMA is done)
+constexpr int kNumBars = 23;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // [0] TMEM base, [1] abort flag
 constexpr uint32_t kOffRed = kOffMisc + 16;              // softmax halves: maxima [2][2][128] f32
 constexpr uint32_t kOffOk = kOffRed + 2048;              // and warp status [2][2][4] i32
@@ -72,6 +73,10 @@ constexpr uint32_t kTmemCols = 512;
 // Softmax set t (block parity) owns S_t (P_t is written over its first 64
 // columns) and the accumulator O_t.
 __device__ __forceinline__ uint32_t col_s(int t) { return 128u * (uint32_t)t; }
+// P (bf16, two keys per column) of keys [16kk, 16kk+16) within S_t: each softmax
+// half writes the P of its 64 keys into the first 32 columns of its own 64 S
+// columns, so the halves never overwrite scores the other half still reads.
+__device__ __forceinline__ uint32_t p_col(int kk) { return kk < 4 ? 8u * kk : 64u + 8u * (kk - 4); }
 __device__ __forceinline__ uint32_t col_o(int t) { return 256u + 128u * (uint32_t)t; }
 
 // kind::f16 instruction descriptors: fp32 accumulate, bf16 A and B, M = 128, N = 128.
@@ -100,6 +105,29 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 // Test the phase; if it is incomplete the thread may sleep in hardware until
 // the phase completes or the hint (ns) expires, whichever is first.
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -253,6 +281,58 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+
+// ---- packed fp32x2 helpers (sm_100) and the exponential split --------------
+__device__ __forceinline__ uint64_t f2_make(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// (lo, hi) -> bf16x2, round to nearest even
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// 2^v for a pair, on the FMA pipe: Cody-Waite split v = j + f with j = rint(v)
+// (magic-number rounding), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// coefficients are a relative-error minimax fit computed for this library
+// (max relative error 7.5e-5); 2^j added to the exponent field.  Inputs are
+// clamped at -126 (results there are below every bf16 P that matters).
+__device__ __forceinline__ void exp2_poly_pair(float v0, float v1, float& r0, float& r1) {
+  constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
+  const uint64_t vc = f2_make(fmaxf(v0, -126.0f), fmaxf(v1, -126.0f));
+  const uint64_t t = f2_add(vc, f2_make(kMagic, kMagic));
+  const uint64_t tf = f2_add(t, f2_make(-kMagic, -kMagic));
+  const uint64_t f = f2_fma(tf, f2_make(-1.0f, -1.0f), vc);
+  uint64_t p = f2_fma(f2_make(0.0551716685f, 0.0551716685f), f, f2_make(0.242611125f, 0.242611125f));
+  p = f2_fma(p, f, f2_make(0.693260968f, 0.693260968f));
+  p = f2_fma(p, f, f2_make(0.999928057f, 0.999928057f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  r0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(p0));   // + (j << 23)
+  r1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1));
+}
+
 // Two non-negative floats -> packed bf16x2 (low half = a), rounded to nearest
 // with ties away from zero, using integer ops only (keeps the conversion off
 // the transcendental pipe that ex2 saturates).
@@ -297,7 +377,9 @@ __device__ __forceinline__ BlockPlan make_block_plan(const AttnArgs& a, int P, i
 __device__ __forceinline__ bool page_ok(int page, int num_pages) { return page >= 0 && page < num_pages; }
 
 // ------------------------------------------------------------------ the kernel
-__global__ void __launch_bounds__(kThreads, 1)
+// 18 warps: two SMSPs host five of them, so a thread may hold at most
+// 16384 / (5 * 32) -> 96 registers.
+__global__ void __maxnreg__(96)
 attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
                  const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_ks,
                  const __grid_constant__ CUtensorMap tm_vs, const Tc05Params prm) {
@@ -337,7 +419,7 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #endif
     for (int i = 0; i < kNumBars; ++i) {
       const bool pfull = i >= BAR_PFULL && i < BAR_PFULL + kStages;
-      mbar_init(bar(i), pfull ? 4u : 1u);
+      mbar_init(bar(i), pfull ? 8u : 1u);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -373,62 +455,84 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
+    // Separate K and V rings (3 stages each): a K stage is refilled as soon as
+    // its S MMA is done, a V stage when its PV is done, so K runs up to three
+    // blocks ahead of the scores.  One thread polls both rings.
     if (lane == 0) {
-      int issued_phase[kStages] = {-1, -1, -1};
+      int k_phase[kStages] = {-1, -1, -1}, v_phase[kStages] = {-1, -1, -1};
       mbar_expect_tx(bar(BAR_Q), 2u * 128u * (uint32_t)(prm.rho_per_tile * a.G));
       tma_load_4d(sb + kOffQ, &tm_q, 0, g * a.G, rho0, b, bar(BAR_Q));
       tma_load_4d(sb + kOffQ + kChunkBytes, &tm_q, 64, g * a.G, rho0, b, bar(BAR_Q));
       bool bad = false;
-      for (int i = 0; i < bp.nb; ++i) {
+      // one ring's tile of block i: two 64-row pages of the cache, or a window
+      auto issue = [&](int i, bool is_v) {
         const int s = i % kStages;
-        if (i >= kStages && !wait_bar(bar(BAR_EMPTY + s), (uint32_t)((i / kStages - 1) & 1), abort_flag, a.err)) break;
-        const uint32_t kdst = sb + kOffK + s * kTileBytes, vdst = sb + kOffV + s * kTileBytes;
+        const uint32_t dst = sb + (is_v ? kOffV : kOffK) + s * kTileBytes;
+        const uint32_t full = bar((is_v ? BAR_VFULL : BAR_KFULL) + s);
         if (i < bp.npb) {
+          const CUtensorMap* map = is_v ? &tm_vp : &tm_kp;
           const int start = bp.k0 + i * 128;
           const int pa = table[start / 64];
           const bool need_b = start + 64 < bp.kend;
           const int pb = need_b ? table[start / 64 + 1] : -1;
           const bool oka = page_ok(pa, a.num_pages), okb = need_b && page_ok(pb, a.num_pages);
           if (!oka || (need_b && !okb)) bad = true;
-          const uint32_t bytes = (uint32_t)(oka + okb) * 2u * 8192u;
-          mbar_expect_tx(bar(BAR_KFULL + s), bytes);
+          mbar_expect_tx(full, (uint32_t)(oka + okb) * 2u * 8192u);
           if (oka) {
-            tma_load_2d(kdst, &tm_kp, 0, (pa * a.Hkv + g) * 64, bar(BAR_KFULL + s));
-            tma_load_2d(kdst + kChunkBytes, &tm_kp, 64, (pa * a.Hkv + g) * 64, bar(BAR_KFULL + s));
+            tma_load_2d(dst, map, 0, (pa * a.Hkv + g) * 64, full);
+            tma_load_2d(dst + kChunkBytes, map, 64, (pa * a.Hkv + g) * 64, full);
           }
           if (okb) {
-            tma_load_2d(kdst + 8192, &tm_kp, 0, (pb * a.Hkv + g) * 64, bar(BAR_KFULL + s));
-            tma_load_2d(kdst + kChunkBytes + 8192, &tm_kp, 64, (pb * a.Hkv + g) * 64, bar(BAR_KFULL + s));
-          }
-          mbar_expect_tx(bar(BAR_VFULL + s), bytes);
-          if (oka) {
-            tma_load_2d(vdst, &tm_vp, 0, (pa * a.Hkv + g) * 64, bar(BAR_VFULL + s));
-            tma_load_2d(vdst + kChunkBytes, &tm_vp, 64, (pa * a.Hkv + g) * 64, bar(BAR_VFULL + s));
-          }
-          if (okb) {
-            tma_load_2d(vdst + 8192, &tm_vp, 0, (pb * a.Hkv + g) * 64, bar(BAR_VFULL + s));
-            tma_load_2d(vdst + kChunkBytes + 8192, &tm_vp, 64, (pb * a.Hkv + g) * 64, bar(BAR_VFULL + s));
+            tma_load_2d(dst + 8192, map, 0, (pb * a.Hkv + g) * 64, full);
+            tma_load_2d(dst + kChunkBytes + 8192, map, 64, (pb * a.Hkv + g) * 64, full);
           }
         } else {
+          const CUtensorMap* map = is_v ? &tm_vs : &tm_ks;
           const int w = bp.wins[i - bp.npb];
-          mbar_expect_tx(bar(BAR_KFULL + s), kTileBytes);
-          tma_load_4d(kdst, &tm_ks, 0, g, w * 128, b, bar(BAR_KFULL + s));
-          tma_load_4d(kdst + kChunkBytes, &tm_ks, 64, g, w * 128, b, bar(BAR_KFULL + s));
-          mbar_expect_tx(bar(BAR_VFULL + s), kTileBytes);
-          tma_load_4d(vdst, &tm_vs, 0, g, w * 128, b, bar(BAR_VFULL + s));
-          tma_load_4d(vdst + kChunkBytes, &tm_vs, 64, g, w * 128, b, bar(BAR_VFULL + s));
+          mbar_expect_tx(full, kTileBytes);
+          tma_load_4d(dst, map, 0, g, w * 128, b, full);
+          tma_load_4d(dst + kChunkBytes, map, 64, g, w * 128, b, full);
         }
-        issued_phase[s] = i / kStages;
-        TIDAR_TRACE_AT(16 + min(i, 239));
+        (is_v ? v_phase : k_phase)[s] = i / kStages;
+      };
+      int ik = 0, iv = 0;
+      uint64_t last = global_ns();
+      while ((ik < bp.nb || iv < bp.nb) && !*abort_flag) {
+        bool progress = false;
+        if (ik < bp.nb &&
+            (ik < kStages || mbar_test(bar(BAR_KEMPTY + ik % kStages), (uint32_t)((ik / kStages - 1) & 1)))) {
+          issue(ik, false);
+          TIDAR_TRACE_AT(16 + min(ik, 239));
+          ++ik;
+          progress = true;
+        }
+        if (iv < ik &&
+            (iv < kStages || mbar_test(bar(BAR_VEMPTY + iv % kStages), (uint32_t)((iv / kStages - 1) & 1)))) {
+          issue(iv, true);
+          ++iv;
+          progress = true;
+        }
+        if (progress) {
+          last = global_ns();
+        } else {
+          // sleep briefly on the ring that is further behind, then re-check both
+          if (ik < bp.nb && ik - iv < kStages)
+            mbar_try_wait_ns(bar(BAR_KEMPTY + ik % kStages), (uint32_t)((ik / kStages - 1) & 1), 500u);
+          else
+            mbar_try_wait_ns(bar(BAR_VEMPTY + iv % kStages), (uint32_t)((iv / kStages - 1) & 1), 500u);
+          if (global_ns() - last > kWaitLimitNs) {
+            *abort_flag = 1;
+            raise_error(a.err, TIDAR_DEVERR_TIMEOUT);
+          }
+        }
       }
       if (bad) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
       // Drain: on the normal path every load was consumed; after a timeout make
       // sure no copy is still writing shared memory when the CTA exits.
       if (*abort_flag) {
-        for (int s = 0; s < kStages; ++s) {
-          if (issued_phase[s] < 0) continue;
-          wait_quiet(bar(BAR_KFULL + s), issued_phase[s] & 1);
-          wait_quiet(bar(BAR_VFULL + s), issued_phase[s] & 1);
+        for (int s2 = 0; s2 < kStages; ++s2) {
+          if (k_phase[s2] >= 0) wait_quiet(bar(BAR_KFULL + s2), k_phase[s2] & 1);
+          if (v_phase[s2] >= 0) wait_quiet(bar(BAR_VFULL + s2), v_phase[s2] & 1);
         }
         wait_quiet(bar(BAR_Q), 0);
       }
@@ -454,6 +558,7 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           mma_ss(tmem + col_s(t), desc_k_sw128(qa + off), desc_k_sw128(ka + off), kIdescS, kc > 0);
         }
         mma_commit(bar(BAR_SFULL + t));
+        mma_commit(bar(BAR_KEMPTY + st));
         TIDAR_TRACE_AT(512 + min(blk, 255));
         return true;
       };
@@ -467,10 +572,10 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t va = sb + kOffV + st * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, desc_mn_sw128(va + kk * 2048, kChunkBytes), kIdescPV,
+          mma_ts(tmem + col_o(t), tmem + col_s(t) + p_col(kk), desc_mn_sw128(va + kk * 2048, kChunkBytes), kIdescPV,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(BAR_PVDONE + t));
-        mma_commit(bar(BAR_EMPTY + st));
+        mma_commit(bar(BAR_VEMPTY + st));
         TIDAR_TRACE_AT(768 + min(b2, 255));
         if (b2 + 2 < bp.nb && !issue_s(b2 + 2)) break;
       }
@@ -480,26 +585,30 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else {
     // ---------------------------------------------------------------- softmax
-    // Set t (warps 2..5: t = 0, warps 6..9: t = 1) takes blocks b with b & 1 == t
-    // and keeps its own running max, row sum and O_t; the two sets' results are
-    // merged in the epilogue like two split-KV partials.  One thread per TMEM
-    // lane (= packed query row), all 128 columns of the block.
+    // Warps 2..17.  Set t (block parity) = (warp-2)/8 owns S_t and O_t; within a
+    // set, half hf = ((warp-2)/4)&1 takes columns [64hf, 64hf+64) of the rows of
+    // TMEM lane quarter warp%4.  One thread = one half row.  The two halves of a
+    // row swap block maxima at a named barrier (id 1 + 4t + quarter, 64
+    // threads); row sums and the two sets are merged in the epilogue.
     const int q4 = warp & 3;
-    const int t = (warp - 2) >> 2;
+    const int t = (warp - 2) >> 3;
+    const int hf = ((warp - 2) >> 2) & 1;
     const int r = 32 * q4 + lane;
     const int rho_c = min(rho0 + r / a.G, a.R - 1);
     const StepVis vis = step_visibility(a.k, rho_c);
     const uint32_t trow = tmem + ((uint32_t)(32 * q4) << 16);
-    const int gt = threadIdx.x - 64 - 128 * t;          // 0..127 within the set
+    const int gt = (warp - 2 - 8 * t) * 32 + lane;     // 0..255 within the set
     const bool live = 32 * q4 < rows_valid;             // the warp holds at least one real row
     const float sl2 = prm.scale_log2;
     const int nbt = (bp.nb - t + 1) >> 1;               // blocks of this set
+    float* xmax = reinterpret_cast<float*>(smem + kOffRed);          // [2 set][2 half][128]
+    int* xok = reinterpret_cast<int*>(smem + kOffOk);                // [2 set][2 half][4 quarter]
+    const uint32_t pair_bar = 1 + 4 * t + q4;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nbt; ++j) {
       const int b2 = 2 * j + t;
-      if (t == 0 && warp == 4 && lane == 0) TIDAR_TRACE_AT(1700 + min(b2, 255));
-      if (!warp_wait_bar(bar(BAR_SFULL + t), (uint32_t)(j & 1), abort_flag, a.err)) { ok = false; break; }
+      if (!warp_wait_bar(bar(BAR_SFULL + t), (uint32_t)(j & 1), abort_flag, a.err)) ok = false;
       fence_after();
       if (warp == 4 && lane == 0) TIDAR_TRACE_AT(1024 + min(b2, 255));
       TIDAR_TRACE_PH(b2, 0);
@@ -517,90 +626,121 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         kb = bp.wins[b2 - bp.npb] * 128;
       }
       const bool full = !window && lo_valid == 64 && hi_valid == 64;
-      const uint32_t scol = col_s(t);
-      // visibility of column c of this block for this thread's row (masked blocks)
-      auto visible = [&](int c) -> bool {
-        if (window) {
-          const int key = kb + c;
-          return key < a.R && step_visible(vis, key);
-        }
-        return c < 64 ? c < lo_valid : c - 64 < hi_valid;
-      };
-      // pass 1: block maximum of the raw scores (the positive scale commutes)
+      const uint32_t scol = col_s(t) + 64 * hf;          // this half's 64 score columns
+      // pass 1: maximum of this half's raw scores (the positive scale commutes)
       float mb = -INFINITY;
-      if (live) {
-        uint32_t x[128];
-        tmem_ld32(trow + scol + 0, *reinterpret_cast<uint32_t(*)[32]>(x + 0));
-        tmem_ld32(trow + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-        tmem_ld32(trow + scol + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
-        tmem_ld32(trow + scol + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
-        tmem_wait_ld();
-        TIDAR_TRACE_PH(b2, 2);
-        if (!full) {
-          // masked block (rare): invisible keys become -inf in TMEM as well, so
-          // pass 2 needs no mask (2^-inf = 0)
+      if (live && ok) {
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (!visible(c)) x[c] = 0xff800000u;
-          tmem_st32(trow + scol + 0, *reinterpret_cast<uint32_t(*)[32]>(x + 0));
-          tmem_st32(trow + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-          tmem_st32(trow + scol + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
-          tmem_st32(trow + scol + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
-          tmem_wait_st();
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t x[32];
+          tmem_ld32(trow + scol + 32 * h2, x);
+          tmem_wait_ld();
+          if (!full) {
+            // masked block (rare): invisible keys become -inf in TMEM too, so
+            // the exponential pass needs no mask (2^-inf = 0)
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int col = 64 * hf + 32 * h2 + c;
+              bool v;
+              if (window) {
+                const int key = kb + col;
+                v = key < a.R && step_visible(vis, key);
+              } else {
+                v = col < 64 ? col < lo_valid : col - 64 < hi_valid;
+              }
+              if (!v) x[c] = 0xff800000u;
+            }
+            tmem_st32(trow + scol + 32 * h2, x);
+            tmem_wait_st();
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            mx[0] = max3(mx[0], __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+            mx[1] = max3(mx[1], __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+            mx[2] = max3(mx[2], __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
+            mx[3] = max3(mx[3], __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
+          }
         }
-        float mx[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) mx[e] = __uint_as_float(x[e]);
-#pragma unroll
-        for (int c = 4; c < 128; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(x[c]));
         mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       }
       TIDAR_TRACE_PH(b2, 3);
-      const float m_new = fmaxf(m, mb);
+      // swap block maxima and status with the other half of the row
+      const int slot = t * 256;
+      xmax[slot + hf * 128 + r] = mb;
+      if (lane == 0) xok[t * 8 + hf * 4 + q4] = ok ? 1 : 0;            // ok is warp-uniform
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      const float mrow = fmaxf(mb, xmax[slot + (hf ^ 1) * 128 + r]);
+      const bool both_ok = ok && xok[t * 8 + (hf ^ 1) * 4 + q4] != 0;
+      // the slots are rewritten next block only after the partner has read them:
+      // it cannot pass the next barrier before this thread arrives there
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      if (!both_ok) { ok = false; break; }               // both halves leave together
+      const float m_new = fmaxf(m, mrow);
       const bool need = m_new > m + 8.0f;
       const float f_resc = need ? ex2(m - m_new) : 1.0f;   // factor for O_t and l (m = -inf -> 0)
       if (need) m = m_new;
       const float nbase = m == -INFINITY ? 0.f : -m;
       TIDAR_TRACE_PH(b2, 4);
-      // pass 2: P = 2^(score * scale - m) in bf16, packed in registers from two
-      // 64-column reloads of S and stored to TMEM (over S) only after both
-      // reloads; the row sum keeps the fp32 values
+      // pass 2: P = 2^(score * scale - m) in bf16 for this half's 64 keys; the P
+      // of each 32 keys goes over 16 columns of this half's S already reloaded
       float lblk = 0.f;
       if (live) {
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[64];
+        const uint64_t sl2x2 = f2_make(sl2, sl2), nbx2 = f2_make(nbase, nbase);
+        uint64_t ls2[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t x[64];
-          tmem_ld32(trow + scol + 64 * h2, *reinterpret_cast<uint32_t(*)[32]>(x + 0));
-          tmem_ld32(trow + scol + 64 * h2 + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+          uint32_t x[32];
+          tmem_ld32(trow + scol + 32 * h2, x);
           tmem_wait_ld();
+          uint32_t pk[16];
+          if (full) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(fmaf(__uint_as_float(x[2 * c]), sl2, nbase));
-            const float p1 = ex2(fmaf(__uint_as_float(x[2 * c + 1]), sl2, nbase));
-            ls[c & 3] += p0 + p1;
-            pk[32 * h2 + c] = pack_bf16x2_pos(p0, p1);
+            for (int c = 0; c < 16; ++c) {
+              float v0, v1, p0, p1;
+              f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
+              if ((c & 7) < 3) {
+                exp2_poly_pair(v0, v1, p0, p1);
+              } else {
+                p0 = ex2(v0);
+                p1 = ex2(v1);
+              }
+              ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
+              pk[c] = cvt_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              float v0, v1;
+              f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
+              const float p0 = ex2(v0), p1 = ex2(v1);
+              ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
+              pk[c] = cvt_bf16x2(p0, p1);
+            }
           }
+          tmem_st16(trow + scol + 16 * h2, pk);
         }
-        tmem_st32(trow + scol + 0, *reinterpret_cast<uint32_t(*)[32]>(pk + 0));
-        tmem_st32(trow + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
-        lblk = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        float la, lb, lc, ld;
+        f2_split(ls2[0], la, lb);
+        f2_split(ls2[1], lc, ld);
+        lblk = (la + lb) + (lc + ld);
       }
       TIDAR_TRACE_PH(b2, 5);
       if (__any_sync(0xffffffffu, need) && j > 0) {
         // O_t holds PV of this set's earlier blocks: wait for the last one and
-        // rescale it before this block's PV is released to the MMA warp
-        if (!warp_wait_bar(bar(BAR_PVDONE + t), (uint32_t)((j - 1) & 1), abort_flag, a.err)) { ok = false; break; }
+        // rescale this half's 64 columns before this block's PV is released
+        if (!warp_wait_bar(bar(BAR_PVDONE + t), (uint32_t)((j - 1) & 1), abort_flag, a.err)) ok = false;
         fence_after();
+        if (ok) {
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t o[16];
-          tmem_ld16(trow + col_o(t) + 16 * c, o);
-          tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[16];
+            tmem_ld16(trow + col_o(t) + 64 * hf + 16 * c, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f_resc);
-          tmem_st16(trow + col_o(t) + 16 * c, o);
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f_resc);
+            tmem_st16(trow + col_o(t) + 64 * hf + 16 * c, o);
+          }
         }
       }
       l = l * f_resc + lblk;
@@ -608,16 +748,18 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // keys past the prefix end or on an unmapped page: zero their V rows so
         // that 0 * (whatever the page holds) cannot turn into NaN
         const int st = b2 % kStages;
-        if (!warp_wait_bar(bar(BAR_VFULL + st), (uint32_t)((b2 / kStages) & 1), abort_flag, a.err)) { ok = false; break; }
-        uint8_t* vs = smem + kOffV + st * kTileBytes;
-        for (int idx = gt; idx < 128 * 16; idx += 128) {
-          const int row = idx >> 4, piece = idx & 15;
-          const bool inval = row < 64 ? row >= lo_valid : row - 64 >= hi_valid;
-          if (inval)
-            *reinterpret_cast<uint4*>(vs + (piece >> 3) * kChunkBytes + row * 128 + (piece & 7) * 16) =
-                make_uint4(0, 0, 0, 0);
+        if (!warp_wait_bar(bar(BAR_VFULL + st), (uint32_t)((b2 / kStages) & 1), abort_flag, a.err)) ok = false;
+        if (ok) {
+          uint8_t* vs = smem + kOffV + st * kTileBytes;
+          for (int idx = gt; idx < 128 * 16; idx += 256) {
+            const int row = idx >> 4, piece = idx & 15;
+            const bool inval = row < 64 ? row >= lo_valid : row - 64 >= hi_valid;
+            if (inval)
+              *reinterpret_cast<uint4*>(vs + (piece >> 3) * kChunkBytes + row * 128 + (piece & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       tmem_wait_st();
       TIDAR_TRACE_PH(b2, 6);
@@ -625,26 +767,28 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_PFULL + t));
       if (warp == 4 && lane == 0) TIDAR_TRACE_AT(1280 + min(b2, 255));
-      if (b2 == 2 && lane == 0) TIDAR_TRACE_AT(1632 + warp);
     }
-    // ---- epilogue: merge the two sets' partials; set t writes columns [64t, 64t+64)
-    float* xm = reinterpret_cast<float*>(smem + kOffRed);            // [2 set][128] running max
-    float* xl = xm + 256;                                            // [2 set][128] row sums
-    xm[t * 128 + r] = m;
-    xl[t * 128 + r] = l;
-    int* xok = reinterpret_cast<int*>(smem + kOffOk);
-    if (lane == 0) xok[t * 4 + q4] = ok ? 1 : 0;
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + q4) : "memory");
-    const float mo = xm[(t ^ 1) * 128 + r], lo = xl[(t ^ 1) * 128 + r];
-    ok = ok && xok[(t ^ 1) * 4 + q4] != 0;
-    // both sets' last PV must be complete before O_0 and O_1 are read
+    // ---- epilogue: merge sets and halves.  The four warps of a lane quarter
+    // (2 sets x 2 halves) meet at barrier 9 + quarter; each then writes 32 of
+    // the 128 output columns of its rows.
     const int nb0 = (bp.nb + 1) >> 1, nb1 = bp.nb >> 1;
+    // both sets' last PV must be complete before O_0 and O_1 are read; after it
+    // no MMA reads shared memory, so the Q tile holds the exchange arrays
     if (ok && nb0 > 0 && !warp_wait_bar(bar(BAR_PVDONE + 0), (uint32_t)((nb0 - 1) & 1), abort_flag, a.err)) ok = false;
     if (ok && nb1 > 0 && !warp_wait_bar(bar(BAR_PVDONE + 1), (uint32_t)((nb1 - 1) & 1), abort_flag, a.err)) ok = false;
     fence_after();
+    float* xm = reinterpret_cast<float*>(smem + kOffQ);              // [2 set][128] max
+    float* xs = xm + 256;                                            // [2 set][2 half][128] sums
+    int* xk = reinterpret_cast<int*>(xs + 512);                      // [2 set][2 half][4] status
+    asm volatile("bar.sync %0, 128;" ::"r"(9 + q4) : "memory");
+    if (hf == 0) xm[t * 128 + r] = m;
+    xs[(t * 2 + hf) * 128 + r] = l;
+    if (lane == 0) xk[t * 8 + hf * 4 + q4] = ok ? 1 : 0;
+    asm volatile("bar.sync %0, 128;" ::"r"(9 + q4) : "memory");
+    const float m0 = xm[r], m1 = xm[128 + r];
+    const float l0 = xs[r] + xs[128 + r], l1 = xs[256 + r] + xs[384 + r];
+    ok = xk[q4] && xk[4 + q4] && xk[8 + q4] && xk[12 + q4];
     if (warp == 4 && lane == 0) TIDAR_TRACE_AT(1536);
-    const float m0 = t == 0 ? m : mo, m1 = t == 0 ? mo : m;
-    const float l0 = t == 0 ? l : lo, l1 = t == 0 ? lo : l;
     const float mt = fmaxf(m0, m1);
     const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - mt);
     const float f1 = (m1 == -INFINITY || nb1 == 0) ? 0.f : ex2(m1 - mt);
@@ -655,39 +799,35 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const bool write = r < rows_valid && ok;
     const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
     const size_t row = (size_t)(b * a.R + (r < rows_valid ? rho : 0)) * a.Hq + h;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    const int col0 = 32 * (2 * t + hf);                  // this thread's 32 output columns
+    {
       uint32_t o0[32], o1[32];
-      const int col0 = 64 * t + 32 * c;
       tmem_ld32(trow + col_o(0) + col0, o0);
       if (nb1 > 0) tmem_ld32(trow + col_o(1) + col0, o1);
       tmem_wait_ld();
-      if (!write) continue;
-      float* v = reinterpret_cast<float*>(o0);
+      if (write) {
+        float* v = reinterpret_cast<float*>(o0);
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        v[e] = __uint_as_float(o0[e]) * g0 + (nb1 > 0 ? __uint_as_float(o1[e]) * g1 : 0.f);
-      if (a.nsplit == 1) {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + row * 128 + col0;
+        for (int e = 0; e < 32; ++e)
+          v[e] = __uint_as_float(o0[e]) * g0 + (nb1 > 0 ? __uint_as_float(o1[e]) * g1 : 0.f);
+        if (a.nsplit == 1) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + row * 128 + col0;
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 u;
-          __nv_bfloat162 t0 = __floats2bfloat162_rn(v[e], v[e + 1]);
-          __nv_bfloat162 t1 = __floats2bfloat162_rn(v[e + 2], v[e + 3]);
-          __nv_bfloat162 t2 = __floats2bfloat162_rn(v[e + 4], v[e + 5]);
-          __nv_bfloat162 t3 = __floats2bfloat162_rn(v[e + 6], v[e + 7]);
-          u.x = *reinterpret_cast<uint32_t*>(&t0); u.y = *reinterpret_cast<uint32_t*>(&t1);
-          u.z = *reinterpret_cast<uint32_t*>(&t2); u.w = *reinterpret_cast<uint32_t*>(&t3);
-          *reinterpret_cast<uint4*>(dst + e) = u;
+          for (int e = 0; e < 32; e += 8) {
+            uint4 u;
+            u.x = cvt_bf16x2(v[e], v[e + 1]); u.y = cvt_bf16x2(v[e + 2], v[e + 3]);
+            u.z = cvt_bf16x2(v[e + 4], v[e + 5]); u.w = cvt_bf16x2(v[e + 6], v[e + 7]);
+            *reinterpret_cast<uint4*>(dst + e) = u;
+          }
+        } else {
+          const size_t prow = (size_t)split * a.B * a.R * a.Hq + row;
+          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 128 + col0);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) dst[e / 4] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         }
-      } else {
-        const size_t prow = (size_t)split * a.B * a.R * a.Hq + row;
-        float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 128 + col0);
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) dst[e / 4] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
       }
     }
-    if (write && t == 0) {
+    if (write && t == 0 && hf == 0) {
       if (a.nsplit == 1) {
         if (a.lse_out) a.lse_out[row] = lse;
       } else {

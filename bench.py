@@ -12,12 +12,13 @@ Inputs are seeded synthetic tensors generated on the device.  One rank per GPU
 collective on the data path).
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
-cudaDeviceSynchronize.  Each step replays CUDA graphs captured from the public
-API calls (step attention; verify + commit) and is timed on the device with
-CUDA events on the launching stream.  Steps rotate over enough independent
+cudaDeviceSynchronize.  Each step replays a CUDA graph captured from the public
+API calls (step attention, verify, commit) and is timed on the device with CUDA
+events on the launching stream.  Steps rotate over enough independent
 input/cache copies that each step's working set is evicted from L2 (126 MB)
-before it is reused.  Between steps (outside the events) a third graph restores
-the copy's prefix length and page table so every step does identical work.
+before it is reused.  Between steps (outside the events) a second graph
+restores the copy's prefix length and page table so every step does identical
+work.  The attention call alone is timed the same way in a second pass.
 ms_per_step / value is the mean step time, max over ranks.
 
 Prints one JSON line (rank 0).
@@ -188,22 +189,25 @@ class Step:
         c["cache"]["page_table"].copy_(c["pt0"], non_blocking=True)
 
     def capture(self):
-        """One CUDA graph per copy for each of: step attention, verify + commit,
-        restore.  Replaying them keeps the host out of the timed device work."""
+        """Per copy, one CUDA graph of the whole step (attention, verify, commit),
+        one of the attention call alone, and one that restores the copy's
+        prefix length and page table.  Replaying them keeps the host out of the
+        timed device work."""
         n = len(self.copies)
         for i in range(n):          # first calls outside capture (module load, attributes)
             self.attn(i); self.verify_commit(i); self.restore(i)
         torch.cuda.synchronize()
         self.graphs = []
         for i in range(n):
-            ga, gv, gr = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            gs, ga, gr = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gs):
+                self.attn(i)
+                self.verify_commit(i)
             with torch.cuda.graph(ga):
                 self.attn(i)
-            with torch.cuda.graph(gv):
-                self.verify_commit(i)
             with torch.cuda.graph(gr):
                 self.restore(i)
-            self.graphs.append((ga, gv, gr))
+            self.graphs.append((gs, ga, gr))
         torch.cuda.synchronize()
 
 
@@ -280,33 +284,35 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- timing
 def time_steps(st: Step, K: int, W: int, world: int):
-    """Returns per-step device µs and per-step step_attn µs (lists).  Each step
-    replays the copy's captured graphs; events sit between the graphs on the
-    launching stream, and the restore graph runs outside the timed span."""
+    """Returns per-step device µs and per-call step_attn µs (lists).  Each timed
+    step replays its copy's whole-step graph between two events on the launching
+    stream; the restore graph runs outside the events.  The attention call is
+    timed the same way in a second pass with the attention-only graphs."""
     n = len(st.copies)
     st.capture()
     stream = torch.cuda.current_stream()
-    for i in range(W):
-        ga, gv, gr = st.graphs[i % n]
-        ga.replay(); gv.replay(); gr.replay()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(K):
-        ga, gv, gr = st.graphs[(W + i) % n]
-        e0, e1, e2 = ev[i]
-        e0.record(stream)
-        ga.replay()
-        e1.record(stream)
-        gv.replay()
-        e2.record(stream)
-        gr.replay()
-    torch.cuda.synchronize()
-    barrier(world)
-    step_us = [e0.elapsed_time(e2) * 1e3 for e0, _, e2 in ev]
-    attn_us = [e0.elapsed_time(e1) * 1e3 for e0, e1, _ in ev]
+
+    def run(which, count, warm):
+        for i in range(warm):
+            g = st.graphs[i % n]
+            g[which].replay(); g[2].replay()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(count)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(count):
+            g = st.graphs[(warm + i) % n]
+            ev[i][0].record(stream)
+            g[which].replay()
+            ev[i][1].record(stream)
+            g[2].replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        return [a.elapsed_time(b) * 1e3 for a, b in ev]
+
+    step_us = run(0, K, W)
+    attn_us = run(1, K, W)
     return step_us, attn_us
 
 

@@ -87,6 +87,8 @@ def lib():
         L.tidar_status_string.restype = ctypes.c_char_p
         L.tidar_last_cuda_error.argtypes = []
         L.tidar_last_cuda_error.restype = ctypes.c_char_p
+        L.tidar_debug_set.argtypes = [ctypes.c_int, I]
+        L.tidar_debug_set.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -257,6 +259,16 @@ def commit(cache, accept_count, k, *, max_prefix_len, head_dim=None, num_q_heads
                             _ptr(released), _ptr(num_released), _stream_handle(stream))
     _check(st, "tidar_commit")
     return released, num_released
+
+
+DEBUG_STARVE_ATTENTION_LOADS, DEBUG_FORCE_SPLIT_PARTIALS = 1, 2
+
+
+def debug_set(knob: int, value: int) -> None:
+    """Test hooks (include/tidar.h): DEBUG_STARVE_ATTENTION_LOADS makes the
+    tensor-core attention's bounded waits run out; DEBUG_FORCE_SPLIT_PARTIALS
+    sends key splits through workspace partials instead of the on-chip merge."""
+    _check(lib().tidar_debug_set(knob, int(value)), "tidar_debug_set")
 
 
 def device_status(stream=None) -> tuple[int, int]:

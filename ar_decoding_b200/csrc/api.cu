@@ -81,10 +81,13 @@ bool tc05_supported(const tidar_step_desc* d) {
 
 constexpr int kNumSMs = 148;
 
+int g_force_partials = 0;   // TIDAR_DEBUG_FORCE_SPLIT_PARTIALS
+
 struct Plan {
   int path;    // 1 SIMT, 2 TC05
   int nsplit;
   int keys_per_split;
+  bool cluster_merge;   // TC05: splits merged on chip in one cluster (no partials, no finalize)
 };
 
 // Key ranges are multiples of 128 keys.  SIMT: aim for ~2 waves of 4-warp CTAs.
@@ -121,10 +124,28 @@ Plan make_plan(const tidar_step_desc* d, int path) {
   if (ns > max_ns) ns = max_ns;
   if (ns > 64) ns = 64;
   if (ns < 1) ns = 1;
-  const int bps = (blocks128 + ns - 1) / ns;
-  p.keys_per_split = (bps > 0 ? bps : 1) * 128;
-  p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
-  if (p.nsplit < 1) p.nsplit = 1;
+  auto split_keys = [&](int n) {
+    const int bps = (blocks128 + n - 1) / n;
+    p.keys_per_split = (bps > 0 ? bps : 1) * 128;
+    p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
+    if (p.nsplit < 1) p.nsplit = 1;
+  };
+  split_keys(ns);
+  p.cluster_merge = false;
+  if (path == 2 && p.nsplit > 1 && !g_force_partials) {
+    // Merge on chip when one cluster per (b, g, tile) -- all of them at once --
+    // fits the device: the largest split count of at least half the wanted
+    // one whose clusters are all resident together.  Otherwise the splits
+    // write partials that a second launch merges.
+    for (int n = ns < 16 ? ns : 16; n >= 2 && 2 * n >= ns; --n) {
+      split_keys(n);
+      if (p.nsplit <= n && tidar::tc05_resident_clusters(p.nsplit) >= units) {
+        p.cluster_merge = true;
+        break;
+      }
+    }
+    if (!p.cluster_merge) split_keys(ns);
+  }
   return p;
 }
 
@@ -167,7 +188,7 @@ size_t tidar_step_attn_workspace_bytes(const tidar_step_desc* d) {
   if (check_desc(d) != TIDAR_OK) return 0;
   const int pth = choose_path(d);
   const Plan p = make_plan(d, pth);
-  if (p.nsplit <= 1) return 0;
+  if (p.nsplit <= 1 || p.cluster_merge) return 0;     // merged on chip
   const size_t rows = (size_t)d->batch * tidar::rows_per_seq(d->k) * d->num_q_heads;
   return align256((size_t)p.nsplit * rows * d->head_dim * sizeof(float)) +
          align256((size_t)p.nsplit * rows * sizeof(float));
@@ -206,7 +227,7 @@ tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, 
   a.nsplit = p.nsplit; a.keys_per_split = p.keys_per_split;
   a.bf16 = d->dtype == TIDAR_BF16;
   a.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->head_dim);
-  if (p.nsplit > 1) {
+  if (p.nsplit > 1 && !p.cluster_merge) {
     const size_t rows = (size_t)a.B * a.R * a.Hq;
     a.part_o = static_cast<float*>(workspace);
     a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -216,8 +237,13 @@ tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, 
   cudaError_t e = pth == 2 ? tidar::launch_attn_tc05(a, s) : tidar::launch_attn_simt(a, s);
   if (e == cudaErrorNotSupported) return TIDAR_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return cuda_fail(e);
-  e = tidar::launch_finalize(a, s);
-  if (e != cudaSuccess) return cuda_fail(e);
+  // Split merge and draft-row append: a second launch for the CUDA-core path
+  // and for tensor-core split partials; the tensor-core kernel does both
+  // itself with one split or with the on-chip cluster merge.
+  if (pth == 1 || (p.nsplit > 1 && !p.cluster_merge)) {
+    e = tidar::launch_finalize(a, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   return TIDAR_OK;
 }
 
@@ -241,8 +267,10 @@ tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype d
   if (k > 1 && !drafts) return TIDAR_ERR_INVALID_ARG;
   if (mode == TIDAR_REJECTION && (!uniforms || (k > 1 && !draft_logits)))
     return TIDAR_ERR_INVALID_ARG;
+  if (!tidar::verify_grid_ok(batch, k, mode)) return TIDAR_ERR_UNSUPPORTED;
   const size_t need = tidar::verify_workspace_bytes(batch, k, vocab, mode);
-  if (workspace_bytes < need || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  if (workspace_bytes < need ||
+      (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))))
     return TIDAR_ERR_INVALID_ARG;
   tidar::VerifyArgs a;
   a.B = batch; a.k = k; a.n = k > 0 ? k : 1; a.V = vocab; a.bf16 = dtype == TIDAR_BF16; a.mode = mode;
@@ -262,6 +290,7 @@ tidar_status tidar_commit(const tidar_step_desc* d, const tidar_kv_cache* c,
   if (d->batch == 0) return TIDAR_OK;
   if ((st = check_cache(d, c)) != TIDAR_OK) return st;
   if (!accept_count || !released_pages || !num_released) return TIDAR_ERR_INVALID_ARG;
+  if (!tidar::commit_batch_ok(d->batch, d->k, d->page_size)) return TIDAR_ERR_UNSUPPORTED;
   unsigned int* err = nullptr;
   if ((st = error_word(&err)) != TIDAR_OK) return st;
   tidar::CommitArgs a;
@@ -274,6 +303,14 @@ tidar_status tidar_commit(const tidar_step_desc* d, const tidar_kv_cache* c,
   cudaError_t e = tidar::launch_commit(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return TIDAR_OK;
+}
+
+tidar_status tidar_debug_set(tidar_debug_knob knob, int32_t value) {
+  switch (knob) {
+    case TIDAR_DEBUG_STARVE_ATTENTION_LOADS: tidar::set_starve_loads(value != 0); return TIDAR_OK;
+    case TIDAR_DEBUG_FORCE_SPLIT_PARTIALS: g_force_partials = value != 0; return TIDAR_OK;
+  }
+  return TIDAR_ERR_INVALID_ARG;
 }
 
 tidar_status tidar_get_device_status(tidar_stream_t stream, uint32_t* bits_out) {

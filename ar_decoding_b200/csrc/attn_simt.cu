@@ -25,6 +25,8 @@ constexpr int kWarps = 4;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VPL = D / 32;  // elements per lane
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -116,6 +118,8 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(AttnArgs a) {
 // the merge, copy the draft rows' K/V into the cache at P_b .. P_b+n-1.
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32) finalize_kernel(AttnArgs a, int merge_blocks) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VPL = D / 32;
   if ((int)blockIdx.x < merge_blocks) {
     const int lane = threadIdx.x & 31;
@@ -174,8 +178,7 @@ template <typename T, int D>
 cudaError_t launch_simt_t(const AttnArgs& a, cudaStream_t s) {
   const int M = a.R * a.G;
   dim3 grid((M + kWarps - 1) / kWarps, a.nsplit, a.B * a.Hkv);
-  attn_simt_kernel<T, D><<<grid, kWarps * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(attn_simt_kernel<T, D>, grid, kWarps * 32, 0, s, a);
 }
 
 template <typename T, int D>
@@ -184,8 +187,7 @@ cudaError_t launch_finalize_t(const AttnArgs& a, cudaStream_t s) {
   const int merge_blocks = a.nsplit > 1 ? (int)((rows + kWarps - 1) / kWarps) : 0;
   const int blocks = merge_blocks + a.B * a.n;
   if (blocks == 0) return cudaSuccess;
-  finalize_kernel<T, D><<<blocks, kWarps * 32, 0, s>>>(a, merge_blocks);
-  return cudaGetLastError();
+  return launch_pdl(finalize_kernel<T, D>, dim3(blocks), kWarps * 32, 0, s, a, merge_blocks);
 }
 
 }  // namespace

@@ -88,7 +88,10 @@ struct Tc05Params {
   int rho_per_tile;   // query rows per tile (128 / G)
   int tiles;          // tiles per (b, g)
   float scale_log2;   // softmax scale * log2(e)
+  int starve;         // test hook: issue no K/V copies (the waits for them run out)
 };
+
+int g_starve_loads = 0;   // tidar_debug_starve_attention_loads
 
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -153,7 +156,7 @@ __device__ __forceinline__ uint64_t global_ns() {
 __device__ unsigned long long g_tidar_trace[2048 + 2 * 8192];
 __device__ __forceinline__ bool trace_cta() { return blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0; }
 #define TIDAR_TRACE_AT(slot) do { if (trace_cta()) g_tidar_trace[(slot)] = global_ns(); } while (0)
-#define TIDAR_TRACE_PH(i, ph) do { if ((i) == 2 && warp == 4 && lane == 0) TIDAR_TRACE_AT(1600 + (ph)); } while (0)
+#define TIDAR_TRACE_PH(i, ph) do { if (((i) == 10 || (i) == 11) && lane == 0) TIDAR_TRACE_AT(1700 + 8 * warp + (ph)); } while (0)
 #define TIDAR_TRACE_CTA(which) do { const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
     if (cta_ < 8192) g_tidar_trace[2048 + 2 * cta_ + (which)] = global_ns(); } while (0)
 #else
@@ -243,6 +246,36 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
+}
+
+// Distributed shared memory of the split cluster.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+// Every thread of every CTA of the cluster: shared-memory writes before it are
+// visible to the cluster's reads after it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 #define TIDAR_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
@@ -392,6 +425,8 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
   const AttnArgs& a = prm.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();       // the previous kernel on the stream is complete from here on
+  pdl_trigger();
 
   const int tile = blockIdx.x, split = blockIdx.y;
   const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
@@ -400,7 +435,8 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int rows_valid = (rho1 - rho0) * a.G;
 
   int P = a.seq_lens[b];
-  if (P < 0 || P > a.max_prefix) {
+  const bool len_ok = P >= 0 && P <= a.max_prefix;
+  if (!len_ok) {
     if (threadIdx.x == 0 && tile == 0 && split == 0) raise_error(a.err, TIDAR_DEVERR_BAD_LEN);
     P = 0;
   }
@@ -437,46 +473,62 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t tmem = misc[0];
   if (threadIdx.x == 0) TIDAR_TRACE_AT(1);
 
-  if (bp.nb == 0) {
-    // This split holds no prefix keys of sequence b: an empty partial.
-    if (warp >= 2) {
-      const int r = 32 * (warp & 3) + lane;
-      if (r < rows_valid) {
-        const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
-        const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
-        const size_t prow = (size_t)split * a.B * a.R * a.Hq + row;
-        float4* po = reinterpret_cast<float4*>(a.part_o + prow * 128);
-        for (int i = 0; i < 32; ++i) po[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        a.part_lse[prow] = -INFINITY;
-      }
-    }
-    return;
-  }
+  // This CTA's share of the output, carried past the role branches: the
+  // normalised partial O of 32 columns of one row and its log-sum-exp.
+  float ov[32];
+  float olse = -INFINITY;
+  bool owrite = false;
 
-  if (warp == 0) {
+  if (bp.nb == 0) {
+    // This split holds no prefix keys of sequence b (only possible with
+    // nsplit > 1): it contributes an empty partial (lse = -inf) to the merge.
+  } else if (warp == 0) {
     // ---------------------------------------------------------------- producer
     // Separate K and V rings (3 stages each): a K stage is refilled as soon as
     // its S MMA is done, a V stage when its PV is done, so K runs up to three
-    // blocks ahead of the scores.  One thread polls both rings.
+    // blocks ahead of the scores.  The whole warp runs the loop (lane 0 issues);
+    // the page-table entries of this split come from 32-page windows held one
+    // entry per lane, with the next window already loading, so no issue waits
+    // on a page-table read.
+    constexpr unsigned kAll = 0xffffffffu;
+    int k_phase[kStages] = {-1, -1, -1}, v_phase[kStages] = {-1, -1, -1};
     if (lane == 0) {
-      int k_phase[kStages] = {-1, -1, -1}, v_phase[kStages] = {-1, -1, -1};
       mbar_expect_tx(bar(BAR_Q), 2u * 128u * (uint32_t)(prm.rho_per_tile * a.G));
       tma_load_4d(sb + kOffQ, &tm_q, 0, g * a.G, rho0, b, bar(BAR_Q));
       tma_load_4d(sb + kOffQ + kChunkBytes, &tm_q, 64, g * a.G, rho0, b, bar(BAR_Q));
-      bool bad = false;
-      // one ring's tile of block i: two 64-row pages of the cache, or a window
-      auto issue = [&](int i, bool is_v) {
-        const int s = i % kStages;
-        const uint32_t dst = sb + (is_v ? kOffV : kOffK) + s * kTileBytes;
-        const uint32_t full = bar((is_v ? BAR_VFULL : BAR_KFULL) + s);
-        if (i < bp.npb) {
-          const CUtensorMap* map = is_v ? &tm_vp : &tm_kp;
-          const int start = bp.k0 + i * 128;
-          const int pa = table[start / 64];
-          const bool need_b = start + 64 < bp.kend;
-          const int pb = need_b ? table[start / 64 + 1] : -1;
-          const bool oka = page_ok(pa, a.num_pages), okb = need_b && page_ok(pb, a.num_pages);
-          if (!oka || (need_b && !okb)) bad = true;
+    }
+    const int pg0 = bp.k0 / 64;                                   // k0 is a multiple of 128
+    const int npg = bp.kend > bp.k0 ? (bp.kend - bp.k0 + 63) / 64 : 0;
+    auto load_win = [&](int base) -> int {
+      const int pi = base + lane;
+      return pi < npg ? table[pg0 + pi] : -1;
+    };
+    int kwb = 0, kcur = load_win(0), knxt = load_win(32);
+    int vwb = 0, vcur = kcur, vnxt = knxt;
+    // table entry of relative page pi (warp-uniform, non-decreasing per ring)
+    auto entry = [&](int& base, int& cur, int& nxt, int pi) -> int {
+      while (pi >= base + 32) {
+        base += 32;
+        cur = nxt;
+        nxt = load_win(base + 32);
+      }
+      return __shfl_sync(kAll, cur, pi - base);
+    };
+    bool bad = false;
+    // one ring's tile of block i: two 64-row pages of the cache, or a window
+    auto issue = [&](int i, bool is_v) {
+      const int s = i % kStages;
+      const uint32_t dst = sb + (is_v ? kOffV : kOffK) + s * kTileBytes;
+      const uint32_t full = bar((is_v ? BAR_VFULL : BAR_KFULL) + s);
+      if (i < bp.npb) {
+        const CUtensorMap* map = is_v ? &tm_vp : &tm_kp;
+        const int start = bp.k0 + i * 128;
+        const bool need_b = start + 64 < bp.kend;
+        const int pa = is_v ? entry(vwb, vcur, vnxt, 2 * i) : entry(kwb, kcur, knxt, 2 * i);
+        const int pb = is_v ? entry(vwb, vcur, vnxt, 2 * i + 1) : entry(kwb, kcur, knxt, 2 * i + 1);
+        const bool oka = page_ok(pa, a.num_pages), okb = need_b && page_ok(pb, a.num_pages);
+        if (!oka || (need_b && !okb)) bad = true;
+        if (lane == 0) {
           mbar_expect_tx(full, (uint32_t)(oka + okb) * 2u * 8192u);
           if (oka) {
             tma_load_2d(dst, map, 0, (pa * a.Hkv + g) * 64, full);
@@ -486,36 +538,44 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tma_load_2d(dst + 8192, map, 0, (pb * a.Hkv + g) * 64, full);
             tma_load_2d(dst + kChunkBytes + 8192, map, 64, (pb * a.Hkv + g) * 64, full);
           }
-        } else {
-          const CUtensorMap* map = is_v ? &tm_vs : &tm_ks;
-          const int w = bp.wins[i - bp.npb];
-          mbar_expect_tx(full, kTileBytes);
-          tma_load_4d(dst, map, 0, g, w * 128, b, full);
-          tma_load_4d(dst + kChunkBytes, map, 64, g, w * 128, b, full);
         }
-        (is_v ? v_phase : k_phase)[s] = i / kStages;
-      };
-      int ik = 0, iv = 0;
-      uint64_t last = global_ns();
-      while ((ik < bp.nb || iv < bp.nb) && !*abort_flag) {
-        bool progress = false;
-        if (ik < bp.nb &&
-            (ik < kStages || mbar_test(bar(BAR_KEMPTY + ik % kStages), (uint32_t)((ik / kStages - 1) & 1)))) {
-          issue(ik, false);
-          TIDAR_TRACE_AT(16 + min(ik, 239));
-          ++ik;
-          progress = true;
-        }
-        if (iv < ik &&
-            (iv < kStages || mbar_test(bar(BAR_VEMPTY + iv % kStages), (uint32_t)((iv / kStages - 1) & 1)))) {
-          issue(iv, true);
-          ++iv;
-          progress = true;
-        }
-        if (progress) {
-          last = global_ns();
-        } else {
-          // sleep briefly on the ring that is further behind, then re-check both
+      } else if (lane == 0) {
+        const CUtensorMap* map = is_v ? &tm_vs : &tm_ks;
+        const int w = bp.wins[i - bp.npb];
+        mbar_expect_tx(full, kTileBytes);
+        tma_load_4d(dst, map, 0, g, w * 128, b, full);
+        tma_load_4d(dst + kChunkBytes, map, 64, g, w * 128, b, full);
+      }
+      (is_v ? v_phase : k_phase)[s] = i / kStages;
+    };
+    // lane 0's view of a barrier phase / the abort flag, for the whole warp
+    auto test_all = [&](uint32_t bar_addr, uint32_t parity) -> bool {
+      const int t = lane == 0 ? (int)mbar_test(bar_addr, parity) : 0;
+      return __shfl_sync(kAll, t, 0) != 0;
+    };
+    auto aborted = [&]() -> bool { return __shfl_sync(kAll, lane == 0 ? *abort_flag : 0, 0) != 0; };
+    int ik = prm.starve ? bp.nb : 0, iv = ik;
+    uint64_t last = global_ns();
+    while ((ik < bp.nb || iv < bp.nb) && !aborted()) {
+      bool progress = false;
+      if (ik < bp.nb &&
+          (ik < kStages || test_all(bar(BAR_KEMPTY + ik % kStages), (uint32_t)((ik / kStages - 1) & 1)))) {
+        issue(ik, false);
+        if (lane == 0) TIDAR_TRACE_AT(16 + min(ik, 239));
+        ++ik;
+        progress = true;
+      }
+      if (iv < ik &&
+          (iv < kStages || test_all(bar(BAR_VEMPTY + iv % kStages), (uint32_t)((iv / kStages - 1) & 1)))) {
+        issue(iv, true);
+        ++iv;
+        progress = true;
+      }
+      if (progress) {
+        last = global_ns();
+      } else {
+        // sleep briefly on the ring that is further behind, then re-check both
+        if (lane == 0) {
           if (ik < bp.nb && ik - iv < kStages)
             mbar_try_wait_ns(bar(BAR_KEMPTY + ik % kStages), (uint32_t)((ik / kStages - 1) & 1), 500u);
           else
@@ -525,7 +585,10 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             raise_error(a.err, TIDAR_DEVERR_TIMEOUT);
           }
         }
+        __syncwarp();
       }
+    }
+    if (lane == 0) {
       if (bad) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
       // Drain: on the normal path every load was consumed; after a timeout make
       // sure no copy is still writing shared memory when the CTA exits.
@@ -805,39 +868,128 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tmem_ld32(trow + col_o(0) + col0, o0);
       if (nb1 > 0) tmem_ld32(trow + col_o(1) + col0, o1);
       tmem_wait_ld();
-      if (write) {
-        float* v = reinterpret_cast<float*>(o0);
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          v[e] = __uint_as_float(o0[e]) * g0 + (nb1 > 0 ? __uint_as_float(o1[e]) * g1 : 0.f);
-        if (a.nsplit == 1) {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + row * 128 + col0;
+      for (int e = 0; e < 32; ++e)
+        ov[e] = __uint_as_float(o0[e]) * g0 + (nb1 > 0 ? __uint_as_float(o1[e]) * g1 : 0.f);
+      if (write && a.nsplit == 1) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + row * 128 + col0;
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 u;
-            u.x = cvt_bf16x2(v[e], v[e + 1]); u.y = cvt_bf16x2(v[e + 2], v[e + 3]);
-            u.z = cvt_bf16x2(v[e + 4], v[e + 5]); u.w = cvt_bf16x2(v[e + 6], v[e + 7]);
-            *reinterpret_cast<uint4*>(dst + e) = u;
-          }
-        } else {
-          const size_t prow = (size_t)split * a.B * a.R * a.Hq + row;
-          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 128 + col0);
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) dst[e / 4] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        for (int e = 0; e < 32; e += 8) {
+          uint4 u;
+          u.x = cvt_bf16x2(ov[e], ov[e + 1]); u.y = cvt_bf16x2(ov[e + 2], ov[e + 3]);
+          u.z = cvt_bf16x2(ov[e + 4], ov[e + 5]); u.w = cvt_bf16x2(ov[e + 6], ov[e + 7]);
+          *reinterpret_cast<uint4*>(dst + e) = u;
         }
+        if (t == 0 && hf == 0 && a.lse_out) a.lse_out[row] = lse;
       }
     }
-    if (write && t == 0 && hf == 0) {
-      if (a.nsplit == 1) {
-        if (a.lse_out) a.lse_out[row] = lse;
-      } else {
-        a.part_lse[(size_t)split * a.B * a.R * a.Hq + row] = lse;
+    owrite = write;
+    olse = lse;
+  }
+
+  // The producer has drained, every MMA is complete and no copy is in flight:
+  // the K ring is free for the split merge.
+  fence_before();
+  __syncthreads();
+
+  if (a.nsplit > 1 && a.part_o) {
+    // ---------------------------------------------------------------- split partials
+    // Too many splits for one wave of clusters: this split's normalised O and
+    // lse go to the workspace and the finalize launch merges them.
+    if (warp >= 2) {
+      const int r = 32 * (warp & 3) + lane;
+      const int t = (warp - 2) >> 3, hf = ((warp - 2) >> 2) & 1;
+      if (r < rows_valid) {
+        const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
+        const size_t prow = (size_t)split * a.B * a.R * a.Hq + (size_t)(b * a.R + rho) * a.Hq + h;
+        if (owrite) {
+          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 128 + 32 * (2 * t + hf));
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) dst[e / 4] = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
+        }
+        if (t == 0 && hf == 0) a.part_lse[prow] = owrite ? olse : -INFINITY;
       }
+    }
+  } else if (a.nsplit > 1) {
+    // ---------------------------------------------------------------- split merge
+    // The CTAs of this cluster are the splits of one (b, g, tile).  Each leaves
+    // its normalised partial O (fp32 [128 rows][32 float4 chunks], chunk index
+    // XOR (row & 7) against bank conflicts) and per-row lse in its K ring;
+    // after a cluster barrier, CTA `rank` merges rows [rank*rpc, ...) from all
+    // splits over distributed shared memory and writes bf16 O and lse.
+    float* po = reinterpret_cast<float*>(smem + kOffK);
+    float* pl = reinterpret_cast<float*>(smem + kOffK + 128 * 512);
+    if (warp >= 2) {
+      const int r = 32 * (warp & 3) + lane;
+      const int t = (warp - 2) >> 3, hf = ((warp - 2) >> 2) & 1;
+      const int c0 = 8 * (2 * t + hf);                   // first float4 chunk of this thread
+      if (owrite) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<float4*>(po + (r * 32 + ((c0 + c) ^ (r & 7))) * 4) =
+              make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
+      }
+      if (t == 0 && hf == 0) pl[r] = owrite ? olse : -INFINITY;
+    }
+    cluster_sync_all();
+    const int ns = a.nsplit;
+    const uint32_t rank = cluster_rank();
+    const int rpc = (rows_valid + ns - 1) / ns;
+    const int r_lo = (int)rank * rpc, r_hi = min(rows_valid, r_lo + rpc);
+    const uint32_t po_s = smem_u32(po), pl_s = smem_u32(pl);
+    for (int R = r_lo + warp; R < r_hi; R += kThreads / 32) {
+      float l2 = -INFINITY;
+      if (lane < ns) l2 = ld_cluster_f32(mapa(pl_s + 4u * R, (uint32_t)lane)) * 1.4426950408889634f;
+      float mx = l2;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float w = (lane < ns && l2 != -INFINITY) ? ex2(l2 - mx) : 0.f;
+      float wsum = w;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const uint32_t off = 4u * (R * 32 + (lane ^ (R & 7))) * 4u;
+      for (int s2 = 0; s2 < ns; ++s2) {
+        const float ws = __shfl_sync(0xffffffffu, w, s2);
+        if (ws != 0.f) {
+          const float4 x = ld_cluster_f32x4(mapa(po_s + off, (uint32_t)s2));
+          acc.x = fmaf(ws, x.x, acc.x); acc.y = fmaf(ws, x.y, acc.y);
+          acc.z = fmaf(ws, x.z, acc.z); acc.w = fmaf(ws, x.w, acc.w);
+        }
+      }
+      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+      const int rho = rho0 + R / a.G, h = g * a.G + R % a.G;
+      const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
+      uint2 u;
+      u.x = cvt_bf16x2(acc.x * inv, acc.y * inv);
+      u.y = cvt_bf16x2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + row * 128 + 4 * lane) = u;
+      if (lane == 0 && a.lse_out)
+        a.lse_out[row] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
+    }
+    cluster_sync_all();   // no CTA leaves while another may still read its shared memory
+  }
+
+  if (tile == 0 && split == 0 && len_ok && !a.part_o) {
+    // ---------------------------------------------------------------- append
+    // Draft rows D_1..D_n of KV head g into cache rows P .. P+n-1 (the keys
+    // above read them from k_blk / v_blk, not from the cache).
+    for (int c = threadIdx.x; c < a.n * 2 * 16; c += kThreads) {
+      const int r = c >> 5, which = (c >> 4) & 1, piece = c & 15;
+      const int pos = P + r;
+      const int page = table[pos / 64];
+      if (!page_ok(page, a.num_pages)) {
+        if (piece == 0 && which == 0) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
+        continue;
+      }
+      const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(which ? a.v_blk : a.k_blk) +
+                                 ((size_t)(b * a.R + r) * a.Hkv + g) * 128 + piece * 8;
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(const_cast<void*>(which ? a.v_pages : a.k_pages)) +
+                           ((size_t)(page * a.Hkv + g) * 64 + pos % 64) * 128 + piece * 8;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
     }
   }
 
-  fence_before();
-  __syncthreads();
   if (threadIdx.x == 0) {
     TIDAR_TRACE_AT(1537);
     TIDAR_TRACE_CTA(1);
@@ -845,7 +997,7 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (trace_cta()) g_tidar_trace[3] = clock64();
 #endif
   }
-  if (warp == 1) {
+  if (warp == 1 && bp.nb > 0) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
@@ -875,7 +1027,24 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, 
   return r == CUDA_SUCCESS;
 }
 
+// The kernel's dynamic shared memory opt-in, once per device.
+cudaError_t set_smem_attr() {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorNotSupported;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(attn_tc05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
+
+void set_starve_loads(int on) { g_starve_loads = on != 0; }
 
 #ifdef TIDAR_TRACE
 extern "C" int tidar_trace_read(void* dst, size_t bytes) {
@@ -894,6 +1063,7 @@ cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s) {
   prm.rho_per_tile = 128 / a.G;
   prm.tiles = (a.R + prm.rho_per_tile - 1) / prm.rho_per_tile;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
+  prm.starve = g_starve_loads;
 
   CUtensorMap tq, tkp, tvp, tks, tvs;
   {
@@ -916,19 +1086,42 @@ cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s) {
     if (!encode(&tks, a.k_blk, 4, dims, str, box)) return cudaErrorNotSupported;
     if (!encode(&tvs, a.v_blk, 4, dims, str, box)) return cudaErrorNotSupported;
   }
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = set_smem_attr();
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorNotSupported;
-  if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(attn_tc05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+  if (a.nsplit > 1 && !a.part_o && a.nsplit > kMaxCluster) return cudaErrorNotSupported;
+  const dim3 grid(prm.tiles, a.nsplit, a.B * a.Hkv);
+  // with the cluster merge, the splits of one (b, g, tile) form a cluster
+  const dim3 cluster(1, a.part_o ? 1 : a.nsplit, 1);
+  return launch_clustered(attn_tc05_kernel, grid, cluster, kThreads, kSmemAlloc, s, tq, tkp, tvp, tks, tvs,
+                          prm);
+}
+
+int tc05_resident_clusters(int ns) {
+  static int cache[64][kMaxCluster + 1];
+  if (ns < 1 || ns > kMaxCluster) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev][ns]) return cache[dev][ns] - 1;
+  int n = 0;
+  if (set_smem_attr() == cudaSuccess &&
+      (ns <= 8 || cudaFuncSetAttribute(attn_tc05_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                      cudaSuccess)) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, ns, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemAlloc;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = ns;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_tc05_kernel, &cfg) != cudaSuccess) n = 0;
   }
-  dim3 grid(prm.tiles, a.nsplit, a.B * a.Hkv);
-  attn_tc05_kernel<<<grid, kThreads, kSmemAlloc, s>>>(tq, tkp, tvp, tks, tvs, prm);
-  return cudaGetLastError();
+  cudaGetLastError();
+  cache[dev][ns] = n + 1;
+  return n;
 }
 
 }  // namespace tidar

@@ -7,113 +7,189 @@
 // zeroed, the length advances to P+c and pages that held only rejected rows
 // are released.
 //
-// Two launches, no device-side waits:
-//   scrub   grid (B): sequence b validates its own (P, c, pages), zeroes its
-//           rejected rows with 16-byte stores, clears its released page-table
-//           entries and writes their ids to its fixed slot range
-//           released[b*S .. b*S+S) (-1 padded), then advances seq_lens[b].
-//   compact grid (1): stable in-place compaction of `released` to (b, i) order
-//           and the count.
+// One launch: a single thread-block cluster of C <= 16 CTAs; CTA r owns the
+// contiguous sequences [r*per, (r+1)*per).
+//   1. every CTA validates its own sequences (one warp per sequence, the
+//      page-table entries loaded by parallel lanes) and counts the pages each
+//      releases (-1: invalid, left untouched), then an exclusive scan of the
+//      counts over its own range;
+//   2. cluster barrier; each CTA reads the other CTAs' totals over distributed
+//      shared memory, which gives its base in the (b, i)-ordered release list
+//      and the grand total; a second cluster barrier ends all remote reads;
+//   3. each CTA zeroes the rejected rows of its sequences with 16-byte stores,
+//      writes their released page ids at their final positions, clears those
+//      page-table entries and advances seq_lens; the tail of the list is -1.
+// No device-side waits besides the two hardware cluster barriers.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace tidar {
 
+namespace cg = cooperative_groups;
+
 namespace {
 
-__global__ void __launch_bounds__(256) scrub_kernel(CommitArgs a, int slots) {
-  const int b = blockIdx.x;
-  __shared__ int sP, sc, sok;
-  if (threadIdx.x == 0) {
+constexpr int kCThreads = 512;
+constexpr int kCWarps = kCThreads / 32;
+
+// Shared-memory record of one owned sequence: P, c, release count (-1 =
+// invalid), exclusive prefix within the CTA, then the npm page ids that hold
+// rows P .. P+n-1 (npm = min(n, ceil(n/ps) + 1)).
+struct SeqRec { int P, c, cnt, off; };
+
+__global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a, int slots, int per,
+                                                                    int npm) {
+  pdl_wait();
+  pdl_trigger();
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks();
+  const int rank = (int)cl.block_rank();
+  extern __shared__ int s_dyn[];
+  SeqRec* s_rec = reinterpret_cast<SeqRec*>(s_dyn);
+  int* s_pg = s_dyn + 4 * per;                      // [per][npm]
+  __shared__ int s_total, s_base, s_grand;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int b0 = rank * per;
+  const int nown = max(0, min(a.B, b0 + per) - b0);
+  const int ps = a.page_size;
+
+  // 1. validate, count, keep the pages: one warp per sequence
+  for (int i = wid; i < nown; i += kCWarps) {
+    const int b = b0 + i;
     const int P = a.seq_lens[b], c = a.accept_count[b];
     int ok = 1;
-    if (c < 0 || c > a.n) { raise_error(a.err, TIDAR_DEVERR_BAD_COUNT); ok = 0; }
-    if (ok && P < 0) { raise_error(a.err, TIDAR_DEVERR_BAD_LEN); ok = 0; }
-    if (ok && (P + a.n + a.page_size - 1) / a.page_size > a.max_pages) {
-      raise_error(a.err, TIDAR_DEVERR_BAD_LEN); ok = 0;
+    if (c < 0 || c > a.n) { ok = 0; if (lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_COUNT); }
+    if (ok && (P < 0 || (P + a.n + ps - 1) / ps > a.max_pages)) {
+      ok = 0;
+      if (lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_LEN);
     }
-    for (int r = 0; ok && r < a.n; ++r) {
-      const int page = a.page_table[(size_t)b * a.max_pages + (P + r) / a.page_size];
-      if (page < 0 || page >= a.num_pages) { raise_error(a.err, TIDAR_DEVERR_BAD_PAGE); ok = 0; }
+    if (ok) {
+      const int p0 = P / ps, np = (P + a.n - 1) / ps - p0 + 1;   // np <= npm <= 16
+      bool bad = false;
+      if (lane < np) {
+        const int page = a.page_table[(size_t)b * a.max_pages + p0 + lane];
+        bad = page < 0 || page >= a.num_pages;
+        s_pg[i * npm + lane] = page;
+      }
+      if (__any_sync(0xffffffffu, bad)) {
+        ok = 0;
+        if (lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
+      }
     }
-    sP = P; sc = c; sok = ok;
+    if (lane == 0) {
+      SeqRec r;
+      r.P = P; r.c = c; r.off = 0;
+      r.cnt = ok ? (P + a.n + ps - 1) / ps - (P + c + ps - 1) / ps : -1;
+      s_rec[i] = r;
+    }
   }
   __syncthreads();
-  int32_t* rel = a.released + (size_t)b * slots;
-  if (!sok) {
-    for (int i = threadIdx.x; i < slots; i += blockDim.x) rel[i] = -1;
-    return;
-  }
-  const int P = sP, c = sc;
-  // zero rows P+c .. P+n-1 of every KV head, K and V (16-byte chunks)
-  const int row_chunks = a.D * a.elem_bytes / 16;
-  const int per_row = 2 * a.Hkv * row_chunks;
-  const int total = (a.n - c) * per_row;
-  for (int t = threadIdx.x; t < total; t += blockDim.x) {
-    const int r = c + t / per_row;
-    const int rem = t % per_row;
-    const int which = rem / (a.Hkv * row_chunks);
-    const int g = (rem / row_chunks) % a.Hkv;
-    const int ch = rem % row_chunks;
-    const int pos = P + r;
-    const int page = a.page_table[(size_t)b * a.max_pages + pos / a.page_size];
-    char* base = static_cast<char*>(which ? a.v_pages : a.k_pages);
-    const size_t off = (((size_t)page * a.Hkv + g) * a.page_size + pos % a.page_size) * a.D * a.elem_bytes;
-    reinterpret_cast<uint4*>(base + off)[ch] = make_uint4(0, 0, 0, 0);
-  }
-  __syncthreads();   // every thread has read the page table before it changes
-  if (threadIdx.x == 0) {
-    const int first = (P + c + a.page_size - 1) / a.page_size;
-    const int last = (P + a.n + a.page_size - 1) / a.page_size;
-    int cnt = 0;
-    for (int i = first; i < last; ++i) {
-      int32_t* ent = a.page_table + (size_t)b * a.max_pages + i;
-      if (*ent >= 0) { rel[cnt++] = *ent; *ent = -1; }
+  if (wid == 0) {
+    int run = 0;
+    for (int s0 = 0; s0 < nown; s0 += 32) {
+      const int i = s0 + lane;
+      const int v = i < nown ? max(s_rec[i].cnt, 0) : 0;
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (i < nown) s_rec[i].off = run + x - v;
+      run += __shfl_sync(0xffffffffu, x, 31);
     }
-    for (; cnt < slots; ++cnt) rel[cnt] = -1;
-    a.seq_lens[b] = P + c;
+    if (lane == 0) s_total = run;
   }
+
+  // 2. bases across the cluster
+  cl.sync();
+  if (wid == 0) {
+    int t = 0;
+    if (lane < C) t = *cl.map_shared_rank(&s_total, lane);
+    int sb = lane < rank ? t : 0, sg = t;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sb += __shfl_xor_sync(0xffffffffu, sb, o);
+      sg += __shfl_xor_sync(0xffffffffu, sg, o);
+    }
+    if (lane == 0) { s_base = sb; s_grand = sg; }
+  }
+  cl.sync();
+
+  // 3. release and advance (one warp per sequence), then scrub (whole CTA);
+  //    no page-table reads from here on
+  const int base = s_base;
+  for (int i = wid; i < nown; i += kCWarps) {
+    const SeqRec r = s_rec[i];
+    if (r.cnt < 0) continue;                        // invalid: left untouched
+    const int b = b0 + i;
+    const int p0 = r.P / ps, first = (r.P + r.c + ps - 1) / ps;
+    if (lane < r.cnt) {
+      a.released[base + r.off + lane] = s_pg[i * npm + first - p0 + lane];
+      a.page_table[(size_t)b * a.max_pages + first + lane] = -1;
+    }
+    if (lane == 0) a.seq_lens[b] = r.P + r.c;
+  }
+  const int row_chunks = a.D * a.elem_bytes / 16;
+  const int head_chunks = a.Hkv * row_chunks;       // one row of one of K / V, all heads
+  for (int i = 0; i < nown; ++i) {
+    const SeqRec r = s_rec[i];
+    if (r.cnt < 0) continue;
+    const int p0 = r.P / ps;
+    const int total = (a.n - r.c) * 2 * head_chunks;
+    for (int t = threadIdx.x; t < total; t += kCThreads) {
+      const int rr = t / (2 * head_chunks);
+      const int rem = t - rr * 2 * head_chunks;
+      const int which = rem >= head_chunks;
+      const int hc = rem - which * head_chunks;
+      const int g = hc / row_chunks, ch = hc - g * row_chunks;
+      const int pos = r.P + r.c + rr;
+      const int page = s_pg[i * npm + pos / ps - p0];
+      char* dst = static_cast<char*>(which ? a.v_pages : a.k_pages);
+      const size_t off = (((size_t)page * a.Hkv + g) * ps + pos % ps) * a.D * a.elem_bytes;
+      reinterpret_cast<uint4*>(dst + off)[ch] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  const int grand = s_grand;
+  for (int i = grand + rank * kCThreads + (int)threadIdx.x; i < a.B * slots; i += C * kCThreads)
+    a.released[i] = -1;
+  if (rank == 0 && threadIdx.x == 0) *a.num_released = grand;
 }
 
-__global__ void __launch_bounds__(1024) compact_kernel(int32_t* released, int total, int32_t* num_released) {
-  __shared__ int s_warp[32];
-  __shared__ int s_base;
-  if (threadIdx.x == 0) s_base = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  for (int start = 0; start < total; start += blockDim.x) {
-    const int i = start + threadIdx.x;
-    const int v = i < total ? released[i] : -1;
-    const int keep = v >= 0;
-    const unsigned ball = __ballot_sync(0xffffffffu, keep);
-    const int before = __popc(ball & ((1u << lane) - 1));
-    if (lane == 0) s_warp[w] = __popc(ball);
-    __syncthreads();
-    int off = 0;
-    for (int k = 0; k < w; ++k) off += s_warp[k];
-    int chunk_total = 0;
-    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) chunk_total += s_warp[k];
-    const int base = s_base;
-    __syncthreads();                      // all reads of this chunk are done
-    if (keep) released[base + off + before] = v;   // destination <= source index
-    __syncthreads();
-    if (threadIdx.x == 0) s_base = base + chunk_total;
-    __syncthreads();
-  }
-  const int count = s_base;
-  for (int i = count + threadIdx.x; i < total; i += blockDim.x) released[i] = -1;
-  if (threadIdx.x == 0) *num_released = count;
-}
+int commit_npm(int n, int ps) { return min(n, (n + ps - 1) / ps + 1); }
 
 }  // namespace
 
+// Per owned sequence: a 4-int record and up to 16 page ids, in the dynamic
+// shared memory of the portable cluster of 8 (the worst case) within 200 KB.
+constexpr size_t kCommitSmemMax = 200 * 1024;
+size_t commit_smem(int per, int npm) { return (size_t)per * (4 + npm) * sizeof(int); }
+
+bool commit_batch_ok(int B, int k, int page_size) {
+  const int n = k > 0 ? k : 1;
+  return commit_smem((B + 7) / 8, commit_npm(n, page_size)) <= kCommitSmemMax;
+}
+
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t s) {
+  static int limit_cache[64];
+  static bool smem_set[64];
   const int slots = (a.n + a.page_size - 1) / a.page_size + 1;
-  scrub_kernel<<<a.B, 256, 0, s>>>(a, slots);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  compact_kernel<<<1, 1024, 0, s>>>(a.released, a.B * slots, a.num_released);
-  return cudaGetLastError();
+  const int C = min(a.B, cluster_limit(commit_cluster_kernel, kCThreads, limit_cache));
+  const int per = (a.B + C - 1) / C;
+  const int npm = commit_npm(a.n, a.page_size);
+  const size_t smem = commit_smem(per, npm);
+  if (smem > kCommitSmemMax) return cudaErrorNotSupported;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (smem > 48 * 1024 && dev >= 0 && dev < 64 && !smem_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(commit_cluster_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCommitSmemMax);
+    if (e != cudaSuccess) return e;
+    smem_set[dev] = true;
+  }
+  return launch_cluster(commit_cluster_kernel, C, 1, kCThreads, smem, s, a, slots, per, npm);
 }
 
 }  // namespace tidar

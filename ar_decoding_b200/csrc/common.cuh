@@ -14,6 +14,91 @@ __device__ __forceinline__ void raise_error(unsigned int* err, unsigned int bits
   atomicOr(err, bits);
 }
 
+// Thread-block clusters: the verification and commit kernels exchange their
+// partial results over distributed shared memory inside one cluster.
+constexpr int kMaxCluster = 16;
+
+// Largest cluster (16 CTAs if this device schedules non-portable 16-CTA
+// clusters of `kernel` with `threads` threads, else the portable 8).  The
+// answer is cached per device in `cache`, so the first call -- which also sets
+// the kernel's non-portable-cluster attribute -- should come before any
+// stream capture.
+template <typename Kernel>
+inline int cluster_limit(Kernel kernel, int threads, int (&cache)[64], size_t smem = 0) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  if (cache[dev]) return cache[dev];
+  int limit = 8;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kMaxCluster, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = kMaxCluster;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0) limit = kMaxCluster;
+  }
+  cudaGetLastError();   // a refused query leaves no sticky error behind
+  cache[dev] = limit;
+  return limit;
+}
+
+// Programmatic dependent launch.  Every library kernel is launched so that it
+// may start while the previous kernel on the stream is finishing; it runs its
+// own prologue, then pdl_wait() -- which returns once every earlier grid on
+// the stream has completed and its memory is visible -- before it touches any
+// global data, and pdl_trigger() lets the next kernel launch early.  Both
+// are no-ops when there is no such dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch `kernel` on `grid` with clusters of `cluster` CTAs (none if the
+// cluster is 1x1x1), as a programmatic dependent of the previous kernel.
+template <typename Kernel, typename... Args>
+inline cudaError_t launch_clustered(Kernel kernel, dim3 grid, dim3 cluster, int threads, size_t smem,
+                                    cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  int na = 0;
+  at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cluster.x * cluster.y * cluster.z > 1) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = cluster.x;
+    at[na].val.clusterDim.y = cluster.y;
+    at[na].val.clusterDim.z = cluster.z;
+    ++na;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Plain grid, programmatic dependent of the previous kernel.
+template <typename Kernel, typename... Args>
+inline cudaError_t launch_pdl(Kernel kernel, dim3 grid, int threads, size_t smem, cudaStream_t s,
+                              Args... args) {
+  return launch_clustered(kernel, grid, dim3(1, 1, 1), threads, smem, s, args...);
+}
+
+// Launch `kernel` on grid (cx, gy) with clusters of (cx, 1, 1).
+template <typename Kernel, typename... Args>
+inline cudaError_t launch_cluster(Kernel kernel, int cx, int gy, int threads, size_t smem,
+                                  cudaStream_t s, Args... args) {
+  return launch_clustered(kernel, dim3(cx, gy, 1), dim3(cx, 1, 1), threads, smem, s, args...);
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

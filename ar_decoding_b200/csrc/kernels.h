@@ -31,7 +31,16 @@ cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 // tcgen05/TMEM kernel (bf16, D 128, page 64).  Returns cudaErrorNotSupported if
 // the tensor maps cannot be built.
 cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s);
-// Split merge (when nsplit > 1) and the draft-row append, in one launch.
+// How many clusters of `ns` tcgen05 attention CTAs (one per key split) this
+// device holds at once; 0 if none.  The kernel merges its splits on chip
+// through such a cluster (part_o == nullptr) and then also performs the
+// draft-row append; with part_o set it writes split partials instead and
+// launch_finalize merges and appends.
+int tc05_resident_clusters(int ns);
+// Test hook: launches issue no K/V copies (their bounded waits run out).
+void set_starve_loads(int on);
+// Split merge (when nsplit > 1) and the draft-row append, in one launch
+// (CUDA-core path).
 cudaError_t launch_finalize(const AttnArgs& a, cudaStream_t s);
 
 struct VerifyArgs {
@@ -48,6 +57,7 @@ struct VerifyArgs {
   void* workspace;
 };
 size_t verify_workspace_bytes(int B, int k, int V, int mode);
+bool verify_grid_ok(int B, int k, int mode);   // launch grid fits (grid.y <= 65535)
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s);
 
 struct CommitArgs {
@@ -61,6 +71,7 @@ struct CommitArgs {
   int32_t* num_released;
   unsigned int* err;
 };
+bool commit_batch_ok(int B, int k, int page_size);   // per-sequence records fit shared memory
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t s);
 
 }  // namespace tidar

@@ -22,10 +22,14 @@
 #include <climits>
 #include <math.h>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace tidar {
+
+namespace cg = cooperative_groups;
 
 namespace {
 
@@ -88,6 +92,8 @@ __device__ __forceinline__ int load_chunk(const T* row, int V, int c0, float (&x
 template <typename T>
 __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat* stats, int nchunk,
                                                          bool vec_ok) {
+  pdl_wait();
+  pdl_trigger();
   const int c = blockIdx.x, rr = blockIdx.y;
   const int prow = a.B * a.n;
   const T* row = rr < prow ? static_cast<const T*>(a.logits) + (size_t)rr * a.V
@@ -157,25 +163,128 @@ __device__ void write_outputs(const VerifyArgs& a, int b, int j, int t_star) {
   }
 }
 
-__global__ void greedy_kernel(VerifyArgs a, const ChunkStat* stats, int nchunk) {
-  const int b = blockIdx.x;
-  __shared__ int am[16];
-  if ((int)threadIdx.x < a.n) {
-    const ChunkStat* st = stats + ((size_t)b * a.n + threadIdx.x) * nchunk;
+// Greedy verification in one launch: one thread-block cluster per sequence b.
+// The cluster's C CTAs split the n rows of b into n*S (row, slice) items
+// (S = C / n slices per row when n <= C, else S = 1 and a CTA takes several
+// rows); each CTA streams its items' logits with 16-byte loads and leaves one
+// exact (max, argmax) pair per item in its shared memory.  After a cluster
+// barrier, CTA 0 merges the pairs of each row over distributed shared memory,
+// runs the accept scan with a warp ballot and writes the outputs.  A second
+// cluster barrier keeps every CTA's shared memory alive until CTA 0 has read it.
+constexpr int kGThreads = 512;
+constexpr int kGUnroll = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kGThreads) greedy_cluster_kernel(VerifyArgs a, int S, int vec_ok) {
+  pdl_wait();
+  pdl_trigger();
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks();
+  const int rank = (int)cl.block_rank();
+  const int b = blockIdx.y;
+  __shared__ float s_v[kMaxCluster];
+  __shared__ int s_i[kMaxCluster];
+  __shared__ float w_v[kGThreads / 32];
+  __shared__ int w_i[kGThreads / 32];
+  __shared__ int s_d[16];
+  __shared__ int s_am[16];
+  __shared__ int s_g[16 * 16];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const bool want_g = a.next_drafts && a.block_guesses && a.k > 0;
+  // CTA 0 fetches the drafts and every block's guesses now, so those loads
+  // overlap the logits sweep instead of following the accept decision
+  if (rank == 0) {
+    const int t = threadIdx.x;
+    if (t < a.n) s_d[t] = (t >= 1 && a.k > 1) ? a.drafts[(size_t)b * a.k + t] : -1;
+    if (want_g && t < a.k * a.k) s_g[t] = a.block_guesses[(size_t)b * a.k * a.k + t];
+  }
+  const int L = (((a.V + S - 1) / S) + 7) & ~7;
+  for (int it = rank; it < a.n * S; it += C) {
+    const int row = it / S, sl = it % S;
+    const int lo = sl * L, hi = min(a.V, lo + L);
+    const T* p = static_cast<const T*>(a.logits) + ((size_t)b * a.n + row) * a.V;
     float bv = -INFINITY;
     int bi = INT_MAX;
-    for (int c = 0; c < nchunk; ++c) amax_merge(bv, bi, st[c].max, st[c].arg);
-    am[threadIdx.x] = bi;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int j = 1;
-    for (int i = 1; i <= a.n - 1; ++i) {
-      if (a.drafts[(size_t)b * a.k + i] != am[i - 1]) break;
-      j = i + 1;
+    if (vec_ok) {
+      constexpr int kVec = 16 / sizeof(T);
+      constexpr int kStride = kGThreads * kVec;
+      for (int base = lo + (int)threadIdx.x * kVec; base < hi; base += kStride * kGUnroll) {
+        float v[kGUnroll][kVec];
+#pragma unroll
+        for (int u = 0; u < kGUnroll; ++u) {
+          const int e0 = base + u * kStride;
+          if (e0 + kVec <= hi) {
+            load_vec<T, kVec>(p + e0, v[u]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) v[u][e] = e0 + e < hi ? ld(p, e0 + e) : -INFINITY;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kGUnroll; ++u)
+#pragma unroll
+          for (int e = 0; e < kVec; ++e) {
+            const int id = base + u * kStride + e;
+            if (id < hi && (v[u][e] > bv || bi == INT_MAX)) { bv = v[u][e]; bi = id; }
+          }
+      }
+    } else {
+      for (int id = lo + (int)threadIdx.x; id < hi; id += kGThreads) {
+        const float x = ld(p, id);
+        if (x > bv || bi == INT_MAX) { bv = x; bi = id; }
+      }
     }
-    write_outputs(a, b, j, am[j - 1]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+      amax_merge(bv, bi, v2, i2);
+    }
+    if (lane == 0) { w_v[wid] = bv; w_i[wid] = bi; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < kGThreads / 32; ++w) amax_merge(bv, bi, w_v[w], w_i[w]);
+      s_v[it % kMaxCluster] = bv;
+      s_i[it % kMaxCluster] = bi;
+    }
+    __syncthreads();
   }
+  cl.sync();
+  if (rank == 0 && wid == 0) {
+    int am = INT_MAX;
+    if (lane < a.n) {
+      float bv = -INFINITY;
+      int bi = INT_MAX;
+      for (int sl = 0; sl < S; ++sl) {
+        const int it = lane * S + sl;
+        const int owner = it % C;
+        const float* rv = cl.map_shared_rank(s_v, owner);
+        const int* ri = cl.map_shared_rank(s_i, owner);
+        amax_merge(bv, bi, rv[it % kMaxCluster], ri[it % kMaxCluster]);
+      }
+      am = bi;
+      s_am[lane] = am;
+    }
+    __syncwarp();
+    // d_{i+1} is kept while it equals argmax l_i: j = first mismatching i, else n
+    const bool mism = lane >= 1 && lane < a.n && s_d[lane] != s_am[lane - 1];
+    const unsigned bal = __ballot_sync(0xffffffffu, mism);
+    const int j = bal ? __ffs(bal) - 1 : a.n;
+    const int t_star = s_am[j - 1];
+    if (lane < a.n) {
+      const int e = lane;
+      a.out_tokens[(size_t)b * a.n + e] = e < j - 1 ? s_d[e + 1] : (e == j - 1 ? t_star : -1);
+    }
+    if (a.next_drafts && a.k > 0 && lane < a.k) {
+      const int e = lane;
+      a.next_drafts[(size_t)b * a.k + e] = e == 0 ? t_star : (want_g ? s_g[(j - 1) * a.k + e] : -1);
+    }
+    if (lane == 0) {
+      a.accept_count[b] = j;
+      if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
+    }
+  }
+  cl.sync();
 }
 
 // Row normaliser from chunk stats: M = max of chunk maxima, Z = sum_c
@@ -216,6 +325,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const ChunkStat* stats,
                                                             int nchunk, double* wsum, int* jbuf,
                                                             bool vec_ok) {
+  pdl_wait();
+  pdl_trigger();
   const int c = blockIdx.x, b = blockIdx.y;
   __shared__ int sj;
   __shared__ double sMp, sZp, sMq, sZq;
@@ -282,6 +393,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const ChunkStat* stats,
                                                           int nchunk, const double* wsum,
                                                           const int* jbuf) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const int j = jbuf[b];
   __shared__ int s_chunk, s_resid, s_found;
@@ -365,40 +478,51 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
 }
 
 template <typename T>
+cudaError_t launch_greedy(const VerifyArgs& a, cudaStream_t s) {
+  static int limit_cache[64];
+  const int C = cluster_limit(greedy_cluster_kernel<T>, kGThreads, limit_cache);
+  const int S = a.n <= C ? C / a.n : 1;
+  const int vec_ok = ((size_t)a.V * sizeof(T)) % 16 == 0;
+  return launch_cluster(greedy_cluster_kernel<T>, C, a.B, kGThreads, 0, s, a, S, vec_ok);
+}
+
+template <typename T>
 cudaError_t launch_t(const VerifyArgs& a, cudaStream_t s) {
+  if (a.mode == TIDAR_GREEDY) return launch_greedy<T>(a, s);
   const int nchunk = (a.V + kChunk - 1) / kChunk;
   const bool vec_ok = ((size_t)a.V * sizeof(T)) % 16 == 0;
   ChunkStat* stats = static_cast<ChunkStat*>(a.workspace);
   const int rows = a.B * a.n + (a.mode == TIDAR_REJECTION ? a.B * (a.k > 1 ? a.k - 1 : 0) : 0);
-  stats_kernel<T><<<dim3(nchunk, rows), kThreads, 0, s>>>(a, stats, nchunk, vec_ok);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(stats_kernel<T>, dim3(nchunk, rows), kThreads, 0, s, a, stats, nchunk, vec_ok);
   if (e != cudaSuccess) return e;
-  if (a.mode == TIDAR_GREEDY) {
-    greedy_kernel<<<a.B, 32, 0, s>>>(a, stats, nchunk);
-    return cudaGetLastError();
-  }
   char* base = static_cast<char*>(a.workspace) + (((size_t)rows * nchunk * sizeof(ChunkStat) + 255) & ~(size_t)255);
   double* wsum = reinterpret_cast<double*>(base);
   int* jbuf = reinterpret_cast<int*>(base + (((size_t)a.B * nchunk * 2 * sizeof(double) + 255) & ~(size_t)255));
-  residual_kernel<T><<<dim3(nchunk, a.B), kThreads, 0, s>>>(a, stats, nchunk, wsum, jbuf, vec_ok);
-  e = cudaGetLastError();
+  e = launch_pdl(residual_kernel<T>, dim3(nchunk, a.B), kThreads, 0, s, a, (const ChunkStat*)stats, nchunk, wsum, jbuf,
+                 vec_ok);
   if (e != cudaSuccess) return e;
-  select_kernel<T><<<a.B, kThreads, 0, s>>>(a, stats, nchunk, wsum, jbuf);
-  return cudaGetLastError();
+  return launch_pdl(select_kernel<T>, dim3(a.B), kThreads, 0, s, a, (const ChunkStat*)stats, nchunk,
+                    (const double*)wsum, (const int*)jbuf);
 }
 
 }  // namespace
 
 size_t verify_workspace_bytes(int B, int k, int V, int mode) {
+  if (mode != TIDAR_REJECTION) return 0;   // greedy: the cluster kernel keeps everything on chip
   const size_t nchunk = (V + kChunk - 1) / kChunk;
   const int n = k > 0 ? k : 1;
-  const size_t rows = (size_t)B * n + (mode == TIDAR_REJECTION ? (size_t)B * (k > 1 ? k - 1 : 0) : 0);
+  const size_t rows = (size_t)B * n + (size_t)B * (k > 1 ? k - 1 : 0);
   size_t bytes = ((rows * nchunk * sizeof(ChunkStat) + 255) & ~(size_t)255);
-  if (mode == TIDAR_REJECTION) {
-    bytes += (((size_t)B * nchunk * 2 * sizeof(double) + 255) & ~(size_t)255);
-    bytes += (((size_t)B * sizeof(int) + 255) & ~(size_t)255);
-  }
+  bytes += (((size_t)B * nchunk * 2 * sizeof(double) + 255) & ~(size_t)255);
+  bytes += (((size_t)B * sizeof(int) + 255) & ~(size_t)255);
   return bytes;
+}
+
+bool verify_grid_ok(int B, int k, int mode) {
+  const long long n = k > 0 ? k : 1;
+  // grid.y is one sequence (greedy) or one vocab row (rejection statistics)
+  const long long y = mode == TIDAR_REJECTION ? (long long)B * (2 * n - 1) : B;
+  return y <= 65535;
 }
 
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s) {
@@ -450,6 +574,7 @@ extern "C" tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t v
   if (!logits || !accept_count || !out_tokens) return TIDAR_ERR_INVALID_ARG;
   if (k > 1 && !drafts) return TIDAR_ERR_INVALID_ARG;
   if (mode == TIDAR_REJECTION && (!uniforms || (k > 1 && !draft_logits))) return TIDAR_ERR_INVALID_ARG;
+  if (!tidar::verify_grid_ok(batch, k, mode)) return TIDAR_ERR_UNSUPPORTED;
   // too large for the fixed scratch: refuse before touching the device
   if (tidar::verify_workspace_bytes(batch, k, vocab, mode) > tidar::kNoAllocScratchBytes)
     return TIDAR_ERR_UNSUPPORTED;

@@ -167,7 +167,7 @@ class Step:
         cap = cfg.B * ((cfg.n + cfg.page_size - 1) // cfg.page_size + 1)
         self.rel = torch.empty(cap, dtype=torch.int32, device=dev)
         self.nrel = torch.empty(1, dtype=torch.int32, device=dev)
-        self.launches_per_step = 2 + 2 + 2   # attention+finalize, stats+accept, scrub+compact
+        self.launches_per_step = 2 + 1 + 1   # attention+finalize, greedy verify (cluster), commit (cluster)
 
     def attn(self, i):
         c = self.copies[i]

@@ -165,8 +165,10 @@ tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, in
  *   block_guesses [B][k][k] int32 slot guesses of each mask block, or NULL
  *   accept_count  [B] int32      out_tokens [B][n] int32
  *   next_drafts   [B][k] int32 or NULL      selected_block [B] int32 or NULL
- *   workspace: at least tidar_verify_workspace_bytes(...) bytes, 256-aligned.
- * A draft token outside [0, V) is never accepted.
+ *   workspace: at least tidar_verify_workspace_bytes(...) bytes, 256-aligned
+ *     (greedy needs none: 0 bytes, NULL allowed).
+ * A draft token outside [0, V) is never accepted.  TIDAR_ERR_UNSUPPORTED when
+ * the launch grid does not fit: greedy B > 65535, rejection B*(2n-1) > 65535.
  * ------------------------------------------------------------------------- */
 size_t tidar_verify_workspace_bytes(int32_t batch, int32_t k, int32_t vocab,
                                     tidar_accept_mode mode);
@@ -221,7 +223,10 @@ tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t vocab, tidar
  *     (b, i) order, then -1; num_released: [1] int32.
  * tidar_verify produces c in 1..n; c = 0 (evict every draft row) is allowed.
  * Device errors: BAD_COUNT (c out of range) or BAD_PAGE (a draft row without
- * a valid page): that sequence is left untouched.
+ * a valid page): that sequence is left untouched.  TIDAR_ERR_UNSUPPORTED when
+ * the per-sequence bookkeeping of the one launch (a single thread-block
+ * cluster) exceeds its shared memory: B * (4 + min(n, ceil(n/ps) + 1)) * 4
+ * bytes > 8 * 200 KiB (B > 68266 at page 64).
  * ------------------------------------------------------------------------- */
 tidar_status tidar_commit(const tidar_step_desc* desc, const tidar_kv_cache* cache,
                           const int32_t* accept_count, int32_t* released_pages,
@@ -236,6 +241,26 @@ tidar_status tidar_get_device_status(tidar_stream_t stream, uint32_t* bits_out);
 const char* tidar_status_string(tidar_status status);
 /* Text of the last CUDA error seen by this thread's calls (host string). */
 const char* tidar_last_cuda_error(void);
+
+/* ---------------------------------------------------------------------------
+ * Test hooks (no counterpart in the paper).  Process-wide host flags, read
+ * when a call is launched; all off by default.
+ *   TIDAR_DEBUG_STARVE_ATTENTION_LOADS: tensor-core step attentions issue no
+ *     K/V copies, so their bounded mbarrier waits run out (after about 1 s):
+ *     the CTAs record TIDAR_DEVERR_TIMEOUT, release TMEM and exit, the
+ *     outputs are unspecified, tidar_get_device_status returns
+ *     TIDAR_ERR_TIMEOUT and the CUDA context stays usable (failure injection).
+ *   TIDAR_DEBUG_FORCE_SPLIT_PARTIALS: the tensor-core path merges key splits
+ *     through workspace partials and a second launch even where it would
+ *     merge them on chip (so tests reach both merges).  Changes the
+ *     workspace size that tidar_step_attn_workspace_bytes reports.
+ * Returns TIDAR_ERR_INVALID_ARG for an unknown knob.
+ * ------------------------------------------------------------------------- */
+typedef enum {
+  TIDAR_DEBUG_STARVE_ATTENTION_LOADS = 1,
+  TIDAR_DEBUG_FORCE_SPLIT_PARTIALS = 2
+} tidar_debug_knob;
+tidar_status tidar_debug_set(tidar_debug_knob knob, int32_t value);
 
 #ifdef __cplusplus
 }

@@ -71,12 +71,28 @@ def test_step_attn_rejects_null_and_misaligned(L):
 
 
 def test_step_attn_rejects_small_workspace(L):
-    d = _desc(max_prefix_len=8192, batch=1, num_q_heads=32, num_kv_heads=8, k=0)
+    # CUDA-core path: split partials go through the workspace
+    d = _desc(max_prefix_len=8192, batch=1, num_q_heads=32, num_kv_heads=8, k=0,
+              path=tidar.PATH_SIMT)
     c = _cache(max_pages_per_seq=129)
     need = L.tidar_step_attn_workspace_bytes(ctypes.byref(d))
     assert need > 0
     assert _attn(L, d, c, ws=FAKE, wsb=need - 1) == tidar.ERR_INVALID_ARG
     assert _attn(L, d, c, ws=FAKE + 16, wsb=need) == tidar.ERR_INVALID_ARG   # not 256-aligned
+
+
+def test_tensor_core_plan_splits_long_prefixes(L):
+    # one query row per head: the 8192-key prefix is split to fill the SMs; the
+    # workspace holds split partials unless the device merges them on chip
+    d = _desc(max_prefix_len=8192, batch=1, num_q_heads=32, num_kv_heads=8, k=0,
+              path=tidar.PATH_TC05)
+    path, splits = ctypes.c_int32(), ctypes.c_int32()
+    assert L.tidar_step_attn_plan(ctypes.byref(d), ctypes.byref(path), ctypes.byref(splits)) == tidar.OK
+    assert path.value == 2 and splits.value > 1
+    ws = L.tidar_step_attn_workspace_bytes(ctypes.byref(d))
+    rows = 32                                  # B * R * Hq
+    assert ws in (0, ((splits.value * rows * 128 * 4 + 255) // 256 * 256) +
+                  ((splits.value * rows * 4 + 255) // 256 * 256))
 
 
 def test_batch_zero_is_a_noop(L):

@@ -94,6 +94,51 @@ def test_8b_class_k_sweep_sampled(oracle_mod, path, k):
     _check_sampled(oracle_mod, synth.class_8b(k=k), path, 160)
 
 
+class _ForcedPartials:
+    """Tensor-core key splits merged through workspace partials (second launch)."""
+    def __enter__(self):
+        tidar.debug_set(tidar.DEBUG_FORCE_SPLIT_PARTIALS, 1)
+
+    def __exit__(self, *exc):
+        tidar.debug_set(tidar.DEBUG_FORCE_SPLIT_PARTIALS, 0)
+
+
+@pytest.mark.parametrize("merge", ["auto", "partials"])
+def test_8b_class_k0_full_every_split_merged(oracle_mod, merge):
+    # k = 0: one query row per head, the prefix cut into many splits; every
+    # output row and the appended cache row are compared
+    cfg = synth.class_8b(k=0)
+    d = tidar.make_desc(torch.empty(1, 1, 32, 128, dtype=torch.bfloat16, device="cuda"),
+                        torch.empty(1, 1, 8, 128, dtype=torch.bfloat16, device="cuda"),
+                        to_dev(synth.make_cache(cfg)), 0, max(cfg.prefix), path="tc05")
+    if merge == "partials":
+        with _ForcedPartials():
+            assert tidar.plan(d)[1] > 8 and tidar.step_attn_workspace_bytes(d) > 0
+            _check_full(oracle_mod, cfg, "tc05")
+    else:
+        assert tidar.plan(d)[1] > 1
+        _check_full(oracle_mod, cfg, "tc05")
+
+
+@pytest.mark.parametrize("path", PATHS + ["tc05-partials"])
+def test_splits_past_a_short_sequence(oracle_mod, path):
+    # sequence 1 is far shorter than sequence 0: most of its key splits hold no
+    # prefix key and contribute an empty partial to the merge
+    cfg = synth.StepConfig("ragged-splits", B=2, Hq=8, Hkv=2, D=128, k=4, prefix=(4096, 300),
+                           dtype="bf16", seed=57)
+    if path == "tc05-partials":
+        with _ForcedPartials():
+            _check_full(oracle_mod, cfg, "tc05")
+    else:
+        _check_full(oracle_mod, cfg, path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("B,P,k", [(1, 32768, 16), (4, 32768, 4), (1, 131072, 0)])
+def test_long_context_sampled(oracle_mod, path, B, P, k):
+    _check_sampled(oracle_mod, synth.long_context(B, P, k), path, 120)
+
+
 @pytest.mark.parametrize("path", PATHS)
 def test_serving_ragged_sampled(oracle_mod, path):
     cfg = synth.serving()
@@ -116,3 +161,21 @@ def test_step_attn_reports_bad_length():
     tidar.step_attn(step["q"], step["k_blk"], step["v_blk"], cache, cfg.k, max_prefix_len=50)
     st, bits = tidar.device_status()
     assert st == tidar.ERR_DEVICE and bits & tidar.DEVERR_BAD_LEN
+
+
+def test_attention_wait_timeout_is_reported_and_recovered(oracle_mod):
+    # failure injected on the host: the producer issues no copies, so the
+    # kernel's bounded waits run out (~1 s); the call must report a timeout,
+    # and the same context must then compute a correct step
+    cfg = synth.StepConfig("starve", B=1, Hq=4, Hkv=1, D=128, k=2, prefix=(256,), dtype="bf16",
+                           seed=61)
+    cache, step = to_dev(synth.make_cache(cfg)), to_dev(synth.make_step(cfg))
+    tidar.debug_set(tidar.DEBUG_STARVE_ATTENTION_LOADS, 1)
+    try:
+        tidar.step_attn(step["q"], step["k_blk"], step["v_blk"], cache, cfg.k, max_prefix_len=256,
+                        path="tc05")
+    finally:
+        tidar.debug_set(tidar.DEBUG_STARVE_ATTENTION_LOADS, 0)
+    st, bits = tidar.device_status()
+    assert st == tidar.ERR_TIMEOUT and bits & tidar.DEVERR_TIMEOUT
+    _check_full(oracle_mod, cfg, "tc05")

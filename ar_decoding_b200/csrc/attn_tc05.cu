@@ -43,7 +43,6 @@ namespace {
 constexpr int kThreads = 576;       // producer, MMA, 16 softmax warps
 constexpr int kStages = 3;       // K/V ring depth; also the number of S buffers
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // every mbarrier wait gives up after ~1 s
-constexpr uint32_t kSuspendHintNs = 10000000u;      // one try_wait sleeps at most 10 ms
 
 constexpr uint32_t kChunkBytes = 16384;                 // 128 rows x 128 B (64 bf16)
 constexpr uint32_t kTileBytes = 2 * kChunkBytes;        // 128 x 128 bf16
@@ -106,8 +105,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// Test the phase; if it is incomplete the thread may sleep in hardware until
-// the phase completes or the hint (ns) expires, whichever is first.
 // Non-blocking test of a phase.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -120,6 +117,8 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Test the phase; if it is incomplete the thread may sleep in hardware until
+// the phase completes or the hint (ns) expires, whichever is first.
 __device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
@@ -131,14 +130,17 @@ __device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, 
       : "memory");
   return ok != 0;
 }
+// Test the phase; if it is incomplete the thread may be suspended for a
+// system-dependent time (no explicit hint: the hardware wakes it as soon as
+// the phase completes).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }

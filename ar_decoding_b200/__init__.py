@@ -28,9 +28,9 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "tidar.h")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(6)
 F32, BF16 = 0, 1
 GREEDY, REJECTION = 0, 1
-PATH_AUTO, PATH_SIMT, PATH_TC05 = 0, 1, 2
+PATH_AUTO, PATH_SIMT, PATH_TC05, PATH_DEC = 0, 1, 2, 3
 DEVERR_BAD_PAGE, DEVERR_BAD_LEN, DEVERR_BAD_COUNT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 1, 2, 4, 8, 16
-_PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tc05": PATH_TC05}
+_PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tc05": PATH_TC05, "dec": PATH_DEC}
 
 
 class TidarError(RuntimeError):

@@ -57,7 +57,8 @@ tidar_status check_desc(const tidar_step_desc* d) {
   if (d->page_size != 16 && d->page_size != 32 && d->page_size != 64 && d->page_size != 128)
     return TIDAR_ERR_UNSUPPORTED;
   if (d->dtype != TIDAR_F32 && d->dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
-  if (d->path != TIDAR_PATH_AUTO && d->path != TIDAR_PATH_SIMT && d->path != TIDAR_PATH_TC05)
+  if (d->path != TIDAR_PATH_AUTO && d->path != TIDAR_PATH_SIMT && d->path != TIDAR_PATH_TC05 &&
+      d->path != TIDAR_PATH_DEC)
     return TIDAR_ERR_INVALID_ARG;
   return TIDAR_OK;
 }
@@ -79,12 +80,18 @@ bool tc05_supported(const tidar_step_desc* d) {
   return kTc05Built && d->dtype == TIDAR_BF16 && d->head_dim == 128 && d->page_size == 64;
 }
 
+// Warp-MMA decode kernel: at most 16 packed query rows per KV head.
+bool dec_supported(const tidar_step_desc* d) {
+  return tc05_supported(d) &&
+         (long long)tidar::rows_per_seq(d->k) * (d->num_q_heads / d->num_kv_heads) <= 16;
+}
+
 constexpr int kNumSMs = 148;
 
 int g_force_partials = 0;   // TIDAR_DEBUG_FORCE_SPLIT_PARTIALS
 
 struct Plan {
-  int path;    // 1 SIMT, 2 TC05
+  int path;    // 1 SIMT, 2 TC05, 3 DEC
   int nsplit;
   int keys_per_split;
   bool cluster_merge;   // TC05: splits merged on chip in one cluster (no partials, no finalize)
@@ -107,24 +114,37 @@ Plan make_plan(const tidar_step_desc* d, int path) {
     const int tiles = (M + rows_per_tile - 1) / rows_per_tile;
     units = (long long)d->batch * d->num_kv_heads * tiles;
     target = kNumSMs;
+  } else if (path == 3) {
+    units = (long long)d->batch * d->num_kv_heads;   // one CTA per SM, one wave
+    target = kNumSMs;
   } else {
     units = (long long)d->batch * d->num_kv_heads * ((M + 3) / 4);
     target = 2 * kNumSMs * 4;
   }
   int ns = 1;
-  if (path == 2) {
+  if (path == 2 || path == 3) {
     // one CTA per SM: as many splits as fit in a single wave
     if (units > 0 && units < target) ns = (int)(target / units);
   } else if (units > 0 && units < target) {
     ns = (int)((target + units - 1) / units);
   }
-  // at least 2 key blocks of 128 per split (tensor-core path), 1 for SIMT
-  const int min_blocks = path == 2 ? 2 : 1;
-  const int max_ns = blocks128 / min_blocks > 0 ? blocks128 / min_blocks : 1;
+  // at least 2 key blocks of 128 per split (tensor-core path), 2 pages of 64
+  // (decode path), 1 block for SIMT
+  const int max_ns = path == 3 ? ((maxP + 63) / 64 / 2 > 0 ? (maxP + 63) / 64 / 2 : 1)
+                               : (path == 2 ? (blocks128 / 2 > 0 ? blocks128 / 2 : 1)
+                                            : (blocks128 > 0 ? blocks128 : 1));
   if (ns > max_ns) ns = max_ns;
   if (ns > 64) ns = 64;
   if (ns < 1) ns = 1;
   auto split_keys = [&](int n) {
+    if (path == 3) {                                  // pages of 64 keys
+      const int pages = (maxP + 63) / 64;
+      const int pps = (pages + n - 1) / n;
+      p.keys_per_split = (pps > 0 ? pps : 1) * 64;
+      p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
+      if (p.nsplit < 1) p.nsplit = 1;
+      return;
+    }
     const int bps = (blocks128 + n - 1) / n;
     p.keys_per_split = (bps > 0 ? bps : 1) * 128;
     p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
@@ -132,14 +152,16 @@ Plan make_plan(const tidar_step_desc* d, int path) {
   };
   split_keys(ns);
   p.cluster_merge = false;
-  if (path == 2 && p.nsplit > 1 && !g_force_partials) {
+  if ((path == 2 || path == 3) && p.nsplit > 1 && !g_force_partials) {
     // Merge on chip when one cluster per (b, g, tile) -- all of them at once --
     // fits the device: the largest split count of at least half the wanted
     // one whose clusters are all resident together.  Otherwise the splits
     // write partials that a second launch merges.
     for (int n = ns < 16 ? ns : 16; n >= 2 && 2 * n >= ns; --n) {
       split_keys(n);
-      if (p.nsplit <= n && tidar::tc05_resident_clusters(p.nsplit) >= units) {
+      const int resident = path == 2 ? tidar::tc05_resident_clusters(p.nsplit)
+                                     : tidar::dec_resident_clusters(p.nsplit);
+      if (p.nsplit <= n && resident >= units) {
         p.cluster_merge = true;
         break;
       }
@@ -152,7 +174,8 @@ Plan make_plan(const tidar_step_desc* d, int path) {
 int choose_path(const tidar_step_desc* d) {
   if (d->path == TIDAR_PATH_SIMT) return 1;
   if (d->path == TIDAR_PATH_TC05) return 2;
-  return tc05_supported(d) ? 2 : 1;
+  if (d->path == TIDAR_PATH_DEC) return 3;
+  return dec_supported(d) ? 3 : (tc05_supported(d) ? 2 : 1);
 }
 
 }  // namespace
@@ -178,6 +201,7 @@ tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, in
   if (st != TIDAR_OK) return st;
   const int pth = choose_path(desc);
   if (pth == 2 && !tc05_supported(desc)) return TIDAR_ERR_UNSUPPORTED;
+  if (pth == 3 && !dec_supported(desc)) return TIDAR_ERR_UNSUPPORTED;
   const Plan p = make_plan(desc, pth);
   if (path) *path = p.path;
   if (splits) *splits = p.nsplit;
@@ -206,6 +230,7 @@ tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, 
     return TIDAR_ERR_INVALID_ARG;
   const int pth = choose_path(d);
   if (pth == 2 && !tc05_supported(d)) return TIDAR_ERR_UNSUPPORTED;
+  if (pth == 3 && !dec_supported(d)) return TIDAR_ERR_UNSUPPORTED;
   const Plan p = make_plan(d, pth);
   const size_t need = tidar_step_attn_workspace_bytes(d);
   if (workspace_bytes < need) return TIDAR_ERR_INVALID_ARG;
@@ -234,12 +259,13 @@ tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, 
                                           align256((size_t)p.nsplit * rows * a.D * sizeof(float)));
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = pth == 2 ? tidar::launch_attn_tc05(a, s) : tidar::launch_attn_simt(a, s);
+  cudaError_t e = pth == 2 ? tidar::launch_attn_tc05(a, s)
+                           : (pth == 3 ? tidar::launch_attn_dec(a, s) : tidar::launch_attn_simt(a, s));
   if (e == cudaErrorNotSupported) return TIDAR_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return cuda_fail(e);
   // Split merge and draft-row append: a second launch for the CUDA-core path
-  // and for tensor-core split partials; the tensor-core kernel does both
-  // itself with one split or with the on-chip cluster merge.
+  // and for split partials; the tensor-core and decode kernels do both
+  // themselves with one split or with the on-chip cluster merge.
   if (pth == 1 || (p.nsplit > 1 && !p.cluster_merge)) {
     e = tidar::launch_finalize(a, s);
     if (e != cudaSuccess) return cuda_fail(e);

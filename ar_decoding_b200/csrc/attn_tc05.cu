@@ -35,6 +35,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace tidar {
 
@@ -42,7 +43,6 @@ namespace {
 
 constexpr int kThreads = 576;       // producer, MMA, 16 softmax warps
 constexpr int kStages = 3;       // K/V ring depth; also the number of S buffers
-constexpr uint64_t kWaitLimitNs = 1000000000ull;   // every mbarrier wait gives up after ~1 s
 
 constexpr uint32_t kChunkBytes = 16384;                 // 128 rows x 128 B (64 bf16)
 constexpr uint32_t kTileBytes = 2 * kChunkBytes;        // 128 x 128 bf16
@@ -92,63 +92,6 @@ struct Tc05Params {
 
 int g_starve_loads = 0;   // tidar_debug_starve_attention_loads
 
-// ------------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// Non-blocking test of a phase.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Test the phase; if it is incomplete the thread may sleep in hardware until
-// the phase completes or the hint (ns) expires, whichever is first.
-__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-// Test the phase; if it is incomplete the thread may be suspended for a
-// system-dependent time (no explicit hint: the hardware wakes it as soon as
-// the phase completes).
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 // Optional timeline of one CTA and the start/end of every CTA (build with
 // -DTIDAR_TRACE; absent from normal builds).  Slots: [0..15] setup, [16+i]
 // producer issue of block i, [256+i] MMA sees K(i), [512+i] S(i) issued,
@@ -166,54 +109,6 @@ __device__ __forceinline__ bool trace_cta() { return blockIdx.x == 0 && blockIdx
 #define TIDAR_TRACE_PH(i, ph) do {} while (0)
 #define TIDAR_TRACE_CTA(which) do {} while (0)
 #endif
-
-// Wait for a phase with a time limit, no error reporting (drain paths).
-__device__ __forceinline__ bool wait_quiet(uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
-// Bounded wait.  Gives up after kWaitLimitNs (or early once another thread of
-// the CTA has given up), records the timeout and returns false.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         unsigned int* err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_ns() - t0 > kWaitLimitNs) break;
-  }
-  *abort_flag = 1;
-  raise_error(err, TIDAR_DEVERR_TIMEOUT);
-  return false;
-}
-
-// Bounded wait by a whole warp with a warp-uniform result (the tcgen05.ld/st
-// that follow are .sync.aligned and need every lane).
-__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                              unsigned int* err) {
-  const bool ok = wait_bar(bar, parity, abort_flag, err);
-  return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, int c3, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
-      : "memory");
-}
 
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -248,36 +143,6 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
-}
-
-// Distributed shared memory of the split cluster.
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-// Every thread of every CTA of the cluster: shared-memory writes before it are
-// visible to the cluster's reads after it.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 #define TIDAR_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
@@ -375,12 +240,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2_pos(float a, float b) {
   return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // ------------------------------------------------------------------ block plan
 // Blocks 0..npb-1: 128 prefix keys from k0; then nw step-key windows.
 struct BlockPlan {
@@ -429,6 +288,15 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();       // the previous kernel on the stream is complete from here on
   pdl_trigger();
+  // The producer's first two 32-page windows of the page table do not depend on
+  // the prefix length, so they load alongside it.
+  int win_cur = -1, win_nxt = -1;
+  if (warp == 0) {
+    const int32_t* tb = a.page_table + (size_t)(blockIdx.z / a.Hkv) * a.max_pages;
+    const int pg = blockIdx.y * a.keys_per_split / 64;
+    win_cur = pg + lane < a.max_pages ? tb[pg + lane] : -1;
+    win_nxt = pg + 32 + lane < a.max_pages ? tb[pg + 32 + lane] : -1;
+  }
 
   const int tile = blockIdx.x, split = blockIdx.y;
   const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
@@ -500,12 +368,11 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tma_load_4d(sb + kOffQ + kChunkBytes, &tm_q, 64, g * a.G, rho0, b, bar(BAR_Q));
     }
     const int pg0 = bp.k0 / 64;                                   // k0 is a multiple of 128
-    const int npg = bp.kend > bp.k0 ? (bp.kend - bp.k0 + 63) / 64 : 0;
     auto load_win = [&](int base) -> int {
-      const int pi = base + lane;
-      return pi < npg ? table[pg0 + pi] : -1;
+      const int pi = pg0 + base + lane;
+      return pi < a.max_pages ? table[pi] : -1;
     };
-    int kwb = 0, kcur = load_win(0), knxt = load_win(32);
+    int kwb = 0, kcur = win_cur, knxt = win_nxt;
     int vwb = 0, vcur = kcur, vnxt = knxt;
     // table entry of relative page pi (warp-uniform, non-decreasing per ring)
     auto entry = [&](int& base, int& cur, int& nxt, int pi) -> int {
@@ -1006,29 +873,6 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-            const cuuint32_t* box) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 // The kernel's dynamic shared memory opt-in, once per device.
 cudaError_t set_smem_attr() {
   static bool attr_set[64] = {false};

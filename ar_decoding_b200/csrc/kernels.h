@@ -26,6 +26,13 @@ struct AttnArgs {
   float scale;           // softmax scale (natural-log domain)
 };
 
+// Warp-MMA kernel for query blocks of at most 16 packed rows per KV head
+// (bf16, D 128, page 64; splits in multiples of 64 keys).  Like the tcgen05
+// kernel it merges its splits on chip through a cluster of nsplit CTAs when
+// part_o == nullptr (and then appends the draft rows itself); with part_o set
+// launch_finalize merges and appends.
+cudaError_t launch_attn_dec(const AttnArgs& a, cudaStream_t s);
+int dec_resident_clusters(int ns);
 // CUDA-core kernel (fp32 or bf16, D 64 or 128).
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 // tcgen05/TMEM kernel (bf16, D 128, page 64).  Returns cudaErrorNotSupported if

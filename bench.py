@@ -53,7 +53,7 @@ def parse_args():
     ap.add_argument("--prefix", type=int, default=8192)
     ap.add_argument("--no-sweep", action="store_true", help="skip the k sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc05"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc05", "dec"])
     return ap.parse_args()
 
 
@@ -98,6 +98,9 @@ def reduce_sum(x: float, world: int) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+PATH_NAMES = {1: "simt", 2: "tc05", 3: "dec"}
 
 
 def workload(k: int, prefix: int, rank: int = 0):
@@ -467,7 +470,7 @@ def run_ours(args, rank, world, local):
                           "hbm_frac": (b2 / a2 / 1e9) / hbm_peak,
                           "tc_frac": (f2 / a2 / 1e12) / tc_peak,
                           "roofline_frac": max(b2 / (hbm_peak * 1e9), f2 / (tc_peak * 1e12)) / a2,
-                          "path": "tc05" if s2.path_id == 2 else "simt", "splits": s2.splits})
+                          "path": PATH_NAMES[s2.path_id], "splits": s2.splits})
             del s2
             torch.cuda.empty_cache()
 
@@ -490,7 +493,7 @@ def run_ours(args, rank, world, local):
                        "Hkv": cfg.Hkv, "head_dim": cfg.D, "prefix": args.prefix, "k": args.k,
                        "rows": cfg.R, "vocab": cfg.vocab, "page": cfg.page_size,
                        "l2": f"rotating {len(st.copies)} independent input copies (> 3x L2)",
-                       "attn_path": "tc05" if st.path_id == 2 else "simt",
+                       "attn_path": PATH_NAMES[st.path_id],
                        "splits": st.splits},
             "attn_us": mean_attn, "hbm_gbs_attn": bytes_ / attn_s / 1e9,
             "hbm_gbs_all_gpus": agg_gbs,

@@ -63,9 +63,17 @@ typedef enum {
 typedef enum { TIDAR_F32 = 0, TIDAR_BF16 = 1 } tidar_dtype;
 typedef enum { TIDAR_GREEDY = 0, TIDAR_REJECTION = 1 } tidar_accept_mode;
 
-/* Kernel family for the step attention.  AUTO: tcgen05/TMEM tensor-core
- * kernel for bf16, head_dim 128, page 64; CUDA-core kernel otherwise. */
-typedef enum { TIDAR_PATH_AUTO = 0, TIDAR_PATH_SIMT = 1, TIDAR_PATH_TC05 = 2 } tidar_attn_path;
+/* Kernel family for the step attention.  AUTO picks, for bf16, head_dim 128,
+ * page 64: the warp-MMA decode kernel (DEC) when the query block packs into at
+ * most 16 rows per KV head (R * G <= 16, e.g. plain decode k = 0), else the
+ * tcgen05/TMEM tensor-core kernel (TC05); the CUDA-core kernel (SIMT)
+ * otherwise.  Asking for DEC with R * G > 16 returns TIDAR_ERR_UNSUPPORTED. */
+typedef enum {
+  TIDAR_PATH_AUTO = 0,
+  TIDAR_PATH_SIMT = 1,
+  TIDAR_PATH_TC05 = 2,
+  TIDAR_PATH_DEC = 3
+} tidar_attn_path;
 
 /* Bits of the device error word. */
 #define TIDAR_DEVERR_BAD_PAGE 0x1u      /* a needed page-table entry is -1 or >= num_pages */

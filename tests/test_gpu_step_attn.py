@@ -15,16 +15,26 @@ from gpu_harness import (compare_attention, oracle_attention, run_attention, sam
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["simt", "tc05"]
+PATHS = ["simt", "tc05", "dec"]
 
 
 def _tc05_ok(cfg):
     return cfg.dtype == "bf16" and cfg.D == 128 and cfg.page_size == 64
 
 
+def _dec_ok(cfg):
+    return _tc05_ok(cfg) and cfg.R * (cfg.Hq // cfg.Hkv) <= 16
+
+
+def _supported(cfg, path):
+    # the tensor-core kernel takes bf16, head_dim 128, page 64; the warp-MMA
+    # decode kernel in addition at most 16 packed query rows per KV head
+    return {"tc05": _tc05_ok, "dec": _dec_ok}.get(path, lambda c: True)(cfg)
+
+
 def _check_full(oracle_mod, cfg, path):
-    if path == "tc05" and not _tc05_ok(cfg):
-        return                      # the tensor-core kernel takes bf16, head_dim 128 only
+    if not _supported(cfg, path):
+        return
     cache, step = synth.make_cache(cfg), synth.make_step(cfg)
     out, lse, cache_after = run_attention(cfg, path, cache, step)
     want, want_lse = oracle_attention(oracle_mod, cfg, cache, step)
@@ -79,6 +89,8 @@ def test_1p5b_class_full(oracle_mod, path):
 
 
 def _check_sampled(oracle_mod, cfg, path, count, max_prefix=None):
+    if not _supported(cfg, path):
+        return
     cache, step = synth.make_cache(cfg), synth.make_step(cfg)
     out, lse, _ = run_attention(cfg, path, cache, step, max_prefix=max_prefix)
     sel = sample_rows(cfg, count)
@@ -103,21 +115,44 @@ class _ForcedPartials:
         tidar.debug_set(tidar.DEBUG_FORCE_SPLIT_PARTIALS, 0)
 
 
+@pytest.mark.parametrize("path", ["tc05", "dec"])
 @pytest.mark.parametrize("merge", ["auto", "partials"])
-def test_8b_class_k0_full_every_split_merged(oracle_mod, merge):
+def test_8b_class_k0_full_every_split_merged(oracle_mod, merge, path):
     # k = 0: one query row per head, the prefix cut into many splits; every
     # output row and the appended cache row are compared
     cfg = synth.class_8b(k=0)
     d = tidar.make_desc(torch.empty(1, 1, 32, 128, dtype=torch.bfloat16, device="cuda"),
                         torch.empty(1, 1, 8, 128, dtype=torch.bfloat16, device="cuda"),
-                        to_dev(synth.make_cache(cfg)), 0, max(cfg.prefix), path="tc05")
+                        to_dev(synth.make_cache(cfg)), 0, max(cfg.prefix), path=path)
     if merge == "partials":
         with _ForcedPartials():
             assert tidar.plan(d)[1] > 8 and tidar.step_attn_workspace_bytes(d) > 0
-            _check_full(oracle_mod, cfg, "tc05")
+            _check_full(oracle_mod, cfg, path)
     else:
         assert tidar.plan(d)[1] > 1
-        _check_full(oracle_mod, cfg, "tc05")
+        _check_full(oracle_mod, cfg, path)
+
+
+@pytest.mark.parametrize("path", PATHS + ["dec-partials"])
+def test_decode_splits_past_a_short_sequence(oracle_mod, path):
+    # plain decode (k = 0), sequence 1 far shorter than sequence 0: most of its
+    # splits hold no prefix key; unaligned prefix ends inside a page
+    cfg = synth.StepConfig("ragged-decode", B=3, Hq=8, Hkv=2, D=128, k=0, prefix=(5000, 130, 1),
+                           dtype="bf16", seed=58)
+    if path == "dec-partials":
+        with _ForcedPartials():
+            _check_full(oracle_mod, cfg, "dec")
+    else:
+        _check_full(oracle_mod, cfg, path)
+
+
+def test_auto_picks_the_decode_kernel_for_thin_blocks():
+    q = lambda R, Hq: torch.empty(1, R, Hq, 128, dtype=torch.bfloat16, device="cuda")
+    kb = lambda R, Hkv: torch.empty(1, R, Hkv, 128, dtype=torch.bfloat16, device="cuda")
+    cache = to_dev(synth.make_cache(synth.class_8b(k=0)))
+    assert tidar.plan(tidar.make_desc(q(1, 32), kb(1, 8), cache, 0, 8192))[0] == tidar.PATH_DEC
+    cache16 = to_dev(synth.make_cache(synth.class_8b(k=16)))
+    assert tidar.plan(tidar.make_desc(q(272, 32), kb(272, 8), cache16, 16, 8192))[0] == tidar.PATH_TC05
 
 
 @pytest.mark.parametrize("path", PATHS + ["tc05-partials"])

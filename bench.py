@@ -170,7 +170,11 @@ class Step:
         cap = cfg.B * ((cfg.n + cfg.page_size - 1) // cfg.page_size + 1)
         self.rel = torch.empty(cap, dtype=torch.int32, device=dev)
         self.nrel = torch.empty(1, dtype=torch.int32, device=dev)
-        self.launches_per_step = 2 + 1 + 1   # attention+finalize, greedy verify (cluster), commit (cluster)
+        # attention: one launch when the kernel merges its splits on chip (no
+        # workspace) on the tensor-core or decode path, else kernel + finalize;
+        # then greedy verify (one cluster kernel) and commit (one cluster kernel)
+        self.attn_launches = 1 if (need == 0 and self.path_id in (2, 3)) else 2
+        self.launches_per_step = self.attn_launches + 1 + 1
 
     def attn(self, i):
         c = self.copies[i]
@@ -214,11 +218,16 @@ class Step:
         torch.cuda.synchronize()
 
 
-def measured_traffic(k: int):
+KERNEL_SRC = {2: "attn_tc05.cu", 3: "attn_dec.cu"}
+
+
+def measured_traffic(k: int, path_id: int):
     """DRAM bytes of one attention launch from the committed ncu record, if the
     kernel source is unchanged since the capture; else None."""
     import hashlib
-    src = os.path.join(ROOT, "ar_decoding_b200", "csrc", "attn_tc05.cu")
+    if path_id not in KERNEL_SRC:
+        return None
+    src = os.path.join(ROOT, "ar_decoding_b200", "csrc", KERNEL_SRC[path_id])
     rec = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
@@ -317,6 +326,30 @@ def time_steps(st: Step, K: int, W: int, world: int):
     step_us = run(0, K, W)
     attn_us = run(1, K, W)
     return step_us, attn_us
+
+
+def time_attention_launches(st: Step, reps: int):
+    """Average device time of one tidar_step_attn call: a CUDA graph of one call
+    per input copy, back to back (each copy's KV is cold in L2 when its turn
+    comes), replayed `reps` times between two events on the launching stream."""
+    n = len(st.copies)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            st.attn(i)
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * n)
+    del g
+    return us
 
 
 def time_e2e(st: Step, K: int, W: int):
@@ -442,13 +475,14 @@ def run_ours(args, rank, world, local):
     clocks = ClockSampler(local)
     clocks.start()
     step_us, attn_us = time_steps(st, args.steps, args.warmup, world)
+    kern_us = reduce_max(time_attention_launches(st, max(3, args.steps // 3)), world)
     clk = clocks.stop()
     mean_step = reduce_max(statistics.mean(step_us), world)
     mean_attn = reduce_max(statistics.mean(attn_us), world)
     bytes_, flops = algorithmic(cfg)
     t_mem = bytes_ / (hbm_peak * 1e9)
     t_tc = flops / (tc_peak * 1e12)
-    attn_s = mean_attn * 1e-6
+    attn_s = kern_us * 1e-6
     bound = "tensor" if t_tc > t_mem else "hbm"
     if bound == "tensor":
         achieved, peak, unit = flops / attn_s / 1e12, tc_peak, "TFLOP/s"
@@ -464,8 +498,9 @@ def run_ours(args, rank, world, local):
             s2 = Step(c2, copies_for(c2), path=args.path)
             su, au = time_steps(s2, max(10, args.steps // 2), 3, world)
             b2, f2 = algorithmic(c2)
-            a2 = reduce_max(statistics.mean(au), world) * 1e-6
+            a2 = reduce_max(time_attention_launches(s2, 3), world) * 1e-6
             sweep.append({"k": kk, "rows": c2.R, "step_us": reduce_max(statistics.mean(su), world),
+                          "attn_call_us": reduce_max(statistics.mean(au), world),
                           "attn_us": a2 * 1e6, "attn_hbm_gbs": b2 / a2 / 1e9,
                           "hbm_frac": (b2 / a2 / 1e9) / hbm_peak,
                           "tc_frac": (f2 / a2 / 1e12) / tc_peak,
@@ -495,12 +530,14 @@ def run_ours(args, rank, world, local):
                        "l2": f"rotating {len(st.copies)} independent input copies (> 3x L2)",
                        "attn_path": PATH_NAMES[st.path_id],
                        "splits": st.splits},
-            "attn_us": mean_attn, "hbm_gbs_attn": bytes_ / attn_s / 1e9,
+            "attn_call_us": mean_attn, "attn_us": kern_us, "attn_launches": st.attn_launches,
+            "hbm_gbs_attn": bytes_ / attn_s / 1e9,
             "hbm_gbs_all_gpus": agg_gbs,
-            "roofline": {"kernel": "tidar_step_attn", "bound": bound, "achieved": achieved,
+            "roofline": {"kernel": {2: "attn_tc05_kernel", 3: "attn_dec_kernel"}.get(st.path_id, "tidar_step_attn"),
+                         "bound": bound, "achieved": achieved,
                          "peak": peak, "unit": unit, "frac": achieved / peak,
                          "peak_source": peak_src, "peak_kind": "burst",
-                         "traffic": measured_traffic(args.k) if st.path_id == 2 else None,
+                         "traffic": measured_traffic(args.k, st.path_id),
                          "algorithmic_bytes": bytes_, "algorithmic_flops": flops,
                          "roofline_frac_max_of_both": max(t_mem, t_tc) / attn_s},
             "k_sweep": sweep,

@@ -160,7 +160,7 @@ Plan make_plan(const tidar_step_desc* d, int path) {
     for (int n = ns < 16 ? ns : 16; n >= 2 && 2 * n >= ns; --n) {
       split_keys(n);
       const int resident = path == 2 ? tidar::tc05_resident_clusters(p.nsplit)
-                                     : tidar::dec_resident_clusters(p.nsplit);
+                                     : tidar::dec_resident_clusters(p.nsplit, M);
       if (p.nsplit <= n && resident >= units) {
         p.cluster_merge = true;
         break;

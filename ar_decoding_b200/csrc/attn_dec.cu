@@ -7,16 +7,17 @@
 // decode with k = 0, and k = 1 with G <= 8).  Such a block is far too thin for
 // the 128-row tcgen05 tiles and the step is a stream of the paged KV cache,
 // so this kernel is built to keep HBM busy: one TMA producer warp keeps a
-// 6-stage ring of 64-key K/V pages (192 KB) in flight, and eight compute warps
-// work on two pages at a time (pages alternate between two groups of four
-// warps, so every SM sub-partition has two independent warps); each warp takes
-// 16 keys of its page with mma.sync m16n8k16 (bf16, fp32 accumulate): S = Q K^T,
-// an online softmax in registers, and the score fragments reused directly as
-// the A operand of O += P V.  The eight warps' (max, sum, O) merge in shared
-// memory at the end; key splits go to the workspace and the finalize launch
-// merges them and appends the draft rows.
+// 6-stage ring of 64-key K/V pages (192 KB) in flight, and groups of four
+// compute warps take pages in turn (three groups when the rows fit one 8-row
+// MMA tile, two when they need two), each warp 16 keys of its page, with
+// mma.sync m16n8k16 (bf16, fp32 accumulate) in transposed form so the query
+// rows fill the N dimension: S^T = K Q^T, an online softmax in registers, P^T
+// moved into the B-operand layout with movmatrix, O^T += V^T P^T.  The warps'
+// (max, sum, O) merge in shared memory at the end; key splits merge on chip
+// through a cluster when the wave's clusters fit, else through workspace
+// partials and the finalize launch.
 //
-// Grid (split, b * Hkv); 288 threads (warp 0 producer, warps 1..8 compute).
+// Grid (split, b * Hkv); 32 * (1 + 4 * groups) threads (warp 0 producer).
 // Every mbarrier wait is bounded (~1 s): on expiry the CTA records
 // TIDAR_DEVERR_TIMEOUT, the producer drains the copies it issued, and the CTA
 // exits.
@@ -28,8 +29,14 @@ namespace tidar {
 
 namespace {
 
-constexpr int kDecThreads = 288;
-constexpr int kDecCompute = 8;                          // compute warps: 2 page groups x 4 key quarters
+// NT = number of 8-row query tiles (1: M <= 8, 2: M <= 16).  Compute warps come
+// in page groups of four (one per 16-key quarter of a page); NT = 1 leaves
+// room in the register file for three groups, NT = 2 for two.
+template <int NT> struct DecShape {
+  static constexpr int kGroups = NT == 1 ? 3 : 2;
+  static constexpr int kCompute = 4 * kGroups;
+  static constexpr int kThreads = 32 * (1 + kCompute);
+};
 constexpr int kDecStages = 6;
 constexpr uint32_t kHalfPage = 8192;                    // 64 keys x 64 dims bf16 (one 128-byte swizzled box)
 constexpr uint32_t kPageBytes = 2 * kHalfPage;          // 64 keys x 128 dims
@@ -91,6 +98,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// Transpose of an 8x8 matrix of 16-bit elements held as one fragment register
+// per lane (row lane/4, columns 2*(lane%4) and +1).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -102,10 +116,15 @@ __device__ __forceinline__ uint32_t sw128(uint32_t base, int row, int u) {
   return base + (uint32_t)row * 128u + ((uint32_t)(u ^ (row & 7)) << 4);
 }
 
-__global__ void __launch_bounds__(kDecThreads, 1)
+template <int NT>
+__global__ void __launch_bounds__(DecShape<NT>::kThreads, 1)
 attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
                 const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_ks,
                 const __grid_constant__ CUtensorMap tm_vs, const DecParams prm) {
+  constexpr int kDecThreads = DecShape<NT>::kThreads;
+  constexpr int kDecCompute = DecShape<NT>::kCompute;
+  constexpr int kGroups = DecShape<NT>::kGroups;
+  constexpr int kRows = 8 * NT;                 // query rows held by the MMA tiles
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   const AttnArgs& a = prm.a;
@@ -223,33 +242,47 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else {
     // ---------------------------------------------------------------- compute
-    const int cw = (warp - 1) & 3;                // keys [16cw, 16cw+16) of every page of its group
-    const int grp = (warp - 1) >> 2;              // pages i with i % 2 == grp
-    const int wid = warp - 1;                     // 0..7
-    const int gq = lane >> 2, cq = lane & 3;      // fragment row group and column pair
+    // Transposed formulation, query rows in the MMA N dimension:
+    //   S^T (16 keys x 8 rows) = K (16 keys x 16 dims) . Q^T, eight dim chunks;
+    //   O^T (16 dims x 8 rows) += V^T (16 dims x 16 keys) . P^T, eight dim tiles.
+    // A lane holds rows 8nt + 2cq and + 1 of each n-tile nt, keys gq and gq + 8
+    // of its warp's 16 (S^T fragment), and dims 16mt + gq, + 8 of O^T.
+    const int wid = warp - 1;                     // 0 .. kDecCompute - 1
+    const int cw = wid & 3;                       // keys [16cw, 16cw+16) of every page of its group
+    const int grp = wid >> 2;                     // pages i with i % kGroups == grp
+    const int gq = lane >> 2, cq = lane & 3;
     const float sl2 = prm.scale_log2;
-    // the two query rows this lane's fragments hold, and their zone masks
-    const int r0 = gq, r1 = gq + 8;
-    const StepVis vis0 = step_visibility(a.k, min(r0 / a.G, a.R - 1));
-    const StepVis vis1 = step_visibility(a.k, min(r1 / a.G, a.R - 1));
+    StepVis vis[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) vis[nt][h] = step_visibility(a.k, min((8 * nt + 2 * cq + h) / a.G, a.R - 1));
     bool ok = warp_wait_bar(bar(DBAR_Q), 0, abort_flag, a.err);
     if (wid == 0 && lane == 0) DEC_TRACE(3);
-    uint32_t qa[8][4];
+    // Q^T as the B operand: qb[kk][nt] = {dims 16kk + 2cq.., dims 16kk + 8 + 2cq..} of row 8nt + gq
+    uint32_t qb[8][NT][2];
     {
       const int j = lane >> 3, rr = lane & 7;
-      const int row = rr + (j & 1) * 8;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int d = 16 * kk + (j >> 1) * 8;
-        ldsm_x4(sw128(sb + kOffQd + (d >> 6) * kQHalf, row, (d & 63) >> 3), qa[kk][0], qa[kk][1], qa[kk][2],
-                qa[kk][3]);
+      for (int kk = 0; kk < 8; kk += 2) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          // matrices: (rows 8nt.., dims 16kk), (.., 16kk+8), (.., 16(kk+1)), (.., 16(kk+1)+8)
+          const int d = 16 * kk + j * 8;
+          ldsm_x4(sw128(sb + kOffQd + (d >> 6) * kQHalf, 8 * nt + rr, (d & 63) >> 3), qb[kk][nt][0],
+                  qb[kk][nt][1], qb[kk + 1][nt][0], qb[kk + 1][nt][1]);
+        }
       }
     }
-    float o[16][4];
+    float o[8][NT][4];
 #pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    for (int i = grp; ok && i < nb; i += 2) {
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+    float m[NT][2], l[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) m[nt][0] = m[nt][1] = -INFINITY, l[nt][0] = l[nt][1] = 0.f;
+    for (int i = grp; ok && i < nb; i += kGroups) {
       const int s = i % kDecStages;
       if (!warp_wait_bar(bar(DBAR_FULL + s), (uint32_t)((i / kDecStages) & 1), abort_flag, a.err)) {
         ok = false;
@@ -280,90 +313,91 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         __syncwarp();
       }
-      // S = Q K^T for the warp's 16 keys (two n-tiles of 8); even and odd
-      // dimension chunks accumulate separately to halve the dependent chain
-      float sc[2][4], sd[2][4];
+      // S^T = K Q^T: even and odd dim chunks accumulate separately (shorter
+      // dependent chains)
+      float sc[NT][4], sd[NT][4];
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sc[t][e] = sd[t][e] = 0.f;
+        for (int e = 0; e < 4; ++e) sc[nt][e] = sd[nt][e] = 0.f;
       {
         const int j = lane >> 3, rr = lane & 7;
-        const int key = 16 * cw + (j >> 1) * 8 + rr;
+        const int key = 16 * cw + (j & 1) * 8 + rr;   // matrices: keys 0-7 / 8-15 x dims +0 / +8
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const int d = 16 * kk + (j & 1) * 8;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(sw128(kb + (d >> 6) * kHalfPage, key, (d & 63) >> 3), b0, b1, b2, b3);
-          if (kk & 1) {
-            mma16816(sd[0], qa[kk], b0, b1);
-            mma16816(sd[1], qa[kk], b2, b3);
-          } else {
-            mma16816(sc[0], qa[kk], b0, b1);
-            mma16816(sc[1], qa[kk], b2, b3);
+          const int d = 16 * kk + (j >> 1) * 8;
+          uint32_t ka[4];
+          ldsm_x4(sw128(kb + (d >> 6) * kHalfPage, key, (d & 63) >> 3), ka[0], ka[1], ka[2], ka[3]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            if (kk & 1) mma16816(sd[nt], ka, qb[kk][nt][0], qb[kk][nt][1]);
+            else mma16816(sc[nt], ka, qb[kk][nt][0], qb[kk][nt][1]);
           }
         }
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sc[t][e] += sd[t][e];
       }
-      // mask, scale to the log2 domain, online softmax (stale base up to 2^8)
-      float x[2][4];
+      // mask, log2-domain scale, online softmax per row (stale base up to 2^8)
+      float x[NT][4];
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int kl = 8 * t + 2 * cq + (e & 1);          // key within the warp's 16
+          const int kl = gq + (e >> 1) * 8;             // key within the warp's 16
           bool v = kl < nvalid;
-          if (window) v = v && step_visible(e < 2 ? vis0 : vis1, 16 * cw + kl);
-          x[t][e] = v ? sc[t][e] * sl2 : -INFINITY;
+          if (window) v = v && step_visible(vis[nt][e & 1], 16 * cw + kl);
+          x[nt][e] = v ? (sc[nt][e] + sd[nt][e]) * sl2 : -INFINITY;
         }
-      float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-      float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      const bool up0 = n0 > m0 + 8.0f, up1 = n1 > m1 + 8.0f;
-      if (__any_sync(0xffffffffu, up0 || up1)) {
-        const float f0 = up0 ? ex2(m0 - n0) : 1.0f, f1 = up1 ? ex2(m1 - n1) : 1.0f;   // m = -inf -> 0
-        if (up0) m0 = n0;
-        if (up1) m1 = n1;
-        l0 *= f0;
-        l1 *= f1;
+      float f[NT][2];
+      bool any_up = false;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-          o[n][0] *= f0; o[n][1] *= f0;
-          o[n][2] *= f1; o[n][3] *= f1;
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float mx = fmaxf(x[nt][h], x[nt][h + 2]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float nm = fmaxf(m[nt][h], mx);
+          const bool up = nm > m[nt][h] + 8.0f;
+          f[nt][h] = up ? ex2(m[nt][h] - nm) : 1.0f;      // m = -inf -> 0
+          if (up) m[nt][h] = nm;
+          any_up = any_up || up;
+        }
+      if (__any_sync(0xffffffffu, any_up)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          l[nt][0] *= f[nt][0];
+          l[nt][1] *= f[nt][1];
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            o[mt][nt][0] *= f[nt][0]; o[mt][nt][1] *= f[nt][1];
+            o[mt][nt][2] *= f[nt][0]; o[mt][nt][3] *= f[nt][1];
+          }
         }
       }
-      const float b0s = m0 == -INFINITY ? 0.f : m0, b1s = m1 == -INFINITY ? 0.f : m1;
-      float p[2][4];
+      // P^T, transposed in registers into the B operand of the PV MMA
+      uint32_t pb[NT][2];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        p[t][0] = ex2(x[t][0] - b0s);
-        p[t][1] = ex2(x[t][1] - b0s);
-        p[t][2] = ex2(x[t][2] - b1s);
-        p[t][3] = ex2(x[t][3] - b1s);
-        l0 += p[t][0] + p[t][1];
-        l1 += p[t][2] + p[t][3];
+      for (int nt = 0; nt < NT; ++nt) {
+        const float b0s = m[nt][0] == -INFINITY ? 0.f : m[nt][0];
+        const float b1s = m[nt][1] == -INFINITY ? 0.f : m[nt][1];
+        const float p0 = ex2(x[nt][0] - b0s), p1 = ex2(x[nt][1] - b1s);
+        const float p2 = ex2(x[nt][2] - b0s), p3 = ex2(x[nt][3] - b1s);
+        l[nt][0] += p0 + p2;
+        l[nt][1] += p1 + p3;
+        pb[nt][0] = movmatrix_t(pack_bf16(p0, p1));     // keys 0-7 of the warp's 16
+        pb[nt][1] = movmatrix_t(pack_bf16(p2, p3));     // keys 8-15
       }
-      // the score fragments, as bf16, are the A fragment of P (16 x 16 keys)
-      const uint32_t pa[4] = {pack_bf16(p[0][0], p[0][1]), pack_bf16(p[0][2], p[0][3]),
-                              pack_bf16(p[1][0], p[1][1]), pack_bf16(p[1][2], p[1][3])};
-      // O += P V: sixteen n-tiles of 8 dims, V fragments by transposed ldmatrix
+      // O^T += V^T P^T: eight 16-dim tiles, V^T fragments by transposed ldmatrix
       {
         const int j = lane >> 3, rr = lane & 7;
-        const int key = 16 * cw + (j & 1) * 8 + rr;
+        const int key = 16 * cw + (j >> 1) * 8 + rr;   // matrices: (keys 0-7, dims +0 / +8), (keys 8-15, ..)
 #pragma unroll
-        for (int np = 0; np < 8; ++np) {
-          const int d = 16 * np + (j >> 1) * 8;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sw128(vb + (d >> 6) * kHalfPage, key, (d & 63) >> 3), b0, b1, b2, b3);
-          mma16816(o[2 * np], pa, b0, b1);
-          mma16816(o[2 * np + 1], pa, b2, b3);
+        for (int mt = 0; mt < 8; ++mt) {
+          const int d = 16 * mt + (j & 1) * 8;
+          uint32_t va[4];
+          ldsm_x4_t(sw128(vb + (d >> 6) * kHalfPage, key, (d & 63) >> 3), va[0], va[1], va[2], va[3]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma16816(o[mt][nt], va, pb[nt][0], pb[nt][1]);
         }
       }
       // the stage's shared memory has been read into registers: release it
@@ -373,31 +407,43 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (cw == 0 && lane == 0 && i < 64) DEC_TRACE(80 + i);
     }
     if (wid == 0 && lane == 0) DEC_TRACE(150);
-    // ---- merge the eight warps: (max, sum, O) per row through shared memory
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    asm volatile("bar.sync 1, 256;" ::: "memory");       // every compute warp is past its last stage
-    // [8 warps][16 rows][kXo] fp32: rows padded to 136 floats so the eight row
-    // groups of a fragment store land on distinct banks
+    // ---- merge the compute warps: (max, sum, O) per row through shared memory
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        l[nt][h] += __shfl_xor_sync(0xffffffffu, l[nt][h], 4);
+        l[nt][h] += __shfl_xor_sync(0xffffffffu, l[nt][h], 8);
+        l[nt][h] += __shfl_xor_sync(0xffffffffu, l[nt][h], 16);
+      }
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecCompute) : "memory");   // every compute warp is past its last stage
+    // [warps][kRows rows][kXo] fp32, rows padded to 136 floats against bank conflicts
     constexpr int kXo = 136;
     float* xo = reinterpret_cast<float*>(smem + kOffStage);
-    float* xm = xo + kDecCompute * 16 * kXo;                             // [8][16] max
-    float* xl = xm + kDecCompute * 16;                                   // [8][16] sum
-    int* xk = reinterpret_cast<int*>(xl + kDecCompute * 16);             // [8] status
+    float* xm = xo + kDecCompute * kRows * kXo;                        // [warps][kRows] max
+    float* xl = xm + kDecCompute * kRows;                              // [warps][kRows] sum
+    int* xk = reinterpret_cast<int*>(xl + kDecCompute * kRows);        // [warps] status
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      const int col = 8 * n + 2 * cq;
-      *reinterpret_cast<float2*>(xo + (wid * 16 + r0) * kXo + col) = make_float2(o[n][0], o[n][1]);
-      *reinterpret_cast<float2*>(xo + (wid * 16 + r1) * kXo + col) = make_float2(o[n][2], o[n][3]);
-    }
-    if (cq == 0) {
-      xm[wid * 16 + r0] = m0; xm[wid * 16 + r1] = m1;
-      xl[wid * 16 + r0] = l0; xl[wid * 16 + r1] = l1;
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int r0 = 8 * nt + 2 * cq, d0 = 16 * mt + gq;
+        xo[(wid * kRows + r0) * kXo + d0] = o[mt][nt][0];
+        xo[(wid * kRows + r0 + 1) * kXo + d0] = o[mt][nt][1];
+        xo[(wid * kRows + r0) * kXo + d0 + 8] = o[mt][nt][2];
+        xo[(wid * kRows + r0 + 1) * kXo + d0 + 8] = o[mt][nt][3];
+      }
+    if (gq == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          xm[wid * kRows + 8 * nt + 2 * cq + h] = m[nt][h];
+          xl[wid * kRows + 8 * nt + 2 * cq + h] = l[nt][h];
+        }
     }
     if (lane == 0) xk[wid] = ok ? 1 : 0;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecCompute) : "memory");
     // thread -> (row, 8 columns)
     const int t = threadIdx.x - 32;
     const int row = t >> 4, c0 = (t & 15) * 8;
@@ -408,15 +454,15 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* cpl = reinterpret_cast<float*>(smem + kOffCpl);
     if (prm.cluster && row < 16 && c0 == 0) cpl[row] = -INFINITY;   // overwritten below when valid
     if (row < prm.M && all_ok) {
-      float mt = -INFINITY;
+      float mtop = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kDecCompute; ++w) mt = fmaxf(mt, xm[w * 16 + row]);
-      float f[kDecCompute], lt = 0.f;
+      for (int w = 0; w < kDecCompute; ++w) mtop = fmaxf(mtop, xm[w * kRows + row]);
+      float fw[kDecCompute], lt = 0.f;
 #pragma unroll
       for (int w = 0; w < kDecCompute; ++w) {
-        const float mw = xm[w * 16 + row];
-        f[w] = mw == -INFINITY ? 0.f : ex2(mw - mt);
-        lt += f[w] * xl[w * 16 + row];
+        const float mw = xm[w * kRows + row];
+        fw[w] = mw == -INFINITY ? 0.f : ex2(mw - mtop);
+        lt += fw[w] * xl[w * kRows + row];
       }
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       float v[8];
@@ -424,14 +470,14 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int e = 0; e < 8; ++e) v[e] = 0.f;
 #pragma unroll
       for (int w = 0; w < kDecCompute; ++w) {
-        const float4 x0 = *reinterpret_cast<const float4*>(xo + (w * 16 + row) * kXo + c0);
-        const float4 x1 = *reinterpret_cast<const float4*>(xo + (w * 16 + row) * kXo + c0 + 4);
-        v[0] += f[w] * x0.x; v[1] += f[w] * x0.y; v[2] += f[w] * x0.z; v[3] += f[w] * x0.w;
-        v[4] += f[w] * x1.x; v[5] += f[w] * x1.y; v[6] += f[w] * x1.z; v[7] += f[w] * x1.w;
+        const float4 x0 = *reinterpret_cast<const float4*>(xo + (w * kRows + row) * kXo + c0);
+        const float4 x1 = *reinterpret_cast<const float4*>(xo + (w * kRows + row) * kXo + c0 + 4);
+        v[0] += fw[w] * x0.x; v[1] += fw[w] * x0.y; v[2] += fw[w] * x0.z; v[3] += fw[w] * x0.w;
+        v[4] += fw[w] * x1.x; v[5] += fw[w] * x1.y; v[6] += fw[w] * x1.z; v[7] += fw[w] * x1.w;
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] *= inv;
-      const float lse = lt > 0.f ? (mt + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+      const float lse = lt > 0.f ? (mtop + log2f(lt)) * 0.69314718055994531f : -INFINITY;
       const int rho = row / a.G, h = g * a.G + row % a.G;
       const size_t orow = (size_t)(b * a.R + rho) * a.Hq + h;
       if (prm.cluster) {
@@ -522,6 +568,7 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 }
 
 // The kernel's dynamic shared memory opt-in, once per device.
+template <int NT>
 cudaError_t dec_smem_attr() {
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -529,11 +576,40 @@ cudaError_t dec_smem_attr() {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorNotSupported;
   if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(attn_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    e = cudaFuncSetAttribute(attn_dec_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   return cudaSuccess;
+}
+
+template <int NT>
+int resident_clusters_t(int ns) {
+  static int cache[64][kMaxCluster + 1];
+  if (ns < 1 || ns > kMaxCluster) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev][ns]) return cache[dev][ns] - 1;
+  int n = 0;
+  if (dec_smem_attr<NT>() == cudaSuccess &&
+      (ns <= 8 || cudaFuncSetAttribute(attn_dec_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                      cudaSuccess)) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ns, 1, 1);
+    cfg.blockDim = dim3(DecShape<NT>::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kDecSmem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = ns;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_dec_kernel<NT>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cache[dev][ns] = n + 1;
+  return n;
 }
 
 }  // namespace
@@ -544,32 +620,8 @@ extern "C" int tidar_dec_trace_read(void* dst, size_t bytes) {
 }
 #endif
 
-int dec_resident_clusters(int ns) {
-  static int cache[64][kMaxCluster + 1];
-  if (ns < 1 || ns > kMaxCluster) return 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (cache[dev][ns]) return cache[dev][ns] - 1;
-  int n = 0;
-  if (dec_smem_attr() == cudaSuccess &&
-      (ns <= 8 || cudaFuncSetAttribute(attn_dec_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-                      cudaSuccess)) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ns, 1, 1);
-    cfg.blockDim = dim3(kDecThreads, 1, 1);
-    cfg.dynamicSmemBytes = kDecSmem;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = ns;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, attn_dec_kernel, &cfg) != cudaSuccess) n = 0;
-  }
-  cudaGetLastError();
-  cache[dev][ns] = n + 1;
-  return n;
+int dec_resident_clusters(int ns, int M) {
+  return M <= 8 ? resident_clusters_t<1>(ns) : resident_clusters_t<2>(ns);
 }
 
 cudaError_t launch_attn_dec(const AttnArgs& a, cudaStream_t s) {
@@ -602,10 +654,17 @@ cudaError_t launch_attn_dec(const AttnArgs& a, cudaStream_t s) {
     if (!encode(&tks, a.k_blk, 4, dims, str, box)) return cudaErrorNotSupported;
     if (!encode(&tvs, a.v_blk, 4, dims, str, box)) return cudaErrorNotSupported;
   }
-  cudaError_t e = dec_smem_attr();
+  const dim3 grid(a.nsplit, a.B * a.Hkv), cluster(prm.cluster ? a.nsplit : 1, 1, 1);
+  if (M <= 8) {
+    cudaError_t e = dec_smem_attr<1>();
+    if (e != cudaSuccess) return e;
+    return launch_clustered(attn_dec_kernel<1>, grid, cluster, DecShape<1>::kThreads, kDecSmem, s, tq, tkp, tvp,
+                            tks, tvs, prm);
+  }
+  cudaError_t e = dec_smem_attr<2>();
   if (e != cudaSuccess) return e;
-  return launch_clustered(attn_dec_kernel, dim3(a.nsplit, a.B * a.Hkv), dim3(prm.cluster ? a.nsplit : 1, 1, 1),
-                          kDecThreads, kDecSmem, s, tq, tkp, tvp, tks, tvs, prm);
+  return launch_clustered(attn_dec_kernel<2>, grid, cluster, DecShape<2>::kThreads, kDecSmem, s, tq, tkp, tvp, tks,
+                          tvs, prm);
 }
 
 }  // namespace tidar

@@ -32,7 +32,7 @@ struct AttnArgs {
 // part_o == nullptr (and then appends the draft rows itself); with part_o set
 // launch_finalize merges and appends.
 cudaError_t launch_attn_dec(const AttnArgs& a, cudaStream_t s);
-int dec_resident_clusters(int ns);
+int dec_resident_clusters(int ns, int M);   // M = packed query rows per KV head
 // CUDA-core kernel (fp32 or bf16, D 64 or 128).
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 // tcgen05/TMEM kernel (bf16, D 128, page 64).  Returns cudaErrorNotSupported if

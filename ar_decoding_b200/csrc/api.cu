@@ -43,6 +43,17 @@ tidar_status error_word(unsigned int** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
+namespace tidar {
+unsigned int* device_error_word() {
+  unsigned int* p = nullptr;
+  return error_word(&p) == TIDAR_OK ? p : nullptr;
+}
+}  // namespace tidar
+
+namespace {
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Shape checks shared by step_attn and commit.
@@ -303,6 +314,8 @@ tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype d
   a.logits = logits; a.drafts = drafts; a.draft_logits = draft_logits; a.uniforms = uniforms;
   a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;
   a.next_drafts = next_drafts; a.selected_block = selected_block; a.workspace = workspace;
+  tidar_status est = error_word(&a.err);
+  if (est != TIDAR_OK) return est;
   cudaError_t e = tidar::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return TIDAR_OK;

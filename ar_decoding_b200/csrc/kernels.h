@@ -62,7 +62,10 @@ struct VerifyArgs {
   int32_t* next_drafts;
   int32_t* selected_block;
   void* workspace;
+  unsigned int* err;     // device error word (a bounded wait that ran out)
 };
+// This device's error word (looked up once per device); nullptr on failure.
+unsigned int* device_error_word();
 size_t verify_workspace_bytes(int B, int k, int V, int mode);
 bool verify_grid_ok(int B, int k, int mode);   // launch grid fits (grid.y <= 65535)
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s);

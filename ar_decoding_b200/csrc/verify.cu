@@ -26,6 +26,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace tidar {
 
@@ -59,12 +60,19 @@ __device__ __forceinline__ int load_chunk(const T* row, int V, int c0, float (&x
   constexpr int kVec = 16 / sizeof(T);
   int cnt = 0;
   if (vec_ok) {
+    // the 16-byte loads first, so they are in flight together
+    uint4 raw[kPer / kVec];
+#pragma unroll
+    for (int it = 0; it < kPer / kVec; ++it) {
+      const int base = c0 + (it * kThreads + threadIdx.x) * kVec;
+      raw[it] = base + kVec <= V ? __ldg(reinterpret_cast<const uint4*>(row + base)) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
     for (int it = 0; it < kPer / kVec; ++it) {
       const int base = c0 + (it * kThreads + threadIdx.x) * kVec;
       if (base + kVec <= V) {
         float v[kVec];
-        load_vec<T, kVec>(row + base, v);
+        load_vec<T, kVec>(reinterpret_cast<const T*>(&raw[it]), v);
 #pragma unroll
         for (int e = 0; e < kVec; ++e) { x[it * kVec + e] = v[e]; ix[it * kVec + e] = base + e; }
       } else {
@@ -171,25 +179,51 @@ __device__ void write_outputs(const VerifyArgs& a, int b, int j, int t_star) {
 // barrier, CTA 0 merges the pairs of each row over distributed shared memory,
 // runs the accept scan with a warp ballot and writes the outputs.  A second
 // cluster barrier keeps every CTA's shared memory alive until CTA 0 has read it.
+// Optional timeline of sequence 0's cluster (build with -DTIDAR_TRACE; absent
+// from normal builds): [rank*8 + 0] start, +1 after the previous kernel, +2
+// sweep done, +3 past the first cluster barrier, +4 outputs written, +5 end.
+#ifdef TIDAR_TRACE
+__device__ unsigned long long g_verify_trace[16 * 8];
+__device__ __forceinline__ unsigned long long vt_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define VERIFY_TRACE(rank, slot) do { if (blockIdx.y == 0 && threadIdx.x == 0) g_verify_trace[(rank) * 8 + (slot)] = vt_now(); } while (0)
+#else
+#define VERIFY_TRACE(rank, slot) do {} while (0)
+#endif
+
 constexpr int kGThreads = 512;
 constexpr int kGUnroll = 8;
 
 template <typename T>
 __global__ void __launch_bounds__(kGThreads) greedy_cluster_kernel(VerifyArgs a, int S, int vec_ok) {
-  pdl_wait();
-  pdl_trigger();
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks();
   const int rank = (int)cl.block_rank();
   const int b = blockIdx.y;
-  __shared__ float s_v[kMaxCluster];
+  VERIFY_TRACE(rank, 0);
+  __shared__ float s_v[kMaxCluster];          // CTA 0: one (max, argmax) per item, pushed by its owner
   __shared__ int s_i[kMaxCluster];
+  __shared__ __align__(8) uint64_t s_done;    // CTA 0: one arrival per CTA once its items are pushed
   __shared__ float w_v[kGThreads / 32];
   __shared__ int w_i[kGThreads / 32];
   __shared__ int s_d[16];
   __shared__ int s_am[16];
   __shared__ int s_g[16 * 16];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const uint32_t done_bar = static_cast<uint32_t>(__cvta_generic_to_shared(&s_done));
+  if (rank == 0 && threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(done_bar), "r"(C) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // CTA 0's barrier is initialised (and every CTA running) before anyone pushes
+  // to it; the wait comes after the sweep, so this costs nothing
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  pdl_wait();
+  pdl_trigger();
+  VERIFY_TRACE(rank, 1);
   const bool want_g = a.next_drafts && a.block_guesses && a.k > 0;
   // CTA 0 fetches the drafts and every block's guesses now, so those loads
   // overlap the logits sweep instead of following the accept decision
@@ -199,71 +233,119 @@ __global__ void __launch_bounds__(kGThreads) greedy_cluster_kernel(VerifyArgs a,
     if (want_g && t < a.k * a.k) s_g[t] = a.block_guesses[(size_t)b * a.k * a.k + t];
   }
   const int L = (((a.V + S - 1) / S) + 7) & ~7;
+  float item_v[2];
+  int item_i[2], item_n = 0;
   for (int it = rank; it < a.n * S; it += C) {
     const int row = it / S, sl = it % S;
     const int lo = sl * L, hi = min(a.V, lo + L);
     const T* p = static_cast<const T*>(a.logits) + ((size_t)b * a.n + row) * a.V;
-    float bv = -INFINITY;
-    int bi = INT_MAX;
+    // four independent (max, argmax) chains per thread, merged at the end
+    float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    int bi[4] = {INT_MAX, INT_MAX, INT_MAX, INT_MAX};
     if (vec_ok) {
       constexpr int kVec = 16 / sizeof(T);
       constexpr int kStride = kGThreads * kVec;
       for (int base = lo + (int)threadIdx.x * kVec; base < hi; base += kStride * kGUnroll) {
-        float v[kGUnroll][kVec];
+        // all the 16-byte loads first (kept raw, so they are in flight together),
+        // the conversions and compares after
+        uint4 raw[kGUnroll];
 #pragma unroll
         for (int u = 0; u < kGUnroll; ++u) {
           const int e0 = base + u * kStride;
-          if (e0 + kVec <= hi) {
-            load_vec<T, kVec>(p + e0, v[u]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < kVec; ++e) v[u][e] = e0 + e < hi ? ld(p, e0 + e) : -INFINITY;
-          }
+          raw[u] = e0 + kVec <= hi ? __ldg(reinterpret_cast<const uint4*>(p + e0)) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int u = 0; u < kGUnroll; ++u)
+        for (int u = 0; u < kGUnroll; ++u) {
+          const int e0 = base + u * kStride;
+          float v[kVec];
+          if (e0 + kVec <= hi) {
+            load_vec<T, kVec>(reinterpret_cast<const T*>(&raw[u]), v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) v[e] = e0 + e < hi ? ld(p, e0 + e) : -INFINITY;
+          }
 #pragma unroll
           for (int e = 0; e < kVec; ++e) {
-            const int id = base + u * kStride + e;
-            if (id < hi && (v[u][e] > bv || bi == INT_MAX)) { bv = v[u][e]; bi = id; }
+            const int id = e0 + e, q = u & 3;
+            if (id < hi && (v[e] > bv[q] || bi[q] == INT_MAX)) { bv[q] = v[e]; bi[q] = id; }
           }
+        }
       }
     } else {
       for (int id = lo + (int)threadIdx.x; id < hi; id += kGThreads) {
         const float x = ld(p, id);
-        if (x > bv || bi == INT_MAX) { bv = x; bi = id; }
+        if (x > bv[0] || bi[0] == INT_MAX) { bv[0] = x; bi[0] = id; }
       }
     }
+    amax_merge(bv[0], bi[0], bv[1], bi[1]);
+    amax_merge(bv[2], bi[2], bv[3], bi[3]);
+    amax_merge(bv[0], bi[0], bv[2], bi[2]);
+    float fv = bv[0];
+    int fi = bi[0];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
-      amax_merge(bv, bi, v2, i2);
+      const float v2 = __shfl_xor_sync(0xffffffffu, fv, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, fi, o);
+      amax_merge(fv, fi, v2, i2);
     }
-    if (lane == 0) { w_v[wid] = bv; w_i[wid] = bi; }
+    if (lane == 0) { w_v[wid] = fv; w_i[wid] = fi; }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      for (int w = 1; w < kGThreads / 32; ++w) amax_merge(bv, bi, w_v[w], w_i[w]);
-      s_v[it % kMaxCluster] = bv;
-      s_i[it % kMaxCluster] = bi;
+    if (wid == 0) {
+      fv = lane < kGThreads / 32 ? w_v[lane] : -INFINITY;
+      fi = lane < kGThreads / 32 ? w_i[lane] : INT_MAX;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, fv, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, fi, o);
+        amax_merge(fv, fi, v2, i2);
+      }
+      if (lane == 0 && item_n < 2) { item_v[item_n] = fv; item_i[item_n] = fi; }
     }
-    __syncthreads();
+    ++item_n;
+    __syncthreads();                              // w_v / w_i are reused by the next item
   }
-  cl.sync();
-  if (rank == 0 && wid == 0) {
-    int am = INT_MAX;
+  VERIFY_TRACE(rank, 2);
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+  VERIFY_TRACE(rank, 3);
+  if (threadIdx.x == 0) {
+    // push this CTA's items (at most two) into CTA 0, then arrive on its barrier
+    int n_it = 0;
+    for (int it = rank; it < a.n * S; it += C, ++n_it) {
+      const uint32_t rv = mapa(static_cast<uint32_t>(__cvta_generic_to_shared(&s_v[it])), 0);
+      const uint32_t ri = mapa(static_cast<uint32_t>(__cvta_generic_to_shared(&s_i[it])), 0);
+      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(rv), "f"(item_v[n_it]) : "memory");
+      asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(ri), "r"(item_i[n_it]) : "memory");
+    }
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(done_bar, 0))
+                 : "memory");
+  }
+  if (rank != 0) return;                          // nothing of this CTA is read after its push
+  if (wid == 0) {
+    // every CTA's items are in (bounded wait: on expiry, record it and skip)
+    bool ok = false;
+    if (lane == 0) {
+      const uint64_t t0 = global_ns();
+      for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(done_bar)
+            : "memory");
+        if (done) { ok = true; break; }
+        if (global_ns() - t0 > kWaitLimitNs) break;
+      }
+      if (!ok) raise_error(a.err, TIDAR_DEVERR_TIMEOUT);
+    }
+    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
+    __syncwarp();
     if (lane < a.n) {
       float bv = -INFINITY;
       int bi = INT_MAX;
-      for (int sl = 0; sl < S; ++sl) {
-        const int it = lane * S + sl;
-        const int owner = it % C;
-        const float* rv = cl.map_shared_rank(s_v, owner);
-        const int* ri = cl.map_shared_rank(s_i, owner);
-        amax_merge(bv, bi, rv[it % kMaxCluster], ri[it % kMaxCluster]);
-      }
-      am = bi;
-      s_am[lane] = am;
+      for (int sl = 0; sl < S; ++sl) amax_merge(bv, bi, s_v[lane * S + sl], s_i[lane * S + sl]);
+      s_am[lane] = bi;
     }
     __syncwarp();
     // d_{i+1} is kept while it equals argmax l_i: j = first mismatching i, else n
@@ -284,7 +366,7 @@ __global__ void __launch_bounds__(kGThreads) greedy_cluster_kernel(VerifyArgs a,
       if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
     }
   }
-  cl.sync();
+  VERIFY_TRACE(rank, 4);
 }
 
 // Row normaliser from chunk stats: M = max of chunk maxima, Z = sum_c
@@ -507,6 +589,12 @@ cudaError_t launch_t(const VerifyArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+#ifdef TIDAR_TRACE
+extern "C" int tidar_verify_trace_read(void* dst, size_t bytes) {
+  return (int)cudaMemcpyFromSymbol(dst, g_verify_trace, bytes);
+}
+#endif
+
 size_t verify_workspace_bytes(int B, int k, int V, int mode) {
   if (mode != TIDAR_REJECTION) return 0;   // greedy: the cluster kernel keeps everything on chip
   const size_t nchunk = (V + kChunk - 1) / kChunk;
@@ -592,6 +680,8 @@ extern "C" tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t v
   a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;
   a.next_drafts = next_drafts; a.selected_block = selected_block;
   a.workspace = tidar::g_verify_scratch_ptr[dev];
+  a.err = tidar::device_error_word();
+  if (!a.err) return TIDAR_ERR_CUDA;
   if (tidar::launch_verify(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TIDAR_ERR_CUDA;
   return TIDAR_OK;
 }

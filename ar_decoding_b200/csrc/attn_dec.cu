@@ -48,9 +48,17 @@ constexpr uint32_t kOffBarD = kOffStage + kDecStages * kStageBytes;
 constexpr int DBAR_Q = 0;
 constexpr int DBAR_FULL = 1;                            // + stage
 constexpr int DBAR_EMPTY = 1 + kDecStages;              // + stage (count: the page group's 4 warps)
-constexpr int kDecBars = 1 + 2 * kDecStages;
+constexpr int DBAR_MERGE = 1 + 2 * kDecStages;          // split merge: one arrival per CTA of the cluster
+constexpr int kDecBars = 2 + 2 * kDecStages;
 constexpr uint32_t kOffMiscD = kOffBarD + kDecBars * 8;  // [0] abort flag, [1 + s] stage s holds no page
-constexpr uint32_t kDecSmem = kOffMiscD + 4 * (1 + kDecStages);
+// Split-merge receive area of a row-owning CTA, apart from every buffer that
+// is still in use while other CTAs push into it: normalised partial O rows
+// [nsplit][ceil(M / nsplit) slots][128] fp32 (at most 30 rows for M, nsplit
+// <= 16) and their lse.  Row R is merged by CTA R % nsplit in slot R / nsplit.
+constexpr int kRecvRows = 30;
+constexpr uint32_t kOffRecv = (kOffMiscD + 4 * (1 + kDecStages) + 15u) & ~15u;
+constexpr uint32_t kOffRecvL = kOffRecv + kRecvRows * 128 * 4;
+constexpr uint32_t kDecSmem = kOffRecvL + kRecvRows * 4;
 static_assert(kDecSmem <= 232448, "shared memory budget");
 
 // Optional timeline (build with -DTIDAR_TRACE; absent from normal builds):
@@ -59,7 +67,7 @@ static_assert(kDecSmem <= 232448, "shared memory budget");
 // done by warp 1, [150] merge start, [151] end; [256 + 2*cta] start / end of
 // every CTA.
 #ifdef TIDAR_TRACE
-__device__ unsigned long long g_dec_trace[256 + 2 * 4096];
+__device__ unsigned long long g_dec_trace[256 + 2 * 4096 + 4096];   // + per-CTA pages-done time
 #define DEC_TRACE(slot) do { if (blockIdx.x == 0 && blockIdx.y == 0) g_dec_trace[(slot)] = global_ns(); } while (0)
 #define DEC_TRACE_CTA(w) do { const unsigned c_ = blockIdx.x + gridDim.x * blockIdx.y; \
     if (c_ < 4096) g_dec_trace[256 + 2 * c_ + (w)] = global_ns(); } while (0)
@@ -75,10 +83,6 @@ struct DecParams {
   int cluster;        // the nsplit CTAs of one (b, g) form a cluster and merge on chip
 };
 
-// CTA result area for the cluster merge (past the warp-merge scratch):
-// normalised O [16 rows][128] fp32 and lse [16].
-constexpr uint32_t kOffCpo = kOffStage + 96 * 1024;
-constexpr uint32_t kOffCpl = kOffCpo + 16 * 128 * 4;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -143,12 +147,16 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   for (int i = threadIdx.x; i < 4096 / 16; i += kDecThreads)
     reinterpret_cast<uint4*>(smem + kOffQd)[i] = make_uint4(0, 0, 0, 0);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kDecBars; ++i) mbar_init(bar(i), i >= DBAR_EMPTY ? 4u : 1u);
+    for (int i = 0; i < kDecBars; ++i)
+      mbar_init(bar(i), i == DBAR_MERGE ? (uint32_t)a.nsplit : (i >= DBAR_EMPTY ? 4u : 1u));
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
+  // Split cluster: every CTA is running and has initialised its merge barrier
+  // before anyone pushes to it (the matching wait comes after the key sweep).
+  if (prm.cluster) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   if (threadIdx.x == 0) { DEC_TRACE_CTA(0); DEC_TRACE(0); }
 
   pdl_wait();       // the previous kernel on the stream is complete from here on
@@ -407,6 +415,12 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (cw == 0 && lane == 0 && i < 64) DEC_TRACE(80 + i);
     }
     if (wid == 0 && lane == 0) DEC_TRACE(150);
+#ifdef TIDAR_TRACE
+    if (wid == 0 && lane == 0) {
+      const unsigned c_ = blockIdx.x + gridDim.x * blockIdx.y;
+      if (c_ < 4096) g_dec_trace[256 + 2 * 4096 + c_] = global_ns();
+    }
+#endif
     // ---- merge the compute warps: (max, sum, O) per row through shared memory
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -450,9 +464,20 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool all_ok = true;
 #pragma unroll
     for (int w = 0; w < kDecCompute; ++w) all_ok = all_ok && xk[w];
-    float* cpo = reinterpret_cast<float*>(smem + kOffCpo);
-    float* cpl = reinterpret_cast<float*>(smem + kOffCpl);
-    if (prm.cluster && row < 16 && c0 == 0) cpl[row] = -INFINITY;   // overwritten below when valid
+    if (prm.cluster) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    const int nsp = a.nsplit;
+    const uint32_t rank = prm.cluster ? cluster_rank() : 0u;
+    const int slots = (prm.M + nsp - 1) / nsp;        // rows owned per CTA
+    auto recv_addr = [&](int r) -> uint32_t {          // row r's slot for this split in its owner CTA
+      return mapa(sb + kOffRecv + 4u * (((uint32_t)rank * slots + (uint32_t)(r / nsp)) * 128u), (uint32_t)(r % nsp));
+    };
+    auto recvl_addr = [&](int r) -> uint32_t {
+      return mapa(sb + kOffRecvL + 4u * ((uint32_t)rank * slots + (uint32_t)(r / nsp)), (uint32_t)(r % nsp));
+    };
+    if (prm.cluster && row < prm.M && c0 == 0 && !all_ok) {
+      const float ninf = -INFINITY;                   // this split contributes nothing
+      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(recvl_addr(row)), "f"(ninf) : "memory");
+    }
     if (row < prm.M && all_ok) {
       float mtop = -INFINITY;
 #pragma unroll
@@ -481,9 +506,15 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int rho = row / a.G, h = g * a.G + row % a.G;
       const size_t orow = (size_t)(b * a.R + rho) * a.Hq + h;
       if (prm.cluster) {
-        *reinterpret_cast<float4*>(cpo + row * 128 + c0) = make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4*>(cpo + row * 128 + c0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
-        if (c0 == 0) cpl[row] = lse;
+        // push this split's normalised row slice and lse to the row's owner
+        const uint32_t dst = recv_addr(row) + 4u * c0;
+        asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(v[0]), "f"(v[1]),
+                     "f"(v[2]), "f"(v[3])
+                     : "memory");
+        asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16u), "f"(v[4]), "f"(v[5]),
+                     "f"(v[6]), "f"(v[7])
+                     : "memory");
+        if (c0 == 0) asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(recvl_addr(row)), "f"(lse) : "memory");
       } else if (a.nsplit == 1) {
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + orow * 128 + c0;
         uint4 u;
@@ -503,45 +534,82 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (prm.cluster) {
     // ---------------------------------------------------------------- split merge
-    // The CTAs of this cluster are the key splits of one (b, g).  CTA `rank`
-    // merges rows rank, rank + nsplit, ... of the M packed rows from every
-    // split's result over distributed shared memory; one warp per row, one
-    // lane per four columns.
-    cluster_sync_all();
+    // Every CTA of the cluster (the key splits of one (b, g)) has pushed its
+    // rows into their owners; once all of a CTA's pushes are issued, one thread
+    // arrives (release, cluster scope) on each owner's merge barrier.  Owners
+    // (CTAs 0 .. min(nsplit, M) - 1) wait for all nsplit arrivals, merge their
+    // rows from local shared memory and write O and lse; the other CTAs are
+    // done: nothing reads their shared memory.
     const int ns = a.nsplit;
     const uint32_t rank = cluster_rank();
-    const uint32_t cpo_s = sb + kOffCpo, cpl_s = sb + kOffCpl;
-    const int R = (int)rank + ns * warp;
-    if (R < prm.M) {
-      float l2 = -INFINITY;
-      if (lane < ns) l2 = ld_cluster_f32(mapa(cpl_s + 4u * R, (uint32_t)lane)) * 1.4426950408889634f;
-      float mx = l2;
+    if (threadIdx.x == 32) DEC_TRACE(152);
+    __syncthreads();                                   // all of this CTA's pushes are issued
+    if (threadIdx.x == 0) {
+      asm volatile("fence.acq_rel.cluster;" ::: "memory");
+      for (int o = 0; o < min(ns, prm.M); ++o)
+        asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(bar(DBAR_MERGE), o))
+                     : "memory");
+    }
+    if ((int)rank < min(ns, prm.M)) {
+      const int slots = (prm.M + ns - 1) / ns;
+      const int slot = warp;                           // one warp per owned row, one lane per 4 columns
+      const int R = (int)rank + ns * slot;
+      if (slot < slots && R < prm.M) {
+        bool ok = false;
+        {
+          const uint64_t t0 = global_ns();
+          for (;;) {
+            uint32_t done;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(done)
+                : "r"(bar(DBAR_MERGE))
+                : "memory");
+            if (done) { ok = true; break; }
+            if (global_ns() - t0 > kWaitLimitNs) break;
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          if (lane == 0) raise_error(a.err, TIDAR_DEVERR_TIMEOUT);
+        } else {
+          if (threadIdx.x == 32) DEC_TRACE(153);
+          const float* rv = reinterpret_cast<const float*>(smem + kOffRecv);
+          const float* rl = reinterpret_cast<const float*>(smem + kOffRecvL);
+          float l2 = -INFINITY;
+          if (lane < ns) l2 = rl[lane * slots + slot] * 1.4426950408889634f;
+          float mx = l2;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float w = (lane < ns && l2 != -INFINITY) ? ex2(l2 - mx) : 0.f;
-      float wsum = w;
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float w = (lane < ns && l2 != -INFINITY) ? ex2(l2 - mx) : 0.f;
+          float wsum = w;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s2 = 0; s2 < ns; ++s2) {
-        const float ws = __shfl_sync(0xffffffffu, w, s2);
-        if (ws != 0.f) {
-          const float4 x = ld_cluster_f32x4(mapa(cpo_s + 4u * (R * 128 + 4 * lane), (uint32_t)s2));
-          acc.x = fmaf(ws, x.x, acc.x); acc.y = fmaf(ws, x.y, acc.y);
-          acc.z = fmaf(ws, x.z, acc.z); acc.w = fmaf(ws, x.w, acc.w);
+          for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int s2 = 0; s2 < ns; ++s2) {
+            const float ws = __shfl_sync(0xffffffffu, w, s2);
+            // a split with weight 0 may have left its row unwritten: select, not multiply
+            const float4 x = *reinterpret_cast<const float4*>(rv + (s2 * slots + slot) * 128 + 4 * lane);
+            if (ws != 0.f) {
+              acc.x = fmaf(ws, x.x, acc.x); acc.y = fmaf(ws, x.y, acc.y);
+              acc.z = fmaf(ws, x.z, acc.z); acc.w = fmaf(ws, x.w, acc.w);
+            }
+          }
+          const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+          const int rho = R / a.G, h = g * a.G + R % a.G;
+          const size_t orow = (size_t)(b * a.R + rho) * a.Hq + h;
+          uint2 u;
+          u.x = pack_bf16(acc.x * inv, acc.y * inv);
+          u.y = pack_bf16(acc.z * inv, acc.w * inv);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + orow * 128 + 4 * lane) = u;
+          if (lane == 0 && a.lse_out)
+            a.lse_out[orow] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
         }
       }
-      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-      const int rho = R / a.G, h = g * a.G + R % a.G;
-      const size_t orow = (size_t)(b * a.R + rho) * a.Hq + h;
-      uint2 u;
-      u.x = pack_bf16(acc.x * inv, acc.y * inv);
-      u.y = pack_bf16(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + orow * 128 + 4 * lane) = u;
-      if (lane == 0 && a.lse_out)
-        a.lse_out[orow] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
     }
-    cluster_sync_all();   // no CTA leaves while another may still read its shared memory
+    if (threadIdx.x == 32) DEC_TRACE(154);
   }
 
   if (split == 0 && len_ok && !a.part_o) {

@@ -816,14 +816,28 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       float wsum = w;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       const uint32_t off = 4u * (R * 32 + (lane ^ (R & 7))) * 4u;
-      for (int s2 = 0; s2 < ns; ++s2) {
-        const float ws = __shfl_sync(0xffffffffu, w, s2);
-        if (ws != 0.f) {
-          const float4 x = ld_cluster_f32x4(mapa(po_s + off, (uint32_t)s2));
-          acc.x = fmaf(ws, x.x, acc.x); acc.y = fmaf(ws, x.y, acc.y);
-          acc.z = fmaf(ws, x.z, acc.z); acc.w = fmaf(ws, x.w, acc.w);
+      // the splits' partial rows, four remote loads in flight at a time; a
+      // split with weight 0 (no visible key) may have left its row unwritten,
+      // so its value is selected away rather than multiplied
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < ns; s0 += 4) {
+        float4 x[4];
+        float w4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float wl = __shfl_sync(0xffffffffu, w, (s0 + u) & 31);
+          w4[u] = s0 + u < ns ? wl : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          x[u] = s0 + u < ns ? ld_cluster_f32x4(mapa(po_s + off, (uint32_t)(s0 + u))) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (w4[u] != 0.f) {
+            acc.x = fmaf(w4[u], x[u].x, acc.x); acc.y = fmaf(w4[u], x[u].y, acc.y);
+            acc.z = fmaf(w4[u], x[u].z, acc.z); acc.w = fmaf(w4[u], x[u].w, acc.w);
+          }
         }
       }
       const float inv = wsum > 0.f ? 1.f / wsum : 0.f;

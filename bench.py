@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--no-sweep", action="store_true", help="skip the k sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc05", "dec"])
+    ap.add_argument("--configs", action="store_true",
+                    help="also time the serving batch and long-context workloads (extra_configs)")
     return ap.parse_args()
 
 
@@ -509,6 +511,25 @@ def run_ours(args, rank, world, local):
             del s2
             torch.cuda.empty_cache()
 
+    extra = []
+    if args.configs:
+        from ar_decoding_b200 import synth
+        for c2 in (synth.serving(), synth.long_context(1, 32768, 16), synth.long_context(4, 65536, 16),
+                   synth.long_context(8, 131072, 0), synth.long_context(8, 131072, 16)):
+            s2 = Step(c2, copies_for(c2), path=args.path)
+            su, _ = time_steps(s2, max(5, args.steps // 4), 3, world)
+            a2 = reduce_max(time_attention_launches(s2, 2), world) * 1e-6
+            b2, f2 = algorithmic(c2)
+            extra.append({"workload": c2.name, "B": c2.B, "prefix_total": sum(c2.prefix),
+                          "prefix_range": [min(c2.prefix), max(c2.prefix)], "k": c2.k,
+                          "path": PATH_NAMES[s2.path_id], "splits": s2.splits,
+                          "step_us": reduce_max(statistics.mean(su), world), "attn_us": a2 * 1e6,
+                          "attn_hbm_gbs": b2 / a2 / 1e9, "attn_tflops": f2 / a2 / 1e12,
+                          "hbm_frac": (b2 / a2 / 1e9) / hbm_peak, "tc_frac": (f2 / a2 / 1e12) / tc_peak,
+                          "roofline_frac": max(b2 / (hbm_peak * 1e9), f2 / (tc_peak * 1e12)) / a2})
+            del s2
+            torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t, take, total = oracle_step_seconds(cfg, 1.0)
@@ -541,6 +562,7 @@ def run_ours(args, rank, world, local):
                          "algorithmic_bytes": bytes_, "algorithmic_flops": flops,
                          "roofline_frac_max_of_both": max(t_mem, t_tc) / attn_s},
             "k_sweep": sweep,
+            "extra_configs": extra,
             "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": st.launches_per_step * args.steps,

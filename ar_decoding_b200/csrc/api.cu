@@ -156,7 +156,11 @@ Plan make_plan(const tidar_step_desc* d, int path) {
       if (p.nsplit < 1) p.nsplit = 1;
       return;
     }
-    const int bps = (blocks128 + n - 1) / n;
+    // tensor-core path: the last split also runs the tile's step-key windows
+    // (up to ceil(R / 128) blocks of 128), so the split size counts them and
+    // the last split gets that many fewer prefix blocks
+    const int wins = (path == 2 && n > 1) ? (R + 127) / 128 : 0;
+    const int bps = (blocks128 + wins + n - 1) / n;
     p.keys_per_split = (bps > 0 ? bps : 1) * 128;
     p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
     if (p.nsplit < 1) p.nsplit = 1;

@@ -233,13 +233,6 @@ __device__ __forceinline__ void exp2_poly_pair(float v0, float v1, float& r0, fl
   r1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1));
 }
 
-// Two non-negative floats -> packed bf16x2 (low half = a), rounded to nearest
-// with ties away from zero, using integer ops only (keeps the conversion off
-// the transcendental pipe that ex2 saturates).
-__device__ __forceinline__ uint32_t pack_bf16x2_pos(float a, float b) {
-  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
-}
-
 // ------------------------------------------------------------------ block plan
 // Blocks 0..npb-1: 128 prefix keys from k0; then nw step-key windows.
 struct BlockPlan {

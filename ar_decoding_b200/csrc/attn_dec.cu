@@ -437,15 +437,20 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* xm = xo + kDecCompute * kRows * kXo;                        // [warps][kRows] max
     float* xl = xm + kDecCompute * kRows;                              // [warps][kRows] sum
     int* xk = reinterpret_cast<int*>(xl + kDecCompute * kRows);        // [warps] status
+    // only the M real rows are merged (rows past M are tile padding)
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int r0 = 8 * nt + 2 * cq, d0 = 16 * mt + gq;
-        xo[(wid * kRows + r0) * kXo + d0] = o[mt][nt][0];
-        xo[(wid * kRows + r0 + 1) * kXo + d0] = o[mt][nt][1];
-        xo[(wid * kRows + r0) * kXo + d0 + 8] = o[mt][nt][2];
-        xo[(wid * kRows + r0 + 1) * kXo + d0 + 8] = o[mt][nt][3];
+        if (r0 < prm.M) {
+          xo[(wid * kRows + r0) * kXo + d0] = o[mt][nt][0];
+          xo[(wid * kRows + r0) * kXo + d0 + 8] = o[mt][nt][2];
+        }
+        if (r0 + 1 < prm.M) {
+          xo[(wid * kRows + r0 + 1) * kXo + d0] = o[mt][nt][1];
+          xo[(wid * kRows + r0 + 1) * kXo + d0 + 8] = o[mt][nt][3];
+        }
       }
     if (gq == 0) {
 #pragma unroll

@@ -212,27 +212,6 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-// 2^v for a pair, on the FMA pipe: Cody-Waite split v = j + f with j = rint(v)
-// (magic-number rounding), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
-// coefficients are a relative-error minimax fit computed for this library
-// (max relative error 7.5e-5); 2^j added to the exponent field.  Inputs are
-// clamped at -126 (results there are below every bf16 P that matters).
-__device__ __forceinline__ void exp2_poly_pair(float v0, float v1, float& r0, float& r1) {
-  constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
-  const uint64_t vc = f2_make(fmaxf(v0, -126.0f), fmaxf(v1, -126.0f));
-  const uint64_t t = f2_add(vc, f2_make(kMagic, kMagic));
-  const uint64_t tf = f2_add(t, f2_make(-kMagic, -kMagic));
-  const uint64_t f = f2_fma(tf, f2_make(-1.0f, -1.0f), vc);
-  uint64_t p = f2_fma(f2_make(0.0551716685f, 0.0551716685f), f, f2_make(0.242611125f, 0.242611125f));
-  p = f2_fma(p, f, f2_make(0.693260968f, 0.693260968f));
-  p = f2_fma(p, f, f2_make(0.999928057f, 0.999928057f));
-  float p0, p1, t0, t1;
-  f2_split(p, p0, p1);
-  f2_split(t, t0, t1);
-  r0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(p0));   // + (j << 23)
-  r1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1));
-}
-
 // ------------------------------------------------------------------ block plan
 // Blocks 0..npb-1: 128 prefix keys from k0; then nw step-key windows.
 struct BlockPlan {
@@ -619,30 +598,22 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tmem_ld32(trow + scol + 32 * h2, x);
           tmem_wait_ld();
           uint32_t pk[16];
-          if (full) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              float v0, v1, p0, p1;
-              f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
-              if ((c & 7) < 3) {
-                exp2_poly_pair(v0, v1, p0, p1);
-              } else {
-                p0 = ex2(v0);
-                p1 = ex2(v1);
-              }
-              ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
-              pk[c] = cvt_bf16x2(p0, p1);
-            }
-          } else {
+          // The same loop for full and masked blocks (invisible keys hold -inf
+          // in S since pass 1, and 2^-inf = 0).  Compiled as two copies, the
+          // common full-block one is scheduled without register spills.
+          auto exps = [&]() {
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               float v0, v1;
-              f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
+              f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0,
+                       v1);
               const float p0 = ex2(v0), p1 = ex2(v1);
               ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
               pk[c] = cvt_bf16x2(p0, p1);
             }
-          }
+          };
+          if (full) exps();
+          else exps();
           tmem_st16(trow + scol + 16 * h2, pk);
         }
         float la, lb, lc, ld;

@@ -20,10 +20,15 @@
  *   - All pointers are DEVICE pointers unless stated otherwise, on the device
  *     that is current when the call is made.  The caller owns every buffer
  *     (cache, tables, inputs, outputs, workspace); the library allocates no
- *     device memory.  Its only state is a per-device error word (see
- *     tidar_get_device_status).
+ *     device memory.  Its device state is a per-device error word (see
+ *     tidar_get_device_status) and the fixed scratch of tidar_verify_noalloc;
+ *     on the host it caches per-device kernel attributes and cluster
+ *     occupancy, looked up on the first call made with each device current.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
- *     default stream) and returns after the launches are queued.
+ *     default stream) and returns after the launches are queued.  Kernels are
+ *     launched as programmatic dependents of the preceding kernel on the
+ *     stream: they may start early but wait for it to complete before they
+ *     touch global memory, so stream order is kept.
  *   - Argument errors the host can see are returned before anything is
  *     launched.  Errors that depend on device-resident values (page ids, prefix
  *     lengths, accept counts) set bits in the device error word; the affected
@@ -132,7 +137,13 @@ typedef struct {
  *   workspace: device scratch of at least tidar_step_attn_workspace_bytes(desc)
  *     bytes, 256-byte aligned (may be NULL when that size is 0); contents on
  *     entry are ignored.  Calls that share a workspace must be stream-ordered.
- * Device errors: BAD_PAGE (prefix or draft page unmapped), BAD_LEN.
+ * Device errors: BAD_PAGE (prefix or draft page unmapped), BAD_LEN; the TC05
+ * and DEC kernels also TIMEOUT (a bounded wait on a copy or on a cluster
+ * peer ran out) and LAYOUT.  Splits of a long prefix merge on chip (a
+ * thread-block cluster per query tile) when every cluster of the launch can
+ * be resident at once, else through workspace partials and a second launch.
+ * That second launch also writes the draft rows; without it the TC05 and DEC
+ * kernels write them (SIMT always takes the second launch).
  * ------------------------------------------------------------------------- */
 size_t tidar_step_attn_workspace_bytes(const tidar_step_desc* desc);
 tidar_status tidar_step_attn(const tidar_step_desc* desc, const tidar_kv_cache* cache,
@@ -140,8 +151,9 @@ tidar_status tidar_step_attn(const tidar_step_desc* desc, const tidar_kv_cache* 
                              float* lse_out, void* workspace, size_t workspace_bytes,
                              tidar_stream_t stream);
 
-/* The launch plan the library would use: kernel family (1 SIMT, 2 tensor
- * core) and number of KV splits.  Host only, no device access. */
+/* The launch plan the library would use: kernel family (1 SIMT, 2 TC05,
+ * 3 DEC) and number of KV splits.  Host only; with a GPU present the first
+ * call per device queries its SM count and cluster occupancy. */
 tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, int32_t* splits);
 
 /* ---------------------------------------------------------------------------
@@ -258,7 +270,7 @@ const char* tidar_last_cuda_error(void);
  *     the CTAs record TIDAR_DEVERR_TIMEOUT, release TMEM and exit, the
  *     outputs are unspecified, tidar_get_device_status returns
  *     TIDAR_ERR_TIMEOUT and the CUDA context stays usable (failure injection).
- *   TIDAR_DEBUG_FORCE_SPLIT_PARTIALS: the tensor-core path merges key splits
+ *   TIDAR_DEBUG_FORCE_SPLIT_PARTIALS: the TC05 and DEC paths merge key splits
  *     through workspace partials and a second launch even where it would
  *     merge them on chip (so tests reach both merges).  Changes the
  *     workspace size that tidar_step_attn_workspace_bytes reports.

@@ -24,6 +24,7 @@ _lib = None
 
 F32, BF16 = 0, 1
 GREEDY, REJECTION = 0, 1
+RESERVE_FLAG_PAGE, RESERVE_FLAG_LEN, RESERVE_FLAG_POOL = 1, 2, 4
 
 
 def build(force: bool = False) -> str:
@@ -54,6 +55,8 @@ def _load():
         lib.tidar_oracle_verify.restype = i
         lib.tidar_oracle_commit.argtypes = [i, i, i, i, i, i, P, P, P, i, i, P, P, P, P]
         lib.tidar_oracle_commit.restype = i
+        lib.tidar_oracle_reserve.argtypes = [i, i, i, i, P, i, i, P, P, P, i, P, i]
+        lib.tidar_oracle_reserve.restype = i
         _lib = lib
     return _lib
 
@@ -191,3 +194,25 @@ def commit(k_pages, v_pages, page_table, seq_lens, accept_count, k):
                                  _ptr(pt), pt.shape[1], num_pages, _ptr(sl), _ptr(acc), _ptr(rel),
                                  _ptr(nrel))
     return kp, vp, pt, sl, rel, int(nrel[0]), st
+
+
+def reserve(page_table, seq_lens, free_pages, free_count, k, page_size, num_pages, *,
+            max_prefix, returned=None):
+    """Page reservation from a free-page stack, on copies.
+
+    page_table [B][max_pages] int32, seq_lens [B] int32, free_pages [capacity]
+    int32 with free_count valid entries, returned: the ids to push first (or
+    None).  Returns (page_table, free_pages, free_count, flags), flags a
+    combination of RESERVE_FLAG_PAGE / _LEN / _POOL (0 = success).
+    """
+    lib = _load()
+    pt = np.array(page_table, dtype=np.int32, copy=True)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    fp = np.array(free_pages, dtype=np.int32, copy=True)
+    fc = np.array([free_count], dtype=np.int32)
+    ret = None if returned is None else np.ascontiguousarray(returned, dtype=np.int32)
+    nret = 0 if ret is None else int(ret.shape[0])
+    flags = lib.tidar_oracle_reserve(sl.shape[0], k, page_size, int(max_prefix), _ptr(pt),
+                                     pt.shape[1], num_pages, _ptr(sl), _ptr(fp), _ptr(fc),
+                                     fp.shape[0], _ptr(ret), nret)
+    return pt, fp, int(fc[0]), int(flags)

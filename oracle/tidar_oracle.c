@@ -448,3 +448,92 @@ int tidar_oracle_commit(int B, int Hkv, int D, int k, int page_size, int elem_by
   *num_released = count;
   return status;
 }
+
+/*
+ * Page reservation for a step's draft rows, from a stack of free pages.
+ *
+ * The pages evict the rejected entries and reuse the settled cache ([NDfr]
+ * paragraph on the three zones); the step's draft rows P_b .. P_b+n-1 need
+ * cache pages before they are written ([NDfr], same paragraph: candidates
+ * carried from the previous step sit after the settled tokens).  The pages say
+ * nothing about where those pages come from.  The plainest reading, taken
+ * here: the pages a commit released return to a pool, and the pool is a stack
+ * (the last page returned is the first reused).  Flags, not statuses, because
+ * several can arise in one call:
+ *   1. The `returned` ids (num_returned >= 0 of them; returned may be NULL
+ *      when that is 0) are pushed in order: free[count + t] = returned[t].
+ *      If num_returned < 0 or count + num_returned > capacity, nothing at all
+ *      changes and RESERVE_FLAG_POOL is returned.
+ *   2. For each b, with P = seq_lens[b]: if P < 0 or P > max_prefix or
+ *      ceil((P+n)/ps) > max_pages, RESERVE_FLAG_LEN and b is skipped.  Rows
+ *      P .. P+n-1 lie on entries floor(P/ps) .. ceil((P+n)/ps)-1.  An entry
+ *      below ceil(P/ps) also holds prefix rows and must be a page in
+ *      [0, num_pages); an entry at or above it is a page in [0, num_pages)
+ *      (kept) or -1 (needs a page).  Anything else: RESERVE_FLAG_PAGE and b is
+ *      skipped.
+ *   3. If the entries that need a page outnumber count, no entry changes and
+ *      RESERVE_FLAG_POOL is raised (the push of step 1 stands).
+ *   4. Otherwise the needing entries, in (b, i) order, pop the stack one by
+ *      one: the t-th takes free[count - 1 - t]; count drops by their number.
+ * Popped ids are not checked; the step attention reports an out-of-range one.
+ */
+#define RESERVE_FLAG_PAGE 1
+#define RESERVE_FLAG_LEN 2
+#define RESERVE_FLAG_POOL 4
+
+/* Classifies sequence b: returns -1 (and sets *flag) if it is skipped, else the
+ * number of its entries that need a page. */
+static int reserve_need(int b, int n, int page_size, int max_prefix, const int32_t* page_table,
+                        int max_pages, int num_pages, const int32_t* seq_lens, int* flag) {
+  const int64_t P = seq_lens[b];
+  int64_t i, lo, settled, hi;
+  int need = 0;
+  if (P < 0 || P > max_prefix || (P + n + page_size - 1) / page_size > max_pages) {
+    *flag |= RESERVE_FLAG_LEN;
+    return -1;
+  }
+  lo = P / page_size;
+  settled = (P + page_size - 1) / page_size;   /* entries below hold prefix rows */
+  hi = (P + n + page_size - 1) / page_size;
+  for (i = lo; i < hi; ++i) {
+    const int32_t e = page_table[(int64_t)b * max_pages + i];
+    if (e >= 0 && e < num_pages) continue;
+    if (e == -1 && i >= settled) { ++need; continue; }
+    *flag |= RESERVE_FLAG_PAGE;
+    return -1;
+  }
+  return need;
+}
+
+int tidar_oracle_reserve(int B, int k, int page_size, int max_prefix, int32_t* page_table,
+                         int max_pages, int num_pages, const int32_t* seq_lens,
+                         int32_t* free_pages, int32_t* free_count, int capacity,
+                         const int32_t* returned, int num_returned) {
+  const int n = k > 0 ? k : 1;
+  int flag = 0, b, t, total = 0, count = *free_count;
+  int64_t i;
+  if (num_returned < 0 || (int64_t)count + num_returned > capacity) return RESERVE_FLAG_POOL;
+  for (t = 0; t < num_returned; ++t) free_pages[count + t] = returned[t];
+  count += num_returned;
+  *free_count = count;
+  for (b = 0; b < B; ++b) {
+    const int need = reserve_need(b, n, page_size, max_prefix, page_table, max_pages, num_pages,
+                                  seq_lens, &flag);
+    if (need > 0) total += need;
+  }
+  if (total > count) return flag | RESERVE_FLAG_POOL;
+  t = 0;
+  for (b = 0; b < B; ++b) {
+    int unused = 0;
+    const int64_t P = seq_lens[b];
+    if (reserve_need(b, n, page_size, max_prefix, page_table, max_pages, num_pages, seq_lens,
+                     &unused) <= 0)
+      continue;
+    for (i = (P + page_size - 1) / page_size; i < (P + n + page_size - 1) / page_size; ++i) {
+      int32_t* e = &page_table[(int64_t)b * max_pages + i];
+      if (*e == -1) *e = free_pages[count - 1 - t++];
+    }
+  }
+  *free_count = count - total;
+  return flag;
+}

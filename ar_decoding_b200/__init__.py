@@ -8,10 +8,14 @@ libtidar.so is missing or a call fails, an exception is raised.
     out, lse = step_attn(q, k_blk, v_blk, cache, k, max_prefix_len=P)
     res = verify(logits, drafts, k, "greedy", block_guesses=g)
     released, n = commit(cache, res["accept_count"], k, max_prefix_len=P)
+    reserve(cache, pool, k, max_prefix_len=P, returned=released, num_returned=n)
 
 ``cache`` is a mapping with the device tensors ``k_pages``/``v_pages``
 [num_pages][Hkv][page][D], ``page_table`` [B][max_pages] int32 and
-``seq_lens`` [B] int32 (the layout ``synth.make_cache`` produces).
+``seq_lens`` [B] int32 (the layout ``synth.make_cache`` produces).  ``pool``
+maps ``free_pages`` [capacity] and ``free_count`` [1] (int32): the stack of free
+page ids that ``reserve`` pops the next step's draft pages from, after pushing
+the ids the commit released.
 """
 from __future__ import annotations
 
@@ -30,6 +34,7 @@ F32, BF16 = 0, 1
 GREEDY, REJECTION = 0, 1
 PATH_AUTO, PATH_SIMT, PATH_TC05, PATH_DEC = 0, 1, 2, 3
 DEVERR_BAD_PAGE, DEVERR_BAD_LEN, DEVERR_BAD_COUNT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 1, 2, 4, 8, 16
+DEVERR_POOL = 32
 _PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tc05": PATH_TC05, "dec": PATH_DEC}
 
 
@@ -45,6 +50,11 @@ class StepDesc(ctypes.Structure):
                 ("k", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("max_prefix_len", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("path", ctypes.c_int32)]
+
+
+class PagePool(ctypes.Structure):
+    _fields_ = [("free_pages", ctypes.c_void_p), ("free_count", ctypes.c_void_p),
+                ("capacity", ctypes.c_int32)]
 
 
 class KVCacheDesc(ctypes.Structure):
@@ -81,6 +91,8 @@ def lib():
         L.tidar_verify_noalloc.restype = ctypes.c_int
         L.tidar_commit.argtypes = [P, P, P, P, P, P]
         L.tidar_commit.restype = ctypes.c_int
+        L.tidar_reserve.argtypes = [P, P, P, P, P, P]
+        L.tidar_reserve.restype = ctypes.c_int
         L.tidar_get_device_status.argtypes = [P, P]
         L.tidar_get_device_status.restype = ctypes.c_int
         L.tidar_status_string.argtypes = [ctypes.c_int]
@@ -259,6 +271,33 @@ def commit(cache, accept_count, k, *, max_prefix_len, head_dim=None, num_q_heads
                             _ptr(released), _ptr(num_released), _stream_handle(stream))
     _check(st, "tidar_commit")
     return released, num_released
+
+
+def reserve(cache, pool, k, *, max_prefix_len, returned=None, num_returned=None, stream=None):
+    """Pages for the draft rows of the next step, popped from a device stack.
+
+    ``pool`` maps ``free_pages`` [capacity] int32 (ids [0, free_count) free)
+    and ``free_count`` [1] int32, both device tensors.  ``returned`` /
+    ``num_returned`` (e.g. what ``commit`` returned) are pushed first.
+    Updates ``cache["page_table"]`` and the pool in place."""
+    kp = cache["k_pages"]
+    B = cache["seq_lens"].shape[0]
+    Hkv, ps, D = kp.shape[1], kp.shape[2], kp.shape[3]
+    desc = StepDesc(batch=B, num_q_heads=Hkv, num_kv_heads=Hkv, head_dim=D, k=k, page_size=ps,
+                    max_prefix_len=int(max_prefix_len), dtype=_dtype_code(kp), softmax_scale=0.0,
+                    path=PATH_AUTO)
+    cdesc = make_cache_desc(cache)
+    fp, fc = pool["free_pages"], pool["free_count"]
+    _dev(fc, "free_count")
+    if fp.numel():
+        _dev(fp, "free_pages")
+    if fp.dtype != torch.int32 or fc.dtype != torch.int32:
+        raise ValueError("free_pages and free_count must be int32")
+    p = PagePool(free_pages=fp.data_ptr() if fp.numel() else None, free_count=fc.data_ptr(),
+                 capacity=int(fp.numel()))
+    st = lib().tidar_reserve(ctypes.byref(desc), ctypes.byref(cdesc), ctypes.byref(p),
+                             _ptr(returned), _ptr(num_returned), _stream_handle(stream))
+    _check(st, "tidar_reserve")
 
 
 DEBUG_STARVE_ATTENTION_LOADS, DEBUG_FORCE_SPLIT_PARTIALS = 1, 2

@@ -348,6 +348,30 @@ tidar_status tidar_commit(const tidar_step_desc* d, const tidar_kv_cache* c,
   return TIDAR_OK;
 }
 
+tidar_status tidar_reserve(const tidar_step_desc* d, const tidar_kv_cache* c,
+                           const tidar_page_pool* pool, const int32_t* returned_pages,
+                           const int32_t* num_returned, tidar_stream_t stream) {
+  tidar_status st = check_desc(d);
+  if (st != TIDAR_OK) return st;
+  if (d->batch == 0) return TIDAR_OK;
+  if ((st = check_cache(d, c)) != TIDAR_OK) return st;
+  if (!pool || !pool->free_count || pool->capacity < 0 || (pool->capacity > 0 && !pool->free_pages))
+    return TIDAR_ERR_INVALID_ARG;
+  if (!returned_pages != !num_returned) return TIDAR_ERR_INVALID_ARG;
+  if (!tidar::reserve_batch_ok(d->batch)) return TIDAR_ERR_UNSUPPORTED;
+  unsigned int* err = nullptr;
+  if ((st = error_word(&err)) != TIDAR_OK) return st;
+  tidar::ReserveArgs a;
+  a.B = d->batch; a.n = d->k > 0 ? d->k : 1; a.page_size = d->page_size;
+  a.max_prefix = d->max_prefix_len; a.max_pages = c->max_pages_per_seq; a.num_pages = c->num_pages;
+  a.capacity = pool->capacity; a.page_table = c->page_table; a.seq_lens = c->seq_lens;
+  a.free_pages = pool->free_pages; a.free_count = pool->free_count;
+  a.returned = returned_pages; a.num_returned = num_returned; a.err = err;
+  cudaError_t e = tidar::launch_reserve(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
 tidar_status tidar_debug_set(tidar_debug_knob knob, int32_t value) {
   switch (knob) {
     case TIDAR_DEBUG_STARVE_ATTENTION_LOADS: tidar::set_starve_loads(value != 0); return TIDAR_OK;

@@ -84,4 +84,19 @@ struct CommitArgs {
 bool commit_batch_ok(int B, int k, int page_size);   // per-sequence records fit shared memory
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t s);
 
+struct ReserveArgs {
+  int B, n, page_size, max_prefix, max_pages, num_pages, capacity;
+  int32_t* page_table;
+  const int32_t* seq_lens;
+  int32_t* free_pages;
+  int32_t* free_count;
+  const int32_t* returned;       // may be null (then num_returned is null too)
+  const int32_t* num_returned;
+  unsigned int* err;
+};
+// One CTA keeps a byte per sequence in shared memory.
+constexpr int kReserveMaxBatch = 65536;
+bool reserve_batch_ok(int B);
+cudaError_t launch_reserve(const ReserveArgs& a, cudaStream_t s);
+
 }  // namespace tidar

@@ -108,26 +108,30 @@ def _randn(shape, gen, dtype, device="cpu", std=1.0):
     return x.to(dtype)
 
 
-def make_cache(cfg: StepConfig, device="cpu", extra_pages: int = 0):
+def make_cache(cfg: StepConfig, device="cpu", extra_pages: int = 0, draft_pages: bool = True,
+               max_pages: int | None = None):
     """Paged KV cache holding each prefix, with pages reserved for the n draft rows.
 
     Returns dict(k_pages, v_pages [num_pages][Hkv][page][D], page_table
     [B][max_pages] int32 (-1 = none), seq_lens [B] int32).  Page ids are a
     seeded permutation when cfg.shuffle_pages.  Rows past P_b inside reserved
-    pages hold random values too (they are not part of the prefix).
+    pages hold random values too (they are not part of the prefix).  With
+    draft_pages=False only the pages holding prefix rows are mapped (the draft
+    pages stay unmapped and their ids unused); max_pages widens the table.
     """
     gen = torch.Generator(device=device).manual_seed(cfg.seed * 7 + 1)
     ps = cfg.page_size
     need = [-(-(p + cfg.n) // ps) for p in cfg.prefix]
     num_pages = sum(need) + extra_pages
-    max_pages = max(need) + 1
+    width = max(need) + 1 if max_pages is None else max(max_pages, max(need))
     cpu_gen = torch.Generator().manual_seed(cfg.seed * 7 + 2)
     ids = (torch.randperm(num_pages, generator=cpu_gen) if cfg.shuffle_pages
            else torch.arange(num_pages)).to(torch.int32)
-    table = torch.full((cfg.B, max_pages), -1, dtype=torch.int32)
+    table = torch.full((cfg.B, width), -1, dtype=torch.int32)
     pos = 0
     for b, cnt in enumerate(need):
-        table[b, :cnt] = ids[pos:pos + cnt]
+        mapped = cnt if draft_pages else -(-cfg.prefix[b] // ps)
+        table[b, :mapped] = ids[pos:pos + mapped]
         pos += cnt
     shape = (num_pages, cfg.Hkv, ps, cfg.D)
     k_pages = _randn(shape, gen, cfg.torch_dtype, device)
@@ -177,6 +181,91 @@ def make_verify(cfg: StepConfig, mode: str | None = None, seed_offset: int = 0):
     return dict(logits=logits, drafts=drafts.to(torch.int32),
                 draft_logits=draft_logits, uniforms=uniforms,
                 block_guesses=block_guesses.to(torch.int32), mode=mode)
+
+
+def make_pool(cfg: StepConfig, cache, capacity: int | None = None):
+    """Stack of free pages: the ids the cache's page table does not use, in a
+    seeded order.  Returns dict(free_pages [capacity] int32 (-1 past the
+    count), free_count [1] int32); capacity defaults to the number of pages."""
+    num_pages = cache["k_pages"].shape[0]
+    pt = cache["page_table"].cpu()
+    used = set(int(x) for x in pt[pt >= 0])
+    free = torch.tensor([p for p in range(num_pages) if p not in used], dtype=torch.int32)
+    perm = torch.randperm(free.numel(), generator=torch.Generator().manual_seed(cfg.seed * 7 + 6))
+    cap = num_pages if capacity is None else capacity
+    arr = torch.full((cap,), -1, dtype=torch.int32)
+    arr[:free.numel()] = free[perm]
+    return dict(free_pages=arr, free_count=torch.tensor([free.numel()], dtype=torch.int32))
+
+
+def random_pool_state(seed: int):
+    """A random page-reservation problem (numpy): returns dict(table [B][cols],
+    lens [B], free [capacity], count, returned (or None), k, ps, num_pages,
+    max_prefix).  Prefix pages are mapped, some draft pages already are, the
+    stack may be short, and with probability 0.3 one sequence is made invalid
+    (length past max_prefix, or its prefix page unmapped / out of range)."""
+    rng = np.random.default_rng(seed)
+    k = int(rng.choice([0, 1, 3, 8, 16]))
+    ps = int(rng.choice([16, 32, 64, 128]))
+    B = int(rng.integers(1, 12))
+    max_prefix = int(rng.integers(0, 400))
+    n = max(k, 1)
+    cols = -(-(max_prefix + n) // ps) + int(rng.integers(0, 3))
+    num_pages = B * cols + 8
+    lens = rng.integers(0, max_prefix + 1, B).astype(np.int32)
+    ids = rng.permutation(num_pages).astype(np.int32)
+    table = np.full((B, cols), -1, np.int32)
+    pos = 0
+    for b in range(B):
+        for i in range(-(-(int(lens[b]) + n) // ps)):
+            if i * ps < lens[b] or rng.random() < 0.3:       # prefix pages, some draft pages
+                table[b, i] = ids[pos]
+                pos += 1
+    cap = int(rng.integers(0, 3 * B + 4))
+    count = int(rng.integers(0, cap + 1))
+    free = np.full(cap, -1, np.int32)
+    free[:count] = rng.integers(0, num_pages, count)
+    returned = None
+    if rng.random() < 0.6:
+        returned = rng.integers(0, num_pages, int(rng.integers(0, 2 * B + 2))).astype(np.int32)
+    if rng.random() < 0.3:
+        b = int(rng.integers(B))
+        if rng.random() < 0.5:
+            lens[b] = max_prefix + 1 + int(rng.integers(3))
+        elif lens[b] % ps:
+            table[b, int(lens[b]) // ps] = -1
+        else:
+            table[b, int(lens[b]) // ps] = num_pages + 5
+    return dict(table=table, lens=lens, free=free, count=count, returned=returned, k=k, ps=ps,
+                num_pages=num_pages, max_prefix=max_prefix)
+
+
+def make_loop(cfg: StepConfig, steps: int):
+    """Inputs of `steps` chained greedy steps (CPU tensors).
+
+    Returns (attn, ver): attn[s] = make_step of a per-step seed; ver[s] =
+    make_verify(seed_offset=s+1), whose drafts matter only at s = 0 (later
+    steps inherit t*, g_{j,2..k} from the step before).  The block guesses of
+    step s are set so that the drafts step s+1 inherits equal the row argmaxes
+    (first maximal index) of step s+1's logits up to a seeded depth in 1..k, so
+    accept counts spread over 1..k whichever block is selected.
+    """
+    attn = [make_step(StepConfig(**{**cfg.__dict__, "seed": cfg.seed + 101 * (s + 1)}))
+            for s in range(steps)]
+    ver = [make_verify(cfg, "greedy", seed_offset=s + 1) for s in range(steps)]
+    gen = torch.Generator().manual_seed(cfg.seed * 7 + 7)
+    k = cfg.k
+    for s in range(steps - 1):
+        if k < 2:
+            break
+        top = torch.argmax(ver[s + 1]["logits"][:, : k - 1, :].float(), dim=-1)   # [B][k-1]
+        depth = torch.randint(1, k + 1, (cfg.B,), generator=gen)
+        g = ver[s]["block_guesses"].clone()
+        for b in range(cfg.B):
+            for m in range(1, int(depth[b])):
+                g[b, :, m] = top[b, m - 1]
+        ver[s]["block_guesses"] = g
+    return attn, ver
 
 
 def prev_accept_counts(cfg: StepConfig) -> torch.Tensor:

@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--no-sweep", action="store_true", help="skip the k sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc05", "dec"])
+    ap.add_argument("--no-loop", action="store_true", help="skip the chained decode-loop timing")
+    ap.add_argument("--loop-chain", type=int, default=8,
+                    help="steps chained per sequence in the decode-loop graph")
     ap.add_argument("--configs", action="store_true",
                     help="also time the serving batch and long-context workloads (extra_configs)")
     return ap.parse_args()
@@ -218,6 +221,131 @@ class Step:
                 self.restore(i)
             self.graphs.append((gs, ga, gr))
         torch.cuda.synchronize()
+
+
+class Loop:
+    """The decode loop on the device: `chain` steps of reserve -> step attention
+    -> verify -> commit per sequence, each step's drafts, lengths and pages
+    coming from the step before (no host round-trip), for `copies` independent
+    sequences interleaved step by step (each copy's KV is cold in L2 when its
+    turn comes).  One CUDA graph holds the whole loop; a second restores every
+    copy's lengths, page table and free-page stack."""
+
+    def __init__(self, cfg, copies, chain, path="auto"):
+        import ar_decoding_b200 as tidar
+        from ar_decoding_b200 import synth
+        self.tidar, self.cfg, self.chain, self.path = tidar, cfg, chain, path
+        dev = torch.device("cuda")
+        n = cfg.n
+        self.max_prefix = max(cfg.prefix) + chain * n
+        width = -(-(self.max_prefix + n) // cfg.page_size)
+        self.copies = []
+        for c in range(copies):
+            cc = synth.StepConfig(**{**cfg.__dict__, "seed": cfg.seed + 31 * c + 5})
+            cache = synth.make_cache(cc, device=dev, extra_pages=chain * n // cfg.page_size + 2,
+                                     draft_pages=False, max_pages=width)
+            pool = {k: v.to(dev) for k, v in synth.make_pool(cc, cache).items()}
+            attn, ver = synth.make_loop(cc, chain)
+            self.copies.append(dict(
+                cache=cache, pool=pool,
+                attn=[{k: v.to(dev) for k, v in a.items()} for a in attn],
+                logits=[v["logits"].to(dev) for v in ver],
+                guesses=[v["block_guesses"].to(dev) for v in ver],
+                drafts0=ver[0]["drafts"].to(dev),
+                saved={k: t.clone() for k, t in (("seq_lens", cache["seq_lens"]),
+                                                  ("page_table", cache["page_table"]))},
+                saved_pool={k: t.clone() for k, t in pool.items()},
+                drafts=[torch.empty((cfg.B, max(cfg.k, 1)), dtype=torch.int32, device=dev)
+                        for _ in range(2)],
+                rel=[torch.empty(cfg.B * (-(-n // cfg.page_size) + 1), dtype=torch.int32,
+                                 device=dev) for _ in range(2)],
+                nrel=[torch.empty(1, dtype=torch.int32, device=dev) for _ in range(2)]))
+        c0 = self.copies[0]
+        q0 = c0["attn"][0]["q"]
+        self.desc = tidar.make_desc(q0, c0["attn"][0]["k_blk"], c0["cache"], cfg.k,
+                                    self.max_prefix, path=path)
+        self.path_id, self.splits = tidar.plan(self.desc)
+        need = tidar.step_attn_workspace_bytes(self.desc)
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        self.out = torch.empty_like(q0)
+        self.lse = torch.empty(q0.shape[:3], dtype=torch.float32, device=dev)
+        V = c0["logits"][0].shape[2]
+        self.vws = torch.empty(max(tidar.verify_workspace_bytes(cfg.B, cfg.k, V, 0), 256),
+                               dtype=torch.uint8, device=dev)
+        self.vout = dict(accept_count=torch.empty(cfg.B, dtype=torch.int32, device=dev),
+                         out_tokens=torch.empty((cfg.B, n), dtype=torch.int32, device=dev),
+                         selected_block=torch.empty(cfg.B, dtype=torch.int32, device=dev))
+        self.launches_per_step = 1 + (1 if (need == 0 and self.path_id in (2, 3)) else 2) + 2
+
+    def step(self, c, s):
+        """Step s of copy c: pages, attention (with the draft-row append),
+        verification (next drafts into a ping-pong buffer), commit."""
+        t, k = self.tidar, self.cfg.k
+        cp = self.copies[c]
+        prev = (s + 1) % 2
+        t.reserve(cp["cache"], cp["pool"], k, max_prefix_len=self.max_prefix,
+                  returned=cp["rel"][prev] if s else None, num_returned=cp["nrel"][prev] if s else None)
+        a = cp["attn"][s]
+        t.step_attn(a["q"], a["k_blk"], a["v_blk"], cp["cache"], k, max_prefix_len=self.max_prefix,
+                    path=self.path, out=self.out, lse=self.lse, workspace=self.ws)
+        drafts = cp["drafts0"] if s == 0 else cp["drafts"][prev]
+        vout = dict(self.vout, next_drafts=cp["drafts"][s % 2])
+        t.verify(cp["logits"][s], drafts if k else None, k, "greedy",
+                 block_guesses=cp["guesses"][s] if k else None, outputs=vout, workspace=self.vws)
+        t.commit(cp["cache"], self.vout["accept_count"], k, max_prefix_len=self.max_prefix,
+                 released=cp["rel"][s % 2], num_released=cp["nrel"][s % 2])
+
+    def run(self):
+        for s in range(self.chain):
+            for c in range(len(self.copies)):
+                self.step(c, s)
+
+    def restore(self):
+        for cp in self.copies:
+            for k, v in cp["saved"].items():
+                cp["cache"][k].copy_(v, non_blocking=True)
+            for k, v in cp["saved_pool"].items():
+                cp["pool"][k].copy_(v, non_blocking=True)
+
+    def grown(self) -> int:
+        """Tokens the loop committed (sum of accept counts) since the last restore."""
+        return int(sum(int((cp["cache"]["seq_lens"] - cp["saved"]["seq_lens"]).sum())
+                       for cp in self.copies))
+
+    def time(self, reps: int):
+        """Returns (µs per step, committed tokens per loop) over `reps` replays."""
+        self.run(); self.restore()                 # first calls outside capture
+        torch.cuda.synchronize()
+        status, bits = self.tidar.device_status()
+        if status != self.tidar.OK:
+            raise RuntimeError(f"decode loop: device status {status} bits {bits:#x}")
+        gl, gr = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gl):
+            self.run()
+        with torch.cuda.graph(gr):
+            self.restore()
+        stream = torch.cuda.current_stream()
+        gl.replay(); gr.replay()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        tokens = None
+        for i in range(reps):
+            ev[i][0].record(stream)
+            gl.replay()
+            ev[i][1].record(stream)
+            if i == reps - 1:
+                torch.cuda.synchronize()
+                tokens = self.grown()
+            gr.replay()
+        torch.cuda.synchronize()
+        status, bits = self.tidar.device_status()
+        if status != self.tidar.OK:
+            raise RuntimeError(f"decode loop: device status {status} bits {bits:#x}")
+        steps = self.chain * len(self.copies)
+        us = statistics.mean(a.elapsed_time(b) * 1e3 for a, b in ev) / steps
+        del gl, gr
+        return us, tokens
 
 
 KERNEL_SRC = {2: "attn_tc05.cu", 3: "attn_dec.cu"}
@@ -530,6 +658,23 @@ def run_ours(args, rank, world, local):
             del s2
             torch.cuda.empty_cache()
 
+    loop = None
+    if not args.no_loop:
+        lp = Loop(cfg, copies_for(cfg), args.loop_chain, path=args.path)
+        lus, ltok = lp.time(max(3, args.steps // 6))
+        lus = reduce_max(lus, world)
+        nsteps = lp.chain * len(lp.copies)
+        loop = {"workload": f"{cfg.name} decode loop", "chained_steps": lp.chain,
+                "interleaved_sequences": len(lp.copies), "us_per_step": lus,
+                "launches_per_step": lp.launches_per_step,
+                "committed_tokens_per_step": ltok / nsteps,
+                "tokens_per_s_per_sequence": ltok / nsteps / (lus * 1e-6),
+                "acceptance": "planted: drafts match the next step's argmax up to a depth "
+                              "uniform on 1..k (synthetic, not a model's acceptance)",
+                "path": PATH_NAMES[lp.path_id], "splits": lp.splits}
+        del lp
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t, take, total = oracle_step_seconds(cfg, 1.0)
@@ -563,6 +708,7 @@ def run_ours(args, rank, world, local):
                          "roofline_frac_max_of_both": max(t_mem, t_tc) / attn_s},
             "k_sweep": sweep,
             "extra_configs": extra,
+            "decode_loop": loop,
             "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": st.launches_per_step * args.steps,

@@ -86,6 +86,7 @@ typedef enum {
 #define TIDAR_DEVERR_BAD_COUNT 0x4u     /* accept_count[b] outside 0..n (commit) */
 #define TIDAR_DEVERR_TIMEOUT 0x8u       /* a bounded mbarrier wait ran out */
 #define TIDAR_DEVERR_LAYOUT 0x10u       /* a kernel's shared-memory layout check failed (no work done) */
+#define TIDAR_DEVERR_POOL 0x20u         /* tidar_reserve: too few free pages, or no room for the returned ids */
 
 typedef struct {
   int32_t batch;          /* B >= 0 (0: every call is a no-op) */
@@ -251,6 +252,54 @@ tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t vocab, tidar
 tidar_status tidar_commit(const tidar_step_desc* desc, const tidar_kv_cache* cache,
                           const int32_t* accept_count, int32_t* released_pages,
                           int32_t* num_released, tidar_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Page reservation for the next step's draft rows, from a device stack of
+ * free pages (the step the commit's release implies; the pages do not
+ * describe a page pool).  [NDfr] paragraph on the three zones: the candidates
+ * carried from the previous step follow the settled tokens, the settled cache
+ * is reused and rejected entries are evicted.  With the ids that tidar_commit
+ * released passed back in, reserve -> tidar_step_attn -> tidar_verify ->
+ * tidar_commit repeats on the device with no host round-trip, so many steps
+ * can be one CUDA graph.
+ *
+ * The pool is a stack: free_pages[0 .. *free_count) are free page ids, the
+ * last one on top.  In one launch:
+ *   1. the returned ids (*num_returned of them) are pushed in order on top;
+ *      if *num_returned < 0 or they do not fit in `capacity` (or *free_count
+ *      is outside 0..capacity), NOTHING changes and TIDAR_DEVERR_POOL is set;
+ *   2. for each b, with P = seq_lens[b] and n = max(k,1), the draft rows
+ *      P .. P+n-1 lie on page-table entries floor(P/ps) .. ceil((P+n)/ps)-1.
+ *      An entry below ceil(P/ps) also holds prefix rows and must be a valid
+ *      page; an entry at or above it is kept if valid and needs a page if -1.
+ *      P < 0 or P > max_prefix_len sets BAD_LEN, any other entry BAD_PAGE; that
+ *      sequence is skipped;
+ *   3. if the stack holds fewer ids than the entries that need one, no entry
+ *      changes, TIDAR_DEVERR_POOL is set and *free_count is the count after the
+ *      push;
+ *   4. otherwise the needing entries, in (b, i) order, pop the stack: the t-th
+ *      takes free_pages[count-1-t]; *free_count drops by their number.
+ *      Entries at or above the new count keep the ids they held.
+ * Popped ids are not range-checked here (tidar_step_attn reports BAD_PAGE).
+ * With page_size >= 16 and k <= 16 a sequence needs at most one page a step.
+ *
+ *   pool->free_pages [capacity] int32, pool->free_count [1] int32 (device)
+ *   returned_pages [*num_returned] int32 and num_returned [1] int32 (device),
+ *     e.g. tidar_commit's released_pages / num_released; both NULL to push
+ *     nothing, else both non-NULL (TIDAR_ERR_INVALID_ARG).
+ * Only page_table (and the pool) are written; dtype, head counts, head_dim and
+ * path of `desc` are not used beyond validation.  TIDAR_ERR_UNSUPPORTED when
+ * batch > 65536 (one CTA with a byte of shared memory per sequence).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int32_t* free_pages; /* [capacity] page ids; [0, *free_count) are free */
+  int32_t* free_count; /* [1] */
+  int32_t capacity;    /* >= 0 */
+} tidar_page_pool;
+
+tidar_status tidar_reserve(const tidar_step_desc* desc, const tidar_kv_cache* cache,
+                           const tidar_page_pool* pool, const int32_t* returned_pages,
+                           const int32_t* num_returned, tidar_stream_t stream);
 
 /* Synchronises `stream`, reads and clears this device's error word.  Returns
  * TIDAR_ERR_TIMEOUT if the timeout bit was set, TIDAR_ERR_DEVICE for any other

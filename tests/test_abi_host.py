@@ -21,7 +21,8 @@ def L():
 
 def test_exports_every_declared_symbol(L):
     names = tidar.header_functions()
-    assert {"tidar_step_attn", "tidar_verify", "tidar_commit", "tidar_get_device_status"} <= set(names)
+    assert {"tidar_step_attn", "tidar_verify", "tidar_commit", "tidar_reserve",
+            "tidar_get_device_status"} <= set(names)
     for n in names:
         assert hasattr(L, n), n
 
@@ -124,6 +125,25 @@ def test_commit_rejects_bad_args(L):
     assert L.tidar_commit(ctypes.byref(d), ctypes.byref(c), None, FAKE, FAKE, None) == tidar.ERR_INVALID_ARG
     assert L.tidar_commit(ctypes.byref(_desc(k=20)), ctypes.byref(c), FAKE, FAKE, FAKE, None) == tidar.ERR_UNSUPPORTED
     assert L.tidar_commit(ctypes.byref(d), None, FAKE, FAKE, FAKE, None) == tidar.ERR_INVALID_ARG
+
+
+def test_reserve_rejects_bad_args(L):
+    d, c = _desc(), _cache()
+    R = L.tidar_reserve
+    pool = lambda **kw: ctypes.byref(tidar.PagePool(**dict(dict(free_pages=FAKE, free_count=FAKE,
+                                                                 capacity=4), **kw)))
+    assert R(ctypes.byref(d), ctypes.byref(c), None, None, None, None) == tidar.ERR_INVALID_ARG
+    assert R(ctypes.byref(d), ctypes.byref(c), pool(free_count=None), None, None, None) == tidar.ERR_INVALID_ARG
+    assert R(ctypes.byref(d), ctypes.byref(c), pool(capacity=-1), None, None, None) == tidar.ERR_INVALID_ARG
+    assert R(ctypes.byref(d), ctypes.byref(c), pool(free_pages=None), None, None, None) == tidar.ERR_INVALID_ARG
+    assert R(ctypes.byref(d), ctypes.byref(c), pool(), FAKE, None, None) == tidar.ERR_INVALID_ARG
+    assert R(ctypes.byref(d), ctypes.byref(c), pool(), None, FAKE, None) == tidar.ERR_INVALID_ARG
+    assert R(ctypes.byref(_desc(k=20)), ctypes.byref(c), pool(), None, None, None) == tidar.ERR_UNSUPPORTED
+    assert R(ctypes.byref(_desc(batch=65537)), ctypes.byref(c), pool(), None, None, None) == tidar.ERR_UNSUPPORTED
+    assert R(ctypes.byref(d), None, pool(), None, None, None) == tidar.ERR_INVALID_ARG
+    assert R(ctypes.byref(_desc(max_prefix_len=1000)), ctypes.byref(c), pool(), None, None,
+             None) == tidar.ERR_INVALID_ARG                  # table too short for it
+    assert R(ctypes.byref(_desc(batch=0)), None, None, None, None, None) == tidar.OK
 
 
 def test_plan_covers_workloads(L):

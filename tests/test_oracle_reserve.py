@@ -13,6 +13,7 @@
 import numpy as np
 import pytest
 
+from ar_decoding_b200 import synth
 from conftest import read_golden
 
 
@@ -128,42 +129,10 @@ def _model(table, lens, free, count, k, ps, num_pages, max_prefix, returned, fla
 
 @pytest.mark.parametrize("seed", range(40))
 def test_reserve_matches_stack_model(oracle_mod, seed):
-    rng = np.random.default_rng(seed)
-    k = int(rng.choice([0, 1, 3, 8, 16]))
-    ps = int(rng.choice([4, 16, 64]))
-    B = int(rng.integers(1, 12))
-    max_prefix = int(rng.integers(0, 200))
-    n = max(k, 1)
-    cols = -(-(max_prefix + n) // ps) + int(rng.integers(0, 3))
-    num_pages = B * cols + 8
-    lens = rng.integers(0, max_prefix + 1, B).astype(np.int32)
-    ids = rng.permutation(num_pages).astype(np.int32)
-    table = np.full((B, cols), -1, np.int32)
-    pos = 0
-    for b in range(B):
-        hi = -(-(int(lens[b]) + n) // ps)
-        for i in range(hi):
-            if i * ps < lens[b] or rng.random() < 0.3:     # prefix pages, some draft pages
-                table[b, i] = ids[pos]
-                pos += 1
-    cap = int(rng.integers(0, 3 * B + 4))
-    count = int(rng.integers(0, cap + 1))
-    free = np.full(cap, -1, np.int32)
-    free[:count] = rng.integers(0, num_pages, count)
-    returned = None
-    if rng.random() < 0.6:
-        returned = rng.integers(0, num_pages, int(rng.integers(0, 2 * B + 2))).astype(np.int32)
-    if rng.random() < 0.3:                                    # failures
-        b = int(rng.integers(B))
-        if rng.random() < 0.5:
-            lens[b] = max_prefix + 1 + int(rng.integers(3))
-        elif lens[b] % ps:
-            table[b, int(lens[b]) // ps] = -1
-        else:
-            table[b, int(lens[b]) // ps] = num_pages + 5
-    got = oracle_mod.reserve(table, lens, free, count, k, ps, num_pages, max_prefix=max_prefix,
-                             returned=returned)
-    want = _model(table, lens, free, count, k, ps, num_pages, max_prefix, returned, oracle_mod)
+    st = synth.random_pool_state(seed)
+    args = (st["table"], st["lens"], st["free"], st["count"], st["k"], st["ps"], st["num_pages"])
+    got = oracle_mod.reserve(*args, max_prefix=st["max_prefix"], returned=st["returned"])
+    want = _model(*args, st["max_prefix"], st["returned"], oracle_mod)
     np.testing.assert_array_equal(got[0], want[0])
     np.testing.assert_array_equal(got[1], want[1])
     assert got[2] == want[2] and got[3] == want[3]

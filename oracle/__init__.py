@@ -25,6 +25,7 @@ _lib = None
 F32, BF16 = 0, 1
 GREEDY, REJECTION = 0, 1
 RESERVE_FLAG_PAGE, RESERVE_FLAG_LEN, RESERVE_FLAG_POOL = 1, 2, 4
+GATHER_FLAG_BLOCK = 1
 
 
 def build(force: bool = False) -> str:
@@ -57,6 +58,8 @@ def _load():
         lib.tidar_oracle_commit.restype = i
         lib.tidar_oracle_reserve.argtypes = [i, i, i, i, P, i, i, P, P, P, i, P, i]
         lib.tidar_oracle_reserve.restype = i
+        lib.tidar_oracle_gather_block_q.argtypes = [i, i, i, i, P, P, P]
+        lib.tidar_oracle_gather_block_q.restype = i
         _lib = lib
     return _lib
 
@@ -216,3 +219,21 @@ def reserve(page_table, seq_lens, free_pages, free_count, k, page_size, num_page
                                      pt.shape[1], num_pages, _ptr(sl), _ptr(fp), _ptr(fc),
                                      fp.shape[0], _ptr(ret), nret)
     return pt, fp, int(fc[0]), int(flags)
+
+
+def gather_block_q(block_logits, draft_block, k):
+    """Draft distributions from the previous step's mask blocks.
+
+    block_logits [B][k][k][V] (fp32 or bf16 bits), draft_block [B] int32 (1..k).
+    Returns (draft_logits [B][k-1][V], flags): row i-1 is block
+    draft_block[b], slot i+1; a block outside 1..k reads block 1 and sets
+    GATHER_FLAG_BLOCK.
+    """
+    lib = _load()
+    bl = np.ascontiguousarray(block_logits)
+    db = np.ascontiguousarray(draft_block, dtype=np.int32)
+    B, kk, k2, V = bl.shape
+    assert kk == k and k2 == k
+    out = np.zeros((B, max(k - 1, 0), V), bl.dtype)
+    flags = lib.tidar_oracle_gather_block_q(B, k, V, bl.dtype.itemsize, _ptr(bl), _ptr(db), _ptr(out))
+    return out, int(flags)

@@ -537,3 +537,38 @@ int tidar_oracle_reserve(int B, int k, int page_size, int max_prefix, int32_t* p
   *free_count = count - total;
   return flag;
 }
+
+/*
+ * The draft distributions of a step, taken from the previous step's mask
+ * blocks.  Each block of k slots drafts the k tokens that follow one possible
+ * accept count ([NDfr] paragraph on betting on every outcome: one guess block
+ * per future, the matching one is waiting when verification confirms it;
+ * [MS] §2: the pre-drafts are sampled from the diffusion predictions of the
+ * mask slots).  The selected block j becomes the next step's drafts
+ * [t*, g_{j,2}, .., g_{j,k}], so draft d_{i+1} (i >= 1) is slot i+1 of block j
+ * and was drawn from that slot's distribution: q_i = softmax(row (j-1, i) of
+ * the block logits).  Plainest reading of the slot order: slot s of block j is
+ * row (j-1)*k + (s-1) of the [k][k][V] logits, slot 1 being the one t* replaces.
+ *
+ *   block_logits [B][k][k][V] (dtype), draft_block [B] (the previous step's
+ *   selected block, 1..k).  Writes draft_logits [B][k-1][V]: row i-1 = block
+ *   logits row (draft_block[b]-1, i), i = 1..k-1.  A draft_block outside 1..k
+ *   reads block 1 and raises GATHER_FLAG_BLOCK.  Returns the flags.
+ */
+#define GATHER_FLAG_BLOCK 1
+int tidar_oracle_gather_block_q(int B, int k, int V, int elem_bytes, const void* block_logits,
+                                const int32_t* draft_block, void* draft_logits) {
+  int b, i, flags = 0;
+  if (k < 2) return 0;
+  for (b = 0; b < B; ++b) {
+    int j = draft_block[b];
+    if (j < 1 || j > k) { flags |= GATHER_FLAG_BLOCK; j = 1; }
+    for (i = 1; i <= k - 1; ++i) {
+      const int64_t src = (((int64_t)b * k + (j - 1)) * k + i) * V;
+      const int64_t dst = ((int64_t)b * (k - 1) + (i - 1)) * V;
+      memcpy((char*)draft_logits + dst * elem_bytes, (const char*)block_logits + src * elem_bytes,
+             (size_t)V * elem_bytes);
+    }
+  }
+  return flags;
+}

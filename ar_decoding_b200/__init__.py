@@ -89,6 +89,9 @@ def lib():
         L.tidar_verify_noalloc.argtypes = [I, I, I, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P,
                                            P, P, P]
         L.tidar_verify_noalloc.restype = ctypes.c_int
+        L.tidar_verify_blockq.argtypes = [I, I, I, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, P,
+                                          S, P]
+        L.tidar_verify_blockq.restype = ctypes.c_int
         L.tidar_commit.argtypes = [P, P, P, P, P, P]
         L.tidar_commit.restype = ctypes.c_int
         L.tidar_reserve.argtypes = [P, P, P, P, P, P]
@@ -222,6 +225,33 @@ def verify(logits, drafts, k, mode="greedy", *, draft_logits=None, uniforms=None
                             _ptr(outputs["selected_block"]), _ptr(workspace),
                             workspace.numel(), _stream_handle(stream))
     _check(st, "tidar_verify")
+    return outputs
+
+
+def verify_blockq(logits, drafts, k, prev_block_logits, draft_block, uniforms, *,
+                  block_guesses=None, outputs=None, workspace=None, stream=None):
+    """Rejection verification with q read in place from the previous step's mask
+    blocks: prev_block_logits [B][k][k][V], draft_block [B] int32 (last step's
+    selected_block).  Returns the same dict as ``verify``."""
+    _dev(logits, "logits")
+    B, n, V = logits.shape
+    dev = logits.device
+    if outputs is None:
+        outputs = dict(accept_count=torch.empty(B, dtype=torch.int32, device=dev),
+                       out_tokens=torch.empty((B, n), dtype=torch.int32, device=dev),
+                       next_drafts=torch.empty((B, max(k, 1)), dtype=torch.int32, device=dev),
+                       selected_block=torch.empty(B, dtype=torch.int32, device=dev))
+    need = verify_workspace_bytes(B, k, V, REJECTION)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    st = lib().tidar_verify_blockq(B, k, V, _dtype_code(logits), _ptr(logits), _ptr(drafts),
+                                   _ptr(prev_block_logits), _ptr(draft_block), _ptr(uniforms),
+                                   _ptr(block_guesses), _ptr(outputs["accept_count"]),
+                                   _ptr(outputs["out_tokens"]),
+                                   _ptr(outputs["next_drafts"]) if k > 0 else None,
+                                   _ptr(outputs["selected_block"]), _ptr(workspace),
+                                   workspace.numel(), _stream_handle(stream))
+    _check(st, "tidar_verify_blockq")
     return outputs
 
 

@@ -293,12 +293,20 @@ size_t tidar_verify_workspace_bytes(int32_t batch, int32_t k, int32_t vocab, tid
   return tidar::verify_workspace_bytes(batch, k, vocab, mode);
 }
 
-tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
-                          tidar_accept_mode mode, const void* logits, const int32_t* drafts,
-                          const void* draft_logits, const float* uniforms,
-                          const int32_t* block_guesses, int32_t* accept_count,
-                          int32_t* out_tokens, int32_t* next_drafts, int32_t* selected_block,
-                          void* workspace, size_t workspace_bytes, tidar_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by tidar_verify and tidar_verify_blockq: draft_block null means
+// draft_logits is [B][k-1][V]; else it is the previous step's [B][k][k][V]
+// block logits, read through draft_block.
+tidar_status verify_launch(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                           tidar_accept_mode mode, const void* logits, const int32_t* drafts,
+                           const void* draft_logits, const int32_t* draft_block,
+                           const float* uniforms, const int32_t* block_guesses,
+                           int32_t* accept_count, int32_t* out_tokens, int32_t* next_drafts,
+                           int32_t* selected_block, void* workspace, size_t workspace_bytes,
+                           tidar_stream_t stream) {
   if (batch < 0 || k < 0 || vocab <= 0) return TIDAR_ERR_INVALID_ARG;
   if (k > 16) return TIDAR_ERR_UNSUPPORTED;
   if (dtype != TIDAR_F32 && dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
@@ -313,9 +321,10 @@ tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype d
   if (workspace_bytes < need ||
       (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))))
     return TIDAR_ERR_INVALID_ARG;
-  tidar::VerifyArgs a;
+  tidar::VerifyArgs a{};
   a.B = batch; a.k = k; a.n = k > 0 ? k : 1; a.V = vocab; a.bf16 = dtype == TIDAR_BF16; a.mode = mode;
   a.logits = logits; a.drafts = drafts; a.draft_logits = draft_logits; a.uniforms = uniforms;
+  a.draft_block = k > 1 ? draft_block : nullptr;
   a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;
   a.next_drafts = next_drafts; a.selected_block = selected_block; a.workspace = workspace;
   tidar_status est = error_word(&a.err);
@@ -323,6 +332,34 @@ tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype d
   cudaError_t e = tidar::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return TIDAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                          tidar_accept_mode mode, const void* logits, const int32_t* drafts,
+                          const void* draft_logits, const float* uniforms,
+                          const int32_t* block_guesses, int32_t* accept_count,
+                          int32_t* out_tokens, int32_t* next_drafts, int32_t* selected_block,
+                          void* workspace, size_t workspace_bytes, tidar_stream_t stream) {
+  return verify_launch(batch, k, vocab, dtype, mode, logits, drafts, draft_logits, nullptr,
+                       uniforms, block_guesses, accept_count, out_tokens, next_drafts,
+                       selected_block, workspace, workspace_bytes, stream);
+}
+
+tidar_status tidar_verify_blockq(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                                 const void* logits, const int32_t* drafts,
+                                 const void* prev_block_logits, const int32_t* draft_block,
+                                 const float* uniforms, const int32_t* block_guesses,
+                                 int32_t* accept_count, int32_t* out_tokens, int32_t* next_drafts,
+                                 int32_t* selected_block, void* workspace, size_t workspace_bytes,
+                                 tidar_stream_t stream) {
+  if (k > 1 && batch > 0 && (!prev_block_logits || !draft_block)) return TIDAR_ERR_INVALID_ARG;
+  return verify_launch(batch, k, vocab, dtype, TIDAR_REJECTION, logits, drafts, prev_block_logits,
+                       draft_block, uniforms, block_guesses, accept_count, out_tokens, next_drafts,
+                       selected_block, workspace, workspace_bytes, stream);
 }
 
 tidar_status tidar_commit(const tidar_step_desc* d, const tidar_kv_cache* c,

@@ -55,6 +55,11 @@ struct VerifyArgs {
   const void* logits;
   const int32_t* drafts;
   const void* draft_logits;
+  // Rejection: null when draft_logits is [B][k-1][V] (q_i in row i-1); else
+  // draft_logits is the previous step's block logits [B][k][k][V] and q_i is
+  // block draft_block[b] (1..k; outside -> block 1, TIDAR_DEVERR_BAD_COUNT),
+  // slot i+1.
+  const int32_t* draft_block;
   const float* uniforms;
   const int32_t* block_guesses;
   int32_t* accept_count;

@@ -47,6 +47,19 @@ struct ChunkStat {
 template <typename T>
 __device__ __forceinline__ float ld(const T* p, int i) { return to_f32(p[i]); }
 
+// Logit row of q_i (i = 1..k-1: the distribution draft d_{i+1} was drawn
+// from) for sequence b.  With draft_block the rows are read in place from the
+// previous step's mask-block logits: the selected block j supplied the drafts
+// [t*, g_{j,2}, .., g_{j,k}], so d_{i+1} came from slot i+1 of block j.
+template <typename T>
+__device__ __forceinline__ const T* q_row(const VerifyArgs& a, int b, int i) {
+  const T* base = static_cast<const T*>(a.draft_logits);
+  if (!a.draft_block) return base + ((size_t)b * (a.k - 1) + (i - 1)) * a.V;
+  int j = a.draft_block[b];
+  if (j < 1 || j > a.k) j = 1;
+  return base + (((size_t)b * a.k + (j - 1)) * a.k + i) * a.V;
+}
+
 // Exact argmax merge: larger value wins, equal values -> lower index.
 __device__ __forceinline__ void amax_merge(float& v, int& i, float v2, int i2) {
   if (v2 > v || (v2 == v && i2 < i)) { v = v2; i = i2; }
@@ -105,7 +118,7 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat
   const int c = blockIdx.x, rr = blockIdx.y;
   const int prow = a.B * a.n;
   const T* row = rr < prow ? static_cast<const T*>(a.logits) + (size_t)rr * a.V
-                           : static_cast<const T*>(a.draft_logits) + (size_t)(rr - prow) * a.V;
+                           : q_row<T>(a, (rr - prow) / (a.k - 1), (rr - prow) % (a.k - 1) + 1);
   float x[kPer];
   int ix[kPer];
   load_chunk<T>(row, a.V, c * kChunk, x, ix, vec_ok);
@@ -379,26 +392,34 @@ __device__ void row_norm(const ChunkStat* st, int nchunk, double& M, double& Z) 
   for (int c = 0; c < nchunk; ++c) Z += exp((double)st[c].max - M) * st[c].sum;
 }
 
-// The accept scan for sequence b under the rejection rule; returns j.
+// The accept scan for sequence b under the rejection rule; returns j.  Run by
+// a whole warp: the n-1 tests are independent once the chunk statistics exist
+// (only "stop at the first rejection" orders them), so lane i-1 evaluates
+// test i -- the same fp64 arithmetic as a sequential scan -- and a ballot
+// finds the first failure: j = that i, or n when every test passes.
 template <typename T>
-__device__ int rejection_scan(const VerifyArgs& a, int b, const ChunkStat* stats, int nchunk) {
+__device__ int rejection_scan_warp(const VerifyArgs& a, int b, const ChunkStat* stats, int nchunk) {
   const int prow = a.B * a.n;
-  int j = 1;
-  for (int i = 1; i <= a.n - 1; ++i) {
+  const int i = (threadIdx.x & 31) + 1;          // this lane's test decides d_{i+1}
+  bool fail = false;
+  if (i <= a.n - 1) {
     const int d = a.drafts[(size_t)b * a.k + i];
-    if (d < 0 || d >= a.V) break;
-    double Mp, Zp, Mq, Zq;
-    const size_t lrow = (size_t)b * a.n + (i - 1);
-    const size_t qrow = (size_t)b * (a.k - 1) + (i - 1);
-    row_norm(stats + lrow * nchunk, nchunk, Mp, Zp);
-    row_norm(stats + (prow + qrow) * nchunk, nchunk, Mq, Zq);
-    const double p = exp((double)ld(static_cast<const T*>(a.logits) + lrow * a.V, d) - Mp) / Zp;
-    const double q = exp((double)ld(static_cast<const T*>(a.draft_logits) + qrow * a.V, d) - Mq) / Zq;
-    const double u = (double)a.uniforms[(size_t)b * a.n + (i - 1)];
-    if (!(u * q < p)) break;
-    j = i + 1;
+    if (d < 0 || d >= a.V) {
+      fail = true;
+    } else {
+      double Mp, Zp, Mq, Zq;
+      const size_t lrow = (size_t)b * a.n + (i - 1);
+      const size_t qrow = (size_t)b * (a.k - 1) + (i - 1);
+      row_norm(stats + lrow * nchunk, nchunk, Mp, Zp);
+      row_norm(stats + (prow + qrow) * nchunk, nchunk, Mq, Zq);
+      const double p = exp((double)ld(static_cast<const T*>(a.logits) + lrow * a.V, d) - Mp) / Zp;
+      const double q = exp((double)ld(q_row<T>(a, b, i), d) - Mq) / Zq;
+      const double u = (double)a.uniforms[(size_t)b * a.n + (i - 1)];
+      fail = !(u * q < p);
+    }
   }
-  return j;
+  const unsigned bal = __ballot_sync(0xffffffffu, fail);
+  return bal ? __ffs(bal) : a.n;                 // lowest failing lane L is test L+1
 }
 
 // Per (chunk, b): the sampling weights' chunk sums for both candidate weight
@@ -412,12 +433,17 @@ __global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const 
   const int c = blockIdx.x, b = blockIdx.y;
   __shared__ int sj;
   __shared__ double sMp, sZp, sMq, sZq;
-  if (threadIdx.x == 0) {
-    const int j = rejection_scan<T>(a, b, stats, nchunk);
-    sj = j;
-    if (c == 0) jbuf[b] = j;
-    row_norm(stats + ((size_t)b * a.n + (j - 1)) * nchunk, nchunk, sMp, sZp);
-    if (j < a.n) {
+  if (threadIdx.x < 32) {
+    const int j = rejection_scan_warp<T>(a, b, stats, nchunk);
+    if (threadIdx.x == 0) {
+      sj = j;
+      if (c == 0) {
+        jbuf[b] = j;
+        if (a.draft_block && a.k > 1 && (a.draft_block[b] < 1 || a.draft_block[b] > a.k))
+          raise_error(a.err, TIDAR_DEVERR_BAD_COUNT);
+      }
+      row_norm(stats + ((size_t)b * a.n + (j - 1)) * nchunk, nchunk, sMp, sZp);
+    } else if (threadIdx.x == 1 && j < a.n) {      // the q_j normaliser on a second lane
       const size_t qrow = (size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1);
       row_norm(stats + qrow * nchunk, nchunk, sMq, sZq);
     }
@@ -431,7 +457,7 @@ __global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const 
   double sr = 0.0, sp = 0.0;
   const double Mp = sMp, Zp = sZp;
   if (j < a.n) {
-    const T* qrow = static_cast<const T*>(a.draft_logits) + ((size_t)b * (a.k - 1) + (j - 1)) * a.V;
+    const T* qrow = q_row<T>(a, b, j);
     float xq[kPer];
     int iq[kPer];
     load_chunk<T>(qrow, a.V, c * kChunk, xq, iq, vec_ok);
@@ -501,12 +527,13 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
     s_target = target - cum;
     s_found = INT_MAX;
     row_norm(stats + ((size_t)b * a.n + (j - 1)) * nchunk, nchunk, sMp, sZp);
-    if (resid) row_norm(stats + ((size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1)) * nchunk, nchunk, sMq, sZq);
+  } else if (threadIdx.x == 32 && j < a.n) {       // q_j normaliser, in parallel (used if resid)
+    row_norm(stats + ((size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1)) * nchunk, nchunk, sMq, sZq);
   }
   __syncthreads();
   const int c0 = s_chunk * kChunk;
   const T* prow = static_cast<const T*>(a.logits) + ((size_t)b * a.n + (j - 1)) * a.V;
-  const T* qrow = s_resid ? static_cast<const T*>(a.draft_logits) + ((size_t)b * (a.k - 1) + (j - 1)) * a.V : nullptr;
+  const T* qrow = s_resid ? q_row<T>(a, b, j) : nullptr;
   // contiguous kPer elements per thread so a block scan gives index order
   double w[kPer];
   double tsum = 0.0;
@@ -674,7 +701,7 @@ extern "C" tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t v
     if (cudaGetSymbolAddress(&ptr, tidar::g_verify_scratch) != cudaSuccess || !ptr) return TIDAR_ERR_CUDA;
     tidar::g_verify_scratch_ptr[dev] = ptr;
   }
-  tidar::VerifyArgs a;
+  tidar::VerifyArgs a{};
   a.B = batch; a.k = k; a.n = k > 0 ? k : 1; a.V = vocab; a.bf16 = dtype == TIDAR_BF16; a.mode = mode;
   a.logits = logits; a.drafts = drafts; a.draft_logits = draft_logits; a.uniforms = uniforms;
   a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;

@@ -240,21 +240,65 @@ def random_pool_state(seed: int):
                 num_pages=num_pages, max_prefix=max_prefix)
 
 
-def make_loop(cfg: StepConfig, steps: int):
-    """Inputs of `steps` chained greedy steps (CPU tensors).
+def make_block_logits(cfg: StepConfig, seed_offset: int = 0, plant_from=None):
+    """Mask-block logits of a step, [B][k][k][V] (block j-1, slot s-1), N(0,
+    logit_std) in cfg's dtype, and draft_block [B] int32 uniform on 1..k.
+
+    With plant_from (the logits [B][k][V] of the step that will read these
+    blocks as its q), rows (any block, slot i+1) for i below a seeded depth in
+    1..k are copies of plant_from row i-1, so q_i = p_i there and those drafts
+    are accepted whatever they are."""
+    gen = torch.Generator().manual_seed(cfg.seed * 7 + 8 + 1000 * seed_offset)
+    B, k, V = cfg.B, cfg.k, cfg.vocab
+    bl = _randn((B, k, k, V), gen, cfg.torch_dtype, std=cfg.logit_std)
+    blk = torch.randint(1, k + 1, (B,), generator=gen, dtype=torch.int32) if k else \
+        torch.zeros(B, dtype=torch.int32)
+    if plant_from is not None and k > 1:
+        depth = torch.randint(1, k + 1, (B,), generator=gen)
+        for b in range(B):
+            for i in range(1, int(depth[b])):
+                bl[b, :, i] = plant_from[b, i - 1]
+    return bl, blk
+
+
+def make_loop(cfg: StepConfig, steps: int, mode: str = "greedy"):
+    """Inputs of `steps` chained steps (CPU tensors).
 
     Returns (attn, ver): attn[s] = make_step of a per-step seed; ver[s] =
-    make_verify(seed_offset=s+1), whose drafts matter only at s = 0 (later
-    steps inherit t*, g_{j,2..k} from the step before).  The block guesses of
-    step s are set so that the drafts step s+1 inherits equal the row argmaxes
-    (first maximal index) of step s+1's logits up to a seeded depth in 1..k, so
-    accept counts spread over 1..k whichever block is selected.
+    make_verify(mode, seed_offset=s+1), whose drafts matter only at s = 0
+    (later steps inherit t*, g_{j,2..k} from the step before).  Greedy: the
+    block guesses of step s are set so that the drafts step s+1 inherits equal
+    the row argmaxes (first maximal index) of step s+1's logits up to a seeded
+    depth in 1..k.  Rejection: the draft-logit rows of step s below a seeded
+    depth are copies of the matching logit rows (q_i = p_i, so those drafts are
+    accepted whatever they are).  Either way accept counts spread over 1..k.
+    "blockq": rejection where step s+1 draws its q from step s's mask-block
+    logits (ver[s]["block_logits"], planted from step s+1's logits as in
+    make_block_logits) through step s's selected block; step 0 uses
+    ver[0]["draft_logits"].
     """
     attn = [make_step(StepConfig(**{**cfg.__dict__, "seed": cfg.seed + 101 * (s + 1)}))
             for s in range(steps)]
-    ver = [make_verify(cfg, "greedy", seed_offset=s + 1) for s in range(steps)]
+    vmode = "rejection" if mode == "blockq" else mode
+    ver = [make_verify(cfg, vmode, seed_offset=s + 1) for s in range(steps)]
     gen = torch.Generator().manual_seed(cfg.seed * 7 + 7)
     k = cfg.k
+    if mode == "blockq":
+        for s in range(steps):
+            nxt = ver[s + 1]["logits"] if s + 1 < steps else None
+            ver[s]["block_logits"] = make_block_logits(cfg, seed_offset=s + 1, plant_from=nxt)[0]
+        mode = "rejection"
+    if mode == "rejection":
+        for s in range(steps):
+            if k < 2:
+                break
+            depth = torch.randint(1, k + 1, (cfg.B,), generator=gen)
+            dl = ver[s]["draft_logits"].clone()
+            for b in range(cfg.B):
+                for i in range(1, int(depth[b])):
+                    dl[b, i - 1] = ver[s]["logits"][b, i - 1]
+            ver[s]["draft_logits"] = dl
+        return attn, ver
     for s in range(steps - 1):
         if k < 2:
             break

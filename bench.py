@@ -231,10 +231,10 @@ class Loop:
     turn comes).  One CUDA graph holds the whole loop; a second restores every
     copy's lengths, page table and free-page stack."""
 
-    def __init__(self, cfg, copies, chain, path="auto"):
+    def __init__(self, cfg, copies, chain, path="auto", mode="greedy"):
         import ar_decoding_b200 as tidar
         from ar_decoding_b200 import synth
-        self.tidar, self.cfg, self.chain, self.path = tidar, cfg, chain, path
+        self.tidar, self.cfg, self.chain, self.path, self.mode = tidar, cfg, chain, path, mode
         dev = torch.device("cuda")
         n = cfg.n
         self.max_prefix = max(cfg.prefix) + chain * n
@@ -245,12 +245,17 @@ class Loop:
             cache = synth.make_cache(cc, device=dev, extra_pages=chain * n // cfg.page_size + 2,
                                      draft_pages=False, max_pages=width)
             pool = {k: v.to(dev) for k, v in synth.make_pool(cc, cache).items()}
-            attn, ver = synth.make_loop(cc, chain)
+            attn, ver = synth.make_loop(cc, chain, mode)
+            rej = mode != "greedy"
             self.copies.append(dict(
                 cache=cache, pool=pool,
                 attn=[{k: v.to(dev) for k, v in a.items()} for a in attn],
                 logits=[v["logits"].to(dev) for v in ver],
                 guesses=[v["block_guesses"].to(dev) for v in ver],
+                uniforms=[v["uniforms"].to(dev) for v in ver] if rej else None,
+                q0=ver[0]["draft_logits"].to(dev) if rej and cfg.k > 1 else None,
+                blocks=[v["block_logits"].to(dev) for v in ver] if mode == "blockq" else None,
+                sel=[torch.empty(cfg.B, dtype=torch.int32, device=dev) for _ in range(2)],
                 drafts0=ver[0]["drafts"].to(dev),
                 saved={k: t.clone() for k, t in (("seq_lens", cache["seq_lens"]),
                                                   ("page_table", cache["page_table"]))},
@@ -270,12 +275,15 @@ class Loop:
         self.out = torch.empty_like(q0)
         self.lse = torch.empty(q0.shape[:3], dtype=torch.float32, device=dev)
         V = c0["logits"][0].shape[2]
-        self.vws = torch.empty(max(tidar.verify_workspace_bytes(cfg.B, cfg.k, V, 0), 256),
+        vmode = tidar.GREEDY if mode == "greedy" else tidar.REJECTION
+        self.vws = torch.empty(max(tidar.verify_workspace_bytes(cfg.B, cfg.k, V, vmode), 256),
                                dtype=torch.uint8, device=dev)
         self.vout = dict(accept_count=torch.empty(cfg.B, dtype=torch.int32, device=dev),
-                         out_tokens=torch.empty((cfg.B, n), dtype=torch.int32, device=dev),
-                         selected_block=torch.empty(cfg.B, dtype=torch.int32, device=dev))
-        self.launches_per_step = 1 + (1 if (need == 0 and self.path_id in (2, 3)) else 2) + 2
+                         out_tokens=torch.empty((cfg.B, n), dtype=torch.int32, device=dev))
+        # reserve, attention (+ finalize), verify (greedy: one cluster kernel;
+        # rejection: stats, residual, select), commit
+        self.launches_per_step = (1 + (1 if (need == 0 and self.path_id in (2, 3)) else 2) +
+                                  (1 if mode == "greedy" else 3) + 1)
 
     def step(self, c, s):
         """Step s of copy c: pages, attention (with the draft-row append),
@@ -289,9 +297,18 @@ class Loop:
         t.step_attn(a["q"], a["k_blk"], a["v_blk"], cp["cache"], k, max_prefix_len=self.max_prefix,
                     path=self.path, out=self.out, lse=self.lse, workspace=self.ws)
         drafts = cp["drafts0"] if s == 0 else cp["drafts"][prev]
-        vout = dict(self.vout, next_drafts=cp["drafts"][s % 2])
-        t.verify(cp["logits"][s], drafts if k else None, k, "greedy",
-                 block_guesses=cp["guesses"][s] if k else None, outputs=vout, workspace=self.vws)
+        vout = dict(self.vout, next_drafts=cp["drafts"][s % 2], selected_block=cp["sel"][s % 2])
+        g = cp["guesses"][s] if k else None
+        if self.mode == "greedy":
+            t.verify(cp["logits"][s], drafts if k else None, k, "greedy", block_guesses=g,
+                     outputs=vout, workspace=self.vws)
+        elif self.mode == "blockq" and s > 0:
+            # q from the previous step's mask blocks, through its selected block
+            t.verify_blockq(cp["logits"][s], drafts, k, cp["blocks"][s - 1], cp["sel"][prev],
+                            cp["uniforms"][s], block_guesses=g, outputs=vout, workspace=self.vws)
+        else:
+            t.verify(cp["logits"][s], drafts if k else None, k, "rejection", draft_logits=cp["q0"],
+                     uniforms=cp["uniforms"][s], block_guesses=g, outputs=vout, workspace=self.vws)
         t.commit(cp["cache"], self.vout["accept_count"], k, max_prefix_len=self.max_prefix,
                  released=cp["rel"][s % 2], num_released=cp["nrel"][s % 2])
 
@@ -485,7 +502,14 @@ def time_attention_launches(st: Step, reps: int):
 def time_e2e(st: Step, K: int, W: int):
     """Same step through the public API with host buffers: the step's inputs are
     copied from pinned host memory and the verification results read back, inside
-    the timed region.  Returns (µs per step, h2d bytes, d2h bytes)."""
+    the timed region.  The copies and calls of one step are one CUDA graph (as a
+    serving loop would issue them): Q and the step K/V are copied first on the
+    launching stream; then the verification inputs (logits, drafts, guesses)
+    are copied on a second stream while the attention runs (the two sets of
+    copies would otherwise share the host link and delay the attention), joined
+    before verify.  Freshly pinned buffers copy slowly the first few times, so
+    the warm-up is longer than W.  Returns (µs per step, h2d bytes, d2h
+    bytes)."""
     c = st.copies[0]
     host_in = {k: v.cpu().pin_memory() for k, v in
                (("q", c["step"]["q"]), ("k_blk", c["step"]["k_blk"]), ("v_blk", c["step"]["v_blk"]),
@@ -493,32 +517,50 @@ def time_e2e(st: Step, K: int, W: int):
     host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in st.vout.items()}
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(v.numel() * v.element_size() for v in host_out.values())
-    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
 
     def one():
+        main = torch.cuda.current_stream()
         c["step"]["q"].copy_(host_in["q"], non_blocking=True)
         c["step"]["k_blk"].copy_(host_in["k_blk"], non_blocking=True)
         c["step"]["v_blk"].copy_(host_in["v_blk"], non_blocking=True)
-        c["logits"].copy_(host_in["logits"], non_blocking=True)
-        c["drafts"].copy_(host_in["drafts"], non_blocking=True)
-        c["guesses"].copy_(host_in["guesses"], non_blocking=True)
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            c["logits"].copy_(host_in["logits"], non_blocking=True)
+            c["drafts"].copy_(host_in["drafts"], non_blocking=True)
+            c["guesses"].copy_(host_in["guesses"], non_blocking=True)
         st.attn(0)
+        main.wait_stream(side)
         st.verify_commit(0)
         for k2 in host_out:
             host_out[k2].copy_(st.vout[k2], non_blocking=True)
 
-    for _ in range(W):
+    for _ in range(max(W, 10)):              # eager warm-up
         one(); st.restore(0)
+    torch.cuda.synchronize()
+    g, gr = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        one()
+    with torch.cuda.graph(gr):
+        st.restore(0)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(W, 10)):
+        g.replay(); gr.replay()
     torch.cuda.synchronize()
     ts = []
     for _ in range(K):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        one()
+        g.replay()
         e1.record(stream)
-        st.restore(0)
+        gr.replay()
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1) * 1e3)
+    want = {k2: v.clone() for k2, v in st.vout.items()}
+    for k2 in host_out:                      # the results did come back
+        if not torch.equal(host_out[k2], want[k2].cpu()):
+            raise RuntimeError(f"e2e: host copy of {k2} differs from the device result")
+    del g, gr
     return statistics.mean(ts), h2d, d2h
 
 
@@ -618,7 +660,7 @@ def run_ours(args, rank, world, local):
         achieved, peak, unit = flops / attn_s / 1e12, tc_peak, "TFLOP/s"
     else:
         achieved, peak, unit = bytes_ / attn_s / 1e9, hbm_peak, "GB/s"
-    e2e_us, h2d, d2h = time_e2e(st, max(5, args.steps // 2), 2)
+    e2e_us, h2d, d2h = time_e2e(st, max(5, args.steps // 2), 3)
     e2e_us = reduce_max(e2e_us, world)
 
     sweep = []
@@ -660,20 +702,27 @@ def run_ours(args, rank, world, local):
 
     loop = None
     if not args.no_loop:
-        lp = Loop(cfg, copies_for(cfg), args.loop_chain, path=args.path)
-        lus, ltok = lp.time(max(3, args.steps // 6))
-        lus = reduce_max(lus, world)
-        nsteps = lp.chain * len(lp.copies)
-        loop = {"workload": f"{cfg.name} decode loop", "chained_steps": lp.chain,
-                "interleaved_sequences": len(lp.copies), "us_per_step": lus,
-                "launches_per_step": lp.launches_per_step,
+        loop = {}
+        for mode in ("greedy", "blockq"):
+            lp = Loop(cfg, copies_for(cfg), args.loop_chain, path=args.path, mode=mode)
+            lus, ltok = lp.time(max(3, args.steps // 6))
+            lus = reduce_max(lus, world)
+            nsteps = lp.chain * len(lp.copies)
+            loop[mode] = {
+                "workload": f"{cfg.name} decode loop",
+                "verify": ("greedy" if mode == "greedy" else
+                           "rejection, q read from the previous step's selected mask block"),
+                "chained_steps": lp.chain, "interleaved_sequences": len(lp.copies),
+                "us_per_step": lus, "launches_per_step": lp.launches_per_step,
                 "committed_tokens_per_step": ltok / nsteps,
                 "tokens_per_s_per_sequence": ltok / nsteps / (lus * 1e-6),
-                "acceptance": "planted: drafts match the next step's argmax up to a depth "
-                              "uniform on 1..k (synthetic, not a model's acceptance)",
+                "acceptance": ("planted: drafts match the next step's argmax up to a depth "
+                               "uniform on 1..k" if mode == "greedy" else
+                               "planted: q_i = p_i below a depth uniform on 1..k") +
+                              " (synthetic, not a model's acceptance)",
                 "path": PATH_NAMES[lp.path_id], "splits": lp.splits}
-        del lp
-        torch.cuda.empty_cache()
+            del lp
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

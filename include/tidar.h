@@ -83,7 +83,7 @@ typedef enum {
 /* Bits of the device error word. */
 #define TIDAR_DEVERR_BAD_PAGE 0x1u      /* a needed page-table entry is -1 or >= num_pages */
 #define TIDAR_DEVERR_BAD_LEN 0x2u       /* seq_lens[b] < 0 or > max_prefix_len */
-#define TIDAR_DEVERR_BAD_COUNT 0x4u     /* accept_count[b] outside 0..n (commit) */
+#define TIDAR_DEVERR_BAD_COUNT 0x4u     /* accept_count[b] outside 0..n (commit); draft_block[b] outside 1..k (tidar_verify_blockq) */
 #define TIDAR_DEVERR_TIMEOUT 0x8u       /* a bounded mbarrier wait ran out */
 #define TIDAR_DEVERR_LAYOUT 0x10u       /* a kernel's shared-memory layout check failed (no work done) */
 #define TIDAR_DEVERR_POOL 0x20u         /* tidar_reserve: too few free pages, or no room for the returned ids */
@@ -199,6 +199,34 @@ tidar_status tidar_verify(int32_t batch, int32_t k, int32_t vocab, tidar_dtype d
                           const int32_t* block_guesses, int32_t* accept_count,
                           int32_t* out_tokens, int32_t* next_drafts, int32_t* selected_block,
                           void* workspace, size_t workspace_bytes, tidar_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Rejection verification whose draft distributions are read in place from the
+ * previous step's mask-block logits.  [NDfr] paragraph on betting on every
+ * outcome (one guess block per possible accept count, waiting for the
+ * verification that confirms it); [MS] §2 (the pre-drafts come from the
+ * diffusion predictions of the mask slots).  The block j selected last step
+ * supplied this step's drafts [t*, g_{j,2}, .., g_{j,k}], so draft d_{i+1}
+ * (i >= 1) was drawn from slot i+1 of block j: q_i is row
+ * (b, j-1, i) of prev_block_logits.  Nothing is gathered or copied; j comes
+ * from draft_block on the device (last step's selected_block), so a loop of
+ * steps needs no host round-trip.
+ *
+ *   prev_block_logits [B][k][k][V] dtype (block j-1, slot s-1), 16-byte aligned
+ *   draft_block       [B] int32, 1..k (a value outside: block 1 is read and
+ *                     TIDAR_DEVERR_BAD_COUNT is set)
+ * Both may be NULL when k <= 1.  Every other argument, the workspace
+ * (tidar_verify_workspace_bytes(..., TIDAR_REJECTION)) and the results are
+ * those of tidar_verify in TIDAR_REJECTION mode with draft_logits row i-1 =
+ * that block row.
+ * ------------------------------------------------------------------------- */
+tidar_status tidar_verify_blockq(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                                 const void* logits, const int32_t* drafts,
+                                 const void* prev_block_logits, const int32_t* draft_block,
+                                 const float* uniforms, const int32_t* block_guesses,
+                                 int32_t* accept_count, int32_t* out_tokens, int32_t* next_drafts,
+                                 int32_t* selected_block, void* workspace, size_t workspace_bytes,
+                                 tidar_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Verification without a caller workspace (no counterpart in the paper; a

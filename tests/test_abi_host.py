@@ -127,6 +127,20 @@ def test_commit_rejects_bad_args(L):
     assert L.tidar_commit(ctypes.byref(d), None, FAKE, FAKE, FAKE, None) == tidar.ERR_INVALID_ARG
 
 
+def test_verify_blockq_rejects_bad_args(L):
+    Q = L.tidar_verify_blockq
+    ws = L.tidar_verify_workspace_bytes(2, 4, 512, tidar.REJECTION)
+    def call(B=2, k=4, bl=FAKE, db=FAKE, u=FAKE, wsb=ws):
+        return Q(B, k, 512, tidar.F32, FAKE, FAKE, bl, db, u, None, FAKE, FAKE, None, None, FAKE,
+                 wsb, None)
+    assert call(bl=None) == tidar.ERR_INVALID_ARG
+    assert call(db=None) == tidar.ERR_INVALID_ARG
+    assert call(u=None) == tidar.ERR_INVALID_ARG
+    assert call(wsb=ws - 1) == tidar.ERR_INVALID_ARG
+    assert call(k=17) == tidar.ERR_UNSUPPORTED
+    assert call(B=0) == tidar.OK
+
+
 def test_reserve_rejects_bad_args(L):
     d, c = _desc(), _cache()
     R = L.tidar_reserve

@@ -120,19 +120,28 @@ def test_reserve_pool_exhausted_and_overflow(oracle_mod):
 # --- the chained decode loop ---------------------------------------------------
 
 LOOPS = [
-    # (name, cfg kwargs, steps): M = R*G decides the attention kernel
+    # (name, cfg kwargs, steps, verify mode, use tidar_verify_noalloc):
+    # M = R*G decides the attention kernel
     ("tc05", dict(B=4, Hq=8, Hkv=2, D=128, k=4, prefix=(62, 63, 64, 190), dtype="bf16",
-                  page_size=64), 6),
+                  page_size=64), 6, "greedy", False),
+    ("tc05-rejection", dict(B=3, Hq=8, Hkv=2, D=128, k=4, prefix=(60, 127, 5), dtype="bf16",
+                            page_size=64), 6, "rejection", False),
     ("dec", dict(B=3, Hq=4, Hkv=2, D=128, k=2, prefix=(61, 127, 300), dtype="bf16",
-                 page_size=64), 6),
+                 page_size=64), 6, "greedy", False),
+    ("dec-noalloc-rejection", dict(B=3, Hq=4, Hkv=2, D=128, k=2, prefix=(62, 1, 255),
+                                   dtype="bf16", page_size=64), 6, "rejection", True),
     ("dec-k0", dict(B=3, Hq=8, Hkv=2, D=128, k=0, prefix=(62, 63, 129), dtype="bf16",
-                    page_size=64), 5),
+                    page_size=64), 5, "greedy", False),
+    # rejection with q read from the previous step's mask blocks through its
+    # selected block (tidar_verify_blockq), chained on the device
+    ("tc05-blockq", dict(B=3, Hq=8, Hkv=2, D=128, k=4, prefix=(63, 64, 200), dtype="bf16",
+                         page_size=64), 6, "blockq", False),
     ("simt", dict(B=3, Hq=4, Hkv=2, D=64, k=3, prefix=(14, 15, 40), dtype="f32",
-                  page_size=16), 6),
+                  page_size=16), 6, "greedy", True),
 ]
 
 
-def _oracle_loop(oracle_mod, cfg, cache, pool, attn, ver, steps, max_prefix):
+def _oracle_loop(oracle_mod, cfg, cache, pool, attn, ver, steps, max_prefix, mode):
     n = synth.to_np
     kp, vp = n(cache["k_pages"]), n(cache["v_pages"])
     pt, sl = n(cache["page_table"]), n(cache["seq_lens"])
@@ -146,8 +155,16 @@ def _oracle_loop(oracle_mod, cfg, cache, pool, attn, ver, steps, max_prefix):
         kp, vp = oracle_mod.append(kp, vp, pt, sl, n(a["k_blk"]), n(a["v_blk"]), cfg.k)
         out, lse = oracle_mod.step_attn(n(a["q"]), n(a["k_blk"]), n(a["v_blk"]), kp, vp, pt, sl,
                                         cfg.k)
+        dl = n(ver[s]["draft_logits"])
+        if mode == "blockq" and s > 0:
+            dl, fl = oracle_mod.gather_block_q(n(ver[s - 1]["block_logits"]),
+                                               per[-1]["verify"]["selected_block"], cfg.k)
+            assert fl == 0
         v = oracle_mod.verify(n(ver[s]["logits"]), drafts if cfg.k else None, cfg.k,
-                              oracle_mod.GREEDY, block_guesses=n(ver[s]["block_guesses"]))
+                              oracle_mod.GREEDY if mode == "greedy" else oracle_mod.REJECTION,
+                              draft_logits=dl,
+                              uniforms=n(ver[s]["uniforms"]),
+                              block_guesses=n(ver[s]["block_guesses"]))
         kp, vp, pt, sl, rel, nrel, st = oracle_mod.commit(kp, vp, pt, sl, v["accept_count"], cfg.k)
         assert st == 0
         ret = rel[:nrel]
@@ -161,7 +178,7 @@ def _clone(d):
     return {k: v.clone() for k, v in d.items()}
 
 
-def _enqueue_loop(cfg, dc, dpool, dattn, dver, outs, steps, max_prefix, drafts0):
+def _enqueue_loop(cfg, dc, dpool, dattn, dver, outs, steps, max_prefix, drafts0, mode, noalloc):
     """Queues `steps` chained steps on the current stream (graph-capturable)."""
     ret = nret = None
     drafts = drafts0
@@ -171,17 +188,29 @@ def _enqueue_loop(cfg, dc, dpool, dattn, dver, outs, steps, max_prefix, drafts0)
         tidar.step_attn(dattn[s]["q"], dattn[s]["k_blk"], dattn[s]["v_blk"], dc, cfg.k,
                         max_prefix_len=max_prefix, out=o["out"], lse=o["lse"],
                         workspace=o["ws"])
-        tidar.verify(dver[s]["logits"], drafts if cfg.k else None, cfg.k, "greedy",
-                     block_guesses=dver[s]["block_guesses"] if cfg.k else None,
-                     outputs=o["verify"], workspace=o["vws"])
+        vkw = dict(draft_logits=dver[s].get("draft_logits") if cfg.k > 1 else None,
+                   uniforms=dver[s]["uniforms"] if mode != "greedy" else None,
+                   block_guesses=dver[s]["block_guesses"] if cfg.k else None,
+                   outputs=o["verify"])
+        if mode == "blockq" and s > 0:
+            tidar.verify_blockq(dver[s]["logits"], drafts, cfg.k, dver[s - 1]["block_logits"],
+                                outs[s - 1]["verify"]["selected_block"], vkw["uniforms"],
+                                block_guesses=vkw["block_guesses"], outputs=o["verify"],
+                                workspace=o["vws"])
+        elif noalloc:
+            tidar.verify_noalloc(dver[s]["logits"], drafts if cfg.k else None, cfg.k,
+                                 "greedy" if mode == "greedy" else "rejection", **vkw)
+        else:
+            tidar.verify(dver[s]["logits"], drafts if cfg.k else None, cfg.k,
+                         "greedy" if mode == "greedy" else "rejection", workspace=o["vws"], **vkw)
         tidar.commit(dc, o["verify"]["accept_count"], cfg.k, max_prefix_len=max_prefix,
                      num_q_heads=cfg.Hq, released=o["released"], num_released=o["num_released"])
         ret, nret = o["released"], o["num_released"]
         drafts = o["verify"]["next_drafts"]
 
 
-@pytest.mark.parametrize("name,kw,steps", LOOPS, ids=[x[0] for x in LOOPS])
-def test_decode_loop_in_one_cuda_graph(oracle_mod, name, kw, steps):
+@pytest.mark.parametrize("name,kw,steps,mode,noalloc", LOOPS, ids=[x[0] for x in LOOPS])
+def test_decode_loop_in_one_cuda_graph(oracle_mod, name, kw, steps, mode, noalloc):
     cfg = synth.StepConfig(f"loop-{name}", vocab=4096, seed=0x10F + len(name), **kw)
     n = cfg.n
     max_prefix = max(cfg.prefix) + steps * n
@@ -189,8 +218,8 @@ def test_decode_loop_in_one_cuda_graph(oracle_mod, name, kw, steps):
     cache = synth.make_cache(cfg, extra_pages=cfg.B * (steps * n // cfg.page_size + 2),
                              draft_pages=False, max_pages=width)
     pool = synth.make_pool(cfg, cache)
-    attn, ver = synth.make_loop(cfg, steps)
-    per, final = _oracle_loop(oracle_mod, cfg, cache, pool, attn, ver, steps, max_prefix)
+    attn, ver = synth.make_loop(cfg, steps, mode)
+    per, final = _oracle_loop(oracle_mod, cfg, cache, pool, attn, ver, steps, max_prefix, mode)
 
     dc, dpool = to_dev(cache), to_dev(pool)
     dattn = [to_dev(a) for a in attn]
@@ -198,7 +227,8 @@ def test_decode_loop_in_one_cuda_graph(oracle_mod, name, kw, steps):
     drafts0 = dver[0]["drafts"]
     desc = tidar.make_desc(dattn[0]["q"], dattn[0]["k_blk"], dc, cfg.k, max_prefix)
     wsb = tidar.step_attn_workspace_bytes(desc)
-    vwsb = tidar.verify_workspace_bytes(cfg.B, cfg.k, cfg.vocab, tidar.GREEDY)
+    vwsb = tidar.verify_workspace_bytes(cfg.B, cfg.k, cfg.vocab,
+                                        tidar.GREEDY if mode == "greedy" else tidar.REJECTION)
     cap = cfg.B * (-(-n // cfg.page_size) + 1)
     outs = []
     for s in range(steps):
@@ -219,13 +249,14 @@ def test_decode_loop_in_one_cuda_graph(oracle_mod, name, kw, steps):
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
-        _enqueue_loop(cfg, _clone(dc), _clone(dpool), dattn, dver, outs, steps, max_prefix, drafts0)
+        _enqueue_loop(cfg, _clone(dc), _clone(dpool), dattn, dver, outs, steps, max_prefix, drafts0,
+                      mode, noalloc)
     torch.cuda.current_stream().wait_stream(side)
     assert tidar.device_status()[0] == tidar.OK
 
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        _enqueue_loop(cfg, dc, dpool, dattn, dver, outs, steps, max_prefix, drafts0)
+        _enqueue_loop(cfg, dc, dpool, dattn, dver, outs, steps, max_prefix, drafts0, mode, noalloc)
     graph.replay()
     status, bits = tidar.device_status()
     assert status == tidar.OK, f"bits {bits:#x}"

@@ -102,3 +102,49 @@ def test_verify_out_of_range_drafts_rejected(oracle_mod):
         vin = synth.make_verify(cfg, mode)
         vin["drafts"][:, 2] = torch.tensor([-1, 512, 10**6, -5, 0, 511, 3, 9], dtype=torch.int32)
         _compare(cfg, _gpu_verify(cfg, vin, mode), _oracle_verify(oracle_mod, cfg, vin, mode), mode)
+
+
+@pytest.mark.parametrize("k", [1, 2, 4, 16])
+@pytest.mark.parametrize("dtype,V", [("f32", 512), ("bf16", 32768), ("bf16", 333)])
+def test_verify_blockq_matches_oracle(oracle_mod, k, dtype, V):
+    """q read in place from the previous step's mask blocks through draft_block."""
+    cfg = synth.StepConfig("vbq", B=40, Hq=1, Hkv=1, D=64, k=k, prefix=(0,) * 40, dtype=dtype,
+                           vocab=V, logit_std=2.0 if dtype == "f32" else 3.0, seed=700 + k + V)
+    vin = synth.make_verify(cfg, "rejection")
+    bl, blk = synth.make_block_logits(cfg, plant_from=vin["logits"])
+    d = lambda t: t.cuda()
+    res = tidar.verify_blockq(d(vin["logits"]), d(vin["drafts"]) if k else None, k,
+                              d(bl) if k > 1 else None, d(blk) if k > 1 else None,
+                              d(vin["uniforms"]), block_guesses=d(vin["block_guesses"]) if k else None)
+    st, bits = tidar.device_status()
+    assert st == tidar.OK, bits
+    got = {key: v.cpu().numpy() for key, v in res.items()}
+    n = synth.to_np
+    dl = oracle_mod.gather_block_q(n(bl), n(blk), k)[0] if k > 1 else None
+    want = oracle_mod.verify(n(vin["logits"]), n(vin["drafts"]) if k else None, k,
+                             oracle_mod.REJECTION, draft_logits=dl, uniforms=n(vin["uniforms"]),
+                             block_guesses=n(vin["block_guesses"]) if k else None,
+                             with_margins=True)
+    _compare(cfg, got, want, "rejection")
+    if k > 1:
+        assert len(set(int(x) for x in want["accept_count"])) >= 2
+
+
+def test_verify_blockq_bad_block_reads_block_one(oracle_mod):
+    k, V = 4, 512
+    cfg = synth.StepConfig("vbq-bad", B=6, Hq=1, Hkv=1, D=64, k=k, prefix=(0,) * 6, dtype="f32",
+                           vocab=V, logit_std=2.0, seed=733)
+    vin = synth.make_verify(cfg, "rejection")
+    bl, blk = synth.make_block_logits(cfg, plant_from=vin["logits"])
+    blk[1], blk[4] = 0, k + 1
+    res = tidar.verify_blockq(vin["logits"].cuda(), vin["drafts"].cuda(), k, bl.cuda(), blk.cuda(),
+                              vin["uniforms"].cuda(), block_guesses=vin["block_guesses"].cuda())
+    st, bits = tidar.device_status()
+    assert st == tidar.ERR_DEVICE and bits == tidar.DEVERR_BAD_COUNT
+    n = synth.to_np
+    dl, flags = oracle_mod.gather_block_q(n(bl), n(blk), k)
+    assert flags == oracle_mod.GATHER_FLAG_BLOCK
+    want = oracle_mod.verify(n(vin["logits"]), n(vin["drafts"]), k, oracle_mod.REJECTION,
+                             draft_logits=dl, uniforms=n(vin["uniforms"]),
+                             block_guesses=n(vin["block_guesses"]), with_margins=True)
+    _compare(cfg, {key: v.cpu().numpy() for key, v in res.items()}, want, "rejection")

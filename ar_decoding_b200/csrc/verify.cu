@@ -422,23 +422,19 @@ __device__ int rejection_scan_warp(const VerifyArgs& a, int b, const ChunkStat* 
   return bal ? __ffs(bal) : a.n;                 // lowest failing lane L is test L+1
 }
 
-// Per (chunk, b): the sampling weights' chunk sums for both candidate weight
-// laws -- residual max(0, p_j - q_j) (when j < n) and p_j itself.
+// Accept scan and the two normalisers of row j, for sequence b, into shared
+// variables of the calling CTA (warp 0: the scan; lanes 0 and 1: the p_j and
+// q_j normalisers).  Ends with __syncthreads.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const ChunkStat* stats,
-                                                            int nchunk, double* wsum, int* jbuf,
-                                                            bool vec_ok) {
-  pdl_wait();
-  pdl_trigger();
-  const int c = blockIdx.x, b = blockIdx.y;
-  __shared__ int sj;
-  __shared__ double sMp, sZp, sMq, sZq;
+__device__ void scan_and_norms(const VerifyArgs& a, int b, bool first, const ChunkStat* stats,
+                               int nchunk, int* jbuf, int& sj, double& sMp, double& sZp,
+                               double& sMq, double& sZq) {
   if (threadIdx.x < 32) {
     const int j = rejection_scan_warp<T>(a, b, stats, nchunk);
     if (threadIdx.x == 0) {
       sj = j;
-      if (c == 0) {
-        jbuf[b] = j;
+      if (first) {
+        if (jbuf) jbuf[b] = j;
         if (a.draft_block && a.k > 1 && (a.draft_block[b] < 1 || a.draft_block[b] > a.k))
           raise_error(a.err, TIDAR_DEVERR_BAD_COUNT);
       }
@@ -449,19 +445,23 @@ __global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const 
     }
   }
   __syncthreads();
-  const int j = sj;
+}
+
+// Chunk c's sums of both candidate weight laws for row j: the residual
+// max(0, p_j - q_j) (when j < n) and p_j itself; valid in thread 0.
+template <typename T>
+__device__ void chunk_weight_sums(const VerifyArgs& a, int b, int c, int j, double Mp, double Zp,
+                                  double Mq, double Zq, bool vec_ok, double& out_r, double& out_p) {
   const T* prow = static_cast<const T*>(a.logits) + ((size_t)b * a.n + (j - 1)) * a.V;
   float xp[kPer];
   int ix[kPer];
   load_chunk<T>(prow, a.V, c * kChunk, xp, ix, vec_ok);
   double sr = 0.0, sp = 0.0;
-  const double Mp = sMp, Zp = sZp;
   if (j < a.n) {
     const T* qrow = q_row<T>(a, b, j);
     float xq[kPer];
     int iq[kPer];
     load_chunk<T>(qrow, a.V, c * kChunk, xq, iq, vec_ok);
-    const double Mq = sMq, Zq = sZq;
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
       if (ix[e] == INT_MAX) continue;
@@ -490,51 +490,23 @@ __global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const 
   if (threadIdx.x == 0) {
     sr = 0.0; sp = 0.0;
     for (int i = 0; i < kThreads / 32; ++i) { sr += s1[i]; sp += s2[i]; }
-    wsum[((size_t)b * nchunk + c) * 2 + 0] = sr;
-    wsum[((size_t)b * nchunk + c) * 2 + 1] = sp;
+    out_r = sr;
+    out_p = sp;
   }
 }
 
-// Inverse CDF: smallest t with u*sum(w) < sum_{x<=t} w(x).  Chunk located from
-// the chunk sums; inside the chunk an fp64 block scan in index order.
+// Inverse CDF inside the located chunk: smallest t with target < the running
+// sum of w (fp64 block scan in index order, kPer contiguous elements per
+// thread); writes the outputs of sequence b.  Called by the whole CTA.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const ChunkStat* stats,
-                                                          int nchunk, const double* wsum,
-                                                          const int* jbuf) {
-  pdl_wait();
-  pdl_trigger();
-  const int b = blockIdx.x;
-  const int j = jbuf[b];
-  __shared__ int s_chunk, s_resid, s_found;
-  __shared__ double s_target, sMp, sZp, sMq, sZq;
+__device__ void select_in_chunk(const VerifyArgs& a, int b, int j, int chunk, bool resid,
+                                double target, double Mp, double Zp, double Mq, double Zq) {
+  __shared__ int s_found, s_last;
   __shared__ double s_scan[kThreads];
-  if (threadIdx.x == 0) {
-    double tr = 0.0, tp = 0.0;
-    for (int c = 0; c < nchunk; ++c) { tr += wsum[((size_t)b * nchunk + c) * 2]; tp += wsum[((size_t)b * nchunk + c) * 2 + 1]; }
-    const int resid = (j < a.n) && (tr > 0.0);
-    const double total = resid ? tr : tp;
-    const double target = (double)a.uniforms[(size_t)b * a.n + (a.n - 1)] * total;
-    double cum = 0.0;
-    int ch = nchunk - 1;
-    for (int c = 0; c < nchunk; ++c) {
-      const double wc = wsum[((size_t)b * nchunk + c) * 2 + (resid ? 0 : 1)];
-      if (target < cum + wc) { ch = c; break; }
-      cum += wc;
-      if (c == nchunk - 1) cum -= wc;   // not found: scan the last chunk
-    }
-    s_chunk = ch;
-    s_resid = resid;
-    s_target = target - cum;
-    s_found = INT_MAX;
-    row_norm(stats + ((size_t)b * a.n + (j - 1)) * nchunk, nchunk, sMp, sZp);
-  } else if (threadIdx.x == 32 && j < a.n) {       // q_j normaliser, in parallel (used if resid)
-    row_norm(stats + ((size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1)) * nchunk, nchunk, sMq, sZq);
-  }
-  __syncthreads();
-  const int c0 = s_chunk * kChunk;
+  if (threadIdx.x == 0) { s_found = INT_MAX; s_last = -1; }
+  const int c0 = chunk * kChunk;
   const T* prow = static_cast<const T*>(a.logits) + ((size_t)b * a.n + (j - 1)) * a.V;
-  const T* qrow = s_resid ? q_row<T>(a, b, j) : nullptr;
-  // contiguous kPer elements per thread so a block scan gives index order
+  const T* qrow = resid ? q_row<T>(a, b, j) : nullptr;
   double w[kPer];
   double tsum = 0.0;
   int last_nz = -1;
@@ -543,9 +515,9 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
     const int id = c0 + threadIdx.x * kPer + e;
     double v = 0.0;
     if (id < a.V) {
-      const double p = exp((double)ld(prow, id) - sMp) / sZp;
-      if (s_resid) {
-        const double q = exp((double)ld(qrow, id) - sMq) / sZq;
+      const double p = exp((double)ld(prow, id) - Mp) / Zp;
+      if (resid) {
+        const double q = exp((double)ld(qrow, id) - Mq) / Zq;
         v = p - q > 0.0 ? p - q : 0.0;
       } else {
         v = p;
@@ -565,7 +537,6 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
     __syncthreads();
   }
   double cum = threadIdx.x ? s_scan[threadIdx.x - 1] : 0.0;
-  const double target = s_target;
   int hit = INT_MAX;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
@@ -574,9 +545,6 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
     if (hit == INT_MAX && id < a.V && target < cum) hit = id;
   }
   if (hit != INT_MAX) atomicMin(&s_found, hit);
-  __shared__ int s_last;
-  if (threadIdx.x == 0) s_last = -1;
-  __syncthreads();
   if (last_nz >= 0) atomicMax(&s_last, last_nz);
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -584,6 +552,116 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
     if (t == INT_MAX) t = s_last >= 0 ? s_last : min(c0 + kChunk, a.V) - 1;
     write_outputs(a, b, j, t);
   }
+}
+
+// Per (chunk, b): the sampling weights' chunk sums (vocabularies of more
+// chunks than a cluster holds).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const ChunkStat* stats,
+                                                            int nchunk, double* wsum, int* jbuf,
+                                                            bool vec_ok) {
+  pdl_wait();
+  pdl_trigger();
+  const int c = blockIdx.x, b = blockIdx.y;
+  __shared__ int sj;
+  __shared__ double sMp, sZp, sMq, sZq;
+  scan_and_norms<T>(a, b, c == 0, stats, nchunk, jbuf, sj, sMp, sZp, sMq, sZq);
+  double sr = 0.0, sp = 0.0;
+  chunk_weight_sums<T>(a, b, c, sj, sMp, sZp, sMq, sZq, vec_ok, sr, sp);
+  if (threadIdx.x == 0) {
+    wsum[((size_t)b * nchunk + c) * 2 + 0] = sr;
+    wsum[((size_t)b * nchunk + c) * 2 + 1] = sp;
+  }
+}
+
+// Inverse CDF from the chunk sums of residual_kernel (one CTA per sequence).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const ChunkStat* stats,
+                                                          int nchunk, const double* wsum,
+                                                          const int* jbuf) {
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.x;
+  const int j = jbuf[b];
+  __shared__ int s_chunk, s_resid;
+  __shared__ double s_target, sMp, sZp, sMq, sZq;
+  if (threadIdx.x == 0) {
+    double tr = 0.0, tp = 0.0;
+    for (int c = 0; c < nchunk; ++c) { tr += wsum[((size_t)b * nchunk + c) * 2]; tp += wsum[((size_t)b * nchunk + c) * 2 + 1]; }
+    const int resid = (j < a.n) && (tr > 0.0);
+    const double total = resid ? tr : tp;
+    const double target = (double)a.uniforms[(size_t)b * a.n + (a.n - 1)] * total;
+    double cum = 0.0;
+    int ch = nchunk - 1;
+    for (int c = 0; c < nchunk; ++c) {     // first chunk whose running sum exceeds target
+      const double wc = wsum[((size_t)b * nchunk + c) * 2 + (resid ? 0 : 1)];
+      if (target < cum + wc) { ch = c; break; }
+      cum += wc;
+      if (c == nchunk - 1) cum -= wc;
+    }
+    const double rem = target - cum;
+    s_chunk = ch;
+    s_resid = resid;
+    s_target = rem;
+    row_norm(stats + ((size_t)b * a.n + (j - 1)) * nchunk, nchunk, sMp, sZp);
+  } else if (threadIdx.x == 32 && j < a.n) {       // q_j normaliser, in parallel (used if resid)
+    row_norm(stats + ((size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1)) * nchunk, nchunk, sMq, sZq);
+  }
+  __syncthreads();
+  select_in_chunk<T>(a, b, j, s_chunk, s_resid != 0, s_target, sMp, sZp, sMq, sZq);
+}
+
+// Residual sums and inverse CDF in one launch: one thread-block cluster per
+// sequence, CTA c = chunk c.  Each CTA runs the accept scan, sums its chunk's
+// weights and leaves them in shared memory; after a cluster barrier every CTA
+// reads all chunk sums over distributed shared memory (added in chunk order,
+// as select_kernel does), locates the target chunk, and the CTA that owns it
+// runs the inverse CDF.  A second cluster barrier keeps every CTA's shared
+// memory alive until the remote reads are done.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyArgs a,
+                                                                        const ChunkStat* stats,
+                                                                        int nchunk, bool vec_ok) {
+  pdl_wait();
+  pdl_trigger();
+  cg::cluster_group cl = cg::this_cluster();
+  const int c = (int)cl.block_rank(), b = blockIdx.y;
+  __shared__ int sj, s_chunk, s_resid;
+  __shared__ double sMp, sZp, sMq, sZq, s_target;
+  __shared__ double s_sum[2];                         // this chunk's (residual, p) sums
+  scan_and_norms<T>(a, b, c == 0, stats, nchunk, nullptr, sj, sMp, sZp, sMq, sZq);
+  const int j = sj;
+  double sr = 0.0, sp = 0.0;
+  chunk_weight_sums<T>(a, b, c, j, sMp, sZp, sMq, sZq, vec_ok, sr, sp);
+  if (threadIdx.x == 0) { s_sum[0] = sr; s_sum[1] = sp; }
+  cl.sync();
+  if (threadIdx.x == 0) {
+    // the chunk sums in chunk order, read from each CTA's shared memory (the
+    // arithmetic of select_kernel)
+    double tr = 0.0, tp = 0.0;
+    for (int r = 0; r < nchunk; ++r) {
+      const double* peer = cl.map_shared_rank(s_sum, r);
+      tr += peer[0];
+      tp += peer[1];
+    }
+    const int resid = (j < a.n) && (tr > 0.0);
+    const double total = resid ? tr : tp;
+    const double target = (double)a.uniforms[(size_t)b * a.n + (a.n - 1)] * total;
+    double cum = 0.0;
+    int ch = nchunk - 1;
+    for (int r = 0; r < nchunk; ++r) {
+      const double wc = cl.map_shared_rank(s_sum, r)[resid ? 0 : 1];
+      if (target < cum + wc) { ch = r; break; }
+      cum += wc;
+      if (r == nchunk - 1) cum -= wc;   // not found: scan the last chunk
+    }
+    s_chunk = ch;
+    s_resid = resid;
+    s_target = target - cum;
+  }
+  cl.sync();                                          // remote reads done; s_* visible
+  if (s_chunk != c) return;
+  select_in_chunk<T>(a, b, j, c, s_resid != 0, s_target, sMp, sZp, sMq, sZq);
 }
 
 template <typename T>
@@ -607,6 +685,12 @@ cudaError_t launch_t(const VerifyArgs& a, cudaStream_t s) {
   char* base = static_cast<char*>(a.workspace) + (((size_t)rows * nchunk * sizeof(ChunkStat) + 255) & ~(size_t)255);
   double* wsum = reinterpret_cast<double*>(base);
   int* jbuf = reinterpret_cast<int*>(base + (((size_t)a.B * nchunk * 2 * sizeof(double) + 255) & ~(size_t)255));
+  // residual sums + inverse CDF: one cluster per sequence when the chunks fit
+  // one cluster, else two launches through the workspace
+  static int rs_limit[64];
+  if (nchunk <= cluster_limit(resid_select_cluster_kernel<T>, kThreads, rs_limit))
+    return launch_cluster(resid_select_cluster_kernel<T>, nchunk, a.B, kThreads, 0, s, a,
+                          (const ChunkStat*)stats, nchunk, vec_ok);
   e = launch_pdl(residual_kernel<T>, dim3(nchunk, a.B), kThreads, 0, s, a, (const ChunkStat*)stats, nchunk, wsum, jbuf,
                  vec_ok);
   if (e != cudaSuccess) return e;

@@ -281,9 +281,12 @@ class Loop:
         self.vout = dict(accept_count=torch.empty(cfg.B, dtype=torch.int32, device=dev),
                          out_tokens=torch.empty((cfg.B, n), dtype=torch.int32, device=dev))
         # reserve, attention (+ finalize), verify (greedy: one cluster kernel;
-        # rejection: stats, residual, select), commit
+        # rejection: chunk statistics, then residual sums + inverse CDF in one
+        # cluster when the vocabulary's 4096-wide chunks fit a portable cluster
+        # of 8, else two launches), commit
+        nchunk = -(-V // 4096)
         self.launches_per_step = (1 + (1 if (need == 0 and self.path_id in (2, 3)) else 2) +
-                                  (1 if mode == "greedy" else 3) + 1)
+                                  (1 if mode == "greedy" else (2 if nchunk <= 8 else 3)) + 1)
 
     def step(self, c, s):
         """Step s of copy c: pages, attention (with the draft-row append),

@@ -148,3 +148,14 @@ def test_verify_blockq_bad_block_reads_block_one(oracle_mod):
                              draft_logits=dl, uniforms=n(vin["uniforms"]),
                              block_guesses=n(vin["block_guesses"]), with_margins=True)
     _compare(cfg, {key: v.cpu().numpy() for key, v in res.items()}, want, "rejection")
+
+
+@pytest.mark.parametrize("V,dtype", [(69632, "bf16"), (70001, "f32")])
+def test_verify_rejection_vocab_past_one_cluster(oracle_mod, V, dtype):
+    """More 4096-wide chunks than a cluster holds: the residual sums and the
+    inverse CDF take two launches through the workspace instead of the cluster."""
+    cfg = synth.StepConfig("vwide", B=6, Hq=1, Hkv=1, D=64, k=4, prefix=(0,) * 6, dtype=dtype,
+                           vocab=V, logit_std=3.0, seed=900 + V)
+    vin = synth.make_verify(cfg, "rejection")
+    _compare(cfg, _gpu_verify(cfg, vin, "rejection"),
+             _oracle_verify(oracle_mod, cfg, vin, "rejection"), "rejection")

@@ -447,16 +447,17 @@ __device__ void scan_and_norms(const VerifyArgs& a, int b, bool first, const Chu
   __syncthreads();
 }
 
-// Chunk c's sums of both candidate weight laws for row j: the residual
-// max(0, p_j - q_j) (when j < n) and p_j itself; valid in thread 0.
+// Chunk c's weights of both candidate laws for row j, in load_chunk's layout:
+// wp = p_j, wr = max(0, p_j - q_j) (0 when j = n); slots past V hold 0.  The
+// probabilities are exp(x - M) times the normaliser's reciprocal (fp64).
 template <typename T>
-__device__ void chunk_weight_sums(const VerifyArgs& a, int b, int c, int j, double Mp, double Zp,
-                                  double Mq, double Zq, bool vec_ok, double& out_r, double& out_p) {
+__device__ void chunk_weights(const VerifyArgs& a, int b, int c, int j, double Mp, double iZp,
+                              double Mq, double iZq, bool vec_ok, double (&wr)[kPer],
+                              double (&wp)[kPer]) {
   const T* prow = static_cast<const T*>(a.logits) + ((size_t)b * a.n + (j - 1)) * a.V;
   float xp[kPer];
   int ix[kPer];
   load_chunk<T>(prow, a.V, c * kChunk, xp, ix, vec_ok);
-  double sr = 0.0, sp = 0.0;
   if (j < a.n) {
     const T* qrow = q_row<T>(a, b, j);
     float xq[kPer];
@@ -464,20 +465,28 @@ __device__ void chunk_weight_sums(const VerifyArgs& a, int b, int c, int j, doub
     load_chunk<T>(qrow, a.V, c * kChunk, xq, iq, vec_ok);
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
-      if (ix[e] == INT_MAX) continue;
-      const double p = exp((double)xp[e] - Mp) / Zp;
-      const double q = exp((double)xq[e] - Mq) / Zq;
-      const double r = p - q;
-      sr += r > 0.0 ? r : 0.0;
-      sp += p;
+      const bool ok = ix[e] != INT_MAX;
+      const double p = ok ? exp((double)xp[e] - Mp) * iZp : 0.0;
+      const double q = ok ? exp((double)xq[e] - Mq) * iZq : 0.0;
+      wp[e] = p;
+      wr[e] = p - q > 0.0 ? p - q : 0.0;
     }
   } else {
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
-      if (ix[e] == INT_MAX) continue;
-      sp += exp((double)xp[e] - Mp) / Zp;
+      wp[e] = ix[e] != INT_MAX ? exp((double)xp[e] - Mp) * iZp : 0.0;
+      wr[e] = 0.0;
     }
   }
+}
+
+// Block sums of both weight arrays, valid in thread 0 (warp butterflies, then
+// the warps in order).
+__device__ void block_sums(const double (&wr)[kPer], const double (&wp)[kPer], double& out_r,
+                           double& out_p) {
+  double sr = 0.0, sp = 0.0;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) { sr += wr[e]; sp += wp[e]; }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     sr += __shfl_xor_sync(0xffffffffu, sr, o);
@@ -495,12 +504,71 @@ __device__ void chunk_weight_sums(const VerifyArgs& a, int b, int c, int j, doub
   }
 }
 
+// Inverse CDF over this CTA's chunk from weights held in load_chunk's layout:
+// runs of L contiguous elements, run r of thread t starting at
+// c0 + (r * kThreads + t) * L (L = the vector width, or 1 for scalar loads).
+// Index-ordered running sums come from one block scan per run; the smallest
+// id with target < running sum is the sample.  Writes the outputs of b.
+template <int L>
+__device__ void select_from_regs(const VerifyArgs& a, int b, int j, int chunk, double target,
+                                 const double (&w)[kPer]) {
+  __shared__ double s_wsum[kThreads / 32];
+  __shared__ int s_found, s_last;
+  if (threadIdx.x == 0) { s_found = INT_MAX; s_last = -1; }
+  const int c0 = chunk * kChunk;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  double base = 0.0;
+  int hit = INT_MAX, last_nz = -1;
+#pragma unroll
+  for (int r = 0; r < kPer / L; ++r) {
+    double ts = 0.0;
+#pragma unroll
+    for (int e = 0; e < L; ++e) ts += w[r * L + e];
+    double x = ts;                                   // inclusive scan over the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    const double up = __shfl_up_sync(0xffffffffu, x, 1);
+    const double excl = lane ? up : 0.0;             // lanes before this one
+    if (lane == 31) s_wsum[wid] = x;
+    __syncthreads();
+    double wpre = 0.0, tot = 0.0;
+    for (int k2 = 0; k2 < kThreads / 32; ++k2) {
+      const double v = s_wsum[k2];
+      if (k2 < wid) wpre += v;
+      tot += v;
+    }
+    __syncthreads();                                 // s_wsum is rewritten next run
+    double cum = base + wpre + excl;
+#pragma unroll
+    for (int e = 0; e < L; ++e) {
+      const int id = c0 + (r * kThreads + (int)threadIdx.x) * L + e;
+      cum += w[r * L + e];
+      if (id < a.V) {
+        if (hit == INT_MAX && target < cum) hit = id;
+        if (w[r * L + e] > 0.0) last_nz = id;
+      }
+    }
+    base += tot;
+  }
+  if (hit != INT_MAX) atomicMin(&s_found, hit);
+  if (last_nz >= 0) atomicMax(&s_last, last_nz);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = s_found;
+    if (t == INT_MAX) t = s_last >= 0 ? s_last : min(c0 + kChunk, a.V) - 1;
+    write_outputs(a, b, j, t);
+  }
+}
+
 // Inverse CDF inside the located chunk: smallest t with target < the running
 // sum of w (fp64 block scan in index order, kPer contiguous elements per
 // thread); writes the outputs of sequence b.  Called by the whole CTA.
 template <typename T>
 __device__ void select_in_chunk(const VerifyArgs& a, int b, int j, int chunk, bool resid,
-                                double target, double Mp, double Zp, double Mq, double Zq) {
+                                double target, double Mp, double iZp, double Mq, double iZq) {
   __shared__ int s_found, s_last;
   __shared__ double s_scan[kThreads];
   if (threadIdx.x == 0) { s_found = INT_MAX; s_last = -1; }
@@ -515,9 +583,9 @@ __device__ void select_in_chunk(const VerifyArgs& a, int b, int j, int chunk, bo
     const int id = c0 + threadIdx.x * kPer + e;
     double v = 0.0;
     if (id < a.V) {
-      const double p = exp((double)ld(prow, id) - Mp) / Zp;
+      const double p = exp((double)ld(prow, id) - Mp) * iZp;
       if (resid) {
-        const double q = exp((double)ld(qrow, id) - Mq) / Zq;
+        const double q = exp((double)ld(qrow, id) - Mq) * iZq;
         v = p - q > 0.0 ? p - q : 0.0;
       } else {
         v = p;
@@ -566,8 +634,10 @@ __global__ void __launch_bounds__(kThreads) residual_kernel(VerifyArgs a, const 
   __shared__ int sj;
   __shared__ double sMp, sZp, sMq, sZq;
   scan_and_norms<T>(a, b, c == 0, stats, nchunk, jbuf, sj, sMp, sZp, sMq, sZq);
+  double wr[kPer], wp[kPer];
+  chunk_weights<T>(a, b, c, sj, sMp, 1.0 / sZp, sMq, sj < a.n ? 1.0 / sZq : 0.0, vec_ok, wr, wp);
   double sr = 0.0, sp = 0.0;
-  chunk_weight_sums<T>(a, b, c, sj, sMp, sZp, sMq, sZq, vec_ok, sr, sp);
+  block_sums(wr, wp, sr, sp);
   if (threadIdx.x == 0) {
     wsum[((size_t)b * nchunk + c) * 2 + 0] = sr;
     wsum[((size_t)b * nchunk + c) * 2 + 1] = sp;
@@ -608,7 +678,8 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
     row_norm(stats + ((size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1)) * nchunk, nchunk, sMq, sZq);
   }
   __syncthreads();
-  select_in_chunk<T>(a, b, j, s_chunk, s_resid != 0, s_target, sMp, sZp, sMq, sZq);
+  select_in_chunk<T>(a, b, j, s_chunk, s_resid != 0, s_target, sMp, 1.0 / sZp, sMq,
+                     s_resid ? 1.0 / sZq : 0.0);
 }
 
 // Residual sums and inverse CDF in one launch: one thread-block cluster per
@@ -631,8 +702,10 @@ __global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyAr
   __shared__ double s_sum[2];                         // this chunk's (residual, p) sums
   scan_and_norms<T>(a, b, c == 0, stats, nchunk, nullptr, sj, sMp, sZp, sMq, sZq);
   const int j = sj;
+  double wr[kPer], wp[kPer];
+  chunk_weights<T>(a, b, c, j, sMp, 1.0 / sZp, sMq, j < a.n ? 1.0 / sZq : 0.0, vec_ok, wr, wp);
   double sr = 0.0, sp = 0.0;
-  chunk_weight_sums<T>(a, b, c, j, sMp, sZp, sMq, sZq, vec_ok, sr, sp);
+  block_sums(wr, wp, sr, sp);
   if (threadIdx.x == 0) { s_sum[0] = sr; s_sum[1] = sp; }
   cl.sync();
   if (threadIdx.x == 0) {
@@ -661,7 +734,16 @@ __global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyAr
   }
   cl.sync();                                          // remote reads done; s_* visible
   if (s_chunk != c) return;
-  select_in_chunk<T>(a, b, j, c, s_resid != 0, s_target, sMp, sZp, sMq, sZq);
+  // the owner scans the weights it already holds (no reload, no recompute)
+  constexpr int kVec = 16 / sizeof(T);
+  const double target = s_target;
+  if (s_resid) {
+    if (vec_ok) select_from_regs<kVec>(a, b, j, c, target, wr);
+    else select_from_regs<1>(a, b, j, c, target, wr);
+  } else {
+    if (vec_ok) select_from_regs<kVec>(a, b, j, c, target, wp);
+    else select_from_regs<1>(a, b, j, c, target, wp);
+  }
 }
 
 template <typename T>

@@ -15,6 +15,11 @@
  * speculative write of the draft rows' K/V), then tidar_verify (left-to-right
  * acceptance and selection of the matching pre-drafted block), then
  * tidar_commit (keep the accepted drafts' cache rows, evict the rest).
+ * Around it, for a loop of steps that never returns to the host:
+ * tidar_reserve (the next step's draft pages from a device stack of free
+ * pages, fed with the pages the commit released) and tidar_verify_blockq
+ * (rejection verification whose draft distributions are read from the
+ * previous step's mask-block logits through its selected block).
  *
  * Conventions for every call:
  *   - All pointers are DEVICE pointers unless stated otherwise, on the device

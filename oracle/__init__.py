@@ -60,6 +60,12 @@ def _load():
         lib.tidar_oracle_reserve.restype = i
         lib.tidar_oracle_gather_block_q.argtypes = [i, i, i, i, P, P, P]
         lib.tidar_oracle_gather_block_q.restype = i
+        lib.tidar_oracle_zone_positions.argtypes = [i, ctypes.c_int64, P]
+        lib.tidar_oracle_zone_positions.restype = i
+        lib.tidar_oracle_rope.argtypes = [i, i, i, ctypes.c_double, P, P, i, P]
+        lib.tidar_oracle_rope.restype = i
+        lib.tidar_oracle_linear.argtypes = [i, i, i, P, i, P, i, P]
+        lib.tidar_oracle_linear.restype = i
         _lib = lib
     return _lib
 
@@ -237,3 +243,41 @@ def gather_block_q(block_logits, draft_block, k):
     out = np.zeros((B, max(k - 1, 0), V), bl.dtype)
     flags = lib.tidar_oracle_gather_block_q(B, k, V, bl.dtype.itemsize, _ptr(bl), _ptr(db), _ptr(out))
     return out, int(flags)
+
+
+def zone_positions(k, P):
+    """Positions of a step's R query rows (drafts at P + r - 1, slot s of block
+    j at P + j + s - 1, the single row of k = 0 at P), int64 [R]."""
+    out = np.zeros(rows_per_seq(k), np.int64)
+    st = _load().tidar_oracle_zone_positions(k, int(P), _ptr(out))
+    if st != 0:
+        raise ValueError(f"oracle zone_positions failed with status {st}")
+    return out
+
+
+def rope(x, pos, base=10000.0):
+    """Rotate-half rotary embedding of x [rows][H][D] (fp32 or bf16 bits) at
+    pos [rows], fp64 [rows][H][D]."""
+    x = np.ascontiguousarray(x)
+    rows, H, D = x.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    out = np.zeros((rows, H, D), np.float64)
+    st = _load().tidar_oracle_rope(rows, H, D, float(base), _ptr(pos), _ptr(x), _dtype_code(x),
+                                   _ptr(out))
+    if st != 0:
+        raise ValueError(f"oracle rope failed with status {st}")
+    return out
+
+
+def linear(x, w):
+    """y = x w^T for x [M][K], w [N][K] (fp32 or bf16 bits), fp64 [M][N]."""
+    x, w = np.ascontiguousarray(x), np.ascontiguousarray(w)
+    M, K = x.shape
+    N = w.shape[0]
+    assert w.shape[1] == K
+    y = np.zeros((M, N), np.float64)
+    st = _load().tidar_oracle_linear(M, N, K, _ptr(x), _dtype_code(x), _ptr(w), _dtype_code(w),
+                                     _ptr(y))
+    if st != 0:
+        raise ValueError(f"oracle linear failed with status {st}")
+    return y

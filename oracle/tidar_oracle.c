@@ -572,3 +572,69 @@ int tidar_oracle_gather_block_q(int B, int k, int V, int elem_bytes, const void*
   }
   return flags;
 }
+
+/*
+ * Layer-level pieces around the step attention (for a step with synthetic
+ * weights: query/key/value projection, rotary position embedding at the zone
+ * positions, output projection).  The pages describe one backbone doing both
+ * jobs in one pass ([NDfr] paragraph on the three zones) and a mask placed so
+ * that it slides forward as the text grows ([NDfr] masking paragraph); they do
+ * not give the position of each row or the position encoding.  Readings taken
+ * here (the plainest ones the rest supports):
+ *   - draft row r (1..k) sits at position P + r - 1, the cache row it is
+ *     appended at;
+ *   - mask slot s of block j sits at P + j + s - 1: block j drafts the tokens
+ *     that follow d_1..d_j, so slot 1 is where t* lands when j drafts are
+ *     accepted and slots 2..k become the next step's drafts d_2..d_k there;
+ *   - k = 0: the single row sits at P;
+ *   - rotary embedding in the rotate-half form: dims f and f + D/2 of a head
+ *     form a pair rotated by the angle pos * base^(-2f/D), f = 0..D/2-1.
+ */
+
+/* Positions of the R query rows of a step with committed length P. */
+int tidar_oracle_zone_positions(int k, int64_t P, int64_t* pos) {
+  int r, j, s;
+  if (k < 0) return ORACLE_ERR_ARG;
+  if (k == 0) { pos[0] = P; return ORACLE_OK; }
+  for (r = 1; r <= k; ++r) pos[r - 1] = P + r - 1;
+  for (j = 1; j <= k; ++j)
+    for (s = 1; s <= k; ++s) pos[k + (j - 1) * k + (s - 1)] = P + j + s - 1;
+  return ORACLE_OK;
+}
+
+/* Rotary embedding of x [rows][H][D] (fp32 or bf16) at pos[rows], in fp64:
+ *   out[f]       = x[f] cos(a_f) - x[f + D/2] sin(a_f)
+ *   out[f + D/2] = x[f] sin(a_f) + x[f + D/2] cos(a_f),   a_f = pos * base^(-2f/D). */
+int tidar_oracle_rope(int rows, int H, int D, double base, const int64_t* pos, const void* x,
+                      int dtype, double* out) {
+  int r, h, f;
+  if (rows < 0 || H <= 0 || D <= 0 || (D & 1) || base <= 0.0) return ORACLE_ERR_ARG;
+  for (r = 0; r < rows; ++r)
+    for (h = 0; h < H; ++h) {
+      const int64_t o = ((int64_t)r * H + h) * D;
+      for (f = 0; f < D / 2; ++f) {
+        const double ang = (double)pos[r] * pow(base, -2.0 * f / D);
+        const double c = cos(ang), sn = sin(ang);
+        const double a = elem(x, o + f, dtype), b = elem(x, o + f + D / 2, dtype);
+        out[o + f] = a * c - b * sn;
+        out[o + f + D / 2] = a * sn + b * c;
+      }
+    }
+  return ORACLE_OK;
+}
+
+/* y [M][N] = x [M][K] times the transpose of w [N][K] (a linear layer whose
+ * weight rows are its outputs), fp64 sums in index order. */
+int tidar_oracle_linear(int M, int N, int K, const void* x, int x_dtype, const void* w,
+                        int w_dtype, double* y) {
+  int m, n, kk;
+  if (M < 0 || N < 0 || K < 0) return ORACLE_ERR_ARG;
+  for (m = 0; m < M; ++m)
+    for (n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (kk = 0; kk < K; ++kk)
+        acc += elem(x, (int64_t)m * K + kk, x_dtype) * elem(w, (int64_t)n * K + kk, w_dtype);
+      y[(int64_t)m * N + n] = acc;
+    }
+  return ORACLE_OK;
+}

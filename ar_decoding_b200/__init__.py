@@ -141,9 +141,33 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
-def _dev(t: torch.Tensor, name: str):
-    if not t.is_cuda or not t.is_contiguous():
+def _dev(t: torch.Tensor, name: str, dtype=None, device=None):
+    """Every tensor handed to the library is a device pointer: a host tensor
+    (or a strided view) is refused here rather than dereferenced on the GPU."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call's tensors are on {device}")
+
+
+def _devopt(t, name: str, dtype=None, device=None):
+    if t is not None:
+        _dev(t, name, dtype, device)
+
+
+def _check_verify_args(logits, drafts, draft_logits, uniforms, block_guesses, outputs, workspace):
+    _dev(logits, "logits")
+    dev = logits.device
+    _devopt(drafts, "drafts", torch.int32, dev)
+    _devopt(draft_logits, "draft_logits", logits.dtype, dev)
+    _devopt(uniforms, "uniforms", torch.float32, dev)
+    _devopt(block_guesses, "block_guesses", torch.int32, dev)
+    _devopt(workspace, "workspace", None, dev)
+    if outputs is not None:
+        for key, t in outputs.items():
+            _dev(t, key, torch.int32, dev)
 
 
 def make_desc(q, k_blk, cache, k, max_prefix_len, scale=0.0, path="auto") -> StepDesc:
@@ -153,9 +177,9 @@ def make_desc(q, k_blk, cache, k, max_prefix_len, scale=0.0, path="auto") -> Ste
                     dtype=_dtype_code(q), softmax_scale=float(scale), path=_PATHS[path])
 
 
-def make_cache_desc(cache) -> KVCacheDesc:
+def make_cache_desc(cache, device=None) -> KVCacheDesc:
     for n in ("k_pages", "v_pages", "page_table", "seq_lens"):
-        _dev(cache[n], n)
+        _dev(cache[n], n, None, device)
     if cache["page_table"].dtype != torch.int32 or cache["seq_lens"].dtype != torch.int32:
         raise ValueError("page_table and seq_lens must be int32")
     return KVCacheDesc(k_pages=cache["k_pages"].data_ptr(), v_pages=cache["v_pages"].data_ptr(),
@@ -179,17 +203,24 @@ def step_attn_workspace_bytes(desc: StepDesc) -> int:
 def step_attn(q, k_blk, v_blk, cache, k, *, max_prefix_len, scale=0.0, path="auto", out=None,
               lse=None, want_lse=True, workspace=None, stream=None):
     """Three-zone step attention (+ draft-row K/V append).  Returns (out, lse)."""
-    for t, n in ((q, "q"), (k_blk, "k_blk"), (v_blk, "v_blk")):
-        _dev(t, n)
+    _dev(q, "q")
+    dev = q.device
+    _dev(k_blk, "k_blk", q.dtype, dev)
+    _dev(v_blk, "v_blk", q.dtype, dev)
     desc = make_desc(q, k_blk, cache, k, max_prefix_len, scale, path)
-    cdesc = make_cache_desc(cache)
+    cdesc = make_cache_desc(cache, dev)
+    if cache["k_pages"].dtype != q.dtype or cache["v_pages"].dtype != q.dtype:
+        raise ValueError("the cache pages must have q's dtype")
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
-        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    _dev(out, "out", q.dtype, dev)
+    _devopt(lse, "lse", torch.float32, dev)
     need = step_attn_workspace_bytes(desc)
     if workspace is None and need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _devopt(workspace, "workspace", None, dev)
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = lib().tidar_step_attn(ctypes.byref(desc), ctypes.byref(cdesc), _ptr(q), _ptr(k_blk),
                                _ptr(v_blk), _ptr(out), _ptr(lse), _ptr(workspace), wbytes,
@@ -218,6 +249,7 @@ def verify(logits, drafts, k, mode="greedy", *, draft_logits=None, uniforms=None
     need = verify_workspace_bytes(B, k, V, m)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check_verify_args(logits, drafts, draft_logits, uniforms, block_guesses, outputs, workspace)
     st = lib().tidar_verify(B, k, V, _dtype_code(logits), m, _ptr(logits), _ptr(drafts),
                             _ptr(draft_logits), _ptr(uniforms), _ptr(block_guesses),
                             _ptr(outputs["accept_count"]), _ptr(outputs["out_tokens"]),
@@ -244,6 +276,9 @@ def verify_blockq(logits, drafts, k, prev_block_logits, draft_block, uniforms, *
     need = verify_workspace_bytes(B, k, V, REJECTION)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check_verify_args(logits, drafts, prev_block_logits, uniforms, block_guesses, outputs,
+                       workspace)
+    _devopt(draft_block, "draft_block", torch.int32, dev)
     st = lib().tidar_verify_blockq(B, k, V, _dtype_code(logits), _ptr(logits), _ptr(drafts),
                                    _ptr(prev_block_logits), _ptr(draft_block), _ptr(uniforms),
                                    _ptr(block_guesses), _ptr(outputs["accept_count"]),
@@ -272,6 +307,7 @@ def verify_noalloc(logits, drafts, k, mode="greedy", *, draft_logits=None, unifo
                        out_tokens=torch.empty((B, n), dtype=torch.int32, device=dev),
                        next_drafts=torch.empty((B, max(k, 1)), dtype=torch.int32, device=dev),
                        selected_block=torch.empty(B, dtype=torch.int32, device=dev))
+    _check_verify_args(logits, drafts, draft_logits, uniforms, block_guesses, outputs, None)
     st = lib().tidar_verify_noalloc(B, k, V, _dtype_code(logits), m, _ptr(logits), _ptr(drafts),
                                     _ptr(draft_logits), _ptr(uniforms), _ptr(block_guesses),
                                     _ptr(outputs["accept_count"]), _ptr(outputs["out_tokens"]),
@@ -291,12 +327,15 @@ def commit(cache, accept_count, k, *, max_prefix_len, head_dim=None, num_q_heads
     desc = StepDesc(batch=B, num_q_heads=num_q_heads or Hkv, num_kv_heads=Hkv, head_dim=D, k=k,
                     page_size=ps, max_prefix_len=int(max_prefix_len), dtype=_dtype_code(kp),
                     softmax_scale=0.0, path=PATH_AUTO)
-    cdesc = make_cache_desc(cache)
+    cdesc = make_cache_desc(cache, kp.device)
     cap = B * ((n + ps - 1) // ps + 1)
     if released is None:
         released = torch.empty(cap, dtype=torch.int32, device=kp.device)
     if num_released is None:
         num_released = torch.empty(1, dtype=torch.int32, device=kp.device)
+    _dev(accept_count, "accept_count", torch.int32, kp.device)
+    _dev(released, "released", torch.int32, kp.device)
+    _dev(num_released, "num_released", torch.int32, kp.device)
     st = lib().tidar_commit(ctypes.byref(desc), ctypes.byref(cdesc), _ptr(accept_count),
                             _ptr(released), _ptr(num_released), _stream_handle(stream))
     _check(st, "tidar_commit")
@@ -316,13 +355,15 @@ def reserve(cache, pool, k, *, max_prefix_len, returned=None, num_returned=None,
     desc = StepDesc(batch=B, num_q_heads=Hkv, num_kv_heads=Hkv, head_dim=D, k=k, page_size=ps,
                     max_prefix_len=int(max_prefix_len), dtype=_dtype_code(kp), softmax_scale=0.0,
                     path=PATH_AUTO)
-    cdesc = make_cache_desc(cache)
+    cdesc = make_cache_desc(cache, kp.device)
     fp, fc = pool["free_pages"], pool["free_count"]
-    _dev(fc, "free_count")
+    _dev(fc, "free_count", torch.int32, kp.device)
     if fp.numel():
-        _dev(fp, "free_pages")
-    if fp.dtype != torch.int32 or fc.dtype != torch.int32:
-        raise ValueError("free_pages and free_count must be int32")
+        _dev(fp, "free_pages", torch.int32, kp.device)
+    elif fp.dtype != torch.int32:
+        raise ValueError("free_pages must be int32")
+    _devopt(returned, "returned", torch.int32, kp.device)
+    _devopt(num_returned, "num_returned", torch.int32, kp.device)
     p = PagePool(free_pages=fp.data_ptr() if fp.numel() else None, free_count=fc.data_ptr(),
                  capacity=int(fp.numel()))
     st = lib().tidar_reserve(ctypes.byref(desc), ctypes.byref(cdesc), ctypes.byref(p),

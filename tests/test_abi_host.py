@@ -174,3 +174,28 @@ def test_plan_covers_workloads(L):
 def test_status_strings(L):
     for s in range(6):
         assert L.tidar_status_string(s)
+
+
+def test_binding_refuses_host_tensors(L):
+    """No CPU fallback: host tensors are refused before anything reaches the library."""
+    import torch
+    from ar_decoding_b200 import synth
+    cfg = synth.StepConfig("host", B=1, Hq=2, Hkv=2, D=64, k=2, prefix=(10,), dtype="f32",
+                           vocab=64)
+    cache, step = synth.make_cache(cfg), synth.make_step(cfg)
+    vin = synth.make_verify(cfg, "rejection")
+    with pytest.raises(ValueError):
+        tidar.step_attn(step["q"], step["k_blk"], step["v_blk"], cache, cfg.k, max_prefix_len=10)
+    with pytest.raises(ValueError):
+        tidar.verify(vin["logits"], vin["drafts"], cfg.k, "greedy")
+    with pytest.raises(ValueError):
+        tidar.verify_noalloc(vin["logits"], vin["drafts"], cfg.k, "rejection",
+                             draft_logits=vin["draft_logits"], uniforms=vin["uniforms"])
+    bl, blk = synth.make_block_logits(cfg)
+    with pytest.raises(ValueError):
+        tidar.verify_blockq(vin["logits"], vin["drafts"], cfg.k, bl, blk, vin["uniforms"])
+    with pytest.raises(ValueError):
+        tidar.commit(cache, torch.ones(1, dtype=torch.int32), cfg.k, max_prefix_len=10)
+    pool = synth.make_pool(cfg, cache)
+    with pytest.raises(ValueError):
+        tidar.reserve(cache, pool, cfg.k, max_prefix_len=10)

@@ -21,6 +21,13 @@ restores the copy's prefix length and page table so every step does identical
 work.  The attention call alone is timed the same way in a second pass.
 ms_per_step / value is the mean step time, max over ranks.
 
+Also in the line: the attention kernel's roofline (algorithmic bytes or flops
+over its launch duration, against the measured peaks), the k sweep, the same
+step end to end with host buffers (e2e), the chained decode loops
+(decode_loop: reserve -> attention -> verify -> commit for 8 steps of 10
+interleaved sequences in one CUDA graph, greedy and rejection with q read
+from the previous step's mask blocks), and the CPU oracle on the host cores.
+
 Prints one JSON line (rank 0).
 """
 from __future__ import annotations

@@ -7,6 +7,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/tidar.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -18,7 +20,10 @@ namespace {
 
 thread_local char g_cuda_msg[256] = "";
 constexpr int kMaxDevices = 64;
+// Per-device address of the error word.  Filled under g_err_mutex, so two host
+// threads making their first call on a device at once look it up once.
 unsigned int* g_err_ptr[kMaxDevices] = {nullptr};
+std::mutex g_err_mutex;
 
 tidar_status cuda_fail(cudaError_t e) {
   snprintf(g_cuda_msg, sizeof g_cuda_msg, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
@@ -31,6 +36,7 @@ tidar_status error_word(unsigned int** out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return TIDAR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_err_mutex);
   if (!g_err_ptr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_tidar_error_word);
@@ -50,6 +56,8 @@ unsigned int* device_error_word() {
   unsigned int* p = nullptr;
   return error_word(&p) == TIDAR_OK ? p : nullptr;
 }
+tidar_status error_word_status(unsigned int** out) { return error_word(out); }
+tidar_status cuda_status(cudaError_t e) { return cuda_fail(e); }
 }  // namespace tidar
 
 namespace {

@@ -11,23 +11,27 @@
 // cached prefix.  The last split also runs the step-key windows (128 step keys
 // each) that hold keys visible to the tile, with the mask applied in softmax.
 //
-// Roles (10 warps):
-//   warp 0      TMA producer: Q tile once; per 128-key block two 64-row pages
-//               of K and V (paged cache, SWIZZLE_128B) or one step-key window.
-//               3-stage ring.  No multicast.
-//   warp 1      TMEM owner and MMA issuer (one thread):
-//               S = Q K_b^T  (kind::f16, A and B from shared memory, fp32 in
-//               TMEM), O_t += P V_b with P read from TMEM (bf16, written over
-//               S_t) and V as an MN-major operand.  Blocks alternate between
-//               two softmax sets (t = b & 1), each with its own S_t and O_t, so
-//               one set's exponentials overlap the other set's loads, maxima
-//               and hand-offs.
-//   warps 2..9  softmax: set 0 = warps 2..5, set 1 = warps 6..9; one thread
-//               per TMEM lane (= packed query row), all 128 block columns.
-//               tcgen05.ld of S, mask, online softmax in the log2 domain, P
-//               back to TMEM as bf16; O_t is rescaled only when the set's row
-//               maximum grows by more than 2^8.  The epilogue merges the two
-//               sets (max, sums, O) and writes O / l.
+// Roles (18 warps, 576 threads):
+//   warp 0       TMA producer: Q tile once; per 128-key block two 64-row pages
+//                of K and V (paged cache, SWIZZLE_128B) or one step-key window.
+//                Separate 3-stage K and V rings.  No multicast.
+//   warp 1       TMEM owner and MMA issuer (one thread):
+//                S_t = Q K_b^T  (kind::f16, A and B from shared memory, fp32 in
+//                TMEM), O_t += P V_b with P read from TMEM (bf16, written over
+//                S_t) and V as an MN-major operand.  Blocks alternate between
+//                two softmax sets (t = b & 1), each with its own S_t and O_t, so
+//                one set's exponentials overlap the other set's loads, maxima
+//                and hand-offs.
+//   warps 2..17  softmax: set 0 = warps 2..9, set 1 = warps 10..17.  Within a
+//                set, the four warps of each half hf take TMEM lane quarter
+//                warp % 4 (32 packed query rows each) and columns
+//                [64 hf, 64 hf + 64) of the block: one thread holds half a row.
+//                The two halves of a row swap their block maxima at a named
+//                barrier; then tcgen05.ld of S, mask, online softmax in the
+//                log2 domain, P back to TMEM as bf16 (each half over the first
+//                32 columns of its own 64).  O_t is rescaled only when the
+//                row maximum grows by more than 2^8.  The epilogue merges the
+//                two sets and the two halves (max, sums, O) and writes O / l.
 // Every mbarrier wait is bounded: on expiry the CTA records TIDAR_DEVERR_TIMEOUT,
 // stops issuing, drains what it issued (bounded), frees TMEM and exits.
 #include <cuda.h>

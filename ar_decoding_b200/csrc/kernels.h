@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/tidar.h"
+
 namespace tidar {
 
 // Everything a step-attention kernel needs, in device pointers and sizes.
@@ -71,6 +73,12 @@ struct VerifyArgs {
 };
 // This device's error word (looked up once per device); nullptr on failure.
 unsigned int* device_error_word();
+// The same lookup as a status (TIDAR_ERR_CUDA with the message recorded for
+// tidar_last_cuda_error on failure).
+tidar_status error_word_status(unsigned int** out);
+// Records a CUDA error's name and text for tidar_last_cuda_error and returns
+// TIDAR_ERR_CUDA.
+tidar_status cuda_status(cudaError_t e);
 size_t verify_workspace_bytes(int B, int k, int V, int mode);
 bool verify_grid_ok(int B, int k, int mode);   // launch grid fits (grid.y <= 65535)
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s);

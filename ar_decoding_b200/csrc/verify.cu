@@ -22,6 +22,8 @@
 #include <climits>
 #include <math.h>
 
+#include <mutex>
+
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -823,11 +825,14 @@ cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s) {
 // loads the library keeps it until the process exits.
 //
 // The device address of the array is looked up (cudaGetSymbolAddress) on the
-// first call made with each device current; that first call should therefore
+// first call made with each device current, under a mutex, so host threads
+// that make their first calls at once are safe; that first call should still
 // happen before any stream capture.  All calls share the one array and it
 // keeps whatever the last call left there.  Verification needs no part of it
 // zeroed: every statistic is written before it is read.  Calls that overlap on
 // the GPU (different streams, no ordering between them) race on the array.
+// CUDA failures return TIDAR_ERR_CUDA with the message recorded for
+// tidar_last_cuda_error, as every other entry point does.
 namespace tidar {
 namespace {
 
@@ -836,6 +841,25 @@ static __device__ __align__(256) unsigned char g_verify_scratch[kNoAllocScratchB
 
 constexpr int kNoAllocMaxDevices = 64;
 void* g_verify_scratch_ptr[kNoAllocMaxDevices] = {nullptr};
+std::mutex g_verify_scratch_mutex;
+
+// Device address of this device's scratch array (looked up once per device).
+tidar_status scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return TIDAR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_verify_scratch_mutex);
+  if (!g_verify_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_verify_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (!ptr) return TIDAR_ERR_CUDA;
+    g_verify_scratch_ptr[dev] = ptr;
+  }
+  *out = g_verify_scratch_ptr[dev];
+  return TIDAR_OK;
+}
 
 }  // namespace
 }  // namespace tidar
@@ -859,22 +883,17 @@ extern "C" tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t v
   // too large for the fixed scratch: refuse before touching the device
   if (tidar::verify_workspace_bytes(batch, k, vocab, mode) > tidar::kNoAllocScratchBytes)
     return TIDAR_ERR_UNSUPPORTED;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return TIDAR_ERR_CUDA;
-  if (dev < 0 || dev >= tidar::kNoAllocMaxDevices) return TIDAR_ERR_UNSUPPORTED;
-  if (!tidar::g_verify_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, tidar::g_verify_scratch) != cudaSuccess || !ptr) return TIDAR_ERR_CUDA;
-    tidar::g_verify_scratch_ptr[dev] = ptr;
-  }
+  void* scratch = nullptr;
+  tidar_status st = tidar::scratch_address(&scratch);
+  if (st != TIDAR_OK) return st;
   tidar::VerifyArgs a{};
   a.B = batch; a.k = k; a.n = k > 0 ? k : 1; a.V = vocab; a.bf16 = dtype == TIDAR_BF16; a.mode = mode;
   a.logits = logits; a.drafts = drafts; a.draft_logits = draft_logits; a.uniforms = uniforms;
   a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;
   a.next_drafts = next_drafts; a.selected_block = selected_block;
-  a.workspace = tidar::g_verify_scratch_ptr[dev];
-  a.err = tidar::device_error_word();
-  if (!a.err) return TIDAR_ERR_CUDA;
-  if (tidar::launch_verify(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TIDAR_ERR_CUDA;
+  a.workspace = scratch;
+  if ((st = tidar::error_word_status(&a.err)) != TIDAR_OK) return st;
+  const cudaError_t e = tidar::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return tidar::cuda_status(e);
   return TIDAR_OK;
 }

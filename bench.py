@@ -22,11 +22,18 @@ work.  The attention call alone is timed the same way in a second pass.
 ms_per_step / value is the mean step time, max over ranks.
 
 Also in the line: the attention kernel's roofline (algorithmic bytes or flops
-over its launch duration, against the measured peaks), the k sweep, the same
-step end to end with host buffers (e2e), the chained decode loops
+over its launch duration, against the measured peaks), the k sweep, the other
+workloads (extra_configs: the serving batch, long-context corners, 1.5B-class
+and tiny, each with its own roofline fractions), the same step end to end with
+host buffers (e2e, rotating the same cold copies), the chained decode loops
 (decode_loop: reserve -> attention -> verify -> commit for 8 steps of 10
 interleaved sequences in one CUDA graph, greedy and rejection with q read
 from the previous step's mask blocks), and the CPU oracle on the host cores.
+
+--impl reference times the plain CPU oracle instead (the only reference this
+path has): one whole step of the same workload per timed step on every
+allowed host core, plus the oracle's whole-step time on each timed workload
+single-threaded and on all cores (cpu_sweep).
 
 Prints one JSON line (rank 0).
 """
@@ -64,8 +71,11 @@ def parse_args():
     ap.add_argument("--no-loop", action="store_true", help="skip the chained decode-loop timing")
     ap.add_argument("--loop-chain", type=int, default=8,
                     help="steps chained per sequence in the decode-loop graph")
-    ap.add_argument("--configs", action="store_true",
-                    help="also time the serving batch and long-context workloads (extra_configs)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (serving batch, long-context corners, "
+                         "1.5B-class, tiny) reported under extra_configs")
+    ap.add_argument("--no-cpu-sweep", action="store_true",
+                    help="reference arm: skip the per-workload oracle timings (cpu_sweep)")
     return ap.parse_args()
 
 
@@ -402,6 +412,16 @@ def copies_for(cfg):
     return max(3, math.ceil(3 * L2_BYTES / per))
 
 
+def bench_config(cfg, prefix: int, k: int) -> dict:
+    """The `config` object of the JSON line: the workload, identical for the GPU
+    arm and the oracle (reference) arm."""
+    return {"workload": "8B-class TiDAR step", "B_per_gpu": cfg.B, "Hq": cfg.Hq,
+            "Hkv": cfg.Hkv, "head_dim": cfg.D, "prefix": prefix, "k": k, "rows": cfg.R,
+            "vocab": cfg.vocab, "page": cfg.page_size,
+            "l2": f"rotating {copies_for(cfg)} independent input copies (> 3x L2) between "
+                  "timed steps"}
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -517,68 +537,77 @@ def time_e2e(st: Step, K: int, W: int):
     launching stream; then the verification inputs (logits, drafts, guesses)
     are copied on a second stream while the attention runs (the two sets of
     copies would otherwise share the host link and delay the attention), joined
-    before verify.  Freshly pinned buffers copy slowly the first few times, so
+    before verify.  Timed steps rotate over the same independent copies as the
+    device-resident timing, so each step's KV cache is cold in L2, exactly as
+    for `value`.  Freshly pinned buffers copy slowly the first few times, so
     the warm-up is longer than W.  Returns (µs per step, h2d bytes, d2h
     bytes)."""
-    c = st.copies[0]
-    host_in = {k: v.cpu().pin_memory() for k, v in
-               (("q", c["step"]["q"]), ("k_blk", c["step"]["k_blk"]), ("v_blk", c["step"]["v_blk"]),
-                ("logits", c["logits"]), ("drafts", c["drafts"]), ("guesses", c["guesses"]))}
+    n = len(st.copies)
+    names = (("q", "step", "q"), ("k_blk", "step", "k_blk"), ("v_blk", "step", "v_blk"))
+    host_in = []
+    for c in st.copies:
+        h = {k: c[a][b].cpu().pin_memory() for k, a, b in names}
+        h.update({k: c[k].cpu().pin_memory() for k in ("logits", "drafts", "guesses")})
+        host_in.append(h)
     host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in st.vout.items()}
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    h2d = sum(v.numel() * v.element_size() for v in host_in[0].values())
     d2h = sum(v.numel() * v.element_size() for v in host_out.values())
     side = torch.cuda.Stream()
 
-    def one():
+    def one(i):
+        c, h = st.copies[i], host_in[i]
         main = torch.cuda.current_stream()
-        c["step"]["q"].copy_(host_in["q"], non_blocking=True)
-        c["step"]["k_blk"].copy_(host_in["k_blk"], non_blocking=True)
-        c["step"]["v_blk"].copy_(host_in["v_blk"], non_blocking=True)
+        c["step"]["q"].copy_(h["q"], non_blocking=True)
+        c["step"]["k_blk"].copy_(h["k_blk"], non_blocking=True)
+        c["step"]["v_blk"].copy_(h["v_blk"], non_blocking=True)
         side.wait_stream(main)
         with torch.cuda.stream(side):
-            c["logits"].copy_(host_in["logits"], non_blocking=True)
-            c["drafts"].copy_(host_in["drafts"], non_blocking=True)
-            c["guesses"].copy_(host_in["guesses"], non_blocking=True)
-        st.attn(0)
+            c["logits"].copy_(h["logits"], non_blocking=True)
+            c["drafts"].copy_(h["drafts"], non_blocking=True)
+            c["guesses"].copy_(h["guesses"], non_blocking=True)
+        st.attn(i)
         main.wait_stream(side)
-        st.verify_commit(0)
+        st.verify_commit(i)
         for k2 in host_out:
             host_out[k2].copy_(st.vout[k2], non_blocking=True)
 
-    for _ in range(max(W, 10)):              # eager warm-up
-        one(); st.restore(0)
+    for j in range(max(W, 10)):              # eager warm-up
+        one(j % n); st.restore(j % n)
     torch.cuda.synchronize()
-    g, gr = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        one()
-    with torch.cuda.graph(gr):
-        st.restore(0)
+    graphs = []
+    for i in range(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one(i)
+        graphs.append(g)
     stream = torch.cuda.current_stream()
-    for _ in range(max(W, 10)):
-        g.replay(); gr.replay()
+    for j in range(max(W, 10)):
+        graphs[j % n].replay(); st.graphs[j % n][2].replay()
     torch.cuda.synchronize()
     ts = []
-    for _ in range(K):
+    for j in range(K):
+        i = j % n
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        g.replay()
+        graphs[i].replay()
         e1.record(stream)
-        gr.replay()
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1) * 1e3)
-    want = {k2: v.clone() for k2, v in st.vout.items()}
-    for k2 in host_out:                      # the results did come back
-        if not torch.equal(host_out[k2], want[k2].cpu()):
-            raise RuntimeError(f"e2e: host copy of {k2} differs from the device result")
-    del g, gr
+        if j == K - 1:                       # the results did come back
+            for k2 in host_out:
+                if not torch.equal(host_out[k2], st.vout[k2].cpu()):
+                    raise RuntimeError(f"e2e: host copy of {k2} differs from the device result")
+        st.graphs[i][2].replay()             # restore the copy's lengths and table (untimed)
+    torch.cuda.synchronize()
+    del graphs
     return statistics.mean(ts), h2d, d2h
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_step_seconds(cfg, row_fraction=1.0, threads=0):
-    """Wall time of the oracle doing one step (attention over a fraction of the
-    rows, verification and commit), scaled to the full step."""
-    import numpy as np
+def oracle_step_seconds(cfg, threads=0):
+    """Wall time of the oracle doing one whole step of `cfg`: attention over every
+    (b, row, head), the draft-row append, greedy verification and the commit.
+    `threads` = 0 uses every allowed core (OpenMP), else that many."""
     import oracle
     from ar_decoding_b200 import synth
     cache, step = synth.make_cache(cfg), synth.make_step(cfg)
@@ -586,23 +615,15 @@ def oracle_step_seconds(cfg, row_fraction=1.0, threads=0):
     n = synth.to_np
     npc = {k: n(v) for k, v in cache.items()}
     nps = {k: n(v) for k, v in step.items()}
-    rows = [(b, r, h) for b in range(cfg.B) for r in range(cfg.R) for h in range(cfg.Hq)]
-    take = max(1, int(round(len(rows) * row_fraction)))
-    idx = np.linspace(0, len(rows) - 1, take).round().astype(int)
-    sel = [rows[i] for i in idx]
     t0 = time.perf_counter()
     oracle.step_attn(nps["q"], nps["k_blk"], nps["v_blk"], npc["k_pages"], npc["v_pages"],
-                     npc["page_table"], npc["seq_lens"], cfg.k, sel=None if take == len(rows) else sel,
-                     num_threads=threads)
-    t_attn = (time.perf_counter() - t0) * len(rows) / take
-    t0 = time.perf_counter()
+                     npc["page_table"], npc["seq_lens"], cfg.k, num_threads=threads)
     kp, vp = oracle.append(npc["k_pages"], npc["v_pages"], npc["page_table"], npc["seq_lens"],
                            nps["k_blk"], nps["v_blk"], cfg.k)
     res = oracle.verify(n(vin["logits"]), n(vin["drafts"]), cfg.k, oracle.GREEDY,
                         block_guesses=n(vin["block_guesses"]))
     oracle.commit(kp, vp, npc["page_table"], npc["seq_lens"], res["accept_count"], cfg.k)
-    t_rest = time.perf_counter() - t0
-    return t_attn + t_rest, take, len(rows)
+    return time.perf_counter() - t0
 
 
 def oracle_threads():
@@ -613,31 +634,47 @@ def oracle_threads():
 
 
 # ----------------------------------------------------------------------------- main
+def cpu_sweep(cores: int):
+    """The oracle's whole-step time on the workloads it is timed on (tiny,
+    1.5B-class, 8B-class at k = 0, 4, 8, 16, one long-context point), single
+    threaded and on every allowed core."""
+    from ar_decoding_b200 import synth
+    out = []
+    for cfg in (synth.tiny(), synth.class_1p5b(), synth.class_8b(k=0), synth.class_8b(k=4),
+                synth.class_8b(k=8), synth.class_8b(k=16), synth.long_context(1, 32768, 4)):
+        row = {"workload": cfg.name, "B": cfg.B, "prefix": max(cfg.prefix), "k": cfg.k,
+               "rows": cfg.R, "dtype": cfg.dtype}
+        for threads, key in ((1, "us_1_thread"), (cores, f"us_{cores}_threads")):
+            row[key] = oracle_step_seconds(cfg, threads) * 1e6
+        out.append(row)
+    return out
+
+
 def run_reference(args, rank, world):
+    """The oracle arm: the plain CPU oracle timed on the host cores, one whole
+    step of the same workload per timed step (nothing sampled or scaled)."""
     if rank != 0:
         return
     cfg = workload(args.k, args.prefix)
     cores = oracle_threads()
-    # each step: the oracle on an evenly spaced fraction of the query rows (plus
-    # the whole verification and commit), scaled to one full step
-    frac = 0.25
     times = []
     for i in range(args.warmup + args.steps):
-        t, take, total = oracle_step_seconds(cfg, frac)
+        t = oracle_step_seconds(cfg, cores)
         if i >= args.warmup:
             times.append(t)
     us = statistics.mean(times) * 1e6
-    sample = (f"oracle on {take} of {total} (b,row,head) attention rows per step (scaled x{total / take:.2f}),"
-              f" full verify+append+commit; {cores} OpenMP threads")
+    sample = (f"one whole step per timed step: all {cfg.B * cfg.R * cfg.Hq} (b, row, head) "
+              f"attention rows, the draft-row append, greedy verify and commit; {cores} "
+              "OpenMP threads")
+    sweep = None if args.no_cpu_sweep else cpu_sweep(cores)
     line = {"impl": "reference", "metric": METRIC, "value": us, "unit": "us", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)",
-            "config": {"workload": "8B-class TiDAR step", "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv,
-                       "head_dim": cfg.D, "prefix": args.prefix, "k": args.k, "rows": cfg.R,
-                       "vocab": cfg.vocab},
+            "config": bench_config(cfg, args.prefix, args.k),
             "cpu_baseline": {"value": us, "unit": "us", "cores": cores, "kind": "oracle",
                              "sample": sample},
+            "cpu_sweep": sweep,
             "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -692,21 +729,26 @@ def run_ours(args, rank, world, local):
             torch.cuda.empty_cache()
 
     extra = []
-    if args.configs:
+    if not args.no_configs:
         from ar_decoding_b200 import synth
-        for c2 in (synth.serving(), synth.long_context(1, 32768, 16), synth.long_context(4, 65536, 16),
-                   synth.long_context(8, 131072, 0), synth.long_context(8, 131072, 16)):
+        for c2 in (synth.serving(), synth.long_context(1, 32768, 0), synth.long_context(1, 32768, 16),
+                   synth.long_context(4, 65536, 4), synth.long_context(4, 65536, 8),
+                   synth.long_context(8, 131072, 0), synth.long_context(8, 131072, 16),
+                   synth.class_1p5b(), synth.tiny()):
             s2 = Step(c2, copies_for(c2), path=args.path)
             su, _ = time_steps(s2, max(5, args.steps // 4), 3, world)
             a2 = reduce_max(time_attention_launches(s2, 2), world) * 1e-6
             b2, f2 = algorithmic(c2)
             extra.append({"workload": c2.name, "B": c2.B, "prefix_total": sum(c2.prefix),
                           "prefix_range": [min(c2.prefix), max(c2.prefix)], "k": c2.k,
+                          "Hq": c2.Hq, "Hkv": c2.Hkv, "head_dim": c2.D, "dtype": c2.dtype,
                           "path": PATH_NAMES[s2.path_id], "splits": s2.splits,
+                          "copies": len(s2.copies),
                           "step_us": reduce_max(statistics.mean(su), world), "attn_us": a2 * 1e6,
                           "attn_hbm_gbs": b2 / a2 / 1e9, "attn_tflops": f2 / a2 / 1e12,
                           "hbm_frac": (b2 / a2 / 1e9) / hbm_peak, "tc_frac": (f2 / a2 / 1e12) / tc_peak,
-                          "roofline_frac": max(b2 / (hbm_peak * 1e9), f2 / (tc_peak * 1e12)) / a2})
+                          "roofline_frac": max(b2 / (hbm_peak * 1e9), f2 / (tc_peak * 1e12)) / a2,
+                          "bound": "tensor" if f2 / (tc_peak * 1e12) > b2 / (hbm_peak * 1e9) else "hbm"})
             del s2
             torch.cuda.empty_cache()
 
@@ -736,11 +778,11 @@ def run_ours(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t, take, total = oracle_step_seconds(cfg, 1.0)
         cores = oracle_threads()
+        t = oracle_step_seconds(cfg, cores)
         cpu = {"value": t * 1e6, "unit": "us", "cores": cores, "kind": "oracle",
-               "sample": f"one full step of the same workload ({total} attention rows, verify, "
-                         f"append, commit) on {cores} OpenMP threads"}
+               "sample": f"one whole step of the same workload ({cfg.B * cfg.R * cfg.Hq} attention "
+                         f"rows, append, verify, commit) on {cores} OpenMP threads"}
 
     agg_gbs = reduce_sum(bytes_ / attn_s / 1e9, world)
     if rank == 0:
@@ -749,12 +791,8 @@ def run_ours(args, rank, world, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_step / 1e3,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded, generated on device)",
-            "config": {"workload": "8B-class TiDAR step", "B_per_gpu": cfg.B, "Hq": cfg.Hq,
-                       "Hkv": cfg.Hkv, "head_dim": cfg.D, "prefix": args.prefix, "k": args.k,
-                       "rows": cfg.R, "vocab": cfg.vocab, "page": cfg.page_size,
-                       "l2": f"rotating {len(st.copies)} independent input copies (> 3x L2)",
-                       "attn_path": PATH_NAMES[st.path_id],
-                       "splits": st.splits},
+            "config": bench_config(cfg, args.prefix, args.k),
+            "attn_plan": {"path": PATH_NAMES[st.path_id], "splits": st.splits},
             "attn_call_us": mean_attn, "attn_us": kern_us, "attn_launches": st.attn_launches,
             "hbm_gbs_attn": bytes_ / attn_s / 1e9,
             "hbm_gbs_all_gpus": agg_gbs,

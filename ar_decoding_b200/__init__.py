@@ -32,10 +32,11 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "tidar.h")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(6)
 F32, BF16 = 0, 1
 GREEDY, REJECTION = 0, 1
-PATH_AUTO, PATH_SIMT, PATH_TC05, PATH_DEC = 0, 1, 2, 3
+PATH_AUTO, PATH_SIMT, PATH_TC05, PATH_DEC, PATH_PAIR = 0, 1, 2, 3, 4
 DEVERR_BAD_PAGE, DEVERR_BAD_LEN, DEVERR_BAD_COUNT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 1, 2, 4, 8, 16
 DEVERR_POOL = 32
-_PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tc05": PATH_TC05, "dec": PATH_DEC}
+_PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tc05": PATH_TC05, "dec": PATH_DEC,
+          "pair": PATH_PAIR}
 
 
 class TidarError(RuntimeError):
@@ -104,6 +105,14 @@ def lib():
         L.tidar_last_cuda_error.restype = ctypes.c_char_p
         L.tidar_debug_set.argtypes = [ctypes.c_int, I]
         L.tidar_debug_set.restype = ctypes.c_int
+        L.tidar_linear.argtypes = [I, I, I, ctypes.c_int, P, P, P, P]
+        L.tidar_linear.restype = ctypes.c_int
+        L.tidar_qkv_rope.argtypes = [P, I, P, P, P, ctypes.c_float, P, P, P, P]
+        L.tidar_qkv_rope.restype = ctypes.c_int
+        L.tidar_layer_step_workspace_bytes.argtypes = [P, I]
+        L.tidar_layer_step_workspace_bytes.restype = S
+        L.tidar_layer_step.argtypes = [P, P, I, P, P, P, ctypes.c_float, P, P, P, S, P]
+        L.tidar_layer_step.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -226,6 +235,95 @@ def step_attn(q, k_blk, v_blk, cache, k, *, max_prefix_len, scale=0.0, path="aut
                                _ptr(v_blk), _ptr(out), _ptr(lse), _ptr(workspace), wbytes,
                                _stream_handle(stream))
     _check(st, "tidar_step_attn")
+    return out, lse
+
+
+def linear(x, w, *, out=None, stream=None):
+    """y = x w^T (bf16; x [rows][in], w [out][in]) on the tensor cores."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(w, "w", torch.bfloat16, x.device)
+    N, K = w.shape
+    if x.numel() % K:
+        raise ValueError(f"x has {x.numel()} elements, not a whole number of rows of {K} features")
+    rows = x.numel() // K
+    if out is None:
+        shape = (*x.shape[:-1], N) if x.shape[-1] == K else (rows, N)
+        out = torch.empty(shape, dtype=torch.bfloat16, device=x.device)
+    if out.numel() != rows * N:
+        raise ValueError(f"out has {out.numel()} elements, expected {rows} x {N}")
+    _dev(out, "out", torch.bfloat16, x.device)
+    _check(lib().tidar_linear(rows, N, K, BF16, _ptr(x), _ptr(w), _ptr(out), _stream_handle(stream)),
+           "tidar_linear")
+    return out
+
+
+def _layer_desc(x, k, Hq, Hkv, max_prefix_len, page_size=64, path="auto"):
+    B, R, _ = x.shape
+    if R != (1 if k == 0 else k + k * k):
+        raise ValueError(f"x has {R} rows per sequence, k = {k} needs {1 if k == 0 else k + k * k}")
+    return StepDesc(batch=B, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=128, k=k,
+                    page_size=page_size, max_prefix_len=int(max_prefix_len), dtype=BF16,
+                    softmax_scale=0.0, path=_PATHS[path])
+
+
+def qkv_rope(x, w_qkv, seq_lens, k, num_q_heads, num_kv_heads, *, max_prefix_len,
+             rope_base=10000.0, out=None, stream=None):
+    """Query/key/value projection of the step rows x [B][R][d_model] with the
+    rotary embedding at their zone positions.  Returns (q, k_blk, v_blk)."""
+    _dev(x, "x", torch.bfloat16)
+    dev = x.device
+    _dev(w_qkv, "w_qkv", torch.bfloat16, dev)
+    _dev(seq_lens, "seq_lens", torch.int32, dev)
+    B, R, dm = x.shape
+    Hq, Hkv = num_q_heads, num_kv_heads
+    if tuple(w_qkv.shape) != ((Hq + 2 * Hkv) * 128, dm):
+        raise ValueError(f"w_qkv is {tuple(w_qkv.shape)}, expected {((Hq + 2 * Hkv) * 128, dm)}")
+    desc = _layer_desc(x, k, Hq, Hkv, max_prefix_len)
+    if out is None:
+        out = (torch.empty((B, R, Hq, 128), dtype=torch.bfloat16, device=dev),
+               torch.empty((B, R, Hkv, 128), dtype=torch.bfloat16, device=dev),
+               torch.empty((B, R, Hkv, 128), dtype=torch.bfloat16, device=dev))
+    for name, t in zip(("q", "k_blk", "v_blk"), out):
+        _dev(t, name, torch.bfloat16, dev)
+    q, kb, vb = out
+    _check(lib().tidar_qkv_rope(ctypes.byref(desc), dm, _ptr(x), _ptr(w_qkv), _ptr(seq_lens),
+                                float(rope_base), _ptr(q), _ptr(kb), _ptr(vb), _stream_handle(stream)),
+           "tidar_qkv_rope")
+    return q, kb, vb
+
+
+def layer_step_workspace_bytes(desc: StepDesc, d_model: int) -> int:
+    return int(lib().tidar_layer_step_workspace_bytes(ctypes.byref(desc), int(d_model)))
+
+
+def layer_step(x, w_qkv, w_o, cache, k, num_q_heads, num_kv_heads, *, max_prefix_len,
+               rope_base=10000.0, path="auto", out=None, lse=None, want_lse=True,
+               workspace=None, stream=None):
+    """One layer of a TiDAR step: projection + rotary embedding, three-zone
+    step attention (with the draft-row append), output projection.
+    Returns (y [B][R][d_model], lse [B][R][Hq])."""
+    _dev(x, "x", torch.bfloat16)
+    dev = x.device
+    _dev(w_qkv, "w_qkv", torch.bfloat16, dev)
+    _dev(w_o, "w_o", torch.bfloat16, dev)
+    B, R, dm = x.shape
+    desc = _layer_desc(x, k, num_q_heads, num_kv_heads, max_prefix_len,
+                       page_size=cache["k_pages"].shape[2], path=path)
+    cdesc = make_cache_desc(cache, dev)
+    if out is None:
+        out = torch.empty((B, R, dm), dtype=torch.bfloat16, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty((B, R, num_q_heads), dtype=torch.float32, device=dev)
+    _dev(out, "out", torch.bfloat16, dev)
+    _devopt(lse, "lse", torch.float32, dev)
+    need = layer_step_workspace_bytes(desc, dm)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", None, dev)
+    st = lib().tidar_layer_step(ctypes.byref(desc), ctypes.byref(cdesc), dm, _ptr(x), _ptr(w_qkv),
+                                _ptr(w_o), float(rope_base), _ptr(out), _ptr(lse), _ptr(workspace),
+                                workspace.numel(), _stream_handle(stream))
+    _check(st, "tidar_layer_step")
     return out, lse
 
 

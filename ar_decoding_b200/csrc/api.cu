@@ -77,7 +77,7 @@ tidar_status check_desc(const tidar_step_desc* d) {
     return TIDAR_ERR_UNSUPPORTED;
   if (d->dtype != TIDAR_F32 && d->dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
   if (d->path != TIDAR_PATH_AUTO && d->path != TIDAR_PATH_SIMT && d->path != TIDAR_PATH_TC05 &&
-      d->path != TIDAR_PATH_DEC)
+      d->path != TIDAR_PATH_DEC && d->path != TIDAR_PATH_PAIR)
     return TIDAR_ERR_INVALID_ARG;
   return TIDAR_OK;
 }
@@ -110,14 +110,15 @@ constexpr int kNumSMs = 148;
 int g_force_partials = 0;   // TIDAR_DEBUG_FORCE_SPLIT_PARTIALS
 
 struct Plan {
-  int path;    // 1 SIMT, 2 TC05, 3 DEC
+  int path;    // 1 SIMT, 2 TC05, 3 DEC, 4 PAIR
   int nsplit;
   int keys_per_split;
   bool cluster_merge;   // TC05: splits merged on chip in one cluster (no partials, no finalize)
 };
 
-// Key ranges are multiples of 128 keys.  SIMT: aim for ~2 waves of 4-warp CTAs.
-// TC05: one CTA per (b, kv head, 128-row tile, split); aim for one wave.
+// Key ranges are multiples of 128 keys (64 on the decode path).  SIMT: aim for
+// ~2 waves of 4-warp CTAs.  TC05 / PAIR / DEC: one CTA per SM and per (b, kv
+// head, query tile or pair of tiles, split), split count from a cost model.
 Plan make_plan(const tidar_step_desc* d, int path) {
   Plan p;
   p.path = path;
@@ -128,33 +129,23 @@ Plan make_plan(const tidar_step_desc* d, int path) {
   const int blocks128 = (maxP + 127) / 128;
   long long units;
   int target;
-  if (path == 2) {
+  if (path == 2 || path == 4) {
     const int rows_per_tile = (128 / G) * G;
     const int tiles = (M + rows_per_tile - 1) / rows_per_tile;
-    units = (long long)d->batch * d->num_kv_heads * tiles;
+    units = (long long)d->batch * d->num_kv_heads * (path == 4 ? (tiles + 1) / 2 : tiles);
     target = kNumSMs;
   } else if (path == 3) {
-    units = (long long)d->batch * d->num_kv_heads;   // one CTA per SM, one wave
+    units = (long long)d->batch * d->num_kv_heads;
     target = kNumSMs;
   } else {
     units = (long long)d->batch * d->num_kv_heads * ((M + 3) / 4);
     target = 2 * kNumSMs * 4;
   }
-  int ns = 1;
-  if (path == 2 || path == 3) {
-    // one CTA per SM: as many splits as fit in a single wave
-    if (units > 0 && units < target) ns = (int)(target / units);
-  } else if (units > 0 && units < target) {
-    ns = (int)((target + units - 1) / units);
-  }
-  // at least 2 key blocks of 128 per split (tensor-core path), 2 pages of 64
+  // at least 2 key blocks of 128 per split (tensor-core paths), 2 pages of 64
   // (decode path), 1 block for SIMT
   const int max_ns = path == 3 ? ((maxP + 63) / 64 / 2 > 0 ? (maxP + 63) / 64 / 2 : 1)
-                               : (path == 2 ? (blocks128 / 2 > 0 ? blocks128 / 2 : 1)
-                                            : (blocks128 > 0 ? blocks128 : 1));
-  if (ns > max_ns) ns = max_ns;
-  if (ns > 64) ns = 64;
-  if (ns < 1) ns = 1;
+                               : ((path == 2 || path == 4) ? (blocks128 / 2 > 0 ? blocks128 / 2 : 1)
+                                                           : (blocks128 > 0 ? blocks128 : 1));
   auto split_keys = [&](int n) {
     if (path == 3) {                                  // pages of 64 keys
       const int pages = (maxP + 63) / 64;
@@ -164,33 +155,57 @@ Plan make_plan(const tidar_step_desc* d, int path) {
       if (p.nsplit < 1) p.nsplit = 1;
       return;
     }
-    // tensor-core path: the last split also runs the tile's step-key windows
+    // tensor-core paths: the last split also runs the tile's step-key windows
     // (up to ceil(R / 128) blocks of 128), so the split size counts them and
     // the last split gets that many fewer prefix blocks
-    const int wins = (path == 2 && n > 1) ? (R + 127) / 128 : 0;
+    const int wins = ((path == 2 || path == 4) && n > 1) ? (R + 127) / 128 : 0;
     const int bps = (blocks128 + wins + n - 1) / n;
     p.keys_per_split = (bps > 0 ? bps : 1) * 128;
     p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
     if (p.nsplit < 1) p.nsplit = 1;
   };
-  split_keys(ns);
   p.cluster_merge = false;
-  if ((path == 2 || path == 3) && p.nsplit > 1 && !g_force_partials) {
-    // Merge on chip when one cluster per (b, g, tile) -- all of them at once --
-    // fits the device: the largest split count of at least half the wanted
-    // one whose clusters are all resident together.  Otherwise the splits
-    // write partials that a second launch merges.
-    for (int n = ns < 16 ? ns : 16; n >= 2 && 2 * n >= ns; --n) {
-      split_keys(n);
+  if (path == 1) {
+    // SIMT: aim for ~2 waves of 4-warp CTAs
+    int ns = 1;
+    if (units > 0 && units < target) ns = (int)((target + units - 1) / units);
+    if (ns > max_ns) ns = max_ns;
+    if (ns > 64) ns = 64;
+    split_keys(ns < 1 ? 1 : ns);
+    return p;
+  }
+  // Tensor-core and decode paths (one CTA per SM): choose the split count by a
+  // cost model in units of 128-key blocks per CTA -- the waves of CTAs the
+  // launch needs times (the keys of one split + a fixed per-CTA cost), plus
+  // the second launch when splits merge through workspace partials.  A merge
+  // on chip needs a cluster of nsplit CTAs; its waves count the clusters that
+  // can be resident at once.
+  constexpr double kFixedBlocks = 2.5, kFinalizeBlocks = 2.0;
+  double best = 1e300;
+  int best_n = 1;
+  bool best_cluster = false;
+  int last_ns = -1;
+  const int n_hi = max_ns < 64 ? max_ns : 64;
+  for (int n = 1; n <= n_hi; ++n) {
+    split_keys(n);
+    if (p.nsplit == last_ns) continue;
+    last_ns = p.nsplit;
+    const double per = (double)p.keys_per_split / 128.0 + kFixedBlocks;
+    const long long ctas = units * p.nsplit;
+    const double cost_p = (double)((ctas + target - 1) / target) * per + (p.nsplit > 1 ? kFinalizeBlocks : 0.0);
+    if (cost_p < best) { best = cost_p; best_n = n; best_cluster = false; }
+    if (p.nsplit > 1 && p.nsplit <= 16 && !g_force_partials) {
       const int resident = path == 2 ? tidar::tc05_resident_clusters(p.nsplit)
-                                     : tidar::dec_resident_clusters(p.nsplit, M);
-      if (p.nsplit <= n && resident >= units) {
-        p.cluster_merge = true;
-        break;
+                                     : (path == 4 ? tidar::pair_resident_clusters(p.nsplit)
+                                                  : tidar::dec_resident_clusters(p.nsplit, M));
+      if (resident > 0) {
+        const double cost_c = (double)((units + resident - 1) / resident) * per;
+        if (cost_c < best) { best = cost_c; best_n = n; best_cluster = true; }
       }
     }
-    if (!p.cluster_merge) split_keys(ns);
   }
+  split_keys(best_n);
+  p.cluster_merge = best_cluster && p.nsplit > 1;
   return p;
 }
 
@@ -198,6 +213,7 @@ int choose_path(const tidar_step_desc* d) {
   if (d->path == TIDAR_PATH_SIMT) return 1;
   if (d->path == TIDAR_PATH_TC05) return 2;
   if (d->path == TIDAR_PATH_DEC) return 3;
+  if (d->path == TIDAR_PATH_PAIR) return 4;
   return dec_supported(d) ? 3 : (tc05_supported(d) ? 2 : 1);
 }
 
@@ -223,7 +239,7 @@ tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, in
   tidar_status st = check_desc(desc);
   if (st != TIDAR_OK) return st;
   const int pth = choose_path(desc);
-  if (pth == 2 && !tc05_supported(desc)) return TIDAR_ERR_UNSUPPORTED;
+  if ((pth == 2 || pth == 4) && !tc05_supported(desc)) return TIDAR_ERR_UNSUPPORTED;
   if (pth == 3 && !dec_supported(desc)) return TIDAR_ERR_UNSUPPORTED;
   const Plan p = make_plan(desc, pth);
   if (path) *path = p.path;
@@ -252,7 +268,7 @@ tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, 
   if (!aligned16(q) || !aligned16(k_blk) || !aligned16(v_blk) || !aligned16(out))
     return TIDAR_ERR_INVALID_ARG;
   const int pth = choose_path(d);
-  if (pth == 2 && !tc05_supported(d)) return TIDAR_ERR_UNSUPPORTED;
+  if ((pth == 2 || pth == 4) && !tc05_supported(d)) return TIDAR_ERR_UNSUPPORTED;
   if (pth == 3 && !dec_supported(d)) return TIDAR_ERR_UNSUPPORTED;
   const Plan p = make_plan(d, pth);
   const size_t need = tidar_step_attn_workspace_bytes(d);
@@ -282,8 +298,10 @@ tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, 
                                           align256((size_t)p.nsplit * rows * a.D * sizeof(float)));
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = pth == 2 ? tidar::launch_attn_tc05(a, s)
-                           : (pth == 3 ? tidar::launch_attn_dec(a, s) : tidar::launch_attn_simt(a, s));
+  cudaError_t e = pth == 2   ? tidar::launch_attn_tc05(a, s)
+                  : pth == 3 ? tidar::launch_attn_dec(a, s)
+                  : pth == 4 ? tidar::launch_attn_pair(a, s)
+                             : tidar::launch_attn_simt(a, s);
   if (e == cudaErrorNotSupported) return TIDAR_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return cuda_fail(e);
   // Split merge and draft-row append: a second launch for the CUDA-core path
@@ -415,6 +433,106 @@ tidar_status tidar_reserve(const tidar_step_desc* d, const tidar_kv_cache* c,
   cudaError_t e = tidar::launch_reserve(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return TIDAR_OK;
+}
+
+tidar_status tidar_linear(int32_t rows, int32_t out_features, int32_t in_features, tidar_dtype dtype,
+                          const void* x, const void* w, void* y, tidar_stream_t stream) {
+  if (rows < 0 || out_features <= 0 || in_features <= 0) return TIDAR_ERR_INVALID_ARG;
+  if (dtype != TIDAR_BF16 || in_features % 64 || out_features % 128) return TIDAR_ERR_UNSUPPORTED;
+  if (rows == 0) return TIDAR_OK;
+  if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y)) return TIDAR_ERR_INVALID_ARG;
+  if (!tidar::plan_linear(rows, in_features, out_features).ok) return TIDAR_ERR_UNSUPPORTED;
+  tidar::LinearArgs a{};
+  a.T = rows; a.K = in_features; a.N = out_features; a.mode = 0;
+  a.x = x; a.w = w; a.y = y;
+  tidar_status st = error_word(&a.err);
+  if (st != TIDAR_OK) return st;
+  const cudaError_t e = tidar::launch_linear(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return TIDAR_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
+tidar_status tidar_qkv_rope(const tidar_step_desc* d, int32_t d_model, const void* x, const void* w_qkv,
+                            const int32_t* seq_lens, float rope_base, void* q, void* k_blk, void* v_blk,
+                            tidar_stream_t stream) {
+  tidar_status st = check_desc(d);
+  if (st != TIDAR_OK) return st;
+  if (d_model <= 0 || !(rope_base > 1.0f)) return TIDAR_ERR_INVALID_ARG;
+  if (d->dtype != TIDAR_BF16 || d->head_dim != 128 || d_model % 64) return TIDAR_ERR_UNSUPPORTED;
+  if (d->batch == 0) return TIDAR_OK;
+  if (!x || !w_qkv || !seq_lens || !q || !k_blk || !v_blk) return TIDAR_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(k_blk) || !aligned16(v_blk))
+    return TIDAR_ERR_INVALID_ARG;
+  const int R = tidar::rows_per_seq(d->k);
+  const long long T = (long long)d->batch * R;
+  if (T > 0x7fffffffLL) return TIDAR_ERR_UNSUPPORTED;
+  const int N = (d->num_q_heads + 2 * d->num_kv_heads) * 128;
+  if (!tidar::plan_linear((int)T, d_model, N).ok) return TIDAR_ERR_UNSUPPORTED;
+  tidar::LinearArgs a{};
+  a.T = (int)T; a.K = d_model; a.N = N; a.mode = 1;
+  a.x = x; a.w = w_qkv; a.q = q; a.k_blk = k_blk; a.v_blk = v_blk; a.seq_lens = seq_lens;
+  a.Hq = d->num_q_heads; a.Hkv = d->num_kv_heads; a.R = R; a.k = d->k; a.max_prefix = d->max_prefix_len;
+  a.log2_base = log2((double)rope_base);
+  if ((st = error_word(&a.err)) != TIDAR_OK) return st;
+  const cudaError_t e = tidar::launch_linear(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return TIDAR_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// Byte offsets of the layer step's workspace: q, k_blk, v_blk, attention
+// output, then the step attention's own workspace.
+struct LayerWs {
+  size_t q, kb, vb, o, attn, total;
+};
+LayerWs layer_ws(const tidar_step_desc* d) {
+  LayerWs w{};
+  const size_t rows = (size_t)d->batch * tidar::rows_per_seq(d->k);
+  const size_t qb = rows * d->num_q_heads * 128 * 2, kvb = rows * d->num_kv_heads * 128 * 2;
+  w.q = 0;
+  w.kb = w.q + align256(qb);
+  w.vb = w.kb + align256(kvb);
+  w.o = w.vb + align256(kvb);
+  w.attn = w.o + align256(qb);
+  w.total = w.attn + align256(tidar_step_attn_workspace_bytes(d));
+  return w;
+}
+}  // namespace
+
+extern "C" {
+
+size_t tidar_layer_step_workspace_bytes(const tidar_step_desc* d, int32_t d_model) {
+  if (check_desc(d) != TIDAR_OK || d_model <= 0) return 0;
+  return layer_ws(d).total;
+}
+
+tidar_status tidar_layer_step(const tidar_step_desc* d, const tidar_kv_cache* c, int32_t d_model,
+                              const void* x, const void* w_qkv, const void* w_o, float rope_base, void* y,
+                              float* lse_out, void* workspace, size_t workspace_bytes,
+                              tidar_stream_t stream) {
+  tidar_status st = check_desc(d);
+  if (st != TIDAR_OK) return st;
+  if (d_model <= 0) return TIDAR_ERR_INVALID_ARG;
+  if (d->dtype != TIDAR_BF16 || d->head_dim != 128 || d_model % 128) return TIDAR_ERR_UNSUPPORTED;
+  if (d->batch == 0) return TIDAR_OK;
+  if ((st = check_cache(d, c)) != TIDAR_OK) return st;
+  if (!w_o || !y || !aligned16(w_o) || !aligned16(y)) return TIDAR_ERR_INVALID_ARG;
+  const LayerWs w = layer_ws(d);
+  if (workspace_bytes < w.total || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return TIDAR_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  const int rows = d->batch * tidar::rows_per_seq(d->k);
+  if (!tidar::plan_linear(rows, d->num_q_heads * 128, d_model).ok) return TIDAR_ERR_UNSUPPORTED;
+  st = tidar_qkv_rope(d, d_model, x, w_qkv, c->seq_lens, rope_base, ws + w.q, ws + w.kb, ws + w.vb, stream);
+  if (st != TIDAR_OK) return st;
+  st = tidar_step_attn(d, c, ws + w.q, ws + w.kb, ws + w.vb, ws + w.o, lse_out, ws + w.attn,
+                       workspace_bytes - w.attn, stream);
+  if (st != TIDAR_OK) return st;
+  return tidar_linear(rows, d_model, d->num_q_heads * 128, TIDAR_BF16, ws + w.o, w_o, y, stream);
 }
 
 tidar_status tidar_debug_set(tidar_debug_knob knob, int32_t value) {

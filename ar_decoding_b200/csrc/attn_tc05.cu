@@ -40,6 +40,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tc05.cuh"
 
 namespace tidar {
 
@@ -114,137 +115,7 @@ __device__ __forceinline__ bool trace_cta() { return blockIdx.x == 0 && blockIdx
 #define TIDAR_TRACE_CTA(which) do {} while (0)
 #endif
 
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptors (SWIZZLE_128B, sm_100 version bits).
-// K-major: 8-row groups 1024 B apart; the K offset inside the 128-byte swizzle
-// row is added to the start address.
-__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// MN-major: 64-element MN atoms `lbo` bytes apart, 8-row K groups 1024 B apart.
-__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
-         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-
-#define TIDAR_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
-#define TIDAR_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
-
-// 32 consecutive 32-bit TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-      "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : TIDAR_R8(0), TIDAR_R8(8), TIDAR_R8(16), TIDAR_R8(24)
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-      "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
-      ::"r"(taddr), TIDAR_W8(0), TIDAR_W8(8), TIDAR_W8(16), TIDAR_W8(24)
-      : "memory");
-}
-#define TIDAR_R16(i) TIDAR_R8(i), TIDAR_R8(i + 8)
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-      "%13, %14, %15}, [%16];"
-      : TIDAR_R16(0)
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-      "%13, %14, %15, %16};"
-      ::"r"(taddr), TIDAR_W8(0), TIDAR_W8(8)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-
-// ---- packed fp32x2 helpers (sm_100) and the exponential split --------------
-__device__ __forceinline__ uint64_t f2_make(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-// (lo, hi) -> bf16x2, round to nearest even
-__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-// ------------------------------------------------------------------ block plan
-// Blocks 0..npb-1: 128 prefix keys from k0; then nw step-key windows.
-struct BlockPlan {
-  int k0, kend, npb, nw, nb;
-  int wins[4];
-};
-
-__device__ __forceinline__ BlockPlan make_block_plan(const AttnArgs& a, int P, int split, int rho0,
-                                                     int rho1) {
-  BlockPlan bp;
-  bp.k0 = split * a.keys_per_split;
-  bp.kend = min(P, bp.k0 + a.keys_per_split);
-  bp.npb = bp.kend > bp.k0 ? (bp.kend - bp.k0 + 127) / 128 : 0;
-  bp.nw = 0;
-  if (split == a.nsplit - 1) {
-    bp.wins[bp.nw++] = 0;                       // drafts D_1..D_k (k <= 16) live in window 0
-    if (a.k > 0 && rho1 - 1 >= a.k) {           // the tile holds mask-slot rows
-      const int jlo = (max(rho0, a.k) - a.k) / a.k + 1;
-      const int jhi = (rho1 - 1 - a.k) / a.k + 1;
-      const int lo = a.k + (jlo - 1) * a.k, hi = a.k + jhi * a.k;
-      for (int w = lo / 128; w <= (hi - 1) / 128 && bp.nw < 4; ++w)
-        if (w != 0) bp.wins[bp.nw++] = w;
-    }
-  }
-  bp.nb = bp.npb + bp.nw;
-  return bp;
-}
-
-__device__ __forceinline__ bool page_ok(int page, int num_pages) { return page >= 0 && page < num_pages; }
+using namespace tc05;
 
 // ------------------------------------------------------------------ the kernel
 // 18 warps: two SMSPs host five of them, so a thread may hold at most
@@ -873,6 +744,7 @@ cudaError_t set_smem_attr() {
 }  // namespace
 
 void set_starve_loads(int on) { g_starve_loads = on != 0; }
+int tc05_starve_loads() { return g_starve_loads; }
 
 #ifdef TIDAR_TRACE
 extern "C" int tidar_trace_read(void* dst, size_t bytes) {

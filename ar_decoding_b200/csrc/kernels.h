@@ -46,8 +46,14 @@ cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s);
 // draft-row append; with part_o set it writes split partials instead and
 // launch_finalize merges and appends.
 int tc05_resident_clusters(int ns);
+// Tensor-core kernel with two 128-row query tiles per CTA sharing each staged
+// K/V block (bf16, D 128, page 64), for query blocks of more than one tile per
+// KV head.  Split merge and append as launch_attn_tc05.
+cudaError_t launch_attn_pair(const AttnArgs& a, cudaStream_t s);
+int pair_resident_clusters(int ns);
 // Test hook: launches issue no K/V copies (their bounded waits run out).
 void set_starve_loads(int on);
+int tc05_starve_loads();
 // Split merge (when nsplit > 1) and the draft-row append, in one launch
 // (CUDA-core path).
 cudaError_t launch_finalize(const AttnArgs& a, cudaStream_t s);
@@ -111,5 +117,34 @@ struct ReserveArgs {
 constexpr int kReserveMaxBatch = 65536;
 bool reserve_batch_ok(int B);
 cudaError_t launch_reserve(const ReserveArgs& a, cudaStream_t s);
+
+// Projections on either side of the step attention (tcgen05 GEMM, weights
+// [N][K] bf16 as the A operand, token rows [T][K] bf16 as B).  mode 0: y
+// [T][N] bf16.  mode 1: the query/key/value projection of the R rows of each
+// sequence (T = B R, N = (Hq + 2 Hkv) 128), rotary embedding of queries and
+// keys at their zone positions, outputs q / k_blk / v_blk.
+struct LinearArgs {
+  int T, K, N, mode;
+  const void* x;
+  const void* w;
+  void* y;
+  void* q;
+  void* k_blk;
+  void* v_blk;
+  const int32_t* seq_lens;
+  int Hq, Hkv, R, k, max_prefix;
+  double log2_base;
+  unsigned int* err;
+};
+struct LinearPlan {
+  bool ok;
+  int nt, nsub, tiles, stages, ksplit;
+  uint32_t stage_bytes;
+  size_t smem;
+};
+// Tile plan of one projection: ok is false for shapes the kernel does not
+// take (K not a multiple of 64, N not a multiple of 128).
+LinearPlan plan_linear(int T, int K, int N);
+cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s);
 
 }  // namespace tidar

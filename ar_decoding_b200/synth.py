@@ -312,6 +312,25 @@ def make_loop(cfg: StepConfig, steps: int, mode: str = "greedy"):
     return attn, ver
 
 
+D_MODEL = {"tiny": 128, "1.5B-class": 1536, "8B-class": 4096}
+
+
+def make_layer(cfg: StepConfig, d_model: int | None = None, device="cpu"):
+    """Inputs of the layer-level step: the step rows' hidden states x
+    [B][R][d_model] ~ N(0,1), the projection weights w_qkv [(Hq + 2 Hkv) D]
+    [d_model] ~ N(0, 1/d_model) (queries, then keys, then values; unit-variance
+    q, k, v) and w_o [d_model][Hq D] ~ N(0, 1/(Hq D)); bf16, random (no
+    trained weights).  d_model defaults to the model class's hidden size
+    (4096 for 8B-class heads, 1536 for 1.5B-class)."""
+    dm = d_model if d_model is not None else D_MODEL.get(cfg.name, 4096)
+    gen = torch.Generator(device=device).manual_seed(cfg.seed * 7 + 11)
+    N = (cfg.Hq + 2 * cfg.Hkv) * cfg.D
+    x = _randn((cfg.B, cfg.R, dm), gen, torch.bfloat16, device)
+    w_qkv = _randn((N, dm), gen, torch.bfloat16, device, std=dm ** -0.5)
+    w_o = _randn((dm, cfg.Hq * cfg.D), gen, torch.bfloat16, device, std=(cfg.Hq * cfg.D) ** -0.5)
+    return dict(x=x, w_qkv=w_qkv, w_o=w_o, d_model=dm)
+
+
 def prev_accept_counts(cfg: StepConfig) -> torch.Tensor:
     """Previous-step accept counts, uniform on 0..k (serving workload)."""
     gen = torch.Generator().manual_seed(cfg.seed * 7 + 5)

@@ -67,13 +67,15 @@ def parse_args():
     ap.add_argument("--prefix", type=int, default=8192)
     ap.add_argument("--no-sweep", action="store_true", help="skip the k sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc05", "dec"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc05", "dec", "pair"])
     ap.add_argument("--no-loop", action="store_true", help="skip the chained decode-loop timing")
     ap.add_argument("--loop-chain", type=int, default=8,
                     help="steps chained per sequence in the decode-loop graph")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads (serving batch, long-context corners, "
                          "1.5B-class, tiny) reported under extra_configs")
+    ap.add_argument("--no-layer", action="store_true",
+                    help="skip the layer-level k sweep (projections + attention)")
     ap.add_argument("--no-cpu-sweep", action="store_true",
                     help="reference arm: skip the per-workload oracle timings (cpu_sweep)")
     return ap.parse_args()
@@ -122,7 +124,7 @@ def reduce_sum(x: float, world: int) -> float:
     return float(t.item())
 
 
-PATH_NAMES = {1: "simt", 2: "tc05", 3: "dec"}
+PATH_NAMES = {1: "simt", 2: "tc05", 3: "dec", 4: "pair"}
 
 
 def workload(k: int, prefix: int, rank: int = 0):
@@ -385,7 +387,119 @@ class Loop:
         return us, tokens
 
 
-KERNEL_SRC = {2: "attn_tc05.cu", 3: "attn_dec.cu"}
+class LayerStep:
+    """The layer-level step (query/key/value projection with the rotary
+    embedding, step attention with the draft append, output projection) on
+    `copies` independent instances, each with its own random weights and
+    cache, so neither the weights (84 MB at 8B-class sizes) nor the KV cache of
+    a copy are in L2 when its turn comes."""
+
+    def __init__(self, cfg, copies):
+        import ar_decoding_b200 as tidar
+        from ar_decoding_b200 import synth
+        self.tidar, self.cfg = tidar, cfg
+        dev = torch.device("cuda")
+        self.copies = []
+        for c in range(copies):
+            cc = synth.StepConfig(**{**cfg.__dict__, "seed": cfg.seed + 23 * c})
+            lay = synth.make_layer(cc, device=dev)
+            self.copies.append(dict(cache=synth.make_cache(cc, device=dev), **lay))
+        c0 = self.copies[0]
+        self.dm = c0["d_model"]
+        self.max_prefix = max(cfg.prefix)
+        self.desc = tidar._layer_desc(c0["x"], cfg.k, cfg.Hq, cfg.Hkv, self.max_prefix)
+        need = tidar.layer_step_workspace_bytes(self.desc, self.dm)
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        B, R = cfg.B, cfg.R
+        self.y = torch.empty((B, R, self.dm), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, R, cfg.Hq), dtype=torch.float32, device=dev)
+        self.qkv_out = (torch.empty((B, R, cfg.Hq, 128), dtype=torch.bfloat16, device=dev),
+                        torch.empty((B, R, cfg.Hkv, 128), dtype=torch.bfloat16, device=dev),
+                        torch.empty((B, R, cfg.Hkv, 128), dtype=torch.bfloat16, device=dev))
+        self.attn_out = torch.empty((B, R, cfg.Hq, 128), dtype=torch.bfloat16, device=dev)
+
+    def layer(self, i):
+        c, cfg = self.copies[i], self.cfg
+        self.tidar.layer_step(c["x"], c["w_qkv"], c["w_o"], c["cache"], cfg.k, cfg.Hq, cfg.Hkv,
+                              max_prefix_len=self.max_prefix, out=self.y, lse=self.lse,
+                              workspace=self.ws)
+
+    def qkv(self, i):
+        c, cfg = self.copies[i], self.cfg
+        self.tidar.qkv_rope(c["x"], c["w_qkv"], c["cache"]["seq_lens"], cfg.k, cfg.Hq, cfg.Hkv,
+                            max_prefix_len=self.max_prefix, out=self.qkv_out)
+
+    def oproj(self, i):
+        self.tidar.linear(self.attn_out, self.copies[i]["w_o"], out=self.y)
+
+    def time(self, fn, reps):
+        """Average device µs of fn over all copies back to back in one graph."""
+        n = len(self.copies)
+        for i in range(n):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                fn(i)
+        stream = torch.cuda.current_stream()
+        g.replay(); g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / (reps * n)
+
+
+def layer_sweep(hbm_peak, tc_peak, world, ks=(0, 4, 8, 16), reps=5):
+    """Layer-level step at 8B-class sizes (d_model 4096, 32 q / 8 kv heads,
+    prefix 8192) for each k: the whole layer and its projections, with the
+    projections' algorithmic bytes (weights + activations) and flops."""
+    from ar_decoding_b200 import synth
+    out = []
+    for k in ks:
+        cfg = synth.class_8b(k=k)
+        dm = synth.D_MODEL["8B-class"]
+        T = cfg.B * cfg.R
+        nqkv, no = (cfg.Hq + 2 * cfg.Hkv) * 128, dm
+        w_bytes = (nqkv * dm + no * cfg.Hq * 128) * 2
+        per_copy = w_bytes + algorithmic(cfg)[0]
+        ls = LayerStep(cfg, max(3, math.ceil(3 * L2_BYTES / per_copy)))
+        lay_us = reduce_max(ls.time(ls.layer, reps), world)
+        qkv_us = reduce_max(ls.time(ls.qkv, reps), world)
+        o_us = reduce_max(ls.time(ls.oproj, reps), world)
+        qkv_b = nqkv * dm * 2 + T * dm * 2 + T * nqkv * 2
+        o_b = no * cfg.Hq * 128 * 2 + T * cfg.Hq * 128 * 2 + T * no * 2
+        qkv_f, o_f = 2 * T * nqkv * dm, 2 * T * no * cfg.Hq * 128
+        a_b, a_f = algorithmic(cfg)
+
+        def frac(b, f, us):
+            return max(b / (hbm_peak * 1e9), f / (tc_peak * 1e12)) / (us * 1e-6)
+        out.append({"k": k, "rows": T, "d_model": dm, "copies": len(ls.copies),
+                    "layer_us": lay_us, "qkv_rope_us": qkv_us, "o_proj_us": o_us,
+                    "weight_bytes": w_bytes,
+                    "qkv_rope_gbs": qkv_b / (qkv_us * 1e-6) / 1e9,
+                    "qkv_rope_tflops": qkv_f / (qkv_us * 1e-6) / 1e12,
+                    "qkv_rope_roofline_frac": frac(qkv_b, qkv_f, qkv_us),
+                    "o_proj_gbs": o_b / (o_us * 1e-6) / 1e9,
+                    "o_proj_tflops": o_f / (o_us * 1e-6) / 1e12,
+                    "o_proj_roofline_frac": frac(o_b, o_f, o_us),
+                    "layer_roofline_us": (max((qkv_b) / (hbm_peak * 1e9), qkv_f / (tc_peak * 1e12)) +
+                                          max(a_b / (hbm_peak * 1e9), a_f / (tc_peak * 1e12)) +
+                                          max(o_b / (hbm_peak * 1e9), o_f / (tc_peak * 1e12))) * 1e6})
+        del ls
+        torch.cuda.empty_cache()
+    base = out[0]["layer_us"] if out else None
+    for r in out:
+        r["layer_vs_k0"] = r["layer_us"] / base if base else None
+    return out
+
+
+KERNEL_SRC = {2: "attn_tc05.cu", 3: "attn_dec.cu", 4: "attn_pair.cu"}
 
 
 def measured_traffic(k: int, path_id: int):
@@ -752,6 +866,10 @@ def run_ours(args, rank, world, local):
             del s2
             torch.cuda.empty_cache()
 
+    layer = None
+    if not args.no_layer:
+        layer = layer_sweep(hbm_peak, tc_peak, world)
+
     loop = None
     if not args.no_loop:
         loop = {}
@@ -796,7 +914,8 @@ def run_ours(args, rank, world, local):
             "attn_call_us": mean_attn, "attn_us": kern_us, "attn_launches": st.attn_launches,
             "hbm_gbs_attn": bytes_ / attn_s / 1e9,
             "hbm_gbs_all_gpus": agg_gbs,
-            "roofline": {"kernel": {2: "attn_tc05_kernel", 3: "attn_dec_kernel"}.get(st.path_id, "tidar_step_attn"),
+            "roofline": {"kernel": {2: "attn_tc05_kernel", 3: "attn_dec_kernel",
+                                    4: "attn_pair_kernel"}.get(st.path_id, "tidar_step_attn"),
                          "bound": bound, "achieved": achieved,
                          "peak": peak, "unit": unit, "frac": achieved / peak,
                          "peak_source": peak_src, "peak_kind": "burst",
@@ -805,6 +924,7 @@ def run_ours(args, rank, world, local):
                          "roofline_frac_max_of_both": max(t_mem, t_tc) / attn_s},
             "k_sweep": sweep,
             "extra_configs": extra,
+            "layer_sweep": layer,
             "decode_loop": loop,
             "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

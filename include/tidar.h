@@ -76,13 +76,16 @@ typedef enum { TIDAR_GREEDY = 0, TIDAR_REJECTION = 1 } tidar_accept_mode;
 /* Kernel family for the step attention.  AUTO picks, for bf16, head_dim 128,
  * page 64: the warp-MMA decode kernel (DEC) when the query block packs into at
  * most 16 rows per KV head (R * G <= 16, e.g. plain decode k = 0), else the
- * tcgen05/TMEM tensor-core kernel (TC05); the CUDA-core kernel (SIMT)
- * otherwise.  Asking for DEC with R * G > 16 returns TIDAR_ERR_UNSUPPORTED. */
+ * tcgen05/TMEM tensor-core kernel with one 128-row query tile per CTA (TC05);
+ * the CUDA-core kernel (SIMT) otherwise.  PAIR is the tensor-core kernel with
+ * two query tiles per CTA sharing each staged K/V block (same inputs as
+ * TC05).  Asking for DEC with R * G > 16 returns TIDAR_ERR_UNSUPPORTED. */
 typedef enum {
   TIDAR_PATH_AUTO = 0,
   TIDAR_PATH_SIMT = 1,
   TIDAR_PATH_TC05 = 2,
-  TIDAR_PATH_DEC = 3
+  TIDAR_PATH_DEC = 3,
+  TIDAR_PATH_PAIR = 4
 } tidar_attn_path;
 
 /* Bits of the device error word. */
@@ -158,7 +161,7 @@ tidar_status tidar_step_attn(const tidar_step_desc* desc, const tidar_kv_cache* 
                              tidar_stream_t stream);
 
 /* The launch plan the library would use: kernel family (1 SIMT, 2 TC05,
- * 3 DEC) and number of KV splits.  Host only; with a GPU present the first
+ * 3 DEC, 4 PAIR) and number of KV splits.  Host only; with a GPU present the first
  * call per device queries its SM count and cluster occupancy. */
 tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, int32_t* splits);
 
@@ -333,6 +336,61 @@ typedef struct {
 tidar_status tidar_reserve(const tidar_step_desc* desc, const tidar_kv_cache* cache,
                            const tidar_page_pool* pool, const int32_t* returned_pages,
                            const int32_t* num_returned, tidar_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Layer-level step: the projections on either side of the step attention.
+ * [MS] §2 (one forward pass of the model over the three zones); [EN] section
+ * "為什麼 GPU 在 AR 推論時是閒置的" (each AR decode step reloads every weight,
+ * so a memory-bound step leaves the compute units idle); [NDfr] paragraph on
+ * the masking puzzle (the extra blocks cost a small constant factor on that
+ * idle capacity) and [FG] abstract ("free token slots").  Weights are bf16
+ * rows of their output features (a linear layer y = x w^T); the library
+ * computes in fp32 and stores bf16.  The weights here are the caller's
+ * (random ones in this repository's tests and benchmark).
+ *
+ * tidar_linear: y [rows][out_features] = x [rows][in_features] . w^T with
+ *   w [out_features][in_features].  dtype must be TIDAR_BF16, in_features a
+ *   multiple of 64 and out_features a multiple of 128 (else
+ *   TIDAR_ERR_UNSUPPORTED); x, w, y 16-byte aligned.  rows >= 0.
+ *
+ * tidar_qkv_rope: the query/key/value projection of the R step rows of each
+ *   sequence and the rotary embedding at their zone positions.
+ *   x      [B][R][d_model] bf16 hidden states of the step rows (row order as
+ *          tidar_step_attn: drafts, then mask blocks)
+ *   w_qkv  [(Hq + 2 Hkv) D][d_model] bf16: query features of head h at rows
+ *          [h D, h D + D), then the Hkv key heads, then the Hkv value heads
+ *   seq_lens [B] int32 (device): P_b, which places the rows:
+ *          draft d_r at position P_b + r - 1, slot s of mask block j at
+ *          P_b + j + s - 1 (where t* and the next drafts land once j drafts
+ *          are accepted), the single row of k = 0 at P_b
+ *   queries and keys are rotated pairwise (dims f and f + D/2) by the angle
+ *   position * rope_base^(-2f/D) (formed in fp64); values are not rotated.
+ *   q [B][R][Hq][D], k_blk / v_blk [B][R][Hkv][D]: tidar_step_attn's inputs.
+ *   Needs dtype TIDAR_BF16, head_dim 128, d_model a multiple of 64
+ *   (TIDAR_ERR_UNSUPPORTED otherwise), rope_base > 1.  Device error BAD_LEN
+ *   (seq_lens[b] outside 0..max_prefix_len: position P_b = 0 is used).
+ *
+ * tidar_layer_step: tidar_qkv_rope, tidar_step_attn (which also appends the
+ *   drafts' rotated K/V to the cache) and the output projection
+ *   y [B][R][d_model] = attn_out . w_o^T with w_o [d_model][Hq D], as one
+ *   call.  lse_out as tidar_step_attn's.  workspace: at least
+ *   tidar_layer_step_workspace_bytes(desc, d_model) bytes, 256-byte aligned,
+ *   holding q, k_blk, v_blk, the attention output and the attention's own
+ *   workspace.  d_model must also be a multiple of 128.
+ * Device errors: those of the calls it makes; TIMEOUT if a bounded wait in a
+ * projection ran out.
+ * ------------------------------------------------------------------------- */
+tidar_status tidar_linear(int32_t rows, int32_t out_features, int32_t in_features,
+                          tidar_dtype dtype, const void* x, const void* w, void* y,
+                          tidar_stream_t stream);
+tidar_status tidar_qkv_rope(const tidar_step_desc* desc, int32_t d_model, const void* x,
+                            const void* w_qkv, const int32_t* seq_lens, float rope_base,
+                            void* q, void* k_blk, void* v_blk, tidar_stream_t stream);
+size_t tidar_layer_step_workspace_bytes(const tidar_step_desc* desc, int32_t d_model);
+tidar_status tidar_layer_step(const tidar_step_desc* desc, const tidar_kv_cache* cache,
+                              int32_t d_model, const void* x, const void* w_qkv,
+                              const void* w_o, float rope_base, void* y, float* lse_out,
+                              void* workspace, size_t workspace_bytes, tidar_stream_t stream);
 
 /* Synchronises `stream`, reads and clears this device's error word.  Returns
  * TIDAR_ERR_TIMEOUT if the timeout bit was set, TIDAR_ERR_DEVICE for any other

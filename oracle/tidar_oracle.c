@@ -627,14 +627,18 @@ int tidar_oracle_rope(int rows, int H, int D, double base, const int64_t* pos, c
  * weight rows are its outputs), fp64 sums in index order. */
 int tidar_oracle_linear(int M, int N, int K, const void* x, int x_dtype, const void* w,
                         int w_dtype, double* y) {
-  int m, n, kk;
+  int64_t mn;
   if (M < 0 || N < 0 || K < 0) return ORACLE_ERR_ARG;
-  for (m = 0; m < M; ++m)
-    for (n = 0; n < N; ++n) {
-      double acc = 0.0;
-      for (kk = 0; kk < K; ++kk)
-        acc += elem(x, (int64_t)m * K + kk, x_dtype) * elem(w, (int64_t)n * K + kk, w_dtype);
-      y[(int64_t)m * N + n] = acc;
-    }
+  /* each output is its own index-order sum; the outputs are independent, so
+     they are spread over the host's cores (the arithmetic does not change) */
+#pragma omp parallel for schedule(static)
+  for (mn = 0; mn < (int64_t)M * N; ++mn) {
+    const int64_t m = mn / N, n = mn % N;
+    int kk;
+    double acc = 0.0;
+    for (kk = 0; kk < K; ++kk)
+      acc += elem(x, m * K + kk, x_dtype) * elem(w, n * K + kk, w_dtype);
+    y[m * N + n] = acc;
+  }
   return ORACLE_OK;
 }

@@ -17,7 +17,7 @@ from gpu_harness import (compare_attention, oracle_attention, run_attention, sam
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["simt", "tc05", "dec"]
+PATHS = ["simt", "tc05", "dec", "pair"]
 
 
 def _tc05_ok(cfg):
@@ -31,7 +31,7 @@ def _dec_ok(cfg):
 def _supported(cfg, path):
     # the tensor-core kernel takes bf16, head_dim 128, page 64; the warp-MMA
     # decode kernel in addition at most 16 packed query rows per KV head
-    return {"tc05": _tc05_ok, "dec": _dec_ok}.get(path, lambda c: True)(cfg)
+    return {"tc05": _tc05_ok, "pair": _tc05_ok, "dec": _dec_ok}.get(path, lambda c: True)(cfg)
 
 
 def _check_full(oracle_mod, cfg, path):
@@ -150,7 +150,7 @@ class _ForcedPartials:
         tidar.debug_set(tidar.DEBUG_FORCE_SPLIT_PARTIALS, 0)
 
 
-@pytest.mark.parametrize("path", ["tc05", "dec"])
+@pytest.mark.parametrize("path", ["tc05", "dec", "pair"])
 @pytest.mark.parametrize("merge", ["auto", "partials"])
 def test_8b_class_k0_full_every_split_merged(oracle_mod, merge, path):
     # k = 0: one query row per head, the prefix cut into many splits; every
@@ -190,15 +190,15 @@ def test_auto_picks_the_decode_kernel_for_thin_blocks():
     assert tidar.plan(tidar.make_desc(q(272, 32), kb(272, 8), cache16, 16, 8192))[0] == tidar.PATH_TC05
 
 
-@pytest.mark.parametrize("path", PATHS + ["tc05-partials"])
+@pytest.mark.parametrize("path", PATHS + ["tc05-partials", "pair-partials"])
 def test_splits_past_a_short_sequence(oracle_mod, path):
     # sequence 1 is far shorter than sequence 0: most of its key splits hold no
     # prefix key and contribute an empty partial to the merge
     cfg = synth.StepConfig("ragged-splits", B=2, Hq=8, Hkv=2, D=128, k=4, prefix=(4096, 300),
                            dtype="bf16", seed=57)
-    if path == "tc05-partials":
+    if path.endswith("-partials"):
         with _ForcedPartials():
-            _check_full(oracle_mod, cfg, "tc05")
+            _check_full(oracle_mod, cfg, path.split("-")[0])
     else:
         _check_full(oracle_mod, cfg, path)
 

@@ -58,6 +58,10 @@ class PagePool(ctypes.Structure):
                 ("capacity", ctypes.c_int32)]
 
 
+class Sampling(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_float), ("top_p", ctypes.c_float)]
+
+
 class KVCacheDesc(ctypes.Structure):
     _fields_ = [("k_pages", ctypes.c_void_p), ("v_pages", ctypes.c_void_p),
                 ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
@@ -105,6 +109,13 @@ def lib():
         L.tidar_last_cuda_error.restype = ctypes.c_char_p
         L.tidar_debug_set.argtypes = [ctypes.c_int, I]
         L.tidar_debug_set.restype = ctypes.c_int
+        L.tidar_verify_sampled_workspace_bytes.argtypes = [I, I, I, ctypes.c_int]
+        L.tidar_verify_sampled_workspace_bytes.restype = S
+        L.tidar_verify_sampled.argtypes = [I, I, I, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P,
+                                           P, P, P, P, P, P, S, P]
+        L.tidar_verify_sampled.restype = ctypes.c_int
+        L.tidar_sample_drafts.argtypes = [I, I, I, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P]
+        L.tidar_sample_drafts.restype = ctypes.c_int
         L.tidar_linear.argtypes = [I, I, I, ctypes.c_int, P, P, P, P]
         L.tidar_linear.restype = ctypes.c_int
         L.tidar_qkv_rope.argtypes = [P, I, P, P, P, ctypes.c_float, P, P, P, P]
@@ -386,6 +397,64 @@ def verify_blockq(logits, drafts, k, prev_block_logits, draft_block, uniforms, *
                                    workspace.numel(), _stream_handle(stream))
     _check(st, "tidar_verify_blockq")
     return outputs
+
+
+def verify_sampled(logits, drafts, k, mode="rejection", *, temperature=1.0, top_p=1.0,
+                   draft_logits=None, prev_block_logits=None, draft_block=None, uniforms=None,
+                   block_guesses=None, outputs=None, workspace=None, stream=None):
+    """Verification with the sampling transform (temperature, nucleus top_p)
+    applied to p and q.  q comes from draft_logits [B][k-1][V] or, with
+    prev_block_logits [B][k][k][V] and draft_block [B], in place from the
+    previous step's mask blocks.  Returns the same dict as ``verify``."""
+    m = mode if isinstance(mode, int) else {"greedy": GREEDY, "rejection": REJECTION}[mode]
+    _dev(logits, "logits")
+    B, n, V = logits.shape
+    dev = logits.device
+    if outputs is None:
+        outputs = dict(accept_count=torch.empty(B, dtype=torch.int32, device=dev),
+                       out_tokens=torch.empty((B, n), dtype=torch.int32, device=dev),
+                       next_drafts=torch.empty((B, max(k, 1)), dtype=torch.int32, device=dev),
+                       selected_block=torch.empty(B, dtype=torch.int32, device=dev))
+    need = int(lib().tidar_verify_sampled_workspace_bytes(B, k, V, m))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check_verify_args(logits, drafts, draft_logits, uniforms, block_guesses, outputs, workspace)
+    _devopt(prev_block_logits, "prev_block_logits", logits.dtype, dev)
+    _devopt(draft_block, "draft_block", torch.int32, dev)
+    sp = Sampling(temperature=float(temperature), top_p=float(top_p))
+    st = lib().tidar_verify_sampled(B, k, V, _dtype_code(logits), m, ctypes.byref(sp), _ptr(logits),
+                                    _ptr(drafts), _ptr(draft_logits), _ptr(prev_block_logits),
+                                    _ptr(draft_block), _ptr(uniforms), _ptr(block_guesses),
+                                    _ptr(outputs["accept_count"]), _ptr(outputs["out_tokens"]),
+                                    _ptr(outputs["next_drafts"]) if k > 0 else None,
+                                    _ptr(outputs["selected_block"]), _ptr(workspace),
+                                    workspace.numel(), _stream_handle(stream))
+    _check(st, "tidar_verify_sampled")
+    return outputs
+
+
+def sample_drafts(block_logits, selected_block, k, mode="rejection", *, temperature=1.0, top_p=1.0,
+                  uniforms=None, next_drafts=None, stream=None):
+    """The next drafts from slots 2..k of each sequence's selected mask block
+    (block_logits [B][k][k][V], selected_block [B] int32); writes entries
+    1..k-1 of next_drafts [B][k] (entry 0, t*, is left alone).  Returns it."""
+    m = mode if isinstance(mode, int) else {"greedy": GREEDY, "rejection": REJECTION}[mode]
+    _dev(block_logits, "block_logits")
+    dev = block_logits.device
+    B, kk, k2, V = block_logits.shape
+    if kk != k or k2 != k:
+        raise ValueError(f"block_logits is {tuple(block_logits.shape)}, k = {k}")
+    _dev(selected_block, "selected_block", torch.int32, dev)
+    _devopt(uniforms, "uniforms", torch.float32, dev)
+    if next_drafts is None:
+        next_drafts = torch.full((B, max(k, 1)), -1, dtype=torch.int32, device=dev)
+    _dev(next_drafts, "next_drafts", torch.int32, dev)
+    sp = Sampling(temperature=float(temperature), top_p=float(top_p))
+    st = lib().tidar_sample_drafts(B, k, V, _dtype_code(block_logits), m, ctypes.byref(sp),
+                                   _ptr(block_logits), _ptr(selected_block), _ptr(uniforms),
+                                   _ptr(next_drafts), _stream_handle(stream))
+    _check(st, "tidar_sample_drafts")
+    return next_drafts
 
 
 VERIFY_NOALLOC_MAX_SCRATCH_BYTES = 4 << 20

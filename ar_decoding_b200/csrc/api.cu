@@ -388,6 +388,81 @@ tidar_status tidar_verify_blockq(int32_t batch, int32_t k, int32_t vocab, tidar_
                        selected_block, workspace, workspace_bytes, stream);
 }
 
+size_t tidar_verify_sampled_workspace_bytes(int32_t batch, int32_t k, int32_t vocab,
+                                            tidar_accept_mode mode) {
+  if (batch <= 0 || k < 0 || k > 16 || vocab <= 0) return 0;
+  if (mode == TIDAR_GREEDY) return 0;
+  return align256(tidar::sampled_verify_workspace_bytes(batch, k));
+}
+
+static bool sampling_ok(const tidar_sampling* sp) {
+  return sp && sp->temperature > 0.f && sp->top_p > 0.f;   // NaN fails both
+}
+
+tidar_status tidar_verify_sampled(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                                  tidar_accept_mode mode, const tidar_sampling* sampling,
+                                  const void* logits, const int32_t* drafts, const void* draft_logits,
+                                  const void* prev_block_logits, const int32_t* draft_block,
+                                  const float* uniforms, const int32_t* block_guesses,
+                                  int32_t* accept_count, int32_t* out_tokens, int32_t* next_drafts,
+                                  int32_t* selected_block, void* workspace, size_t workspace_bytes,
+                                  tidar_stream_t stream) {
+  if (!sampling_ok(sampling)) return TIDAR_ERR_INVALID_ARG;
+  if (mode == TIDAR_GREEDY)
+    return verify_launch(batch, k, vocab, dtype, mode, logits, drafts, nullptr, nullptr, uniforms,
+                         block_guesses, accept_count, out_tokens, next_drafts, selected_block, workspace,
+                         workspace_bytes, stream);
+  if (batch < 0 || k < 0 || vocab <= 0) return TIDAR_ERR_INVALID_ARG;
+  if (k > 16) return TIDAR_ERR_UNSUPPORTED;
+  if (dtype != TIDAR_F32 && dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
+  if (mode != TIDAR_REJECTION) return TIDAR_ERR_INVALID_ARG;
+  if (batch == 0) return TIDAR_OK;
+  if (batch > 65535) return TIDAR_ERR_UNSUPPORTED;
+  if (!logits || !accept_count || !out_tokens || !uniforms) return TIDAR_ERR_INVALID_ARG;
+  const bool blockq = prev_block_logits != nullptr;
+  if (k > 1 && (!drafts || (!blockq && !draft_logits) || (blockq && !draft_block)))
+    return TIDAR_ERR_INVALID_ARG;
+  const size_t need = tidar_verify_sampled_workspace_bytes(batch, k, vocab, mode);
+  if (workspace_bytes < need || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return TIDAR_ERR_INVALID_ARG;
+  tidar::VerifyArgs a{};
+  a.B = batch; a.k = k; a.n = k > 0 ? k : 1; a.V = vocab; a.bf16 = dtype == TIDAR_BF16; a.mode = mode;
+  a.logits = logits; a.drafts = drafts; a.uniforms = uniforms;
+  a.draft_logits = k > 1 ? (blockq ? prev_block_logits : draft_logits) : nullptr;
+  a.draft_block = (k > 1 && blockq) ? draft_block : nullptr;
+  a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;
+  a.next_drafts = next_drafts; a.selected_block = selected_block; a.workspace = workspace;
+  tidar_status st = error_word(&a.err);
+  if (st != TIDAR_OK) return st;
+  const cudaError_t e = tidar::launch_sampled_verify(a, (double)sampling->temperature,
+                                                     (double)sampling->top_p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
+tidar_status tidar_sample_drafts(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                                 tidar_accept_mode mode, const tidar_sampling* sampling,
+                                 const void* block_logits, const int32_t* selected_block,
+                                 const float* uniforms, int32_t* next_drafts, tidar_stream_t stream) {
+  if (!sampling_ok(sampling)) return TIDAR_ERR_INVALID_ARG;
+  if (batch < 0 || k < 0 || vocab <= 0) return TIDAR_ERR_INVALID_ARG;
+  if (k > 16) return TIDAR_ERR_UNSUPPORTED;
+  if (dtype != TIDAR_F32 && dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
+  if (mode != TIDAR_GREEDY && mode != TIDAR_REJECTION) return TIDAR_ERR_INVALID_ARG;
+  if (batch == 0 || k < 2) return TIDAR_OK;
+  if (batch > 65535) return TIDAR_ERR_UNSUPPORTED;
+  if (!block_logits || !selected_block || !next_drafts || (mode == TIDAR_REJECTION && !uniforms))
+    return TIDAR_ERR_INVALID_ARG;
+  unsigned int* err = nullptr;
+  tidar_status st = error_word(&err);
+  if (st != TIDAR_OK) return st;
+  const cudaError_t e = tidar::launch_sample_drafts(
+      batch, k, vocab, dtype == TIDAR_BF16, mode, (double)sampling->temperature, (double)sampling->top_p,
+      block_logits, selected_block, uniforms, next_drafts, err, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
 tidar_status tidar_commit(const tidar_step_desc* d, const tidar_kv_cache* c,
                           const int32_t* accept_count, int32_t* released_pages,
                           int32_t* num_released, tidar_stream_t stream) {

@@ -93,6 +93,23 @@ __device__ __forceinline__ uint32_t pcol_o(int t) { return 256u + 128u * (uint32
 constexpr uint32_t kPIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kPIdescPV = kPIdescS | (1u << 16);     // B (= V) is MN-major
 
+// Optional timeline of CTA (0, 0, 0) (build with -DTIDAR_TRACE; absent from
+// normal builds): [0] setup, [1] TMEM ready, [16 + 4 i + t] S_t(i) issued,
+// [512 + 4 i + t] PV_t(i) issued, [1024 + 4 i + t] softmax t sees S_t(i),
+// [1536 + 4 i + t] P_t(i) handed over, [2048 + 8 i + ph] warp 0's phases of
+// block i (0 wait done, 1 loaded, 2 max, 3 exps, 4 stored), [2600] epilogue,
+// [2601] end; [4096 + 2 cta] start / end of every CTA.
+#ifdef TIDAR_TRACE
+__device__ unsigned long long g_pair_trace[4096 + 2 * 8192];
+__device__ __forceinline__ bool ptrace_cta() { return blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0; }
+#define PAIR_TRACE(slot) do { if (ptrace_cta() && (slot) < 4096) g_pair_trace[(slot)] = global_ns(); } while (0)
+#define PAIR_TRACE_CTA(w) do { const unsigned c_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+    if (c_ < 8192) g_pair_trace[4096 + 2 * c_ + (w)] = global_ns(); } while (0)
+#else
+#define PAIR_TRACE(slot) do {} while (0)
+#define PAIR_TRACE_CTA(w) do {} while (0)
+#endif
+
 struct PairParams {
   AttnArgs a;
   int rho_per_tile;   // query rows per tile (128 / G)
@@ -128,6 +145,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
   if (threadIdx.x == 0) {
+    PAIR_TRACE_CTA(0);
+    PAIR_TRACE(0);
     *abort_flag = layout_ok ? 0 : 1;
     if (layout_ok) {
       for (int i = 0; i < kPBars; ++i) mbar_init(bar(i), (i == PB_PFULL || i == PB_PFULL + 1) ? 4u : 1u);
@@ -147,6 +166,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   __syncthreads();
   fence_after();
   const uint32_t tmem = layout_ok ? misc[0] : 0u;
+  if (threadIdx.x == 0) PAIR_TRACE(1);
 
   pdl_wait();       // the previous kernel on the stream is complete from here on
   pdl_trigger();
@@ -300,6 +320,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         mma_commit(bar(PB_SFULL + t));
         if (t == ntile - 1) mma_commit(bar(PB_KEMPTY + st));
+        PAIR_TRACE(16 + 4 * min(blk, 120) + t);
         return true;
       };
       for (int t = 0; ok && t < ntile; ++t) ok = issue_s(t, 0);
@@ -315,6 +336,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mma_ts(tmem + pcol_o(t), tmem + pcol_s(t) + 8u * kk, desc_mn_sw128(va + kk * 2048, kPChunk), kPIdescPV,
                    (b2 > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(PB_PVDONE + t));
+          PAIR_TRACE(512 + 4 * min(b2, 120) + t);
           if (t == ntile - 1) mma_commit(bar(PB_VEMPTY + vs));
           if (b2 + 1 < nb && !issue_s(t, b2 + 1)) ok = false;
         }
@@ -337,6 +359,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int b2 = 0; b2 < nb; ++b2) {
         if (!warp_wait_bar(bar(PB_SFULL + t), (uint32_t)(b2 & 1), abort_flag, a.err)) { ok = false; break; }
         fence_after();
+        if (r == 0) PAIR_TRACE(1024 + 4 * min(b2, 120) + t);
+        if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 0);
         int lo_valid = 64, hi_valid = 64, kb = 0;
         const bool window = b2 >= bp.npb;
         if (!window) {
@@ -357,6 +381,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_ld32(trow + pcol_s(t) + 64, *reinterpret_cast<uint32_t(*)[32]>(&x[64]));
         tmem_ld32(trow + pcol_s(t) + 96, *reinterpret_cast<uint32_t(*)[32]>(&x[96]));
         tmem_wait_ld();
+        if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 1);
         if (!full) {
           // invisible keys (zone mask, past the prefix end, unmapped page) get
           // -inf: their probability is 2^-inf = 0
@@ -381,6 +406,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           mx[3] = max3(mx[3], __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
         }
         const float mrow = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+        if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 2);
         const float m_new = fmaxf(m, mrow);
         const bool need = m_new > m + 8.0f;
         const float f_resc = need ? ex2(m - m_new) : 1.0f;  // factor for O and l (m = -inf -> 0)
@@ -397,6 +423,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
           x[c] = cvt_bf16x2(p0, p1);
         }
+        if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 3);
         tmem_st32(trow + pcol_s(t), *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
         tmem_st32(trow + pcol_s(t) + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
         float la, lb, lc, ld;
@@ -448,8 +475,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncwarp();
         if (!__all_sync(0xffffffffu, ok)) { ok = false; }
         if (lane == 0) mbar_arrive(bar(PB_PFULL + t));
+        if (r == 0) PAIR_TRACE(1536 + 4 * min(b2, 120) + t);
+        if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 4);
         if (!ok) break;
       }
+      if (threadIdx.x == 0) PAIR_TRACE(2600);
       // ---- this tile's row of O: wait for the last PV, normalise
       if (ok && nb > 0 && !warp_wait_bar(bar(PB_PVDONE + t), (uint32_t)((nb - 1) & 1), abort_flag, a.err)) ok = false;
       ok = __all_sync(0xffffffffu, ok && !*abort_flag);
@@ -598,6 +628,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   }
 
+  if (threadIdx.x == 0) { PAIR_TRACE(2601); PAIR_TRACE_CTA(1); }
   if (layout_ok && warp == 9) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPTmemCols) : "memory");
@@ -620,6 +651,16 @@ cudaError_t pair_smem_attr() {
 }
 
 }  // namespace
+
+#ifdef TIDAR_TRACE
+extern "C" int tidar_pair_trace_read(void* dst, size_t bytes) {
+  return (int)cudaMemcpyFromSymbol(dst, g_pair_trace, bytes);
+}
+extern "C" int tidar_pair_trace_clear(void) {
+  static unsigned long long zeros[4096 + 2 * 8192];
+  return (int)cudaMemcpyToSymbol(g_pair_trace, zeros, sizeof zeros);
+}
+#endif
 
 cudaError_t launch_attn_pair(const AttnArgs& a, cudaStream_t s) {
   if (!a.bf16 || a.D != 128 || a.page_size != 64 || a.G > 128) return cudaErrorNotSupported;

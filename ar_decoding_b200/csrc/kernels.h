@@ -88,6 +88,15 @@ tidar_status cuda_status(cudaError_t e);
 size_t verify_workspace_bytes(int B, int k, int V, int mode);
 bool verify_grid_ok(int B, int k, int mode);   // launch grid fits (grid.y <= 65535)
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s);
+// Rejection verification under temperature / nucleus truncation: per-row
+// distribution descriptors into a.workspace, then one CTA per sequence.
+size_t sampled_verify_workspace_bytes(int B, int k);
+cudaError_t launch_sampled_verify(const VerifyArgs& a, double temp, double top_p, cudaStream_t s);
+// The next drafts from slots 2..k of each sequence's selected mask block.
+cudaError_t launch_sample_drafts(int B, int k, int V, int bf16, int mode, double temp, double top_p,
+                                 const void* block_logits, const int32_t* selected_block,
+                                 const float* uniforms, int32_t* next_drafts, unsigned int* err,
+                                 cudaStream_t s);
 
 struct CommitArgs {
   int B, Hkv, D, k, n, page_size, elem_bytes, max_pages, num_pages;

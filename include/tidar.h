@@ -267,6 +267,70 @@ tidar_status tidar_verify_noalloc(int32_t batch, int32_t k, int32_t vocab, tidar
                                   tidar_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Sampling controls: verification and the next drafts under a temperature and
+ * a nucleus (top-p) truncation.  The pages fix neither; they speak of sampling
+ * from the AR distribution ([EN] section "TiDAR 在做什麼") and of drafting from
+ * the mask blocks' predictions ([MS] §2; [NDfr] paragraph on betting on every
+ * outcome).  The speculative-sampling rule is exact for any pair (p, q), so the
+ * same transform is applied to the AR rows and to the draft rows:
+ *   temperature T > 0:  p(x) proportional to exp(l(x) / T);
+ *   top_p in (0, 1]:    order the tokens larger logit first, lower index first
+ *                       on equal logits; keep token x iff the probability of
+ *                       the tokens before it is below top_p (the shortest run
+ *                       reaching top_p); renormalise the kept tokens.
+ *                       top_p >= 1 keeps every token.
+ * Probabilities, the cut and the sums are fp64 (the cut is exact up to
+ * summation order: a cut within ~1e-15 of top_p may fall either way).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  float temperature; /* > 0 */
+  float top_p;       /* > 0; >= 1 disables the truncation */
+} tidar_sampling;
+
+/* tidar_verify / tidar_verify_blockq with the transform.
+ *   Greedy mode ignores the transform (the most likely token is always kept
+ *   and T keeps the order) and runs tidar_verify's greedy kernel; draft rows
+ *   and uniforms are not read.
+ *   Rejection mode: draft_logits [B][k-1][V] (q_i in row i-1), or -- when
+ *   prev_block_logits is non-NULL -- q_i read in place from the previous
+ *   step's mask blocks as tidar_verify_blockq does (draft_logits then unused).
+ *   workspace: at least tidar_verify_sampled_workspace_bytes(batch, k, vocab,
+ *   mode) bytes, 256-byte aligned.  Everything else as tidar_verify.
+ * TIDAR_ERR_INVALID_ARG for a NULL `sampling`, T <= 0 or top_p <= 0 (or NaN).
+ */
+size_t tidar_verify_sampled_workspace_bytes(int32_t batch, int32_t k, int32_t vocab,
+                                            tidar_accept_mode mode);
+tidar_status tidar_verify_sampled(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                                  tidar_accept_mode mode, const tidar_sampling* sampling,
+                                  const void* logits, const int32_t* drafts,
+                                  const void* draft_logits, const void* prev_block_logits,
+                                  const int32_t* draft_block, const float* uniforms,
+                                  const int32_t* block_guesses, int32_t* accept_count,
+                                  int32_t* out_tokens, int32_t* next_drafts,
+                                  int32_t* selected_block, void* workspace,
+                                  size_t workspace_bytes, tidar_stream_t stream);
+
+/* The next step's drafts from the selected mask block, on the device.  With
+ * j = selected_block[b] (a value outside 1..k reads block 1 and sets
+ * TIDAR_DEVERR_BAD_COUNT), slot s = 2..k of block j -- row
+ * block_logits[b][j-1][s-1] -- gives next_drafts[b][s-1]:
+ *   TIDAR_GREEDY:    its argmax (lowest index on ties);
+ *   TIDAR_REJECTION: a draw from its transformed distribution, the smallest t
+ *                    with uniforms[b][s-1] * sum(q) < sum_{x<=t} q(x) (index
+ *                    order), so that next step's tidar_verify_sampled /
+ *                    tidar_verify_blockq, reading q from the same rows, sees
+ *                    drafts drawn from q.
+ * next_drafts[b][0] (t*, written by verification) is not touched.  k < 2: no
+ * work.  block_logits [B][k][k][V] dtype, 16-byte aligned; uniforms [B][k]
+ * fp32 in [0,1) (TIDAR_REJECTION only; entry 0 unused).  No workspace.
+ */
+tidar_status tidar_sample_drafts(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                                 tidar_accept_mode mode, const tidar_sampling* sampling,
+                                 const void* block_logits, const int32_t* selected_block,
+                                 const float* uniforms, int32_t* next_drafts,
+                                 tidar_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * KV commit / evict, in place.  [NDfr] paragraph on the three zones (the
  * settled cache is reused, rejected entries are evicted); [MS] "KV Cache" and
  * [FG] abstract (exact KV cache).  Accepted drafts are a prefix of the draft

@@ -66,6 +66,14 @@ def _load():
         lib.tidar_oracle_rope.restype = i
         lib.tidar_oracle_linear.argtypes = [i, i, i, P, i, P, i, P]
         lib.tidar_oracle_linear.restype = i
+        d = ctypes.c_double
+        lib.tidar_oracle_verify_sampled.argtypes = [i, i, i, i, i, d, d, P, P, P, P, P, P, P, P, P,
+                                                    P, P]
+        lib.tidar_oracle_verify_sampled.restype = i
+        lib.tidar_oracle_sample_drafts.argtypes = [i, i, i, i, i, d, d, P, P, P, P, P]
+        lib.tidar_oracle_sample_drafts.restype = i
+        lib.tidar_oracle_dist_row.argtypes = [i, i, d, d, P, P, P]
+        lib.tidar_oracle_dist_row.restype = i
         _lib = lib
     return _lib
 
@@ -130,6 +138,77 @@ def step_attn(q, k_blk, v_blk, k_pages, v_pages, page_table, seq_lens, k, *, sca
     if st != 0:
         raise ValueError(f"oracle step_attn failed with status {st}")
     return out, lse
+
+
+def dist_row(row, temperature=1.0, top_p=1.0):
+    """The sampling transform of one logit row (fp32 or bf16 bits): returns
+    (p [V] fp64, cut margin)."""
+    row = np.ascontiguousarray(row)
+    V = row.shape[0]
+    p = np.zeros(V, np.float64)
+    cm = np.zeros(1, np.float64)
+    st = _load().tidar_oracle_dist_row(V, _dtype_code(row), float(temperature), float(top_p),
+                                       _ptr(row), _ptr(p), _ptr(cm))
+    if st != 0:
+        raise ValueError(f"oracle dist_row failed with status {st}")
+    return p, float(cm[0])
+
+
+def verify_sampled(logits, drafts, k, mode, *, temperature=1.0, top_p=1.0, draft_logits=None,
+                   uniforms=None, block_guesses=None):
+    """tidar_oracle_verify with the sampling transform (temperature, nucleus
+    top_p) applied to p and q.  Returns verify's dict plus margins [B][n] and
+    cut_margins [B] (the smallest nucleus-cut margin the sequence's decisions
+    read; +inf without truncation)."""
+    lib = _load()
+    logits = np.ascontiguousarray(logits)
+    dt = _dtype_code(logits)
+    B, n, V = logits.shape
+    assert n == max(k, 1)
+    drafts = None if drafts is None else np.ascontiguousarray(drafts, dtype=np.int32)
+    if draft_logits is not None:
+        draft_logits = np.ascontiguousarray(draft_logits)
+        assert draft_logits.dtype == logits.dtype
+    if uniforms is not None:
+        uniforms = np.ascontiguousarray(uniforms, dtype=np.float32)
+    if block_guesses is not None:
+        block_guesses = np.ascontiguousarray(block_guesses, dtype=np.int32)
+    acc = np.zeros(B, np.int32)
+    toks = np.zeros((B, n), np.int32)
+    nxt = np.zeros((B, max(k, 1)), np.int32)
+    selb = np.zeros(B, np.int32)
+    marg = np.zeros((B, n), np.float64)
+    cut = np.zeros(B, np.float64)
+    st = lib.tidar_oracle_verify_sampled(B, k, V, dt, mode, float(temperature), float(top_p),
+                                         _ptr(logits), _ptr(drafts), _ptr(draft_logits),
+                                         _ptr(uniforms), _ptr(block_guesses), _ptr(acc), _ptr(toks),
+                                         _ptr(nxt), _ptr(selb), _ptr(marg), _ptr(cut))
+    if st != 0:
+        raise ValueError(f"oracle verify_sampled failed with status {st}")
+    return dict(accept_count=acc, out_tokens=toks, next_drafts=nxt[:, :k], selected_block=selb,
+                margins=marg, cut_margins=cut)
+
+
+def sample_drafts(block_logits, selected_block, k, mode, *, temperature=1.0, top_p=1.0,
+                  uniforms=None, next_drafts=None):
+    """The next drafts from the selected mask block: slot s = 2..k of block
+    selected_block[b] gives next_drafts[b][s-1] (argmax in mode GREEDY, inverse
+    CDF of the transformed slot distribution with uniforms[b][s-1] in mode
+    REJECTION).  Returns (next_drafts [B][k] int32, margins [B][k], status);
+    entry 0 keeps next_drafts' value (or -1)."""
+    lib = _load()
+    bl = np.ascontiguousarray(block_logits)
+    dt = _dtype_code(bl)
+    B, kk, k2, V = bl.shape
+    assert kk == k and k2 == k
+    sb = np.ascontiguousarray(selected_block, dtype=np.int32)
+    u = None if uniforms is None else np.ascontiguousarray(uniforms, dtype=np.float32)
+    out = (np.full((B, k), -1, np.int32) if next_drafts is None
+           else np.array(next_drafts, dtype=np.int32, copy=True))
+    marg = np.zeros((B, k), np.float64)
+    st = lib.tidar_oracle_sample_drafts(B, k, V, dt, mode, float(temperature), float(top_p),
+                                        _ptr(bl), _ptr(sb), _ptr(u), _ptr(out), _ptr(marg))
+    return out, marg, int(st)
 
 
 def append(k_pages, v_pages, page_table, seq_lens, k_blk, v_blk, k):

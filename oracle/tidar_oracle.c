@@ -399,6 +399,245 @@ int tidar_oracle_verify(int B, int k, int V, int dtype, int mode, const void* lo
 }
 
 /*
+ * The sampling transform of a logit row, applied alike to the AR
+ * distribution p and to the draft distribution q.  The pages fix no
+ * temperature or truncation (they speak only of sampling from the AR
+ * distribution, [EN] section "TiDAR 在做什麼", and of drafting from the mask
+ * blocks' marginals, [MS] §2); this is the plainest reading of the usual
+ * sampling controls, and the speculative-sampling rule stays exact for any
+ * pair (p, q) it produces:
+ *   temperature T > 0:   p(x) proportional to exp(l(x) / T);
+ *   nucleus top_p:       order the tokens larger logit first, lower index first
+ *                        among equal logits; keep token x iff the probability
+ *                        of the tokens before it is below top_p (so the kept run
+ *                        is the shortest one reaching top_p); renormalise the
+ *                        kept tokens (sum in index order).  top_p >= 1 keeps
+ *                        every token.
+ * Writes p[0..V-1] (fp64).  cut_margin (may be NULL) receives the distance of
+ * top_p to the nearest cumulative sum around the cut -- min(top_p - mass before
+ * the last kept token, mass through it - top_p) / top_p -- or +inf without
+ * truncation: a decision that close to a tie is fixed by summation order only.
+ */
+typedef struct {
+  double v;
+  int x;
+} oracle_tok;
+
+static int tok_order(const void* a, const void* b) {
+  const oracle_tok* p = (const oracle_tok*)a;
+  const oracle_tok* q = (const oracle_tok*)b;
+  if (p->v > q->v) return -1;
+  if (p->v < q->v) return 1;
+  return p->x < q->x ? -1 : (p->x > q->x ? 1 : 0);
+}
+
+static int dist_row(const void* base, int64_t off, int V, int dtype, double T, double top_p,
+                    double* p, double* cut_margin) {
+  double m = -INFINITY, z = 0.0;
+  int x;
+  if (cut_margin) *cut_margin = INFINITY;
+  for (x = 0; x < V; ++x) { double v = elem(base, off + x, dtype) / T; if (v > m) m = v; }
+  for (x = 0; x < V; ++x) { p[x] = exp(elem(base, off + x, dtype) / T - m); z += p[x]; }
+  for (x = 0; x < V; ++x) p[x] /= z;
+  if (top_p < 1.0) {
+    oracle_tok* t = (oracle_tok*)malloc(sizeof(oracle_tok) * (size_t)V);
+    char* keep = (char*)malloc((size_t)V);
+    double cum = 0.0, before_last = 0.0, through_last = 0.0, s = 0.0;
+    int i;
+    if (!t || !keep) { free(t); free(keep); return ORACLE_ERR_ARG; }
+    for (x = 0; x < V; ++x) { t[x].v = elem(base, off + x, dtype); t[x].x = x; keep[x] = 0; }
+    qsort(t, (size_t)V, sizeof(oracle_tok), tok_order);
+    for (i = 0; i < V; ++i) {
+      if (cum < top_p) {
+        keep[t[i].x] = 1;
+        before_last = cum;
+        through_last = cum + p[t[i].x];
+      }
+      cum += p[t[i].x];
+    }
+    for (x = 0; x < V; ++x) if (keep[x]) s += p[x];
+    for (x = 0; x < V; ++x) p[x] = keep[x] ? p[x] / s : 0.0;
+    if (cut_margin) {
+      double lo = top_p - before_last, hi = through_last - top_p;
+      *cut_margin = (lo < hi ? lo : hi) / top_p;
+    }
+    free(t);
+    free(keep);
+  }
+  return ORACLE_OK;
+}
+
+/* The transformed distribution of one logit row (for the pins in tests/). */
+int tidar_oracle_dist_row(int V, int dtype, double T, double top_p, const void* row, double* p,
+                          double* cut_margin) {
+  if (V <= 0 || !(T > 0.0) || !(top_p > 0.0)) return ORACLE_ERR_ARG;
+  return dist_row(row, 0, V, dtype, T, top_p, p, cut_margin);
+}
+
+/*
+ * Verification with the sampling transform: the algorithm of
+ * tidar_oracle_verify, step by step, with p_i and q_i taken through
+ * dist_row(T, top_p).  Greedy acceptance is unchanged by the transform (the
+ * most likely token is always kept and T > 0 keeps the order), so greedy
+ * ignores T and top_p.  cut_margins [B] (may be NULL) receives, per sequence,
+ * the smallest cut margin of the rows its decisions read (+inf without
+ * truncation).
+ */
+int tidar_oracle_verify_sampled(int B, int k, int V, int dtype, int mode, double T, double top_p,
+                                const void* logits, const int32_t* drafts, const void* draft_logits,
+                                const float* uniforms, const int32_t* block_guesses,
+                                int32_t* accept_count, int32_t* out_tokens, int32_t* next_drafts,
+                                int32_t* selected_block, double* margins, double* cut_margins) {
+  const int n = k > 0 ? k : 1;
+  double *p, *qd, *w;
+  int b;
+  if (B < 0 || k < 0 || V <= 0 || (mode != 0 && mode != 1) || !(T > 0.0) || !(top_p > 0.0))
+    return ORACLE_ERR_ARG;
+  if (k > 1 && !drafts) return ORACLE_ERR_ARG;
+  if (mode == 1 && (!uniforms || (k > 1 && !draft_logits))) return ORACLE_ERR_ARG;
+  p = (double*)malloc(sizeof(double) * V);
+  qd = (double*)malloc(sizeof(double) * V);
+  w = (double*)malloc(sizeof(double) * V);
+  if (!p || !qd || !w) { free(p); free(qd); free(w); return ORACLE_ERR_ARG; }
+
+  for (b = 0; b < B; ++b) {
+    int i, j = 1, x, t_star = 0, e;
+    double cm = INFINITY, c1;
+    if (margins) for (i = 0; i < n; ++i) margins[(int64_t)b * n + i] = INFINITY;
+
+    /* accept scan, left to right */
+    for (i = 1; i <= n - 1; ++i) {
+      int d_next = drafts[(int64_t)b * k + i];   /* d_{i+1} */
+      int64_t lrow = ((int64_t)b * n + (i - 1)) * V;
+      int accept;
+      if (d_next < 0 || d_next >= V) { accept = 0; }
+      else if (mode == 0) {
+        accept = (d_next == argmax_row(logits, lrow, V, dtype));
+      } else {
+        double u = (double)uniforms[(int64_t)b * n + (i - 1)];
+        int64_t qrow = ((int64_t)b * (k - 1) + (i - 1)) * V;
+        dist_row(logits, lrow, V, dtype, T, top_p, p, &c1);
+        if (c1 < cm) cm = c1;
+        dist_row(draft_logits, qrow, V, dtype, T, top_p, qd, &c1);
+        if (c1 < cm) cm = c1;
+        accept = (u * qd[d_next] < p[d_next]);
+        if (margins && p[d_next] > 0.0)
+          margins[(int64_t)b * n + (i - 1)] = fabs(u * qd[d_next] - p[d_next]) / p[d_next];
+      }
+      if (!accept) break;
+      j = i + 1;
+    }
+
+    /* the token at row j */
+    {
+      int64_t lrow = ((int64_t)b * n + (j - 1)) * V;
+      if (mode == 0) {
+        t_star = argmax_row(logits, lrow, V, dtype);
+      } else {
+        double u = (double)uniforms[(int64_t)b * n + (n - 1)];
+        double total = 0.0, c = 0.0, target, prev = 0.0;
+        dist_row(logits, lrow, V, dtype, T, top_p, p, &c1);
+        if (c1 < cm) cm = c1;
+        if (j < n) {
+          int64_t qrow = ((int64_t)b * (k - 1) + (j - 1)) * V;
+          dist_row(draft_logits, qrow, V, dtype, T, top_p, qd, &c1);
+          if (c1 < cm) cm = c1;
+          for (x = 0; x < V; ++x) { double r = p[x] - qd[x]; w[x] = r > 0.0 ? r : 0.0; total += w[x]; }
+          if (!(total > 0.0)) { for (x = 0; x < V; ++x) w[x] = p[x]; total = 0.0; for (x = 0; x < V; ++x) total += w[x]; }
+        } else {
+          for (x = 0; x < V; ++x) { w[x] = p[x]; total += w[x]; }
+        }
+        target = u * total;
+        t_star = V - 1;
+        for (x = 0; x < V; ++x) {
+          prev = c;
+          c += w[x];
+          if (target < c) { t_star = x; break; }
+        }
+        if (margins) {
+          double lo = target - prev, hi = c - target;
+          margins[(int64_t)b * n + (n - 1)] = (lo < hi ? lo : hi) / total;
+        }
+      }
+    }
+    if (cut_margins) cut_margins[b] = cm;
+
+    /* outputs */
+    accept_count[b] = j;
+    for (e = 0; e < n; ++e) out_tokens[(int64_t)b * n + e] = -1;
+    for (e = 0; e < j - 1; ++e) out_tokens[(int64_t)b * n + e] = drafts[(int64_t)b * k + e + 1];
+    out_tokens[(int64_t)b * n + j - 1] = t_star;
+    if (selected_block) selected_block[b] = k > 0 ? j : 0;
+    if (next_drafts && k > 0) {
+      next_drafts[(int64_t)b * k] = t_star;
+      for (e = 1; e < k; ++e)
+        next_drafts[(int64_t)b * k + e] =
+            block_guesses ? block_guesses[((int64_t)b * k + (j - 1)) * k + e] : -1;
+    }
+  }
+  free(p); free(qd); free(w);
+  return ORACLE_OK;
+}
+
+/*
+ * The next step's drafts from the selected mask block ([MS] §2: the mask slots
+ * give the diffusion predictions the next drafts come from; [NDfr] paragraph on
+ * betting on every outcome: the block matching the accept count is the one
+ * waiting).  With j = selected_block[b] (a value outside 1..k reads block 1 and
+ * the call returns ORACLE_ERR_COUNT), slot s = 2..k of block j supplies
+ * next_drafts[b][s-1]:
+ *   greedy (mode 0): the slot row's argmax (lowest index on ties);
+ *   sampling (mode 1): the smallest t with u[b][s-1] * 1 < sum_{x<=t} q_s(x),
+ *     q_s = dist_row(T, top_p) of the slot row, summed in index order (the
+ *     same inverse CDF as t*).
+ * next_drafts[b][0] (t*, from verification) is left as it is.
+ *   block_logits [B][k][k][V] (block j-1, slot s-1), uniforms [B][k] (mode 1).
+ * margins [B][k] (may be NULL): the distance of u to the nearest cumulative
+ * sum (mode 1), +inf elsewhere.
+ */
+int tidar_oracle_sample_drafts(int B, int k, int V, int dtype, int mode, double T, double top_p,
+                               const void* block_logits, const int32_t* selected_block,
+                               const float* uniforms, int32_t* next_drafts, double* margins) {
+  double* q;
+  int b, status = ORACLE_OK;
+  if (B < 0 || k < 0 || V <= 0 || (mode != 0 && mode != 1) || !(T > 0.0) || !(top_p > 0.0))
+    return ORACLE_ERR_ARG;
+  if (mode == 1 && !uniforms) return ORACLE_ERR_ARG;
+  q = (double*)malloc(sizeof(double) * V);
+  if (!q) return ORACLE_ERR_ARG;
+  for (b = 0; b < B; ++b) {
+    int j = selected_block[b], s;
+    if (margins) for (s = 0; s < k; ++s) margins[(int64_t)b * k + s] = INFINITY;
+    if (j < 1 || j > k) { j = 1; status = ORACLE_ERR_COUNT; }
+    for (s = 2; s <= k; ++s) {
+      const int64_t row = (((int64_t)b * k + (j - 1)) * k + (s - 1)) * V;
+      int tok;
+      if (mode == 0) {
+        tok = argmax_row(block_logits, row, V, dtype);
+      } else {
+        double u = (double)uniforms[(int64_t)b * k + (s - 1)], c = 0.0, prev = 0.0, total = 0.0, c1;
+        int x;
+        dist_row(block_logits, row, V, dtype, T, top_p, q, &c1);
+        for (x = 0; x < V; ++x) total += q[x];
+        tok = V - 1;
+        for (x = 0; x < V; ++x) {
+          prev = c;
+          c += q[x];
+          if (u * total < c) { tok = x; break; }
+        }
+        if (margins) {
+          double lo = u * total - prev, hi = c - u * total, mm = (lo < hi ? lo : hi) / total;
+          margins[(int64_t)b * k + (s - 1)] = mm < c1 ? mm : c1;
+        }
+      }
+      next_drafts[(int64_t)b * k + (s - 1)] = tok;
+    }
+  }
+  free(q);
+  return status;
+}
+
+/*
  * KV commit / evict ("the settled cache is reused, the rejected entries are
  * evicted", [NDfr] paragraph on the three zones; exact KV cache, [MS] "KV
  * Cache" and [FG] abstract).  Accepted drafts are always a prefix of the draft

@@ -180,12 +180,14 @@ Plan make_plan(const tidar_step_desc* d, int path) {
   // the second launch when splits merge through workspace partials.  A merge
   // on chip needs a cluster of nsplit CTAs; its waves count the clusters that
   // can be resident at once.
-  constexpr double kFixedBlocks = 2.5, kFinalizeBlocks = 2.0;
+  // A launch that already fills the device (units >= one wave) keeps one split:
+  // with ragged batches the longest sequence, not the wave count, sets its time.
+  constexpr double kFixedBlocks = 3.0, kFinalizeBlocks = 2.0;
   double best = 1e300;
   int best_n = 1;
   bool best_cluster = false;
   int last_ns = -1;
-  const int n_hi = max_ns < 64 ? max_ns : 64;
+  const int n_hi = units >= target ? 1 : (max_ns < 64 ? max_ns : 64);
   for (int n = 1; n <= n_hi; ++n) {
     split_keys(n);
     if (p.nsplit == last_ns) continue;
@@ -291,6 +293,8 @@ tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, 
   a.nsplit = p.nsplit; a.keys_per_split = p.keys_per_split;
   a.bf16 = d->dtype == TIDAR_BF16;
   a.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->head_dim);
+  a.step_keys = step_keys;
+  a.append = append;
   if (p.nsplit > 1 && !p.cluster_merge) {
     const size_t rows = (size_t)a.B * a.R * a.Hq;
     a.part_o = static_cast<float*>(workspace);

@@ -186,7 +186,7 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int kend = min(P, k0 + a.keys_per_split);
   const int npg = kend > k0 ? (kend - k0 + 63) / 64 : 0;
   const bool last = split == a.nsplit - 1;
-  const int nb = npg + (last ? 1 : 0);                   // + the step-key window (R <= 16 keys)
+  const int nb = npg + ((last && a.step_keys) ? 1 : 0);   // + the step-key window (R <= 16 keys)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -617,7 +617,7 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (threadIdx.x == 32) DEC_TRACE(154);
   }
 
-  if (split == 0 && len_ok && !a.part_o) {
+  if (split == 0 && len_ok && !a.part_o && a.append) {
     // ---------------------------------------------------------------- append
     // Draft rows D_1..D_n of KV head g into cache rows P .. P+n-1 (the step
     // keys above were read from k_blk / v_blk, not from the cache).

@@ -47,6 +47,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -80,11 +82,12 @@ constexpr int kPBars = 18;
 constexpr uint32_t kPOffMisc = kPOffBar + kPBars * 8;      // [0] TMEM base, [1] abort flag
 constexpr uint32_t kPSmem = kPOffMisc + 16;
 static_assert(kPSmem <= 232448, "shared memory budget");
-// split merge, in the K/V rings once they are idle: [2 tiles][128 rows][32
-// float4 chunks] fp32 partial O, then [2][128] lse
+// split merge receive area, in the K/V rings once they are idle: [slot][split]
+// [32 float4] fp32 partial rows for at most 256 + 16 (slot, split) pairs, then
+// their lse
 constexpr uint32_t kPOffPart = kPOffK;
-constexpr uint32_t kPOffPartL = kPOffPart + 2 * 128 * 512;
-static_assert(kPOffPartL + 2 * 128 * 4 <= kPOffBar, "split partials fit the rings");
+constexpr uint32_t kPOffPartL = kPOffPart + 272 * 512;
+static_assert(kPOffPartL + 272 * 4 <= kPOffBar, "split partials fit the rings");
 
 constexpr uint32_t kPTmemCols = 512;
 __device__ __forceinline__ uint32_t pcol_s(int t) { return 128u * (uint32_t)t; }
@@ -397,32 +400,47 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (!v) x[c] = 0xff800000u;
           }
         }
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // row maximum: eight independent chains
+        float mx[8];
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
-          mx[0] = max3(mx[0], __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
-          mx[1] = max3(mx[1], __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
-          mx[2] = max3(mx[2], __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
-          mx[3] = max3(mx[3], __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
-        }
-        const float mrow = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+        for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], __uint_as_float(x[c + 2 * i]), __uint_as_float(x[c + 2 * i + 1]));
+        const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
         if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 2);
         const float m_new = fmaxf(m, mrow);
         const bool need = m_new > m + 8.0f;
         const float f_resc = need ? ex2(m - m_new) : 1.0f;  // factor for O and l (m = -inf -> 0)
         if (need) m = m_new;
         const float nbase = m == -INFINITY ? 0.f : -m;
-        // P = 2^(score * scale - m), bf16 pairs packed in place over x[0..63]
+        // P = 2^(score * scale - m), bf16 pairs packed in place over x[0..63];
+        // in unmasked blocks one pair in four goes through the FMA-pipe
+        // exponential (masked scores are -inf: those blocks keep the MUFU,
+        // whose 2^-inf is exactly 0)
         const uint64_t sl2x2 = f2_make(sl2, sl2), nbx2 = f2_make(nbase, nbase);
         uint64_t ls2[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
+        auto exps = [&](auto poly) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          float v0, v1;
-          f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
-          const float p0 = ex2(v0), p1 = ex2(v1);
-          ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
-          x[c] = cvt_bf16x2(p0, p1);
-        }
+          for (int c = 0; c < 64; ++c) {
+            float v0, v1;
+            f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
+            float p0, p1;
+            if (decltype(poly)::value && (c & 3) == 3) {
+              p0 = exp2_poly(v0);
+              p1 = exp2_poly(v1);
+            } else {
+              p0 = ex2(v0);
+              p1 = ex2(v1);
+            }
+            ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
+            x[c] = pack_bf16_int(p0, p1);
+          }
+        };
+        if (full) exps(std::true_type{});
+        else exps(std::false_type{});
         if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 3);
         tmem_st32(trow + pcol_s(t), *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
         tmem_st32(trow + pcol_s(t) + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
@@ -535,80 +553,58 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else if (cluster) {
     // ---------------------------------------------------------------- split merge
-    // Each CTA leaves its normalised partial O of both tiles (fp32 [t][128
-    // rows][32 float4 chunks], chunk index XOR (row & 7) against bank
-    // conflicts) and per-row lse in its rings; after a cluster barrier CTA
-    // `rank` merges its share of the (tile, row) list over distributed shared
-    // memory and writes bf16 O and lse.
-    float* po = reinterpret_cast<float*>(smem + kPOffPart);
-    float* pl = reinterpret_cast<float*>(smem + kPOffPartL);
-    if (warp < 8) {
-      const int t = warp >> 2, r = threadIdx.x & 127;
-      if (owrite) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          *reinterpret_cast<float4*>(po + ((t * 128 + r) * 32 + (c ^ (r & 7))) * 4) =
-              make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
-      }
-      pl[t * 128 + r] = owrite ? olse : -INFINITY;
-    }
-    cluster_sync_all();
+    // Row i = t * 128 + r of the pair is owned by CTA i % ns (slot i / ns).
+    // Once every CTA is past its main loop (first barrier: the K/V rings are
+    // idle) each softmax thread pushes its row's normalised partial O and lse
+    // into the owner's rings; after the second barrier the owners merge their
+    // rows locally.
     const int ns = a.nsplit;
     const uint32_t rank = cluster_rank();
-    const int total = rows_valid[0] + rows_valid[1];
-    const int rpc = (total + ns - 1) / ns;
-    const int r_lo = (int)rank * rpc, r_hi = min(total, r_lo + rpc);
-    const uint32_t po_s = smem_u32(po), pl_s = smem_u32(pl);
-    for (int i = r_lo + warp; i < r_hi; i += kPThreads / 32) {
-      const int t = i < rows_valid[0] ? 0 : 1;
-      const int rr = t == 0 ? i : i - rows_valid[0];
-      const int slot = t * 128 + rr;
-      float l2 = -INFINITY;
-      if (lane < ns) l2 = ld_cluster_f32(mapa(pl_s + 4u * slot, (uint32_t)lane)) * 1.4426950408889634f;
-      float mx = l2;
+    float* recv = reinterpret_cast<float*>(smem + kPOffPart);        // [slot][split][32 float4]
+    float* recv_l = reinterpret_cast<float*>(smem + kPOffPartL);     // [slot][split]
+    cluster_sync_all();
+    if (warp < 8) {
+      const int t = warp >> 2, r = threadIdx.x & 127;
+      if (r < rows_valid[t]) {
+        const int i = t * 128 + r;
+        const uint32_t owner = (uint32_t)(i % ns);
+        const int slot = i / ns;
+        if (owrite) {
+          const uint32_t dst = mapa(smem_u32(recv) + 16u * (uint32_t)((slot * ns + split) * 32), owner);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float w = (lane < ns && l2 != -INFINITY) ? ex2(l2 - mx) : 0.f;
-      float wsum = w;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-      const uint32_t off = 4u * (slot * 32 + (lane ^ (rr & 7))) * 4u;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < ns; s0 += 4) {
-        float4 xv[4];
-        float w4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float wl = __shfl_sync(0xffffffffu, w, (s0 + u) & 31);
-          w4[u] = s0 + u < ns ? wl : 0.f;
+          for (int c = 0; c < 32; ++c)
+            st_cluster_f32x4(dst + 16u * c, make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]));
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          xv[u] = s0 + u < ns ? ld_cluster_f32x4(mapa(po_s + off, (uint32_t)(s0 + u))) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          // a split with weight 0 (no visible key) may have left its row
-          // unwritten: select, do not multiply
-          if (w4[u] != 0.f) {
-            acc.x = fmaf(w4[u], xv[u].x, acc.x); acc.y = fmaf(w4[u], xv[u].y, acc.y);
-            acc.z = fmaf(w4[u], xv[u].z, acc.z); acc.w = fmaf(w4[u], xv[u].w, acc.w);
-          }
-        }
+        st_cluster_f32(mapa(smem_u32(recv_l) + 4u * (uint32_t)(slot * ns + split), owner), owrite ? olse : -INFINITY);
       }
-      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-      const int rho = rho0[t] + rr / a.G, h = g * a.G + rr % a.G;
-      const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
-      uint2 u;
-      u.x = cvt_bf16x2(acc.x * inv, acc.y * inv);
-      u.y = cvt_bf16x2(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + row * 128 + 4 * lane) = u;
-      if (lane == 0 && a.lse_out)
-        a.lse_out[row] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
     }
-    cluster_sync_all();   // no CTA leaves while another may still read its shared memory
+    cluster_sync_all();
+    const int slots = (256 - (int)rank + ns - 1) / ns;
+    merge_pushed_rows(recv, recv_l, slots, ns, warp, kPThreads / 32, lane,
+                      [&](int sl) -> long long {
+                        const int i = sl * ns + (int)rank;
+                        const int t = i >> 7, rr = i & 127;
+                        if (t >= ntile || rr >= rows_valid[t]) return -1;
+                        const int rho = rho0[t] + rr / a.G, h = g * a.G + rr % a.G;
+                        return (long long)(b * a.R + rho) * a.Hq + h;
+                      },
+                      static_cast<__nv_bfloat16*>(a.out), a.lse_out);
   }
 
-  if (pair == 0 && split == 0 && len_ok && !a.part_o) {
+  if (nb == 0 && layout_ok && a.nsplit == 1 && warp < 8) {
+    // no key at all for this pair (a prefix-only call on an empty slice):
+    // O = 0 and lse = -inf, so a later merge gives these rows no weight
+    const int t = warp >> 2, r = threadIdx.x & 127;
+    if (r < rows_valid[t]) {
+      const int rho = rho0[t] + r / a.G, h = g * a.G + r % a.G;
+      const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * 128);
+      for (int e = 0; e < 16; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+      if (a.lse_out) a.lse_out[row] = -INFINITY;
+    }
+  }
+
+  if (pair == 0 && split == 0 && len_ok && !a.part_o && a.append) {
     // ---------------------------------------------------------------- append
     // Draft rows D_1..D_n of KV head g into cache rows P .. P+n-1 (the keys
     // above read them from k_blk / v_blk, not from the cache).

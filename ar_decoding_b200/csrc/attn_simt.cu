@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(AttnArgs a) {
   if (bad_page && lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
 
   // step keys (drafts and mask slots), last split only
-  if (split == a.nsplit - 1) {
+  if (split == a.nsplit - 1 && a.step_keys) {
     const StepVis vis = step_visibility(a.k, rho);
     const T* kb = static_cast<const T*>(a.k_blk);
     const T* vb = static_cast<const T*>(a.v_blk);
@@ -207,7 +207,7 @@ template <typename T, int D>
 cudaError_t launch_finalize_t(const AttnArgs& a, cudaStream_t s) {
   const size_t rows = (size_t)a.B * a.R * a.Hq;
   const int merge_blocks = a.nsplit > 1 ? (int)((rows + kWarps - 1) / kWarps) : 0;
-  const int blocks = merge_blocks + a.B * a.n;
+  const int blocks = merge_blocks + (a.append ? a.B * a.n : 0);
   if (blocks == 0) return cudaSuccess;
   return launch_pdl(finalize_kernel<T, D>, dim3(blocks), kWarps * 32, 0, s, a, merge_blocks);
 }

@@ -620,79 +620,59 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else if (a.nsplit > 1) {
     // ---------------------------------------------------------------- split merge
-    // The CTAs of this cluster are the splits of one (b, g, tile).  Each leaves
-    // its normalised partial O (fp32 [128 rows][32 float4 chunks], chunk index
-    // XOR (row & 7) against bank conflicts) and per-row lse in its K ring;
-    // after a cluster barrier, CTA `rank` merges rows [rank*rpc, ...) from all
-    // splits over distributed shared memory and writes bf16 O and lse.
-    float* po = reinterpret_cast<float*>(smem + kOffK);
-    float* pl = reinterpret_cast<float*>(smem + kOffK + 128 * 512);
+    // The CTAs of this cluster are the splits of one (b, g, tile).  Row r is
+    // owned by CTA r % ns (slot r / ns).  Once every CTA is past its main loop
+    // (first barrier: the K rings are idle) each thread pushes its 32 columns
+    // of normalised partial O and the row's lse into the owner's K ring; after
+    // the second barrier the owners merge their rows locally.
+    const int ns = a.nsplit;
+    const uint32_t rank = cluster_rank();
+    float* recv = reinterpret_cast<float*>(smem + kOffK);            // [slot][split][32 float4]
+    float* recv_l = reinterpret_cast<float*>(smem + kOffK + 144 * 512);   // [slot][split]
+    cluster_sync_all();
     if (warp >= 2) {
       const int r = 32 * (warp & 3) + lane;
       const int t = (warp - 2) >> 3, hf = ((warp - 2) >> 2) & 1;
       const int c0 = 8 * (2 * t + hf);                   // first float4 chunk of this thread
-      if (owrite) {
+      if (r < rows_valid) {
+        const uint32_t owner = (uint32_t)(r % ns);
+        const int slot = r / ns;
+        if (owrite) {
+          const uint32_t dst = mapa(smem_u32(recv) + 16u * (uint32_t)((slot * ns + split) * 32 + c0), owner);
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<float4*>(po + (r * 32 + ((c0 + c) ^ (r & 7))) * 4) =
-              make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
+          for (int c = 0; c < 8; ++c)
+            st_cluster_f32x4(dst + 16u * c, make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]));
+        }
+        if (t == 0 && hf == 0)
+          st_cluster_f32(mapa(smem_u32(recv_l) + 4u * (uint32_t)(slot * ns + split), owner), owrite ? olse : -INFINITY);
       }
-      if (t == 0 && hf == 0) pl[r] = owrite ? olse : -INFINITY;
     }
     cluster_sync_all();
-    const int ns = a.nsplit;
-    const uint32_t rank = cluster_rank();
-    const int rpc = (rows_valid + ns - 1) / ns;
-    const int r_lo = (int)rank * rpc, r_hi = min(rows_valid, r_lo + rpc);
-    const uint32_t po_s = smem_u32(po), pl_s = smem_u32(pl);
-    for (int R = r_lo + warp; R < r_hi; R += kThreads / 32) {
-      float l2 = -INFINITY;
-      if (lane < ns) l2 = ld_cluster_f32(mapa(pl_s + 4u * R, (uint32_t)lane)) * 1.4426950408889634f;
-      float mx = l2;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float w = (lane < ns && l2 != -INFINITY) ? ex2(l2 - mx) : 0.f;
-      float wsum = w;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-      const uint32_t off = 4u * (R * 32 + (lane ^ (R & 7))) * 4u;
-      // the splits' partial rows, four remote loads in flight at a time; a
-      // split with weight 0 (no visible key) may have left its row unwritten,
-      // so its value is selected away rather than multiplied
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < ns; s0 += 4) {
-        float4 x[4];
-        float w4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float wl = __shfl_sync(0xffffffffu, w, (s0 + u) & 31);
-          w4[u] = s0 + u < ns ? wl : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          x[u] = s0 + u < ns ? ld_cluster_f32x4(mapa(po_s + off, (uint32_t)(s0 + u))) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (w4[u] != 0.f) {
-            acc.x = fmaf(w4[u], x[u].x, acc.x); acc.y = fmaf(w4[u], x[u].y, acc.y);
-            acc.z = fmaf(w4[u], x[u].z, acc.z); acc.w = fmaf(w4[u], x[u].w, acc.w);
-          }
-        }
-      }
-      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-      const int rho = rho0 + R / a.G, h = g * a.G + R % a.G;
-      const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
-      uint2 u;
-      u.x = cvt_bf16x2(acc.x * inv, acc.y * inv);
-      u.y = cvt_bf16x2(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + row * 128 + 4 * lane) = u;
-      if (lane == 0 && a.lse_out)
-        a.lse_out[row] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
-    }
-    cluster_sync_all();   // no CTA leaves while another may still read its shared memory
+    const int slots = (rows_valid - (int)rank + ns - 1) / ns;
+    merge_pushed_rows(recv, recv_l, slots > 0 ? slots : 0, ns, warp, kThreads / 32, lane,
+                      [&](int sl) -> long long {
+                        const int R = sl * ns + (int)rank;
+                        const int rho = rho0 + R / a.G, h = g * a.G + R % a.G;
+                        return (long long)(b * a.R + rho) * a.Hq + h;
+                      },
+                      static_cast<__nv_bfloat16*>(a.out), a.lse_out);
   }
 
-  if (tile == 0 && split == 0 && len_ok && !a.part_o) {
+  if (bp.nb == 0 && a.nsplit == 1 && warp >= 2) {
+    // no key at all for this tile (a prefix-only call on an empty slice):
+    // O = 0 and lse = -inf, so a later merge gives the tile no weight
+    const int r = 32 * (warp & 3) + lane;
+    const int t = (warp - 2) >> 3, hf = ((warp - 2) >> 2) & 1;
+    if (r < rows_valid) {
+      const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
+      const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * 128 + 32 * (2 * t + hf));
+      for (int e = 0; e < 4; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+      if (t == 0 && hf == 0 && a.lse_out) a.lse_out[row] = -INFINITY;
+    }
+  }
+
+  if (tile == 0 && split == 0 && len_ok && !a.part_o && a.append) {
     // ---------------------------------------------------------------- append
     // Draft rows D_1..D_n of KV head g into cache rows P .. P+n-1 (the keys
     // above read them from k_blk / v_blk, not from the cache).

@@ -26,6 +26,8 @@ struct AttnArgs {
   int nsplit, keys_per_split;
   int bf16;              // 1: bf16 tensors, 0: fp32
   float scale;           // softmax scale (natural-log domain)
+  int step_keys;         // 1: the last split also attends the step keys (the zone mask); 0: prefix only
+  int append;            // 1: write the draft rows' K/V into the cache
 };
 
 // Warp-MMA kernel for query blocks of at most 16 packed rows per KV head

@@ -115,6 +115,25 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// 2^v on the FMA pipe, for a share of the softmax exponentials (the MUFU is the
+// softmax's busiest unit): v = j + f with j = floor(v); 2^f by a degree-3
+// polynomial, a least-squares fit of 2^f on [0, 1) weighted for relative
+// error with p(0) = 1 (maximum relative error 1.7e-4, below the 2^-9 of the
+// bf16 P it feeds); 2^j by adding j to the exponent field.  Valid for
+// finite v; v is clamped at -127 (the result is then ~0).
+__device__ __forceinline__ float exp2_poly(float v) {
+  v = fmaxf(v, -127.f);
+  const float j = floorf(v);
+  const float f = v - j;
+  const float p = fmaf(fmaf(fmaf(0.07632546f, f, 0.22830825f), f, 0.69503617f), f, 1.0f);
+  return __int_as_float(__float_as_int(p) + ((int)j << 23));
+}
+// (lo, hi) -> bf16x2 with integer operations (round half up on the magnitude),
+// keeping the conversion off the XU pipe; for finite inputs.
+__device__ __forceinline__ uint32_t pack_bf16_int(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
+  return __byte_perm(a, b, 0x7632);
+}
 // ------------------------------------------------------------------ block plan
 // Blocks 0..npb-1: 128 prefix keys from k0; then nw step-key windows.
 struct BlockPlan {
@@ -129,7 +148,7 @@ __device__ __forceinline__ BlockPlan make_block_plan(const AttnArgs& a, int P, i
   bp.kend = min(P, bp.k0 + a.keys_per_split);
   bp.npb = bp.kend > bp.k0 ? (bp.kend - bp.k0 + 127) / 128 : 0;
   bp.nw = 0;
-  if (split == a.nsplit - 1) {
+  if (split == a.nsplit - 1 && a.step_keys) {
     bp.wins[bp.nw++] = 0;                       // drafts D_1..D_k (k <= 16) live in window 0
     if (a.k > 0 && rho1 - 1 >= a.k) {           // the tile holds mask-slot rows
       const int jlo = (max(rho0, a.k) - a.k) / a.k + 1;
@@ -144,6 +163,52 @@ __device__ __forceinline__ BlockPlan make_block_plan(const AttnArgs& a, int P, i
 }
 
 __device__ __forceinline__ bool page_ok(int page, int num_pages) { return page >= 0 && page < num_pages; }
+
+// ------------------------------------------------------------------ split merge
+// Key splits of one query tile run as the CTAs of a thread-block cluster.  After
+// a cluster barrier each CTA pushes its normalised partial rows (fp32) and
+// their lse into the row's owner CTA -- remote stores, no round trip -- laid
+// out [slot][split][32 float4 chunks] and [slot][split]; after a second
+// barrier each owner merges its rows from its own shared memory.
+__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+// One warp per slot, lane = float4 chunk of the row.  row_of(slot) gives the
+// output row (or -1 for a slot holding no row).  A split whose lse is -inf saw
+// no key and may have pushed no values: it is selected away, not multiplied.
+template <typename RowOf>
+__device__ __forceinline__ void merge_pushed_rows(const float* recv, const float* recv_l, int slots, int ns,
+                                                  int warp, int nwarps, int lane, RowOf row_of,
+                                                  __nv_bfloat16* out, float* lse_out) {
+  for (int sl = warp; sl < slots; sl += nwarps) {
+    const long long row = row_of(sl);
+    if (row < 0) continue;
+    float mx = -INFINITY;
+    for (int s2 = 0; s2 < ns; ++s2) mx = fmaxf(mx, recv_l[sl * ns + s2] * 1.4426950408889634f);
+    float wsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s2 = 0; s2 < ns; ++s2) {
+      const float l2 = recv_l[sl * ns + s2] * 1.4426950408889634f;
+      if (l2 == -INFINITY) continue;
+      const float w = ex2(l2 - mx);
+      wsum += w;
+      const float4 x = reinterpret_cast<const float4*>(recv)[(sl * ns + s2) * 32 + lane];
+      acc.x = fmaf(w, x.x, acc.x); acc.y = fmaf(w, x.y, acc.y);
+      acc.z = fmaf(w, x.z, acc.z); acc.w = fmaf(w, x.w, acc.w);
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    uint2 u;
+    u.x = cvt_bf16x2(acc.x * inv, acc.y * inv);
+    u.y = cvt_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(out + row * 128 + 4 * lane) = u;
+    if (lane == 0 && lse_out) lse_out[row] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
+  }
+}
 
 }  // namespace tc05
 }  // namespace tidar

@@ -197,7 +197,7 @@ class Step:
         # attention: one launch when the kernel merges its splits on chip (no
         # workspace) on the tensor-core or decode path, else kernel + finalize;
         # then greedy verify (one cluster kernel) and commit (one cluster kernel)
-        self.attn_launches = 1 if (need == 0 and self.path_id in (2, 3)) else 2
+        self.attn_launches = 1 if (need == 0 and self.path_id in (2, 3, 4)) else 2
         self.launches_per_step = self.attn_launches + 1 + 1
 
     def attn(self, i):
@@ -304,7 +304,7 @@ class Loop:
         # cluster when the vocabulary's 4096-wide chunks fit a portable cluster
         # of 8, else two launches), commit
         nchunk = -(-V // 4096)
-        self.launches_per_step = (1 + (1 if (need == 0 and self.path_id in (2, 3)) else 2) +
+        self.launches_per_step = (1 + (1 if (need == 0 and self.path_id in (2, 3, 4)) else 2) +
                                   (1 if mode == "greedy" else (2 if nchunk <= 8 else 3)) + 1)
 
     def step(self, c, s):

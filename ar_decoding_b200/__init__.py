@@ -35,6 +35,7 @@ GREEDY, REJECTION = 0, 1
 PATH_AUTO, PATH_SIMT, PATH_TC05, PATH_DEC, PATH_PAIR = 0, 1, 2, 3, 4
 DEVERR_BAD_PAGE, DEVERR_BAD_LEN, DEVERR_BAD_COUNT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 1, 2, 4, 8, 16
 DEVERR_POOL = 32
+PART_STEP_KEYS, PART_APPEND = 1, 2
 _PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tc05": PATH_TC05, "dec": PATH_DEC,
           "pair": PATH_PAIR}
 
@@ -116,6 +117,10 @@ def lib():
         L.tidar_verify_sampled.restype = ctypes.c_int
         L.tidar_sample_drafts.argtypes = [I, I, I, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P]
         L.tidar_sample_drafts.restype = ctypes.c_int
+        L.tidar_step_attn_part.argtypes = [P, P, P, P, P, I, P, P, P, S, P]
+        L.tidar_step_attn_part.restype = ctypes.c_int
+        L.tidar_merge_attn.argtypes = [I, ctypes.c_int64, I, ctypes.c_int, P, P, P, P, P]
+        L.tidar_merge_attn.restype = ctypes.c_int
         L.tidar_linear.argtypes = [I, I, I, ctypes.c_int, P, P, P, P]
         L.tidar_linear.restype = ctypes.c_int
         L.tidar_qkv_rope.argtypes = [P, I, P, P, P, ctypes.c_float, P, P, P, P]
@@ -335,6 +340,57 @@ def layer_step(x, w_qkv, w_o, cache, k, num_q_heads, num_kv_heads, *, max_prefix
                                 _ptr(w_o), float(rope_base), _ptr(out), _ptr(lse), _ptr(workspace),
                                 workspace.numel(), _stream_handle(stream))
     _check(st, "tidar_layer_step")
+    return out, lse
+
+
+def step_attn_part(q, k_blk, v_blk, cache, k, flags, *, max_prefix_len, scale=0.0, path="auto",
+                   out=None, lse=None, workspace=None, stream=None):
+    """Step attention over one slice of a sequence's prefix (context
+    parallelism): flags PART_STEP_KEYS also attends the step keys,
+    PART_APPEND writes the draft rows.  Returns (out, lse)."""
+    _dev(q, "q")
+    dev = q.device
+    _dev(k_blk, "k_blk", q.dtype, dev)
+    _dev(v_blk, "v_blk", q.dtype, dev)
+    desc = make_desc(q, k_blk, cache, k, max_prefix_len, scale, path)
+    cdesc = make_cache_desc(cache, dev)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    _dev(out, "out", q.dtype, dev)
+    _dev(lse, "lse", torch.float32, dev)
+    need = step_attn_workspace_bytes(desc)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _devopt(workspace, "workspace", None, dev)
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().tidar_step_attn_part(ctypes.byref(desc), ctypes.byref(cdesc), _ptr(q), _ptr(k_blk),
+                                    _ptr(v_blk), int(flags), _ptr(out), _ptr(lse), _ptr(workspace),
+                                    wbytes, _stream_handle(stream))
+    _check(st, "tidar_step_attn_part")
+    return out, lse
+
+
+def merge_attn(parts_out, parts_lse, *, out=None, lse=None, stream=None):
+    """Log-sum-exp merge of attention results over disjoint key sets:
+    parts_out [nparts][...][D], parts_lse [nparts][...] -> (out, lse)."""
+    _dev(parts_out, "parts_out")
+    dev = parts_out.device
+    _dev(parts_lse, "parts_lse", torch.float32, dev)
+    nparts, D = parts_out.shape[0], parts_out.shape[-1]
+    rows = parts_lse[0].numel()
+    if tuple(parts_out.shape[:-1]) != tuple(parts_lse.shape):
+        raise ValueError("parts_out and parts_lse disagree in shape")
+    if out is None:
+        out = torch.empty(parts_out.shape[1:], dtype=parts_out.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty(parts_lse.shape[1:], dtype=torch.float32, device=dev)
+    _dev(out, "out", parts_out.dtype, dev)
+    _dev(lse, "lse", torch.float32, dev)
+    st = lib().tidar_merge_attn(nparts, rows, D, _dtype_code(parts_out), _ptr(parts_out),
+                                _ptr(parts_lse), _ptr(out), _ptr(lse), _stream_handle(stream))
+    _check(st, "tidar_merge_attn")
     return out, lse
 
 

@@ -156,9 +156,10 @@ Plan make_plan(const tidar_step_desc* d, int path) {
       return;
     }
     // tensor-core paths: the last split also runs the tile's step-key windows
-    // (up to ceil(R / 128) blocks of 128), so the split size counts them and
-    // the last split gets that many fewer prefix blocks
-    const int wins = ((path == 2 || path == 4) && n > 1) ? (R + 127) / 128 : 0;
+    // (up to ceil(R / 128) blocks of 128, masked: each costs about 1.5 prefix
+    // blocks), so the split size counts them and the last split gets
+    // correspondingly fewer prefix blocks
+    const int wins = ((path == 2 || path == 4) && n > 1) ? (3 * ((R + 127) / 128) + 1) / 2 : 0;
     const int bps = (blocks128 + wins + n - 1) / n;
     p.keys_per_split = (bps > 0 ? bps : 1) * 128;
     p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
@@ -259,9 +260,16 @@ size_t tidar_step_attn_workspace_bytes(const tidar_step_desc* d) {
          align256((size_t)p.nsplit * rows * sizeof(float));
 }
 
-tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, const void* q,
-                             const void* k_blk, const void* v_blk, void* out, float* lse_out,
-                             void* workspace, size_t workspace_bytes, tidar_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The step attention; step_keys = 0 restricts every row to the cache's prefix
+// (a slice of a longer sequence), append = 0 leaves the cache untouched.
+tidar_status step_attn_impl(const tidar_step_desc* d, const tidar_kv_cache* c, const void* q,
+                            const void* k_blk, const void* v_blk, void* out, float* lse_out,
+                            void* workspace, size_t workspace_bytes, tidar_stream_t stream, int step_keys,
+                            int append) {
   tidar_status st = check_desc(d);
   if (st != TIDAR_OK) return st;
   if (d->batch == 0) return TIDAR_OK;
@@ -311,10 +319,44 @@ tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, 
   // Split merge and draft-row append: a second launch for the CUDA-core path
   // and for split partials; the tensor-core and decode kernels do both
   // themselves with one split or with the on-chip cluster merge.
-  if (pth == 1 || (p.nsplit > 1 && !p.cluster_merge)) {
+  if ((pth == 1 && append) || (p.nsplit > 1 && !p.cluster_merge)) {
     e = tidar::launch_finalize(a, s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
+  return TIDAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tidar_status tidar_step_attn(const tidar_step_desc* d, const tidar_kv_cache* c, const void* q,
+                             const void* k_blk, const void* v_blk, void* out, float* lse_out,
+                             void* workspace, size_t workspace_bytes, tidar_stream_t stream) {
+  return step_attn_impl(d, c, q, k_blk, v_blk, out, lse_out, workspace, workspace_bytes, stream, 1, 1);
+}
+
+tidar_status tidar_step_attn_part(const tidar_step_desc* d, const tidar_kv_cache* c, const void* q,
+                                  const void* k_blk, const void* v_blk, int32_t flags, void* out,
+                                  float* lse_out, void* workspace, size_t workspace_bytes,
+                                  tidar_stream_t stream) {
+  if (flags & ~(TIDAR_PART_STEP_KEYS | TIDAR_PART_APPEND)) return TIDAR_ERR_INVALID_ARG;
+  if (!lse_out) return TIDAR_ERR_INVALID_ARG;
+  return step_attn_impl(d, c, q, k_blk, v_blk, out, lse_out, workspace, workspace_bytes, stream,
+                        (flags & TIDAR_PART_STEP_KEYS) ? 1 : 0, (flags & TIDAR_PART_APPEND) ? 1 : 0);
+}
+
+tidar_status tidar_merge_attn(int32_t nparts, int64_t rows, int32_t head_dim, tidar_dtype dtype,
+                              const void* part_o, const float* part_lse, void* out, float* lse_out,
+                              tidar_stream_t stream) {
+  if (nparts <= 0 || rows < 0) return TIDAR_ERR_INVALID_ARG;
+  if (nparts > 64 || (head_dim != 64 && head_dim != 128)) return TIDAR_ERR_UNSUPPORTED;
+  if (dtype != TIDAR_F32 && dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
+  if (rows == 0) return TIDAR_OK;
+  if (!part_o || !part_lse || !out || !aligned16(part_o) || !aligned16(out)) return TIDAR_ERR_INVALID_ARG;
+  const cudaError_t e = tidar::launch_merge_parts(nparts, rows, head_dim, dtype == TIDAR_BF16, part_o, part_lse,
+                                                  out, lse_out, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
   return TIDAR_OK;
 }
 

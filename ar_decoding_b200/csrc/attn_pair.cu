@@ -47,8 +47,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <type_traits>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -388,17 +386,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!full) {
           // invisible keys (zone mask, past the prefix end, unmapped page) get
           // -inf: their probability is 2^-inf = 0
+          uint32_t mw[4];
+          block_mask(window, kb, vis, a.R, lo_valid, hi_valid, mw);
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            bool v;
-            if (window) {
-              const int key = kb + c;
-              v = key < a.R && step_visible(vis, key);
-            } else {
-              v = c < 64 ? c < lo_valid : c - 64 < hi_valid;
-            }
-            if (!v) x[c] = 0xff800000u;
-          }
+          for (int c = 0; c < 128; ++c)
+            if (!(mw[c >> 5] & (1u << (c & 31)))) x[c] = 0xff800000u;
         }
         // row maximum: eight independent chains
         float mx[8];
@@ -416,31 +408,20 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float f_resc = need ? ex2(m - m_new) : 1.0f;  // factor for O and l (m = -inf -> 0)
         if (need) m = m_new;
         const float nbase = m == -INFINITY ? 0.f : -m;
-        // P = 2^(score * scale - m), bf16 pairs packed in place over x[0..63];
-        // in unmasked blocks one pair in four goes through the FMA-pipe
-        // exponential (masked scores are -inf: those blocks keep the MUFU,
-        // whose 2^-inf is exactly 0)
+        // P = 2^(score * scale - m), bf16 pairs packed in place over x[0..63]
+        // (every exponential on the MUFU: moving a share to an FMA-pipe
+        // polynomial and the bf16 packing to integer operations was measured
+        // slower -- the softmax warp is issue-bound, not MUFU-bound)
         const uint64_t sl2x2 = f2_make(sl2, sl2), nbx2 = f2_make(nbase, nbase);
         uint64_t ls2[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
-        auto exps = [&](auto poly) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            float v0, v1;
-            f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
-            float p0, p1;
-            if (decltype(poly)::value && (c & 3) == 3) {
-              p0 = exp2_poly(v0);
-              p1 = exp2_poly(v1);
-            } else {
-              p0 = ex2(v0);
-              p1 = ex2(v1);
-            }
-            ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
-            x[c] = pack_bf16_int(p0, p1);
-          }
-        };
-        if (full) exps(std::true_type{});
-        else exps(std::false_type{});
+        for (int c = 0; c < 64; ++c) {
+          float v0, v1;
+          f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
+          const float p0 = ex2(v0), p1 = ex2(v1);
+          ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
+          x[c] = cvt_bf16x2(p0, p1);
+        }
         if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 3);
         tmem_st32(trow + pcol_s(t), *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
         tmem_st32(trow + pcol_s(t) + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));

@@ -196,6 +196,56 @@ __global__ void __launch_bounds__(kWarps * 32) finalize_kernel(AttnArgs a, int m
   }
 }
 
+// Log-sum-exp merge of nparts attention results over disjoint key sets (one
+// warp per row): O = sum_r w_r O_r / sum_r w_r with w_r = exp(lse_r - max);
+// lse = max + log(sum_r w_r).  A part with lse = -inf (no key) gets no weight
+// and its row is not read.
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32) merge_parts_kernel(int nparts, long long rows, const T* part_o,
+                                                                  const float* part_lse, T* out, float* lse_out) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int VPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float la = lane < nparts ? part_lse[(size_t)lane * rows + row] : -INFINITY;
+  const float lb = lane + 32 < nparts ? part_lse[(size_t)(lane + 32) * rows + row] : -INFINITY;
+  float mx = fmaxf(la, lb);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float wa = la == -INFINITY ? 0.f : expf(la - mx);
+  const float wb = lb == -INFINITY ? 0.f : expf(lb - mx);
+  float wsum = wa + wb;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+  float acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+  for (int r = 0; r < nparts; ++r) {
+    const float w = __shfl_sync(0xffffffffu, r < 32 ? wa : wb, r & 31);
+    if (w == 0.f) continue;
+    float v[VPL];
+    load_vec<T, VPL>(part_o + ((size_t)r * rows + row) * D + lane * VPL, v);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] *= inv;
+  store_vec<T, VPL>(out + (size_t)row * D + lane * VPL, acc);
+  if (lse_out && lane == 0) lse_out[row] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+}
+
+template <typename T, int D>
+cudaError_t launch_merge_t(int nparts, long long rows, const void* part_o, const float* part_lse, void* out,
+                           float* lse_out, cudaStream_t s) {
+  const long long blocks = (rows + kWarps - 1) / kWarps;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  return launch_pdl(merge_parts_kernel<T, D>, dim3((unsigned)blocks), kWarps * 32, 0, s, nparts, rows,
+                    static_cast<const T*>(part_o), part_lse, static_cast<T*>(out), lse_out);
+}
+
 template <typename T, int D>
 cudaError_t launch_simt_t(const AttnArgs& a, cudaStream_t s) {
   const int M = a.R * a.G;
@@ -217,6 +267,14 @@ cudaError_t launch_finalize_t(const AttnArgs& a, cudaStream_t s) {
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s) {
   if (a.bf16) return a.D == 64 ? launch_simt_t<__nv_bfloat16, 64>(a, s) : launch_simt_t<__nv_bfloat16, 128>(a, s);
   return a.D == 64 ? launch_simt_t<float, 64>(a, s) : launch_simt_t<float, 128>(a, s);
+}
+
+cudaError_t launch_merge_parts(int nparts, long long rows, int D, int bf16, const void* part_o,
+                               const float* part_lse, void* out, float* lse_out, cudaStream_t s) {
+  if (bf16) return D == 64 ? launch_merge_t<__nv_bfloat16, 64>(nparts, rows, part_o, part_lse, out, lse_out, s)
+                           : launch_merge_t<__nv_bfloat16, 128>(nparts, rows, part_o, part_lse, out, lse_out, s);
+  return D == 64 ? launch_merge_t<float, 64>(nparts, rows, part_o, part_lse, out, lse_out, s)
+                 : launch_merge_t<float, 128>(nparts, rows, part_o, part_lse, out, lse_out, s);
 }
 
 cudaError_t launch_finalize(const AttnArgs& a, cudaStream_t s) {

@@ -405,6 +405,8 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         kb = bp.wins[b2 - bp.npb] * 128;
       }
       const bool full = !window && lo_valid == 64 && hi_valid == 64;
+      uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
+      if (!full) block_mask(window, kb, vis, a.R, lo_valid, hi_valid, mw);
       const uint32_t scol = col_s(t) + 64 * hf;          // this half's 64 score columns
       // pass 1: maximum of this half's raw scores (the positive scale commutes)
       float mb = -INFINITY;
@@ -418,18 +420,10 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           if (!full) {
             // masked block (rare): invisible keys become -inf in TMEM too, so
             // the exponential pass needs no mask (2^-inf = 0)
+            const uint32_t mwd = mw[2 * hf + h2];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int col = 64 * hf + 32 * h2 + c;
-              bool v;
-              if (window) {
-                const int key = kb + col;
-                v = key < a.R && step_visible(vis, key);
-              } else {
-                v = col < 64 ? col < lo_valid : col - 64 < hi_valid;
-              }
-              if (!v) x[c] = 0xff800000u;
-            }
+            for (int c = 0; c < 32; ++c)
+              if (!(mwd & (1u << c))) x[c] = 0xff800000u;
             tmem_st32(trow + scol + 32 * h2, x);
             tmem_wait_st();
           }

@@ -59,6 +59,10 @@ int tc05_starve_loads();
 // Split merge (when nsplit > 1) and the draft-row append, in one launch
 // (CUDA-core path).
 cudaError_t launch_finalize(const AttnArgs& a, cudaStream_t s);
+// Log-sum-exp merge of attention results over disjoint key sets: part_o
+// [nparts][rows][D] (dtype), part_lse [nparts][rows] -> out, lse_out.
+cudaError_t launch_merge_parts(int nparts, long long rows, int D, int bf16, const void* part_o,
+                               const float* part_lse, void* out, float* lse_out, cudaStream_t s);
 
 struct VerifyArgs {
   int B, k, n, V, bf16, mode;

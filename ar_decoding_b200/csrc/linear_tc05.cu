@@ -75,6 +75,23 @@ struct LinParams {
   unsigned int* err;
 };
 
+// Optional timeline of CTA (0, 0, 0) (build with -DTIDAR_TRACE; absent from
+// normal builds): [0] setup, [1] weights of the first stages issued, [2]
+// after the wait on the previous kernel, [16 + i] producer issues k-block i,
+// [144 + i] the MMA thread sees k-block i, [272] accumulator done, [273]
+// partials in shared memory, [274] merged and written; [512 + 2 cta] start /
+// end of every CTA.
+#ifdef TIDAR_TRACE
+__device__ unsigned long long g_lin_trace[512 + 2 * 4096];
+#define LIN_TRACE(slot) do { if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (slot) < 512) \
+    g_lin_trace[(slot)] = global_ns(); } while (0)
+#define LIN_TRACE_CTA(w) do { const unsigned c_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+    if (c_ < 4096) g_lin_trace[512 + 2 * c_ + (w)] = global_ns(); } while (0)
+#else
+#define LIN_TRACE(slot) do {} while (0)
+#define LIN_TRACE_CTA(w) do {} while (0)
+#endif
+
 __device__ __forceinline__ void lin_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void lin_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -142,6 +159,7 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   double* invf = reinterpret_cast<double*>(smem + ring + 8u * (2 * kLinMaxStages + 1) + 16);   // [64]
 
+  if (threadIdx.x == 0) { LIN_TRACE_CTA(0); LIN_TRACE(0); }
   if (threadIdx.x == 0) {
     // the other CTAs of the cluster read this flag before trusting this CTA's
     // partials, so it is set even when the layout check fails
@@ -185,9 +203,11 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
         mbar_expect_tx(bar(BAR_FULL + i), a_bytes + b_bytes);
         tma_load_2d(dst, &tm_w, (kb0 + i) * 64, ft * 128, bar(BAR_FULL + i));
       }
+      LIN_TRACE(1);
     }
     pdl_wait();
     pdl_trigger();
+    if (lane == 0) LIN_TRACE(2);
     if (lane == 0) {
       int issued = pre;          // stages whose copies were (at least partly) issued
       for (int i = 0; i < nkb; ++i) {
@@ -199,6 +219,7 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
           tma_load_2d(dst, &tm_w, (kb0 + i) * 64, ft * 128, bar(BAR_FULL + s));
           issued = i + 1;
         }
+        LIN_TRACE(16 + min(i, 127));
         for (int u = 0; u < prm.nsub; ++u)
           tma_load_2d(dst + a_bytes + (uint32_t)u * nsubn * 128u, &tm_x, (kb0 + i) * 64, t0 + u * nsubn,
                       bar(BAR_FULL + s));
@@ -220,6 +241,7 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
       for (; i < nkb; ++i) {
         const int s = i % prm.stages;
         if (!wait_bar(bar(BAR_FULL + s), (uint32_t)((i / prm.stages) & 1), abort_flag, prm.err)) break;
+        LIN_TRACE(144 + min(i, 127));
         lin_fence_after();
         const uint32_t a = sb + (uint32_t)s * prm.stage_bytes, b = a + a_bytes;
 #pragma unroll
@@ -240,6 +262,7 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
     const int f = 32 * q4 + lane;
     bool ok = warp_wait_bar(bar(BAR_DONE), 0, abort_flag, prm.err);
     ok = __all_sync(0xffffffffu, ok && !*abort_flag);     // tcgen05.ld needs the whole warp
+    if (threadIdx.x == 64) LIN_TRACE(272);
     lin_fence_after();
     if (ok) {
       float* part = reinterpret_cast<float*>(smem);      // [nt][128]: the ring is idle now
@@ -255,6 +278,7 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
   lin_fence_before();
   __syncthreads();
   const bool cta_ok = layout_ok && !*abort_flag;
+  if (threadIdx.x == 0) LIN_TRACE(273);
   // every CTA of the cluster has its partials in shared memory
   if (prm.ksplit > 1) cluster_sync_all();
 
@@ -337,6 +361,7 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
   // no CTA leaves (or frees TMEM) while another may still read its shared memory
   if (prm.ksplit > 1) cluster_sync_all();
   else __syncthreads();
+  if (threadIdx.x == 0) { LIN_TRACE(274); LIN_TRACE_CTA(1); }
   if (layout_ok && warp == 1) {
     lin_fence_after();
     if (lane == 0) wait_quiet(bar(BAR_DONE), 0);
@@ -361,6 +386,12 @@ cudaError_t lin_smem_attr() {
 }
 
 }  // namespace
+
+#ifdef TIDAR_TRACE
+extern "C" int tidar_lin_trace_read(void* dst, size_t bytes) {
+  return (int)cudaMemcpyFromSymbol(dst, g_lin_trace, bytes);
+}
+#endif
 
 LinearPlan plan_linear(int T, int K, int N) {
   LinearPlan p{};

@@ -115,24 +115,35 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-// 2^v on the FMA pipe, for a share of the softmax exponentials (the MUFU is the
-// softmax's busiest unit): v = j + f with j = floor(v); 2^f by a degree-3
-// polynomial, a least-squares fit of 2^f on [0, 1) weighted for relative
-// error with p(0) = 1 (maximum relative error 1.7e-4, below the 2^-9 of the
-// bf16 P it feeds); 2^j by adding j to the exponent field.  Valid for
-// finite v; v is clamped at -127 (the result is then ~0).
-__device__ __forceinline__ float exp2_poly(float v) {
-  v = fmaxf(v, -127.f);
-  const float j = floorf(v);
-  const float f = v - j;
-  const float p = fmaf(fmaf(fmaf(0.07632546f, f, 0.22830825f), f, 0.69503617f), f, 1.0f);
-  return __int_as_float(__float_as_int(p) + ((int)j << 23));
+// ------------------------------------------------------------------ key masks
+// Bits [a, b) of the 32-column word w (columns 32 w .. 32 w + 31).
+__device__ __forceinline__ uint32_t col_bits(int lo, int hi, int w) {
+  const int a = max(lo - 32 * w, 0), b = min(hi - 32 * w, 32);
+  if (b <= a) return 0u;
+  const uint32_t run = b - a == 32 ? 0xffffffffu : ((1u << (b - a)) - 1u);
+  return run << a;
 }
-// (lo, hi) -> bf16x2 with integer operations (round half up on the magnitude),
-// keeping the conversion off the XU pipe; for finite inputs.
-__device__ __forceinline__ uint32_t pack_bf16_int(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
-  return __byte_perm(a, b, 0x7632);
+// Visibility of the 128 columns of a key block as four 32-bit words.  A
+// step-key window starting at step key kb: the row's visible step keys are
+// the intervals [0, e1) and [b0, b1) (zone mask), below R.  A prefix block:
+// columns [0, lo_valid) of its first page and [64, 64 + hi_valid) of its second.
+__device__ __forceinline__ void block_mask(bool window, int kb, const StepVis& vis, int R, int lo_valid,
+                                           int hi_valid, uint32_t (&mw)[4]) {
+  int l1, h1, l2, h2;
+  if (window) {
+    const int top = R - kb;                              // keys past R are not step keys
+    l1 = 0;
+    h1 = min(vis.e1 - kb, top);
+    l2 = vis.b0 - kb;
+    h2 = min(vis.b1 - kb, top);
+  } else {
+    l1 = 0;
+    h1 = lo_valid;
+    l2 = 64;
+    h2 = 64 + hi_valid;
+  }
+#pragma unroll
+  for (int w = 0; w < 4; ++w) mw[w] = col_bits(l1, h1, w) | col_bits(l2, h2, w);
 }
 // ------------------------------------------------------------------ block plan
 // Blocks 0..npb-1: 128 prefix keys from k0; then nw step-key windows.

@@ -160,6 +160,41 @@ tidar_status tidar_step_attn(const tidar_step_desc* desc, const tidar_kv_cache* 
                              float* lse_out, void* workspace, size_t workspace_bytes,
                              tidar_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Context parallelism: one long sequence whose prefix pages are spread over
+ * several GPUs (no counterpart on the pages, which speak of one standalone
+ * model on one device; the split follows from softmax attention over a union
+ * of disjoint key sets being the log-sum-exp merge of the attention over each
+ * set).  Each GPU runs tidar_step_attn_part on its slice -- a tidar_kv_cache
+ * holding its share of the prefix rows, seq_lens = the slice's length -- and
+ * the GPUs exchange (out, lse) and merge them with tidar_merge_attn.  Exactly
+ * one slice, the one holding the sequence's tail pages, takes the step keys
+ * and appends the draft rows.
+ *
+ * tidar_step_attn_part: tidar_step_attn with
+ *   flags & TIDAR_PART_STEP_KEYS: also attend the step keys (the zone mask);
+ *                                 else every row sees only the slice's prefix;
+ *   flags & TIDAR_PART_APPEND:    write the draft rows' K/V at the slice's
+ *                                 rows P_b .. P_b+n-1 (its pages reserved);
+ *   lse_out is required.  A row with no key in the call (an empty slice
+ *   without step keys) gets out = 0 and lse = -inf.
+ *   tidar_step_attn is flags = TIDAR_PART_STEP_KEYS | TIDAR_PART_APPEND.
+ * tidar_merge_attn: out[i] = sum_r w_r part_o[r][i] / sum_r w_r with
+ *   w_r = exp(part_lse[r][i] - max_r part_lse[r][i]); lse_out[i] = max +
+ *   log(sum w) (fp32; may be NULL).  part_o [nparts][rows][head_dim] and out
+ *   [rows][head_dim] of `dtype`; part_lse [nparts][rows] fp32.  A part with
+ *   lse -inf gets no weight.  nparts <= 64, head_dim 64 or 128.
+ * ------------------------------------------------------------------------- */
+#define TIDAR_PART_STEP_KEYS 0x1
+#define TIDAR_PART_APPEND 0x2
+tidar_status tidar_step_attn_part(const tidar_step_desc* desc, const tidar_kv_cache* cache,
+                                  const void* q, const void* k_blk, const void* v_blk,
+                                  int32_t flags, void* out, float* lse_out, void* workspace,
+                                  size_t workspace_bytes, tidar_stream_t stream);
+tidar_status tidar_merge_attn(int32_t nparts, int64_t rows, int32_t head_dim, tidar_dtype dtype,
+                              const void* part_o, const float* part_lse, void* out,
+                              float* lse_out, tidar_stream_t stream);
+
 /* The launch plan the library would use: kernel family (1 SIMT, 2 TC05,
  * 3 DEC, 4 PAIR) and number of KV splits.  Host only; with a GPU present the first
  * call per device queries its SM count and cluster occupancy. */

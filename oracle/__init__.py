@@ -50,6 +50,11 @@ def _load():
         lib.tidar_oracle_step_attn.argtypes = [i, i, i, i, i, i, i, ctypes.c_double, P, P, P, i, i,
                                                P, P, P, P, i, P, P, P, i]
         lib.tidar_oracle_step_attn.restype = i
+        lib.tidar_oracle_step_attn_keys.argtypes = [i, i, i, i, i, i, i, ctypes.c_double, P, P, P, i, i,
+                                                    P, P, P, P, i, i, P, P, P, i]
+        lib.tidar_oracle_step_attn_keys.restype = i
+        lib.tidar_oracle_merge.argtypes = [i, ctypes.c_int64, i, P, P, P, P]
+        lib.tidar_oracle_merge.restype = i
         lib.tidar_oracle_append.argtypes = [i, i, i, i, i, i, P, P, P, i, i, P, P, P]
         lib.tidar_oracle_append.restype = i
         lib.tidar_oracle_verify.argtypes = [i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
@@ -100,14 +105,15 @@ def step_key_visible(k: int, row: int, key: int) -> bool:
 
 
 def step_attn(q, k_blk, v_blk, k_pages, v_pages, page_table, seq_lens, k, *, scale=0.0,
-              sel=None, num_threads=0):
+              sel=None, num_threads=0, step_keys=True):
     """Three-zone step attention in fp64.
 
     q [B][R][Hq][D], k_blk/v_blk [B][R][Hkv][D], k_pages/v_pages
     [num_pages][Hkv][page][D] (fp32 or uint16 bf16 bits), page_table
     [B][max_pages] int32, seq_lens [B] int32.  Returns (out, lse): out
     [B][R][Hq][D] and lse [B][R][Hq] (natural log), or [n][D] / [n] for the
-    (b, rho, h) triples in ``sel``.
+    (b, rho, h) triples in ``sel``.  step_keys=False: every row sees only the
+    cache's prefix rows (one slice of a longer sequence; no key: 0 and -inf).
     """
     lib = _load()
     q = np.ascontiguousarray(q)
@@ -131,12 +137,30 @@ def step_attn(q, k_blk, v_blk, k_pages, v_pages, page_table, seq_lens, k, *, sca
         n_sel = sel_arr.shape[0]
         out = np.zeros((n_sel, D), np.float64)
         lse = np.zeros((n_sel,), np.float64)
-    st = lib.tidar_oracle_step_attn(B, Hq, Hkv, D, k, page_size, dt, float(scale), _ptr(k_pages),
-                                    _ptr(v_pages), _ptr(page_table), page_table.shape[1], num_pages,
-                                    _ptr(seq_lens), _ptr(q), _ptr(k_blk), _ptr(v_blk), n_sel,
-                                    _ptr(sel_arr), _ptr(out), _ptr(lse), int(num_threads))
+    st = lib.tidar_oracle_step_attn_keys(B, Hq, Hkv, D, k, page_size, dt, float(scale),
+                                         _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+                                         page_table.shape[1], num_pages, _ptr(seq_lens), _ptr(q),
+                                         _ptr(k_blk), _ptr(v_blk), 1 if step_keys else 0, n_sel,
+                                         _ptr(sel_arr), _ptr(out), _ptr(lse), int(num_threads))
     if st != 0:
         raise ValueError(f"oracle step_attn failed with status {st}")
+    return out, lse
+
+
+def merge(parts_o, parts_lse):
+    """Attention over a union of disjoint key sets from the per-set results:
+    parts_o [nparts][...][D], parts_lse [nparts][...] -> (out [...][D], lse
+    [...]) in fp64 (the log-sum-exp merge)."""
+    po = np.ascontiguousarray(parts_o, dtype=np.float64)
+    pl = np.ascontiguousarray(parts_lse, dtype=np.float64)
+    nparts, D = po.shape[0], po.shape[-1]
+    rows = int(np.prod(pl.shape[1:]))
+    assert po.shape[:-1] == pl.shape
+    out = np.zeros(pl.shape[1:] + (D,), np.float64)
+    lse = np.zeros(pl.shape[1:], np.float64)
+    st = _load().tidar_oracle_merge(nparts, rows, D, _ptr(po), _ptr(pl), _ptr(out), _ptr(lse))
+    if st != 0:
+        raise ValueError(f"oracle merge failed with status {st}")
     return out, lse
 
 

@@ -109,7 +109,7 @@ static int64_t cache_row(const int32_t* page_table, int max_pages, int num_pages
 static int attend_one(int b, int rho, int h, int Hq, int Hkv, int D, int k, int page_size,
                       int dtype, double scale, const void* k_pages, const void* v_pages,
                       const int32_t* page_table, int max_pages, int num_pages, int P,
-                      const void* q, const void* k_blk, const void* v_blk,
+                      const void* q, const void* k_blk, const void* v_blk, int with_step_keys,
                       double* s /* scratch, P + R */, double* out, double* lse) {
   const int R = rows_per_seq(k);
   const int G = Hq / Hkv;
@@ -126,7 +126,7 @@ static int attend_one(int b, int rho, int h, int Hq, int Hkv, int D, int k, int 
     for (d = 0; d < D; ++d) dot += elem(q, qoff + d, dtype) * elem(k_pages, ko + d, dtype);
     s[nkeys++] = dot * scale;
   }
-  for (i = 0; i < R; ++i) {
+  for (i = 0; with_step_keys && i < R; ++i) {
     if (tidar_oracle_step_key_visible(k, rho, i)) {
       int64_t ko = (((int64_t)b * R + i) * Hkv + g) * D;
       double dot = 0.0;
@@ -144,14 +144,14 @@ static int attend_one(int b, int rho, int h, int Hq, int Hkv, int D, int k, int 
     double w = s[nkeys++] / z;
     for (d = 0; d < D; ++d) out[d] += w * elem(v_pages, vo + d, dtype);
   }
-  for (i = 0; i < R; ++i) {
+  for (i = 0; with_step_keys && i < R; ++i) {
     if (tidar_oracle_step_key_visible(k, rho, i)) {
       int64_t vo = (((int64_t)b * R + i) * Hkv + g) * D;
       double w = s[nkeys++] / z;
       for (d = 0; d < D; ++d) out[d] += w * elem(v_blk, vo + d, dtype);
     }
   }
-  *lse = m + log(z);
+  *lse = nkeys > 0 ? m + log(z) : -INFINITY;   /* no key: out = 0, lse = -inf */
   return ORACLE_OK;
 }
 
@@ -165,12 +165,35 @@ static int attend_one(int b, int rho, int h, int Hq, int Hkv, int D, int k, int 
  * into out [n_sel][D], lse [n_sel].  lse is the natural log of the softmax
  * normaliser including the maximum.  scale <= 0 selects 1/sqrt(D).
  */
+int tidar_oracle_step_attn_keys(int B, int Hq, int Hkv, int D, int k, int page_size, int dtype,
+                                double scale, const void* k_pages, const void* v_pages,
+                                const int32_t* page_table, int max_pages, int num_pages,
+                                const int32_t* seq_lens, const void* q, const void* k_blk,
+                                const void* v_blk, int with_step_keys, int n_sel,
+                                const int32_t* sel, double* out, double* lse, int num_threads);
+
 int tidar_oracle_step_attn(int B, int Hq, int Hkv, int D, int k, int page_size, int dtype,
                            double scale, const void* k_pages, const void* v_pages,
                            const int32_t* page_table, int max_pages, int num_pages,
                            const int32_t* seq_lens, const void* q, const void* k_blk,
                            const void* v_blk, int n_sel, const int32_t* sel, double* out,
                            double* lse, int num_threads) {
+  return tidar_oracle_step_attn_keys(B, Hq, Hkv, D, k, page_size, dtype, scale, k_pages, v_pages,
+                                     page_table, max_pages, num_pages, seq_lens, q, k_blk, v_blk, 1,
+                                     n_sel, sel, out, lse, num_threads);
+}
+
+/*
+ * The same with the step keys optional: with_step_keys = 0 restricts every row
+ * to the cache's prefix rows (attention over one slice of a longer sequence's
+ * keys; a row with no key gets out = 0, lse = -inf).
+ */
+int tidar_oracle_step_attn_keys(int B, int Hq, int Hkv, int D, int k, int page_size, int dtype,
+                                double scale, const void* k_pages, const void* v_pages,
+                                const int32_t* page_table, int max_pages, int num_pages,
+                                const int32_t* seq_lens, const void* q, const void* k_blk,
+                                const void* v_blk, int with_step_keys, int n_sel,
+                                const int32_t* sel, double* out, double* lse, int num_threads) {
   const int R = rows_per_seq(k);
   int64_t total, t;
   int Pmax = 0, b, status = ORACLE_OK;
@@ -204,8 +227,8 @@ int tidar_oracle_step_attn(int B, int Hq, int Hkv, int D, int k, int page_size, 
         st = ORACLE_ERR_ARG;
       } else {
         st = attend_one(bb, rho, h, Hq, Hkv, D, k, page_size, dtype, scale, k_pages, v_pages,
-                        page_table, max_pages, num_pages, seq_lens[bb], q, k_blk, v_blk, s,
-                        out + t * D, lse + t);
+                        page_table, max_pages, num_pages, seq_lens[bb], q, k_blk, v_blk,
+                        with_step_keys, s, out + t * D, lse + t);
       }
       if (st != ORACLE_OK) {
 #ifdef _OPENMP
@@ -217,6 +240,38 @@ int tidar_oracle_step_attn(int B, int Hq, int Hkv, int D, int k, int page_size, 
     free(s);
   }
   return status;
+}
+
+/*
+ * Attention over a union of disjoint key sets from the attention over each
+ * set: softmax over the union is the mixture of the per-set softmaxes, each set
+ * weighted by its normaliser exp(lse_r).  With M = max_r lse_r and
+ * w_r = exp(lse_r - M) (0 when lse_r = -inf):
+ *   out = sum_r w_r o_r / sum_r w_r,   lse = M + log(sum_r w_r).
+ * parts_o [nparts][rows][D], parts_lse [nparts][rows] (fp64) -> out [rows][D],
+ * lse [rows].  All parts -inf: out = 0, lse = -inf.
+ */
+int tidar_oracle_merge(int nparts, int64_t rows, int D, const double* parts_o, const double* parts_lse,
+                       double* out, double* lse) {
+  int64_t i;
+  int r, d;
+  if (nparts <= 0 || rows < 0 || D <= 0) return ORACLE_ERR_ARG;
+  for (i = 0; i < rows; ++i) {
+    double M = -INFINITY, z = 0.0;
+    for (r = 0; r < nparts; ++r) if (parts_lse[(int64_t)r * rows + i] > M) M = parts_lse[(int64_t)r * rows + i];
+    for (d = 0; d < D; ++d) out[i * D + d] = 0.0;
+    if (M == -INFINITY) { lse[i] = -INFINITY; continue; }
+    for (r = 0; r < nparts; ++r) {
+      const double l = parts_lse[(int64_t)r * rows + i];
+      const double w = l == -INFINITY ? 0.0 : exp(l - M);
+      z += w;
+      if (w != 0.0)
+        for (d = 0; d < D; ++d) out[i * D + d] += w * parts_o[((int64_t)r * rows + i) * D + d];
+    }
+    for (d = 0; d < D; ++d) out[i * D + d] /= z;
+    lse[i] = M + log(z);
+  }
+  return ORACLE_OK;
 }
 
 /*

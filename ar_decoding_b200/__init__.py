@@ -85,7 +85,7 @@ def lib():
         L.tidar_step_attn_workspace_bytes.restype = S
         L.tidar_step_attn.argtypes = [P, P, P, P, P, P, P, P, S, P]
         L.tidar_step_attn.restype = ctypes.c_int
-        L.tidar_step_attn_plan.argtypes = [P, P, P]
+        L.tidar_step_attn_plan.argtypes = [P, P, P, P]
         L.tidar_step_attn_plan.restype = ctypes.c_int
         L.tidar_verify_workspace_bytes.argtypes = [I, I, I, ctypes.c_int]
         L.tidar_verify_workspace_bytes.restype = S
@@ -121,9 +121,13 @@ def lib():
         L.tidar_step_attn_part.restype = ctypes.c_int
         L.tidar_merge_attn.argtypes = [I, ctypes.c_int64, I, ctypes.c_int, P, P, P, P, P]
         L.tidar_merge_attn.restype = ctypes.c_int
-        L.tidar_linear.argtypes = [I, I, I, ctypes.c_int, P, P, P, P]
+        L.tidar_linear_workspace_bytes.argtypes = [I, I, I]
+        L.tidar_linear_workspace_bytes.restype = S
+        L.tidar_linear.argtypes = [I, I, I, ctypes.c_int, P, P, P, P, S, P]
         L.tidar_linear.restype = ctypes.c_int
-        L.tidar_qkv_rope.argtypes = [P, I, P, P, P, ctypes.c_float, P, P, P, P]
+        L.tidar_qkv_rope_workspace_bytes.argtypes = [P, I]
+        L.tidar_qkv_rope_workspace_bytes.restype = S
+        L.tidar_qkv_rope.argtypes = [P, I, P, P, P, ctypes.c_float, P, P, P, P, S, P]
         L.tidar_qkv_rope.restype = ctypes.c_int
         L.tidar_layer_step_workspace_bytes.argtypes = [P, I]
         L.tidar_layer_step_workspace_bytes.restype = S
@@ -215,10 +219,16 @@ def make_cache_desc(cache, device=None) -> KVCacheDesc:
 
 
 def plan(desc: StepDesc) -> tuple[int, int]:
-    path, splits = ctypes.c_int32(), ctypes.c_int32()
-    _check(lib().tidar_step_attn_plan(ctypes.byref(desc), ctypes.byref(path), ctypes.byref(splits)),
-           "tidar_step_attn_plan")
-    return path.value, splits.value
+    """(kernel family, KV splits) of the launch plan."""
+    return plan_full(desc)[:2]
+
+
+def plan_full(desc: StepDesc) -> tuple[int, int, int]:
+    """(kernel family, KV splits, merge: 0 one split, 1 in the kernel, 2 a second launch)."""
+    path, splits, merge = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().tidar_step_attn_plan(ctypes.byref(desc), ctypes.byref(path), ctypes.byref(splits),
+                                      ctypes.byref(merge)), "tidar_step_attn_plan")
+    return path.value, splits.value, merge.value
 
 
 def step_attn_workspace_bytes(desc: StepDesc) -> int:
@@ -254,7 +264,19 @@ def step_attn(q, k_blk, v_blk, cache, k, *, max_prefix_len, scale=0.0, path="aut
     return out, lse
 
 
-def linear(x, w, *, out=None, stream=None):
+def _scratch(need, workspace, dev):
+    """A workspace of at least `need` bytes on `dev` (allocated when None)."""
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _devopt(workspace, "workspace", None, dev)
+    return workspace, (workspace.numel() * workspace.element_size() if workspace is not None else 0)
+
+
+def linear_workspace_bytes(rows: int, out_features: int, in_features: int) -> int:
+    return int(lib().tidar_linear_workspace_bytes(int(rows), int(out_features), int(in_features)))
+
+
+def linear(x, w, *, out=None, workspace=None, stream=None):
     """y = x w^T (bf16; x [rows][in], w [out][in]) on the tensor cores."""
     _dev(x, "x", torch.bfloat16)
     _dev(w, "w", torch.bfloat16, x.device)
@@ -268,8 +290,9 @@ def linear(x, w, *, out=None, stream=None):
     if out.numel() != rows * N:
         raise ValueError(f"out has {out.numel()} elements, expected {rows} x {N}")
     _dev(out, "out", torch.bfloat16, x.device)
-    _check(lib().tidar_linear(rows, N, K, BF16, _ptr(x), _ptr(w), _ptr(out), _stream_handle(stream)),
-           "tidar_linear")
+    ws, wbytes = _scratch(linear_workspace_bytes(rows, N, K) if rows else 0, workspace, x.device)
+    _check(lib().tidar_linear(rows, N, K, BF16, _ptr(x), _ptr(w), _ptr(out), _ptr(ws), wbytes,
+                              _stream_handle(stream)), "tidar_linear")
     return out
 
 
@@ -283,7 +306,7 @@ def _layer_desc(x, k, Hq, Hkv, max_prefix_len, page_size=64, path="auto"):
 
 
 def qkv_rope(x, w_qkv, seq_lens, k, num_q_heads, num_kv_heads, *, max_prefix_len,
-             rope_base=10000.0, out=None, stream=None):
+             rope_base=10000.0, out=None, workspace=None, stream=None):
     """Query/key/value projection of the step rows x [B][R][d_model] with the
     rotary embedding at their zone positions.  Returns (q, k_blk, v_blk)."""
     _dev(x, "x", torch.bfloat16)
@@ -302,9 +325,10 @@ def qkv_rope(x, w_qkv, seq_lens, k, num_q_heads, num_kv_heads, *, max_prefix_len
     for name, t in zip(("q", "k_blk", "v_blk"), out):
         _dev(t, name, torch.bfloat16, dev)
     q, kb, vb = out
+    ws, wbytes = _scratch(int(lib().tidar_qkv_rope_workspace_bytes(ctypes.byref(desc), dm)), workspace, dev)
     _check(lib().tidar_qkv_rope(ctypes.byref(desc), dm, _ptr(x), _ptr(w_qkv), _ptr(seq_lens),
-                                float(rope_base), _ptr(q), _ptr(kb), _ptr(vb), _stream_handle(stream)),
-           "tidar_qkv_rope")
+                                float(rope_base), _ptr(q), _ptr(kb), _ptr(vb), _ptr(ws), wbytes,
+                                _stream_handle(stream)), "tidar_qkv_rope")
     return q, kb, vb
 
 

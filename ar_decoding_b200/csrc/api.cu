@@ -113,7 +113,7 @@ struct Plan {
   int path;    // 1 SIMT, 2 TC05, 3 DEC, 4 PAIR
   int nsplit;
   int keys_per_split;
-  bool cluster_merge;   // TC05: splits merged on chip in one cluster (no partials, no finalize)
+  bool cluster_merge;   // splits of a tile form one cluster and merge in the attention kernel
 };
 
 // Key ranges are multiples of 128 keys (64 on the decode path).  SIMT: aim for
@@ -178,12 +178,12 @@ Plan make_plan(const tidar_step_desc* d, int path) {
   // Tensor-core and decode paths (one CTA per SM): choose the split count by a
   // cost model in units of 128-key blocks per CTA -- the waves of CTAs the
   // launch needs times (the keys of one split + a fixed per-CTA cost), plus
-  // the second launch when splits merge through workspace partials.  A merge
-  // on chip needs a cluster of nsplit CTAs; its waves count the clusters that
-  // can be resident at once.
+  // the merge: a second launch, or (the splits of a tile forming a cluster of
+  // nsplit CTAs) a merge from L2 at the end of the attention kernel, whose
+  // waves count the clusters that can be resident at once.
   // A launch that already fills the device (units >= one wave) keeps one split:
   // with ragged batches the longest sequence, not the wave count, sets its time.
-  constexpr double kFixedBlocks = 3.0, kFinalizeBlocks = 2.0;
+  constexpr double kFixedBlocks = 3.0, kFinalizeBlocks = 2.0, kClusterMergeBlocks = 1.0;
   double best = 1e300;
   int best_n = 1;
   bool best_cluster = false;
@@ -202,7 +202,7 @@ Plan make_plan(const tidar_step_desc* d, int path) {
                                      : (path == 4 ? tidar::pair_resident_clusters(p.nsplit)
                                                   : tidar::dec_resident_clusters(p.nsplit, M));
       if (resident > 0) {
-        const double cost_c = (double)((units + resident - 1) / resident) * per;
+        const double cost_c = (double)((units + resident - 1) / resident) * per + kClusterMergeBlocks;
         if (cost_c < best) { best = cost_c; best_n = n; best_cluster = true; }
       }
     }
@@ -238,7 +238,8 @@ const char* tidar_status_string(tidar_status s) {
 
 const char* tidar_last_cuda_error(void) { return g_cuda_msg; }
 
-tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, int32_t* splits) {
+tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, int32_t* splits,
+                                  int32_t* merge) {
   tidar_status st = check_desc(desc);
   if (st != TIDAR_OK) return st;
   const int pth = choose_path(desc);
@@ -247,6 +248,7 @@ tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, in
   const Plan p = make_plan(desc, pth);
   if (path) *path = p.path;
   if (splits) *splits = p.nsplit;
+  if (merge) *merge = p.nsplit <= 1 ? 0 : (p.cluster_merge ? 1 : 2);
   return TIDAR_OK;
 }
 
@@ -254,7 +256,7 @@ size_t tidar_step_attn_workspace_bytes(const tidar_step_desc* d) {
   if (check_desc(d) != TIDAR_OK) return 0;
   const int pth = choose_path(d);
   const Plan p = make_plan(d, pth);
-  if (p.nsplit <= 1 || p.cluster_merge) return 0;     // merged on chip
+  if (p.nsplit <= 1) return 0;                        // one split: nothing to merge
   const size_t rows = (size_t)d->batch * tidar::rows_per_seq(d->k) * d->num_q_heads;
   return align256((size_t)p.nsplit * rows * d->head_dim * sizeof(float)) +
          align256((size_t)p.nsplit * rows * sizeof(float));
@@ -303,7 +305,8 @@ tidar_status step_attn_impl(const tidar_step_desc* d, const tidar_kv_cache* c, c
   a.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->head_dim);
   a.step_keys = step_keys;
   a.append = append;
-  if (p.nsplit > 1 && !p.cluster_merge) {
+  a.cluster_merge = p.cluster_merge ? 1 : 0;
+  if (p.nsplit > 1) {
     const size_t rows = (size_t)a.B * a.R * a.Hq;
     a.part_o = static_cast<float*>(workspace);
     a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -556,16 +559,27 @@ tidar_status tidar_reserve(const tidar_step_desc* d, const tidar_kv_cache* c,
   return TIDAR_OK;
 }
 
+size_t tidar_linear_workspace_bytes(int32_t rows, int32_t out_features, int32_t in_features) {
+  if (rows <= 0 || out_features <= 0 || in_features <= 0) return 0;
+  const tidar::LinearPlan p = tidar::plan_linear(rows, in_features, out_features);
+  return p.ok ? p.ws_bytes : 0;
+}
+
 tidar_status tidar_linear(int32_t rows, int32_t out_features, int32_t in_features, tidar_dtype dtype,
-                          const void* x, const void* w, void* y, tidar_stream_t stream) {
+                          const void* x, const void* w, void* y, void* workspace, size_t workspace_bytes,
+                          tidar_stream_t stream) {
   if (rows < 0 || out_features <= 0 || in_features <= 0) return TIDAR_ERR_INVALID_ARG;
   if (dtype != TIDAR_BF16 || in_features % 64 || out_features % 128) return TIDAR_ERR_UNSUPPORTED;
   if (rows == 0) return TIDAR_OK;
   if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y)) return TIDAR_ERR_INVALID_ARG;
-  if (!tidar::plan_linear(rows, in_features, out_features).ok) return TIDAR_ERR_UNSUPPORTED;
+  const tidar::LinearPlan p = tidar::plan_linear(rows, in_features, out_features);
+  if (!p.ok) return TIDAR_ERR_UNSUPPORTED;
+  if (workspace_bytes < p.ws_bytes || (p.ws_bytes && !workspace) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return TIDAR_ERR_INVALID_ARG;
   tidar::LinearArgs a{};
   a.T = rows; a.K = in_features; a.N = out_features; a.mode = 0;
-  a.x = x; a.w = w; a.y = y;
+  a.x = x; a.w = w; a.y = y; a.ws = workspace;
   tidar_status st = error_word(&a.err);
   if (st != TIDAR_OK) return st;
   const cudaError_t e = tidar::launch_linear(a, reinterpret_cast<cudaStream_t>(stream));
@@ -574,9 +588,16 @@ tidar_status tidar_linear(int32_t rows, int32_t out_features, int32_t in_feature
   return TIDAR_OK;
 }
 
+size_t tidar_qkv_rope_workspace_bytes(const tidar_step_desc* d, int32_t d_model) {
+  if (check_desc(d) != TIDAR_OK || d_model <= 0 || d->batch <= 0) return 0;
+  const long long T = (long long)d->batch * tidar::rows_per_seq(d->k);
+  if (T > 0x7fffffffLL) return 0;
+  return tidar_linear_workspace_bytes((int32_t)T, (d->num_q_heads + 2 * d->num_kv_heads) * 128, d_model);
+}
+
 tidar_status tidar_qkv_rope(const tidar_step_desc* d, int32_t d_model, const void* x, const void* w_qkv,
                             const int32_t* seq_lens, float rope_base, void* q, void* k_blk, void* v_blk,
-                            tidar_stream_t stream) {
+                            void* workspace, size_t workspace_bytes, tidar_stream_t stream) {
   tidar_status st = check_desc(d);
   if (st != TIDAR_OK) return st;
   if (d_model <= 0 || !(rope_base > 1.0f)) return TIDAR_ERR_INVALID_ARG;
@@ -589,9 +610,13 @@ tidar_status tidar_qkv_rope(const tidar_step_desc* d, int32_t d_model, const voi
   const long long T = (long long)d->batch * R;
   if (T > 0x7fffffffLL) return TIDAR_ERR_UNSUPPORTED;
   const int N = (d->num_q_heads + 2 * d->num_kv_heads) * 128;
-  if (!tidar::plan_linear((int)T, d_model, N).ok) return TIDAR_ERR_UNSUPPORTED;
+  const tidar::LinearPlan p = tidar::plan_linear((int)T, d_model, N);
+  if (!p.ok) return TIDAR_ERR_UNSUPPORTED;
+  if (workspace_bytes < p.ws_bytes || (p.ws_bytes && !workspace) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return TIDAR_ERR_INVALID_ARG;
   tidar::LinearArgs a{};
-  a.T = (int)T; a.K = d_model; a.N = N; a.mode = 1;
+  a.T = (int)T; a.K = d_model; a.N = N; a.mode = 1; a.ws = workspace;
   a.x = x; a.w = w_qkv; a.q = q; a.k_blk = k_blk; a.v_blk = v_blk; a.seq_lens = seq_lens;
   a.Hq = d->num_q_heads; a.Hkv = d->num_kv_heads; a.R = R; a.k = d->k; a.max_prefix = d->max_prefix_len;
   a.log2_base = log2((double)rope_base);
@@ -606,19 +631,23 @@ tidar_status tidar_qkv_rope(const tidar_step_desc* d, int32_t d_model, const voi
 
 namespace {
 // Byte offsets of the layer step's workspace: q, k_blk, v_blk, attention
-// output, then the step attention's own workspace.
+// output, the projections' split partials (the two projections run one after
+// the other and share them), then the step attention's own workspace.
 struct LayerWs {
-  size_t q, kb, vb, o, attn, total;
+  size_t q, kb, vb, o, lin, attn, total;
 };
-LayerWs layer_ws(const tidar_step_desc* d) {
+LayerWs layer_ws(const tidar_step_desc* d, int d_model) {
   LayerWs w{};
   const size_t rows = (size_t)d->batch * tidar::rows_per_seq(d->k);
   const size_t qb = rows * d->num_q_heads * 128 * 2, kvb = rows * d->num_kv_heads * 128 * 2;
+  const size_t lin_qkv = tidar_qkv_rope_workspace_bytes(d, d_model);
+  const size_t lin_o = tidar_linear_workspace_bytes((int32_t)rows, d_model, d->num_q_heads * 128);
   w.q = 0;
   w.kb = w.q + align256(qb);
   w.vb = w.kb + align256(kvb);
   w.o = w.vb + align256(kvb);
-  w.attn = w.o + align256(qb);
+  w.lin = w.o + align256(qb);
+  w.attn = w.lin + align256(lin_qkv > lin_o ? lin_qkv : lin_o);
   w.total = w.attn + align256(tidar_step_attn_workspace_bytes(d));
   return w;
 }
@@ -628,7 +657,7 @@ extern "C" {
 
 size_t tidar_layer_step_workspace_bytes(const tidar_step_desc* d, int32_t d_model) {
   if (check_desc(d) != TIDAR_OK || d_model <= 0) return 0;
-  return layer_ws(d).total;
+  return layer_ws(d, d_model).total;
 }
 
 tidar_status tidar_layer_step(const tidar_step_desc* d, const tidar_kv_cache* c, int32_t d_model,
@@ -642,18 +671,20 @@ tidar_status tidar_layer_step(const tidar_step_desc* d, const tidar_kv_cache* c,
   if (d->batch == 0) return TIDAR_OK;
   if ((st = check_cache(d, c)) != TIDAR_OK) return st;
   if (!w_o || !y || !aligned16(w_o) || !aligned16(y)) return TIDAR_ERR_INVALID_ARG;
-  const LayerWs w = layer_ws(d);
+  const LayerWs w = layer_ws(d, d_model);
   if (workspace_bytes < w.total || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return TIDAR_ERR_INVALID_ARG;
   char* ws = static_cast<char*>(workspace);
   const int rows = d->batch * tidar::rows_per_seq(d->k);
   if (!tidar::plan_linear(rows, d->num_q_heads * 128, d_model).ok) return TIDAR_ERR_UNSUPPORTED;
-  st = tidar_qkv_rope(d, d_model, x, w_qkv, c->seq_lens, rope_base, ws + w.q, ws + w.kb, ws + w.vb, stream);
+  st = tidar_qkv_rope(d, d_model, x, w_qkv, c->seq_lens, rope_base, ws + w.q, ws + w.kb, ws + w.vb,
+                      ws + w.lin, w.attn - w.lin, stream);
   if (st != TIDAR_OK) return st;
   st = tidar_step_attn(d, c, ws + w.q, ws + w.kb, ws + w.vb, ws + w.o, lse_out, ws + w.attn,
                        workspace_bytes - w.attn, stream);
   if (st != TIDAR_OK) return st;
-  return tidar_linear(rows, d_model, d->num_q_heads * 128, TIDAR_BF16, ws + w.o, w_o, y, stream);
+  return tidar_linear(rows, d_model, d->num_q_heads * 128, TIDAR_BF16, ws + w.o, w_o, y, ws + w.lin,
+                      w.attn - w.lin, stream);
 }
 
 tidar_status tidar_debug_set(tidar_debug_knob knob, int32_t value) {

@@ -617,7 +617,7 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (threadIdx.x == 32) DEC_TRACE(154);
   }
 
-  if (split == 0 && len_ok && !a.part_o && a.append) {
+  if (split == 0 && len_ok && (a.nsplit == 1 || a.cluster_merge) && a.append) {
     // ---------------------------------------------------------------- append
     // Draft rows D_1..D_n of KV head g into cache rows P .. P+n-1 (the step
     // keys above were read from k_blk / v_blk, not from the cache).
@@ -704,7 +704,7 @@ cudaError_t launch_attn_dec(const AttnArgs& a, cudaStream_t s) {
   prm.a = a;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
   prm.M = M;
-  prm.cluster = a.nsplit > 1 && !a.part_o;
+  prm.cluster = a.nsplit > 1 && a.cluster_merge;
   if (prm.cluster && a.nsplit > kMaxCluster) return cudaErrorNotSupported;
   CUtensorMap tq, tkp, tvp, tks, tvs;
   {

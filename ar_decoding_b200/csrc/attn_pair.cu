@@ -37,10 +37,10 @@
 //   warps 10, 11 only the split merge and the draft-row append.
 // The last split also runs the step-key windows holding keys visible to
 // either tile, with the zone mask applied in the softmax.  Key splits of one
-// (b, g, pair) merge on chip through a thread-block cluster (each CTA leaves
-// its normalised partial O and lse in its idle K/V rings; CTA `rank` merges a
-// share of the rows over distributed shared memory), or go to workspace
-// partials when the clusters of a launch cannot all be resident.
+// (b, g, pair) write their normalised partial O and lse to the workspace and
+// either merge in this kernel (the splits form a thread-block cluster; after
+// a cluster barrier CTA `rank` merges a share of the rows from L2) or leave
+// the merge to a finalize launch.
 // Every mbarrier wait is bounded (~1 s): on expiry the CTA records
 // TIDAR_DEVERR_TIMEOUT, stops issuing, drains what it issued, frees TMEM and
 // exits through the same cluster barriers as the other CTAs.
@@ -83,9 +83,6 @@ static_assert(kPSmem <= 232448, "shared memory budget");
 // split merge receive area, in the K/V rings once they are idle: [slot][split]
 // [32 float4] fp32 partial rows for at most 256 + 16 (slot, split) pairs, then
 // their lse
-constexpr uint32_t kPOffPart = kPOffK;
-constexpr uint32_t kPOffPartL = kPOffPart + 272 * 512;
-static_assert(kPOffPartL + 272 * 4 <= kPOffBar, "split partials fit the rings");
 
 constexpr uint32_t kPTmemCols = 512;
 __device__ __forceinline__ uint32_t pcol_s(int t) { return 128u * (uint32_t)t; }
@@ -128,7 +125,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t sb = smem_u32(smem);
   const AttnArgs& a = prm.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool cluster = a.nsplit > 1 && !a.part_o;
+  const bool cluster = a.nsplit > 1 && a.cluster_merge;
   // A CTA whose layout check fails does no work but still meets its cluster.
   const bool layout_ok = (sb & 1023u) == 0;
   const int pair = blockIdx.x, split = blockIdx.y;
@@ -512,12 +509,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   }
 
-  // The producer has drained, every MMA is complete and no copy is in flight:
-  // the K/V rings are free for the split merge.
+  // The producer has drained, every MMA is complete and no copy is in flight.
   fence_before();
   __syncthreads();
 
-  if (a.nsplit > 1 && a.part_o) {
+  if (a.nsplit > 1) {
     // ---------------------------------------------------------------- split partials
     if (warp < 8) {
       const int t = warp >> 2, r = threadIdx.x & 127;
@@ -532,44 +528,24 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         a.part_lse[prow] = owrite ? olse : -INFINITY;
       }
     }
-  } else if (cluster) {
-    // ---------------------------------------------------------------- split merge
-    // Row i = t * 128 + r of the pair is owned by CTA i % ns (slot i / ns).
-    // Once every CTA is past its main loop (first barrier: the K/V rings are
-    // idle) each softmax thread pushes its row's normalised partial O and lse
-    // into the owner's rings; after the second barrier the owners merge their
-    // rows locally.
-    const int ns = a.nsplit;
-    const uint32_t rank = cluster_rank();
-    float* recv = reinterpret_cast<float*>(smem + kPOffPart);        // [slot][split][32 float4]
-    float* recv_l = reinterpret_cast<float*>(smem + kPOffPartL);     // [slot][split]
-    cluster_sync_all();
-    if (warp < 8) {
-      const int t = warp >> 2, r = threadIdx.x & 127;
-      if (r < rows_valid[t]) {
-        const int i = t * 128 + r;
-        const uint32_t owner = (uint32_t)(i % ns);
-        const int slot = i / ns;
-        if (owrite) {
-          const uint32_t dst = mapa(smem_u32(recv) + 16u * (uint32_t)((slot * ns + split) * 32), owner);
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            st_cluster_f32x4(dst + 16u * c, make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]));
-        }
-        st_cluster_f32(mapa(smem_u32(recv_l) + 4u * (uint32_t)(slot * ns + split), owner), owrite ? olse : -INFINITY);
-      }
+    if (cluster) {
+      // -------------------------------------------------------------- split merge
+      // Row i = t * 128 + r of the pair is merged by CTA i % ns once every
+      // split has written its partials (the cluster barrier), from L2.
+      const int ns = a.nsplit;
+      const int rank = (int)cluster_rank();
+      cluster_sync_all();
+      const int owned = (256 - rank + ns - 1) / ns;
+      merge_l2_rows(a.part_o, a.part_lse, (long long)a.B * a.R * a.Hq, ns, owned,
+                    [&](int sl) -> long long {
+                      const int i = sl * ns + rank;
+                      const int t = i >> 7, rr = i & 127;
+                      if (t >= ntile || rr >= rows_valid[t]) return -1;
+                      const int rho = rho0[t] + rr / a.G, h = g * a.G + rr % a.G;
+                      return (long long)(b * a.R + rho) * a.Hq + h;
+                    },
+                    static_cast<__nv_bfloat16*>(a.out), a.lse_out);
     }
-    cluster_sync_all();
-    const int slots = (256 - (int)rank + ns - 1) / ns;
-    merge_pushed_rows(recv, recv_l, slots, ns, warp, kPThreads / 32, lane,
-                      [&](int sl) -> long long {
-                        const int i = sl * ns + (int)rank;
-                        const int t = i >> 7, rr = i & 127;
-                        if (t >= ntile || rr >= rows_valid[t]) return -1;
-                        const int rho = rho0[t] + rr / a.G, h = g * a.G + rr % a.G;
-                        return (long long)(b * a.R + rho) * a.Hq + h;
-                      },
-                      static_cast<__nv_bfloat16*>(a.out), a.lse_out);
   }
 
   if (nb == 0 && layout_ok && a.nsplit == 1 && warp < 8) {
@@ -585,7 +561,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   }
 
-  if (pair == 0 && split == 0 && len_ok && !a.part_o && a.append) {
+  if (pair == 0 && split == 0 && len_ok && (a.nsplit == 1 || cluster) && a.append) {
     // ---------------------------------------------------------------- append
     // Draft rows D_1..D_n of KV head g into cache rows P .. P+n-1 (the keys
     // above read them from k_blk / v_blk, not from the cache).
@@ -672,9 +648,11 @@ cudaError_t launch_attn_pair(const AttnArgs& a, cudaStream_t s) {
   }
   cudaError_t e = pair_smem_attr();
   if (e != cudaSuccess) return e;
-  if (a.nsplit > 1 && !a.part_o && a.nsplit > kMaxCluster) return cudaErrorNotSupported;
+  if (a.nsplit > 1 && (!a.part_o || !a.part_lse)) return cudaErrorInvalidValue;   // partials are staged
+  const bool clu = a.nsplit > 1 && a.cluster_merge;
+  if (clu && a.nsplit > kMaxCluster) return cudaErrorNotSupported;
   const dim3 grid(prm.pairs, a.nsplit, a.B * a.Hkv);
-  const dim3 cluster(1, a.part_o ? 1 : a.nsplit, 1);
+  const dim3 cluster(1, clu ? a.nsplit : 1, 1);
   return launch_clustered(attn_pair_kernel, grid, cluster, kPThreads, kPSmem, s, tq, tkp, tvp, tks, tvs, prm);
 }
 

@@ -32,6 +32,10 @@
 //                32 columns of its own 64).  O_t is rescaled only when the
 //                row maximum grows by more than 2^8.  The epilogue merges the
 //                two sets and the two halves (max, sums, O) and writes O / l.
+// Key splits of one (b, g, tile) write their normalised partial O and lse to
+// the workspace; with cluster_merge they form one thread-block cluster and
+// merge in this kernel (from L2, after a cluster barrier), else a finalize
+// launch merges them.
 // Every mbarrier wait is bounded: on expiry the CTA records TIDAR_DEVERR_TIMEOUT,
 // stops issuing, drains what it issued (bounded), frees TMEM and exits.
 #include <cuda.h>
@@ -589,15 +593,13 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     olse = lse;
   }
 
-  // The producer has drained, every MMA is complete and no copy is in flight:
-  // the K ring is free for the split merge.
+  // The producer has drained, every MMA is complete and no copy is in flight.
   fence_before();
   __syncthreads();
 
-  if (a.nsplit > 1 && a.part_o) {
+  if (a.nsplit > 1) {
     // ---------------------------------------------------------------- split partials
-    // Too many splits for one wave of clusters: this split's normalised O and
-    // lse go to the workspace and the finalize launch merges them.
+    // This split's normalised O rows and their lse go to the workspace.
     if (warp >= 2) {
       const int r = 32 * (warp & 3) + lane;
       const int t = (warp - 2) >> 3, hf = ((warp - 2) >> 2) & 1;
@@ -612,44 +614,24 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (t == 0 && hf == 0) a.part_lse[prow] = owrite ? olse : -INFINITY;
       }
     }
-  } else if (a.nsplit > 1) {
-    // ---------------------------------------------------------------- split merge
-    // The CTAs of this cluster are the splits of one (b, g, tile).  Row r is
-    // owned by CTA r % ns (slot r / ns).  Once every CTA is past its main loop
-    // (first barrier: the K rings are idle) each thread pushes its 32 columns
-    // of normalised partial O and the row's lse into the owner's K ring; after
-    // the second barrier the owners merge their rows locally.
-    const int ns = a.nsplit;
-    const uint32_t rank = cluster_rank();
-    float* recv = reinterpret_cast<float*>(smem + kOffK);            // [slot][split][32 float4]
-    float* recv_l = reinterpret_cast<float*>(smem + kOffK + 144 * 512);   // [slot][split]
-    cluster_sync_all();
-    if (warp >= 2) {
-      const int r = 32 * (warp & 3) + lane;
-      const int t = (warp - 2) >> 3, hf = ((warp - 2) >> 2) & 1;
-      const int c0 = 8 * (2 * t + hf);                   // first float4 chunk of this thread
-      if (r < rows_valid) {
-        const uint32_t owner = (uint32_t)(r % ns);
-        const int slot = r / ns;
-        if (owrite) {
-          const uint32_t dst = mapa(smem_u32(recv) + 16u * (uint32_t)((slot * ns + split) * 32 + c0), owner);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_cluster_f32x4(dst + 16u * c, make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]));
-        }
-        if (t == 0 && hf == 0)
-          st_cluster_f32(mapa(smem_u32(recv_l) + 4u * (uint32_t)(slot * ns + split), owner), owrite ? olse : -INFINITY);
-      }
+    if (a.cluster_merge) {
+      // -------------------------------------------------------------- split merge
+      // The CTAs of this cluster are the splits of one (b, g, tile).  Once all
+      // of them have written their partials (the cluster barrier), CTA j
+      // merges rows j, j + ns, j + 2 ns, ... of the tile from L2.  Without
+      // cluster_merge a finalize launch does this.
+      const int ns = a.nsplit;
+      const int rank = (int)cluster_rank();
+      cluster_sync_all();
+      const int owned = rows_valid > rank ? (rows_valid - rank + ns - 1) / ns : 0;
+      merge_l2_rows(a.part_o, a.part_lse, (long long)a.B * a.R * a.Hq, ns, owned,
+                    [&](int i) -> long long {
+                      const int r = i * ns + rank;
+                      const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
+                      return (long long)(b * a.R + rho) * a.Hq + h;
+                    },
+                    static_cast<__nv_bfloat16*>(a.out), a.lse_out);
     }
-    cluster_sync_all();
-    const int slots = (rows_valid - (int)rank + ns - 1) / ns;
-    merge_pushed_rows(recv, recv_l, slots > 0 ? slots : 0, ns, warp, kThreads / 32, lane,
-                      [&](int sl) -> long long {
-                        const int R = sl * ns + (int)rank;
-                        const int rho = rho0 + R / a.G, h = g * a.G + R % a.G;
-                        return (long long)(b * a.R + rho) * a.Hq + h;
-                      },
-                      static_cast<__nv_bfloat16*>(a.out), a.lse_out);
   }
 
   if (bp.nb == 0 && a.nsplit == 1 && warp >= 2) {
@@ -666,7 +648,7 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   }
 
-  if (tile == 0 && split == 0 && len_ok && !a.part_o && a.append) {
+  if (tile == 0 && split == 0 && len_ok && (a.nsplit == 1 || a.cluster_merge) && a.append) {
     // ---------------------------------------------------------------- append
     // Draft rows D_1..D_n of KV head g into cache rows P .. P+n-1 (the keys
     // above read them from k_blk / v_blk, not from the cache).
@@ -762,10 +744,12 @@ cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s) {
   }
   cudaError_t e = set_smem_attr();
   if (e != cudaSuccess) return e;
-  if (a.nsplit > 1 && !a.part_o && a.nsplit > kMaxCluster) return cudaErrorNotSupported;
+  if (a.nsplit > 1 && (!a.part_o || !a.part_lse)) return cudaErrorInvalidValue;   // partials are staged
+  const bool clu = a.nsplit > 1 && a.cluster_merge;
+  if (clu && a.nsplit > kMaxCluster) return cudaErrorNotSupported;
   const dim3 grid(prm.tiles, a.nsplit, a.B * a.Hkv);
   // with the cluster merge, the splits of one (b, g, tile) form a cluster
-  const dim3 cluster(1, a.part_o ? 1 : a.nsplit, 1);
+  const dim3 cluster(1, clu ? a.nsplit : 1, 1);
   return launch_clustered(attn_tc05_kernel, grid, cluster, kThreads, kSmemAlloc, s, tq, tkp, tvp, tks, tvs,
                           prm);
 }

@@ -39,10 +39,23 @@ constexpr int kCWarps = kCThreads / 32;
 // rows P .. P+n-1 (npm = min(n, ceil(n/ps) + 1)).
 struct SeqRec { int P, c, cnt, off; };
 
+// Optional timeline of CTA 0 (build with -DTIDAR_TRACE; absent from normal
+// builds): [0] start, [1] after the wait on the previous kernel, [2] validated,
+// [3] past the cluster barriers, [4] end.
+#ifdef TIDAR_TRACE
+__device__ unsigned long long g_commit_trace[8];
+#define COMMIT_TRACE(slot) do { if (blockIdx.x == 0 && threadIdx.x == 0) { unsigned long long t_; \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_)); g_commit_trace[(slot)] = t_; } } while (0)
+#else
+#define COMMIT_TRACE(slot) do {} while (0)
+#endif
+
 __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a, int slots, int per,
                                                                     int npm) {
+  COMMIT_TRACE(0);
   pdl_wait();
   pdl_trigger();
+  COMMIT_TRACE(1);
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks();
   const int rank = (int)cl.block_rank();
@@ -86,6 +99,7 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
     }
   }
   __syncthreads();
+  COMMIT_TRACE(2);
   if (wid == 0) {
     int run = 0;
     for (int s0 = 0; s0 < nown; s0 += 32) {
@@ -117,6 +131,7 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
     if (lane == 0) { s_base = sb; s_grand = sg; }
   }
   cl.sync();
+  COMMIT_TRACE(3);
 
   // 3. release and advance (one warp per sequence), then scrub (whole CTA);
   //    no page-table reads from here on
@@ -156,11 +171,18 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
   for (int i = grand + rank * kCThreads + (int)threadIdx.x; i < a.B * slots; i += C * kCThreads)
     a.released[i] = -1;
   if (rank == 0 && threadIdx.x == 0) *a.num_released = grand;
+  COMMIT_TRACE(4);
 }
 
 int commit_npm(int n, int ps) { return min(n, (n + ps - 1) / ps + 1); }
 
 }  // namespace
+
+#ifdef TIDAR_TRACE
+extern "C" int tidar_commit_trace_read(void* dst, size_t bytes) {
+  return (int)cudaMemcpyFromSymbol(dst, g_commit_trace, bytes);
+}
+#endif
 
 // Per owned sequence: a 4-int record and up to 16 page ids, in the dynamic
 // shared memory of the portable cluster of 8 (the worst case) within 200 KB.

@@ -28,13 +28,15 @@ struct AttnArgs {
   float scale;           // softmax scale (natural-log domain)
   int step_keys;         // 1: the last split also attends the step keys (the zone mask); 0: prefix only
   int append;            // 1: write the draft rows' K/V into the cache
+  int cluster_merge;     // nsplit > 1: the splits of a tile are one cluster and merge in the kernel
+                         // (partials through part_o / part_lse in L2); 0: a finalize launch merges
 };
 
 // Warp-MMA kernel for query blocks of at most 16 packed rows per KV head
-// (bf16, D 128, page 64; splits in multiples of 64 keys).  Like the tcgen05
-// kernel it merges its splits on chip through a cluster of nsplit CTAs when
-// part_o == nullptr (and then appends the draft rows itself); with part_o set
-// launch_finalize merges and appends.
+// (bf16, D 128, page 64; splits in multiples of 64 keys).  With cluster_merge
+// its nsplit CTAs form a cluster and merge over distributed shared memory (and
+// the kernel appends the draft rows itself); without it the splits write
+// part_o / part_lse and launch_finalize merges and appends.
 cudaError_t launch_attn_dec(const AttnArgs& a, cudaStream_t s);
 int dec_resident_clusters(int ns, int M);   // M = packed query rows per KV head
 // CUDA-core kernel (fp32 or bf16, D 64 or 128).
@@ -43,9 +45,9 @@ cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 // the tensor maps cannot be built.
 cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s);
 // How many clusters of `ns` tcgen05 attention CTAs (one per key split) this
-// device holds at once; 0 if none.  The kernel merges its splits on chip
-// through such a cluster (part_o == nullptr) and then also performs the
-// draft-row append; with part_o set it writes split partials instead and
+// device holds at once; 0 if none.  The splits always write part_o / part_lse;
+// with cluster_merge they form such a cluster and merge those partials in the
+// kernel (which then also performs the draft-row append), else
 // launch_finalize merges and appends.
 int tc05_resident_clusters(int ns);
 // Tensor-core kernel with two 128-row query tiles per CTA sharing each staged
@@ -150,15 +152,18 @@ struct LinearArgs {
   int Hq, Hkv, R, k, max_prefix;
   double log2_base;
   unsigned int* err;
+  void* ws;          // plan.ws_bytes of device scratch (split partials), 256-byte aligned
 };
 struct LinearPlan {
   bool ok;
   int nt, nsub, tiles, stages, ksplit;
   uint32_t stage_bytes;
   size_t smem;
+  size_t ws_bytes;   // split-K partials and status words (0 with one split)
 };
 // Tile plan of one projection: ok is false for shapes the kernel does not
-// take (K not a multiple of 64, N not a multiple of 128).
+// take (K not a multiple of 64, N not a multiple of 128).  The split count
+// depends on the current device's cluster occupancy (queried once).
 LinearPlan plan_linear(int T, int K, int N);
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s);
 

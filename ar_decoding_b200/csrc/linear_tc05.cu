@@ -17,10 +17,11 @@
 // TMEM lanes), the rows the B operand (N = tokens in the TMEM columns: one MMA
 // of N = tile, or two of N = tile / 2 above 256), so every token count from 1
 // up fills the 128-wide M dimension.  The K ranges of one (feature tile, token
-// tile) form a thread-block cluster; each CTA leaves its fp32 partial sums in
-// its shared memory and, after a cluster barrier, CTA `rank` adds the splits'
-// partials of its share of the tokens over distributed shared memory (in rank
-// order, so the sum is deterministic) and writes them.
+// tile) form a thread-block cluster; each CTA writes its fp32 partial sums to
+// the workspace (they stay in L2) and, after a cluster barrier, CTA `rank`
+// adds the splits' partials of its share of the tokens (in split order, so the
+// sum is deterministic) and writes them.  The split count is the largest
+// whose clusters all fit on the device at once (one wave).
 //
 // Epilogues:
 //   plain   y [T][N] bf16.
@@ -35,10 +36,12 @@
 // Roles (6 warps): warp 0 TMA producer (the weight tiles of the first stages
 // are issued before the wait on the previous kernel: they do not depend on
 // it); warp 1 TMEM owner and MMA issuer; warps 2..5 move the accumulator from
-// TMEM (lane quarter warp % 4) to shared memory; all six warps then reduce
-// and write.  Every mbarrier wait is bounded (~1 s): on expiry the CTA records
-// TIDAR_DEVERR_TIMEOUT, skips the rest of its work but still meets its
-// cluster at both cluster barriers, frees TMEM and exits.
+// TMEM (lane quarter warp % 4) to the workspace (to shared memory with one
+// split); all six warps then reduce and write, one warp per token and several
+// tokens' loads in flight.  Every mbarrier wait is bounded (~1 s): on expiry
+// the CTA records TIDAR_DEVERR_TIMEOUT, skips the rest of its work, marks its
+// partials invalid (the other splits of its cluster then write nothing for
+// the tile), still meets its cluster at the barrier, frees TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -55,6 +58,7 @@ constexpr int kLinMaxStages = 8;
 constexpr uint32_t kLinATile = 128u * 128u;              // 128 features x 64 bf16 (128 B rows)
 constexpr uint32_t kLinSmemBudget = 225u * 1024u;        // ring + barriers, under the 227 KB limit
 constexpr int kLinMaxTile = 288;                         // tokens per CTA (TMEM columns)
+constexpr int kLinMaxSplit = 8;                          // K splits (cluster size)
 
 struct LinParams {
   int T, K, N;        // tokens, reduction length, output features
@@ -73,6 +77,8 @@ struct LinParams {
   int Hq, Hkv, R, kdraft, max_prefix;
   double log2_base;
   unsigned int* err;
+  float* part;        // [tiles][N / 128][ksplit][nt][128] fp32 split partials (ksplit > 1)
+  int* stat;          // [tiles][N / 128][ksplit]: 0 when that split's partials are valid
 };
 
 // Optional timeline of CTA (0, 0, 0) (build with -DTIDAR_TRACE; absent from
@@ -117,6 +123,11 @@ __device__ __forceinline__ void lin_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
 }
+__device__ __forceinline__ uint32_t lin_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 #define LIN_R16(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
     "=r"(r[i + 6]), "=r"(r[i + 7]), "=r"(r[i + 8]), "=r"(r[i + 9]), "=r"(r[i + 10]), "=r"(r[i + 11]),         \
     "=r"(r[i + 12]), "=r"(r[i + 13]), "=r"(r[i + 14]), "=r"(r[i + 15])
@@ -135,6 +146,89 @@ __device__ __forceinline__ long long zone_position(int k, int row, int P) {
   if (k == 0 || row < k) return (long long)P + row;     // d_r (r = row + 1) at P + r - 1
   const int j = (row - k) / k + 1, s = (row - k) % k + 1;
   return (long long)P + j + s - 1;
+}
+
+// (token tile, feature tile) group of a CTA, and the first float of split
+// `split`'s partials in the workspace.
+__device__ __forceinline__ int lin_group(const LinParams& prm, int tt, int ft) { return tt * (prm.N / 128) + ft; }
+__device__ __forceinline__ size_t lin_part_offset(const LinParams& prm, int tt, int ft, int split) {
+  return ((size_t)lin_group(prm, tt, ft) * prm.ksplit + split) * (size_t)prm.nt * 128;
+}
+
+// Sum of the KS splits' partials of tokens [tlo, thi) of the tile and the
+// epilogue.  One warp per token, lane l holding features 4l .. 4l+3; each warp
+// has U tokens' loads (KS float4 each, from L2 -- other SMs wrote them -- or
+// from shared memory with one split) in flight before it adds them in split
+// order.  The rotary pairs (f, f + 64) sit in lanes l and l ^ 16.
+template <int KS>
+__device__ __forceinline__ void lin_reduce(const LinParams& prm, const float* part, int tlo, int thi, int t0,
+                                           int ft, int warp, int lane, const double* invf) {
+  constexpr int U = KS == 1 ? 4 : (KS <= 2 ? 8 : (KS <= 4 ? 4 : 2));
+  constexpr int W = kLinThreads / 32;
+  const size_t split_stride = (size_t)prm.nt * 128;
+  for (int tb = tlo + warp; tb < thi; tb += W * U) {
+    float4 v[U][KS];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = tb + W * u;
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        if (t < thi) {
+          const float4* src = reinterpret_cast<const float4*>(part + s * split_stride + (size_t)t * 128) + lane;
+          v[u][s] = KS == 1 ? *src : __ldcg(src);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = tb + W * u;
+      if (t >= thi) break;                                // warp-uniform
+      float acc[4] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w};
+#pragma unroll
+      for (int s = 1; s < KS; ++s) {
+        acc[0] += v[u][s].x; acc[1] += v[u][s].y; acc[2] += v[u][s].z; acc[3] += v[u][s].w;
+      }
+      const int tg = t0 + t;
+      __nv_bfloat16* dst;
+      if (prm.mode == 0) {
+        dst = static_cast<__nv_bfloat16*>(prm.y) + (size_t)tg * prm.N + ft * 128;
+      } else {
+        const int b = tg / prm.R, row = tg % prm.R;
+        bool rotate = true;
+        if (ft < prm.Hq) {
+          dst = static_cast<__nv_bfloat16*>(prm.q) + ((size_t)tg * prm.Hq + ft) * 128;
+        } else if (ft < prm.Hq + prm.Hkv) {
+          dst = static_cast<__nv_bfloat16*>(prm.kb) + ((size_t)tg * prm.Hkv + (ft - prm.Hq)) * 128;
+        } else {
+          dst = static_cast<__nv_bfloat16*>(prm.vb) + ((size_t)tg * prm.Hkv + (ft - prm.Hq - prm.Hkv)) * 128;
+          rotate = false;
+        }
+        if (rotate) {                                     // warp-uniform
+          int P = prm.seq_lens[b];
+          if (P < 0 || P > prm.max_prefix) {
+            if (lane == 0 && row == 0 && ft == 0 && blockIdx.y == 0) raise_error(prm.err, TIDAR_DEVERR_BAD_LEN);
+            P = 0;
+          }
+          const double pos = (double)zone_position(prm.kdraft, row, P);
+          const bool hi = lane >= 16;                     // features 64 .. 127: the second of each pair
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float other = __shfl_xor_sync(0xffffffffu, acc[e], 16);
+            const double ang = pos * invf[4 * (lane & 15) + e];
+            const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+            float sn, cs;
+            sincosf((float)red, &sn, &cs);
+            // (x_f, x_{f+64}) -> (x_f cos - x_{f+64} sin, x_f sin + x_{f+64} cos)
+            acc[e] = hi ? other * sn + acc[e] * cs : acc[e] * cs - other * sn;
+          }
+        }
+      }
+      uint2 u2;
+      u2.x = lin_bf16x2(acc[0], acc[1]);
+      u2.y = lin_bf16x2(acc[2], acc[3]);
+      *reinterpret_cast<uint2*>(dst + 4 * lane) = u2;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kLinThreads, 1)
@@ -255,7 +349,7 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
       lin_commit(bar(BAR_DONE));
     }
   } else {
-    // ---------------------------------------------------------------- TMEM -> smem
+    // ---------------------------------------------------------------- TMEM -> partials
     pdl_wait();
     pdl_trigger();
     const int q4 = warp & 3;
@@ -265,13 +359,17 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
     if (threadIdx.x == 64) LIN_TRACE(272);
     lin_fence_after();
     if (ok) {
-      float* part = reinterpret_cast<float*>(smem);      // [nt][128]: the ring is idle now
+      // one split: [nt][128] in shared memory (the ring is idle now); several:
+      // this split's slice of the workspace, token-major, so a warp's 32
+      // features of one token are one 128-byte line
+      float* part = prm.ksplit > 1 ? prm.part + lin_part_offset(prm, tt, ft, split) : reinterpret_cast<float*>(smem);
       const uint32_t trow = tmem + ((uint32_t)(32 * q4) << 16);
-      for (int c = 0; c < prm.nt; c += 16) {
+      for (int c = 0; c < nvalid; c += 16) {
         uint32_t r[16];
         lin_tmem_ld16(trow + (uint32_t)c, r);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) part[(c + e) * 128 + f] = __uint_as_float(r[e]);
+        for (int e = 0; e < 16; ++e)
+          if (c + e < nvalid) part[(c + e) * 128 + f] = __uint_as_float(r[e]);
       }
     }
   }
@@ -279,88 +377,40 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
   __syncthreads();
   const bool cta_ok = layout_ok && !*abort_flag;
   if (threadIdx.x == 0) LIN_TRACE(273);
-  // every CTA of the cluster has its partials in shared memory
-  if (prm.ksplit > 1) cluster_sync_all();
+  const int ks = prm.ksplit;
+  if (ks > 1) {
+    // every split's partials and status word are written before any CTA of
+    // the cluster reads them (release / acquire at cluster scope)
+    if (threadIdx.x == 0) prm.stat[lin_group(prm, tt, ft) * ks + split] = cta_ok ? 0 : 1;
+    cluster_sync_all();
+  }
 
   // ------------------------------------------------------------------ reduce + write
-  // CTA `rank` owns tokens [rank * per, (rank + 1) * per) of the tile; one warp
-  // per token, lane l adds features l, l + 32, l + 64, l + 96 over the splits.
-  const int ks = prm.ksplit;
+  // CTA `rank` owns tokens [rank * per, (rank + 1) * per) of the tile.  A
+  // split that timed out or failed its layout check leaves garbage, so every
+  // CTA checks all status words first and writes nothing for the tile if one
+  // is set (the error word already says why).
   const uint32_t rank = ks > 1 ? cluster_rank() : 0u;
   const int per = (nvalid + ks - 1) / ks;
   const int tlo = (int)rank * per, thi = min(nvalid, tlo + per);
-  // a split that timed out contributes garbage: every CTA of the cluster checks
-  // every split's status word before trusting its partials
   bool all_ok = cta_ok;
   if (ks > 1) {
-    for (int r2 = 0; r2 < ks; ++r2) {
-      const uint32_t st = mapa(smem_u32(misc + 1), (uint32_t)r2);
-      int flag;
-      asm volatile("ld.shared::cluster.b32 %0, [%1];" : "=r"(flag) : "r"(st) : "memory");
-      all_ok = all_ok && flag == 0;
-    }
+    const int* st = prm.stat + lin_group(prm, tt, ft) * ks;
+    for (int r2 = 0; r2 < ks; ++r2) all_ok = all_ok && __ldcg(st + r2) == 0;
   }
   if (all_ok) {
-    const uint32_t part_s = sb;
-    for (int t = tlo + warp; t < thi; t += kLinThreads / 32) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int r2 = 0; r2 < ks; ++r2) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t off = 4u * (uint32_t)(t * 128 + lane + 32 * e);
-          float v;
-          if (ks > 1) {
-            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(mapa(part_s + off, (uint32_t)r2)) : "memory");
-          } else {
-            v = reinterpret_cast<const float*>(smem)[t * 128 + lane + 32 * e];
-          }
-          acc[e] += v;
-        }
-      }
-      const int tg = t0 + t;
-      if (prm.mode == 0) {
-        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(prm.y) + (size_t)tg * prm.N + ft * 128;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) y[lane + 32 * e] = __float2bfloat16_rn(acc[e]);
-      } else {
-        const int b = tg / prm.R, row = tg % prm.R;
-        __nv_bfloat16* dst;
-        bool rotate = true;
-        if (ft < prm.Hq) {
-          dst = static_cast<__nv_bfloat16*>(prm.q) + ((size_t)tg * prm.Hq + ft) * 128;
-        } else if (ft < prm.Hq + prm.Hkv) {
-          dst = static_cast<__nv_bfloat16*>(prm.kb) + ((size_t)tg * prm.Hkv + (ft - prm.Hq)) * 128;
-        } else {
-          dst = static_cast<__nv_bfloat16*>(prm.vb) + ((size_t)tg * prm.Hkv + (ft - prm.Hq - prm.Hkv)) * 128;
-          rotate = false;
-        }
-        if (rotate) {
-          int P = prm.seq_lens[b];
-          if (P < 0 || P > prm.max_prefix) {
-            if (lane == 0 && row == 0 && ft == 0 && split == 0) raise_error(prm.err, TIDAR_DEVERR_BAD_LEN);
-            P = 0;
-          }
-          const double pos = (double)zone_position(prm.kdraft, row, P);
-          // pairs (f, f + 64) for f = lane and lane + 32
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const double ang = pos * invf[lane + 32 * h];
-            const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
-            float sn, cs;
-            sincosf((float)red, &sn, &cs);
-            const float a = acc[h], c = acc[h + 2];
-            acc[h] = a * cs - c * sn;
-            acc[h + 2] = a * sn + c * cs;
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[lane + 32 * e] = __float2bfloat16_rn(acc[e]);
-      }
+    switch (ks) {
+      case 1: lin_reduce<1>(prm, reinterpret_cast<const float*>(smem), tlo, thi, t0, ft, warp, lane, invf); break;
+      case 2: lin_reduce<2>(prm, prm.part + lin_part_offset(prm, tt, ft, 0), tlo, thi, t0, ft, warp, lane, invf); break;
+      case 3: lin_reduce<3>(prm, prm.part + lin_part_offset(prm, tt, ft, 0), tlo, thi, t0, ft, warp, lane, invf); break;
+      case 4: lin_reduce<4>(prm, prm.part + lin_part_offset(prm, tt, ft, 0), tlo, thi, t0, ft, warp, lane, invf); break;
+      case 5: lin_reduce<5>(prm, prm.part + lin_part_offset(prm, tt, ft, 0), tlo, thi, t0, ft, warp, lane, invf); break;
+      case 6: lin_reduce<6>(prm, prm.part + lin_part_offset(prm, tt, ft, 0), tlo, thi, t0, ft, warp, lane, invf); break;
+      case 7: lin_reduce<7>(prm, prm.part + lin_part_offset(prm, tt, ft, 0), tlo, thi, t0, ft, warp, lane, invf); break;
+      default: lin_reduce<8>(prm, prm.part + lin_part_offset(prm, tt, ft, 0), tlo, thi, t0, ft, warp, lane, invf); break;
     }
   }
-  // no CTA leaves (or frees TMEM) while another may still read its shared memory
-  if (prm.ksplit > 1) cluster_sync_all();
-  else __syncthreads();
+  __syncthreads();
   if (threadIdx.x == 0) { LIN_TRACE(274); LIN_TRACE_CTA(1); }
   if (layout_ok && warp == 1) {
     lin_fence_after();
@@ -385,11 +435,46 @@ cudaError_t lin_smem_attr() {
   return cudaSuccess;
 }
 
+// Clusters of `ks` CTAs (the K splits of one output tile) with `smem` bytes
+// each that this device holds at once; 0 if none (or no device).
+int lin_resident_clusters(int ks, size_t smem) {
+  static int cache[64][kLinMaxSplit + 1][4];
+  static size_t cache_smem[64][kLinMaxSplit + 1][4];
+  if (ks < 1 || ks > kLinMaxSplit) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 0; }
+  for (int i = 0; i < 4; ++i)
+    if (cache[dev][ks][i] && cache_smem[dev][ks][i] == smem) return cache[dev][ks][i] - 1;
+  int n = 0;
+  if (lin_smem_attr() == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, ks, 1);
+    cfg.blockDim = dim3(kLinThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = ks;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, linear_tc05_kernel, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  for (int i = 0; i < 4; ++i)
+    if (!cache[dev][ks][i]) { cache[dev][ks][i] = n + 1; cache_smem[dev][ks][i] = smem; break; }
+  return n;
+}
+
 }  // namespace
 
 #ifdef TIDAR_TRACE
 extern "C" int tidar_lin_trace_read(void* dst, size_t bytes) {
   return (int)cudaMemcpyFromSymbol(dst, g_lin_trace, bytes);
+}
+extern "C" int tidar_lin_trace_clear() {
+  static unsigned long long zero[512 + 2 * 4096];
+  return (int)cudaMemcpyToSymbol(g_lin_trace, zero, sizeof zero);
 }
 #endif
 
@@ -408,14 +493,27 @@ LinearPlan plan_linear(int T, int K, int N) {
   const uint32_t extra = 8u * (2 * kLinMaxStages + 1) + 16u + 64u * 8u;
   p.stages = (int)((kLinSmemBudget - extra) / p.stage_bytes);
   if (p.stages > kLinMaxStages) p.stages = kLinMaxStages;
+  p.smem = p.stages * p.stage_bytes + extra;
+  // Split count: the waves of clusters the launch needs times (the k-blocks
+  // of one split + a fixed per-CTA cost), plus the reduction through L2, in
+  // units of one 64-wide k-block.  Without a device (host-only planning) the
+  // occupancy is taken as one cluster per ks SMs.
   const int kb = K / 64;
   const long long base = (long long)(N / 128) * p.tiles;
-  int ks = base >= 148 ? 1 : (int)(148 / base);
-  if (ks > 8) ks = 8;
-  if (ks > kb) ks = kb;
-  if (ks < 1) ks = 1;
-  p.ksplit = ks;
-  p.smem = p.stages * p.stage_bytes + extra;
+  constexpr double kFixed = 4.0, kReduce = 1.5;
+  double best = 1e300;
+  int best_ks = 1;
+  for (int ks = 1; ks <= kLinMaxSplit && ks <= kb; ++ks) {
+    int resident = ks == 1 ? 148 : lin_resident_clusters(ks, p.smem);
+    if (resident <= 0) resident = 148 / ks;
+    const long long waves = (base + resident - 1) / resident;
+    const double cost = (double)waves * ((double)kb / ks + kFixed) + (ks > 1 ? kReduce : 0.0);
+    if (cost < best - 1e-9) { best = cost; best_ks = ks; }
+  }
+  p.ksplit = best_ks;
+  p.ws_bytes = p.ksplit > 1 ? ((base * p.ksplit * (size_t)p.nt * 128 * sizeof(float) + 255) / 256 * 256 +
+                                (base * p.ksplit * sizeof(int) + 255) / 256 * 256)
+                            : 0;
   p.ok = p.stages >= 4 && (uint32_t)p.nt * 512u <= (uint32_t)p.stages * p.stage_bytes;
   return p;
 }
@@ -423,6 +521,7 @@ LinearPlan plan_linear(int T, int K, int N) {
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s) {
   const LinearPlan p = plan_linear(a.T, a.K, a.N);
   if (!p.ok) return cudaErrorNotSupported;
+  if (p.ws_bytes && (!a.ws || (reinterpret_cast<uintptr_t>(a.ws) & 255u))) return cudaErrorInvalidValue;
   LinParams prm{};
   prm.T = a.T; prm.K = a.K; prm.N = a.N;
   prm.nt = p.nt; prm.nsub = p.nsub; prm.stages = p.stages; prm.ksplit = p.ksplit;
@@ -430,6 +529,12 @@ cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s) {
   prm.mode = a.mode; prm.y = a.y; prm.q = a.q; prm.kb = a.k_blk; prm.vb = a.v_blk;
   prm.seq_lens = a.seq_lens; prm.Hq = a.Hq; prm.Hkv = a.Hkv; prm.R = a.R; prm.kdraft = a.k;
   prm.max_prefix = a.max_prefix; prm.log2_base = a.log2_base; prm.err = a.err;
+  if (p.ws_bytes) {
+    const size_t groups = (size_t)(a.N / 128) * p.tiles;
+    prm.part = static_cast<float*>(a.ws);
+    prm.stat = reinterpret_cast<int*>(static_cast<char*>(a.ws) +
+                                      (groups * p.ksplit * (size_t)p.nt * 128 * sizeof(float) + 255) / 256 * 256);
+  }
   CUtensorMap tw, tx;
   {
     const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.N};

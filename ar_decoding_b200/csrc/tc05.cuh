@@ -176,49 +176,80 @@ __device__ __forceinline__ BlockPlan make_block_plan(const AttnArgs& a, int P, i
 __device__ __forceinline__ bool page_ok(int page, int num_pages) { return page >= 0 && page < num_pages; }
 
 // ------------------------------------------------------------------ split merge
-// Key splits of one query tile run as the CTAs of a thread-block cluster.  After
-// a cluster barrier each CTA pushes its normalised partial rows (fp32) and
-// their lse into the row's owner CTA -- remote stores, no round trip -- laid
-// out [slot][split][32 float4 chunks] and [slot][split]; after a second
-// barrier each owner merges its rows from its own shared memory.
-__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr, float4 v) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
-               "f"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-// One warp per slot, lane = float4 chunk of the row.  row_of(slot) gives the
-// output row (or -1 for a slot holding no row).  A split whose lse is -inf saw
-// no key and may have pushed no values: it is selected away, not multiplied.
-template <typename RowOf>
-__device__ __forceinline__ void merge_pushed_rows(const float* recv, const float* recv_l, int slots, int ns,
-                                                  int warp, int nwarps, int lane, RowOf row_of,
-                                                  __nv_bfloat16* out, float* lse_out) {
-  for (int sl = warp; sl < slots; sl += nwarps) {
-    const long long row = row_of(sl);
+// Key splits of one query tile run as the CTAs of a thread-block cluster and
+// merge through L2.  Every split has written its normalised partial rows (fp32
+// O of 128 columns, and the row's lse) to part_o / part_lse, laid out
+// [split][stride rows]; a cluster barrier (release / acquire at cluster scope)
+// orders those writes before these reads.  This CTA merges `owned` rows,
+// row_of(i) giving the i-th one's row index (negative: skip).  A group of
+// 32 / CPT threads merges one row, CPT float4 columns each, so that with
+// enough threads every owned row is in flight at once: one round trip for the
+// lse of all splits, one for the rows.  Loads bypass L1 (other SMs wrote the
+// partials).  The weights are exp(lse_s - max); a split with lse = -inf saw no
+// key and may have written no values: it is selected away, not multiplied.
+template <int CPT, class RowOf>
+__device__ __forceinline__ void merge_l2_rows_t(const float* __restrict__ part_o,
+                                                const float* __restrict__ part_lse, long long stride, int ns,
+                                                int owned, RowOf row_of, __nv_bfloat16* out, float* lse_out) {
+  constexpr int kG = 32 / CPT;
+  const int sub = (int)threadIdx.x % kG;
+  const int groups = (int)blockDim.x / kG;
+  for (int i = (int)threadIdx.x / kG; i < owned; i += groups) {
+    const long long row = row_of(i);
     if (row < 0) continue;
+    float l2[kMaxCluster];
     float mx = -INFINITY;
-    for (int s2 = 0; s2 < ns; ++s2) mx = fmaxf(mx, recv_l[sl * ns + s2] * 1.4426950408889634f);
+#pragma unroll
+    for (int s = 0; s < kMaxCluster; ++s) {
+      l2[s] = s < ns ? __ldcg(part_lse + s * stride + row) * 1.4426950408889634f : -INFINITY;
+      mx = fmaxf(mx, l2[s]);
+    }
+    float4 acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     float wsum = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s2 = 0; s2 < ns; ++s2) {
-      const float l2 = recv_l[sl * ns + s2] * 1.4426950408889634f;
-      if (l2 == -INFINITY) continue;
-      const float w = ex2(l2 - mx);
-      wsum += w;
-      const float4 x = reinterpret_cast<const float4*>(recv)[(sl * ns + s2) * 32 + lane];
-      acc.x = fmaf(w, x.x, acc.x); acc.y = fmaf(w, x.y, acc.y);
-      acc.z = fmaf(w, x.z, acc.z); acc.w = fmaf(w, x.w, acc.w);
+#pragma unroll
+    for (int s = 0; s < kMaxCluster; ++s) {
+      if (s < ns) {
+        const float4* src = reinterpret_cast<const float4*>(part_o + (s * stride + row) * 128) + sub * CPT;
+        float4 x[CPT];
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) x[c] = __ldcg(src + c);
+        if (l2[s] != -INFINITY) {
+          const float w = ex2(l2[s] - mx);
+          wsum += w;
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) {
+            acc[c].x = fmaf(w, x[c].x, acc[c].x); acc[c].y = fmaf(w, x[c].y, acc[c].y);
+            acc[c].z = fmaf(w, x[c].z, acc[c].z); acc[c].w = fmaf(w, x[c].w, acc[c].w);
+          }
+        }
+      }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    uint2 u;
-    u.x = cvt_bf16x2(acc.x * inv, acc.y * inv);
-    u.y = cvt_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(out + row * 128 + 4 * lane) = u;
-    if (lane == 0 && lse_out) lse_out[row] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      uint2 u;
+      u.x = cvt_bf16x2(acc[c].x * inv, acc[c].y * inv);
+      u.y = cvt_bf16x2(acc[c].z * inv, acc[c].w * inv);
+      *reinterpret_cast<uint2*>(out + row * 128 + 4 * (sub * CPT + c)) = u;
+    }
+    if (sub == 0 && lse_out) lse_out[row] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
   }
+}
+
+// This CTA's share of the merge, the group size picked so that all `owned`
+// rows go in one pass when the block has the threads (at most 8 columns of 4
+// per thread).
+template <class RowOf>
+__device__ __forceinline__ void merge_l2_rows(const float* part_o, const float* part_lse, long long stride,
+                                              int ns, int owned, RowOf row_of, __nv_bfloat16* out,
+                                              float* lse_out) {
+  const int per = (32 * owned + (int)blockDim.x - 1) / (int)blockDim.x;
+  if (per <= 1) merge_l2_rows_t<1>(part_o, part_lse, stride, ns, owned, row_of, out, lse_out);
+  else if (per <= 2) merge_l2_rows_t<2>(part_o, part_lse, stride, ns, owned, row_of, out, lse_out);
+  else if (per <= 4) merge_l2_rows_t<4>(part_o, part_lse, stride, ns, owned, row_of, out, lse_out);
+  else merge_l2_rows_t<8>(part_o, part_lse, stride, ns, owned, row_of, out, lse_out);
 }
 
 }  // namespace tc05

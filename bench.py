@@ -197,7 +197,8 @@ class Step:
         # attention: one launch when the kernel merges its splits on chip (no
         # workspace) on the tensor-core or decode path, else kernel + finalize;
         # then greedy verify (one cluster kernel) and commit (one cluster kernel)
-        self.attn_launches = 1 if (need == 0 and self.path_id in (2, 3, 4)) else 2
+        self.merge = tidar.plan_full(self.desc)[2]
+        self.attn_launches = 2 if (self.merge == 2 or self.path_id == 1) else 1
         self.launches_per_step = self.attn_launches + 1 + 1
 
     def attn(self, i):
@@ -304,7 +305,8 @@ class Loop:
         # cluster when the vocabulary's 4096-wide chunks fit a portable cluster
         # of 8, else two launches), commit
         nchunk = -(-V // 4096)
-        self.launches_per_step = (1 + (1 if (need == 0 and self.path_id in (2, 3, 4)) else 2) +
+        merge = tidar.plan_full(self.desc)[2]
+        self.launches_per_step = (1 + (2 if (merge == 2 or self.path_id == 1) else 1) +
                                   (1 if mode == "greedy" else (2 if nchunk <= 8 else 3)) + 1)
 
     def step(self, c, s):
@@ -427,10 +429,10 @@ class LayerStep:
     def qkv(self, i):
         c, cfg = self.copies[i], self.cfg
         self.tidar.qkv_rope(c["x"], c["w_qkv"], c["cache"]["seq_lens"], cfg.k, cfg.Hq, cfg.Hkv,
-                            max_prefix_len=self.max_prefix, out=self.qkv_out)
+                            max_prefix_len=self.max_prefix, out=self.qkv_out, workspace=self.ws)
 
     def oproj(self, i):
-        self.tidar.linear(self.attn_out, self.copies[i]["w_o"], out=self.y)
+        self.tidar.linear(self.attn_out, self.copies[i]["w_o"], out=self.y, workspace=self.ws)
 
     def time(self, fn, reps):
         """Average device µs of fn over all copies back to back in one graph."""

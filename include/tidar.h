@@ -144,15 +144,18 @@ typedef struct {
  *   q        [B][R][Hq][D]     k_blk, v_blk [B][R][Hkv][D]     (dtype)
  *   out      [B][R][Hq][D]     (dtype)     lse_out [B][R][Hq] fp32 or NULL
  *   workspace: device scratch of at least tidar_step_attn_workspace_bytes(desc)
- *     bytes, 256-byte aligned (may be NULL when that size is 0); contents on
- *     entry are ignored.  Calls that share a workspace must be stream-ordered.
+ *     bytes, 256-byte aligned (may be NULL when that size is 0: one split);
+ *     the splits' partial rows pass through it.  Contents on entry are
+ *     ignored.  Calls that share a workspace must be stream-ordered.
  * Device errors: BAD_PAGE (prefix or draft page unmapped), BAD_LEN; the TC05
  * and DEC kernels also TIMEOUT (a bounded wait on a copy or on a cluster
- * peer ran out) and LAYOUT.  Splits of a long prefix merge on chip (a
- * thread-block cluster per query tile) when every cluster of the launch can
- * be resident at once, else through workspace partials and a second launch.
- * That second launch also writes the draft rows; without it the TC05 and DEC
- * kernels write them (SIMT always takes the second launch).
+ * peer ran out) and LAYOUT.  Splits of a long prefix merge inside the
+ * attention kernel (the splits of a query tile form a thread-block cluster;
+ * the tensor-core kernels pass the partial rows through the workspace in L2,
+ * the decode kernel through distributed shared memory) when such clusters
+ * can be scheduled, else in a second launch.  That second launch also writes the
+ * draft rows; without it the tensor-core and decode kernels write them (SIMT
+ * always takes the second launch).
  * ------------------------------------------------------------------------- */
 size_t tidar_step_attn_workspace_bytes(const tidar_step_desc* desc);
 tidar_status tidar_step_attn(const tidar_step_desc* desc, const tidar_kv_cache* cache,
@@ -196,9 +199,12 @@ tidar_status tidar_merge_attn(int32_t nparts, int64_t rows, int32_t head_dim, ti
                               float* lse_out, tidar_stream_t stream);
 
 /* The launch plan the library would use: kernel family (1 SIMT, 2 TC05,
- * 3 DEC, 4 PAIR) and number of KV splits.  Host only; with a GPU present the first
- * call per device queries its SM count and cluster occupancy. */
-tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, int32_t* splits);
+ * 3 DEC, 4 PAIR), number of KV splits, and how the splits merge (0: one
+ * split; 1: in the attention kernel, its splits forming a thread-block
+ * cluster; 2: a second launch).  Any pointer may be NULL.  Host only; with a
+ * GPU present the first call per device queries its cluster occupancy. */
+tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, int32_t* splits,
+                                  int32_t* merge);
 
 /* ---------------------------------------------------------------------------
  * Verification, acceptance and selection.  [NDfr] paragraph on betting on
@@ -451,6 +457,12 @@ tidar_status tidar_reserve(const tidar_step_desc* desc, const tidar_kv_cache* ca
  *   w [out_features][in_features].  dtype must be TIDAR_BF16, in_features a
  *   multiple of 64 and out_features a multiple of 128 (else
  *   TIDAR_ERR_UNSUPPORTED); x, w, y 16-byte aligned.  rows >= 0.
+ *   workspace: device scratch of at least tidar_linear_workspace_bytes(rows,
+ *   out_features, in_features) bytes, 256-byte aligned (NULL when that is 0):
+ *   the fp32 partial sums of the reduction's splits.  Contents on entry are
+ *   ignored; calls sharing a workspace must be stream-ordered.  The size
+ *   depends on the current device (its cluster occupancy sets the number of
+ *   splits): query it on the device that runs the call.
  *
  * tidar_qkv_rope: the query/key/value projection of the R step rows of each
  *   sequence and the rotary embedding at their zone positions.
@@ -468,23 +480,27 @@ tidar_status tidar_reserve(const tidar_step_desc* desc, const tidar_kv_cache* ca
  *   Needs dtype TIDAR_BF16, head_dim 128, d_model a multiple of 64
  *   (TIDAR_ERR_UNSUPPORTED otherwise), rope_base > 1.  Device error BAD_LEN
  *   (seq_lens[b] outside 0..max_prefix_len: position P_b = 0 is used).
+ *   workspace as tidar_linear's, sized by tidar_qkv_rope_workspace_bytes.
  *
  * tidar_layer_step: tidar_qkv_rope, tidar_step_attn (which also appends the
  *   drafts' rotated K/V to the cache) and the output projection
  *   y [B][R][d_model] = attn_out . w_o^T with w_o [d_model][Hq D], as one
  *   call.  lse_out as tidar_step_attn's.  workspace: at least
  *   tidar_layer_step_workspace_bytes(desc, d_model) bytes, 256-byte aligned,
- *   holding q, k_blk, v_blk, the attention output and the attention's own
- *   workspace.  d_model must also be a multiple of 128.
+ *   holding q, k_blk, v_blk, the attention output, the projections' and the
+ *   attention's own workspaces.  d_model must also be a multiple of 128.
  * Device errors: those of the calls it makes; TIMEOUT if a bounded wait in a
  * projection ran out.
  * ------------------------------------------------------------------------- */
+size_t tidar_linear_workspace_bytes(int32_t rows, int32_t out_features, int32_t in_features);
 tidar_status tidar_linear(int32_t rows, int32_t out_features, int32_t in_features,
                           tidar_dtype dtype, const void* x, const void* w, void* y,
-                          tidar_stream_t stream);
+                          void* workspace, size_t workspace_bytes, tidar_stream_t stream);
+size_t tidar_qkv_rope_workspace_bytes(const tidar_step_desc* desc, int32_t d_model);
 tidar_status tidar_qkv_rope(const tidar_step_desc* desc, int32_t d_model, const void* x,
                             const void* w_qkv, const int32_t* seq_lens, float rope_base,
-                            void* q, void* k_blk, void* v_blk, tidar_stream_t stream);
+                            void* q, void* k_blk, void* v_blk, void* workspace,
+                            size_t workspace_bytes, tidar_stream_t stream);
 size_t tidar_layer_step_workspace_bytes(const tidar_step_desc* desc, int32_t d_model);
 tidar_status tidar_layer_step(const tidar_step_desc* desc, const tidar_kv_cache* cache,
                               int32_t d_model, const void* x, const void* w_qkv,
@@ -509,10 +525,10 @@ const char* tidar_last_cuda_error(void);
  *     the CTAs record TIDAR_DEVERR_TIMEOUT, release TMEM and exit, the
  *     outputs are unspecified, tidar_get_device_status returns
  *     TIDAR_ERR_TIMEOUT and the CUDA context stays usable (failure injection).
- *   TIDAR_DEBUG_FORCE_SPLIT_PARTIALS: the TC05 and DEC paths merge key splits
- *     through workspace partials and a second launch even where it would
- *     merge them on chip (so tests reach both merges).  Changes the
- *     workspace size that tidar_step_attn_workspace_bytes reports.
+ *   TIDAR_DEBUG_FORCE_SPLIT_PARTIALS: the TC05, PAIR and DEC paths merge key
+ *     splits in a second launch even where they would merge them in the
+ *     attention kernel (so tests reach both merges).  May change the split
+ *     count, and with it the size tidar_step_attn_workspace_bytes reports.
  * Returns TIDAR_ERR_INVALID_ARG for an unknown knob.
  * ------------------------------------------------------------------------- */
 typedef enum {

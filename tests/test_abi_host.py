@@ -84,16 +84,19 @@ def test_step_attn_rejects_small_workspace(L):
 
 def test_tensor_core_plan_splits_long_prefixes(L):
     # one query row per head: the 8192-key prefix is split to fill the SMs; the
-    # workspace holds split partials unless the device merges them on chip
+    # split partials pass through the workspace whichever way they merge
     d = _desc(max_prefix_len=8192, batch=1, num_q_heads=32, num_kv_heads=8, k=0,
               path=tidar.PATH_TC05)
-    path, splits = ctypes.c_int32(), ctypes.c_int32()
-    assert L.tidar_step_attn_plan(ctypes.byref(d), ctypes.byref(path), ctypes.byref(splits)) == tidar.OK
-    assert path.value == 2 and splits.value > 1
+    path, splits, merge = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    assert L.tidar_step_attn_plan(ctypes.byref(d), ctypes.byref(path), ctypes.byref(splits),
+                                  ctypes.byref(merge)) == tidar.OK
+    assert path.value == 2 and splits.value > 1 and merge.value in (1, 2)
+    assert L.tidar_step_attn_plan(ctypes.byref(d), None, None, None) == tidar.OK
     ws = L.tidar_step_attn_workspace_bytes(ctypes.byref(d))
     rows = 32                                  # B * R * Hq
-    assert ws in (0, ((splits.value * rows * 128 * 4 + 255) // 256 * 256) +
-                  ((splits.value * rows * 4 + 255) // 256 * 256))
+    assert ws == ((splits.value * rows * 128 * 4 + 255) // 256 * 256) + \
+        ((splits.value * rows * 4 + 255) // 256 * 256)
+    assert tidar.plan_full(d) == (path.value, splits.value, merge.value)
 
 
 def test_batch_zero_is_a_noop(L):
@@ -199,3 +202,25 @@ def test_binding_refuses_host_tensors(L):
     pool = synth.make_pool(cfg, cache)
     with pytest.raises(ValueError):
         tidar.reserve(cache, pool, cfg.k, max_prefix_len=10)
+
+
+def test_projection_workspace_is_checked(L):
+    # split-K partials pass through the caller's workspace: an 8B-class query /
+    # key / value projection of a 272-row step splits its reduction, a single
+    # 64-wide reduction cannot split (no workspace)
+    need = L.tidar_linear_workspace_bytes(272, 6144, 4096)
+    assert need > 0 and need % 256 == 0
+    assert L.tidar_linear_workspace_bytes(16, 128, 64) == 0
+    assert L.tidar_linear_workspace_bytes(0, 128, 64) == 0
+    lin = lambda ws, wsb: L.tidar_linear(272, 6144, 4096, tidar.BF16, FAKE, FAKE, FAKE, ws, wsb, None)
+    assert lin(None, 0) == tidar.ERR_INVALID_ARG
+    assert lin(FAKE, need - 1) == tidar.ERR_INVALID_ARG
+    assert lin(FAKE + 16, need) == tidar.ERR_INVALID_ARG               # not 256-aligned
+    assert L.tidar_linear(272, 6144, 4000, tidar.BF16, FAKE, FAKE, FAKE, None, 0, None) == \
+        tidar.ERR_UNSUPPORTED                                             # in_features % 64
+    d = _desc(batch=1, num_q_heads=32, num_kv_heads=8, k=16, max_prefix_len=8192, head_dim=128,
+              dtype=tidar.BF16)
+    assert L.tidar_qkv_rope_workspace_bytes(ctypes.byref(d), 4096) == need
+    assert L.tidar_qkv_rope(ctypes.byref(d), 4096, FAKE, FAKE, FAKE, ctypes.c_float(10000.0), FAKE, FAKE,
+                            FAKE, None, 0, None) == tidar.ERR_INVALID_ARG
+    assert L.tidar_layer_step_workspace_bytes(ctypes.byref(d), 4096) > need

@@ -156,10 +156,10 @@ Plan make_plan(const tidar_step_desc* d, int path) {
       return;
     }
     // tensor-core paths: the last split also runs the tile's step-key windows
-    // (up to ceil(R / 128) blocks of 128, masked: each costs about 1.5 prefix
-    // blocks), so the split size counts them and the last split gets
-    // correspondingly fewer prefix blocks
-    const int wins = ((path == 2 || path == 4) && n > 1) ? (3 * ((R + 127) / 128) + 1) / 2 : 0;
+    // (up to ceil(R / 128) blocks of 128; a masked block costs about what a
+    // prefix block does), so the split size counts them and the last split
+    // gets correspondingly fewer prefix blocks
+    const int wins = ((path == 2 || path == 4) && n > 1) ? (R + 127) / 128 : 0;
     const int bps = (blocks128 + wins + n - 1) / n;
     p.keys_per_split = (bps > 0 ? bps : 1) * 128;
     p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
@@ -256,7 +256,7 @@ size_t tidar_step_attn_workspace_bytes(const tidar_step_desc* d) {
   if (check_desc(d) != TIDAR_OK) return 0;
   const int pth = choose_path(d);
   const Plan p = make_plan(d, pth);
-  if (p.nsplit <= 1) return 0;                        // one split: nothing to merge
+  if (p.nsplit <= 1 || p.cluster_merge) return 0;     // one split, or merged in the kernel
   const size_t rows = (size_t)d->batch * tidar::rows_per_seq(d->k) * d->num_q_heads;
   return align256((size_t)p.nsplit * rows * d->head_dim * sizeof(float)) +
          align256((size_t)p.nsplit * rows * sizeof(float));
@@ -306,7 +306,7 @@ tidar_status step_attn_impl(const tidar_step_desc* d, const tidar_kv_cache* c, c
   a.step_keys = step_keys;
   a.append = append;
   a.cluster_merge = p.cluster_merge ? 1 : 0;
-  if (p.nsplit > 1) {
+  if (p.nsplit > 1 && !p.cluster_merge) {
     const size_t rows = (size_t)a.B * a.R * a.Hq;
     a.part_o = static_cast<float*>(workspace);
     a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +

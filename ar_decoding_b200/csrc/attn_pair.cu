@@ -37,10 +37,10 @@
 //   warps 10, 11 only the split merge and the draft-row append.
 // The last split also runs the step-key windows holding keys visible to
 // either tile, with the zone mask applied in the softmax.  Key splits of one
-// (b, g, pair) write their normalised partial O and lse to the workspace and
-// either merge in this kernel (the splits form a thread-block cluster; after
-// a cluster barrier CTA `rank` merges a share of the rows from L2) or leave
-// the merge to a finalize launch.
+// (b, g, pair) either form a thread-block cluster and merge in this kernel
+// (each CTA stages its normalised rows in shared memory; after a cluster
+// barrier CTA `rank` merges a share of the rows over distributed shared
+// memory) or write fp32 partials to the workspace for a finalize launch.
 // Every mbarrier wait is bounded (~1 s): on expiry the CTA records
 // TIDAR_DEVERR_TIMEOUT, stops issuing, drains what it issued, frees TMEM and
 // exits through the same cluster barriers as the other CTAs.
@@ -80,6 +80,7 @@ constexpr int kPBars = 18;
 constexpr uint32_t kPOffMisc = kPOffBar + kPBars * 8;      // [0] TMEM base, [1] abort flag
 constexpr uint32_t kPSmem = kPOffMisc + 16;
 static_assert(kPSmem <= 232448, "shared memory budget");
+static_assert((256 * kStageStride + 512) * 4 <= (kKSt + kVSt) * kPTile, "row staging fits the K/V rings");
 // split merge receive area, in the K/V rings once they are idle: [slot][split]
 // [32 float4] fp32 partial rows for at most 256 + 16 (slot, split) pairs, then
 // their lse
@@ -98,11 +99,11 @@ constexpr uint32_t kPIdescPV = kPIdescS | (1u << 16);     // B (= V) is MN-major
 // block i (0 wait done, 1 loaded, 2 max, 3 exps, 4 stored), [2600] epilogue,
 // [2601] end; [4096 + 2 cta] start / end of every CTA.
 #ifdef TIDAR_TRACE
-__device__ unsigned long long g_pair_trace[4096 + 2 * 8192];
+__device__ unsigned long long g_pair_trace[4096 + 4 * 8192];
 __device__ __forceinline__ bool ptrace_cta() { return blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0; }
 #define PAIR_TRACE(slot) do { if (ptrace_cta() && (slot) < 4096) g_pair_trace[(slot)] = global_ns(); } while (0)
 #define PAIR_TRACE_CTA(w) do { const unsigned c_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
-    if (c_ < 8192) g_pair_trace[4096 + 2 * c_ + (w)] = global_ns(); } while (0)
+    if (c_ < 8192) g_pair_trace[4096 + 4 * c_ + (w)] = global_ns(); } while (0)
 #else
 #define PAIR_TRACE(slot) do {} while (0)
 #define PAIR_TRACE_CTA(w) do {} while (0)
@@ -475,7 +476,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (threadIdx.x == 0) PAIR_TRACE(2048 + 8 * min(b2, 60) + 4);
         if (!ok) break;
       }
-      if (threadIdx.x == 0) PAIR_TRACE(2600);
+      if (threadIdx.x == 0) { PAIR_TRACE(2600); PAIR_TRACE_CTA(2); }
       // ---- this tile's row of O: wait for the last PV, normalise
       if (ok && nb > 0 && !warp_wait_bar(bar(PB_PVDONE + t), (uint32_t)((nb - 1) & 1), abort_flag, a.err)) ok = false;
       ok = __all_sync(0xffffffffu, ok && !*abort_flag);
@@ -493,72 +494,71 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       }
       owrite = ok && r < rows_valid[t];
-      if (owrite && a.nsplit == 1) {
-        const int rho = rho0[t] + r / a.G, h = g * a.G + r % a.G;
-        const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + row * 128;
-#pragma unroll
-        for (int e = 0; e < 128; e += 8) {
-          uint4 u;
-          u.x = cvt_bf16x2(ov[e], ov[e + 1]); u.y = cvt_bf16x2(ov[e + 2], ov[e + 3]);
-          u.z = cvt_bf16x2(ov[e + 4], ov[e + 5]); u.w = cvt_bf16x2(ov[e + 6], ov[e + 7]);
-          *reinterpret_cast<uint4*>(dst + e) = u;
-        }
-        if (a.lse_out) a.lse_out[row] = olse;
-      }
+      if (threadIdx.x == 0) PAIR_TRACE(2602);
     }
   }
 
   // The producer has drained, every MMA is complete and no copy is in flight.
+  if (lane == 0) PAIR_TRACE(2610 + warp);
   fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) PAIR_TRACE(2606);
 
-  if (a.nsplit > 1) {
-    // ---------------------------------------------------------------- split partials
-    if (warp < 8) {
-      const int t = warp >> 2, r = threadIdx.x & 127;
-      if (r < rows_valid[t]) {
-        const int rho = rho0[t] + r / a.G, h = g * a.G + r % a.G;
-        const size_t prow = (size_t)split * a.B * a.R * a.Hq + (size_t)(b * a.R + rho) * a.Hq + h;
-        if (owrite) {
-          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 128);
-#pragma unroll
-          for (int e = 0; e < 128; e += 4) dst[e / 4] = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
-        }
-        a.part_lse[prow] = owrite ? olse : -INFINITY;
-      }
-    }
-    if (cluster) {
-      // -------------------------------------------------------------- split merge
-      // Row i = t * 128 + r of the pair is merged by CTA i % ns once every
-      // split has written its partials (the cluster barrier), from L2.
-      const int ns = a.nsplit;
-      const int rank = (int)cluster_rank();
-      cluster_sync_all();
-      const int owned = (256 - rank + ns - 1) / ns;
-      merge_l2_rows(a.part_o, a.part_lse, (long long)a.B * a.R * a.Hq, ns, owned,
-                    [&](int sl) -> long long {
-                      const int i = sl * ns + rank;
-                      const int t = i >> 7, rr = i & 127;
-                      if (t >= ntile || rr >= rows_valid[t]) return -1;
-                      const int rho = rho0[t] + rr / a.G, h = g * a.G + rr % a.G;
-                      return (long long)(b * a.R + rho) * a.Hq + h;
-                    },
-                    static_cast<__nv_bfloat16*>(a.out), a.lse_out);
-    }
-  }
-
-  if (nb == 0 && layout_ok && a.nsplit == 1 && warp < 8) {
-    // no key at all for this pair (a prefix-only call on an empty slice):
-    // O = 0 and lse = -inf, so a later merge gives these rows no weight
+  // ------------------------------------------------------------------ write-out
+  // Staged row i = t * 128 + r (tile t) in the idle K/V rings, then whole-row
+  // stores: the bf16 output (one split) or this split's fp32 partials, merged
+  // by the cluster (cluster_merge) or a finalize launch.  A pair without keys
+  // (an empty slice of a prefix-only call, or a split past a short sequence's
+  // prefix) contributes O = 0 with lse = -inf.
+  float* ost = reinterpret_cast<float*>(smem + kPOffK);
+  float* lst = ost + 256 * kStageStride;
+  int* wst = reinterpret_cast<int*>(lst + 256);
+  if (warp < 8) {
     const int t = warp >> 2, r = threadIdx.x & 127;
-    if (r < rows_valid[t]) {
-      const int rho = rho0[t] + r / a.G, h = g * a.G + r % a.G;
-      const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * 128);
-      for (int e = 0; e < 16; ++e) dst[e] = make_uint4(0, 0, 0, 0);
-      if (a.lse_out) a.lse_out[row] = -INFINITY;
+    if (nb == 0) {
+#pragma unroll
+      for (int e = 0; e < 128; ++e) ov[e] = 0.f;
+      olse = -INFINITY;
+      owrite = layout_ok && r < rows_valid[t];
     }
+    float4* d = reinterpret_cast<float4*>(ost + (t * 128 + r) * kStageStride);
+#pragma unroll
+    for (int e = 0; e < 128; e += 4) d[e / 4] = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
+    lst[t * 128 + r] = owrite ? olse : -INFINITY;
+    wst[t * 128 + r] = owrite ? 1 : 0;
+    if (threadIdx.x == 0) PAIR_TRACE(2607);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) PAIR_TRACE(2608);
+  auto out_row = [&](int i) -> long long {
+    const int t = i >> 7, rr = i & 127;
+    if (t >= ntile || rr >= rows_valid[t]) return -1;
+    const int rho = rho0[t] + rr / a.G, h = g * a.G + rr % a.G;
+    return (long long)(b * a.R + rho) * a.Hq + h;
+  };
+  if (a.nsplit == 1) {
+    store_rows_bf16(ost, lst, wst, 256, out_row, static_cast<__nv_bfloat16*>(a.out), a.lse_out);
+  } else if (cluster) {
+    // ---------------------------------------------------------------- split merge
+    // Staged row i of the pair is merged by CTA i % ns from every split's
+    // shared memory once all have staged (first cluster barrier); the second
+    // keeps each CTA's shared memory alive until its peers are done.
+    const int ns = a.nsplit;
+    const int rank = (int)cluster_rank();
+    cluster_sync_all();
+    if (threadIdx.x == 0) { PAIR_TRACE(2604); PAIR_TRACE_CTA(3); }
+    const int owned = (256 - rank + ns - 1) / ns;
+    merge_rows<4, 4>(ost, lst, ns, rank, owned, out_row, static_cast<__nv_bfloat16*>(a.out), a.lse_out);
+    if (threadIdx.x == 0) PAIR_TRACE(2605);
+    cluster_sync_all();
+  } else {
+    const long long stride = (long long)a.B * a.R * a.Hq;
+    store_rows_partial(ost, lst, wst, 256, [&](int i) -> long long {
+                         const long long r = out_row(i);
+                         return r < 0 ? -1 : split * stride + r;
+                       },
+                       a.part_o, a.part_lse);
+    if (threadIdx.x == 0) PAIR_TRACE(2603);
   }
 
   if (pair == 0 && split == 0 && len_ok && (a.nsplit == 1 || cluster) && a.append) {
@@ -610,7 +610,7 @@ extern "C" int tidar_pair_trace_read(void* dst, size_t bytes) {
   return (int)cudaMemcpyFromSymbol(dst, g_pair_trace, bytes);
 }
 extern "C" int tidar_pair_trace_clear(void) {
-  static unsigned long long zeros[4096 + 2 * 8192];
+  static unsigned long long zeros[4096 + 4 * 8192];
   return (int)cudaMemcpyToSymbol(g_pair_trace, zeros, sizeof zeros);
 }
 #endif
@@ -648,8 +648,8 @@ cudaError_t launch_attn_pair(const AttnArgs& a, cudaStream_t s) {
   }
   cudaError_t e = pair_smem_attr();
   if (e != cudaSuccess) return e;
-  if (a.nsplit > 1 && (!a.part_o || !a.part_lse)) return cudaErrorInvalidValue;   // partials are staged
   const bool clu = a.nsplit > 1 && a.cluster_merge;
+  if (a.nsplit > 1 && !clu && (!a.part_o || !a.part_lse)) return cudaErrorInvalidValue;
   if (clu && a.nsplit > kMaxCluster) return cudaErrorNotSupported;
   const dim3 grid(prm.pairs, a.nsplit, a.B * a.Hkv);
   const dim3 cluster(1, clu ? a.nsplit : 1, 1);

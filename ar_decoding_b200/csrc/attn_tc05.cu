@@ -32,10 +32,10 @@
 //                32 columns of its own 64).  O_t is rescaled only when the
 //                row maximum grows by more than 2^8.  The epilogue merges the
 //                two sets and the two halves (max, sums, O) and writes O / l.
-// Key splits of one (b, g, tile) write their normalised partial O and lse to
-// the workspace; with cluster_merge they form one thread-block cluster and
-// merge in this kernel (from L2, after a cluster barrier), else a finalize
-// launch merges them.
+// Key splits of one (b, g, tile) either form one thread-block cluster and
+// merge in this kernel (cluster_merge: each CTA stages its normalised rows in
+// shared memory and owners read their peers' rows over distributed shared
+// memory), or write fp32 partials to the workspace for a finalize launch.
 // Every mbarrier wait is bounded: on expiry the CTA records TIDAR_DEVERR_TIMEOUT,
 // stops issuing, drains what it issued (bounded), frees TMEM and exits.
 #include <cuda.h>
@@ -105,14 +105,16 @@ int g_starve_loads = 0;   // tidar_debug_starve_attention_loads
 // -DTIDAR_TRACE; absent from normal builds).  Slots: [0..15] setup, [16+i]
 // producer issue of block i, [256+i] MMA sees K(i), [512+i] S(i) issued,
 // [768+i] PV(i) issued, [1024+i] softmax sees S(i), [1280+i] P(i) handed over,
-// [1536..] epilogue, [2048 + 2*cta] CTA start / end.
+// [1536..] epilogue (1536 sets merged, 1538 O formed, 1539 partials stored,
+// 1540 past the cluster barrier, 1541 merged, 1537 end), [2048 + 4*cta] CTA
+// start / end / epilogue / past the cluster barrier.
 #ifdef TIDAR_TRACE
-__device__ unsigned long long g_tidar_trace[2048 + 2 * 8192];
+__device__ unsigned long long g_tidar_trace[2048 + 4 * 8192];
 __device__ __forceinline__ bool trace_cta() { return blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0; }
 #define TIDAR_TRACE_AT(slot) do { if (trace_cta()) g_tidar_trace[(slot)] = global_ns(); } while (0)
 #define TIDAR_TRACE_PH(i, ph) do { if (((i) == 10 || (i) == 11) && lane == 0) TIDAR_TRACE_AT(1700 + 8 * warp + (ph)); } while (0)
 #define TIDAR_TRACE_CTA(which) do { const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
-    if (cta_ < 8192) g_tidar_trace[2048 + 2 * cta_ + (which)] = global_ns(); } while (0)
+    if (cta_ < 8192) g_tidar_trace[2048 + 4 * cta_ + (which)] = global_ns(); } while (0)
 #else
 #define TIDAR_TRACE_AT(slot) do {} while (0)
 #define TIDAR_TRACE_PH(i, ph) do {} while (0)
@@ -120,6 +122,7 @@ __device__ __forceinline__ bool trace_cta() { return blockIdx.x == 0 && blockIdx
 #endif
 
 using namespace tc05;
+static_assert((128 * kStageStride + 256) * 4 <= kStages * kTileBytes, "row staging fits the K ring");
 
 // ------------------------------------------------------------------ the kernel
 // 18 warps: two SMSPs host five of them, so a thread may hold at most
@@ -557,7 +560,7 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float m0 = xm[r], m1 = xm[128 + r];
     const float l0 = xs[r] + xs[128 + r], l1 = xs[256 + r] + xs[384 + r];
     ok = xk[q4] && xk[4 + q4] && xk[8 + q4] && xk[12 + q4];
-    if (warp == 4 && lane == 0) TIDAR_TRACE_AT(1536);
+    if (warp == 4 && lane == 0) { TIDAR_TRACE_AT(1536); TIDAR_TRACE_CTA(2); }
     const float mt = fmaxf(m0, m1);
     const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - mt);
     const float f1 = (m1 == -INFINITY || nb1 == 0) ? 0.f : ex2(m1 - mt);
@@ -566,8 +569,6 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float g0 = f0 * inv, g1 = f1 * inv;
     const float lse = lt > 0.f ? (mt + log2f(lt)) * 0.69314718055994531f : -INFINITY;
     const bool write = r < rows_valid && ok;
-    const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
-    const size_t row = (size_t)(b * a.R + (r < rows_valid ? rho : 0)) * a.Hq + h;
     const int col0 = 32 * (2 * t + hf);                  // this thread's 32 output columns
     {
       uint32_t o0[32], o1[32];
@@ -577,75 +578,74 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
       for (int e = 0; e < 32; ++e)
         ov[e] = __uint_as_float(o0[e]) * g0 + (nb1 > 0 ? __uint_as_float(o1[e]) * g1 : 0.f);
-      if (write && a.nsplit == 1) {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + row * 128 + col0;
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 u;
-          u.x = cvt_bf16x2(ov[e], ov[e + 1]); u.y = cvt_bf16x2(ov[e + 2], ov[e + 3]);
-          u.z = cvt_bf16x2(ov[e + 4], ov[e + 5]); u.w = cvt_bf16x2(ov[e + 6], ov[e + 7]);
-          *reinterpret_cast<uint4*>(dst + e) = u;
-        }
-        if (t == 0 && hf == 0 && a.lse_out) a.lse_out[row] = lse;
-      }
     }
     owrite = write;
     olse = lse;
+    if (warp == 4 && lane == 0) TIDAR_TRACE_AT(1538);
   }
 
   // The producer has drained, every MMA is complete and no copy is in flight.
+  if (lane == 0) TIDAR_TRACE_AT(1550 + warp);
   fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) TIDAR_TRACE_AT(1542);
 
-  if (a.nsplit > 1) {
-    // ---------------------------------------------------------------- split partials
-    // This split's normalised O rows and their lse go to the workspace.
-    if (warp >= 2) {
-      const int r = 32 * (warp & 3) + lane;
-      const int t = (warp - 2) >> 3, hf = ((warp - 2) >> 2) & 1;
-      if (r < rows_valid) {
-        const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
-        const size_t prow = (size_t)split * a.B * a.R * a.Hq + (size_t)(b * a.R + rho) * a.Hq + h;
-        if (owrite) {
-          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 128 + 32 * (2 * t + hf));
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) dst[e / 4] = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
-        }
-        if (t == 0 && hf == 0) a.part_lse[prow] = owrite ? olse : -INFINITY;
-      }
-    }
-    if (a.cluster_merge) {
-      // -------------------------------------------------------------- split merge
-      // The CTAs of this cluster are the splits of one (b, g, tile).  Once all
-      // of them have written their partials (the cluster barrier), CTA j
-      // merges rows j, j + ns, j + 2 ns, ... of the tile from L2.  Without
-      // cluster_merge a finalize launch does this.
-      const int ns = a.nsplit;
-      const int rank = (int)cluster_rank();
-      cluster_sync_all();
-      const int owned = rows_valid > rank ? (rows_valid - rank + ns - 1) / ns : 0;
-      merge_l2_rows(a.part_o, a.part_lse, (long long)a.B * a.R * a.Hq, ns, owned,
-                    [&](int i) -> long long {
-                      const int r = i * ns + rank;
-                      const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
-                      return (long long)(b * a.R + rho) * a.Hq + h;
-                    },
-                    static_cast<__nv_bfloat16*>(a.out), a.lse_out);
-    }
-  }
-
-  if (bp.nb == 0 && a.nsplit == 1 && warp >= 2) {
-    // no key at all for this tile (a prefix-only call on an empty slice):
-    // O = 0 and lse = -inf, so a later merge gives the tile no weight
+  // ------------------------------------------------------------------ write-out
+  // The softmax threads stage their normalised O (32 columns of one row each)
+  // and the rows' lse in the idle K ring; then every warp stores whole rows:
+  // the bf16 output (one split), or this split's fp32 partials, which the
+  // splits of a cluster then merge (cluster_merge) or a finalize launch does.
+  // A CTA without keys (an empty slice of a prefix-only call, or a split past
+  // a short sequence's prefix) contributes O = 0 with lse = -inf.
+  float* ost = reinterpret_cast<float*>(smem + kOffK);
+  float* lst = ost + 128 * kStageStride;
+  int* wst = reinterpret_cast<int*>(lst + 128);
+  if (warp >= 2) {
     const int r = 32 * (warp & 3) + lane;
     const int t = (warp - 2) >> 3, hf = ((warp - 2) >> 2) & 1;
-    if (r < rows_valid) {
-      const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
-      const size_t row = (size_t)(b * a.R + rho) * a.Hq + h;
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * 128 + 32 * (2 * t + hf));
-      for (int e = 0; e < 4; ++e) dst[e] = make_uint4(0, 0, 0, 0);
-      if (t == 0 && hf == 0 && a.lse_out) a.lse_out[row] = -INFINITY;
+    if (bp.nb == 0) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ov[e] = 0.f;
+      olse = -INFINITY;
+      owrite = r < rows_valid;
     }
+    float4* d = reinterpret_cast<float4*>(ost + r * kStageStride + 32 * (2 * t + hf));
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) d[e / 4] = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
+    if (t == 0 && hf == 0) {
+      lst[r] = owrite ? olse : -INFINITY;
+      wst[r] = owrite ? 1 : 0;
+    }
+    if (warp == 4 && lane == 0) TIDAR_TRACE_AT(1543);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) TIDAR_TRACE_AT(1544);
+  auto out_row = [&](int r) -> long long {
+    const int rho = rho0 + r / a.G, h = g * a.G + r % a.G;
+    return (long long)(b * a.R + rho) * a.Hq + h;
+  };
+  if (a.nsplit == 1) {
+    store_rows_bf16(ost, lst, wst, rows_valid, out_row, static_cast<__nv_bfloat16*>(a.out), a.lse_out);
+  } else if (a.cluster_merge) {
+    // ---------------------------------------------------------------- split merge
+    // The CTAs of this cluster are the splits of one (b, g, tile) (cluster
+    // rank = split): once all of them have staged their rows (first cluster
+    // barrier), CTA j merges rows j, j + ns, j + 2 ns, ... of the tile from
+    // every split's shared memory; the second barrier keeps each CTA's shared
+    // memory alive until its peers are done.
+    const int ns = a.nsplit;
+    const int rank = (int)cluster_rank();
+    cluster_sync_all();
+    if (threadIdx.x == 0) { TIDAR_TRACE_AT(1540); TIDAR_TRACE_CTA(3); }
+    const int owned = rows_valid > rank ? (rows_valid - rank + ns - 1) / ns : 0;
+    merge_rows<4, 2>(ost, lst, ns, rank, owned, out_row, static_cast<__nv_bfloat16*>(a.out), a.lse_out);
+    if (threadIdx.x == 0) TIDAR_TRACE_AT(1541);
+    cluster_sync_all();
+  } else {
+    const long long stride = (long long)a.B * a.R * a.Hq;
+    store_rows_partial(ost, lst, wst, rows_valid, [&](int r) -> long long { return split * stride + out_row(r); },
+                       a.part_o, a.part_lse);
+    if (warp == 4 && lane == 0) TIDAR_TRACE_AT(1539);
   }
 
   if (tile == 0 && split == 0 && len_ok && (a.nsplit == 1 || a.cluster_merge) && a.append) {
@@ -707,7 +707,7 @@ extern "C" int tidar_trace_read(void* dst, size_t bytes) {
   return (int)cudaMemcpyFromSymbol(dst, g_tidar_trace, bytes);
 }
 extern "C" int tidar_trace_clear(void) {
-  static unsigned long long zeros[2048 + 2 * 8192];
+  static unsigned long long zeros[2048 + 4 * 8192];
   return (int)cudaMemcpyToSymbol(g_tidar_trace, zeros, sizeof zeros);
 }
 #endif
@@ -744,8 +744,8 @@ cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s) {
   }
   cudaError_t e = set_smem_attr();
   if (e != cudaSuccess) return e;
-  if (a.nsplit > 1 && (!a.part_o || !a.part_lse)) return cudaErrorInvalidValue;   // partials are staged
   const bool clu = a.nsplit > 1 && a.cluster_merge;
+  if (a.nsplit > 1 && !clu && (!a.part_o || !a.part_lse)) return cudaErrorInvalidValue;
   if (clu && a.nsplit > kMaxCluster) return cudaErrorNotSupported;
   const dim3 grid(prm.tiles, a.nsplit, a.B * a.Hkv);
   // with the cluster merge, the splits of one (b, g, tile) form a cluster

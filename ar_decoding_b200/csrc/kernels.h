@@ -29,7 +29,7 @@ struct AttnArgs {
   int step_keys;         // 1: the last split also attends the step keys (the zone mask); 0: prefix only
   int append;            // 1: write the draft rows' K/V into the cache
   int cluster_merge;     // nsplit > 1: the splits of a tile are one cluster and merge in the kernel
-                         // (partials through part_o / part_lse in L2); 0: a finalize launch merges
+                         // (part_o unused); 0: partials in part_o / part_lse, a finalize launch merges
 };
 
 // Warp-MMA kernel for query blocks of at most 16 packed rows per KV head
@@ -45,9 +45,9 @@ cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 // the tensor maps cannot be built.
 cudaError_t launch_attn_tc05(const AttnArgs& a, cudaStream_t s);
 // How many clusters of `ns` tcgen05 attention CTAs (one per key split) this
-// device holds at once; 0 if none.  The splits always write part_o / part_lse;
-// with cluster_merge they form such a cluster and merge those partials in the
-// kernel (which then also performs the draft-row append), else
+// device holds at once; 0 if none.  With cluster_merge the splits form such a
+// cluster and merge over distributed shared memory (and the kernel performs
+// the draft-row append), else they write part_o / part_lse and
 // launch_finalize merges and appends.
 int tc05_resident_clusters(int ns);
 // Tensor-core kernel with two 128-row query tiles per CTA sharing each staged

@@ -495,12 +495,14 @@ LinearPlan plan_linear(int T, int K, int N) {
   if (p.stages > kLinMaxStages) p.stages = kLinMaxStages;
   p.smem = p.stages * p.stage_bytes + extra;
   // Split count: the waves of clusters the launch needs times (the k-blocks
-  // of one split + a fixed per-CTA cost), plus the reduction through L2, in
-  // units of one 64-wide k-block.  Without a device (host-only planning) the
-  // occupancy is taken as one cluster per ks SMs.
+  // of one split + a fixed per-CTA cost: ramp-up, partials, the wait for the
+  // slowest split of the cluster), plus the reduction through L2, in units of
+  // one 64-wide k-block (about 0.5 us with every SM streaming).  Without a
+  // device (host-only planning) the occupancy is taken as one cluster per ks
+  // SMs.
   const int kb = K / 64;
   const long long base = (long long)(N / 128) * p.tiles;
-  constexpr double kFixed = 4.0, kReduce = 1.5;
+  constexpr double kFixed = 10.0, kReduce = 1.5;
   double best = 1e300;
   int best_ks = 1;
   for (int ks = 1; ks <= kLinMaxSplit && ks <= kb; ++ks) {

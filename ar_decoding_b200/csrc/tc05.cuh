@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace tidar {
 namespace tc05 {
@@ -175,81 +176,169 @@ __device__ __forceinline__ BlockPlan make_block_plan(const AttnArgs& a, int P, i
 
 __device__ __forceinline__ bool page_ok(int page, int num_pages) { return page >= 0 && page < num_pages; }
 
-// ------------------------------------------------------------------ split merge
-// Key splits of one query tile run as the CTAs of a thread-block cluster and
-// merge through L2.  Every split has written its normalised partial rows (fp32
-// O of 128 columns, and the row's lse) to part_o / part_lse, laid out
-// [split][stride rows]; a cluster barrier (release / acquire at cluster scope)
-// orders those writes before these reads.  This CTA merges `owned` rows,
-// row_of(i) giving the i-th one's row index (negative: skip).  A group of
-// 32 / CPT threads merges one row, CPT float4 columns each, so that with
-// enough threads every owned row is in flight at once: one round trip for the
-// lse of all splits, one for the rows.  Loads bypass L1 (other SMs wrote the
-// partials).  The weights are exp(lse_s - max); a split with lse = -inf saw no
-// key and may have written no values: it is selected away, not multiplied.
-template <int CPT, class RowOf>
-__device__ __forceinline__ void merge_l2_rows_t(const float* __restrict__ part_o,
-                                                const float* __restrict__ part_lse, long long stride, int ns,
-                                                int owned, RowOf row_of, __nv_bfloat16* out, float* lse_out) {
-  constexpr int kG = 32 / CPT;
-  const int sub = (int)threadIdx.x % kG;
-  const int groups = (int)blockDim.x / kG;
-  for (int i = (int)threadIdx.x / kG; i < owned; i += groups) {
+// ------------------------------------------------------------------ row write-out
+// After the main loop a CTA's normalised O rows pass through shared memory,
+// `kStageStride` floats per row (the padding keeps the softmax threads' row
+// writes -- one row per lane -- free of bank conflicts), so that every global
+// store and load below moves whole rows: one warp instruction per row of 128
+// columns, lane l holding columns 4l .. 4l+3.  lst / wst hold each row's lse
+// (-inf where the row could not be computed) and whether it is valid (a CTA
+// whose bounded wait ran out writes no output rows, and its partial rows get
+// lse = -inf).
+constexpr int kStageStride = 132;
+
+// Final bf16 rows and their lse; row_of(i) = output row of staged row i
+// (negative: no such row).
+template <class RowOf>
+__device__ __forceinline__ void store_rows_bf16(const float* ost, const float* lst, const int* wst, int nrows,
+                                                RowOf row_of, __nv_bfloat16* out, float* lse_out) {
+  const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31, nw = (int)blockDim.x >> 5;
+  for (int i = warp; i < nrows; i += nw) {
+    if (!wst[i]) continue;
     const long long row = row_of(i);
     if (row < 0) continue;
-    float l2[kMaxCluster];
-    float mx = -INFINITY;
+    const float4 v = *reinterpret_cast<const float4*>(ost + i * kStageStride + 4 * lane);
+    uint2 u;
+    u.x = cvt_bf16x2(v.x, v.y);
+    u.y = cvt_bf16x2(v.z, v.w);
+    *reinterpret_cast<uint2*>(out + row * 128 + 4 * lane) = u;
+    if (lane == 0 && lse_out) lse_out[row] = lst[i];
+  }
+}
+
+// fp32 partial rows of one key split; prow_of(i) = row of staged row i in the
+// partials, laid out [split][rows][128] and [split][rows] (negative: no such
+// row).
+template <class RowOf>
+__device__ __forceinline__ void store_rows_partial(const float* ost, const float* lst, const int* wst, int nrows,
+                                                   RowOf prow_of, float* part_o, float* part_lse) {
+  const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31, nw = (int)blockDim.x >> 5;
+  for (int i = warp; i < nrows; i += nw) {
+    const long long prow = prow_of(i);
+    if (prow < 0) continue;
+    const bool w = wst[i] != 0;
+    if (w) reinterpret_cast<float4*>(part_o + prow * 128)[lane] = *reinterpret_cast<const float4*>(ost + i * kStageStride + 4 * lane);
+    if (lane == 0) part_lse[prow] = w ? lst[i] : -INFINITY;
+  }
+}
+
+// Split merge over distributed shared memory.  The splits of a query tile are
+// the CTAs of one thread-block cluster (cluster rank = split); every CTA has
+// staged its normalised rows (ost, kStageStride floats per row) and their lse
+// (lst; -inf for a row it could not compute) in its own shared memory, and a
+// cluster barrier orders that before these reads.  This CTA merges staged
+// rows r = i * ns + rank for i < owned: lane s < ns reads split s's lse, the
+// weights exp(lse_s - max) and their sum come from warp shuffles, then every
+// lane reads its 4 columns of each split's row -- 512 contiguous bytes per
+// warp and split, so the owner's banks see no conflicts -- U rows per warp in
+// flight.  A split with lse = -inf saw no key: its weight is 0 and its row is
+// selected away, not multiplied.  out_row(r) = output row of staged row r
+// (negative: no such row).  The caller keeps its shared memory alive (a second
+// cluster barrier) until every peer is done reading.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+template <int U, int NC, class RowOf>
+__device__ __forceinline__ void merge_rows_t(const float* ost, const float* lst, int ns, int rank, int owned,
+                                             RowOf out_row, __nv_bfloat16* out, float* lse_out) {
+  const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31, nw = (int)blockDim.x >> 5;
+  constexpr unsigned kAll = 0xffffffffu;
+  const uint32_t ost_a = smem_u32(ost), lst_a = smem_u32(lst);
+  for (int i0 = warp * U; i0 < owned; i0 += nw * U) {
+    int r[U];
+    long long orow[U];
+    float w[U], wsum[U], mx[U];
+    float4 x[U][NC];
+    // the lse of every split and the rows of the first NC splits are all in
+    // flight before the first of them is used
+    auto load_chunk = [&](int s0) {
 #pragma unroll
-    for (int s = 0; s < kMaxCluster; ++s) {
-      l2[s] = s < ns ? __ldcg(part_lse + s * stride + row) * 1.4426950408889634f : -INFINITY;
-      mx = fmaxf(mx, l2[s]);
+      for (int j = 0; j < NC; ++j) {
+        const int sp = s0 + j;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          x[u][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (orow[u] >= 0 && sp < ns) {
+            const int e = r[u] * kStageStride + 4 * lane;
+            x[u][j] = sp == rank ? *reinterpret_cast<const float4*>(ost + e)
+                                 : ld_cluster_f32x4(mapa(ost_a + 4u * (uint32_t)e, (uint32_t)sp));
+          }
+        }
+      }
+    };
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      r[u] = (i0 + u) * ns + rank;
+      orow[u] = i0 + u < owned ? out_row(r[u]) : -1;
+      w[u] = (orow[u] >= 0 && lane < ns)
+                 ? ld_cluster_f32(mapa(lst_a + 4u * (uint32_t)r[u], (uint32_t)lane)) * 1.4426950408889634f
+                 : -INFINITY;
     }
-    float4 acc[CPT];
+    load_chunk(0);
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float wsum = 0.f;
+    for (int u = 0; u < U; ++u) {
+      float m = w[u];
 #pragma unroll
-    for (int s = 0; s < kMaxCluster; ++s) {
-      if (s < ns) {
-        const float4* src = reinterpret_cast<const float4*>(part_o + (s * stride + row) * 128) + sub * CPT;
-        float4 x[CPT];
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kAll, m, o));
+      mx[u] = m;
+      w[u] = w[u] == -INFINITY ? 0.f : ex2(w[u] - m);
+      float sm = w[u];
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) x[c] = __ldcg(src + c);
-        if (l2[s] != -INFINITY) {
-          const float w = ex2(l2[s] - mx);
-          wsum += w;
+      for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(kAll, sm, o);
+      wsum[u] = sm;
+    }
+    float4 acc[U];
 #pragma unroll
-          for (int c = 0; c < CPT; ++c) {
-            acc[c].x = fmaf(w, x[c].x, acc[c].x); acc[c].y = fmaf(w, x[c].y, acc[c].y);
-            acc[c].z = fmaf(w, x[c].z, acc[c].z); acc[c].w = fmaf(w, x[c].w, acc[c].w);
+    for (int u = 0; u < U; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < ns; s0 += NC) {
+      if (s0 > 0) load_chunk(s0);
+#pragma unroll
+      for (int j = 0; j < NC; ++j) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const float ws = __shfl_sync(kAll, w[u], (s0 + j) & 31);
+          if (s0 + j < ns && ws > 0.f) {
+            acc[u].x = fmaf(ws, x[u][j].x, acc[u].x); acc[u].y = fmaf(ws, x[u][j].y, acc[u].y);
+            acc[u].z = fmaf(ws, x[u][j].z, acc[u].z); acc[u].w = fmaf(ws, x[u][j].w, acc[u].w);
           }
         }
       }
     }
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-      uint2 u;
-      u.x = cvt_bf16x2(acc[c].x * inv, acc[c].y * inv);
-      u.y = cvt_bf16x2(acc[c].z * inv, acc[c].w * inv);
-      *reinterpret_cast<uint2*>(out + row * 128 + 4 * (sub * CPT + c)) = u;
+    for (int u = 0; u < U; ++u) {
+      if (orow[u] < 0) continue;
+      const float inv = wsum[u] > 0.f ? 1.f / wsum[u] : 0.f;
+      uint2 o;
+      o.x = cvt_bf16x2(acc[u].x * inv, acc[u].y * inv);
+      o.y = cvt_bf16x2(acc[u].z * inv, acc[u].w * inv);
+      *reinterpret_cast<uint2*>(out + orow[u] * 128 + 4 * lane) = o;
+      if (lane == 0 && lse_out)
+        lse_out[orow[u]] = wsum[u] > 0.f ? (mx[u] + log2f(wsum[u])) * 0.69314718055994531f : -INFINITY;
     }
-    if (sub == 0 && lse_out) lse_out[row] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -INFINITY;
   }
 }
 
-// This CTA's share of the merge, the group size picked so that all `owned`
-// rows go in one pass when the block has the threads (at most 8 columns of 4
-// per thread).
-template <class RowOf>
-__device__ __forceinline__ void merge_l2_rows(const float* part_o, const float* part_lse, long long stride,
-                                              int ns, int owned, RowOf row_of, __nv_bfloat16* out,
-                                              float* lse_out) {
-  const int per = (32 * owned + (int)blockDim.x - 1) / (int)blockDim.x;
-  if (per <= 1) merge_l2_rows_t<1>(part_o, part_lse, stride, ns, owned, row_of, out, lse_out);
-  else if (per <= 2) merge_l2_rows_t<2>(part_o, part_lse, stride, ns, owned, row_of, out, lse_out);
-  else if (per <= 4) merge_l2_rows_t<4>(part_o, part_lse, stride, ns, owned, row_of, out, lse_out);
-  else merge_l2_rows_t<8>(part_o, part_lse, stride, ns, owned, row_of, out, lse_out);
+// This CTA's share of the merge: U rows per warp (at most kMaxU), NC splits'
+// rows in flight per chunk, U picked so that the block's warps take all
+// `owned` rows in one pass where they can (ns <= 32).
+template <int kMaxU, int NC, class RowOf>
+__device__ __forceinline__ void merge_rows(const float* ost, const float* lst, int ns, int rank, int owned,
+                                           RowOf out_row, __nv_bfloat16* out, float* lse_out) {
+  const int nw = (int)blockDim.x >> 5;
+  const int per = (owned + nw - 1) / nw;
+  if (per <= 1 || kMaxU == 1) merge_rows_t<1, NC>(ost, lst, ns, rank, owned, out_row, out, lse_out);
+  else if (per <= 2 || kMaxU == 2) merge_rows_t<2, NC>(ost, lst, ns, rank, owned, out_row, out, lse_out);
+  else merge_rows_t<4, NC>(ost, lst, ns, rank, owned, out_row, out, lse_out);
 }
 
 }  // namespace tc05

@@ -144,16 +144,16 @@ typedef struct {
  *   q        [B][R][Hq][D]     k_blk, v_blk [B][R][Hkv][D]     (dtype)
  *   out      [B][R][Hq][D]     (dtype)     lse_out [B][R][Hq] fp32 or NULL
  *   workspace: device scratch of at least tidar_step_attn_workspace_bytes(desc)
- *     bytes, 256-byte aligned (may be NULL when that size is 0: one split);
- *     the splits' partial rows pass through it.  Contents on entry are
- *     ignored.  Calls that share a workspace must be stream-ordered.
+ *     bytes, 256-byte aligned (may be NULL when that size is 0: one split, or
+ *     splits merged inside the kernel); it holds split partials for the
+ *     second launch.  Contents on entry are ignored.  Calls that share a
+ *     workspace must be stream-ordered.
  * Device errors: BAD_PAGE (prefix or draft page unmapped), BAD_LEN; the TC05
  * and DEC kernels also TIMEOUT (a bounded wait on a copy or on a cluster
  * peer ran out) and LAYOUT.  Splits of a long prefix merge inside the
- * attention kernel (the splits of a query tile form a thread-block cluster;
- * the tensor-core kernels pass the partial rows through the workspace in L2,
- * the decode kernel through distributed shared memory) when such clusters
- * can be scheduled, else in a second launch.  That second launch also writes the
+ * attention kernel (the splits of a query tile form a thread-block cluster and
+ * read each other's rows over distributed shared memory) when such clusters
+ * can be scheduled, else through workspace partials in a second launch.  That second launch also writes the
  * draft rows; without it the tensor-core and decode kernels write them (SIMT
  * always takes the second launch).
  * ------------------------------------------------------------------------- */

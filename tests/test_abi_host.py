@@ -84,7 +84,7 @@ def test_step_attn_rejects_small_workspace(L):
 
 def test_tensor_core_plan_splits_long_prefixes(L):
     # one query row per head: the 8192-key prefix is split to fill the SMs; the
-    # split partials pass through the workspace whichever way they merge
+    # workspace holds split partials unless the kernel merges them itself
     d = _desc(max_prefix_len=8192, batch=1, num_q_heads=32, num_kv_heads=8, k=0,
               path=tidar.PATH_TC05)
     path, splits, merge = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
@@ -94,8 +94,8 @@ def test_tensor_core_plan_splits_long_prefixes(L):
     assert L.tidar_step_attn_plan(ctypes.byref(d), None, None, None) == tidar.OK
     ws = L.tidar_step_attn_workspace_bytes(ctypes.byref(d))
     rows = 32                                  # B * R * Hq
-    assert ws == ((splits.value * rows * 128 * 4 + 255) // 256 * 256) + \
-        ((splits.value * rows * 4 + 255) // 256 * 256)
+    assert ws == (0 if merge.value == 1 else ((splits.value * rows * 128 * 4 + 255) // 256 * 256) +
+                  ((splits.value * rows * 4 + 255) // 256 * 256))
     assert tidar.plan_full(d) == (path.value, splits.value, merge.value)
 
 

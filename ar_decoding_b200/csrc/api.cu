@@ -440,7 +440,7 @@ tidar_status tidar_verify_blockq(int32_t batch, int32_t k, int32_t vocab, tidar_
 size_t tidar_verify_sampled_workspace_bytes(int32_t batch, int32_t k, int32_t vocab,
                                             tidar_accept_mode mode) {
   if (batch <= 0 || k < 0 || k > 16 || vocab <= 0) return 0;
-  if (mode == TIDAR_GREEDY) return 0;
+  if (mode == TIDAR_GREEDY) return tidar_verify_workspace_bytes(batch, k, vocab, mode);   // tidar_verify's
   return align256(tidar::sampled_verify_workspace_bytes(batch, k));
 }
 

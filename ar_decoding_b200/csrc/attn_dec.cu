@@ -151,6 +151,14 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(bar(i), i == DBAR_MERGE ? (uint32_t)a.nsplit : (i >= DBAR_EMPTY ? 4u : 1u));
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&tm_q);      // kernel parameters: safe before the dependency wait
+    prefetch_tmap(&tm_kp);
+    prefetch_tmap(&tm_vp);
+    prefetch_tmap(&tm_ks);
+    prefetch_tmap(&tm_vs);
+    const int bq = blockIdx.y / a.Hkv;
+    prefetch_l2(a.seq_lens + bq, 4, 0, 1);
+    prefetch_l2(a.page_table + (size_t)bq * a.max_pages + blockIdx.x * a.keys_per_split / 64, 256, 0, 1);
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();

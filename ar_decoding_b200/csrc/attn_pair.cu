@@ -150,6 +150,13 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (layout_ok) {
       for (int i = 0; i < kPBars; ++i) mbar_init(bar(i), (i == PB_PFULL || i == PB_PFULL + 1) ? 4u : 1u);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_kp);
+      prefetch_tmap(&tm_vp);
+      prefetch_tmap(&tm_ks);
+      prefetch_tmap(&tm_vs);
+      prefetch_l2(a.seq_lens + b, 4, 0, 1);
+      prefetch_l2(a.page_table + (size_t)b * a.max_pages + split * a.keys_per_split / 64, 256, 0, 1);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     } else {
       raise_error(a.err, TIDAR_DEVERR_LAYOUT);

@@ -140,6 +140,31 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
   const AttnArgs& a = prm.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Set-up that reads nothing the previous kernel on the stream may write
+  // (barriers, the tensor maps) runs before the dependency wait, so it
+  // overlaps that kernel's tail.
+  if (threadIdx.x == 0) {
+    TIDAR_TRACE_CTA(0);
+    TIDAR_TRACE_AT(0);
+#ifdef TIDAR_TRACE
+    if (trace_cta()) g_tidar_trace[2] = clock64();
+#endif
+    for (int i = 0; i < kNumBars; ++i) {
+      const bool pfull = i >= BAR_PFULL && i < BAR_PFULL + kStages;
+      mbar_init(sb + kOffBar + 8u * i, pfull ? 8u : 1u);
+    }
+    reinterpret_cast<volatile int*>(smem + kOffMisc)[1] = 0;     // abort flag
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_kp);
+    prefetch_tmap(&tm_vp);
+    prefetch_tmap(&tm_ks);
+    prefetch_tmap(&tm_vs);
+    const int bq = blockIdx.z / prm.a.Hkv;
+    prefetch_l2(prm.a.seq_lens + bq, 4, 0, 1);
+    prefetch_l2(prm.a.page_table + (size_t)bq * prm.a.max_pages + blockIdx.y * prm.a.keys_per_split / 64, 256, 0, 1);
+  }
   pdl_wait();       // the previous kernel on the stream is complete from here on
   pdl_trigger();
   // The producer's first two 32-page windows of the page table do not depend on
@@ -170,27 +195,13 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8u * i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-
-  if (threadIdx.x == 0) {
-    TIDAR_TRACE_CTA(0);
-    TIDAR_TRACE_AT(0);
-#ifdef TIDAR_TRACE
-    if (trace_cta()) g_tidar_trace[2] = clock64();
-#endif
-    for (int i = 0; i < kNumBars; ++i) {
-      const bool pfull = i >= BAR_PFULL && i < BAR_PFULL + kStages;
-      mbar_init(bar(i), pfull ? 8u : 1u);
-    }
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-  if (warp == 1 && bp.nb > 0) {
+  if (warp == 1) {      // every CTA holds TMEM (released at the end), keys or not
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sb + kOffMisc),
                  "r"(kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+
   fence_before();
   __syncthreads();
   fence_after();
@@ -675,7 +686,7 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (trace_cta()) g_tidar_trace[3] = clock64();
 #endif
   }
-  if (warp == 1 && bp.nb > 0) {
+  if (warp == 1) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }

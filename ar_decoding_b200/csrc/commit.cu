@@ -8,7 +8,8 @@
 // are released.
 //
 // One launch: a single thread-block cluster of C <= 16 CTAs; CTA r owns the
-// contiguous sequences [r*per, (r+1)*per).
+// contiguous sequences [r*per, (r+1)*per) (with fewer sequences than CTAs,
+// the zeroing of step 3 is shared by the whole cluster).
 //   1. every CTA validates its own sequences (one warp per sequence, the
 //      page-table entries loaded by parallel lanes) and counts the pages each
 //      releases (-1: invalid, left untouched), then an exclusive scan of the
@@ -62,6 +63,12 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
   extern __shared__ int s_dyn[];
   SeqRec* s_rec = reinterpret_cast<SeqRec*>(s_dyn);
   int* s_pg = s_dyn + 4 * per;                      // [per][npm]
+  // With fewer sequences than CTAs every CTA also keeps a record of every
+  // sequence (read in step 1, before any CTA advances a length), so that the
+  // whole cluster zeroes the rejected rows instead of their owners alone.
+  const bool spread = a.B < C;
+  SeqRec* s_all = reinterpret_cast<SeqRec*>(s_pg + per * npm);   // [B] when spread
+  int* s_allpg = s_pg + per * npm + 4 * (spread ? a.B : 0);      // [B][npm] when spread
   __shared__ int s_total, s_base, s_grand;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int b0 = rank * per;
@@ -96,6 +103,28 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
       r.P = P; r.c = c; r.off = 0;
       r.cnt = ok ? (P + a.n + ps - 1) / ps - (P + c + ps - 1) / ps : -1;
       s_rec[i] = r;
+    }
+  }
+  if (spread) {
+    // the same reads as above without the error reports (owners make those)
+    for (int b = wid; b < a.B; b += kCWarps) {
+      const int P = a.seq_lens[b], c = a.accept_count[b];
+      bool ok = c >= 0 && c <= a.n && P >= 0 && (P + a.n + ps - 1) / ps <= a.max_pages;
+      if (ok) {
+        const int p0 = P / ps, np = (P + a.n - 1) / ps - p0 + 1;
+        bool bad = false;
+        if (lane < np) {
+          const int page = a.page_table[(size_t)b * a.max_pages + p0 + lane];
+          bad = page < 0 || page >= a.num_pages;
+          s_allpg[b * npm + lane] = page;
+        }
+        ok = !__any_sync(0xffffffffu, bad);
+      }
+      if (lane == 0) {
+        SeqRec r;
+        r.P = P; r.c = c; r.off = 0; r.cnt = ok ? 0 : -1;
+        s_all[b] = r;
+      }
     }
   }
   __syncthreads();
@@ -149,19 +178,23 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
   }
   const int row_chunks = a.D * a.elem_bytes / 16;
   const int head_chunks = a.Hkv * row_chunks;       // one row of one of K / V, all heads
-  for (int i = 0; i < nown; ++i) {
-    const SeqRec r = s_rec[i];
+  const int nscrub = spread ? a.B : nown;
+  const int t0 = spread ? rank * kCThreads + (int)threadIdx.x : (int)threadIdx.x;
+  const int tstep = spread ? C * kCThreads : kCThreads;
+  for (int i = 0; i < nscrub; ++i) {
+    const SeqRec r = spread ? s_all[i] : s_rec[i];
+    const int* pg = spread ? s_allpg + i * npm : s_pg + i * npm;
     if (r.cnt < 0) continue;
     const int p0 = r.P / ps;
     const int total = (a.n - r.c) * 2 * head_chunks;
-    for (int t = threadIdx.x; t < total; t += kCThreads) {
+    for (int t = t0; t < total; t += tstep) {
       const int rr = t / (2 * head_chunks);
       const int rem = t - rr * 2 * head_chunks;
       const int which = rem >= head_chunks;
       const int hc = rem - which * head_chunks;
       const int g = hc / row_chunks, ch = hc - g * row_chunks;
       const int pos = r.P + r.c + rr;
-      const int page = s_pg[i * npm + pos / ps - p0];
+      const int page = pg[pos / ps - p0];
       char* dst = static_cast<char*>(which ? a.v_pages : a.k_pages);
       const size_t off = (((size_t)page * a.Hkv + g) * ps + pos % ps) * a.D * a.elem_bytes;
       reinterpret_cast<uint4*>(dst + off)[ch] = make_uint4(0, 0, 0, 0);
@@ -198,10 +231,12 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t s) {
   static int limit_cache[64];
   static bool smem_set[64];
   const int slots = (a.n + a.page_size - 1) / a.page_size + 1;
-  const int C = min(a.B, cluster_limit(commit_cluster_kernel, kCThreads, limit_cache));
+  // at least as many CTAs as the cluster allows: with a small batch the idle
+  // ones share the zeroing of the rejected rows
+  const int C = cluster_limit(commit_cluster_kernel, kCThreads, limit_cache);
   const int per = (a.B + C - 1) / C;
   const int npm = commit_npm(a.n, a.page_size);
-  const size_t smem = commit_smem(per, npm);
+  const size_t smem = commit_smem(per + (a.B < C ? a.B : 0), npm);
   if (smem > kCommitSmemMax) return cudaErrorNotSupported;
   int dev = 0;
   cudaGetDevice(&dev);

@@ -259,6 +259,8 @@ linear_tc05_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
     // partials, so it is set even when the layout check fails
     *abort_flag = layout_ok ? 0 : 1;
     if (layout_ok) {
+      prefetch_tmap(&tm_w);      // kernel parameters: safe before the dependency wait
+      prefetch_tmap(&tm_x);
       for (int i = 0; i < 2 * kLinMaxStages + 1; ++i) mbar_init(bar(i), 1u);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

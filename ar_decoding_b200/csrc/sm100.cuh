@@ -101,6 +101,25 @@ __device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, vol
   return __all_sync(0xffffffffu, ok);
 }
 
+// Fetch a tensor map (a __grid_constant__ kernel parameter) into the
+// descriptor cache ahead of its first copy.  Kernel parameters are not outputs
+// of the previous kernel, so this may run before the dependency wait.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// L2 prefetch of [p, p + bytes), spread over `nthreads` threads: warms L2 and
+// the address translation for data read after the dependency wait.  Only a
+// hint -- it returns no data, and anything the previous kernel writes
+// meanwhile is what the real loads see (L2 is the point of coherence) -- so
+// it may run before the wait; its addresses must come from kernel arguments,
+// never from memory the previous kernel may write.
+__device__ __forceinline__ void prefetch_l2(const void* p, size_t bytes, int tid, int nthreads) {
+  const char* c = static_cast<const char*>(p);
+  for (size_t off = (size_t)tid * 128; off < bytes; off += (size_t)nthreads * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(c + off));
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             uint32_t bar) {
   asm volatile(

@@ -14,7 +14,8 @@
 //   stats:     grid (chunks, rows).  One CTA sweeps CHUNK logits of one row with
 //              16-byte loads: exact max / argmax (lowest index on ties) and,
 //              for rejection, the fp64 sum of exp(x - chunk max).
-//   greedy:    grid (B).  Merges the chunk argmaxes, scans, writes outputs.
+//   greedy:    one warp per sequence.  Merges the chunk argmaxes, scans, writes
+//              the outputs.
 //   rejection: residual (grid (chunks, B)) recomputes the row normalisers from
 //              the chunk stats, runs the accept scan (fp64), and sums the
 //              sampling weights of its chunk; select (grid (B)) locates the
@@ -112,11 +113,33 @@ __device__ __forceinline__ int load_chunk(const T* row, int V, int c0, float (&x
   return cnt;
 }
 
+// Optional timeline (build with -DTIDAR_TRACE; absent from normal builds):
+// statistics CTA (0, 0) [0] start, [1] after the wait on the previous kernel,
+// [2] end; acceptance warp of sequence 0 [8] start, [9] after the wait, [10]
+// end.
+#ifdef TIDAR_TRACE
+__device__ unsigned long long g_verify_trace[16 * 8];
+#define VERIFY_TRACE(cond, slot) do { if (cond) { unsigned long long t_; \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_)); g_verify_trace[(slot)] = t_; } } while (0)
+#else
+#define VERIFY_TRACE(cond, slot) do {} while (0)
+#endif
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat* stats, int nchunk,
                                                          bool vec_ok) {
+  const bool tr = blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0;
+  VERIFY_TRACE(tr, 0);
+  if ((int)blockIdx.y < a.B * a.n) {
+    // this CTA's chunk of its logits row into L2 while the previous kernel ends
+    const int lo = (int)blockIdx.x * kChunk, hi = min(a.V, lo + kChunk);
+    if (hi > lo)
+      prefetch_l2(static_cast<const T*>(a.logits) + (size_t)blockIdx.y * a.V + lo, (size_t)(hi - lo) * sizeof(T),
+                  (int)threadIdx.x, kThreads);
+  }
   pdl_wait();
   pdl_trigger();
+  VERIFY_TRACE(tr, 1);
   const int c = blockIdx.x, rr = blockIdx.y;
   const int prow = a.B * a.n;
   const T* row = rr < prow ? static_cast<const T*>(a.logits) + (size_t)rr * a.V
@@ -166,6 +189,7 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat
     st.max = cmax; st.arg = carg; st.sum = sum;
     stats[(size_t)rr * nchunk + c] = st;
   }
+  VERIFY_TRACE(tr, 2);
 }
 
 // Writes accept_count, out_tokens, selected_block, next_drafts for sequence b.
@@ -186,202 +210,54 @@ __device__ void write_outputs(const VerifyArgs& a, int b, int j, int t_star) {
   }
 }
 
-// Greedy verification in one launch: one thread-block cluster per sequence b.
-// The cluster's C CTAs split the n rows of b into n*S (row, slice) items
-// (S = C / n slices per row when n <= C, else S = 1 and a CTA takes several
-// rows); each CTA streams its items' logits with 16-byte loads and leaves one
-// exact (max, argmax) pair per item in its shared memory.  After a cluster
-// barrier, CTA 0 merges the pairs of each row over distributed shared memory,
-// runs the accept scan with a warp ballot and writes the outputs.  A second
-// cluster barrier keeps every CTA's shared memory alive until CTA 0 has read it.
-// Optional timeline of sequence 0's cluster (build with -DTIDAR_TRACE; absent
-// from normal builds): [rank*8 + 0] start, +1 after the previous kernel, +2
-// sweep done, +3 past the first cluster barrier, +4 outputs written, +5 end.
-#ifdef TIDAR_TRACE
-__device__ unsigned long long g_verify_trace[16 * 8];
-__device__ __forceinline__ unsigned long long vt_now() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-#define VERIFY_TRACE(rank, slot) do { if (blockIdx.y == 0 && threadIdx.x == 0) g_verify_trace[(rank) * 8 + (slot)] = vt_now(); } while (0)
-#else
-#define VERIFY_TRACE(rank, slot) do {} while (0)
-#endif
-
-constexpr int kGThreads = 512;
-constexpr int kGUnroll = 8;
-
-template <typename T>
-__global__ void __launch_bounds__(kGThreads) greedy_cluster_kernel(VerifyArgs a, int S, int vec_ok) {
-  cg::cluster_group cl = cg::this_cluster();
-  const int C = (int)cl.num_blocks();
-  const int rank = (int)cl.block_rank();
-  const int b = blockIdx.y;
-  VERIFY_TRACE(rank, 0);
-  __shared__ float s_v[kMaxCluster];          // CTA 0: one (max, argmax) per item, pushed by its owner
-  __shared__ int s_i[kMaxCluster];
-  __shared__ __align__(8) uint64_t s_done;    // CTA 0: one arrival per CTA once its items are pushed
-  __shared__ float w_v[kGThreads / 32];
-  __shared__ int w_i[kGThreads / 32];
-  __shared__ int s_d[16];
-  __shared__ int s_am[16];
-  __shared__ int s_g[16 * 16];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const uint32_t done_bar = static_cast<uint32_t>(__cvta_generic_to_shared(&s_done));
-  if (rank == 0 && threadIdx.x == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(done_bar), "r"(C) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  // CTA 0's barrier is initialised (and every CTA running) before anyone pushes
-  // to it; the wait comes after the sweep, so this costs nothing
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+// Greedy acceptance from the chunk statistics (one warp per sequence b).  The
+// statistics kernel has left an exact (max, argmax) per 4096-wide chunk of
+// every logits row -- that sweep runs on as many CTAs as there are chunks,
+// since a single SM pulls only some tens of GB/s -- so lane i merges the
+// chunks of row i in chunk order (equal values keep the lower index), and the
+// drafts and block guesses are fetched before the statistics are needed.
+// d_{i+1} is kept while it equals argmax l_i: j = the first mismatching i,
+// else n; t* = argmax l_{j-1}.
+constexpr int kAccWarps = 4;
+__global__ void __launch_bounds__(kAccWarps * 32) greedy_accept_kernel(VerifyArgs a, const ChunkStat* stats,
+                                                                       int nchunk) {
+  __shared__ int s_g[kAccWarps][16 * 16];
+  const bool tr = blockIdx.x == 0 && threadIdx.x == 0;
+  VERIFY_TRACE(tr, 8);
   pdl_wait();
   pdl_trigger();
-  VERIFY_TRACE(rank, 1);
+  VERIFY_TRACE(tr, 9);
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x * kAccWarps + wid;
+  if (b >= a.B) return;                           // warp-uniform; no block-wide barrier below
   const bool want_g = a.next_drafts && a.block_guesses && a.k > 0;
-  // CTA 0 fetches the drafts and every block's guesses now, so those loads
-  // overlap the logits sweep instead of following the accept decision
-  if (rank == 0) {
-    const int t = threadIdx.x;
-    if (t < a.n) s_d[t] = (t >= 1 && a.k > 1) ? a.drafts[(size_t)b * a.k + t] : -1;
-    if (want_g && t < a.k * a.k) s_g[t] = a.block_guesses[(size_t)b * a.k * a.k + t];
+  // d_lane (lane >= 1) and every block's guesses: independent of the logits
+  const int d = (lane >= 1 && lane < a.n && a.k > 1) ? a.drafts[(size_t)b * a.k + lane] : -1;
+  if (want_g)
+    for (int t = lane; t < a.k * a.k; t += 32) s_g[wid][t] = a.block_guesses[(size_t)b * a.k * a.k + t];
+  float mv = -INFINITY;
+  int am = INT_MAX;
+  if (lane < a.n) {
+    const ChunkStat* st = stats + ((size_t)b * a.n + lane) * nchunk;
+    for (int c = 0; c < nchunk; ++c) amax_merge(mv, am, st[c].max, st[c].arg);
   }
-  const int L = (((a.V + S - 1) / S) + 7) & ~7;
-  float item_v[2];
-  int item_i[2], item_n = 0;
-  for (int it = rank; it < a.n * S; it += C) {
-    const int row = it / S, sl = it % S;
-    const int lo = sl * L, hi = min(a.V, lo + L);
-    const T* p = static_cast<const T*>(a.logits) + ((size_t)b * a.n + row) * a.V;
-    // four independent (max, argmax) chains per thread, merged at the end
-    float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    int bi[4] = {INT_MAX, INT_MAX, INT_MAX, INT_MAX};
-    if (vec_ok) {
-      constexpr int kVec = 16 / sizeof(T);
-      constexpr int kStride = kGThreads * kVec;
-      for (int base = lo + (int)threadIdx.x * kVec; base < hi; base += kStride * kGUnroll) {
-        // all the 16-byte loads first (kept raw, so they are in flight together),
-        // the conversions and compares after
-        uint4 raw[kGUnroll];
-#pragma unroll
-        for (int u = 0; u < kGUnroll; ++u) {
-          const int e0 = base + u * kStride;
-          raw[u] = e0 + kVec <= hi ? __ldg(reinterpret_cast<const uint4*>(p + e0)) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < kGUnroll; ++u) {
-          const int e0 = base + u * kStride;
-          float v[kVec];
-          if (e0 + kVec <= hi) {
-            load_vec<T, kVec>(reinterpret_cast<const T*>(&raw[u]), v);
-          } else {
-#pragma unroll
-            for (int e = 0; e < kVec; ++e) v[e] = e0 + e < hi ? ld(p, e0 + e) : -INFINITY;
-          }
-#pragma unroll
-          for (int e = 0; e < kVec; ++e) {
-            const int id = e0 + e, q = u & 3;
-            if (id < hi && (v[e] > bv[q] || bi[q] == INT_MAX)) { bv[q] = v[e]; bi[q] = id; }
-          }
-        }
-      }
-    } else {
-      for (int id = lo + (int)threadIdx.x; id < hi; id += kGThreads) {
-        const float x = ld(p, id);
-        if (x > bv[0] || bi[0] == INT_MAX) { bv[0] = x; bi[0] = id; }
-      }
-    }
-    amax_merge(bv[0], bi[0], bv[1], bi[1]);
-    amax_merge(bv[2], bi[2], bv[3], bi[3]);
-    amax_merge(bv[0], bi[0], bv[2], bi[2]);
-    float fv = bv[0];
-    int fi = bi[0];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float v2 = __shfl_xor_sync(0xffffffffu, fv, o);
-      const int i2 = __shfl_xor_sync(0xffffffffu, fi, o);
-      amax_merge(fv, fi, v2, i2);
-    }
-    if (lane == 0) { w_v[wid] = fv; w_i[wid] = fi; }
-    __syncthreads();
-    if (wid == 0) {
-      fv = lane < kGThreads / 32 ? w_v[lane] : -INFINITY;
-      fi = lane < kGThreads / 32 ? w_i[lane] : INT_MAX;
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) {
-        const float v2 = __shfl_xor_sync(0xffffffffu, fv, o);
-        const int i2 = __shfl_xor_sync(0xffffffffu, fi, o);
-        amax_merge(fv, fi, v2, i2);
-      }
-      if (lane == 0 && item_n < 2) { item_v[item_n] = fv; item_i[item_n] = fi; }
-    }
-    ++item_n;
-    __syncthreads();                              // w_v / w_i are reused by the next item
+  __syncwarp();
+  constexpr unsigned kAll = 0xffffffffu;
+  const int am_prev = __shfl_up_sync(kAll, am, 1);            // argmax l_{lane-1}
+  const bool mism = lane >= 1 && lane < a.n && d != am_prev;
+  const unsigned bal = __ballot_sync(kAll, mism);
+  const int j = bal ? __ffs(bal) - 1 : a.n;
+  const int t_star = __shfl_sync(kAll, am, j - 1);
+  const int d_next = __shfl_down_sync(kAll, d, 1);            // d_{lane+1}
+  if (lane < a.n)
+    a.out_tokens[(size_t)b * a.n + lane] = lane < j - 1 ? d_next : (lane == j - 1 ? t_star : -1);
+  if (a.next_drafts && a.k > 0 && lane < a.k)
+    a.next_drafts[(size_t)b * a.k + lane] = lane == 0 ? t_star : (want_g ? s_g[wid][(j - 1) * a.k + lane] : -1);
+  if (lane == 0) {
+    a.accept_count[b] = j;
+    if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
   }
-  VERIFY_TRACE(rank, 2);
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-  VERIFY_TRACE(rank, 3);
-  if (threadIdx.x == 0) {
-    // push this CTA's items (at most two) into CTA 0, then arrive on its barrier
-    int n_it = 0;
-    for (int it = rank; it < a.n * S; it += C, ++n_it) {
-      const uint32_t rv = mapa(static_cast<uint32_t>(__cvta_generic_to_shared(&s_v[it])), 0);
-      const uint32_t ri = mapa(static_cast<uint32_t>(__cvta_generic_to_shared(&s_i[it])), 0);
-      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(rv), "f"(item_v[n_it]) : "memory");
-      asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(ri), "r"(item_i[n_it]) : "memory");
-    }
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(done_bar, 0))
-                 : "memory");
-  }
-  if (rank != 0) return;                          // nothing of this CTA is read after its push
-  if (wid == 0) {
-    // every CTA's items are in (bounded wait: on expiry, record it and skip)
-    bool ok = false;
-    if (lane == 0) {
-      const uint64_t t0 = global_ns();
-      for (;;) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(done_bar)
-            : "memory");
-        if (done) { ok = true; break; }
-        if (global_ns() - t0 > kWaitLimitNs) break;
-      }
-      if (!ok) raise_error(a.err, TIDAR_DEVERR_TIMEOUT);
-    }
-    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
-    __syncwarp();
-    if (lane < a.n) {
-      float bv = -INFINITY;
-      int bi = INT_MAX;
-      for (int sl = 0; sl < S; ++sl) amax_merge(bv, bi, s_v[lane * S + sl], s_i[lane * S + sl]);
-      s_am[lane] = bi;
-    }
-    __syncwarp();
-    // d_{i+1} is kept while it equals argmax l_i: j = first mismatching i, else n
-    const bool mism = lane >= 1 && lane < a.n && s_d[lane] != s_am[lane - 1];
-    const unsigned bal = __ballot_sync(0xffffffffu, mism);
-    const int j = bal ? __ffs(bal) - 1 : a.n;
-    const int t_star = s_am[j - 1];
-    if (lane < a.n) {
-      const int e = lane;
-      a.out_tokens[(size_t)b * a.n + e] = e < j - 1 ? s_d[e + 1] : (e == j - 1 ? t_star : -1);
-    }
-    if (a.next_drafts && a.k > 0 && lane < a.k) {
-      const int e = lane;
-      a.next_drafts[(size_t)b * a.k + e] = e == 0 ? t_star : (want_g ? s_g[(j - 1) * a.k + e] : -1);
-    }
-    if (lane == 0) {
-      a.accept_count[b] = j;
-      if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
-    }
-  }
-  VERIFY_TRACE(rank, 4);
+  VERIFY_TRACE(tr, 10);
 }
 
 // Row normaliser from chunk stats: M = max of chunk maxima, Z = sum_c
@@ -750,11 +626,13 @@ __global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyAr
 
 template <typename T>
 cudaError_t launch_greedy(const VerifyArgs& a, cudaStream_t s) {
-  static int limit_cache[64];
-  const int C = cluster_limit(greedy_cluster_kernel<T>, kGThreads, limit_cache);
-  const int S = a.n <= C ? C / a.n : 1;
-  const int vec_ok = ((size_t)a.V * sizeof(T)) % 16 == 0;
-  return launch_cluster(greedy_cluster_kernel<T>, C, a.B, kGThreads, 0, s, a, S, vec_ok);
+  const int nchunk = (a.V + kChunk - 1) / kChunk;
+  const bool vec_ok = ((size_t)a.V * sizeof(T)) % 16 == 0;
+  ChunkStat* stats = static_cast<ChunkStat*>(a.workspace);
+  cudaError_t e = launch_pdl(stats_kernel<T>, dim3(nchunk, a.B * a.n), kThreads, 0, s, a, stats, nchunk, vec_ok);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(greedy_accept_kernel, dim3((a.B + kAccWarps - 1) / kAccWarps), kAccWarps * 32, 0, s, a,
+                    (const ChunkStat*)stats, nchunk);
 }
 
 template <typename T>
@@ -791,9 +669,10 @@ extern "C" int tidar_verify_trace_read(void* dst, size_t bytes) {
 #endif
 
 size_t verify_workspace_bytes(int B, int k, int V, int mode) {
-  if (mode != TIDAR_REJECTION) return 0;   // greedy: the cluster kernel keeps everything on chip
   const size_t nchunk = (V + kChunk - 1) / kChunk;
   const int n = k > 0 ? k : 1;
+  if (mode != TIDAR_REJECTION)                      // greedy: the chunk statistics of the B n rows
+    return (((size_t)B * n * nchunk * sizeof(ChunkStat) + 255) & ~(size_t)255);
   const size_t rows = (size_t)B * n + (size_t)B * (k > 1 ? k - 1 : 0);
   size_t bytes = ((rows * nchunk * sizeof(ChunkStat) + 255) & ~(size_t)255);
   bytes += (((size_t)B * nchunk * 2 * sizeof(double) + 255) & ~(size_t)255);
@@ -803,8 +682,8 @@ size_t verify_workspace_bytes(int B, int k, int V, int mode) {
 
 bool verify_grid_ok(int B, int k, int mode) {
   const long long n = k > 0 ? k : 1;
-  // grid.y is one sequence (greedy) or one vocab row (rejection statistics)
-  const long long y = mode == TIDAR_REJECTION ? (long long)B * (2 * n - 1) : B;
+  // grid.y is one vocab row of the chunk statistics (rejection: also the q rows)
+  const long long y = mode == TIDAR_REJECTION ? (long long)B * (2 * n - 1) : (long long)B * n;
   return y <= 65535;
 }
 

@@ -194,12 +194,13 @@ class Step:
         cap = cfg.B * ((cfg.n + cfg.page_size - 1) // cfg.page_size + 1)
         self.rel = torch.empty(cap, dtype=torch.int32, device=dev)
         self.nrel = torch.empty(1, dtype=torch.int32, device=dev)
-        # attention: one launch when the kernel merges its splits on chip (no
-        # workspace) on the tensor-core or decode path, else kernel + finalize;
-        # then greedy verify (one cluster kernel) and commit (one cluster kernel)
+        # attention: one launch when the kernel merges its splits itself on the
+        # tensor-core or decode path, else kernel + finalize; then greedy
+        # verify (chunk statistics, then acceptance) and commit (one cluster
+        # kernel)
         self.merge = tidar.plan_full(self.desc)[2]
         self.attn_launches = 2 if (self.merge == 2 or self.path_id == 1) else 1
-        self.launches_per_step = self.attn_launches + 1 + 1
+        self.launches_per_step = self.attn_launches + 2 + 1
 
     def attn(self, i):
         c = self.copies[i]
@@ -300,14 +301,14 @@ class Loop:
                                dtype=torch.uint8, device=dev)
         self.vout = dict(accept_count=torch.empty(cfg.B, dtype=torch.int32, device=dev),
                          out_tokens=torch.empty((cfg.B, n), dtype=torch.int32, device=dev))
-        # reserve, attention (+ finalize), verify (greedy: one cluster kernel;
-        # rejection: chunk statistics, then residual sums + inverse CDF in one
-        # cluster when the vocabulary's 4096-wide chunks fit a portable cluster
-        # of 8, else two launches), commit
+        # reserve, attention (+ finalize), verify (chunk statistics, then --
+        # greedy -- acceptance, or -- rejection -- residual sums + inverse CDF
+        # in one cluster when the vocabulary's 4096-wide chunks fit a portable
+        # cluster of 8, else two launches), commit
         nchunk = -(-V // 4096)
         merge = tidar.plan_full(self.desc)[2]
         self.launches_per_step = (1 + (2 if (merge == 2 or self.path_id == 1) else 1) +
-                                  (1 if mode == "greedy" else (2 if nchunk <= 8 else 3)) + 1)
+                                  (2 if (mode == "greedy" or nchunk <= 8) else 3) + 1)
 
     def step(self, c, s):
         """Step s of copy c: pages, attention (with the draft-row append),

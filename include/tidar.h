@@ -236,9 +236,9 @@ tidar_status tidar_step_attn_plan(const tidar_step_desc* desc, int32_t* path, in
  *   accept_count  [B] int32      out_tokens [B][n] int32
  *   next_drafts   [B][k] int32 or NULL      selected_block [B] int32 or NULL
  *   workspace: at least tidar_verify_workspace_bytes(...) bytes, 256-aligned
- *     (greedy needs none: 0 bytes, NULL allowed).
+ *     (per-chunk statistics of the logits rows).
  * A draft token outside [0, V) is never accepted.  TIDAR_ERR_UNSUPPORTED when
- * the launch grid does not fit: greedy B > 65535, rejection B*(2n-1) > 65535.
+ * the launch grid does not fit: greedy B*n > 65535, rejection B*(2n-1) > 65535.
  * ------------------------------------------------------------------------- */
 size_t tidar_verify_workspace_bytes(int32_t batch, int32_t k, int32_t vocab,
                                     tidar_accept_mode mode);

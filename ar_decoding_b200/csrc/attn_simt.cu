@@ -123,8 +123,11 @@ __global__ void __launch_bounds__(kWarps * 32) finalize_kernel(AttnArgs a, int m
   constexpr int VPL = D / 32;
   if ((int)blockIdx.x < merge_blocks) {
     // one warp per output row.  The split weights are computed lane-parallel
-    // (lane s holds splits s and s + 32; at most 64 splits), then the partial
-    // rows are read four splits at a time so their loads are in flight together.
+    // (lane s holds splits s and s + 32; at most 64 splits).  The partial rows
+    // of up to kFinChunk splits are loaded in the same round trip as the lse
+    // values -- unconditionally, since an empty split's row may be unwritten,
+    // and then selected away rather than multiplied by its zero weight.
+    constexpr int kFinChunk = 16;
     const int lane = threadIdx.x & 31;
     const size_t rows = (size_t)a.B * a.R * a.Hq;
     const size_t row = (size_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -132,38 +135,35 @@ __global__ void __launch_bounds__(kWarps * 32) finalize_kernel(AttnArgs a, int m
     const int ns = a.nsplit;
     const float la = lane < ns ? a.part_lse[lane * rows + row] : -INFINITY;
     const float lb = lane + 32 < ns ? a.part_lse[(lane + 32) * rows + row] : -INFINITY;
-    float mx = fmaxf(la, lb);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float wa = la == -INFINITY ? 0.f : expf(la - mx);
-    const float wb = lb == -INFINITY ? 0.f : expf(lb - mx);
-    float wsum = wa + wb;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     float acc[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
-    for (int s0 = 0; s0 < ns; s0 += 4) {
-      float w4[4], v[4][VPL];
+    float wa = 0.f, wb = 0.f, mx = -INFINITY, wsum = 0.f;
+    for (int s0 = 0; s0 < ns; s0 += kFinChunk) {
+      float v[kFinChunk][VPL];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int sp = s0 + u;
-        const float wl = __shfl_sync(0xffffffffu, sp < 32 ? wa : wb, sp & 31);
-        w4[u] = sp < ns ? wl : 0.f;
+      for (int u = 0; u < kFinChunk; ++u) {
+        if (s0 + u < ns) load_vec<float, VPL>(a.part_o + ((s0 + u) * rows + row) * D + lane * VPL, v[u]);
+      }
+      if (s0 == 0) {
+        mx = fmaxf(la, lb);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        wa = la == -INFINITY ? 0.f : expf(la - mx);
+        wb = lb == -INFINITY ? 0.f : expf(lb - mx);
+        wsum = wa + wb;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (w4[u] != 0.f) {          // an empty split's partial row may be unwritten
-          load_vec<float, VPL>(a.part_o + ((s0 + u) * rows + row) * D + lane * VPL, v[u]);
-        } else {
+      for (int u = 0; u < kFinChunk; ++u) {
+        const int sp = s0 + u;
+        const float w = __shfl_sync(0xffffffffu, sp < 32 ? wa : wb, sp & 31);
+        if (sp < ns && w > 0.f) {
 #pragma unroll
-          for (int i = 0; i < VPL; ++i) v[u][i] = 0.f;
+          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(w, v[u][i], acc[i]);
         }
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) acc[i] = fmaf(w4[u], v[u][i], acc[i]);
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
 #pragma unroll

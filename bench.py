@@ -503,18 +503,28 @@ def layer_sweep(hbm_peak, tc_peak, world, ks=(0, 4, 8, 16), reps=5):
 
 
 KERNEL_SRC = {2: "attn_tc05.cu", 3: "attn_dec.cu", 4: "attn_pair.cu"}
+KERNEL_HEADERS = ("tc05.cuh", "sm100.cuh", "common.cuh", "kernels.h")
+
+
+def kernel_source_hash(path_id: int) -> str:
+    """sha256 prefix of an attention kernel's source and the headers it
+    includes (the key of profiles/traffic.txt)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in (KERNEL_SRC[path_id],) + KERNEL_HEADERS:
+        with open(os.path.join(ROOT, "ar_decoding_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def measured_traffic(k: int, path_id: int):
     """DRAM bytes of one attention launch from the committed ncu record, if the
     kernel source is unchanged since the capture; else None."""
-    import hashlib
     if path_id not in KERNEL_SRC:
         return None
-    src = os.path.join(ROOT, "ar_decoding_b200", "csrc", KERNEL_SRC[path_id])
     rec = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        sha = kernel_source_hash(path_id)
         for line in open(rec):
             parts = line.split()
             if len(parts) == 3 and not line.startswith("#") and parts[0] == sha and int(parts[1]) == k:

@@ -183,7 +183,7 @@ Plan make_plan(const tidar_step_desc* d, int path) {
   // waves count the clusters that can be resident at once.
   // A launch that already fills the device (units >= one wave) keeps one split:
   // with ragged batches the longest sequence, not the wave count, sets its time.
-  constexpr double kFixedBlocks = 3.0, kFinalizeBlocks = 3.0, kClusterMergeBlocks = 1.0;
+  constexpr double kFixedBlocks = 3.0, kFinalizeBlocks = 2.0, kClusterMergeBlocks = 1.0;
   double best = 1e300;
   int best_n = 1;
   bool best_cluster = false;

@@ -100,6 +100,9 @@ def lib():
         L.tidar_verify_blockq.restype = ctypes.c_int
         L.tidar_commit.argtypes = [P, P, P, P, P, P]
         L.tidar_commit.restype = ctypes.c_int
+        L.tidar_verify_commit.argtypes = [P, P, I, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, P,
+                                          P, S, P]
+        L.tidar_verify_commit.restype = ctypes.c_int
         L.tidar_reserve.argtypes = [P, P, P, P, P, P]
         L.tidar_reserve.restype = ctypes.c_int
         L.tidar_get_device_status.argtypes = [P, P]
@@ -587,6 +590,50 @@ def commit(cache, accept_count, k, *, max_prefix_len, head_dim=None, num_q_heads
                             _ptr(released), _ptr(num_released), _stream_handle(stream))
     _check(st, "tidar_commit")
     return released, num_released
+
+
+def verify_commit(logits, drafts, cache, k, mode="greedy", *, max_prefix_len, draft_logits=None,
+                  uniforms=None, block_guesses=None, outputs=None, released=None, num_released=None,
+                  workspace=None, stream=None):
+    """``verify`` then ``commit`` on its accept counts, as one call (greedy:
+    two launches).  Returns (outputs dict as ``verify``, released, num_released)."""
+    m = mode if isinstance(mode, int) else {"greedy": GREEDY, "rejection": REJECTION}[mode]
+    _dev(logits, "logits")
+    B, n, V = logits.shape
+    dev = logits.device
+    kp = cache["k_pages"]
+    if cache["seq_lens"].shape[0] != B:
+        raise ValueError(f"the cache holds {cache['seq_lens'].shape[0]} sequences, the logits {B}")
+    Hkv, ps, D = kp.shape[1], kp.shape[2], kp.shape[3]
+    desc = StepDesc(batch=B, num_q_heads=Hkv, num_kv_heads=Hkv, head_dim=D, k=k, page_size=ps,
+                    max_prefix_len=int(max_prefix_len), dtype=_dtype_code(kp), softmax_scale=0.0,
+                    path=PATH_AUTO)
+    cdesc = make_cache_desc(cache, dev)
+    if outputs is None:
+        outputs = dict(accept_count=torch.empty(B, dtype=torch.int32, device=dev),
+                       out_tokens=torch.empty((B, n), dtype=torch.int32, device=dev),
+                       next_drafts=torch.empty((B, max(k, 1)), dtype=torch.int32, device=dev),
+                       selected_block=torch.empty(B, dtype=torch.int32, device=dev))
+    cap = B * ((max(k, 1) + ps - 1) // ps + 1)
+    if released is None:
+        released = torch.empty(cap, dtype=torch.int32, device=dev)
+    if num_released is None:
+        num_released = torch.empty(1, dtype=torch.int32, device=dev)
+    _dev(released, "released", torch.int32, dev)
+    _dev(num_released, "num_released", torch.int32, dev)
+    need = verify_workspace_bytes(B, k, V, m)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check_verify_args(logits, drafts, draft_logits, uniforms, block_guesses, outputs, workspace)
+    st = lib().tidar_verify_commit(ctypes.byref(desc), ctypes.byref(cdesc), V, _dtype_code(logits), m,
+                                   _ptr(logits), _ptr(drafts), _ptr(draft_logits), _ptr(uniforms),
+                                   _ptr(block_guesses), _ptr(outputs["accept_count"]),
+                                   _ptr(outputs["out_tokens"]),
+                                   _ptr(outputs["next_drafts"]) if k > 0 else None,
+                                   _ptr(outputs["selected_block"]), _ptr(released), _ptr(num_released),
+                                   _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(st, "tidar_verify_commit")
+    return outputs, released, num_released
 
 
 def reserve(cache, pool, k, *, max_prefix_len, returned=None, num_returned=None, stream=None):

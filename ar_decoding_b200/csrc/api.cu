@@ -375,13 +375,14 @@ namespace {
 // Shared by tidar_verify and tidar_verify_blockq: draft_block null means
 // draft_logits is [B][k-1][V]; else it is the previous step's [B][k][k][V]
 // block logits, read through draft_block.
-tidar_status verify_launch(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
-                           tidar_accept_mode mode, const void* logits, const int32_t* drafts,
-                           const void* draft_logits, const int32_t* draft_block,
-                           const float* uniforms, const int32_t* block_guesses,
-                           int32_t* accept_count, int32_t* out_tokens, int32_t* next_drafts,
-                           int32_t* selected_block, void* workspace, size_t workspace_bytes,
-                           tidar_stream_t stream) {
+// Host checks of a verification and its launch arguments (nothing queued).
+tidar_status verify_prepare(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                            tidar_accept_mode mode, const void* logits, const int32_t* drafts,
+                            const void* draft_logits, const int32_t* draft_block,
+                            const float* uniforms, const int32_t* block_guesses,
+                            int32_t* accept_count, int32_t* out_tokens, int32_t* next_drafts,
+                            int32_t* selected_block, void* workspace, size_t workspace_bytes,
+                            tidar::VerifyArgs& a) {
   if (batch < 0 || k < 0 || vocab <= 0) return TIDAR_ERR_INVALID_ARG;
   if (k > 16) return TIDAR_ERR_UNSUPPORTED;
   if (dtype != TIDAR_F32 && dtype != TIDAR_BF16) return TIDAR_ERR_UNSUPPORTED;
@@ -396,16 +397,49 @@ tidar_status verify_launch(int32_t batch, int32_t k, int32_t vocab, tidar_dtype 
   if (workspace_bytes < need ||
       (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))))
     return TIDAR_ERR_INVALID_ARG;
-  tidar::VerifyArgs a{};
+  a = tidar::VerifyArgs{};
   a.B = batch; a.k = k; a.n = k > 0 ? k : 1; a.V = vocab; a.bf16 = dtype == TIDAR_BF16; a.mode = mode;
   a.logits = logits; a.drafts = drafts; a.draft_logits = draft_logits; a.uniforms = uniforms;
   a.draft_block = k > 1 ? draft_block : nullptr;
   a.block_guesses = block_guesses; a.accept_count = accept_count; a.out_tokens = out_tokens;
   a.next_drafts = next_drafts; a.selected_block = selected_block; a.workspace = workspace;
-  tidar_status est = error_word(&a.err);
-  if (est != TIDAR_OK) return est;
+  return error_word(&a.err);
+}
+
+tidar_status verify_launch(int32_t batch, int32_t k, int32_t vocab, tidar_dtype dtype,
+                           tidar_accept_mode mode, const void* logits, const int32_t* drafts,
+                           const void* draft_logits, const int32_t* draft_block,
+                           const float* uniforms, const int32_t* block_guesses,
+                           int32_t* accept_count, int32_t* out_tokens, int32_t* next_drafts,
+                           int32_t* selected_block, void* workspace, size_t workspace_bytes,
+                           tidar_stream_t stream) {
+  tidar::VerifyArgs a;
+  tidar_status st = verify_prepare(batch, k, vocab, dtype, mode, logits, drafts, draft_logits, draft_block,
+                                   uniforms, block_guesses, accept_count, out_tokens, next_drafts,
+                                   selected_block, workspace, workspace_bytes, a);
+  if (st != TIDAR_OK || batch == 0) return st;
   cudaError_t e = tidar::launch_verify(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
+// Host checks of a commit and its launch arguments (nothing queued).
+tidar_status commit_prepare(const tidar_step_desc* d, const tidar_kv_cache* c, const int32_t* accept_count,
+                            int32_t* released_pages, int32_t* num_released, tidar::CommitArgs& a) {
+  tidar_status st = check_desc(d);
+  if (st != TIDAR_OK) return st;
+  if (d->batch == 0) return TIDAR_OK;
+  if ((st = check_cache(d, c)) != TIDAR_OK) return st;
+  if (!accept_count || !released_pages || !num_released) return TIDAR_ERR_INVALID_ARG;
+  if (!tidar::commit_batch_ok(d->batch, d->k, d->page_size)) return TIDAR_ERR_UNSUPPORTED;
+  unsigned int* err = nullptr;
+  if ((st = error_word(&err)) != TIDAR_OK) return st;
+  a.B = d->batch; a.Hkv = d->num_kv_heads; a.D = d->head_dim; a.k = d->k; a.n = d->k > 0 ? d->k : 1;
+  a.page_size = d->page_size; a.elem_bytes = d->dtype == TIDAR_BF16 ? 2 : 4;
+  a.max_pages = c->max_pages_per_seq; a.num_pages = c->num_pages;
+  a.k_pages = c->k_pages; a.v_pages = c->v_pages; a.page_table = c->page_table;
+  a.seq_lens = c->seq_lens; a.accept_count = accept_count; a.released = released_pages;
+  a.num_released = num_released; a.err = err;
   return TIDAR_OK;
 }
 
@@ -515,22 +549,45 @@ tidar_status tidar_sample_drafts(int32_t batch, int32_t k, int32_t vocab, tidar_
 tidar_status tidar_commit(const tidar_step_desc* d, const tidar_kv_cache* c,
                           const int32_t* accept_count, int32_t* released_pages,
                           int32_t* num_released, tidar_stream_t stream) {
-  tidar_status st = check_desc(d);
+  tidar::CommitArgs a{};
+  const tidar_status st = commit_prepare(d, c, accept_count, released_pages, num_released, a);
+  if (st != TIDAR_OK || d->batch == 0) return st;
+  cudaError_t e = tidar::launch_commit(a, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TIDAR_OK;
+}
+
+tidar_status tidar_verify_commit(const tidar_step_desc* d, const tidar_kv_cache* c, int32_t vocab,
+                                 tidar_dtype dtype, tidar_accept_mode mode, const void* logits,
+                                 const int32_t* drafts, const void* draft_logits, const float* uniforms,
+                                 const int32_t* block_guesses, int32_t* accept_count, int32_t* out_tokens,
+                                 int32_t* next_drafts, int32_t* selected_block, int32_t* released_pages,
+                                 int32_t* num_released, void* workspace, size_t workspace_bytes,
+                                 tidar_stream_t stream) {
+  // every host check of both halves before anything is queued
+  tidar::CommitArgs ca{};
+  tidar_status st = commit_prepare(d, c, accept_count, released_pages, num_released, ca);
   if (st != TIDAR_OK) return st;
-  if (d->batch == 0) return TIDAR_OK;
-  if ((st = check_cache(d, c)) != TIDAR_OK) return st;
-  if (!accept_count || !released_pages || !num_released) return TIDAR_ERR_INVALID_ARG;
-  if (!tidar::commit_batch_ok(d->batch, d->k, d->page_size)) return TIDAR_ERR_UNSUPPORTED;
-  unsigned int* err = nullptr;
-  if ((st = error_word(&err)) != TIDAR_OK) return st;
-  tidar::CommitArgs a;
-  a.B = d->batch; a.Hkv = d->num_kv_heads; a.D = d->head_dim; a.k = d->k; a.n = d->k > 0 ? d->k : 1;
-  a.page_size = d->page_size; a.elem_bytes = d->dtype == TIDAR_BF16 ? 2 : 4;
-  a.max_pages = c->max_pages_per_seq; a.num_pages = c->num_pages;
-  a.k_pages = c->k_pages; a.v_pages = c->v_pages; a.page_table = c->page_table;
-  a.seq_lens = c->seq_lens; a.accept_count = accept_count; a.released = released_pages;
-  a.num_released = num_released; a.err = err;
-  cudaError_t e = tidar::launch_commit(a, reinterpret_cast<cudaStream_t>(stream));
+  tidar::VerifyArgs va;
+  st = verify_prepare(d->batch, d->k, vocab, dtype, mode, logits, drafts, draft_logits, nullptr, uniforms,
+                      block_guesses, accept_count, out_tokens, next_drafts, selected_block, workspace,
+                      workspace_bytes, va);
+  if (st != TIDAR_OK || d->batch == 0) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (mode == TIDAR_REJECTION) {
+    cudaError_t e = tidar::launch_verify(va, s);
+    if (e == cudaSuccess) e = tidar::launch_commit(ca, nullptr, s);
+    return e == cudaSuccess ? TIDAR_OK : cuda_fail(e);
+  }
+  // greedy: the chunk statistics, then acceptance and commit in one launch
+  cudaError_t e = tidar::launch_greedy_stats(va, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  tidar::GreedyAcceptArgs f{};
+  f.stats = static_cast<const tidar::ChunkStat*>(workspace);
+  f.nchunk = tidar::verify_chunks(vocab);
+  f.drafts = drafts; f.block_guesses = block_guesses; f.accept_count = accept_count;
+  f.out_tokens = out_tokens; f.next_drafts = next_drafts; f.selected_block = selected_block;
+  e = tidar::launch_commit(ca, &f, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return TIDAR_OK;
 }

@@ -426,32 +426,30 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
       if (!full) block_mask(window, kb, vis, a.R, lo_valid, hi_valid, mw);
       const uint32_t scol = col_s(t) + 64 * hf;          // this half's 64 score columns
-      // pass 1: maximum of this half's raw scores (the positive scale commutes)
+      // pass 1: maximum of this half's raw scores (the positive scale commutes);
+      // its 64 columns come in one TMEM round trip
       float mb = -INFINITY;
       if (live && ok) {
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        uint32_t x[64];
+        tmem_ld64(trow + scol, x);
+        tmem_wait_ld();
+        if (!full) {
+          // masked block (rare): invisible keys become -inf in TMEM too, so
+          // the exponential pass needs no mask (2^-inf = 0)
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t x[32];
-          tmem_ld32(trow + scol + 32 * h2, x);
-          tmem_wait_ld();
-          if (!full) {
-            // masked block (rare): invisible keys become -inf in TMEM too, so
-            // the exponential pass needs no mask (2^-inf = 0)
-            const uint32_t mwd = mw[2 * hf + h2];
+          for (int c = 0; c < 64; ++c)
+            if (!(mw[2 * hf + (c >> 5)] & (1u << (c & 31)))) x[c] = 0xff800000u;
+          tmem_st32(trow + scol, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
+          tmem_st32(trow + scol + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
+          tmem_wait_st();
+        }
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (!(mwd & (1u << c))) x[c] = 0xff800000u;
-            tmem_st32(trow + scol + 32 * h2, x);
-            tmem_wait_st();
-          }
-#pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            mx[0] = max3(mx[0], __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
-            mx[1] = max3(mx[1], __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
-            mx[2] = max3(mx[2], __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
-            mx[3] = max3(mx[3], __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
-          }
+        for (int c = 0; c < 64; c += 8) {
+          mx[0] = max3(mx[0], __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+          mx[1] = max3(mx[1], __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+          mx[2] = max3(mx[2], __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
+          mx[3] = max3(mx[3], __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
         }
         mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       }
@@ -473,36 +471,32 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (need) m = m_new;
       const float nbase = m == -INFINITY ? 0.f : -m;
       TIDAR_TRACE_PH(b2, 4);
-      // pass 2: P = 2^(score * scale - m) in bf16 for this half's 64 keys; the P
-      // of each 32 keys goes over 16 columns of this half's S already reloaded
+      // pass 2: P = 2^(score * scale - m) in bf16 for this half's 64 keys, over
+      // the first 32 columns of this half's S (one TMEM load, one store)
       float lblk = 0.f;
       if (live) {
         const uint64_t sl2x2 = f2_make(sl2, sl2), nbx2 = f2_make(nbase, nbase);
         uint64_t ls2[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
+        uint32_t x[64];
+        tmem_ld64(trow + scol, x);
+        tmem_wait_ld();
+        uint32_t pk[32];
+        // The same loop for full and masked blocks (invisible keys hold -inf
+        // in S since pass 1, and 2^-inf = 0).  Compiled as two copies, the
+        // common full-block one is scheduled without register spills.
+        auto exps = [&]() {
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t x[32];
-          tmem_ld32(trow + scol + 32 * h2, x);
-          tmem_wait_ld();
-          uint32_t pk[16];
-          // The same loop for full and masked blocks (invisible keys hold -inf
-          // in S since pass 1, and 2^-inf = 0).  Compiled as two copies, the
-          // common full-block one is scheduled without register spills.
-          auto exps = [&]() {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              float v0, v1;
-              f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0,
-                       v1);
-              const float p0 = ex2(v0), p1 = ex2(v1);
-              ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
-              pk[c] = cvt_bf16x2(p0, p1);
-            }
-          };
-          if (full) exps();
-          else exps();
-          tmem_st16(trow + scol + 16 * h2, pk);
-        }
+          for (int c = 0; c < 32; ++c) {
+            float v0, v1;
+            f2_split(f2_fma(f2_make(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sl2x2, nbx2), v0, v1);
+            const float p0 = ex2(v0), p1 = ex2(v1);
+            ls2[c & 1] = f2_add(ls2[c & 1], f2_make(p0, p1));
+            pk[c] = cvt_bf16x2(p0, p1);
+          }
+        };
+        if (full) exps();
+        else exps();
+        tmem_st32(trow + scol, pk);
         float la, lb, lc, ld;
         f2_split(ls2[0], la, lb);
         f2_split(ls2[1], lc, ld);

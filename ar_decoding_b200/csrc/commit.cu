@@ -23,6 +23,7 @@
 // No device-side waits besides the two hardware cluster barriers.
 #include <cooperative_groups.h>
 
+#include "accept.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -51,8 +52,13 @@ __device__ unsigned long long g_commit_trace[8];
 #define COMMIT_TRACE(slot) do {} while (0)
 #endif
 
-__global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a, int slots, int per,
-                                                                    int npm) {
+// kFused: the accept counts are not read but computed here from the chunk
+// statistics of a greedy verification (`f`), whose outputs the owner of each
+// sequence also writes (tidar_verify_commit).
+template <bool kFused>
+__global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a, int slots, int per, int npm,
+                                                                    GreedyAcceptArgs f) {
+  __shared__ int s_g[kFused ? kCWarps : 1][kFused ? 16 * 16 : 1];   // per-warp block guesses
   COMMIT_TRACE(0);
   pdl_wait();
   pdl_trigger();
@@ -75,10 +81,12 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
   const int nown = max(0, min(a.B, b0 + per) - b0);
   const int ps = a.page_size;
 
-  // 1. validate, count, keep the pages: one warp per sequence
-  for (int i = wid; i < nown; i += kCWarps) {
+  // 1. validate, count, keep the pages: one warp per sequence (its own
+  //    sequences; with `spread`, every sequence -- the loop below)
+  for (int i = wid; i < (spread ? 0 : nown); i += kCWarps) {
     const int b = b0 + i;
-    const int P = a.seq_lens[b], c = a.accept_count[b];
+    const int P = a.seq_lens[b];
+    const int c = kFused ? greedy_accept_warp(f, a.n, a.k, b, s_g[kFused ? wid : 0], true) : a.accept_count[b];
     int ok = 1;
     if (c < 0 || c > a.n) { ok = 0; if (lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_COUNT); }
     if (ok && (P < 0 || (P + a.n + ps - 1) / ps > a.max_pages)) {
@@ -106,10 +114,18 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
     }
   }
   if (spread) {
-    // the same reads as above without the error reports (owners make those)
+    // the same per sequence, in every CTA; the owner (CTA b / per) reports the
+    // errors and, fused, writes the verification outputs
     for (int b = wid; b < a.B; b += kCWarps) {
-      const int P = a.seq_lens[b], c = a.accept_count[b];
-      bool ok = c >= 0 && c <= a.n && P >= 0 && (P + a.n + ps - 1) / ps <= a.max_pages;
+      const bool owner = b / per == rank;
+      const int P = a.seq_lens[b];
+      const int c = kFused ? greedy_accept_warp(f, a.n, a.k, b, s_g[kFused ? wid : 0], owner) : a.accept_count[b];
+      bool ok = true;
+      if (c < 0 || c > a.n) { ok = false; if (owner && lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_COUNT); }
+      if (ok && (P < 0 || (P + a.n + ps - 1) / ps > a.max_pages)) {
+        ok = false;
+        if (owner && lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_LEN);
+      }
       if (ok) {
         const int p0 = P / ps, np = (P + a.n - 1) / ps - p0 + 1;
         bool bad = false;
@@ -119,17 +135,36 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
           s_allpg[b * npm + lane] = page;
         }
         ok = !__any_sync(0xffffffffu, bad);
+        if (!ok && owner && lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
       }
       if (lane == 0) {
         SeqRec r;
-        r.P = P; r.c = c; r.off = 0; r.cnt = ok ? 0 : -1;
+        r.P = P; r.c = c; r.off = 0;
+        r.cnt = ok ? (P + a.n + ps - 1) / ps - (P + c + ps - 1) / ps : -1;
         s_all[b] = r;
       }
     }
   }
   __syncthreads();
   COMMIT_TRACE(2);
-  if (wid == 0) {
+  if (spread) {
+    // Every CTA holds every sequence's record: the release-list offsets and
+    // the total come from a local scan, and one cluster barrier orders every
+    // CTA's reads of the lengths and tables before the owners' writes.
+    if (wid == 0) {
+      const int v = lane < a.B ? max(s_all[lane].cnt, 0) : 0;      // B < C <= 16 <= 32
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane < a.B) s_all[lane].off = x - v;
+      if (lane == 31) s_grand = x;
+      if (lane == 0) s_base = 0;
+    }
+    cl.sync();
+  } else if (wid == 0) {
     int run = 0;
     for (int s0 = 0; s0 < nown; s0 += 32) {
       const int i = s0 + lane;
@@ -147,8 +182,8 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
   }
 
   // 2. bases across the cluster
-  cl.sync();
-  if (wid == 0) {
+  if (!spread) cl.sync();
+  if (!spread && wid == 0) {
     int t = 0;
     if (lane < C) t = *cl.map_shared_rank(&s_total, lane);
     int sb = lane < rank ? t : 0, sg = t;
@@ -159,19 +194,20 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
     }
     if (lane == 0) { s_base = sb; s_grand = sg; }
   }
-  cl.sync();
+  if (!spread) cl.sync();
   COMMIT_TRACE(3);
 
   // 3. release and advance (one warp per sequence), then scrub (whole CTA);
   //    no page-table reads from here on
   const int base = s_base;
   for (int i = wid; i < nown; i += kCWarps) {
-    const SeqRec r = s_rec[i];
-    if (r.cnt < 0) continue;                        // invalid: left untouched
     const int b = b0 + i;
+    const SeqRec r = spread ? s_all[b] : s_rec[i];
+    if (r.cnt < 0) continue;                        // invalid: left untouched
     const int p0 = r.P / ps, first = (r.P + r.c + ps - 1) / ps;
+    const int* pg = spread ? s_allpg + b * npm : s_pg + i * npm;
     if (lane < r.cnt) {
-      a.released[base + r.off + lane] = s_pg[i * npm + first - p0 + lane];
+      a.released[base + r.off + lane] = pg[first - p0 + lane];
       a.page_table[(size_t)b * a.max_pages + first + lane] = -1;
     }
     if (lane == 0) a.seq_lens[b] = r.P + r.c;
@@ -227,13 +263,14 @@ bool commit_batch_ok(int B, int k, int page_size) {
   return commit_smem((B + 7) / 8, commit_npm(n, page_size)) <= kCommitSmemMax;
 }
 
-cudaError_t launch_commit(const CommitArgs& a, cudaStream_t s) {
+template <bool kFused>
+cudaError_t launch_commit_t(const CommitArgs& a, const GreedyAcceptArgs& f, cudaStream_t s) {
   static int limit_cache[64];
   static bool smem_set[64];
   const int slots = (a.n + a.page_size - 1) / a.page_size + 1;
   // at least as many CTAs as the cluster allows: with a small batch the idle
   // ones share the zeroing of the rejected rows
-  const int C = cluster_limit(commit_cluster_kernel, kCThreads, limit_cache);
+  const int C = cluster_limit(commit_cluster_kernel<kFused>, kCThreads, limit_cache);
   const int per = (a.B + C - 1) / C;
   const int npm = commit_npm(a.n, a.page_size);
   const size_t smem = commit_smem(per + (a.B < C ? a.B : 0), npm);
@@ -241,12 +278,17 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (smem > 48 * 1024 && dev >= 0 && dev < 64 && !smem_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(commit_cluster_kernel,
+    cudaError_t e = cudaFuncSetAttribute(commit_cluster_kernel<kFused>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCommitSmemMax);
     if (e != cudaSuccess) return e;
     smem_set[dev] = true;
   }
-  return launch_cluster(commit_cluster_kernel, C, 1, kCThreads, smem, s, a, slots, per, npm);
+  return launch_cluster(commit_cluster_kernel<kFused>, C, 1, kCThreads, smem, s, a, slots, per, npm, f);
+}
+
+cudaError_t launch_commit(const CommitArgs& a, const GreedyAcceptArgs* fused, cudaStream_t s) {
+  if (fused) return launch_commit_t<true>(a, *fused, s);
+  return launch_commit_t<false>(a, GreedyAcceptArgs{}, s);
 }
 
 }  // namespace tidar

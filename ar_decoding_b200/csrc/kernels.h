@@ -106,6 +106,30 @@ cudaError_t launch_sample_drafts(int B, int k, int V, int bf16, int mode, double
                                  const float* uniforms, int32_t* next_drafts, unsigned int* err,
                                  cudaStream_t s);
 
+// Exact (max, argmax) of one 4096-wide chunk of a logits row (lowest index on
+// ties) and, in rejection mode, the fp64 sum of exp(x - max) over it.
+struct ChunkStat {
+  float max;
+  int arg;
+  double sum;
+};
+// Launches the per-chunk statistics of the B n logits rows of a greedy
+// verification into a.workspace ([B n][chunks] ChunkStat).
+cudaError_t launch_greedy_stats(const VerifyArgs& a, cudaStream_t s);
+int verify_chunks(int V);
+// Greedy acceptance from those statistics, for the commit kernel to run it in
+// the same launch (tidar_verify_commit): its outputs as tidar_verify's.
+struct GreedyAcceptArgs {
+  const ChunkStat* stats;
+  int nchunk;
+  const int32_t* drafts;
+  const int32_t* block_guesses;
+  int32_t* accept_count;
+  int32_t* out_tokens;
+  int32_t* next_drafts;
+  int32_t* selected_block;
+};
+
 struct CommitArgs {
   int B, Hkv, D, k, n, page_size, elem_bytes, max_pages, num_pages;
   void* k_pages;
@@ -118,7 +142,10 @@ struct CommitArgs {
   unsigned int* err;
 };
 bool commit_batch_ok(int B, int k, int page_size);   // per-sequence records fit shared memory
-cudaError_t launch_commit(const CommitArgs& a, cudaStream_t s);
+// fused == nullptr: the accept counts come from a.accept_count; else the
+// kernel computes them (greedy) from fused->stats and writes the
+// verification outputs too.
+cudaError_t launch_commit(const CommitArgs& a, const GreedyAcceptArgs* fused, cudaStream_t s);
 
 struct ReserveArgs {
   int B, n, page_size, max_prefix, max_pages, num_pages, capacity;

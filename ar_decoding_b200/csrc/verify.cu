@@ -28,6 +28,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "accept.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -40,12 +41,6 @@ namespace {
 constexpr int kChunk = 4096;
 constexpr int kThreads = 256;
 constexpr int kPer = kChunk / kThreads;   // 16 elements per thread
-
-struct ChunkStat {
-  float max;
-  int arg;
-  double sum;   // sum exp(x - max) over the chunk (rejection only)
-};
 
 template <typename T>
 __device__ __forceinline__ float ld(const T* p, int i) { return to_f32(p[i]); }
@@ -128,7 +123,7 @@ __device__ unsigned long long g_verify_trace[16 * 8];
 template <typename T>
 __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat* stats, int nchunk,
                                                          bool vec_ok) {
-  const bool tr = blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0;
+  [[maybe_unused]] const bool tr = blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0;
   VERIFY_TRACE(tr, 0);
   if ((int)blockIdx.y < a.B * a.n) {
     // this CTA's chunk of its logits row into L2 while the previous kernel ends
@@ -210,53 +205,28 @@ __device__ void write_outputs(const VerifyArgs& a, int b, int j, int t_star) {
   }
 }
 
-// Greedy acceptance from the chunk statistics (one warp per sequence b).  The
-// statistics kernel has left an exact (max, argmax) per 4096-wide chunk of
-// every logits row -- that sweep runs on as many CTAs as there are chunks,
-// since a single SM pulls only some tens of GB/s -- so lane i merges the
-// chunks of row i in chunk order (equal values keep the lower index), and the
-// drafts and block guesses are fetched before the statistics are needed.
-// d_{i+1} is kept while it equals argmax l_i: j = the first mismatching i,
-// else n; t* = argmax l_{j-1}.
+// Greedy acceptance from the chunk statistics (one warp per sequence b,
+// `greedy_accept_warp`).  The statistics kernel has left an exact
+// (max, argmax) per 4096-wide chunk of every logits row -- that sweep runs on
+// as many CTAs as there are chunks, since a single SM pulls only some tens of
+// GB/s.
 constexpr int kAccWarps = 4;
 __global__ void __launch_bounds__(kAccWarps * 32) greedy_accept_kernel(VerifyArgs a, const ChunkStat* stats,
                                                                        int nchunk) {
   __shared__ int s_g[kAccWarps][16 * 16];
-  const bool tr = blockIdx.x == 0 && threadIdx.x == 0;
+  [[maybe_unused]] const bool tr = blockIdx.x == 0 && threadIdx.x == 0;
   VERIFY_TRACE(tr, 8);
   pdl_wait();
   pdl_trigger();
   VERIFY_TRACE(tr, 9);
-  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
   const int b = blockIdx.x * kAccWarps + wid;
   if (b >= a.B) return;                           // warp-uniform; no block-wide barrier below
-  const bool want_g = a.next_drafts && a.block_guesses && a.k > 0;
-  // d_lane (lane >= 1) and every block's guesses: independent of the logits
-  const int d = (lane >= 1 && lane < a.n && a.k > 1) ? a.drafts[(size_t)b * a.k + lane] : -1;
-  if (want_g)
-    for (int t = lane; t < a.k * a.k; t += 32) s_g[wid][t] = a.block_guesses[(size_t)b * a.k * a.k + t];
-  float mv = -INFINITY;
-  int am = INT_MAX;
-  if (lane < a.n) {
-    const ChunkStat* st = stats + ((size_t)b * a.n + lane) * nchunk;
-    for (int c = 0; c < nchunk; ++c) amax_merge(mv, am, st[c].max, st[c].arg);
-  }
-  __syncwarp();
-  constexpr unsigned kAll = 0xffffffffu;
-  const int am_prev = __shfl_up_sync(kAll, am, 1);            // argmax l_{lane-1}
-  const bool mism = lane >= 1 && lane < a.n && d != am_prev;
-  const unsigned bal = __ballot_sync(kAll, mism);
-  const int j = bal ? __ffs(bal) - 1 : a.n;
-  const int t_star = __shfl_sync(kAll, am, j - 1);
-  const int d_next = __shfl_down_sync(kAll, d, 1);            // d_{lane+1}
-  if (lane < a.n)
-    a.out_tokens[(size_t)b * a.n + lane] = lane < j - 1 ? d_next : (lane == j - 1 ? t_star : -1);
-  if (a.next_drafts && a.k > 0 && lane < a.k)
-    a.next_drafts[(size_t)b * a.k + lane] = lane == 0 ? t_star : (want_g ? s_g[wid][(j - 1) * a.k + lane] : -1);
-  if (lane == 0) {
-    a.accept_count[b] = j;
-    if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
-  }
+  GreedyAcceptArgs f;
+  f.stats = stats; f.nchunk = nchunk; f.drafts = a.drafts; f.block_guesses = a.block_guesses;
+  f.accept_count = a.accept_count; f.out_tokens = a.out_tokens; f.next_drafts = a.next_drafts;
+  f.selected_block = a.selected_block;
+  greedy_accept_warp(f, a.n, a.k, b, s_g[wid], true);
   VERIFY_TRACE(tr, 10);
 }
 
@@ -625,14 +595,20 @@ __global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyAr
 }
 
 template <typename T>
-cudaError_t launch_greedy(const VerifyArgs& a, cudaStream_t s) {
+cudaError_t launch_greedy_stats_t(const VerifyArgs& a, cudaStream_t s) {
   const int nchunk = (a.V + kChunk - 1) / kChunk;
   const bool vec_ok = ((size_t)a.V * sizeof(T)) % 16 == 0;
   ChunkStat* stats = static_cast<ChunkStat*>(a.workspace);
-  cudaError_t e = launch_pdl(stats_kernel<T>, dim3(nchunk, a.B * a.n), kThreads, 0, s, a, stats, nchunk, vec_ok);
+  return launch_pdl(stats_kernel<T>, dim3(nchunk, a.B * a.n), kThreads, 0, s, a, stats, nchunk, vec_ok);
+}
+
+template <typename T>
+cudaError_t launch_greedy(const VerifyArgs& a, cudaStream_t s) {
+  cudaError_t e = launch_greedy_stats_t<T>(a, s);
   if (e != cudaSuccess) return e;
+  const int nchunk = (a.V + kChunk - 1) / kChunk;
   return launch_pdl(greedy_accept_kernel, dim3((a.B + kAccWarps - 1) / kAccWarps), kAccWarps * 32, 0, s, a,
-                    (const ChunkStat*)stats, nchunk);
+                    (const ChunkStat*)a.workspace, nchunk);
 }
 
 template <typename T>
@@ -690,6 +666,12 @@ bool verify_grid_ok(int B, int k, int mode) {
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t s) {
   return a.bf16 ? launch_t<__nv_bfloat16>(a, s) : launch_t<float>(a, s);
 }
+
+cudaError_t launch_greedy_stats(const VerifyArgs& a, cudaStream_t s) {
+  return a.bf16 ? launch_greedy_stats_t<__nv_bfloat16>(a, s) : launch_greedy_stats_t<float>(a, s);
+}
+
+int verify_chunks(int V) { return (V + kChunk - 1) / kChunk; }
 
 }  // namespace tidar
 

@@ -196,11 +196,11 @@ class Step:
         self.nrel = torch.empty(1, dtype=torch.int32, device=dev)
         # attention: one launch when the kernel merges its splits itself on the
         # tensor-core or decode path, else kernel + finalize; then greedy
-        # verify (chunk statistics, then acceptance) and commit (one cluster
-        # kernel)
+        # verification and commit (tidar_verify_commit: the chunk statistics,
+        # then acceptance + commit in one cluster kernel)
         self.merge = tidar.plan_full(self.desc)[2]
         self.attn_launches = 2 if (self.merge == 2 or self.path_id == 1) else 1
-        self.launches_per_step = self.attn_launches + 2 + 1
+        self.launches_per_step = self.attn_launches + 2
 
     def attn(self, i):
         c = self.copies[i]
@@ -210,11 +210,10 @@ class Step:
 
     def verify_commit(self, i):
         c = self.copies[i]
-        self.tidar.verify(c["logits"], c["drafts"], self.cfg.k, "greedy",
-                          block_guesses=c["guesses"], outputs=self.vout, workspace=self.vws)
-        self.tidar.commit(c["cache"], self.vout["accept_count"], self.cfg.k,
-                          max_prefix_len=self.max_prefix, released=self.rel,
-                          num_released=self.nrel)
+        self.tidar.verify_commit(c["logits"], c["drafts"], c["cache"], self.cfg.k, "greedy",
+                                 max_prefix_len=self.max_prefix, block_guesses=c["guesses"],
+                                 outputs=self.vout, released=self.rel, num_released=self.nrel,
+                                 workspace=self.vws)
 
     def restore(self, i):
         c = self.copies[i]
@@ -301,14 +300,15 @@ class Loop:
                                dtype=torch.uint8, device=dev)
         self.vout = dict(accept_count=torch.empty(cfg.B, dtype=torch.int32, device=dev),
                          out_tokens=torch.empty((cfg.B, n), dtype=torch.int32, device=dev))
-        # reserve, attention (+ finalize), verify (chunk statistics, then --
-        # greedy -- acceptance, or -- rejection -- residual sums + inverse CDF
-        # in one cluster when the vocabulary's 4096-wide chunks fit a portable
-        # cluster of 8, else two launches), commit
+        # reserve, attention (+ finalize), verify + commit (greedy: chunk
+        # statistics, then acceptance + commit in one launch; rejection: chunk
+        # statistics, residual sums + inverse CDF in one cluster when the
+        # vocabulary's 4096-wide chunks fit a portable cluster of 8, else two
+        # launches, then the commit)
         nchunk = -(-V // 4096)
         merge = tidar.plan_full(self.desc)[2]
         self.launches_per_step = (1 + (2 if (merge == 2 or self.path_id == 1) else 1) +
-                                  (2 if (mode == "greedy" or nchunk <= 8) else 3) + 1)
+                                  (1 if mode == "greedy" else (2 if nchunk <= 8 else 3)) + 1)
 
     def step(self, c, s):
         """Step s of copy c: pages, attention (with the draft-row append),
@@ -325,8 +325,12 @@ class Loop:
         vout = dict(self.vout, next_drafts=cp["drafts"][s % 2], selected_block=cp["sel"][s % 2])
         g = cp["guesses"][s] if k else None
         if self.mode == "greedy":
-            t.verify(cp["logits"][s], drafts if k else None, k, "greedy", block_guesses=g,
-                     outputs=vout, workspace=self.vws)
+            # verification and commit as one call (acceptance inside the commit's launch)
+            t.verify_commit(cp["logits"][s], drafts if k else None, cp["cache"], k, "greedy",
+                            max_prefix_len=self.max_prefix, block_guesses=g, outputs=vout,
+                            released=cp["rel"][s % 2], num_released=cp["nrel"][s % 2],
+                            workspace=self.vws)
+            return
         elif self.mode == "blockq" and s > 0:
             # q from the previous step's mask blocks, through its selected block
             t.verify_blockq(cp["logits"][s], drafts, k, cp["blocks"][s - 1], cp["sel"][prev],

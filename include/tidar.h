@@ -395,6 +395,29 @@ tidar_status tidar_commit(const tidar_step_desc* desc, const tidar_kv_cache* cac
                           int32_t* num_released, tidar_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * tidar_verify followed by tidar_commit on the accept counts it produces, as
+ * one call: the verification after a step's forward pass and the eviction it
+ * implies ([NDfr] paragraphs on betting on every outcome and on the three
+ * zones).  Arguments as the two calls (batch and k from desc; dtype is the
+ * logits' type), accept_count both the verification's output and the
+ * commit's input; workspace as tidar_verify's
+ * (tidar_verify_workspace_bytes(batch, k, vocab, mode)).  Every host check of
+ * both runs before anything is queued.  Greedy mode computes the acceptance
+ * inside the commit's launch (two launches: the chunk statistics, then
+ * acceptance + commit); rejection mode queues tidar_verify's launches and
+ * then the commit's.  Results and device errors are those of the two calls.
+ * ------------------------------------------------------------------------- */
+tidar_status tidar_verify_commit(const tidar_step_desc* desc, const tidar_kv_cache* cache,
+                                 int32_t vocab, tidar_dtype dtype, tidar_accept_mode mode,
+                                 const void* logits, const int32_t* drafts,
+                                 const void* draft_logits, const float* uniforms,
+                                 const int32_t* block_guesses, int32_t* accept_count,
+                                 int32_t* out_tokens, int32_t* next_drafts,
+                                 int32_t* selected_block, int32_t* released_pages,
+                                 int32_t* num_released, void* workspace, size_t workspace_bytes,
+                                 tidar_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Page reservation for the next step's draft rows, from a device stack of
  * free pages (the step the commit's release implies; the pages do not
  * describe a page pool).  [NDfr] paragraph on the three zones: the candidates

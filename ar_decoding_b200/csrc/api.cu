@@ -116,6 +116,30 @@ struct Plan {
   bool cluster_merge;   // splits of a tile form one cluster and merge in the attention kernel
 };
 
+// Step-key windows (128 step keys each) the last split of the busiest query
+// tile runs on the tensor-core paths (PAIR: a pair of tiles): window 0 (the
+// drafts) plus those holding the tile's own mask blocks -- the windows the
+// kernels' block plans add, at most 4.
+int max_step_windows(const tidar_step_desc* d, int path) {
+  const int k = d->k, R = tidar::rows_per_seq(k);
+  const int G = d->num_q_heads / d->num_kv_heads;
+  const int rows = (path == 4 ? 2 : 1) * (128 / G);
+  int most = 1;
+  for (int rho0 = 0; rho0 < R; rho0 += rows) {
+    const int rho1 = rho0 + rows < R ? rho0 + rows : R;
+    int nw = 1;
+    if (k > 0 && rho1 - 1 >= k) {
+      const int jlo = ((rho0 > k ? rho0 : k) - k) / k + 1;
+      const int jhi = (rho1 - 1 - k) / k + 1;
+      const int lo = k + (jlo - 1) * k, hi = k + jhi * k;
+      for (int w = lo / 128; w <= (hi - 1) / 128 && nw < 4; ++w)
+        if (w != 0) ++nw;
+    }
+    if (nw > most) most = nw;
+  }
+  return most;
+}
+
 // Key ranges are multiples of 128 keys (64 on the decode path).  SIMT: aim for
 // ~2 waves of 4-warp CTAs.  TC05 / PAIR / DEC: one CTA per SM and per (b, kv
 // head, query tile or pair of tiles, split), split count from a cost model.
@@ -156,13 +180,14 @@ Plan make_plan(const tidar_step_desc* d, int path) {
       return;
     }
     // tensor-core paths: the last split also runs the tile's step-key windows
-    // (up to ceil(R / 128) blocks of 128; a masked block costs about what a
-    // prefix block does), so the split size counts them and the last split
-    // gets correspondingly fewer prefix blocks
-    const int wins = ((path == 2 || path == 4) && n > 1) ? (R + 127) / 128 : 0;
+    // (blocks of 128 step keys; a masked block costs about what a prefix block
+    // does), so the blocks are dealt out with the busiest tile's windows counted
+    // as the last ones: every split holds at most bps blocks, and the last
+    // split holds what remains of the prefix (possibly nothing) and the windows
+    const int wins = ((path == 2 || path == 4) && n > 1) ? max_step_windows(d, path) : 0;
     const int bps = (blocks128 + wins + n - 1) / n;
     p.keys_per_split = (bps > 0 ? bps : 1) * 128;
-    p.nsplit = maxP > 0 ? (maxP + p.keys_per_split - 1) / p.keys_per_split : 1;
+    p.nsplit = maxP > 0 ? (blocks128 + wins + bps - 1) / (bps > 0 ? bps : 1) : 1;
     if (p.nsplit < 1) p.nsplit = 1;
   };
   p.cluster_merge = false;
@@ -179,7 +204,7 @@ Plan make_plan(const tidar_step_desc* d, int path) {
   // cost model in units of 128-key blocks per CTA -- the waves of CTAs the
   // launch needs times (the keys of one split + a fixed per-CTA cost), plus
   // the merge: a second launch, or (the splits of a tile forming a cluster of
-  // nsplit CTAs) a merge from L2 at the end of the attention kernel, whose
+  // nsplit CTAs) an on-chip merge at the end of the attention kernel, whose
   // waves count the clusters that can be resident at once.
   // A launch that already fills the device (units >= one wave) keeps one split:
   // with ragged batches the longest sequence, not the wave count, sets its time.
@@ -203,7 +228,7 @@ Plan make_plan(const tidar_step_desc* d, int path) {
                                                   : tidar::dec_resident_clusters(p.nsplit, M));
       if (resident > 0) {
         const double cost_c = (double)((units + resident - 1) / resident) * per + kClusterMergeBlocks;
-        if (cost_c < best) { best = cost_c; best_n = n; best_cluster = true; }
+        if (cost_c <= best) { best = cost_c; best_n = n; best_cluster = true; }   // ties: on chip
       }
     }
   }

@@ -158,7 +158,9 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     prefetch_tmap(&tm_vs);
     const int bq = blockIdx.y / a.Hkv;
     prefetch_l2(a.seq_lens + bq, 4, 0, 1);
-    prefetch_l2(a.page_table + (size_t)bq * a.max_pages + blockIdx.x * a.keys_per_split / 64, 256, 0, 1);
+    const int pgq = blockIdx.x * a.keys_per_split / 64;
+    if (pgq < a.max_pages)
+      prefetch_l2(a.page_table + (size_t)bq * a.max_pages + pgq, min(256, 4 * (a.max_pages - pgq)), 0, 1);
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();

@@ -156,7 +156,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       prefetch_tmap(&tm_ks);
       prefetch_tmap(&tm_vs);
       prefetch_l2(a.seq_lens + b, 4, 0, 1);
-      prefetch_l2(a.page_table + (size_t)b * a.max_pages + split * a.keys_per_split / 64, 256, 0, 1);
+      const int pgq = split * a.keys_per_split / 64;     // the last split may start past the table
+      if (pgq < a.max_pages)
+        prefetch_l2(a.page_table + (size_t)b * a.max_pages + pgq, min(256, 4 * (a.max_pages - pgq)), 0, 1);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     } else {
       raise_error(a.err, TIDAR_DEVERR_LAYOUT);

@@ -163,7 +163,9 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     prefetch_tmap(&tm_vs);
     const int bq = blockIdx.z / prm.a.Hkv;
     prefetch_l2(prm.a.seq_lens + bq, 4, 0, 1);
-    prefetch_l2(prm.a.page_table + (size_t)bq * prm.a.max_pages + blockIdx.y * prm.a.keys_per_split / 64, 256, 0, 1);
+    const int pgq = blockIdx.y * prm.a.keys_per_split / 64;   // the last split may start past the table
+    if (pgq < prm.a.max_pages)
+      prefetch_l2(prm.a.page_table + (size_t)bq * prm.a.max_pages + pgq, min(256, 4 * (prm.a.max_pages - pgq)), 0, 1);
   }
   pdl_wait();       // the previous kernel on the stream is complete from here on
   pdl_trigger();

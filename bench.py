@@ -376,6 +376,7 @@ class Loop:
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(reps)]
         tokens = None
+        hold_stream(reps)
         for i in range(reps):
             ev[i][0].record(stream)
             gl.replay()
@@ -453,6 +454,7 @@ class LayerStep:
         g.replay(); g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        hold_stream(reps)
         e0.record(stream)
         for _ in range(reps):
             g.replay()
@@ -572,6 +574,15 @@ def flush_l2():
     buf.zero_()
 
 
+def hold_stream(items: int, us_per_item: float = 40.0) -> None:
+    """Queue a GPU-side wait (a spin of about 0.2 ms + `us_per_item` per timed
+    item) ahead of the timed launches, so that the host has enqueued all of
+    them before the first one runs: the events then bracket device work only,
+    never a gap in which the device waits for the host to submit the next
+    graph.  The work between the events is unchanged."""
+    torch.cuda._sleep(int((200.0 + items * us_per_item) * 2000))   # clock cycles, ~2 GHz
+
+
 def bench_config(cfg, prefix: int, k: int) -> dict:
     """The `config` object of the JSON line: the workload, identical for the GPU
     arm and the oracle (reference) arm."""
@@ -649,6 +660,7 @@ def time_steps(st: Step, K: int, W: int, world: int):
               for _ in range(count)]
         barrier(world)
         torch.cuda.synchronize()
+        hold_stream(count, 60.0 if flush else 40.0)
         for i in range(count):
             g = st.graphs[(warm + i) % n]
             ev[i][0].record(stream)
@@ -684,6 +696,7 @@ def time_attention_launches(st: Step, reps: int, attn_call_us=None):
         g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hold_stream(reps)
     e0.record(stream)
     for _ in range(reps):
         g.replay()

@@ -82,6 +82,15 @@ def test_step_attn_rejects_small_workspace(L):
     assert _attn(L, d, c, ws=FAKE + 16, wsb=need) == tidar.ERR_INVALID_ARG   # not 256-aligned
 
 
+def test_last_split_may_hold_only_the_step_windows(L):
+    # 8B-class k = 4 (one query tile of 20 rows x 4 heads): 64 prefix blocks of
+    # 128 keys plus the tile's one step-key window are dealt out 4 per split,
+    # so 16 splits take the prefix and a 17th only the window
+    d = _desc(max_prefix_len=8192, batch=1, num_q_heads=32, num_kv_heads=8, k=4,
+              path=tidar.PATH_TC05)
+    assert tidar.plan_full(d)[:2] == (tidar.PATH_TC05, 17)
+
+
 def test_tensor_core_plan_splits_long_prefixes(L):
     # one query row per head: the 8192-key prefix is split to fill the SMs; the
     # workspace holds split partials unless the kernel merges them itself

@@ -71,4 +71,27 @@ __device__ __forceinline__ int greedy_accept_warp(const GreedyAcceptArgs& f, int
   return j;
 }
 
+// Writes accept_count, out_tokens, selected_block, next_drafts for sequence b.
+// Called by a whole warp (n, k <= 16): every lane loads its draft and its
+// block guess first, all in flight at once, then the lanes store (one thread
+// storing as it loads would wait a memory round trip per element, the loads
+// not being movable past stores that might alias).
+__device__ __forceinline__ void write_outputs_warp(const VerifyArgs& a, int b, int j, int t_star) {
+  const int e = (int)threadIdx.x & 31;
+  int v = -1, gv = -1;
+  if (e < a.n) {
+    if (e < j - 1) v = a.drafts[(size_t)b * a.k + e + 1];
+    else if (e == j - 1) v = t_star;
+  }
+  const bool nd = a.next_drafts && a.k > 0;
+  if (nd && e >= 1 && e < a.k && a.block_guesses) gv = a.block_guesses[((size_t)b * a.k + (j - 1)) * a.k + e];
+  __syncwarp();
+  if (e < a.n) a.out_tokens[(size_t)b * a.n + e] = v;
+  if (nd && e < a.k) a.next_drafts[(size_t)b * a.k + e] = e == 0 ? t_star : gv;
+  if (e == 0) {
+    a.accept_count[b] = j;
+    if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
+  }
+}
+
 }  // namespace tidar

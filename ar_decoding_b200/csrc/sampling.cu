@@ -36,6 +36,7 @@
 #include <climits>
 #include <math.h>
 
+#include "accept.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -341,23 +342,25 @@ __global__ void __launch_bounds__(kSThreads) accept_kernel(SampledArgs sa) {
   const int b = blockIdx.x;
   const int rows = a.n + a.k - 1 > a.n ? a.n + a.k - 1 : a.n;
   const RowDist* dd = sa.dist + (size_t)b * rows;
-  if (threadIdx.x == 0) {
-    // accept scan, left to right, fp64
-    int j = 1;
-    for (int i = 1; i <= a.n - 1; ++i) {
+  if (threadIdx.x < 32) {
+    // accept scan: the n-1 tests are independent (only "stop at the first
+    // rejection" orders them), so lane i-1 evaluates test i in fp64 and a
+    // ballot finds the first failure: j = that i, else n
+    const int i = (int)threadIdx.x + 1;
+    bool fail = false;
+    if (i <= a.n - 1) {
       const int d = a.drafts[(size_t)b * a.k + i];
-      bool acc = false;
+      fail = true;
       if (d >= 0 && d < a.V) {
         const double u = (double)a.uniforms[(size_t)b * a.n + (i - 1)];
         const float lp = ld_logit(dist_row_ptr<T>(a, b, i - 1), d);
         const float lq = ld_logit(dist_row_ptr<T>(a, b, a.n + i - 1), d);
         const double p = prob(dd[i - 1], lp, d, sa.temp), q = prob(dd[a.n + i - 1], lq, d, sa.temp);
-        acc = u * q < p;
+        fail = !(u * q < p);
       }
-      if (!acc) break;
-      j = i + 1;
     }
-    s_j = j;
+    const unsigned bal = __ballot_sync(0xffffffffu, fail);
+    if (threadIdx.x == 0) s_j = bal ? __ffs(bal) : a.n;
   }
   __syncthreads();
   const int j = s_j;
@@ -379,22 +382,7 @@ __global__ void __launch_bounds__(kSThreads) accept_kernel(SampledArgs sa) {
   } else {
     t_star = inverse_cdf(a.V, u, [&](int x) { return prob(dp, ld_logit(prow, x), x, sa.temp); }, s, nullptr);
   }
-  if (threadIdx.x == 0) {
-    a.accept_count[b] = j;
-    for (int e = 0; e < a.n; ++e) {
-      int v = -1;
-      if (e < j - 1) v = a.drafts[(size_t)b * a.k + e + 1];
-      else if (e == j - 1) v = t_star;
-      a.out_tokens[(size_t)b * a.n + e] = v;
-    }
-    if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
-    if (a.next_drafts && a.k > 0) {
-      a.next_drafts[(size_t)b * a.k] = t_star;
-      for (int e = 1; e < a.k; ++e)
-        a.next_drafts[(size_t)b * a.k + e] =
-            a.block_guesses ? a.block_guesses[((size_t)b * a.k + (j - 1)) * a.k + e] : -1;
-    }
-  }
+  if (threadIdx.x < 32) write_outputs_warp(a, b, j, t_star);
 }
 
 struct DraftArgs {

@@ -187,24 +187,6 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat
   VERIFY_TRACE(tr, 2);
 }
 
-// Writes accept_count, out_tokens, selected_block, next_drafts for sequence b.
-__device__ void write_outputs(const VerifyArgs& a, int b, int j, int t_star) {
-  a.accept_count[b] = j;
-  for (int e = 0; e < a.n; ++e) {
-    int v = -1;
-    if (e < j - 1) v = a.drafts[(size_t)b * a.k + e + 1];
-    else if (e == j - 1) v = t_star;
-    a.out_tokens[(size_t)b * a.n + e] = v;
-  }
-  if (a.selected_block) a.selected_block[b] = a.k > 0 ? j : 0;
-  if (a.next_drafts && a.k > 0) {
-    a.next_drafts[(size_t)b * a.k] = t_star;
-    for (int e = 1; e < a.k; ++e)
-      a.next_drafts[(size_t)b * a.k + e] =
-          a.block_guesses ? a.block_guesses[((size_t)b * a.k + (j - 1)) * a.k + e] : -1;
-  }
-}
-
 // Greedy acceptance from the chunk statistics (one warp per sequence b,
 // `greedy_accept_warp`).  The statistics kernel has left an exact
 // (max, argmax) per 4096-wide chunk of every logits row -- that sweep runs on
@@ -232,11 +214,15 @@ __global__ void __launch_bounds__(kAccWarps * 32) greedy_accept_kernel(VerifyArg
 
 // Row normaliser from chunk stats: M = max of chunk maxima, Z = sum_c
 // exp(max_c - M) * sum_c (fp64).
+// The loops are unrolled by 8 so that the loads of 8 chunks' statistics go
+// out together (one memory round trip per 8 chunks, not one per chunk).
 __device__ void row_norm(const ChunkStat* st, int nchunk, double& M, double& Z) {
   float mf = -INFINITY;
+#pragma unroll 8
   for (int c = 0; c < nchunk; ++c) mf = fmaxf(mf, st[c].max);
   M = (double)mf;
   Z = 0.0;
+#pragma unroll 8
   for (int c = 0; c < nchunk; ++c) Z += exp((double)st[c].max - M) * st[c].sum;
 }
 
@@ -252,14 +238,15 @@ __device__ int rejection_scan_warp(const VerifyArgs& a, int b, const ChunkStat* 
   bool fail = false;
   if (i <= a.n - 1) {
     const int d = a.drafts[(size_t)b * a.k + i];
+    // the normalisers do not depend on the draft: their loads go out with its
+    const size_t lrow = (size_t)b * a.n + (i - 1);
+    const size_t qrow = (size_t)b * (a.k - 1) + (i - 1);
+    double Mp, Zp, Mq, Zq;
+    row_norm(stats + lrow * nchunk, nchunk, Mp, Zp);
+    row_norm(stats + (prow + qrow) * nchunk, nchunk, Mq, Zq);
     if (d < 0 || d >= a.V) {
       fail = true;
     } else {
-      double Mp, Zp, Mq, Zq;
-      const size_t lrow = (size_t)b * a.n + (i - 1);
-      const size_t qrow = (size_t)b * (a.k - 1) + (i - 1);
-      row_norm(stats + lrow * nchunk, nchunk, Mp, Zp);
-      row_norm(stats + (prow + qrow) * nchunk, nchunk, Mq, Zq);
       const double p = exp((double)ld(static_cast<const T*>(a.logits) + lrow * a.V, d) - Mp) / Zp;
       const double q = exp((double)ld(q_row<T>(a, b, i), d) - Mq) / Zq;
       const double u = (double)a.uniforms[(size_t)b * a.n + (i - 1)];
@@ -290,6 +277,83 @@ __device__ void scan_and_norms(const VerifyArgs& a, int b, bool first, const Chu
     } else if (threadIdx.x == 1 && j < a.n) {      // the q_j normaliser on a second lane
       const size_t qrow = (size_t)a.B * a.n + (size_t)b * (a.k - 1) + (j - 1);
       row_norm(stats + qrow * nchunk, nchunk, sMq, sZq);
+    }
+  }
+  __syncthreads();
+}
+
+// The same scan and normalisers with the whole CTA (nchunk <= kNormChunks):
+// the chunk statistics of every row the scan can touch -- the n p rows and the
+// n-1 q rows of sequence b -- are loaded by all threads at once into shared
+// memory, one thread per row then forms (M, Z) with row_norm's arithmetic and
+// order, and warp 0 runs the tests from that table.  The lanes' drafts and
+// logits at the drafts are loaded before, alongside the statistics.  Ends with
+// __syncthreads.
+constexpr int kNormChunks = 16, kNormRows = 31;   // n <= 16: 2n - 1 rows
+static_assert(kMaxCluster <= kNormChunks, "a cluster's chunks fit the table");
+template <typename T>
+__device__ void scan_and_norms_block(const VerifyArgs& a, int b, bool first, const ChunkStat* stats,
+                                     int nchunk, int& sj, double& sMp, double& sZp, double& sMq,
+                                     double& sZq) {
+  __shared__ float s_cm[kNormRows * kNormChunks];
+  __shared__ double s_cs[kNormRows * kNormChunks];
+  __shared__ double s_M[kNormRows], s_Z[kNormRows];
+  const int R = 2 * a.n - 1;                          // p rows 0..n-1, then q rows 0..n-2
+  // the lanes' test operands: lane i-1 decides d_{i+1}
+  const int i = (int)(threadIdx.x & 31) + 1;
+  int d = -1;
+  float lp = 0.f, lq = 0.f;
+  if (threadIdx.x < 32 && i <= a.n - 1) {
+    d = a.drafts[(size_t)b * a.k + i];
+    if (d >= 0 && d < a.V) {
+      lp = ld(static_cast<const T*>(a.logits) + ((size_t)b * a.n + (i - 1)) * a.V, d);
+      lq = ld(q_row<T>(a, b, i), d);
+    }
+  }
+  for (int idx = threadIdx.x; idx < R * nchunk; idx += blockDim.x) {
+    const int r = idx / nchunk, c = idx - r * nchunk;
+    const size_t srow = r < a.n ? (size_t)b * a.n + r : (size_t)a.B * a.n + (size_t)b * (a.k - 1) + (r - a.n);
+    const ChunkStat st = stats[srow * nchunk + c];
+    s_cm[idx] = st.max;
+    s_cs[idx] = st.sum;
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < R) {
+    const float* cm = s_cm + threadIdx.x * nchunk;
+    const double* cs = s_cs + threadIdx.x * nchunk;
+    float mf = -INFINITY;
+    for (int c = 0; c < nchunk; ++c) mf = fmaxf(mf, cm[c]);
+    const double M = (double)mf;
+    double Z = 0.0;
+    for (int c = 0; c < nchunk; ++c) Z += exp((double)cm[c] - M) * cs[c];
+    s_M[threadIdx.x] = M;
+    s_Z[threadIdx.x] = Z;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    bool fail = false;
+    if (i <= a.n - 1) {
+      if (d < 0 || d >= a.V) {
+        fail = true;
+      } else {
+        const double p = exp((double)lp - s_M[i - 1]) / s_Z[i - 1];
+        const double q = exp((double)lq - s_M[a.n + i - 1]) / s_Z[a.n + i - 1];
+        const double u = (double)a.uniforms[(size_t)b * a.n + (i - 1)];
+        fail = !(u * q < p);
+      }
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, fail);
+    const int j = bal ? __ffs(bal) : a.n;             // lowest failing lane L is test L+1
+    if (threadIdx.x == 0) {
+      sj = j;
+      if (first && a.draft_block && a.k > 1 && (a.draft_block[b] < 1 || a.draft_block[b] > a.k))
+        raise_error(a.err, TIDAR_DEVERR_BAD_COUNT);
+      sMp = s_M[j - 1];
+      sZp = s_Z[j - 1];
+      if (j < a.n) {
+        sMq = s_M[a.n + j - 1];
+        sZq = s_Z[a.n + j - 1];
+      }
     }
   }
   __syncthreads();
@@ -404,10 +468,10 @@ __device__ void select_from_regs(const VerifyArgs& a, int b, int j, int chunk, d
   if (hit != INT_MAX) atomicMin(&s_found, hit);
   if (last_nz >= 0) atomicMax(&s_last, last_nz);
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
     int t = s_found;
     if (t == INT_MAX) t = s_last >= 0 ? s_last : min(c0 + kChunk, a.V) - 1;
-    write_outputs(a, b, j, t);
+    write_outputs_warp(a, b, j, t);
   }
 }
 
@@ -463,10 +527,10 @@ __device__ void select_in_chunk(const VerifyArgs& a, int b, int j, int chunk, bo
   if (hit != INT_MAX) atomicMin(&s_found, hit);
   if (last_nz >= 0) atomicMax(&s_last, last_nz);
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
     int t = s_found;
     if (t == INT_MAX) t = s_last >= 0 ? s_last : min(c0 + kChunk, a.V) - 1;
-    write_outputs(a, b, j, t);
+    write_outputs_warp(a, b, j, t);
   }
 }
 
@@ -541,46 +605,64 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyArgs a,
                                                                         const ChunkStat* stats,
                                                                         int nchunk, bool vec_ok) {
+  [[maybe_unused]] const bool tr = blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0;
+  VERIFY_TRACE(tr, 16);
   pdl_wait();
   pdl_trigger();
+  VERIFY_TRACE(tr, 17);
   cg::cluster_group cl = cg::this_cluster();
   const int c = (int)cl.block_rank(), b = blockIdx.y;
   __shared__ int sj, s_chunk, s_resid;
   __shared__ double sMp, sZp, sMq, sZq, s_target;
   __shared__ double s_sum[2];                         // this chunk's (residual, p) sums
-  scan_and_norms<T>(a, b, c == 0, stats, nchunk, nullptr, sj, sMp, sZp, sMq, sZq);
+  scan_and_norms_block<T>(a, b, c == 0, stats, nchunk, sj, sMp, sZp, sMq, sZq);
+  VERIFY_TRACE(tr, 18);
   const int j = sj;
   double wr[kPer], wp[kPer];
   chunk_weights<T>(a, b, c, j, sMp, 1.0 / sZp, sMq, j < a.n ? 1.0 / sZq : 0.0, vec_ok, wr, wp);
+  VERIFY_TRACE(tr, 19);
   double sr = 0.0, sp = 0.0;
   block_sums(wr, wp, sr, sp);
   if (threadIdx.x == 0) { s_sum[0] = sr; s_sum[1] = sp; }
+  VERIFY_TRACE(tr, 20);
   cl.sync();
-  if (threadIdx.x == 0) {
-    // the chunk sums in chunk order, read from each CTA's shared memory (the
-    // arithmetic of select_kernel)
-    double tr = 0.0, tp = 0.0;
-    for (int r = 0; r < nchunk; ++r) {
-      const double* peer = cl.map_shared_rank(s_sum, r);
-      tr += peer[0];
-      tp += peer[1];
+  VERIFY_TRACE(tr, 21);
+  if (threadIdx.x < 32) {
+    // every CTA's chunk sums, one peer per lane (all distributed shared memory
+    // reads in flight at once), into local shared memory; then thread 0 adds
+    // them in chunk order (the arithmetic of select_kernel)
+    __shared__ double s_all[kMaxCluster][2];
+    if ((int)threadIdx.x < nchunk) {
+      const double* peer = cl.map_shared_rank(s_sum, (int)threadIdx.x);
+      s_all[threadIdx.x][0] = peer[0];
+      s_all[threadIdx.x][1] = peer[1];
     }
-    const int resid = (j < a.n) && (tr > 0.0);
-    const double total = resid ? tr : tp;
-    const double target = (double)a.uniforms[(size_t)b * a.n + (a.n - 1)] * total;
-    double cum = 0.0;
-    int ch = nchunk - 1;
-    for (int r = 0; r < nchunk; ++r) {
-      const double wc = cl.map_shared_rank(s_sum, r)[resid ? 0 : 1];
-      if (target < cum + wc) { ch = r; break; }
-      cum += wc;
-      if (r == nchunk - 1) cum -= wc;   // not found: scan the last chunk
+    __syncwarp();
+    if (threadIdx.x == 0) {
+      double tr = 0.0, tp = 0.0;
+      for (int r = 0; r < nchunk; ++r) {
+        tr += s_all[r][0];
+        tp += s_all[r][1];
+      }
+      const int resid = (j < a.n) && (tr > 0.0);
+      const double total = resid ? tr : tp;
+      const double target = (double)a.uniforms[(size_t)b * a.n + (a.n - 1)] * total;
+      double cum = 0.0;
+      int ch = nchunk - 1;
+      for (int r = 0; r < nchunk; ++r) {
+        const double wc = s_all[r][resid ? 0 : 1];
+        if (target < cum + wc) { ch = r; break; }
+        cum += wc;
+        if (r == nchunk - 1) cum -= wc;   // not found: scan the last chunk
+      }
+      s_chunk = ch;
+      s_resid = resid;
+      s_target = target - cum;
     }
-    s_chunk = ch;
-    s_resid = resid;
-    s_target = target - cum;
   }
+  VERIFY_TRACE(tr, 22);
   cl.sync();                                          // remote reads done; s_* visible
+  VERIFY_TRACE(tr, 23);
   if (s_chunk != c) return;
   // the owner scans the weights it already holds (no reload, no recompute)
   constexpr int kVec = 16 / sizeof(T);
@@ -592,6 +674,7 @@ __global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyAr
     if (vec_ok) select_from_regs<kVec>(a, b, j, c, target, wp);
     else select_from_regs<1>(a, b, j, c, target, wp);
   }
+  VERIFY_TRACE(blockIdx.y == 0 && threadIdx.x == 0, 24);
 }
 
 template <typename T>
@@ -672,6 +755,7 @@ cudaError_t launch_greedy_stats(const VerifyArgs& a, cudaStream_t s) {
 }
 
 int verify_chunks(int V) { return (V + kChunk - 1) / kChunk; }
+
 
 }  // namespace tidar
 

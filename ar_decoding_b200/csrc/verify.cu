@@ -63,12 +63,15 @@ __device__ __forceinline__ void amax_merge(float& v, int& i, float v2, int i2) {
   if (v2 > v || (v2 == v && i2 < i)) { v = v2; i = i2; }
 }
 
-// Loads this thread's kPer elements of the chunk (index order t*8.., strided by
-// 8*kThreads for 16-byte vector loads when the row is vector aligned).
-template <typename T>
-__device__ __forceinline__ int load_chunk(const T* row, int V, int c0, float (&x)[kPer],
-                                          int (&ix)[kPer], bool vec_ok) {
+// Loads this thread's kChunk / TH elements of the chunk (runs of one 16-byte
+// vector, run r of thread t at c0 + (r * TH + t) * (16 / sizeof(T)), when the
+// row is vector aligned; else single elements strided by TH).
+template <typename T, int TH = kThreads>
+__device__ __forceinline__ int load_chunk(const T* row, int V, int c0, float (&x)[kChunk / TH],
+                                          int (&ix)[kChunk / TH], bool vec_ok) {
+  constexpr int kPer = kChunk / TH, kThreads = TH;
   constexpr int kVec = 16 / sizeof(T);
+  static_assert(kPer % kVec == 0, "whole vectors per thread");
   int cnt = 0;
   if (vec_ok) {
     // the 16-byte loads first, so they are in flight together
@@ -362,19 +365,20 @@ __device__ void scan_and_norms_block(const VerifyArgs& a, int b, bool first, con
 // Chunk c's weights of both candidate laws for row j, in load_chunk's layout:
 // wp = p_j, wr = max(0, p_j - q_j) (0 when j = n); slots past V hold 0.  The
 // probabilities are exp(x - M) times the normaliser's reciprocal (fp64).
-template <typename T>
+template <typename T, int TH = kThreads>
 __device__ void chunk_weights(const VerifyArgs& a, int b, int c, int j, double Mp, double iZp,
-                              double Mq, double iZq, bool vec_ok, double (&wr)[kPer],
-                              double (&wp)[kPer]) {
+                              double Mq, double iZq, bool vec_ok, double (&wr)[kChunk / TH],
+                              double (&wp)[kChunk / TH]) {
+  constexpr int kPer = kChunk / TH;
   const T* prow = static_cast<const T*>(a.logits) + ((size_t)b * a.n + (j - 1)) * a.V;
   float xp[kPer];
   int ix[kPer];
-  load_chunk<T>(prow, a.V, c * kChunk, xp, ix, vec_ok);
+  load_chunk<T, TH>(prow, a.V, c * kChunk, xp, ix, vec_ok);
   if (j < a.n) {
     const T* qrow = q_row<T>(a, b, j);
     float xq[kPer];
     int iq[kPer];
-    load_chunk<T>(qrow, a.V, c * kChunk, xq, iq, vec_ok);
+    load_chunk<T, TH>(qrow, a.V, c * kChunk, xq, iq, vec_ok);
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
       const bool ok = ix[e] != INT_MAX;
@@ -394,8 +398,10 @@ __device__ void chunk_weights(const VerifyArgs& a, int b, int c, int j, double M
 
 // Block sums of both weight arrays, valid in thread 0 (warp butterflies, then
 // the warps in order).
-__device__ void block_sums(const double (&wr)[kPer], const double (&wp)[kPer], double& out_r,
+template <int TH = kThreads>
+__device__ void block_sums(const double (&wr)[kChunk / TH], const double (&wp)[kChunk / TH], double& out_r,
                            double& out_p) {
+  constexpr int kPer = kChunk / TH, kThreads = TH;
   double sr = 0.0, sp = 0.0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) { sr += wr[e]; sp += wp[e]; }
@@ -408,22 +414,34 @@ __device__ void block_sums(const double (&wr)[kPer], const double (&wp)[kPer], d
   const int w = threadIdx.x >> 5;
   if ((threadIdx.x & 31) == 0) { s1[w] = sr; s2[w] = sp; }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    sr = 0.0; sp = 0.0;
-    for (int i = 0; i < kThreads / 32; ++i) { sr += s1[i]; sp += s2[i]; }
-    out_r = sr;
-    out_p = sp;
+  if constexpr (kThreads / 32 <= 8) {
+    if (threadIdx.x == 0) {
+      sr = 0.0; sp = 0.0;
+      for (int i = 0; i < kThreads / 32; ++i) { sr += s1[i]; sp += s2[i]; }
+      out_r = sr;
+      out_p = sp;
+    }
+  } else if (threadIdx.x < 32) {              // many warps: their sums by one more butterfly
+    sr = threadIdx.x < kThreads / 32 ? s1[threadIdx.x] : 0.0;
+    sp = threadIdx.x < kThreads / 32 ? s2[threadIdx.x] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sr += __shfl_xor_sync(0xffffffffu, sr, o);
+      sp += __shfl_xor_sync(0xffffffffu, sp, o);
+    }
+    if (threadIdx.x == 0) { out_r = sr; out_p = sp; }
   }
 }
 
 // Inverse CDF over this CTA's chunk from weights held in load_chunk's layout:
 // runs of L contiguous elements, run r of thread t starting at
-// c0 + (r * kThreads + t) * L (L = the vector width, or 1 for scalar loads).
+// c0 + (r * TH + t) * L (L = the vector width, or 1 for scalar loads).
 // Index-ordered running sums come from one block scan per run; the smallest
 // id with target < running sum is the sample.  Writes the outputs of b.
-template <int L>
+template <int L, int TH = kThreads>
 __device__ void select_from_regs(const VerifyArgs& a, int b, int j, int chunk, double target,
-                                 const double (&w)[kPer]) {
+                                 const double (&w)[kChunk / TH]) {
+  constexpr int kPer = kChunk / TH, kThreads = TH;
   __shared__ double s_wsum[kThreads / 32];
   __shared__ int s_found, s_last;
   if (threadIdx.x == 0) { s_found = INT_MAX; s_last = -1; }
@@ -601,10 +619,17 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
 // as select_kernel does), locates the target chunk, and the CTA that owns it
 // runs the inverse CDF.  A second cluster barrier keeps every CTA's shared
 // memory alive until the remote reads are done.
+// One 16-byte vector of the chunk per thread: 1024 threads for fp32 logits,
+// 512 for bf16 (the fp64 exponentials of the weights are latency bound at
+// fewer threads; one run per thread also makes the inverse CDF one block scan).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyArgs a,
+constexpr int rej_threads() { return kChunk / (16 / (int)sizeof(T)); }
+
+template <typename T>
+__global__ void __launch_bounds__(rej_threads<T>()) resid_select_cluster_kernel(VerifyArgs a,
                                                                         const ChunkStat* stats,
                                                                         int nchunk, bool vec_ok) {
+  constexpr int TH = rej_threads<T>(), kPer = kChunk / TH;
   [[maybe_unused]] const bool tr = blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0;
   VERIFY_TRACE(tr, 16);
   pdl_wait();
@@ -619,10 +644,10 @@ __global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyAr
   VERIFY_TRACE(tr, 18);
   const int j = sj;
   double wr[kPer], wp[kPer];
-  chunk_weights<T>(a, b, c, j, sMp, 1.0 / sZp, sMq, j < a.n ? 1.0 / sZq : 0.0, vec_ok, wr, wp);
+  chunk_weights<T, TH>(a, b, c, j, sMp, 1.0 / sZp, sMq, j < a.n ? 1.0 / sZq : 0.0, vec_ok, wr, wp);
   VERIFY_TRACE(tr, 19);
   double sr = 0.0, sp = 0.0;
-  block_sums(wr, wp, sr, sp);
+  block_sums<TH>(wr, wp, sr, sp);
   if (threadIdx.x == 0) { s_sum[0] = sr; s_sum[1] = sp; }
   VERIFY_TRACE(tr, 20);
   cl.sync();
@@ -668,11 +693,11 @@ __global__ void __launch_bounds__(kThreads) resid_select_cluster_kernel(VerifyAr
   constexpr int kVec = 16 / sizeof(T);
   const double target = s_target;
   if (s_resid) {
-    if (vec_ok) select_from_regs<kVec>(a, b, j, c, target, wr);
-    else select_from_regs<1>(a, b, j, c, target, wr);
+    if (vec_ok) select_from_regs<kVec, TH>(a, b, j, c, target, wr);
+    else select_from_regs<1, TH>(a, b, j, c, target, wr);
   } else {
-    if (vec_ok) select_from_regs<kVec>(a, b, j, c, target, wp);
-    else select_from_regs<1>(a, b, j, c, target, wp);
+    if (vec_ok) select_from_regs<kVec, TH>(a, b, j, c, target, wp);
+    else select_from_regs<1, TH>(a, b, j, c, target, wp);
   }
   VERIFY_TRACE(blockIdx.y == 0 && threadIdx.x == 0, 24);
 }
@@ -709,8 +734,8 @@ cudaError_t launch_t(const VerifyArgs& a, cudaStream_t s) {
   // residual sums + inverse CDF: one cluster per sequence when the chunks fit
   // one cluster, else two launches through the workspace
   static int rs_limit[64];
-  if (nchunk <= cluster_limit(resid_select_cluster_kernel<T>, kThreads, rs_limit))
-    return launch_cluster(resid_select_cluster_kernel<T>, nchunk, a.B, kThreads, 0, s, a,
+  if (nchunk <= cluster_limit(resid_select_cluster_kernel<T>, rej_threads<T>(), rs_limit))
+    return launch_cluster(resid_select_cluster_kernel<T>, nchunk, a.B, rej_threads<T>(), 0, s, a,
                           (const ChunkStat*)stats, nchunk, vec_ok);
   e = launch_pdl(residual_kernel<T>, dim3(nchunk, a.B), kThreads, 0, s, a, (const ChunkStat*)stats, nchunk, wsum, jbuf,
                  vec_ok);

@@ -123,17 +123,43 @@ __device__ unsigned long long g_verify_trace[16 * 8];
 #define VERIFY_TRACE(cond, slot) do {} while (0)
 #endif
 
+// One 16-byte vector of the chunk per thread: 1024 threads for fp32 logits,
+// 512 for bf16 (the fp64 exponentials of the weights are latency bound at
+// fewer threads; one run per thread also makes the inverse CDF one block scan).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat* stats, int nchunk,
-                                                         bool vec_ok) {
+constexpr int rej_threads() { return kChunk / (16 / (int)sizeof(T)); }
+
+// TH threads per chunk: 256 for greedy (no exponentials); rejection uses
+// rej_threads<T>() (fp64 exponentials, latency bound at fewer threads).
+template <typename T, int TH = kThreads>
+__global__ void __launch_bounds__(TH) stats_kernel(VerifyArgs a, ChunkStat* stats, int nchunk,
+                                                   bool vec_ok) {
+  constexpr int kThreads = TH, kPer = kChunk / TH;
   [[maybe_unused]] const bool tr = blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0;
   VERIFY_TRACE(tr, 0);
-  if ((int)blockIdx.y < a.B * a.n) {
-    // this CTA's chunk of its logits row into L2 while the previous kernel ends
+  {
+    // this CTA's chunk of its row into L2 while the previous kernel ends (a
+    // hint: for a q row read through draft_block, the block index is read
+    // ahead of the dependency wait with a relaxed load and clamped, so a
+    // stale value only prefetches another row of the same tensor)
     const int lo = (int)blockIdx.x * kChunk, hi = min(a.V, lo + kChunk);
-    if (hi > lo)
-      prefetch_l2(static_cast<const T*>(a.logits) + (size_t)blockIdx.y * a.V + lo, (size_t)(hi - lo) * sizeof(T),
-                  (int)threadIdx.x, kThreads);
+    const T* row = nullptr;
+    const int prow = a.B * a.n;
+    if ((int)blockIdx.y < prow) {
+      row = static_cast<const T*>(a.logits) + (size_t)blockIdx.y * a.V;
+    } else if (a.mode == TIDAR_REJECTION && a.k > 1) {
+      const int qb = ((int)blockIdx.y - prow) / (a.k - 1), qi = ((int)blockIdx.y - prow) % (a.k - 1) + 1;
+      const T* base = static_cast<const T*>(a.draft_logits);
+      if (!a.draft_block) {
+        row = base + ((size_t)qb * (a.k - 1) + (qi - 1)) * a.V;
+      } else {
+        int jb;
+        asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(jb) : "l"(a.draft_block + qb));
+        if (jb < 1 || jb > a.k) jb = 1;
+        row = base + (((size_t)qb * a.k + (jb - 1)) * a.k + qi) * a.V;
+      }
+    }
+    if (row && hi > lo) prefetch_l2(row + lo, (size_t)(hi - lo) * sizeof(T), (int)threadIdx.x, kThreads);
   }
   pdl_wait();
   pdl_trigger();
@@ -144,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat
                            : q_row<T>(a, (rr - prow) / (a.k - 1), (rr - prow) % (a.k - 1) + 1);
   float x[kPer];
   int ix[kPer];
-  load_chunk<T>(row, a.V, c * kChunk, x, ix, vec_ok);
+  load_chunk<T, TH>(row, a.V, c * kChunk, x, ix, vec_ok);
   float bv = -INFINITY;
   int bi = INT_MAX;
 #pragma unroll
@@ -161,9 +187,22 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) { sv[w] = bv; si[w] = bi; }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int i = 1; i < kThreads / 32; ++i) amax_merge(bv, bi, sv[i], si[i]);
-    sv[0] = bv; si[0] = bi;
+  if constexpr (kThreads / 32 <= 8) {
+    if (threadIdx.x == 0) {
+      for (int i = 1; i < kThreads / 32; ++i) amax_merge(bv, bi, sv[i], si[i]);
+      sv[0] = bv; si[0] = bi;
+    }
+  } else if (threadIdx.x < 32) {             // many warps: one more exact butterfly
+    bv = lane < kThreads / 32 ? sv[lane] : -INFINITY;
+    bi = lane < kThreads / 32 ? si[lane] : INT_MAX;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+      amax_merge(bv, bi, v2, i2);
+    }
+    __syncwarp();
+    if (lane == 0) { sv[0] = bv; si[0] = bi; }
   }
   __syncthreads();
   const float cmax = sv[0];
@@ -177,9 +216,15 @@ __global__ void __launch_bounds__(kThreads) stats_kernel(VerifyArgs a, ChunkStat
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (lane == 0) sd[w] = sum;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      sum = 0.0;
-      for (int i = 0; i < kThreads / 32; ++i) sum += sd[i];
+    if constexpr (kThreads / 32 <= 8) {
+      if (threadIdx.x == 0) {
+        sum = 0.0;
+        for (int i = 0; i < kThreads / 32; ++i) sum += sd[i];
+      }
+    } else if (threadIdx.x < 32) {
+      sum = lane < kThreads / 32 ? sd[lane] : 0.0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     }
   }
   if (threadIdx.x == 0) {
@@ -321,15 +366,21 @@ __device__ void scan_and_norms_block(const VerifyArgs& a, int b, bool first, con
     s_cs[idx] = st.sum;
   }
   __syncthreads();
-  if ((int)threadIdx.x < R) {
-    const float* cm = s_cm + threadIdx.x * nchunk;
-    const double* cs = s_cs + threadIdx.x * nchunk;
+  // row_norm's terms exp(max_c - M) sum_c, one thread per (row, chunk), then
+  // one thread per row adds them in chunk order (the same arithmetic)
+  for (int idx = threadIdx.x; idx < R * nchunk; idx += blockDim.x) {
+    const int r = idx / nchunk;
+    const float* cm = s_cm + r * nchunk;
     float mf = -INFINITY;
     for (int c = 0; c < nchunk; ++c) mf = fmaxf(mf, cm[c]);
-    const double M = (double)mf;
+    s_cs[idx] = exp((double)s_cm[idx] - (double)mf) * s_cs[idx];
+    if (idx == r * nchunk) s_M[r] = (double)mf;
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < R) {
+    const double* terms = s_cs + threadIdx.x * nchunk;
     double Z = 0.0;
-    for (int c = 0; c < nchunk; ++c) Z += exp((double)cm[c] - M) * cs[c];
-    s_M[threadIdx.x] = M;
+    for (int c = 0; c < nchunk; ++c) Z += terms[c];
     s_Z[threadIdx.x] = Z;
   }
   __syncthreads();
@@ -619,12 +670,6 @@ __global__ void __launch_bounds__(kThreads) select_kernel(VerifyArgs a, const Ch
 // as select_kernel does), locates the target chunk, and the CTA that owns it
 // runs the inverse CDF.  A second cluster barrier keeps every CTA's shared
 // memory alive until the remote reads are done.
-// One 16-byte vector of the chunk per thread: 1024 threads for fp32 logits,
-// 512 for bf16 (the fp64 exponentials of the weights are latency bound at
-// fewer threads; one run per thread also makes the inverse CDF one block scan).
-template <typename T>
-constexpr int rej_threads() { return kChunk / (16 / (int)sizeof(T)); }
-
 template <typename T>
 __global__ void __launch_bounds__(rej_threads<T>()) resid_select_cluster_kernel(VerifyArgs a,
                                                                         const ChunkStat* stats,
@@ -726,7 +771,10 @@ cudaError_t launch_t(const VerifyArgs& a, cudaStream_t s) {
   const bool vec_ok = ((size_t)a.V * sizeof(T)) % 16 == 0;
   ChunkStat* stats = static_cast<ChunkStat*>(a.workspace);
   const int rows = a.B * a.n + (a.mode == TIDAR_REJECTION ? a.B * (a.k > 1 ? a.k - 1 : 0) : 0);
-  cudaError_t e = launch_pdl(stats_kernel<T>, dim3(nchunk, rows), kThreads, 0, s, a, stats, nchunk, vec_ok);
+  cudaError_t e = a.mode == TIDAR_REJECTION
+                      ? launch_pdl(stats_kernel<T, rej_threads<T>()>, dim3(nchunk, rows), rej_threads<T>(), 0, s, a,
+                                   stats, nchunk, vec_ok)
+                      : launch_pdl(stats_kernel<T>, dim3(nchunk, rows), kThreads, 0, s, a, stats, nchunk, vec_ok);
   if (e != cudaSuccess) return e;
   char* base = static_cast<char*>(a.workspace) + (((size_t)rows * nchunk * sizeof(ChunkStat) + 255) & ~(size_t)255);
   double* wsum = reinterpret_cast<double*>(base);

@@ -12,14 +12,17 @@ Inputs are seeded synthetic tensors generated on the device.  One rank per GPU
 collective on the data path).
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
-cudaDeviceSynchronize.  Each step replays a CUDA graph captured from the public
-API calls (step attention, verify, commit) and is timed on the device with CUDA
-events on the launching stream.  Steps rotate over enough independent
-input/cache copies that each step's working set is evicted from L2 (126 MB)
-before it is reused.  Between steps (outside the events) a second graph
-restores the copy's prefix length and page table so every step does identical
-work.  The attention call alone is timed the same way in a second pass.
-ms_per_step / value is the mean step time, max over ranks.
+cudaDeviceSynchronize.  The steps (step attention, then verification and
+commit, captured from the public API calls) run back to back as a serving loop
+issues them: replays of CUDA graphs that each hold the steps of up to n
+independent input/cache copies in a row, timed on the device with CUDA events
+on the launching stream, one event pair per replay.  The copies are enough
+that each step's working set is evicted from L2 (126 MB) before it is reused;
+after each replay (outside the events) a second graph restores those copies'
+prefix lengths and page tables, so every step does identical work.
+ms_per_step / value is the mean step time, max over ranks.  For reference the
+line also carries step_call_us: each step alone, its own one-step graph between
+two events (adding the device-side cost of one graph launch per step).
 
 Also in the line: the attention kernel's roofline (algorithmic bytes or flops
 over its launch duration, against the measured peaks), the k sweep, the other
@@ -219,6 +222,25 @@ class Step:
         c = self.copies[i]
         c["cache"]["seq_lens"].copy_(c["seq0"], non_blocking=True)
         c["cache"]["page_table"].copy_(c["pt0"], non_blocking=True)
+
+    def round_graph(self, m):
+        """(graph of the steps of copies 0..m-1 back to back, graph restoring
+        those copies), captured once per m."""
+        rg = self.__dict__.setdefault("_rounds", {})
+        if m not in rg:
+            gs, gr = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gs):
+                for i in range(m):
+                    self.attn(i)
+                    self.verify_commit(i)
+            with torch.cuda.graph(gr):
+                for i in range(m):
+                    self.restore(i)
+            torch.cuda.synchronize()
+            gr.replay()
+            torch.cuda.synchronize()
+            rg[m] = (gs, gr)
+        return rg[m]
 
     def capture(self):
         """Per copy, one CUDA graph of the whole step (attention, verify, commit),
@@ -642,10 +664,14 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- timing
 def time_steps(st: Step, K: int, W: int, world: int):
-    """Returns per-step device µs and per-call step_attn µs (lists).  Each timed
-    step replays its copy's whole-step graph between two events on the launching
-    stream; the restore graph runs outside the events.  The attention call is
-    timed the same way in a second pass with the attention-only graphs."""
+    """Returns (per-step device µs, per-call step_attn µs, per-step µs of a
+    one-step graph) as lists.  The step: graphs of consecutive steps of
+    different copies, back to back as a serving loop issues them (the
+    attention's own figure is taken the same way), each replay between two
+    events on the launching stream, the restore graphs outside the events.
+    For reference each step is also timed alone, its copy's one-step graph
+    between two events (that adds the device-side cost of launching a graph
+    to every step), and the attention call likewise."""
     n = len(st.copies)
     st.capture()
     stream = torch.cuda.current_stream()
@@ -673,9 +699,37 @@ def time_steps(st: Step, K: int, W: int, world: int):
         barrier(world)
         return [a.elapsed_time(b) * 1e3 for a, b in ev]
 
-    step_us = run(0, K, W)
+    def run_rounds(count, warm):
+        """Steps back to back: one graph holds the steps of m <= n copies in
+        a row (each copy once, so every step does the same work), replayed
+        between two events; the restore of those copies runs after the second
+        event.  Each timed step gets its round's mean."""
+        for i in range(warm):
+            st.round_graph(n)[0].replay(); st.round_graph(n)[1].replay()
+        torch.cuda.synchronize()
+        sizes = [n] * (count // n) + ([count % n] if count % n else [])
+        graphs = [st.round_graph(m) for m in sizes]
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in sizes]
+        barrier(world)
+        torch.cuda.synchronize()
+        hold_stream(count)
+        for (gs, gr), (e0, e1) in zip(graphs, ev):
+            e0.record(stream)
+            gs.replay()
+            e1.record(stream)
+            gr.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        out = []
+        for m, (e0, e1) in zip(sizes, ev):
+            out += [e0.elapsed_time(e1) * 1e3 / m] * m
+        return out
+
+    step_call_us = run(0, K, W)
     attn_us = run(1, K, W)
-    return step_us, attn_us
+    # small workloads flush L2 between steps: there every step keeps its own graph
+    step_us = step_call_us if flush else run_rounds(K, W)
+    return step_us, attn_us, step_call_us
 
 
 def time_attention_launches(st: Step, reps: int, attn_call_us=None):
@@ -871,7 +925,7 @@ def run_ours(args, rank, world, local):
     st = Step(cfg, copies_for(cfg), path=args.path)
     clocks = ClockSampler(local)
     clocks.start()
-    step_us, attn_us = time_steps(st, args.steps, args.warmup, world)
+    step_us, attn_us, step_call_us = time_steps(st, args.steps, args.warmup, world)
     kern_us = reduce_max(time_attention_launches(st, max(3, args.steps // 3)), world)
     clk = clocks.stop()
     mean_step = reduce_max(statistics.mean(step_us), world)
@@ -893,10 +947,11 @@ def run_ours(args, rank, world, local):
         for kk in (0, 4, 8, 16):
             c2 = workload(kk, args.prefix, rank)
             s2 = Step(c2, copies_for(c2), path=args.path)
-            su, au = time_steps(s2, max(10, args.steps // 2), 3, world)
+            su, au, sc = time_steps(s2, max(10, args.steps // 2), 3, world)
             b2, f2 = algorithmic(c2)
             a2 = reduce_max(time_attention_launches(s2, 3), world) * 1e-6
             sweep.append({"k": kk, "rows": c2.R, "step_us": reduce_max(statistics.mean(su), world),
+                          "step_call_us": reduce_max(statistics.mean(sc), world),
                           "attn_call_us": reduce_max(statistics.mean(au), world),
                           "attn_us": a2 * 1e6, "attn_hbm_gbs": b2 / a2 / 1e9,
                           "hbm_frac": (b2 / a2 / 1e9) / hbm_peak,
@@ -914,7 +969,7 @@ def run_ours(args, rank, world, local):
                    synth.long_context(8, 131072, 0), synth.long_context(8, 131072, 16),
                    synth.class_1p5b(), synth.tiny()):
             s2 = Step(c2, copies_for(c2), path=args.path)
-            su, au = time_steps(s2, max(5, args.steps // 4), 3, world)
+            su, au, _ = time_steps(s2, max(5, args.steps // 4), 3, world)
             a2 = reduce_max(time_attention_launches(s2, 2, statistics.mean(au)), world) * 1e-6
             b2, f2 = algorithmic(c2)
             extra.append({"workload": c2.name, "B": c2.B, "prefix_total": sum(c2.prefix),
@@ -975,6 +1030,7 @@ def run_ours(args, rank, world, local):
             "data": "synthetic (seeded, generated on device)",
             "config": bench_config(cfg, args.prefix, args.k),
             "attn_plan": {"path": PATH_NAMES[st.path_id], "splits": st.splits},
+            "step_call_us": reduce_max(statistics.mean(step_call_us), world),
             "attn_call_us": mean_attn, "attn_us": kern_us, "attn_launches": st.attn_launches,
             "hbm_gbs_attn": bytes_ / attn_s / 1e9,
             "hbm_gbs_all_gpus": agg_gbs,

@@ -344,18 +344,25 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 0) {
       bool ok = wait_bar(bar(BAR_Q), 0, abort_flag, a.err);
       fence_after();
-      const uint32_t qa = sb + kOffQ;
+      // Operand descriptors: a descriptor's start-address field is the shared
+      // address / 16 (below 2^14 here), so a tile at base + delta has the
+      // descriptor of base plus delta / 16.  Q's eight are fixed; a stage's
+      // K and V ones are its ring slot's base plus constants, formed ahead of
+      // the eight-MMA asm blocks.
+      uint64_t dq[8];
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) dq[kc] = desc_k_sw128(sb + kOffQ + (kc >> 2) * kChunkBytes + (kc & 3) * 32);
+      const uint64_t dk0 = desc_k_sw128(sb + kOffK), dv0 = desc_mn_sw128(sb + kOffV, kChunkBytes);
       auto issue_s = [&](int blk) -> bool {
         const int st = blk % kStages, t = blk & 1;
         if (!wait_bar(bar(BAR_KFULL + st), (uint32_t)((blk / kStages) & 1), abort_flag, a.err)) return false;
         TIDAR_TRACE_AT(256 + min(blk, 255));
         fence_after();
-        const uint32_t ka = sb + kOffK + st * kTileBytes;
+        const uint64_t kbase = dk0 + (uint64_t)((st * kTileBytes) >> 4);
+        uint64_t dk[8];
 #pragma unroll
-        for (int kc = 0; kc < 8; ++kc) {
-          const uint32_t off = (kc >> 2) * kChunkBytes + (kc & 3) * 32;
-          mma_ss(tmem + col_s(t), desc_k_sw128(qa + off), desc_k_sw128(ka + off), kIdescS, kc > 0);
-        }
+        for (int kc = 0; kc < 8; ++kc) dk[kc] = kbase + (uint64_t)(((kc >> 2) * kChunkBytes + (kc & 3) * 32) >> 4);
+        mma_ss_x8(tmem + col_s(t), dq, dk, kIdescS, 0u);
         mma_commit(bar(BAR_SFULL + t));
         mma_commit(bar(BAR_KEMPTY + st));
         TIDAR_TRACE_AT(512 + min(blk, 255));
@@ -368,11 +375,15 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_bar(bar(BAR_VFULL + st), (uint32_t)((b2 / kStages) & 1), abort_flag, a.err)) break;
         if (!wait_bar(bar(BAR_PFULL + t), (uint32_t)(j & 1), abort_flag, a.err)) break;
         fence_after();
-        const uint32_t va = sb + kOffV + st * kTileBytes;
+        const uint64_t vbase = dv0 + (uint64_t)((st * kTileBytes) >> 4);
+        uint32_t pa[8];
+        uint64_t dv[8];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + col_o(t), tmem + col_s(t) + p_col(kk), desc_mn_sw128(va + kk * 2048, kChunkBytes), kIdescPV,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) {
+          pa[kk] = tmem + col_s(t) + p_col(kk);
+          dv[kk] = vbase + (uint64_t)((kk * 2048) >> 4);
+        }
+        mma_ts_x8(tmem + col_o(t), pa, dv, kIdescPV, j > 0 ? 1u : 0u);
         mma_commit(bar(BAR_PVDONE + t));
         mma_commit(bar(BAR_VEMPTY + st));
         TIDAR_TRACE_AT(768 + min(b2, 255));

@@ -54,22 +54,46 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(AttnArgs a) {
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
 
-  auto update = [&](const T* kp, const T* vp) {
-    float kv[VPL], vv[VPL];
-    load_vec<T, VPL>(kp, kv);
-    float dot = 0.f;
+  // Online-softmax update with a batch of up to kKB keys whose K and V slices
+  // are in registers (ok[u]: key u exists): all the batch's dot products and
+  // warp sums first, then one rescale of (l, acc) by the batch's new maximum.
+  constexpr int kKB = 8;
+  auto update = [&](const float (&kv)[kKB][VPL], const float (&vv)[kKB][VPL], const bool (&ok)[kKB]) {
+    float sc[kKB];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) dot = fmaf(qv[i], kv[i], dot);
-    const float s = warp_sum(dot);
-    load_vec<T, VPL>(vp, vv);
-    const float mn = fmaxf(mx, s);
-    const float corr = expf(mx - mn);   // 0 on the first key (mx = -inf)
-    const float pe = expf(s - mn);
-    l = fmaf(l, corr, pe);
+    for (int u = 0; u < kKB; ++u) {
+      float dot = 0.f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) acc[i] = fmaf(acc[i], corr, pe * vv[i]);
+      for (int i = 0; i < VPL; ++i) dot = fmaf(qv[i], kv[u][i], dot);
+      sc[u] = dot;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < kKB; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+    float mn = mx;
+#pragma unroll
+    for (int u = 0; u < kKB; ++u)
+      if (ok[u]) mn = fmaxf(mn, sc[u]);
+    if (mn == -INFINITY) return;                    // no key in the batch (and none before)
+    const float corr = expf(mx - mn);               // 0 while mx = -inf
+    float ps = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] *= corr;
+#pragma unroll
+    for (int u = 0; u < kKB; ++u) {
+      if (!ok[u]) continue;                          // its K/V registers were never loaded
+      const float pe = expf(sc[u] - mn);
+      ps += pe;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) acc[i] = fmaf(pe, vv[u][i], acc[i]);
+    }
+    l = fmaf(l, corr, ps);
     mx = mn;
   };
+  // Keys go in batches of kKB: the K and V slices of a batch are all loaded
+  // before the first is used (one memory round trip per batch, not two per
+  // key).
 
   // prefix keys of this split
   const int k0 = split * a.keys_per_split;
@@ -78,11 +102,26 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(AttnArgs a) {
   const T* vpages = static_cast<const T*>(a.v_pages);
   const int32_t* table = a.page_table + (size_t)b * a.max_pages;
   bool bad_page = false;
-  for (int key = k0; key < k1; ++key) {
-    const int page = table[key / a.page_size];
-    if (page < 0 || page >= a.num_pages) { bad_page = true; continue; }
-    const size_t off = ((size_t)(page * a.Hkv + g) * a.page_size + key % a.page_size) * D + lane * VPL;
-    update(kpages + off, vpages + off);
+  for (int key0 = k0; key0 < k1; key0 += kKB) {
+    float kv[kKB][VPL], vv[kKB][VPL];
+    bool ok[kKB];
+#pragma unroll
+    for (int u = 0; u < kKB; ++u) {
+      const int key = key0 + u;
+      ok[u] = false;
+      if (key < k1) {
+        const int page = table[key / a.page_size];
+        if (page < 0 || page >= a.num_pages) {
+          bad_page = true;
+        } else {
+          const size_t off = ((size_t)(page * a.Hkv + g) * a.page_size + key % a.page_size) * D + lane * VPL;
+          load_vec<T, VPL>(kpages + off, kv[u]);
+          load_vec<T, VPL>(vpages + off, vv[u]);
+          ok[u] = true;
+        }
+      }
+    }
+    update(kv, vv, ok);
   }
   if (bad_page && lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_PAGE);
 
@@ -91,10 +130,20 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(AttnArgs a) {
     const StepVis vis = step_visibility(a.k, rho);
     const T* kb = static_cast<const T*>(a.k_blk);
     const T* vb = static_cast<const T*>(a.v_blk);
-    for (int key = 0; key < a.R; ++key) {
-      if (!step_visible(vis, key)) continue;
-      const size_t off = ((size_t)(b * a.R + key) * a.Hkv + g) * D + lane * VPL;
-      update(kb + off, vb + off);
+    for (int key0 = 0; key0 < a.R; key0 += kKB) {
+      float kv[kKB][VPL], vv[kKB][VPL];
+      bool ok[kKB];
+#pragma unroll
+      for (int u = 0; u < kKB; ++u) {
+        const int key = key0 + u;
+        ok[u] = key < a.R && step_visible(vis, key);
+        if (ok[u]) {
+          const size_t off = ((size_t)(b * a.R + key) * a.Hkv + g) * D + lane * VPL;
+          load_vec<T, VPL>(kb + off, kv[u]);
+          load_vec<T, VPL>(vb + off, vv[u]);
+        }
+      }
+      update(kv, vv, ok);
     }
   }
 

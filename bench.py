@@ -580,7 +580,7 @@ def needs_flush(cfg) -> bool:
 
 def l2_policy(cfg) -> str:
     if needs_flush(cfg):
-        return (f"rotating {copies_for(cfg)} input copies and writing a {2 * L2_BYTES >> 20} MiB "
+        return (f"rotating {copies_for(cfg)} input copies and reading a {2 * L2_BYTES >> 20} MiB "
                 "buffer (> L2) between timed steps")
     return f"rotating {copies_for(cfg)} independent input copies (> 3x L2) between timed steps"
 
@@ -589,11 +589,14 @@ _FLUSH = {}
 
 
 def flush_l2():
-    """Write a buffer twice the size of L2 (evicts every earlier line)."""
+    """Read a buffer twice the size of L2 (evicts every earlier line).  A read,
+    not a write: a flush that leaves L2 full of dirty lines makes the next
+    kernel wait for their write-back (~100 µs), which is not the workload's."""
     buf = _FLUSH.get("buf")
     if buf is None:
-        buf = _FLUSH["buf"] = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
-    buf.zero_()
+        buf = _FLUSH["buf"] = torch.zeros(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+        _FLUSH["sink"] = torch.empty((), dtype=torch.uint8, device="cuda")
+    torch.amax(buf, dim=0, out=_FLUSH["sink"])
 
 
 def hold_stream(items: int, us_per_item: float = 40.0) -> None:

@@ -7,9 +7,10 @@
 // zeroed, the length advances to P+c and pages that held only rejected rows
 // are released.
 //
-// One launch: a single thread-block cluster of C <= 16 CTAs; CTA r owns the
-// contiguous sequences [r*per, (r+1)*per) (with fewer sequences than CTAs,
-// the zeroing of step 3 is shared by the whole cluster).
+// One launch: a single thread-block cluster of C <= 16 CTAs (one per 16 KB
+// of rows to zero; one CTA up to 32 KB); CTA r owns the contiguous sequences
+// [r*per, (r+1)*per) (with fewer sequences than CTAs, the zeroing of step 3
+// is shared by the whole cluster).
 //   1. every CTA validates its own sequences (one warp per sequence, the
 //      page-table entries loaded by parallel lanes) and counts the pages each
 //      releases (-1: invalid, left untouched), then an exclusive scan of the
@@ -22,6 +23,8 @@
 //      page-table entries and advances seq_lens; the tail of the list is -1.
 // No device-side waits besides the two hardware cluster barriers.
 #include <cooperative_groups.h>
+
+#include <algorithm>
 
 #include "accept.cuh"
 #include "common.cuh"
@@ -60,9 +63,6 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
                                                                     GreedyAcceptArgs f) {
   __shared__ int s_g[kFused ? kCWarps : 1][kFused ? 16 * 16 : 1];   // per-warp block guesses
   COMMIT_TRACE(0);
-  pdl_wait();
-  pdl_trigger();
-  COMMIT_TRACE(1);
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks();
   const int rank = (int)cl.block_rank();
@@ -80,13 +80,39 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
   const int b0 = rank * per;
   const int nown = max(0, min(a.B, b0 + per) - b0);
   const int ps = a.page_size;
+  // Fused with a greedy verification, the kernel before this one is the
+  // verification's statistics, which write neither lengths nor page tables;
+  // and that kernel passed its own dependency wait before this one could
+  // start, so everything earlier on the stream is complete.  The lengths and
+  // the page-table entries of the draft rows are therefore read before the
+  // wait (relaxed loads, so no stale L1 copy is used), overlapping the
+  // statistics' tail.
+  const bool early = kFused;
+  if (early) {
+    // own sequences (spread: every sequence, into the all-sequence records)
+    for (int i = wid; i < (spread ? a.B : nown); i += kCWarps) {
+      const int b = spread ? i : b0 + i;
+      int* pgs = spread ? s_allpg + i * npm : s_pg + i * npm;
+      const int P = ld_relaxed(a.seq_lens + b);
+      if (P >= 0 && (P + a.n + ps - 1) / ps <= a.max_pages) {
+        const int p0 = P / ps, np = (P + a.n - 1) / ps - p0 + 1;
+        if (lane < np) pgs[lane] = ld_relaxed(a.page_table + (size_t)b * a.max_pages + p0 + lane);
+      }
+      if (lane == 0) (spread ? s_all : s_rec)[i].P = P;
+    }
+    __syncwarp();
+  }
+  pdl_wait();
+  pdl_trigger();
+  COMMIT_TRACE(1);
 
   // 1. validate, count, keep the pages: one warp per sequence (its own
   //    sequences; with `spread`, every sequence -- the loop below)
   for (int i = wid; i < (spread ? 0 : nown); i += kCWarps) {
     const int b = b0 + i;
-    const int P = a.seq_lens[b];
+    const int P = early ? s_rec[i].P : a.seq_lens[b];
     const int c = kFused ? greedy_accept_warp(f, a.n, a.k, b, s_g[kFused ? wid : 0], true) : a.accept_count[b];
+    COMMIT_TRACE(5);
     int ok = 1;
     if (c < 0 || c > a.n) { ok = 0; if (lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_COUNT); }
     if (ok && (P < 0 || (P + a.n + ps - 1) / ps > a.max_pages)) {
@@ -97,7 +123,7 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
       const int p0 = P / ps, np = (P + a.n - 1) / ps - p0 + 1;   // np <= npm <= 16
       bool bad = false;
       if (lane < np) {
-        const int page = a.page_table[(size_t)b * a.max_pages + p0 + lane];
+        const int page = early ? s_pg[i * npm + lane] : a.page_table[(size_t)b * a.max_pages + p0 + lane];
         bad = page < 0 || page >= a.num_pages;
         s_pg[i * npm + lane] = page;
       }
@@ -118,7 +144,7 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
     // errors and, fused, writes the verification outputs
     for (int b = wid; b < a.B; b += kCWarps) {
       const bool owner = b / per == rank;
-      const int P = a.seq_lens[b];
+      const int P = early ? s_all[b].P : a.seq_lens[b];
       const int c = kFused ? greedy_accept_warp(f, a.n, a.k, b, s_g[kFused ? wid : 0], owner) : a.accept_count[b];
       bool ok = true;
       if (c < 0 || c > a.n) { ok = false; if (owner && lane == 0) raise_error(a.err, TIDAR_DEVERR_BAD_COUNT); }
@@ -130,7 +156,7 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
         const int p0 = P / ps, np = (P + a.n - 1) / ps - p0 + 1;
         bool bad = false;
         if (lane < np) {
-          const int page = a.page_table[(size_t)b * a.max_pages + p0 + lane];
+          const int page = early ? s_allpg[b * npm + lane] : a.page_table[(size_t)b * a.max_pages + p0 + lane];
           bad = page < 0 || page >= a.num_pages;
           s_allpg[b * npm + lane] = page;
         }
@@ -181,9 +207,14 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
     if (lane == 0) s_total = run;
   }
 
-  // 2. bases across the cluster
-  if (!spread) cl.sync();
-  if (!spread && wid == 0) {
+  // 2. bases across the cluster (one CTA: its own totals, no cluster barrier)
+  if (C == 1) {
+    __syncthreads();
+    if (threadIdx.x == 0) { s_base = 0; s_grand = s_total; }
+    __syncthreads();
+  }
+  if (!spread && C > 1) cl.sync();
+  if (!spread && C > 1 && wid == 0) {
     int t = 0;
     if (lane < C) t = *cl.map_shared_rank(&s_total, lane);
     int sb = lane < rank ? t : 0, sg = t;
@@ -194,7 +225,7 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
     }
     if (lane == 0) { s_base = sb; s_grand = sg; }
   }
-  if (!spread) cl.sync();
+  if (!spread && C > 1) cl.sync();
   COMMIT_TRACE(3);
 
   // 3. release and advance (one warp per sequence), then scrub (whole CTA);
@@ -214,26 +245,52 @@ __global__ void __launch_bounds__(kCThreads) commit_cluster_kernel(CommitArgs a,
   }
   const int row_chunks = a.D * a.elem_bytes / 16;
   const int head_chunks = a.Hkv * row_chunks;       // one row of one of K / V, all heads
+  const int cols = 2 * head_chunks;                  // 16-byte pieces of one cache row, K and V
   const int nscrub = spread ? a.B : nown;
   const int t0 = spread ? rank * kCThreads + (int)threadIdx.x : (int)threadIdx.x;
   const int tstep = spread ? C * kCThreads : kCThreads;
-  for (int i = 0; i < nscrub; ++i) {
-    const SeqRec r = spread ? s_all[i] : s_rec[i];
-    const int* pg = spread ? s_allpg + i * npm : s_pg + i * npm;
-    if (r.cnt < 0) continue;
-    const int p0 = r.P / ps;
-    const int total = (a.n - r.c) * 2 * head_chunks;
-    for (int t = t0; t < total; t += tstep) {
-      const int rr = t / (2 * head_chunks);
-      const int rem = t - rr * 2 * head_chunks;
-      const int which = rem >= head_chunks;
-      const int hc = rem - which * head_chunks;
-      const int g = hc / row_chunks, ch = hc - g * row_chunks;
-      const int pos = r.P + r.c + rr;
-      const int page = pg[pos / ps - p0];
-      char* dst = static_cast<char*>(which ? a.v_pages : a.k_pages);
-      const size_t off = (((size_t)page * a.Hkv + g) * ps + pos % ps) * a.D * a.elem_bytes;
-      reinterpret_cast<uint4*>(dst + off)[ch] = make_uint4(0, 0, 0, 0);
+  const size_t row_bytes = (size_t)a.D * a.elem_bytes;
+  if (tstep % cols == 0) {
+    // Each thread keeps one 16-byte column (K or V, head, piece) and walks
+    // the rejected rows tstep / cols apart: the column's decomposition is
+    // computed once, each store costs a page lookup.
+    const int col = t0 % cols, rstep = tstep / cols;
+    const int which = col >= head_chunks;
+    const int hc = col - which * head_chunks;
+    const int g = hc / row_chunks, ch = hc - g * row_chunks;
+    char* dbase = static_cast<char*>(which ? a.v_pages : a.k_pages) + (size_t)g * ps * row_bytes + (size_t)ch * 16;
+    const size_t page_bytes = (size_t)a.Hkv * ps * row_bytes;
+    for (int i = 0; i < nscrub; ++i) {
+      const SeqRec r = spread ? s_all[i] : s_rec[i];
+      const int* pg = spread ? s_allpg + i * npm : s_pg + i * npm;
+      if (r.cnt < 0) continue;
+      const int p0 = r.P / ps;
+      for (int rr = t0 / cols; rr < a.n - r.c; rr += rstep) {
+        const int pos = r.P + r.c + rr;
+        const int pq = pos / ps;
+        *reinterpret_cast<uint4*>(dbase + (size_t)pg[pq - p0] * page_bytes + (size_t)(pos - pq * ps) * row_bytes) =
+            make_uint4(0, 0, 0, 0);
+      }
+    }
+  } else {
+    for (int i = 0; i < nscrub; ++i) {
+      const SeqRec r = spread ? s_all[i] : s_rec[i];
+      const int* pg = spread ? s_allpg + i * npm : s_pg + i * npm;
+      if (r.cnt < 0) continue;
+      const int p0 = r.P / ps;
+      const int total = (a.n - r.c) * cols;
+      for (int t = t0; t < total; t += tstep) {
+        const int rr = t / cols;
+        const int rem = t - rr * cols;
+        const int which = rem >= head_chunks;
+        const int hc = rem - which * head_chunks;
+        const int g = hc / row_chunks, ch = hc - g * row_chunks;
+        const int pos = r.P + r.c + rr;
+        const int page = pg[pos / ps - p0];
+        char* dst = static_cast<char*>(which ? a.v_pages : a.k_pages);
+        const size_t off = (((size_t)page * a.Hkv + g) * ps + pos % ps) * row_bytes;
+        reinterpret_cast<uint4*>(dst + off)[ch] = make_uint4(0, 0, 0, 0);
+      }
     }
   }
   const int grand = s_grand;
@@ -268,9 +325,15 @@ cudaError_t launch_commit_t(const CommitArgs& a, const GreedyAcceptArgs& f, cuda
   static int limit_cache[64];
   static bool smem_set[64];
   const int slots = (a.n + a.page_size - 1) / a.page_size + 1;
-  // at least as many CTAs as the cluster allows: with a small batch the idle
-  // ones share the zeroing of the rejected rows
-  const int C = cluster_limit(commit_cluster_kernel<kFused>, kCThreads, limit_cache);
+  // One CTA per 16 KB of rows to zero (at most 32 KB: one CTA, which stores
+  // them faster than a cluster barrier takes), up to the largest cluster: with
+  // a small batch the CTAs share the zeroing, and a small cluster finds its
+  // SMs free while the previous kernel's CTAs still hold most of the others.
+  const size_t scrub = (size_t)a.B * a.n * 2 * a.Hkv * a.D * a.elem_bytes;
+  const int C = scrub <= (32u << 10)
+                    ? 1
+                    : (int)std::min<size_t>(cluster_limit(commit_cluster_kernel<kFused>, kCThreads, limit_cache),
+                                            (scrub + (16u << 10) - 1) >> 14);
   const int per = (a.B + C - 1) / C;
   const int npm = commit_npm(a.n, a.page_size);
   const size_t smem = commit_smem(per + (a.B < C ? a.B : 0), npm);

@@ -58,6 +58,15 @@ inline int cluster_limit(Kernel kernel, int threads, int (&cache)[64], size_t sm
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Relaxed load at device scope: served by L2 (the point of coherence), never
+// by a stale L1 line.  For data read before pdl_wait() that kernels further
+// back on the stream wrote.
+__device__ __forceinline__ int ld_relaxed(const int32_t* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Launch `kernel` on `grid` with clusters of `cluster` CTAs (none if the
 // cluster is 1x1x1), as a programmatic dependent of the previous kernel.
 template <typename Kernel, typename... Args>

@@ -53,6 +53,23 @@ def test_commit_matches_oracle(oracle_mod, k, ps, dtype):
     _assert_same(got, rel, nrel, _oracle_commit(oracle_mod, cache, acc, k))
 
 
+@pytest.mark.parametrize("B,k,Hkv", [(1, 16, 3), (2, 8, 6), (5, 4, 3), (1, 2, 8), (1, 16, 5)])
+def test_commit_zeroing_shapes(oracle_mod, B, k, Hkv):
+    # rows of 2 * Hkv * 16 sixteen-byte pieces that do (Hkv 8) and do not
+    # (Hkv 3, 6) divide the CTA's threads, with one CTA (up to 32 KB of rows
+    # to zero) or a cluster sharing them
+    g = torch.Generator().manual_seed(100 * B + 10 * k + Hkv)
+    prefix = tuple(int(x) for x in torch.randint(0, 700, (B,), generator=g))
+    cfg = synth.StepConfig("cz", B=B, Hq=2 * Hkv, Hkv=Hkv, D=128, k=k, prefix=prefix, dtype="bf16",
+                           page_size=64, seed=B + k + Hkv)
+    cache = synth.make_cache(cfg)
+    acc = torch.randint(0, cfg.n + 1, (B,), generator=g, dtype=torch.int32)
+    acc[0] = 0                                            # every draft row rejected
+    got, rel, nrel, st, bits = _gpu_commit(cache, acc, k, max(prefix))
+    assert st == tidar.OK, bits
+    _assert_same(got, rel, nrel, _oracle_commit(oracle_mod, cache, acc, k))
+
+
 def test_commit_bad_count_and_page_leave_sequence_untouched(oracle_mod):
     cfg = synth.StepConfig("cbad", B=4, Hq=2, Hkv=2, D=64, k=4, prefix=(10, 70, 5, 64),
                            dtype="f32", page_size=16, seed=4)

@@ -138,7 +138,7 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x;
-  const int b = blockIdx.y / a.Hkv, g = blockIdx.y % a.Hkv;
+  const int g = blockIdx.y % a.Hkv;
   auto bar = [&](int i) -> uint32_t { return sb + kOffBarD + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMiscD);
   volatile int* stage_bad = abort_flag + 1;
@@ -171,6 +171,8 @@ attn_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   pdl_wait();       // the previous kernel on the stream is complete from here on
   pdl_trigger();
+  // longest sequences first (ragged batches of up to 32 sequences)
+  const int b = longest_first(a.seq_lens, a.B, (int)blockIdx.y / a.Hkv);
 
   // The producer's first two 32-page windows of the page table do not depend on
   // the prefix length, so they load alongside it.

@@ -169,18 +169,20 @@ attn_tc05_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
   pdl_wait();       // the previous kernel on the stream is complete from here on
   pdl_trigger();
+  // longest sequences first (ragged batches of up to 32 sequences)
+  const int b = longest_first(a.seq_lens, a.B, (int)blockIdx.z / a.Hkv);
   // The producer's first two 32-page windows of the page table do not depend on
   // the prefix length, so they load alongside it.
   int win_cur = -1, win_nxt = -1;
   if (warp == 0) {
-    const int32_t* tb = a.page_table + (size_t)(blockIdx.z / a.Hkv) * a.max_pages;
+    const int32_t* tb = a.page_table + (size_t)b * a.max_pages;
     const int pg = blockIdx.y * a.keys_per_split / 64;
     win_cur = pg + lane < a.max_pages ? tb[pg + lane] : -1;
     win_nxt = pg + 32 + lane < a.max_pages ? tb[pg + 32 + lane] : -1;
   }
 
   const int tile = blockIdx.x, split = blockIdx.y;
-  const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
+  const int g = blockIdx.z % a.Hkv;
   const int rho0 = tile * prm.rho_per_tile;
   const int rho1 = min(a.R, rho0 + prm.rho_per_tile);
   const int rows_valid = (rho1 - rho0) * a.G;

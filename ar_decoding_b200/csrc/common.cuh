@@ -58,6 +58,26 @@ inline int cluster_limit(Kernel kernel, int threads, int (&cache)[64], size_t sm
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Order of a ragged batch over the grid: the CTAs of grid row r (rows are
+// dispatched roughly in order) take the sequence with the r-th longest
+// prefix (ties: the lower index first), so that the longest work starts
+// first and the launch ends with a short tail instead of a long sequence
+// started last.  Batches of 2..32 sequences (identity otherwise).  Called by
+// whole warps after the dependency wait (the lengths may come from the
+// previous kernel); every lane returns the same sequence.
+__device__ __forceinline__ int longest_first(const int32_t* seq_lens, int B, int r) {
+  if (B <= 1 || B > 32) return r;
+  const int lane = (int)threadIdx.x & 31;
+  const int len = lane < B ? seq_lens[lane] : 0;
+  int rank = 0;
+  for (int j = 0; j < B; ++j) {
+    const int lj = __shfl_sync(0xffffffffu, len, j);
+    rank += (lj > len || (lj == len && j < lane)) ? 1 : 0;
+  }
+  const unsigned m = __ballot_sync(0xffffffffu, lane < B && rank == r);
+  return m ? __ffs(m) - 1 : r;
+}
+
 // Relaxed load at device scope: served by L2 (the point of coherence), never
 // by a stale L1 line.  For data read before pdl_wait() that kernels further
 // back on the stream wrote.
